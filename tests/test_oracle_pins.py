@@ -1,0 +1,63 @@
+"""The CPU oracle against what the pages and the mathematics fix (no GPU)."""
+
+import pytest
+import torch
+
+import oracle
+from oracle_pins import ALL_PINS, load_table, table_names
+
+
+def _run(xs, mode, chunked):
+    return oracle.ulysses_a2a(xs, mode, chunked)
+
+
+@pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
+def test_pin(pin):
+    pin(_run)
+
+
+@pytest.mark.parametrize("E", [1, 2, 4, 8])
+def test_hand_tables_every_element_size(E):
+    from oracle_pins import pin_hand_tables
+    pin_hand_tables(_run, elem_bytes=E)
+
+
+def test_tables_are_well_formed():
+    # each table lists every input symbol exactly once across its outputs
+    for name in table_names():
+        w, (B, S, H, D), ins, outs = load_table(name)
+        assert len(ins) == w and len(outs) == w
+        assert sorted(s for l in ins for s in l) == sorted(s for l in outs for s in l)
+        assert all(len(l) == B * S * H * D for l in ins + outs)
+
+
+def test_output_shapes_follow_run_armed():
+    # FastVideo API docs, ulysses_a2a `run_armed`: mode 0 -> [B, S_local*w, H//w, D];
+    # mode 1 -> [B, S_global//w, H_local*w, D]
+    assert oracle.output_shape((2, 4725, 40, 128), 0, 8) == (2, 4725 * 8, 5, 128)
+    assert oracle.output_shape((2, 4725 * 8, 5, 128), 1, 8) == (2, 4725, 40, 128)
+    assert oracle.mode0_local_tuple((2, 4725 * 8, 5, 128), 1, 8) == (2, 4725, 40, 128)
+    w = 4
+    x = [torch.zeros(1, 3, 8, 2, dtype=torch.bfloat16) for _ in range(w)]
+    y = oracle.ulysses_a2a(x, 0)
+    assert all(tuple(t.shape) == (1, 12, 2, 2) for t in y)
+    z = oracle.ulysses_a2a(y, 1)
+    assert all(tuple(t.shape) == (1, 3, 8, 2) for t in z)
+
+
+def test_rejects_bad_arguments():
+    x = [torch.zeros(1, 2, 3, 4) for _ in range(2)]
+    with pytest.raises(ValueError):
+        oracle.ulysses_a2a(x, 0)          # H = 3 not divisible by w = 2
+    with pytest.raises(ValueError):
+        oracle.ulysses_a2a([torch.zeros(1, 3, 2, 4) for _ in range(2)], 1)  # S_global % w
+    lib = oracle._get_lib()
+    import ctypes
+    arr = (ctypes.c_void_p * 2)(None, None)
+    assert lib.oracle_ulysses_a2a(arr, arr, 1, 1, 2, 1, 2, 0, 2) == -1
+    good = [torch.zeros(4) for _ in range(4)]
+    a = (ctypes.c_void_p * 2)(good[0].data_ptr(), good[1].data_ptr())
+    b = (ctypes.c_void_p * 2)(good[2].data_ptr(), good[3].data_ptr())
+    assert lib.oracle_ulysses_a2a(a, b, 1, 1, 2, 1, 2, 2, 4) == -1    # mode 2
+    assert lib.oracle_ulysses_a2a(a, b, 0, 1, 2, 1, 2, 0, 4) == -1    # B = 0
+    assert lib.oracle_ulysses_a2a(a, b, 1, 1, 2, 1, 2, 0, 4) == 0
