@@ -1,0 +1,462 @@
+#!/usr/bin/env python3
+"""Benchmark of the B200 Ulysses 4D all-to-all re-layout.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+mode 0 (scatter heads, gather sequence) on the w input slabs, then mode 1 (the
+inverse) on its result, each through the C ABI (host checks, descriptor table,
+tile scheduler, copy kernel). Workload: w=4, B=1, S_local=8192, H=24, D=128,
+bf16, N(0,1) values (payload P = 192 MiB per call).
+
+Metric: payload GB/s (P per call / device time, 1 GB = 1e9 B) and the fraction
+of the measured HBM copy bandwidth, counting 2P bytes moved per call. The L2 is
+flushed (a write of 2x its size) before every timed call, outside the timed
+interval; each call is timed with CUDA events on its stream.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own independent
+instance of the workload (the w logical ranks all live in one GPU's memory, so
+nothing is exchanged); `value` = payload of all ranks / the slowest rank's time
+("weak" scaling). The only collective is the max-over-ranks of the timings.
+
+`--impl reference` times the CPU oracle (the plain nested-loop definition) on
+the host cores, on a bounded sample of the same workload, as a baseline only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "payload GB/s and % of HBM roofline (2x bytes) per mode at w=2/4/8, 1xB200"
+WORKLOAD = dict(w=4, B=1, S_local=8192, H=24, D=128, dtype="bf16")
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 2 * 126 * 1024 * 1024 + (4 << 20)
+
+
+# ---------------------------------------------------------------- helpers
+def env_rank():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs: torch copy, 1 Gi bf16)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sequence_all_re_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_hash):
+    """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None, "no ncu traffic summary"
+    if d.get("kernel_source_hash") != kernel_hash:
+        return None, "kernel changed since the ncu counters were taken"
+    return d, "ncu"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.lines = []
+        try:
+            p = torch.cuda.get_device_properties(device_index)
+            self.bus = "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+        except Exception:
+            self.bus = None
+
+    def start(self):
+        if self.bus is None:
+            return
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.bus, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                maxes.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes),
+                "samples": len(sms), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- our arm
+def make_inputs(w, B, S, H, D, dtype, device, seed0=1234):
+    """Seeded N(0,1) slabs drawn on the device generator (values do not affect timing)."""
+    dt = {"bf16": torch.bfloat16, "fp32": torch.float32}[dtype]
+    xs = []
+    for k in range(w):
+        g = torch.Generator(device=device)
+        g.manual_seed(seed0 + k)
+        xs.append(torch.randn((B, S, H, D), generator=g, device=device, dtype=torch.float32).to(dt))
+    return xs
+
+
+def timed_calls(a2a, xs, ys, flush, steps, warmup, stream, sampler=None):
+    """Per-call device times (ms) of mode 0 (xs->ys) and mode 1 (ys->xs2) over `steps` steps."""
+    xs2 = [torch.empty_like(t) for t in xs]
+    for _ in range(warmup):
+        a2a.run(xs, 0, out=ys, stream=stream)
+        a2a.run(ys, 1, out=xs2, stream=stream)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    launches0 = a2a.launch_count
+    if sampler:
+        sampler.start()
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            a2a.run(xs, 0, out=ys, stream=stream)
+            ev[i][1].record(stream)
+            flush.fill_((i + 1) & 0xFF)
+            ev[i][2].record(stream)
+            a2a.run(ys, 1, out=xs2, stream=stream)
+            ev[i][3].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    launches = a2a.launch_count - launches0
+    t0 = [ev[i][0].elapsed_time(ev[i][1]) for i in range(steps)]
+    t1 = [ev[i][2].elapsed_time(ev[i][3]) for i in range(steps)]
+    return t0, t1, launches, clocks, xs2
+
+
+def bench_sweep_point(a2a, w, payload, dtype, device, flush, stream, reps):
+    E = 2 if dtype == "bf16" else 4
+    H, D = 8 * w, 128
+    S = payload // (w * H * D * E)
+    xs = make_inputs(w, 1, S, H, D, dtype, device)
+    ys = [torch.empty((1, S * w, H // w, D), dtype=xs[0].dtype, device=device) for _ in range(w)]
+    t0, t1, _, _, _ = timed_calls(a2a, xs, ys, flush, reps, 3, stream)
+    P = w * S * H * D * E
+    del xs, ys
+    return P, statistics.median(t0), statistics.median(t1)
+
+
+def cpu_oracle_baseline(w, B, S, H, D, budget_s=12.0):
+    """The oracle, as it stands, on the host: full workload steps until ~budget_s."""
+    import oracle
+    from synth import normal_slabs
+
+    xs = normal_slabs((B, S, H, D), w, "bf16")
+    done = 0
+    t_start = time.perf_counter()
+    while True:
+        y = oracle.ulysses_a2a(xs, 0)
+        oracle.ulysses_a2a(y, 1)
+        done += 1
+        if time.perf_counter() - t_start > budget_s:
+            break
+    el = time.perf_counter() - t_start
+    P = w * B * S * H * D * 2
+    return {"value": round(2 * P * done / el / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{done} full steps (mode 0 + mode 1 on w={w},B={B},S_local={S},H={H},"
+                      f"D={D} bf16) in {el:.1f} s, single-threaded C nested loops"}
+
+
+def run_ours(args):
+    rank, local_rank, world = env_rank()
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=device, timeout=datetime.timedelta(seconds=120))
+
+    from sequence_all_re_b200 import UlyssesA2A
+
+    w, B, S, H, D = (WORKLOAD[k] for k in ("w", "B", "S_local", "H", "D"))
+    E = 2
+    P = w * B * S * H * D * E
+    a2a = UlyssesA2A(local_rank, E)
+    stream = torch.cuda.Stream(device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    xs = make_inputs(w, B, S, H, D, "bf16", device)
+    ys = [torch.empty((B, S * w, H // w, D), dtype=torch.bfloat16, device=device) for _ in range(w)]
+    plan = a2a.plan(xs, 0, out=ys)
+
+    sampler = ClockSampler(local_rank)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0, t1, launches, clocks, xs2 = timed_calls(a2a, xs, ys, flush, args.steps, args.warmup,
+                                                stream, sampler)
+    a2a.status(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    # round trip must reproduce the input bit for bit (cheap on-device check)
+    for k in range(w):
+        if not torch.equal(xs2[k].view(torch.int16), xs[k].view(torch.int16)):
+            raise SystemExit("round trip mismatch: mode1(mode0(x)) != x")
+    total_ms = sum(t0) + sum(t1)
+    if dist:
+        t = torch.tensor([total_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * 2 * P * args.steps / (total_ms / 1e3) / 1e9
+
+    peak, peak_src = hbm_peak()
+    m0 = statistics.mean(t0)
+    m1 = statistics.mean(t1)
+    gbs0 = P / (m0 / 1e3) / 1e9
+    gbs1 = P / (m1 / 1e3) / 1e9
+    avg_launch_ms = (m0 + m1) / 2
+    achieved = 2 * P / (avg_launch_ms / 1e3) / 1e9
+    khash = kernel_source_hash()
+    traffic, traffic_src = ncu_traffic(khash)
+    traffic_bytes = None
+    if traffic:
+        traffic_bytes = traffic.get("workloads", {}).get("w4_B1_S8192_H24_D128_bf16", {}).get(
+            "dram_bytes_per_launch")
+
+    # e2e: the same step through the host-buffer entry point (pinned host slabs)
+    e2e = None
+    if not args.no_e2e:
+        hx = [t.cpu().pin_memory() for t in xs]
+        hy = [torch.empty((B, S * w, H // w, D), dtype=torch.bfloat16).pin_memory() for _ in range(w)]
+        hz = [torch.empty_like(t).pin_memory() for t in hx]
+        for _ in range(2):
+            a2a.run_host(hx, 0, out=hy, stream=stream)
+            a2a.run_host(hy, 1, out=hz, stream=stream)
+        e_steps = max(3, min(args.e2e_steps, args.steps))
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ea = torch.cuda.Event(enable_timing=True)
+        eb = torch.cuda.Event(enable_timing=True)
+        ea.record(stream)
+        for _ in range(e_steps):
+            a2a.run_host(hx, 0, out=hy, stream=stream)
+            a2a.run_host(hy, 1, out=hz, stream=stream)
+        eb.record(stream)
+        torch.cuda.synchronize()
+        e_ms = ea.elapsed_time(eb)
+        if dist:
+            t = torch.tensor([e_ms], device=device, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        for k in range(w):
+            if not torch.equal(hz[k].view(torch.int16), hx[k].view(torch.int16)):
+                raise SystemExit("host-path round trip mismatch")
+        e2e = {"value": round(world * 2 * P * e_steps / (e_ms / 1e3) / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": 2 * P, "d2h_bytes_per_step": 2 * P,
+               "steps": e_steps, "via": "ulysses_a2a_run_host, pinned host slabs"}
+
+    # per-mode figures at w = 2/4/8 on a 512 MiB payload (the >= 256 MB target regime)
+    w_sweep = None
+    if not args.no_sweep and rank == 0 or (not args.no_sweep and world == 1):
+        w_sweep = {}
+        for ww in (2, 4, 8):
+            Pw, a, b = bench_sweep_point(a2a, ww, 512 << 20, "bf16", device, flush, stream,
+                                         args.sweep_reps)
+            w_sweep[f"w{ww}"] = {
+                "payload_bytes": Pw,
+                "mode0_gbs": round(Pw / (a / 1e3) / 1e9, 1),
+                "mode1_gbs": round(Pw / (b / 1e3) / 1e9, 1),
+                "mode0_frac": round(2 * Pw / (a / 1e3) / 1e9 / peak, 4),
+                "mode1_frac": round(2 * Pw / (b / 1e3) / 1e9 / peak, 4),
+            }
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_baseline(w, B, S, H, D, budget_s=args.cpu_budget)
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": "ulysses_a2a w=4 B=1 S_local=8192 H=24 D=128 bf16, step = mode 0 + mode 1",
+            "w": w, "B": B, "S_local": S, "H": H, "D": D,
+            "payload_bytes_per_call": P,
+            "path": {1: "tma", 2: "vec"}[plan["path"]],
+            "rows_per_tile": plan["rows_per_tile"], "stages": plan["stages"], "grid": plan["grid"],
+            "l2": "flushed (2x L2 write) before every timed call, outside its events",
+            "parallelism": f"{world} independent instance(s), one per GPU",
+        },
+        "per_mode": {"mode0_gbs": round(gbs0, 1), "mode1_gbs": round(gbs1, 1),
+                     "mode0_frac": round(2 * gbs0 / peak, 4), "mode1_frac": round(2 * gbs1 / peak, 4)},
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "ua2a_tma_kernel<0>/<1>" if plan["path"] == 1 else "ua2a_vec_kernel",
+            "achieved": round(achieved, 1),
+            "peak": peak,
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "peak_source": peak_src,
+            "algorithmic_bytes_per_launch": 2 * P,
+            "traffic": traffic_bytes,
+            "traffic_source": traffic_src,
+        },
+        "gpu_launches": launches,
+        "e2e": e2e,
+        "clocks": clocks,
+        "w_sweep_512MiB": w_sweep,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    a2a.close()
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank, _, world = env_rank()
+    if rank != 0:
+        return
+    import oracle
+    from synth import normal_slabs
+
+    w, B, S, H, D = (WORKLOAD[k] for k in ("w", "B", "S_local", "H", "D"))
+    E = 2
+    # size each step's sample so warmup + steps finish in about two minutes
+    probe_S = 256
+    xs = normal_slabs((B, probe_S, H, D), w, "bf16")
+    t = time.perf_counter()
+    y = oracle.ulysses_a2a(xs, 0)
+    oracle.ulysses_a2a(y, 1)
+    per_row = (time.perf_counter() - t) / probe_S
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    S_sample = int(max(1, min(S, budget / max(per_row, 1e-9))))
+    xs = normal_slabs((B, S_sample, H, D), w, "bf16")
+    for _ in range(args.warmup):
+        y = oracle.ulysses_a2a(xs, 0)
+        oracle.ulysses_a2a(y, 1)
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        y = oracle.ulysses_a2a(xs, 0)
+        oracle.ulysses_a2a(y, 1)
+        times.append(time.perf_counter() - t)
+    P = w * B * S_sample * H * D * E
+    total = sum(times)
+    value = 2 * P * args.steps / total / 1e9
+    sample = (f"each step: mode 0 + mode 1 on S_local={S_sample} of {S} rows "
+              f"(w={w},B={B},H={H},D={D} bf16), single-threaded C nested loops")
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total / args.steps * 1e3 * (S / S_sample), 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "ulysses_a2a w=4 B=1 S_local=8192 H=24 D=128 bf16, "
+                               "step = mode 0 + mode 1", "w": w, "B": B, "S_local": S, "H": H,
+                   "D": D},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "note": "ms_per_step is scaled from the sample to the full workload",
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--sweep-reps", type=int, default=30)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: warm-up raised to 3 steps", file=sys.stderr)
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

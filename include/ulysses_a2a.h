@@ -1,0 +1,166 @@
+/*
+ * ulysses_a2a.h - C ABI of the B200 Ulysses 4D all-to-all re-layout library
+ * (libulysses_a2a.so).
+ *
+ * The operation (FastVideo API docs, fastvideo.distributed.device_communicators
+ * .ulysses_a2a, `run_armed`): Ulysses sequence parallelism keeps, on each of w
+ * ranks, a sequence shard x_r of shape [B, S_local, H, D]. Before attention,
+ * "mode 0" scatters heads and gathers sequence, so that every rank holds the
+ * whole sequence for H/w heads, [B, S_local*w, H/w, D]; after attention "mode 1"
+ * undoes it. Here all w rank slabs live in one GPU's memory, so the all-to-all
+ * is a pure permutation of bytes:
+ *
+ *   mode 0:  out_r[b, j*S_local + s, h', d] = x_j[b, s, r*(H/w) + h', d]
+ *   mode 1:  out_j[b, s, r*(H/w) + h', d]   = x_r[b, j*S_local + s, h', d]
+ *
+ * for ranks r, j in [0, w), b in [0, B), s in [0, S_local), h' in [0, H/w),
+ * d in [0, D). Rank r receives head group [r*H/w, (r+1)*H/w); the gathered
+ * sequence is rank-major. Values are moved as raw elem_bytes-byte words: no
+ * arithmetic, bit-exact, NaN payloads and -0.0 preserved.
+ *
+ * Layout: every slab is a dense row-major C array. In mode 0 each in_slabs[j]
+ * is [B, S_local, H, D] and each out_slabs[r] is [B, S_local*w, H/w, D]; in
+ * mode 1 the roles are swapped. (B, S_local, H, D) are ALWAYS passed in
+ * mode-0-local terms, whichever the mode, as the page's native op receives them.
+ *
+ * Ownership: the caller owns every slab and the stream. The context owns a tiny
+ * device status word, a cache of TMA descriptors, and (only if
+ * ulysses_a2a_run_host is used) device staging buffers that grow on demand.
+ * Nothing returned by this API ever aliases caller memory.
+ *
+ * Errors: every entry point returns an int status (ULYSSES_A2A_OK = 0). All
+ * arguments are checked on the host BEFORE anything is launched; a rejected
+ * call launches nothing, leaves the outputs untouched and the context usable,
+ * and ulysses_a2a_last_error() describes why. Misalignment is not an error: it
+ * only selects a narrower copy path. Thread safety: one context must not be
+ * used from two host threads at once; distinct contexts are independent.
+ */
+#ifndef ULYSSES_A2A_H
+#define ULYSSES_A2A_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define ULYSSES_A2A_OK              0
+#define ULYSSES_A2A_ERR_INVALID     1  /* bad argument: null, size, H % w, mode */
+#define ULYSSES_A2A_ERR_OVERLAP     2  /* an output slab overlaps another slab  */
+#define ULYSSES_A2A_ERR_DEVICE      3  /* pointer not in ctx's device memory, or
+                                          its allocation is smaller than the slab */
+#define ULYSSES_A2A_ERR_CUDA        4  /* a CUDA runtime/driver call failed     */
+#define ULYSSES_A2A_ERR_UNSUPPORTED 5  /* forced path cannot express the shape  */
+#define ULYSSES_A2A_ERR_NOMEM       6  /* host or device allocation failed      */
+#define ULYSSES_A2A_ERR_TIMEOUT     7  /* a kernel's bounded wait gave up       */
+
+/* ---- copy paths ------------------------------------------------------- */
+#define ULYSSES_A2A_PATH_AUTO 0  /* TMA when the shape allows it, else VEC     */
+#define ULYSSES_A2A_PATH_TMA  1  /* cp.async.bulk.tensor load -> smem -> store */
+#define ULYSSES_A2A_PATH_VEC  2  /* 16/8/4/2/1-byte LDG/STG copy               */
+
+#define ULYSSES_A2A_MAX_W     64 /* largest rank count any path accepts        */
+#define ULYSSES_A2A_MAX_W_TMA 8  /* largest rank count of the TMA path         */
+
+typedef struct ulysses_a2a_ctx ulysses_a2a_ctx; /* opaque */
+
+/* Geometry and path the library picks for one call (see ulysses_a2a_plan). */
+typedef struct ulysses_a2a_plan_t {
+    int32_t path;            /* ULYSSES_A2A_PATH_TMA or _VEC                  */
+    int32_t vec_bytes;       /* VEC path: bytes per load/store (16..1)        */
+    int64_t row_bytes;       /* one contiguous run: (H/w)*D*elem_bytes        */
+    int64_t rows_per_tile;   /* S_tile: sequence rows per work unit           */
+    int64_t tiles_per_block; /* ceil(S_local / S_tile)                        */
+    int64_t tail_rows;       /* S_local % S_tile (0 = no ragged tile)         */
+    int64_t units;           /* work units per launch: w * B_launch * w * T   */
+    int64_t payload_bytes;   /* sum of input slab bytes = w*B*S_local*H*D*E   */
+    int32_t launches;        /* kernel launches per call: 1, or B if chunked  */
+    int32_t grid;            /* CTAs per launch                               */
+    int32_t block;           /* threads per CTA                               */
+    int32_t stages;          /* TMA path: shared-memory ring depth            */
+    int64_t smem_bytes;      /* dynamic shared memory per CTA                 */
+} ulysses_a2a_plan_t;
+
+/* Create a context on CUDA device `device` for elements of `elem_bytes` bytes
+ * (1, 2, 4 or 8; bf16 = 2, fp32 = 4). On success *out holds a new context that
+ * ulysses_a2a_destroy must release. Allocates a few bytes of device memory. */
+int ulysses_a2a_create(ulysses_a2a_ctx **out, int device, int elem_bytes);
+
+/* Release a context. NULL is accepted. Always consumes the handle, even when a
+ * CUDA cleanup call reports an error (returned as ULYSSES_A2A_ERR_CUDA); never
+ * call it twice on the same pointer. Waits for the context's own work first. */
+int ulysses_a2a_destroy(ulysses_a2a_ctx *ctx);
+
+/* The re-layout (FastVideo API docs, ulysses_a2a `run_armed`: output shapes of
+ * both modes, the mode-0-local argument tuple, and the chunked loop).
+ *   in_slabs  : host array of w device pointers, the input slab of each rank.
+ *   out_slabs : host array of w device pointers, caller-allocated outputs. No
+ *               output may overlap any input or any other output.
+ *   B, S_local, H, D : mode-0-local sizes, all >= 1, H % w == 0.
+ *   w         : rank count, 1 <= w <= ULYSSES_A2A_MAX_W (w = 1 is a copy).
+ *   mode      : 0 (scatter heads, gather sequence) or 1 (the inverse).
+ *   chunked   : 0 = one launch over all B planes; 1 = the per-plane variant:
+ *               one launch per plane b on the one-plane views, in stream
+ *               order, so plane b is complete before plane b+1 starts. Same
+ *               bytes either way.
+ *   stream    : a cudaStream_t (NULL = legacy default stream).
+ * Asynchronous on `stream`; no host synchronisation and no allocation. */
+int ulysses_a2a_run(ulysses_a2a_ctx *ctx, const void *const *in_slabs,
+                    void *const *out_slabs, int64_t B, int64_t S_local,
+                    int64_t H, int64_t D, int w, int mode, int chunked,
+                    void *stream);
+
+/* Same operation on HOST slabs (pageable or pinned): copies every input to
+ * context-owned device buffers, runs the re-layout on `stream`, copies every
+ * output back, and returns once out_slabs hold the result. Device buffers grow
+ * on demand and are kept until ulysses_a2a_destroy. */
+int ulysses_a2a_run_host(ulysses_a2a_ctx *ctx, const void *const *in_slabs,
+                         void *const *out_slabs, int64_t B, int64_t S_local,
+                         int64_t H, int64_t D, int w, int mode, int chunked,
+                         void *stream);
+
+/* Human-readable reason for the last failed call on ctx ("" if none). The
+ * string belongs to ctx and stays valid until the next call on it. */
+const char *ulysses_a2a_last_error(const ulysses_a2a_ctx *ctx);
+
+/* Synchronise `stream` and read (then clear) the context's device status word.
+ * Returns ULYSSES_A2A_ERR_TIMEOUT if any kernel launched by this context gave
+ * up a bounded wait since the last check, else ULYSSES_A2A_OK. */
+int ulysses_a2a_status(ulysses_a2a_ctx *ctx, void *stream);
+
+/* Force a copy path (ULYSSES_A2A_PATH_*) for later runs; AUTO restores the
+ * default choice. A forced path that cannot express a shape makes run fail
+ * with ULYSSES_A2A_ERR_UNSUPPORTED instead of silently switching. */
+int ulysses_a2a_set_path(ulysses_a2a_ctx *ctx, int path);
+
+/* Tuning overrides for later runs; 0 keeps the library's default for that
+ * knob. rows_per_tile caps S_tile (1..256); ctas_per_sm sets the persistent
+ * grid (1..32); stages sets the TMA ring depth (2..16). Results never depend
+ * on these, only speed does. */
+int ulysses_a2a_set_tuning(ulysses_a2a_ctx *ctx, int rows_per_tile,
+                           int ctas_per_sm, int stages);
+
+/* Kernel launches this context has issued since creation. */
+uint64_t ulysses_a2a_launch_count(const ulysses_a2a_ctx *ctx);
+
+/* Host-only planning: validates the arguments exactly as ulysses_a2a_run does
+ * (except the device-residency check, which needs a GPU) and reports the path
+ * and geometry it would use. Makes no CUDA call, so it runs without a GPU.
+ * Pointer values are only compared and tested for alignment, never read.
+ * forced_path / rows_per_tile / ctas_per_sm / stages as in the setters above;
+ * num_sms = streaming multiprocessors of the target device (148 on B200).
+ * On failure writes a message of at most errlen bytes into err (if non-NULL). */
+int ulysses_a2a_plan(const void *const *in_slabs, void *const *out_slabs,
+                     int64_t B, int64_t S_local, int64_t H, int64_t D, int w,
+                     int mode, int chunked, int elem_bytes, int forced_path,
+                     int rows_per_tile, int ctas_per_sm, int stages,
+                     int num_sms, ulysses_a2a_plan_t *out, char *err,
+                     size_t errlen);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* ULYSSES_A2A_H */

@@ -1,0 +1,169 @@
+"""B200-native Ulysses 4D all-to-all re-layout.
+
+All ``w`` logical rank slabs live in one GPU's memory, so the Ulysses
+all-to-all is a pure permutation (FastVideo API docs,
+device_communicators/ulysses_a2a, ``run_armed``):
+
+* mode 0 scatters heads and gathers sequence: each rank's ``[B, S_local, H, D]``
+  becomes ``[B, S_local*w, H//w, D]`` with
+  ``out_r[b, j*S_local+s, h', d] = x_j[b, s, r*(H//w)+h', d]``;
+* mode 1 is the exact inverse;
+* ``chunked=True`` runs one launch per batch plane, in stream order.
+
+The work happens in ``libulysses_a2a.so`` (hand-written CUDA for sm_100a,
+C ABI in ``include/ulysses_a2a.h``). This package only marshals tensors into
+that ABI; PyTorch supplies device memory and streams. There is no CPU or
+PyTorch fallback: if the library is missing, importing this package fails.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+from ._lib import A2AError, PATH_AUTO, PATH_TMA, PATH_VEC  # noqa: F401
+
+__all__ = ["UlyssesA2A", "A2AError", "output_shape", "mode0_local_tuple",
+           "PATH_AUTO", "PATH_TMA", "PATH_VEC"]
+
+
+def output_shape(in_shape, mode: int, w: int) -> tuple:
+    """Output slab shape for an input slab shape, as ``run_armed`` derives it."""
+    if mode == 0:
+        B, S_local, H, D = in_shape
+        return (B, S_local * w, H // w, D)
+    B, S_global, H_local, D = in_shape
+    return (B, S_global // w, H_local * w, D)
+
+
+def mode0_local_tuple(in_shape, mode: int, w: int) -> tuple:
+    """(B, S_local, H, D) handed to the native op in either mode."""
+    if mode == 0:
+        return tuple(int(v) for v in in_shape)
+    B, S_global, H_local, D = in_shape
+    return (int(B), int(S_global) // w, int(H_local) * w, int(D))
+
+
+class UlyssesA2A:
+    """A library context bound to one CUDA device and one element size."""
+
+    def __init__(self, device=0, elem_bytes: int = 2):
+        dev = torch.device("cuda", device) if isinstance(device, int) else torch.device(device)
+        self.device = dev
+        self.elem_bytes = int(elem_bytes)
+        self._ctx = _lib.ulysses_a2a_create(dev.index or 0, self.elem_bytes)
+
+    # ------------------------------------------------------------------ knobs
+    def set_path(self, path: int) -> None:
+        self._check(_lib.ulysses_a2a_set_path(self._ctx, path))
+
+    def set_tuning(self, rows_per_tile: int = 0, ctas_per_sm: int = 0, stages: int = 0) -> None:
+        self._check(_lib.ulysses_a2a_set_tuning(self._ctx, rows_per_tile, ctas_per_sm, stages))
+
+    @property
+    def launch_count(self) -> int:
+        return _lib.ulysses_a2a_launch_count(self._ctx)
+
+    def last_error(self) -> str:
+        return _lib.ulysses_a2a_last_error(self._ctx)
+
+    def _check(self, rc: int) -> None:
+        if rc != _lib.OK:
+            raise A2AError(rc, self.last_error())
+
+    # ------------------------------------------------------------- the op
+    def _prepare(self, xs, mode, out, device_type):
+        w = len(xs)
+        if w < 1:
+            raise ValueError("need at least one rank slab")
+        shape = tuple(xs[0].shape)
+        if len(shape) != 4:
+            raise ValueError("rank slabs are 4D")
+        for t in xs:
+            if tuple(t.shape) != shape or t.dtype != xs[0].dtype:
+                raise ValueError("rank slabs must share shape and dtype")
+            if t.element_size() != self.elem_bytes:
+                raise ValueError(f"context handles {self.elem_bytes}-byte elements")
+            if not t.is_contiguous():
+                raise ValueError("rank slabs must be contiguous")
+            if t.device.type != device_type:
+                raise ValueError(f"rank slabs must be on {device_type}")
+        if mode not in (0, 1):
+            raise ValueError("mode must be 0 or 1")
+        B, S, H, D = mode0_local_tuple(shape, mode, w)
+        oshape = output_shape(shape, mode, w)
+        if out is None:
+            kw = {"dtype": xs[0].dtype, "device": xs[0].device}
+            if device_type == "cpu":
+                kw["pin_memory"] = xs[0].is_pinned()
+            out = [torch.empty(oshape, **kw) for _ in range(w)]
+        else:
+            if len(out) != w:
+                raise ValueError("need one output per rank")
+            for o in out:
+                if tuple(o.shape) != oshape or o.dtype != xs[0].dtype or not o.is_contiguous():
+                    raise ValueError(f"outputs must be contiguous {oshape} {xs[0].dtype}")
+        return w, (B, S, H, D), out
+
+    def run(self, xs, mode: int, chunked: bool = False, out=None, stream=None):
+        """Re-layout device slabs ``xs`` (list of w tensors); returns the w outputs.
+
+        Asynchronous on ``stream`` (default: torch's current stream on the device).
+        """
+        w, (B, S, H, D), out = self._prepare(xs, mode, out, "cuda")
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        rc = _lib.ulysses_a2a_run(self._ctx, [t.data_ptr() for t in xs],
+                                  [o.data_ptr() for o in out], B, S, H, D, w, mode,
+                                  int(bool(chunked)), handle)
+        self._check(rc)
+        return out
+
+    def run_host(self, xs, mode: int, chunked: bool = False, out=None, stream=None):
+        """Same op on host slabs: H2D copies, the kernel, D2H copies; returns when done."""
+        w, (B, S, H, D), out = self._prepare(xs, mode, out, "cpu")
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        rc = _lib.ulysses_a2a_run_host(self._ctx, [t.data_ptr() for t in xs],
+                                       [o.data_ptr() for o in out], B, S, H, D, w, mode,
+                                       int(bool(chunked)), handle)
+        self._check(rc)
+        return out
+
+    def status(self, stream=None) -> None:
+        """Synchronise ``stream``; raise if a kernel of this context gave up a wait."""
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        self._check(_lib.ulysses_a2a_status(self._ctx, handle))
+
+    def plan(self, xs, mode: int, chunked: bool = False, out=None) -> dict:
+        """The path and geometry a run with these tensors would use (host only)."""
+        w, (B, S, H, D), out = self._prepare(xs, mode, out, xs[0].device.type)
+        rc, p, msg = _lib.ulysses_a2a_plan([t.data_ptr() for t in xs], [o.data_ptr() for o in out],
+                                           B, S, H, D, w, mode, int(bool(chunked)),
+                                           self.elem_bytes)
+        if rc != _lib.OK:
+            raise A2AError(rc, msg)
+        return p.as_dict()
+
+    def close(self) -> None:
+        if self._ctx is not None:
+            ctx, self._ctx = self._ctx, None
+            rc = _lib.ulysses_a2a_destroy(ctx)
+            if rc != _lib.OK:
+                raise A2AError(rc, "destroy reported a CUDA error (the handle is released)")
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()

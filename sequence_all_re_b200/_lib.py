@@ -1,0 +1,177 @@
+"""ctypes binding of libulysses_a2a.so (include/ulysses_a2a.h), same names.
+
+Argument marshalling only: every step of the re-layout runs inside the CUDA
+library. If the library is missing this module raises at import; there is no
+fallback of any kind.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libulysses_a2a.so")
+
+OK = 0
+ERR_INVALID = 1
+ERR_OVERLAP = 2
+ERR_DEVICE = 3
+ERR_CUDA = 4
+ERR_UNSUPPORTED = 5
+ERR_NOMEM = 6
+ERR_TIMEOUT = 7
+
+PATH_AUTO = 0
+PATH_TMA = 1
+PATH_VEC = 2
+
+MAX_W = 64
+MAX_W_TMA = 8
+
+EXPORTED = (
+    "ulysses_a2a_create",
+    "ulysses_a2a_destroy",
+    "ulysses_a2a_run",
+    "ulysses_a2a_run_host",
+    "ulysses_a2a_last_error",
+    "ulysses_a2a_status",
+    "ulysses_a2a_set_path",
+    "ulysses_a2a_set_tuning",
+    "ulysses_a2a_launch_count",
+    "ulysses_a2a_plan",
+)
+
+
+class PlanT(ctypes.Structure):
+    """Mirror of ``ulysses_a2a_plan_t``."""
+
+    _fields_ = [
+        ("path", ctypes.c_int32),
+        ("vec_bytes", ctypes.c_int32),
+        ("row_bytes", ctypes.c_int64),
+        ("rows_per_tile", ctypes.c_int64),
+        ("tiles_per_block", ctypes.c_int64),
+        ("tail_rows", ctypes.c_int64),
+        ("units", ctypes.c_int64),
+        ("payload_bytes", ctypes.c_int64),
+        ("launches", ctypes.c_int32),
+        ("grid", ctypes.c_int32),
+        ("block", ctypes.c_int32),
+        ("stages", ctypes.c_int32),
+        ("smem_bytes", ctypes.c_int64),
+    ]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+class A2AError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"ulysses_a2a error {code}: {msg}")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is not built; run `python -m sequence_all_re_b200.build` "
+            "(the CUDA library is required: there is no fallback path)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    PP = ctypes.POINTER(ctypes.c_void_p)
+    i64 = ctypes.c_int64
+    c_int = ctypes.c_int
+    lib.ulysses_a2a_create.argtypes = [ctypes.POINTER(P), c_int, c_int]
+    lib.ulysses_a2a_create.restype = c_int
+    lib.ulysses_a2a_destroy.argtypes = [P]
+    lib.ulysses_a2a_destroy.restype = c_int
+    run_args = [P, PP, PP, i64, i64, i64, i64, c_int, c_int, c_int, P]
+    lib.ulysses_a2a_run.argtypes = run_args
+    lib.ulysses_a2a_run.restype = c_int
+    lib.ulysses_a2a_run_host.argtypes = run_args
+    lib.ulysses_a2a_run_host.restype = c_int
+    lib.ulysses_a2a_last_error.argtypes = [P]
+    lib.ulysses_a2a_last_error.restype = ctypes.c_char_p
+    lib.ulysses_a2a_status.argtypes = [P, P]
+    lib.ulysses_a2a_status.restype = c_int
+    lib.ulysses_a2a_set_path.argtypes = [P, c_int]
+    lib.ulysses_a2a_set_path.restype = c_int
+    lib.ulysses_a2a_set_tuning.argtypes = [P, c_int, c_int, c_int]
+    lib.ulysses_a2a_set_tuning.restype = c_int
+    lib.ulysses_a2a_launch_count.argtypes = [P]
+    lib.ulysses_a2a_launch_count.restype = ctypes.c_uint64
+    lib.ulysses_a2a_plan.argtypes = [PP, PP, i64, i64, i64, i64, c_int, c_int, c_int, c_int,
+                                     c_int, c_int, c_int, c_int, c_int,
+                                     ctypes.POINTER(PlanT), ctypes.c_char_p, ctypes.c_size_t]
+    lib.ulysses_a2a_plan.restype = c_int
+    return lib
+
+
+lib = _load()
+
+
+def ptr_array(ptrs) -> ctypes.Array:
+    return (ctypes.c_void_p * len(ptrs))(*[int(p) for p in ptrs])
+
+
+# ---- same-named thin wrappers -------------------------------------------------
+
+def ulysses_a2a_create(device: int, elem_bytes: int) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    rc = lib.ulysses_a2a_create(ctypes.byref(h), int(device), int(elem_bytes))
+    if rc != OK:
+        raise A2AError(rc, f"create(device={device}, elem_bytes={elem_bytes}) failed")
+    return h
+
+
+def ulysses_a2a_destroy(ctx) -> int:
+    return lib.ulysses_a2a_destroy(ctx)
+
+
+def ulysses_a2a_last_error(ctx) -> str:
+    s = lib.ulysses_a2a_last_error(ctx)
+    return s.decode() if s else ""
+
+
+def ulysses_a2a_run(ctx, in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, stream) -> int:
+    return lib.ulysses_a2a_run(ctx, ptr_array(in_ptrs), ptr_array(out_ptrs), int(B), int(S_local),
+                               int(H), int(D), int(w), int(mode), int(chunked),
+                               ctypes.c_void_p(int(stream)))
+
+
+def ulysses_a2a_run_host(ctx, in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, stream) -> int:
+    return lib.ulysses_a2a_run_host(ctx, ptr_array(in_ptrs), ptr_array(out_ptrs), int(B),
+                                    int(S_local), int(H), int(D), int(w), int(mode), int(chunked),
+                                    ctypes.c_void_p(int(stream)))
+
+
+def ulysses_a2a_status(ctx, stream) -> int:
+    return lib.ulysses_a2a_status(ctx, ctypes.c_void_p(int(stream)))
+
+
+def ulysses_a2a_set_path(ctx, path: int) -> int:
+    return lib.ulysses_a2a_set_path(ctx, int(path))
+
+
+def ulysses_a2a_set_tuning(ctx, rows_per_tile: int = 0, ctas_per_sm: int = 0, stages: int = 0) -> int:
+    return lib.ulysses_a2a_set_tuning(ctx, int(rows_per_tile), int(ctas_per_sm), int(stages))
+
+
+def ulysses_a2a_launch_count(ctx) -> int:
+    return int(lib.ulysses_a2a_launch_count(ctx))
+
+
+def ulysses_a2a_plan(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, elem_bytes,
+                     forced_path=PATH_AUTO, rows_per_tile=0, ctas_per_sm=0, stages=0,
+                     num_sms=148):
+    """Host-only planning (no CUDA call). Returns (rc, PlanT, message)."""
+    plan = PlanT()
+    buf = ctypes.create_string_buffer(256)
+    ins = ptr_array(in_ptrs) if in_ptrs is not None else None
+    outs = ptr_array(out_ptrs) if out_ptrs is not None else None
+    rc = lib.ulysses_a2a_plan(ins, outs, int(B), int(S_local), int(H), int(D), int(w), int(mode),
+                              int(chunked), int(elem_bytes), int(forced_path), int(rows_per_tile),
+                              int(ctas_per_sm), int(stages), int(num_sms), ctypes.byref(plan),
+                              buf, len(buf))
+    return rc, plan, buf.value.decode()

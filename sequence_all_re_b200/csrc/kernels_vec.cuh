@@ -1,0 +1,126 @@
+// kernels_vec.cuh - vectorised LDG/STG copy path of the Ulysses 4D all-to-all
+// re-layout (any shape, any alignment).
+//
+// Mode 0 (FastVideo API docs, device_communicators/ulysses_a2a, `run_armed`,
+// mode-0 branch): out_r[b, j*S_local + s, h', d] = x_j[b, s, r*(H/w) + h', d].
+// Mode 1 (the else branch, the inverse): out_j[b, s, r*(H/w) + h', d] =
+// x_r[b, j*S_local + s, h', d].
+//
+// For fixed (r, b, j) the (h', d) pairs of one sequence row form a contiguous
+// run of L = (H/w)*D elements on BOTH sides, so the copy moves whole runs:
+// vectors of V bytes (16 when every base address and the run length allow it,
+// otherwise 8/4/2/1), with `ld.global.cs` / `st.global.cs` (streaming, evict
+// first: every byte is touched exactly once). A CTA owns one work unit at a
+// time: up to S_tile rows of one (r, b, j) block, the last tile of a block
+// holding only the S_local % S_tile remaining rows (ceil-div tiling, clamped
+// row count). Each thread keeps U vectors in flight before storing them.
+#pragma once
+
+#include <cstdint>
+
+#include "ulysses_a2a.h"
+
+namespace ua2a {
+
+// Division by a run-time invariant divisor d (1 <= d < 2^31) for dividends
+// n < 2^31, by multiply-high and shift: the round-up method of Granlund and
+// Montgomery, "Division by invariant integers using multiplication" (PLDI 1994).
+// With s = ceil(log2 d) and m = floor(2^32 (2^s - d) / d) + 1, the quotient is
+// (umulhi(n, m) + n) >> s.
+struct FastDiv {
+  uint32_t d = 1, m = 1, s = 0;
+  FastDiv() = default;
+  explicit FastDiv(uint32_t div) : d(div) {
+    s = 0;
+    while ((uint64_t(1) << s) < div) ++s;
+    m = (uint32_t)((((uint64_t(1) << s) - div) << 32) / div + 1);
+  }
+};
+
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+  return (__umulhi(n, f.m) + n) >> f.s;
+}
+
+struct VecParams {
+  const char* in[ULYSSES_A2A_MAX_W];
+  char* out[ULYSSES_A2A_MAX_W];
+  int64_t S_local;
+  int64_t b0;            // first plane of this launch
+  int64_t nv;            // vectors per run: L*E / V
+  int32_t w;
+  int32_t rows_per_tile;
+  uint32_t units;        // w * nb * w * T
+  FastDiv div_T;         // tiles per (r, b, j) block
+  FastDiv div_w;
+  FastDiv div_nb;        // planes in this launch
+  FastDiv div_nv;
+};
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) { return __ldcs(p); }
+__device__ __forceinline__ uint2 ld_stream(const uint2* p) { return __ldcs(p); }
+__device__ __forceinline__ unsigned int ld_stream(const unsigned int* p) { return __ldcs(p); }
+__device__ __forceinline__ unsigned short ld_stream(const unsigned short* p) { return __ldcs(p); }
+__device__ __forceinline__ unsigned char ld_stream(const unsigned char* p) { return __ldcs(p); }
+__device__ __forceinline__ void st_stream(uint4* p, uint4 v) { __stcs(p, v); }
+__device__ __forceinline__ void st_stream(uint2* p, uint2 v) { __stcs(p, v); }
+__device__ __forceinline__ void st_stream(unsigned int* p, unsigned int v) { __stcs(p, v); }
+__device__ __forceinline__ void st_stream(unsigned short* p, unsigned short v) { __stcs(p, v); }
+__device__ __forceinline__ void st_stream(unsigned char* p, unsigned char v) { __stcs(p, v); }
+
+template <typename V, int MODE, int U>
+__global__ void __launch_bounds__(256) ua2a_vec_kernel(const __grid_constant__ VecParams p) {
+  const uint32_t nv = (uint32_t)p.nv;
+  const int64_t strided_row = (int64_t)p.w * p.nv;  // vectors between rows s, s+1 of [B,S,H,D]
+  const uint32_t step = blockDim.x * U;
+  for (uint32_t u = blockIdx.x; u < p.units; u += gridDim.x) {
+    // u = ((r * nb + b_rel) * w + j) * T + t
+    const uint32_t q = fdiv(u, p.div_T);
+    const uint32_t t = u - q * p.div_T.d;
+    const uint32_t q2 = fdiv(q, p.div_w);
+    const uint32_t j = q - q2 * p.div_w.d;
+    const uint32_t r = fdiv(q2, p.div_nb);
+    const uint32_t bl = q2 - r * p.div_nb.d;
+    const int64_t b = p.b0 + bl;
+    const int64_t s0 = (int64_t)t * p.rows_per_tile;
+    const int64_t rows_left = p.S_local - s0;
+    const int64_t rows = rows_left < p.rows_per_tile ? rows_left : p.rows_per_tile;
+    // strided side: row (b, s0), head group r; gathered side: row (b, j*S_local + s0)
+    const int64_t soff = (b * p.S_local + s0) * strided_row + (int64_t)r * p.nv;
+    const int64_t goff = ((b * p.w + j) * p.S_local + s0) * p.nv;
+    const V* src;
+    V* dst;
+    if (MODE == 0) {
+      src = reinterpret_cast<const V*>(p.in[j]) + soff;
+      dst = reinterpret_cast<V*>(p.out[r]) + goff;
+    } else {
+      src = reinterpret_cast<const V*>(p.in[r]) + goff;
+      dst = reinterpret_cast<V*>(p.out[j]) + soff;
+    }
+    const uint32_t n = (uint32_t)(rows * p.nv);
+    for (uint32_t base = threadIdx.x; base < n; base += step) {
+      V v[U];
+#pragma unroll
+      for (int k = 0; k < U; ++k) {
+        const uint32_t e = base + k * blockDim.x;
+        if (e < n) {
+          const uint32_t row = fdiv(e, p.div_nv);
+          const uint32_t c = e - row * nv;
+          const int64_t off = (MODE == 0) ? (int64_t)row * strided_row + c : (int64_t)e;
+          v[k] = ld_stream(src + off);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < U; ++k) {
+        const uint32_t e = base + k * blockDim.x;
+        if (e < n) {
+          const uint32_t row = fdiv(e, p.div_nv);
+          const uint32_t c = e - row * nv;
+          const int64_t off = (MODE == 0) ? (int64_t)e : (int64_t)row * strided_row + c;
+          st_stream(dst + off, v[k]);
+        }
+      }
+    }
+  }
+}
+
+}  // namespace ua2a

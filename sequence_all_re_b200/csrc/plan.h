@@ -1,0 +1,246 @@
+// plan.h - host-only argument checks and work geometry for the Ulysses 4D
+// all-to-all re-layout (FastVideo API docs, device_communicators/ulysses_a2a,
+// `run_armed`: shapes of both modes and the per-plane chunked loop).
+//
+// Nothing here touches CUDA: the same code validates ulysses_a2a_run's
+// arguments and answers ulysses_a2a_plan on a machine without a GPU.
+//
+// Work decomposition. For ranks r (destination head group) and j (source
+// sequence shard), plane b and sequence tile t, one work unit moves rows
+// s in [t*S_tile, min((t+1)*S_tile, S_local)) of the (r, b, j) block:
+//   strided side  [B, S_local, H, D]     : rows of L = (H/w)*D elements,
+//                                          stride H*D, at head offset r*L;
+//   gathered side [B, S_local*w, H/w, D] : the same rows, contiguous, at
+//                                          sequence offset j*S_local.
+// Mode 0 reads the strided side and writes the gathered side; mode 1 the
+// reverse. Units are numbered (r, b, j, t) with t fastest, so consecutive
+// CTAs touch consecutive bytes of the contiguous side.
+#pragma once
+
+#include <cstdint>
+#include <cstdio>
+#include <string>
+
+#include "ulysses_a2a.h"
+
+namespace ua2a {
+
+// Bytes of one work unit the planner aims for (shared-memory stage size).
+constexpr int64_t kTileTargetBytes = 32 * 1024;
+// Largest TMA tile; a single row longer than this goes to the VEC path.
+constexpr int64_t kTmaMaxTileBytes = 64 * 1024;
+// Dynamic shared memory the TMA ring may use per CTA by default (of 227 KB).
+constexpr int64_t kTmaSmemBudget = 192 * 1024;
+constexpr int64_t kTmaSmemMax = 220 * 1024;
+constexpr int kTmaMaxStages = 16;
+constexpr int kTmaBlock = 32;
+constexpr int kTmaDefaultCtasPerSm = 1;
+constexpr int kTmaMaxBoxDim = 256;
+constexpr int kVecBlock = 256;
+constexpr int kVecDefaultCtasPerSm = 8;
+
+struct Tuning {
+  int rows_per_tile = 0;  // 0 = default
+  int ctas_per_sm = 0;
+  int stages = 0;
+};
+
+inline bool mul_overflows(int64_t a, int64_t b, int64_t* out) {
+  return __builtin_mul_overflow(a, b, out);
+}
+
+inline void set_err(std::string* err, const char* fmt, long long a = 0, long long b = 0) {
+  if (!err) return;
+  char buf[256];
+  std::snprintf(buf, sizeof(buf), fmt, a, b);
+  *err = buf;
+}
+
+// [lo, hi) ranges intersect?
+inline bool overlaps(uintptr_t a, uintptr_t a_end, uintptr_t b, uintptr_t b_end) {
+  return a < b_end && b < a_end;
+}
+
+// Why the TMA path cannot take a shape (nullptr if it can).
+inline const char* tma_blocker(const void* const* in, void* const* out, int64_t B,
+                               int64_t S, int64_t H, int64_t D, int w, int E,
+                               int64_t row_bytes) {
+  const int64_t Hw = H / w;
+  if (w > ULYSSES_A2A_MAX_W_TMA) return "w exceeds the TMA path's rank limit";
+  if (D > kTmaMaxBoxDim || Hw > kTmaMaxBoxDim) return "D or H/w exceeds a TMA box dimension (256)";
+  if ((D * E) % 16 != 0) return "D*elem_bytes is not a multiple of 16 bytes";
+  if (row_bytes > kTmaMaxTileBytes) return "one row run exceeds the TMA tile limit";
+  if (S > INT32_MAX || B > INT32_MAX) return "S_local or B exceeds a TMA coordinate";
+  // global strides must stay below 2^40 bytes: the largest is one plane
+  if (S * H * D * E >= (int64_t(1) << 40)) return "plane stride exceeds the TMA stride limit";
+  for (int k = 0; k < w; ++k) {
+    if ((reinterpret_cast<uintptr_t>(in[k]) & 15u) != 0 ||
+        (reinterpret_cast<uintptr_t>(out[k]) & 15u) != 0)
+      return "a slab base address is not 16-byte aligned";
+  }
+  return nullptr;
+}
+
+// Validate and plan one call. Returns a ULYSSES_A2A_* status.
+inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t S,
+                     int64_t H, int64_t D, int w, int mode, int chunked, int E,
+                     int forced_path, const Tuning& tune, int num_sms,
+                     ulysses_a2a_plan_t* p, std::string* err) {
+  if (p == nullptr) { set_err(err, "plan output is NULL"); return ULYSSES_A2A_ERR_INVALID; }
+  *p = ulysses_a2a_plan_t{};
+  if (in == nullptr || out == nullptr) {
+    set_err(err, "in_slabs/out_slabs array is NULL");
+    return ULYSSES_A2A_ERR_INVALID;
+  }
+  if (w < 1 || w > ULYSSES_A2A_MAX_W) {
+    set_err(err, "w=%lld outside [1, %lld]", w, ULYSSES_A2A_MAX_W);
+    return ULYSSES_A2A_ERR_INVALID;
+  }
+  if (!(E == 1 || E == 2 || E == 4 || E == 8)) {
+    set_err(err, "elem_bytes=%lld not in {1,2,4,8}", E);
+    return ULYSSES_A2A_ERR_INVALID;
+  }
+  if (mode != 0 && mode != 1) { set_err(err, "mode=%lld not 0 or 1", mode); return ULYSSES_A2A_ERR_INVALID; }
+  if (chunked != 0 && chunked != 1) { set_err(err, "chunked=%lld not 0 or 1", chunked); return ULYSSES_A2A_ERR_INVALID; }
+  if (B < 1 || S < 1 || H < 1 || D < 1) {
+    set_err(err, "sizes must be >= 1 (B, S_local, H, D)");
+    return ULYSSES_A2A_ERR_INVALID;
+  }
+  if (H % w != 0) { set_err(err, "H=%lld not divisible by w=%lld", H, w); return ULYSSES_A2A_ERR_INVALID; }
+  if (forced_path < ULYSSES_A2A_PATH_AUTO || forced_path > ULYSSES_A2A_PATH_VEC) {
+    set_err(err, "unknown path %lld", forced_path);
+    return ULYSSES_A2A_ERR_INVALID;
+  }
+  if (num_sms < 1) { set_err(err, "num_sms must be >= 1"); return ULYSSES_A2A_ERR_INVALID; }
+
+  // sizes, overflow-checked
+  int64_t plane_elems, slab_elems, slab_bytes, payload, tmp;
+  if (mul_overflows(S, H, &tmp) || mul_overflows(tmp, D, &plane_elems) ||
+      mul_overflows(plane_elems, B, &slab_elems) || mul_overflows(slab_elems, E, &slab_bytes) ||
+      mul_overflows(slab_bytes, (int64_t)w, &payload) || payload > (int64_t(1) << 56)) {
+    set_err(err, "slab sizes overflow");
+    return ULYSSES_A2A_ERR_INVALID;
+  }
+  for (int k = 0; k < w; ++k) {
+    if (in[k] == nullptr || out[k] == nullptr) {
+      set_err(err, "slab pointer %lld is NULL", k);
+      return ULYSSES_A2A_ERR_INVALID;
+    }
+  }
+  // No output may overlap an input or another output (inputs may alias each other).
+  for (int k = 0; k < w; ++k) {
+    const uintptr_t o = reinterpret_cast<uintptr_t>(out[k]);
+    const uintptr_t oe = o + (uintptr_t)slab_bytes;
+    if (oe < o) { set_err(err, "output slab %lld wraps the address space", k); return ULYSSES_A2A_ERR_INVALID; }
+    for (int m = 0; m < w; ++m) {
+      const uintptr_t i = reinterpret_cast<uintptr_t>(in[m]);
+      if (overlaps(o, oe, i, i + (uintptr_t)slab_bytes)) {
+        set_err(err, "output slab %lld overlaps input slab %lld", k, m);
+        return ULYSSES_A2A_ERR_OVERLAP;
+      }
+      if (m != k) {
+        const uintptr_t q = reinterpret_cast<uintptr_t>(out[m]);
+        if (overlaps(o, oe, q, q + (uintptr_t)slab_bytes)) {
+          set_err(err, "output slab %lld overlaps output slab %lld", k, m);
+          return ULYSSES_A2A_ERR_OVERLAP;
+        }
+      }
+    }
+  }
+
+  const int64_t Hw = H / w;
+  const int64_t row_bytes = Hw * D * E;  // one contiguous run, L*E
+  const char* blocker = tma_blocker(in, out, B, S, H, D, w, E, row_bytes);
+  int path;
+  if (forced_path == ULYSSES_A2A_PATH_TMA) {
+    if (blocker) {
+      if (err) *err = std::string("TMA path forced but unusable: ") + blocker;
+      return ULYSSES_A2A_ERR_UNSUPPORTED;
+    }
+    path = ULYSSES_A2A_PATH_TMA;
+  } else if (forced_path == ULYSSES_A2A_PATH_VEC) {
+    path = ULYSSES_A2A_PATH_VEC;
+  } else {
+    path = blocker ? ULYSSES_A2A_PATH_VEC : ULYSSES_A2A_PATH_TMA;
+  }
+
+  // sequence rows per work unit
+  int64_t rows = kTileTargetBytes / row_bytes;
+  if (tune.rows_per_tile > 0) rows = tune.rows_per_tile;
+  if (rows < 1) rows = 1;
+  if (rows > kTmaMaxBoxDim) rows = kTmaMaxBoxDim;
+  if (path == ULYSSES_A2A_PATH_TMA) {
+    while (rows > 1 && rows * row_bytes > kTmaMaxTileBytes) --rows;
+  }
+  if (rows > S) rows = S;
+
+  const int64_t T = (S + rows - 1) / rows;  // ceil-div: the ragged last tile is a unit too
+  const int64_t nb = chunked ? 1 : B;
+  int64_t units;
+  if (mul_overflows((int64_t)w * w, nb, &tmp) || mul_overflows(tmp, T, &units)) {
+    set_err(err, "unit count overflows");
+    return ULYSSES_A2A_ERR_INVALID;
+  }
+
+  p->path = path;
+  p->row_bytes = row_bytes;
+  p->rows_per_tile = rows;
+  p->tiles_per_block = T;
+  p->tail_rows = S % rows;
+  p->units = units;
+  p->payload_bytes = payload;
+  p->launches = chunked ? (int32_t)(B > INT32_MAX ? INT32_MAX : B) : 1;
+
+  if (path == ULYSSES_A2A_PATH_TMA) {
+    const int64_t tile_bytes = rows * row_bytes;
+    const int64_t stage_bytes = (tile_bytes + 1023) / 1024 * 1024;
+    int ctas = tune.ctas_per_sm > 0 ? tune.ctas_per_sm : kTmaDefaultCtasPerSm;
+    int64_t stages = tune.stages > 0 ? tune.stages : kTmaSmemBudget / stage_bytes;
+    if (stages > kTmaMaxStages) stages = kTmaMaxStages;
+    while (stages > 2 && stages * stage_bytes > kTmaSmemMax) --stages;
+    if (stages < 2 || stages * stage_bytes > kTmaSmemMax) {
+      // cannot hold two tiles: let the VEC path take it (or fail if forced)
+      if (forced_path == ULYSSES_A2A_PATH_TMA) {
+        set_err(err, "TMA ring of two %lld-byte tiles does not fit shared memory", tile_bytes);
+        return ULYSSES_A2A_ERR_UNSUPPORTED;
+      }
+      p->path = path = ULYSSES_A2A_PATH_VEC;
+    } else {
+      p->stages = (int32_t)stages;
+      p->smem_bytes = stages * stage_bytes;
+      p->block = kTmaBlock;
+      int64_t g = (int64_t)num_sms * ctas;
+      p->grid = (int32_t)(units < g ? units : g);
+      p->vec_bytes = 16;
+    }
+  }
+  if (path == ULYSSES_A2A_PATH_VEC) {
+    int v = 16;
+    while (v > 1) {
+      bool ok = (row_bytes % v) == 0;
+      for (int k = 0; k < w && ok; ++k)
+        ok = (reinterpret_cast<uintptr_t>(in[k]) % v) == 0 &&
+             (reinterpret_cast<uintptr_t>(out[k]) % v) == 0;
+      if (ok) break;
+      v >>= 1;
+    }
+    if (units >= (int64_t(1) << 31)) {
+      set_err(err, "%lld work units exceed the VEC path's 2^31 limit", units);
+      return ULYSSES_A2A_ERR_UNSUPPORTED;
+    }
+    if (rows * (row_bytes / v) >= (int64_t(1) << 31)) {
+      set_err(err, "one VEC tile exceeds 2^31 vectors");
+      return ULYSSES_A2A_ERR_UNSUPPORTED;
+    }
+    int ctas = tune.ctas_per_sm > 0 ? tune.ctas_per_sm : kVecDefaultCtasPerSm;
+    int64_t g = (int64_t)num_sms * ctas;
+    p->vec_bytes = v;
+    p->stages = 0;
+    p->smem_bytes = 0;
+    p->block = kVecBlock;
+    p->grid = (int32_t)(units < g ? units : g);
+  }
+  return ULYSSES_A2A_OK;
+}
+
+}  // namespace ua2a

@@ -1,0 +1,541 @@
+// ulysses_a2a.cu - C ABI of the B200 Ulysses 4D all-to-all re-layout.
+//
+// Implements include/ulysses_a2a.h. The operation and its argument convention
+// follow the FastVideo API docs, fastvideo.distributed.device_communicators
+// .ulysses_a2a, `run_armed`: the native op always receives the mode-0-local
+// tuple (B, S_local, H, D); mode 0 produces [B, S_local*w, H/w, D] per rank,
+// mode 1 produces [B, S_local, H, D]; the chunked variant runs the op once per
+// plane on one-plane views, each plane finishing (stream order) before the
+// next starts.
+//
+// On one GPU every rank slab is local, so the all-to-all is a permutation and
+// the work is pure data movement: two kernels (kernels_tma.cuh,
+// kernels_vec.cuh), picked per shape by the host planner (plan.h). The context
+// plays the part of the page's reusable communication handle: it holds the
+// rank-slab descriptor table (TMA tensor maps, cached per pointer set and
+// shape), the device status word of the bounded waits, and the device staging
+// buffers of the host-buffer entry point (grown on demand, like the page's
+// window `_build`/grow).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "kernels_tma.cuh"
+#include "kernels_vec.cuh"
+#include "plan.h"
+#include "ulysses_a2a.h"
+
+using ua2a::TmaParams;
+using ua2a::VecParams;
+
+namespace {
+
+constexpr int kTmaCacheEntries = 16;
+
+struct TmaCacheEntry {
+  bool valid = false;
+  uint64_t stamp = 0;
+  int mode = 0, w = 0;
+  int64_t B = 0, S = 0, H = 0, D = 0, rows = 0;
+  const void* in[ULYSSES_A2A_MAX_W_TMA] = {};
+  void* out[ULYSSES_A2A_MAX_W_TMA] = {};
+  TmaParams params;  // tensor maps + geometry (b0/nb/status filled per launch)
+};
+
+}  // namespace
+
+struct ulysses_a2a_ctx {
+  int device = 0;
+  int elem_bytes = 2;
+  int num_sms = 148;
+  int forced_path = ULYSSES_A2A_PATH_AUTO;
+  ua2a::Tuning tuning;
+  unsigned int* d_status = nullptr;  // 4 words, see kernels_tma.cuh
+  std::string last_error;
+  uint64_t launches = 0;
+  uint64_t stamp = 0;
+  TmaCacheEntry tma_cache[kTmaCacheEntries];
+  bool tma_smem_set[2] = {false, false};
+  int64_t tma_smem_set_bytes[2] = {0, 0};
+  // run_host staging: one device buffer carved into 2w slabs
+  void* d_stage = nullptr;
+  size_t stage_bytes = 0;
+  PFN_cuTensorMapEncodeTiled_v12000 encode_tiled = nullptr;
+  PFN_cuMemGetAddressRange_v3020 get_range = nullptr;
+};
+
+namespace {
+
+// Switch to the context's device for the lifetime of the guard.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    ok = cudaSetDevice(dev) == cudaSuccess;
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+int fail(ulysses_a2a_ctx* ctx, int code, const std::string& msg) {
+  if (ctx) ctx->last_error = msg;
+  return code;
+}
+
+int cuda_fail(ulysses_a2a_ctx* ctx, const char* what, cudaError_t e) {
+  return fail(ctx, ULYSSES_A2A_ERR_CUDA,
+              std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")");
+}
+
+int env_int(const char* name, int dflt) {
+  const char* v = std::getenv(name);
+  if (!v || !*v) return dflt;
+  return std::atoi(v);
+}
+
+CUtensorMapDataType map_dtype(int E) {
+  switch (E) {
+    case 1: return CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    case 2: return CU_TENSOR_MAP_DATA_TYPE_UINT16;
+    case 4: return CU_TENSOR_MAP_DATA_TYPE_UINT32;
+    default: return CU_TENSOR_MAP_DATA_TYPE_UINT64;
+  }
+}
+
+// Tensor maps of one strided-side slab [B, S, H, D] and one gathered-side slab
+// [B, S*w, H/w, D] (viewed as [B, w, S, H/w, D] so rows stop at S per block).
+int encode_strided(ulysses_a2a_ctx* ctx, CUtensorMap* m, const void* base, int64_t B, int64_t S,
+                   int64_t H, int64_t D, int64_t Hw, int64_t rows) {
+  const int64_t E = ctx->elem_bytes;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)(D * E), (cuuint64_t)(H * D * E), (cuuint64_t)(S * H * D * E)};
+  cuuint32_t box[4] = {(cuuint32_t)D, (cuuint32_t)Hw, (cuuint32_t)rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = ctx->encode_tiled(m, map_dtype((int)E), 4, const_cast<void*>(base), dims, strides, box,
+                                 estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(ctx, ULYSSES_A2A_ERR_CUDA, "cuTensorMapEncodeTiled (strided side) failed: " + std::to_string((int)r));
+  return ULYSSES_A2A_OK;
+}
+
+int encode_gathered(ulysses_a2a_ctx* ctx, CUtensorMap* m, const void* base, int64_t B, int64_t S,
+                    int64_t Hw, int64_t D, int w, int64_t rows) {
+  const int64_t E = ctx->elem_bytes;
+  cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)Hw, (cuuint64_t)S, (cuuint64_t)w, (cuuint64_t)B};
+  cuuint64_t strides[4] = {(cuuint64_t)(D * E), (cuuint64_t)(Hw * D * E), (cuuint64_t)(S * Hw * D * E),
+                           (cuuint64_t)(w * S * Hw * D * E)};
+  cuuint32_t box[5] = {(cuuint32_t)D, (cuuint32_t)Hw, (cuuint32_t)rows, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = ctx->encode_tiled(m, map_dtype((int)E), 5, const_cast<void*>(base), dims, strides, box,
+                                 estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(ctx, ULYSSES_A2A_ERR_CUDA, "cuTensorMapEncodeTiled (gathered side) failed: " + std::to_string((int)r));
+  return ULYSSES_A2A_OK;
+}
+
+// Find or build the descriptor table for this pointer set and shape.
+int tma_params_for(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, int64_t B,
+                   int64_t S, int64_t H, int64_t D, int w, int mode, const ulysses_a2a_plan_t& pl,
+                   TmaParams** result) {
+  const int64_t rows = pl.rows_per_tile;
+  TmaCacheEntry* victim = &ctx->tma_cache[0];
+  for (auto& e : ctx->tma_cache) {
+    if (e.valid && e.mode == mode && e.w == w && e.B == B && e.S == S && e.H == H && e.D == D &&
+        e.rows == rows) {
+      bool same = true;
+      for (int k = 0; k < w && same; ++k) same = e.in[k] == in[k] && e.out[k] == out[k];
+      if (same) {
+        e.stamp = ++ctx->stamp;
+        e.params.stages = pl.stages;
+        *result = &e.params;
+        return ULYSSES_A2A_OK;
+      }
+    }
+    if (!e.valid || e.stamp < victim->stamp) victim = &e;
+  }
+  TmaCacheEntry fresh;
+  const int64_t Hw = H / w;
+  // mode 0 reads the strided side (inputs) and writes the gathered side (outputs);
+  // mode 1 the reverse
+  for (int k = 0; k < w; ++k) {
+    const void* strided = mode == 0 ? in[k] : out[k];
+    const void* gathered = mode == 0 ? out[k] : in[k];
+    int rc = encode_strided(ctx, &fresh.params.strided[k], strided, B, S, H, D, Hw, rows);
+    if (rc) return rc;
+    rc = encode_gathered(ctx, &fresh.params.gathered[k], gathered, B, S, Hw, D, w, rows);
+    if (rc) return rc;
+    fresh.in[k] = in[k];
+    fresh.out[k] = out[k];
+  }
+  fresh.valid = true;
+  fresh.stamp = ++ctx->stamp;
+  fresh.mode = mode;
+  fresh.w = w;
+  fresh.B = B;
+  fresh.S = S;
+  fresh.H = H;
+  fresh.D = D;
+  fresh.rows = rows;
+  TmaParams& p = fresh.params;
+  p.status = ctx->d_status;
+  p.w = w;
+  p.Hw = (int32_t)Hw;
+  p.rows_per_tile = (int32_t)rows;
+  p.tiles_per_block = (int32_t)pl.tiles_per_block;
+  p.tile_bytes = (uint32_t)(rows * pl.row_bytes);
+  p.stage_bytes = (uint32_t)((p.tile_bytes + 1023u) / 1024u * 1024u);
+  p.stages = pl.stages;
+  *victim = fresh;
+  *result = &victim->params;
+  return ULYSSES_A2A_OK;
+}
+
+// Every slab must sit in device memory of ctx's device, inside one allocation.
+int check_residency(ulysses_a2a_ctx* ctx, const void* const* ptrs, int w, int64_t bytes,
+                    const char* what) {
+  for (int k = 0; k < w; ++k) {
+    cudaPointerAttributes a;
+    cudaError_t e = cudaPointerGetAttributes(&a, ptrs[k]);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(ctx, ULYSSES_A2A_ERR_DEVICE, std::string(what) + " slab " + std::to_string(k) +
+                                                   ": not a CUDA pointer");
+    }
+    if (!(a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) || a.device != ctx->device)
+      return fail(ctx, ULYSSES_A2A_ERR_DEVICE, std::string(what) + " slab " + std::to_string(k) +
+                                                   " is not device memory of device " +
+                                                   std::to_string(ctx->device));
+    if (ctx->get_range && a.type == cudaMemoryTypeDevice) {
+      CUdeviceptr base = 0;
+      size_t size = 0;
+      if (ctx->get_range(&base, &size, (CUdeviceptr)(uintptr_t)ptrs[k]) == CUDA_SUCCESS) {
+        const uintptr_t p = (uintptr_t)ptrs[k];
+        if (p + (uintptr_t)bytes > (uintptr_t)base + size)
+          return fail(ctx, ULYSSES_A2A_ERR_DEVICE, std::string(what) + " slab " + std::to_string(k) +
+                                                       " runs past the end of its allocation");
+      }
+    }
+  }
+  return ULYSSES_A2A_OK;
+}
+
+template <typename V>
+cudaError_t launch_vec_t(const VecParams& p, int mode, int grid, int block, cudaStream_t st) {
+  if (mode == 0)
+    ua2a::ua2a_vec_kernel<V, 0, 4><<<grid, block, 0, st>>>(p);
+  else
+    ua2a::ua2a_vec_kernel<V, 1, 4><<<grid, block, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_vec(const VecParams& p, int vec_bytes, int mode, int grid, int block,
+                       cudaStream_t st) {
+  switch (vec_bytes) {
+    case 16: return launch_vec_t<uint4>(p, mode, grid, block, st);
+    case 8: return launch_vec_t<uint2>(p, mode, grid, block, st);
+    case 4: return launch_vec_t<unsigned int>(p, mode, grid, block, st);
+    case 2: return launch_vec_t<unsigned short>(p, mode, grid, block, st);
+    default: return launch_vec_t<unsigned char>(p, mode, grid, block, st);
+  }
+}
+
+int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, int64_t B, int64_t S,
+               int64_t H, int64_t D, int w, int mode, int chunked, cudaStream_t st,
+               const ulysses_a2a_plan_t& pl) {
+  const int64_t nb = chunked ? 1 : B;
+  const int launches = chunked ? (int)B : 1;
+  if (pl.path == ULYSSES_A2A_PATH_TMA) {
+    TmaParams* cached = nullptr;
+    int rc = tma_params_for(ctx, in, out, B, S, H, D, w, mode, pl, &cached);
+    if (rc) return rc;
+    TmaParams p = *cached;
+    p.status = ctx->d_status;
+    p.nb = (int32_t)nb;
+    p.units = pl.units;
+    const int mi = mode ? 1 : 0;
+    if (!ctx->tma_smem_set[mi] || ctx->tma_smem_set_bytes[mi] < pl.smem_bytes) {
+      cudaError_t e = mode == 0 ? cudaFuncSetAttribute(ua2a::ua2a_tma_kernel<0>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       (int)ua2a::kTmaSmemMax)
+                                : cudaFuncSetAttribute(ua2a::ua2a_tma_kernel<1>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       (int)ua2a::kTmaSmemMax);
+      if (e != cudaSuccess) return cuda_fail(ctx, "cudaFuncSetAttribute", e);
+      ctx->tma_smem_set[mi] = true;
+      ctx->tma_smem_set_bytes[mi] = ua2a::kTmaSmemMax;
+    }
+    for (int l = 0; l < launches; ++l) {
+      p.b0 = chunked ? l : 0;
+      if (mode == 0)
+        ua2a::ua2a_tma_kernel<0><<<pl.grid, pl.block, (size_t)pl.smem_bytes, st>>>(p);
+      else
+        ua2a::ua2a_tma_kernel<1><<<pl.grid, pl.block, (size_t)pl.smem_bytes, st>>>(p);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(ctx, "TMA kernel launch", e);
+      ctx->launches++;
+    }
+    return ULYSSES_A2A_OK;
+  }
+  VecParams p;
+  std::memset(&p, 0, sizeof(p));
+  for (int k = 0; k < w; ++k) {
+    p.in[k] = static_cast<const char*>(in[k]);
+    p.out[k] = static_cast<char*>(out[k]);
+  }
+  p.S_local = S;
+  p.nv = pl.row_bytes / pl.vec_bytes;
+  p.w = w;
+  p.rows_per_tile = (int32_t)pl.rows_per_tile;
+  p.units = (uint32_t)pl.units;
+  p.div_T = ua2a::FastDiv((uint32_t)pl.tiles_per_block);
+  p.div_w = ua2a::FastDiv((uint32_t)w);
+  p.div_nb = ua2a::FastDiv((uint32_t)nb);
+  p.div_nv = ua2a::FastDiv((uint32_t)p.nv);
+  for (int l = 0; l < launches; ++l) {
+    p.b0 = chunked ? l : 0;
+    cudaError_t e = launch_vec(p, pl.vec_bytes, mode, pl.grid, pl.block, st);
+    if (e != cudaSuccess) return cuda_fail(ctx, "VEC kernel launch", e);
+    ctx->launches++;
+  }
+  return ULYSSES_A2A_OK;
+}
+
+int plan_for(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, int64_t B, int64_t S,
+             int64_t H, int64_t D, int w, int mode, int chunked, ulysses_a2a_plan_t* pl) {
+  std::string err;
+  int rc = ua2a::make_plan(in, out, B, S, H, D, w, mode, chunked, ctx->elem_bytes, ctx->forced_path,
+                           ctx->tuning, ctx->num_sms, pl, &err);
+  if (rc) return fail(ctx, rc, err);
+  return ULYSSES_A2A_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ulysses_a2a_create(ulysses_a2a_ctx** out, int device, int elem_bytes) {
+  if (out == nullptr) return ULYSSES_A2A_ERR_INVALID;
+  *out = nullptr;
+  if (!(elem_bytes == 1 || elem_bytes == 2 || elem_bytes == 4 || elem_bytes == 8))
+    return ULYSSES_A2A_ERR_INVALID;
+  int count = 0;
+  if (cudaGetDeviceCount(&count) != cudaSuccess || device < 0 || device >= count) {
+    cudaGetLastError();
+    return ULYSSES_A2A_ERR_DEVICE;
+  }
+  ulysses_a2a_ctx* ctx = new (std::nothrow) ulysses_a2a_ctx();
+  if (!ctx) return ULYSSES_A2A_ERR_NOMEM;
+  ctx->device = device;
+  ctx->elem_bytes = elem_bytes;
+  DeviceGuard g(device);
+  if (!g.ok) {
+    delete ctx;
+    return ULYSSES_A2A_ERR_DEVICE;
+  }
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess || prop.major < 10) {
+    delete ctx;
+    return ULYSSES_A2A_ERR_DEVICE;  // built for sm_100a only
+  }
+  ctx->num_sms = prop.multiProcessorCount;
+  cudaDriverEntryPointQueryResult q;
+  void* fn = nullptr;
+  if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr) {
+    delete ctx;
+    return ULYSSES_A2A_ERR_CUDA;
+  }
+  ctx->encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  fn = nullptr;
+  if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &fn, 12000, cudaEnableDefault, &q) ==
+          cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    ctx->get_range = reinterpret_cast<PFN_cuMemGetAddressRange_v3020>(fn);
+  if (cudaMalloc(&ctx->d_status, 4 * sizeof(unsigned int)) != cudaSuccess) {
+    cudaGetLastError();
+    delete ctx;
+    return ULYSSES_A2A_ERR_NOMEM;
+  }
+  if (cudaMemset(ctx->d_status, 0, 4 * sizeof(unsigned int)) != cudaSuccess) {
+    cudaFree(ctx->d_status);
+    delete ctx;
+    return ULYSSES_A2A_ERR_CUDA;
+  }
+  // tuning knobs from the environment (for sweeps only; results never change)
+  ctx->tuning.rows_per_tile = env_int("ULYSSES_A2A_ROWS_PER_TILE", 0);
+  ctx->tuning.ctas_per_sm = env_int("ULYSSES_A2A_CTAS_PER_SM", 0);
+  ctx->tuning.stages = env_int("ULYSSES_A2A_STAGES", 0);
+  *out = ctx;
+  return ULYSSES_A2A_OK;
+}
+
+int ulysses_a2a_destroy(ulysses_a2a_ctx* ctx) {
+  if (ctx == nullptr) return ULYSSES_A2A_OK;
+  int rc = ULYSSES_A2A_OK;
+  {
+    DeviceGuard g(ctx->device);
+    if (cudaDeviceSynchronize() != cudaSuccess) rc = ULYSSES_A2A_ERR_CUDA;
+    if (ctx->d_status && cudaFree(ctx->d_status) != cudaSuccess) rc = ULYSSES_A2A_ERR_CUDA;
+    if (ctx->d_stage && cudaFree(ctx->d_stage) != cudaSuccess) rc = ULYSSES_A2A_ERR_CUDA;
+    cudaGetLastError();
+  }
+  delete ctx;  // the handle is consumed whatever the cleanup calls reported
+  return rc;
+}
+
+int ulysses_a2a_run(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void* const* out_slabs,
+                    int64_t B, int64_t S_local, int64_t H, int64_t D, int w, int mode, int chunked,
+                    void* stream) {
+  if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
+  ctx->last_error.clear();
+  ulysses_a2a_plan_t pl;
+  int rc = plan_for(ctx, in_slabs, out_slabs, B, S_local, H, D, w, mode, chunked, &pl);
+  if (rc) return rc;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "cannot select the context's device");
+  const int64_t slab_bytes = pl.payload_bytes / w;
+  rc = check_residency(ctx, in_slabs, w, slab_bytes, "input");
+  if (rc) return rc;
+  rc = check_residency(ctx, reinterpret_cast<const void* const*>(out_slabs), w, slab_bytes, "output");
+  if (rc) return rc;
+  return run_device(ctx, in_slabs, out_slabs, B, S_local, H, D, w, mode, chunked,
+                    static_cast<cudaStream_t>(stream), pl);
+}
+
+int ulysses_a2a_run_host(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void* const* out_slabs,
+                         int64_t B, int64_t S_local, int64_t H, int64_t D, int w, int mode,
+                         int chunked, void* stream) {
+  if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
+  ctx->last_error.clear();
+  // validate the host pointers (overlap, sizes) before touching the device
+  ulysses_a2a_plan_t host_pl;
+  int rc = plan_for(ctx, in_slabs, out_slabs, B, S_local, H, D, w, mode, chunked, &host_pl);
+  if (rc) return rc;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "cannot select the context's device");
+  const int64_t slab_bytes = host_pl.payload_bytes / w;
+  const size_t slot = ((size_t)slab_bytes + 255) / 256 * 256;
+  const size_t need = slot * 2 * (size_t)w;
+  if (ctx->stage_bytes < need) {
+    if (ctx->d_stage) {
+      cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+      if (e != cudaSuccess) return cuda_fail(ctx, "cudaStreamSynchronize", e);
+      cudaFree(ctx->d_stage);
+      ctx->d_stage = nullptr;
+      ctx->stage_bytes = 0;
+      for (auto& c : ctx->tma_cache) c.valid = false;  // maps may point into the old buffer
+    }
+    cudaError_t e = cudaMalloc(&ctx->d_stage, need);
+    if (e != cudaSuccess) {
+      ctx->d_stage = nullptr;
+      return cuda_fail(ctx, "cudaMalloc (host-path staging)", e);
+    }
+    ctx->stage_bytes = need;
+  }
+  std::vector<const void*> din(w);
+  std::vector<void*> dout(w);
+  char* base = static_cast<char*>(ctx->d_stage);
+  for (int k = 0; k < w; ++k) {
+    din[k] = base + slot * k;
+    dout[k] = base + slot * (w + k);
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int k = 0; k < w; ++k) {
+    cudaError_t e = cudaMemcpyAsync(const_cast<void*>(din[k]), in_slabs[k], (size_t)slab_bytes,
+                                    cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(ctx, "cudaMemcpyAsync H2D", e);
+  }
+  ulysses_a2a_plan_t pl;
+  rc = plan_for(ctx, din.data(), dout.data(), B, S_local, H, D, w, mode, chunked, &pl);
+  if (rc) return rc;
+  rc = run_device(ctx, din.data(), dout.data(), B, S_local, H, D, w, mode, chunked, st, pl);
+  if (rc) return rc;
+  for (int k = 0; k < w; ++k) {
+    cudaError_t e = cudaMemcpyAsync(out_slabs[k], dout[k], (size_t)slab_bytes,
+                                    cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return cuda_fail(ctx, "cudaMemcpyAsync D2H", e);
+  }
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(ctx, "cudaStreamSynchronize", e);
+  return ULYSSES_A2A_OK;
+}
+
+const char* ulysses_a2a_last_error(const ulysses_a2a_ctx* ctx) {
+  if (ctx == nullptr) return "NULL context";
+  return ctx->last_error.c_str();
+}
+
+int ulysses_a2a_status(ulysses_a2a_ctx* ctx, void* stream) {
+  if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
+  DeviceGuard g(ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(ctx, "cudaStreamSynchronize", e);
+  unsigned int h[4] = {0, 0, 0, 0};
+  e = cudaMemcpy(h, ctx->d_status, sizeof(h), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(ctx, "cudaMemcpy (status word)", e);
+  if (h[0] == 0) return ULYSSES_A2A_OK;
+  e = cudaMemset(ctx->d_status, 0, sizeof(h));
+  if (e != cudaSuccess) return cuda_fail(ctx, "cudaMemset (status word)", e);
+  char buf[160];
+  std::snprintf(buf, sizeof(buf),
+                "a TMA wait gave up (flags=0x%x, block %u, tile %u)%s", h[0],
+                h[1] ? h[1] - 1 : 0u, h[2],
+                (h[0] & ua2a::kStatusDrainTimeout) ? "; draining also timed out" : "");
+  return fail(ctx, ULYSSES_A2A_ERR_TIMEOUT, buf);
+}
+
+int ulysses_a2a_set_path(ulysses_a2a_ctx* ctx, int path) {
+  if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
+  if (path < ULYSSES_A2A_PATH_AUTO || path > ULYSSES_A2A_PATH_VEC)
+    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "unknown path");
+  ctx->forced_path = path;
+  return ULYSSES_A2A_OK;
+}
+
+int ulysses_a2a_set_tuning(ulysses_a2a_ctx* ctx, int rows_per_tile, int ctas_per_sm, int stages) {
+  if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
+  if (rows_per_tile < 0 || rows_per_tile > 256 || ctas_per_sm < 0 || ctas_per_sm > 32 ||
+      stages < 0 || stages == 1 || stages > ua2a::kTmaMaxStages)
+    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "tuning value out of range");
+  ctx->tuning.rows_per_tile = rows_per_tile;
+  ctx->tuning.ctas_per_sm = ctas_per_sm;
+  ctx->tuning.stages = stages;
+  return ULYSSES_A2A_OK;
+}
+
+uint64_t ulysses_a2a_launch_count(const ulysses_a2a_ctx* ctx) {
+  return ctx ? ctx->launches : 0;
+}
+
+int ulysses_a2a_plan(const void* const* in_slabs, void* const* out_slabs, int64_t B,
+                     int64_t S_local, int64_t H, int64_t D, int w, int mode, int chunked,
+                     int elem_bytes, int forced_path, int rows_per_tile, int ctas_per_sm,
+                     int stages, int num_sms, ulysses_a2a_plan_t* out, char* err, size_t errlen) {
+  ua2a::Tuning t;
+  t.rows_per_tile = rows_per_tile;
+  t.ctas_per_sm = ctas_per_sm;
+  t.stages = stages;
+  std::string msg;
+  int rc = ua2a::make_plan(in_slabs, out_slabs, B, S_local, H, D, w, mode, chunked, elem_bytes,
+                           forced_path, t, num_sms, out, &msg);
+  if (err && errlen) {
+    std::snprintf(err, errlen, "%s", rc ? msg.c_str() : "");
+  }
+  return rc;
+}
+
+}  // extern "C"

@@ -114,6 +114,12 @@ def rank_tagged_slabs(shape, w: int) -> list:
     return out
 
 
+def random_byte_slabs(shape, w: int, seed0: int = SEED0) -> list:
+    """w uint8 CPU tensors of ``shape``, uniform random bytes, rank k seeded seed0+k."""
+    return [torch.randint(0, 256, tuple(shape), dtype=torch.uint8, generator=_gen(seed0 + k))
+            for k in range(w)]
+
+
 def poison_like(t: torch.Tensor) -> torch.Tensor:
     """A tensor shaped like ``t`` with every byte 0xFF (an unwritten-output marker)."""
     out = torch.empty_like(t)

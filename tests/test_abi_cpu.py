@@ -1,0 +1,245 @@
+"""The C-ABI library without a GPU: it loads, exports what the header declares,
+and its host-only planner validates arguments and lays out work correctly."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from sequence_all_re_b200 import _lib
+from sequence_all_re_b200._lib import (ERR_INVALID, ERR_OVERLAP, ERR_UNSUPPORTED, OK, PATH_AUTO,
+                                       PATH_TMA, PATH_VEC, ulysses_a2a_plan)
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ulysses_a2a.h")
+
+MiB = 1 << 20
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ulysses_a2a_\w+)\s*\(", text)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    for n in ("ulysses_a2a_create", "ulysses_a2a_destroy", "ulysses_a2a_run"):
+        assert n in names
+    assert sorted(names) == sorted(_lib.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(_lib.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_plan_struct_layout_matches_header():
+    # int32 path, vec_bytes; 6 x int64; 4 x int32; int64 -> 8 + 48 + 16 + 8 = 80 bytes
+    assert ctypes.sizeof(_lib.PlanT) == 80
+
+
+def fake_slabs(w, slab_bytes, base=1 << 40, align=256, gap=0):
+    """Distinct, non-overlapping fake addresses (never dereferenced)."""
+    step = (slab_bytes + gap + align - 1) // align * align
+    ins = [base + k * step for k in range(w)]
+    outs = [base + (w + k) * step for k in range(w)]
+    return ins, outs
+
+
+def plan(w, B, S, H, D, mode=0, chunked=0, E=2, **kw):
+    ins, outs = fake_slabs(w, B * S * H * D * E)
+    return ulysses_a2a_plan(ins, outs, B, S, H, D, w, mode, chunked, E, **kw)
+
+
+# ---- geometry at the benchmark configurations -------------------------------
+
+def test_plan_cfg2_tma():
+    rc, p, msg = plan(4, 1, 8192, 24, 128)
+    assert rc == OK, msg
+    assert p.path == PATH_TMA
+    assert p.row_bytes == 6 * 128 * 2
+    assert p.rows_per_tile == 32 * 1024 // 1536       # 21 rows, ~32 KB
+    assert p.tiles_per_block == -(-8192 // 21)
+    assert p.tail_rows == 8192 % 21
+    assert p.units == 4 * 1 * 4 * p.tiles_per_block
+    assert p.payload_bytes == 192 * MiB
+    assert p.launches == 1 and p.block == 32
+    assert p.grid == 148
+    assert p.stages >= 2 and p.smem_bytes <= 220 * 1024
+
+
+def test_plan_cfg3_tail_rows():
+    rc, p, _ = plan(8, 2, 4725, 40, 128)
+    assert rc == OK and p.path == PATH_TMA
+    assert p.row_bytes == 5 * 128 * 2
+    assert p.rows_per_tile == 25 and p.tail_rows == 0          # 4725 = 189 * 25
+    rc, p, _ = plan(8, 2, 4725, 40, 128, rows_per_tile=32)
+    assert rc == OK
+    assert p.rows_per_tile == 32 and p.tail_rows == 4725 - 147 * 32 == 21
+    assert p.tiles_per_block == 148
+    assert p.units == 8 * 2 * 8 * 148
+    # a 64-row tile would be 80 KB: the TMA path caps tiles at 64 KB (51 rows)
+    rc, p, _ = plan(8, 2, 4725, 40, 128, rows_per_tile=64)
+    assert rc == OK and p.rows_per_tile == 51 and p.tail_rows == 4725 % 51
+    rc, p, _ = plan(8, 2, 4725, 40, 128, rows_per_tile=64, forced_path=PATH_VEC)
+    assert rc == OK and p.rows_per_tile == 64 and p.tail_rows == 53
+
+
+def test_plan_cfg4_chunked_launches():
+    rc, p, _ = plan(4, 4, 16384, 32, 64, chunked=1)
+    assert rc == OK and p.path == PATH_TMA
+    assert p.launches == 4
+    assert p.units == 4 * 1 * 4 * p.tiles_per_block     # one plane per launch
+    rc, q, _ = plan(4, 4, 16384, 32, 64, chunked=0)
+    assert q.launches == 1 and q.units == 4 * p.units
+    assert p.payload_bytes == q.payload_bytes == 1 << 30
+
+
+def test_plan_cfg1_small():
+    rc, p, _ = plan(2, 1, 64, 4, 64)
+    assert rc == OK and p.path == PATH_TMA
+    assert p.rows_per_tile == 64 and p.tail_rows == 0 and p.tiles_per_block == 1
+    assert p.units == 4 and p.grid == 4
+
+
+def test_rows_never_exceed_sequence():
+    rc, p, _ = plan(2, 1, 3, 2, 8)
+    assert rc == OK and p.rows_per_tile == 3 and p.tiles_per_block == 1
+
+
+# ---- path selection --------------------------------------------------------
+
+def test_vec_when_feature_bytes_not_16_aligned():
+    rc, p, _ = plan(2, 1, 16, 4, 3)             # D*E = 6 bytes
+    assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 4   # run = 2*3*2 = 12 B
+    rc, p, _ = plan(2, 1, 16, 2, 5, E=1)        # run = 5 B
+    assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 1
+
+
+def test_vec_when_misaligned_pointer():
+    w, B, S, H, D, E = 2, 1, 8, 4, 64, 2
+    ins, outs = fake_slabs(w, B * S * H * D * E)
+    outs[1] += 8
+    rc, p, _ = ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E)
+    assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 8
+    rc, p, msg = ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E, forced_path=PATH_TMA)
+    assert rc == ERR_UNSUPPORTED and "aligned" in msg
+
+
+def test_vec_when_too_many_ranks_for_tma():
+    rc, p, _ = plan(16, 1, 32, 16, 64)
+    assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 16
+    rc, p, msg = plan(16, 1, 32, 16, 64, forced_path=PATH_TMA)
+    assert rc == ERR_UNSUPPORTED
+
+
+def test_vec_when_box_dim_too_large():
+    rc, p, _ = plan(2, 1, 8, 2, 512)            # D = 512 > 256
+    assert rc == OK and p.path == PATH_VEC
+
+
+def test_forced_vec_geometry():
+    rc, p, _ = plan(4, 1, 8192, 24, 128, forced_path=PATH_VEC)
+    assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 16
+    assert p.block == 256 and p.grid == min(p.units, 148 * 8)
+
+
+def test_tuning_knobs():
+    rc, p, _ = plan(4, 1, 8192, 24, 128, rows_per_tile=16, stages=4, ctas_per_sm=2)
+    assert rc == OK and p.rows_per_tile == 16 and p.stages == 4 and p.grid == 296
+    assert p.smem_bytes == 4 * 24 * 1024
+
+
+# ---- argument validation ----------------------------------------------------
+
+@pytest.mark.parametrize("args,code", [
+    (dict(w=2, B=1, S=4, H=3, D=8), ERR_INVALID),        # H % w
+    (dict(w=2, B=0, S=4, H=4, D=8), ERR_INVALID),
+    (dict(w=2, B=1, S=0, H=4, D=8), ERR_INVALID),
+    (dict(w=2, B=1, S=4, H=4, D=0), ERR_INVALID),
+    (dict(w=0, B=1, S=4, H=4, D=8), ERR_INVALID),
+    (dict(w=65, B=1, S=4, H=65, D=8), ERR_INVALID),
+    (dict(w=2, B=1, S=4, H=4, D=8, mode=2), ERR_INVALID),
+    (dict(w=2, B=1, S=4, H=4, D=8, chunked=3), ERR_INVALID),
+    (dict(w=2, B=1, S=4, H=4, D=8, E=3), ERR_INVALID),
+])
+def test_rejects_bad_arguments(args, code):
+    a = dict(args)
+    w = a.pop("w")
+    B, S, H, D = a.pop("B"), a.pop("S"), a.pop("H"), a.pop("D")
+    mode, chunked, E = a.pop("mode", 0), a.pop("chunked", 0), a.pop("E", 2)
+    ins, outs = fake_slabs(max(w, 1), max(B * S * H * D * E, 1))
+    rc, _, msg = ulysses_a2a_plan(ins[:max(w, 0)] or [0], outs[:max(w, 0)] or [0], B, S, H, D, w,
+                                  mode, chunked, E)
+    assert rc == code and msg
+
+
+def test_rejects_size_overflow():
+    ins, outs = fake_slabs(2, 16)
+    rc, _, msg = ulysses_a2a_plan(ins, outs, 1 << 40, 1 << 20, 2, 8, 2, 0, 0, 2)
+    assert rc == ERR_INVALID and "overflow" in msg
+
+
+def test_rejects_null_pointers():
+    rc, _, _ = ulysses_a2a_plan(None, None, 1, 1, 2, 1, 2, 0, 0, 2)
+    assert rc == ERR_INVALID
+    ins, outs = fake_slabs(2, 64)
+    ins[1] = 0
+    rc, _, msg = ulysses_a2a_plan(ins, outs, 1, 4, 2, 4, 2, 0, 0, 2)
+    assert rc == ERR_INVALID and "NULL" in msg
+
+
+def test_rejects_output_overlapping_input():
+    w, B, S, H, D, E = 2, 1, 4, 4, 8, 2
+    nbytes = B * S * H * D * E
+    ins, outs = fake_slabs(w, nbytes)
+    outs[0] = ins[1] + nbytes - 2             # last element of input 1 shared
+    rc, _, msg = ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E)
+    assert rc == ERR_OVERLAP and "input" in msg
+    outs[0] = ins[1] + nbytes                 # touching but disjoint: fine
+    outs[1] = outs[0] + nbytes
+    rc, _, _ = ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E)
+    assert rc == OK
+
+
+def test_rejects_outputs_overlapping_each_other_and_in_place():
+    w, B, S, H, D, E = 2, 1, 4, 4, 8, 2
+    nbytes = B * S * H * D * E
+    ins, outs = fake_slabs(w, nbytes)
+    outs[1] = outs[0] + 16
+    rc, _, msg = ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E)
+    assert rc == ERR_OVERLAP and "output" in msg
+    rc, _, _ = ulysses_a2a_plan(ins, ins, B, S, H, D, w, 0, 0, E)   # in place
+    assert rc == ERR_OVERLAP
+
+
+def test_inputs_may_alias_each_other():
+    w, B, S, H, D, E = 2, 1, 4, 4, 8, 2
+    ins, outs = fake_slabs(w, B * S * H * D * E)
+    ins[1] = ins[0]
+    rc, _, _ = ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E)
+    assert rc == OK
+
+
+# ---- entry points that need no GPU ------------------------------------------
+
+def test_null_context_handling():
+    lib = _lib.lib
+    assert lib.ulysses_a2a_destroy(None) == OK
+    assert lib.ulysses_a2a_launch_count(None) == 0
+    assert lib.ulysses_a2a_last_error(None) == b"NULL context"
+    assert lib.ulysses_a2a_set_path(None, PATH_AUTO) == ERR_INVALID
+    assert lib.ulysses_a2a_set_tuning(None, 0, 0, 0) == ERR_INVALID
+    arr = _lib.ptr_array([1, 2])
+    assert lib.ulysses_a2a_run(None, arr, arr, 1, 1, 2, 1, 2, 0, 0, None) == ERR_INVALID
+    assert lib.ulysses_a2a_run_host(None, arr, arr, 1, 1, 2, 1, 2, 0, 0, None) == ERR_INVALID
+    assert lib.ulysses_a2a_status(None, None) == ERR_INVALID
+
+
+def test_create_rejects_bad_element_size_before_touching_cuda():
+    h = ctypes.c_void_p()
+    assert _lib.lib.ulysses_a2a_create(ctypes.byref(h), 0, 3) == ERR_INVALID
+    assert _lib.lib.ulysses_a2a_create(None, 0, 2) == ERR_INVALID

@@ -1,0 +1,347 @@
+"""CUDA path vs the CPU oracle, bit for bit (needs a B200).
+
+Every output slab sits inside a larger buffer: the slab itself is pre-filled
+with 0xFF (an element the kernel never writes stays wrong) and the bytes before
+and after it hold a canary pattern that must survive the run (a write past
+either end of a slab is caught). Inputs come from ``synth`` with fixed seeds;
+expected values come from ``oracle`` only.
+"""
+
+import pytest
+import torch
+
+import oracle
+from sequence_all_re_b200 import A2AError, PATH_AUTO, PATH_TMA, PATH_VEC, UlyssesA2A, _lib
+from synth import (normal_slabs, random_byte_slabs, rank_tagged_slabs, slab_shape, uniform_slabs,
+                   unique_slabs)
+
+pytestmark = pytest.mark.gpu
+
+GUARD = 4096          # canary bytes on each side of an output slab (keeps 256 B alignment)
+CANARY = 0xA5
+
+INT_OF = {1: torch.uint8, 2: torch.int16, 4: torch.int32, 8: torch.int64}
+
+
+def bits(t):
+    return t.contiguous().view(INT_OF[t.element_size()])
+
+
+class Guarded:
+    """w output slabs, each poisoned and surrounded by canary bytes."""
+
+    def __init__(self, shape, dtype, w, device="cuda", offset=0):
+        n = 1
+        for v in shape:
+            n *= v
+        esz = torch.empty((), dtype=dtype).element_size()
+        self.nbytes = n * esz
+        self.offset = offset
+        self.bufs, self.slabs = [], []
+        for _ in range(w):
+            buf = torch.full((self.nbytes + 2 * GUARD + offset,), CANARY, dtype=torch.uint8,
+                             device=device)
+            lo = GUARD + offset
+            buf[lo:lo + self.nbytes].fill_(0xFF)
+            self.bufs.append(buf)
+            self.slabs.append(buf[lo:lo + self.nbytes].view(dtype).view(shape))
+
+    def check_guards(self):
+        for buf in self.bufs:
+            lo = GUARD + self.offset
+            head = buf[:lo]
+            tail = buf[lo + self.nbytes:]
+            assert bool((head == CANARY).all()), "bytes before an output slab were written"
+            assert bool((tail == CANARY).all()), "bytes after an output slab were written"
+
+
+def run_case(xs_cpu, mode, *, chunked=False, path=PATH_AUTO, tuning=None, a2a=None,
+             out_offset=0, in_offset=0):
+    """Run the GPU path on xs_cpu (moved to the device) and compare with the oracle."""
+    w = len(xs_cpu)
+    E = xs_cpu[0].element_size()
+    own = a2a is None
+    a2a = a2a or UlyssesA2A(0, E)
+    try:
+        a2a.set_path(path)
+        a2a.set_tuning(*(tuning or (0, 0, 0)))
+        if in_offset:
+            xs = []
+            for t in xs_cpu:
+                raw = torch.empty(t.numel() * E + in_offset, dtype=torch.uint8, device="cuda")
+                v = raw[in_offset:].view(t.dtype).view(t.shape)
+                v.copy_(t)
+                xs.append(v)
+        else:
+            xs = [t.cuda() for t in xs_cpu]
+        oshape = oracle.output_shape(tuple(xs_cpu[0].shape), mode, w)
+        g = Guarded(oshape, xs_cpu[0].dtype, w, offset=out_offset)
+        before = a2a.launch_count
+        a2a.run(xs, mode, chunked=chunked, out=g.slabs)
+        a2a.status()
+        B = xs_cpu[0].shape[0]
+        assert a2a.launch_count - before == (B if chunked else 1)
+        want = oracle.ulysses_a2a(xs_cpu, mode, chunked=False)
+        for k in range(w):
+            got = g.slabs[k].cpu()
+            assert torch.equal(bits(got), bits(want[k])), f"rank {k} differs from the oracle"
+        g.check_guards()
+        return [s.cpu() for s in g.slabs]
+    finally:
+        if own:
+            a2a.close()
+
+
+# ---- small and medium shapes: several tiles, ragged tails, both paths -------
+
+SHAPES = [
+    # (w, B, S_local, H, D)
+    (2, 1, 64, 4, 64),          # the small oracle-size case
+    (2, 3, 37, 4, 64),          # ragged S_local, several planes
+    (4, 2, 100, 8, 128),
+    (8, 2, 53, 40, 128),        # cfg3's head geometry, short sequence
+    (3, 2, 29, 6, 32),          # odd rank count
+    (1, 2, 33, 4, 64),          # w = 1: identity copy
+    (8, 1, 7, 8, 256),          # D at the TMA box limit, H/w = 1
+]
+
+TUNINGS = [(0, 0, 0), (7, 0, 2), (16, 2, 3), (1, 1, 2)]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "w{}B{}S{}H{}D{}".format(*s))
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("path", [PATH_TMA, PATH_VEC], ids=["tma", "vec"])
+def test_parity_small(shape, mode, path):
+    w, B, S, H, D = shape
+    xs = normal_slabs(slab_shape(mode, w, B, S, H, D), w, "bf16", seed0=100 + mode)
+    a2a = UlyssesA2A(0, 2)
+    try:
+        for tuning in TUNINGS:
+            for chunked in (False, True):
+                run_case(xs, mode, chunked=chunked, path=path, tuning=tuning, a2a=a2a)
+    finally:
+        a2a.close()
+
+
+@pytest.mark.parametrize("E", [1, 2, 4, 8])
+@pytest.mark.parametrize("path", [PATH_TMA, PATH_VEC], ids=["tma", "vec"])
+def test_parity_unique_ids_every_element_size(E, path):
+    # every element distinct: a misplaced element can never match by chance.
+    # D*E = 32 bytes keeps every element size expressible by the TMA path.
+    if E == 1:
+        w, B, S, H, D = 2, 1, 2, 2, 32        # 256 ids fill a byte exactly
+    else:
+        w, B, S, H, D = 4, 2, 19, 8, 32 // E
+    xs = unique_slabs((B, S, H, D), w, E)
+    for mode in (0, 1):
+        xin = xs if mode == 0 else oracle.ulysses_a2a(xs, 0)
+        run_case(xin, mode, path=path, tuning=(5, 0, 2))
+        run_case(xin, mode, path=path, tuning=(1, 0, 2), chunked=True)
+
+
+def test_parity_fp32_uniform():
+    w, B, S, H, D = 4, 2, 45, 8, 128
+    for mode in (0, 1):
+        xs = uniform_slabs(slab_shape(mode, w, B, S, H, D), w, "fp32", seed0=7)
+        run_case(xs, mode)
+        run_case(xs, mode, path=PATH_VEC)
+
+
+def test_parity_rank_tagged_bf16_width():
+    w, B, S, H, D = 8, 2, 33, 16, 64
+    xs = rank_tagged_slabs((B, S, H, D), w)
+    y = run_case(xs, 0)
+    run_case(y, 1)
+
+
+def test_round_trip_on_device():
+    w, B, S, H, D = 4, 2, 77, 8, 64
+    xs = normal_slabs((B, S, H, D), w, "bf16", seed0=5)
+    with UlyssesA2A(0, 2) as a2a:
+        xd = [t.cuda() for t in xs]
+        y = a2a.run(xd, 0)
+        z = a2a.run(y, 1)
+        a2a.status()
+        for k in range(w):
+            assert torch.equal(bits(z[k].cpu()), bits(xs[k]))
+
+
+def test_nan_payloads_and_signed_zero_survive():
+    w, B, S, H, D = 2, 1, 8, 2, 8
+    xs = normal_slabs((B, S, H, D), w, "fp32", seed0=9)
+    b0 = xs[0].view(torch.int32)
+    b0.view(-1)[0] = 0x7FC01234
+    b0.view(-1)[3] = 0x7F800001
+    xs[1].view(torch.int32).view(-1)[5] = -(2 ** 31)
+    for path in (PATH_TMA, PATH_VEC):
+        run_case(xs, 0, path=path)
+
+
+# ---- alignment: misaligned slabs take the narrower vector path --------------
+
+@pytest.mark.parametrize("offset,vec", [(8, 8), (4, 4), (2, 2), (1, 1)])
+def test_misaligned_pointers_select_narrower_vectors(offset, vec):
+    w, B, S, H, D = 2, 2, 21, 4, 64
+    E = 2 if offset % 2 == 0 else 1
+    if E == 2:
+        xs = normal_slabs((B, S, H, D), w, "bf16", seed0=3)
+    else:
+        xs = random_byte_slabs((B, S, H, D * 2), w, seed0=3)
+    with UlyssesA2A(0, E) as a2a:
+        xd = [t.cuda() for t in xs]
+        g = Guarded(oracle.output_shape(tuple(xs[0].shape), 0, w), xs[0].dtype, w, offset=offset)
+        plan = a2a.plan(xd, 0, out=g.slabs)
+        assert plan["path"] == PATH_VEC and plan["vec_bytes"] == vec
+    run_case(xs, 0, out_offset=offset)
+    run_case(xs, 0, in_offset=offset)
+
+
+def test_shapes_tma_cannot_express_use_vec():
+    # D*E = 6 bytes: rows of 12 bytes, VEC path with 4-byte vectors
+    w, B, S, H, D = 2, 2, 17, 4, 3
+    for mode in (0, 1):
+        xs = normal_slabs(slab_shape(mode, w, B, S, H, D), w, "bf16", seed0=1)
+        run_case(xs, mode)
+        run_case(xs, mode, chunked=True)
+    # w = 16 exceeds the TMA descriptor table
+    w, B, S, H, D = 16, 1, 9, 16, 64
+    xs = normal_slabs((B, S, H, D), w, "bf16", seed0=2)
+    run_case(xs, 0)
+    with pytest.raises(A2AError):
+        run_case(xs, 0, path=PATH_TMA)
+
+
+# ---- the benchmark's configurations at full size (default launch config) ----
+
+FULL = {
+    "cfg1_w2_S64": (2, 1, 64, 4, 64),
+    "cfg2_w4_S8192": (4, 1, 8192, 24, 128),
+    "cfg3_w8_S4725": (8, 2, 4725, 40, 128),
+    "cfg4_w4_B4_S16384": (4, 4, 16384, 32, 64),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FULL))
+def test_full_size_configs(name):
+    w, B, S, H, D = FULL[name]
+    xs = normal_slabs((B, S, H, D), w, "bf16")
+    y = run_case(xs, 0)
+    run_case(y, 1)
+    if B > 1:
+        run_case(xs, 0, chunked=True)
+        run_case(y, 1, chunked=True)
+    if name.startswith("cfg3"):
+        # the ragged tile: 4725 = 147 * 32 + 21
+        run_case(xs, 0, tuning=(32, 0, 0))
+        run_case(y, 1, tuning=(32, 0, 0), path=PATH_VEC)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("w", [2, 4, 8])
+def test_sweep_points(dtype, w):
+    # bandwidth-sweep geometry: D = 128, H = 8w, B = 1, S_local set by the payload
+    E = 2 if dtype == "bf16" else 4
+    H, D = 8 * w, 128
+    for payload in (256 << 10, 8 << 20, 64 << 20):
+        S = payload // (w * H * D * E)
+        if S < 1:
+            continue
+        for mode in (0, 1):
+            xs = uniform_slabs(slab_shape(mode, w, 1, S, H, D), w, dtype, seed0=payload % 1000)
+            run_case(xs, mode)
+
+
+# ---- the host-buffer entry point -------------------------------------------
+
+def test_run_host_matches_oracle():
+    w, B, S, H, D = 4, 2, 300, 8, 128
+    with UlyssesA2A(0, 2) as a2a:
+        for mode in (0, 1):
+            xs = normal_slabs(slab_shape(mode, w, B, S, H, D), w, "bf16", seed0=21)
+            pinned = [t.pin_memory() for t in xs]
+            for src in (xs, pinned):
+                out = a2a.run_host(src, mode)
+                want = oracle.ulysses_a2a(xs, mode)
+                for k in range(w):
+                    assert torch.equal(bits(out[k]), bits(want[k]))
+        # the staging buffers grow on demand
+        xs = normal_slabs((B, 2 * S, H, D), w, "bf16", seed0=22)
+        out = a2a.run_host(xs, 0, chunked=True)
+        want = oracle.ulysses_a2a(xs, 0)
+        for k in range(w):
+            assert torch.equal(bits(out[k]), bits(want[k]))
+
+
+# ---- argument errors on a live device: nothing is launched ------------------
+
+def test_errors_launch_nothing():
+    w, B, S, H, D = 2, 1, 8, 4, 64
+    with UlyssesA2A(0, 2) as a2a:
+        xs = [t.cuda() for t in normal_slabs((B, S, H, D), w, "bf16")]
+        outs = [torch.empty(B, S * w, H // w, D, dtype=torch.bfloat16, device="cuda")
+                for _ in range(w)]
+        n0 = a2a.launch_count
+        # a host pointer where device memory is required
+        host = [t.cpu() for t in outs]
+        with pytest.raises(A2AError) as e:
+            _raise(a2a, _lib.ulysses_a2a_run(a2a._ctx, [t.data_ptr() for t in xs],
+                                             [t.data_ptr() for t in host], B, S, H, D, w, 0, 0, 0))
+        assert e.value.code == _lib.ERR_DEVICE
+        # output overlapping an input
+        rc = _lib.ulysses_a2a_run(a2a._ctx, [t.data_ptr() for t in xs],
+                                  [xs[0].data_ptr(), outs[1].data_ptr()], B, S, H, D, w, 0, 0, 0)
+        assert rc == _lib.ERR_OVERLAP and "overlaps" in a2a.last_error()
+        # H not divisible by w
+        rc = _lib.ulysses_a2a_run(a2a._ctx, [t.data_ptr() for t in xs],
+                                  [t.data_ptr() for t in outs], B, S, 3, D, w, 0, 0, 0)
+        assert rc == _lib.ERR_INVALID
+        assert a2a.launch_count == n0
+        # the context still works after the rejected calls
+        a2a.run(xs, 0, out=outs)
+        a2a.status()
+        assert a2a.launch_count == n0 + 1
+
+
+def _raise(a2a, rc):
+    if rc != _lib.OK:
+        raise A2AError(rc, a2a.last_error())
+
+
+def test_slab_past_end_of_allocation_is_rejected():
+    from cuda.bindings import runtime as rt
+
+    w, B, S, H, D = 2, 1, 64, 4, 64
+    nbytes = B * S * H * D * 2
+    size = 4 << 20
+    err, base = rt.cudaMalloc(size)            # a dedicated allocation of known extent
+    assert err == rt.cudaError_t.cudaSuccess
+    try:
+        with UlyssesA2A(0, 2) as a2a:
+            xs = [t.cuda() for t in normal_slabs((B, S, H, D), w, "bf16")]
+            out0 = torch.empty(B, S * w, H // w, D, dtype=torch.bfloat16, device="cuda")
+            n0 = a2a.launch_count
+            # second output starts half a slab before the allocation's end
+            rc = _lib.ulysses_a2a_run(a2a._ctx, [t.data_ptr() for t in xs],
+                                      [out0.data_ptr(), int(base) + size - nbytes // 2],
+                                      B, S, H, D, w, 0, 0, 0)
+            assert rc == _lib.ERR_DEVICE and "past the end" in a2a.last_error()
+            # the same slab placed wholly inside the allocation is accepted
+            rc = _lib.ulysses_a2a_run(a2a._ctx, [t.data_ptr() for t in xs],
+                                      [out0.data_ptr(), int(base) + size - nbytes],
+                                      B, S, H, D, w, 0, 0, 0)
+            assert rc == _lib.OK
+            a2a.status()
+            assert a2a.launch_count == n0 + 1
+    finally:
+        torch.cuda.synchronize()
+        rt.cudaFree(base)
+
+
+def test_status_is_clean_and_destroy_is_idempotent_on_null():
+    a2a = UlyssesA2A(0, 2)
+    xs = [t.cuda() for t in normal_slabs((1, 16, 4, 64), 2, "bf16")]
+    a2a.run(xs, 0)
+    a2a.status()
+    a2a.close()
+    a2a.close()
+    assert _lib.lib.ulysses_a2a_destroy(None) == _lib.OK
