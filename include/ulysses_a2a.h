@@ -159,6 +159,40 @@ int ulysses_a2a_plan(const void *const *in_slabs, void *const *out_slabs,
                      int num_sms, ulysses_a2a_plan_t *out, char *err,
                      size_t errlen);
 
+/* Allocation-free variant of ulysses_a2a_run (the pages have no counterpart:
+ * this entry point exists for this library's users, not for the method).
+ *
+ * Who needs it: callers that must not allocate device memory themselves, e.g.
+ * a process whose device memory is owned by another allocator under a fixed
+ * budget, or host code running where a cudaMalloc/cudaFree (which may
+ * synchronise the whole device) is not allowed. ulysses_a2a_create allocates
+ * the TMA kernel's status records; this call needs no context and allocates
+ * nothing: it keeps those records in a file-scope static device array of 64
+ * records x 16 bytes (1 KiB), one record per kernel launch, which every GPU
+ * that loads the library holds until the process exits.
+ *
+ * Arguments and layout as ulysses_a2a_run, plus elem_bytes (1, 2, 4 or 8). It
+ * runs on the CURRENT CUDA device, which must hold every slab. The caller still
+ * owns all inputs and outputs.
+ *   wait = 0 : return once the work is queued on `stream`.
+ *   wait = 1 : also synchronise `stream` and check the status records;
+ *              returns ULYSSES_A2A_ERR_TIMEOUT if a kernel gave up a wait.
+ *   err      : optional buffer (errlen bytes) for a message on failure.
+ * Limit: a chunked call launches once per plane and needs one record per
+ * plane, so chunked calls over more than 64 planes are rejected with
+ * ULYSSES_A2A_ERR_UNSUPPORTED and a message (unchunked calls need one record).
+ *
+ * The first call on a device also does a one-time set-up for that device
+ * (resolving the array's device address and the kernels' shared-memory limit);
+ * make that first call before any stream capture. Every call shares the array
+ * and the array keeps the last call's contents: each call clears the records
+ * it uses, on `stream`, before its kernels run, so calls whose work overlaps
+ * on the GPU (other streams, other host threads) race on the records. */
+int ulysses_a2a_run_noalloc(const void *const *in_slabs, void *const *out_slabs,
+                            int64_t B, int64_t S_local, int64_t H, int64_t D,
+                            int w, int mode, int chunked, int elem_bytes,
+                            void *stream, int wait, char *err, size_t errlen);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif

@@ -40,6 +40,7 @@ EXPORTED = (
     "ulysses_a2a_set_tuning",
     "ulysses_a2a_launch_count",
     "ulysses_a2a_plan",
+    "ulysses_a2a_run_noalloc",
 )
 
 
@@ -105,6 +106,9 @@ def _load() -> ctypes.CDLL:
                                      c_int, c_int, c_int, c_int, c_int,
                                      ctypes.POINTER(PlanT), ctypes.c_char_p, ctypes.c_size_t]
     lib.ulysses_a2a_plan.restype = c_int
+    lib.ulysses_a2a_run_noalloc.argtypes = [PP, PP, i64, i64, i64, i64, c_int, c_int, c_int, c_int,
+                                            P, c_int, ctypes.c_char_p, ctypes.c_size_t]
+    lib.ulysses_a2a_run_noalloc.restype = c_int
     return lib
 
 
@@ -160,6 +164,17 @@ def ulysses_a2a_set_tuning(ctx, rows_per_tile: int = 0, ctas_per_sm: int = 0, st
 
 def ulysses_a2a_launch_count(ctx) -> int:
     return int(lib.ulysses_a2a_launch_count(ctx))
+
+
+def ulysses_a2a_run_noalloc(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, elem_bytes,
+                            stream, wait=1):
+    """The allocation-free entry point (current device). Returns (rc, message)."""
+    buf = ctypes.create_string_buffer(256)
+    rc = lib.ulysses_a2a_run_noalloc(ptr_array(in_ptrs), ptr_array(out_ptrs), int(B), int(S_local),
+                                     int(H), int(D), int(w), int(mode), int(chunked),
+                                     int(elem_bytes), ctypes.c_void_p(int(stream)), int(wait),
+                                     buf, len(buf))
+    return rc, buf.value.decode()
 
 
 def ulysses_a2a_plan(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, elem_bytes,
