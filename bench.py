@@ -8,9 +8,12 @@ tile scheduler, copy kernel). Workload: w=4, B=1, S_local=8192, H=24, D=128,
 bf16, N(0,1) values (payload P = 192 MiB per call).
 
 Metric: payload GB/s (P per call / device time, 1 GB = 1e9 B) and the fraction
-of the measured HBM copy bandwidth, counting 2P bytes moved per call. The L2 is
-flushed (a write of 2x its size) before every timed call, outside the timed
-interval; each call is timed with CUDA events on its stream.
+of the measured HBM copy bandwidth, counting 2P bytes moved per call. The K
+steps run back to back between two CUDA events on the launching stream. Every
+input (192 MiB per call) is larger than the 126 MB L2, and mode 1 reads its own
+input slabs rather than mode 0's fresh output, so no kernel reads what the
+kernel before it touched. As a cross-check, each mode is also timed call by
+call after a 2x-L2 write flush (per-call events, ~2 us resolution).
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own independent
 instance of the workload (the w logical ranks all live in one GPU's memory, so
@@ -151,45 +154,72 @@ def make_inputs(w, B, S, H, D, dtype, device, seed0=1234):
     return xs
 
 
-def timed_calls(a2a, xs, ys, flush, steps, warmup, stream, sampler=None):
-    """Per-call device times (ms) of mode 0 (xs->ys) and mode 1 (ys->xs2) over `steps` steps."""
-    xs2 = [torch.empty_like(t) for t in xs]
+def timed_steps(a2a, x, y, y2, z, steps, warmup, stream, sampler=None):
+    """K back-to-back steps (mode 0: x -> y, mode 1: y2 -> z) between one pair of events.
+
+    Returns (total ms, launches of our kernels in the timed region, clocks)."""
     for _ in range(warmup):
-        a2a.run(xs, 0, out=ys, stream=stream)
-        a2a.run(ys, 1, out=xs2, stream=stream)
+        a2a.run(x, 0, out=y, stream=stream)
+        a2a.run(y2, 1, out=z, stream=stream)
     torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
     launches0 = a2a.launch_count
     if sampler:
         sampler.start()
-    with torch.cuda.stream(stream):
-        for i in range(steps):
-            flush.fill_(i & 0xFF)
-            ev[i][0].record(stream)
-            a2a.run(xs, 0, out=ys, stream=stream)
-            ev[i][1].record(stream)
-            flush.fill_((i + 1) & 0xFF)
-            ev[i][2].record(stream)
-            a2a.run(ys, 1, out=xs2, stream=stream)
-            ev[i][3].record(stream)
+    e0.record(stream)
+    for _ in range(steps):
+        a2a.run(x, 0, out=y, stream=stream)
+        a2a.run(y2, 1, out=z, stream=stream)
+    e1.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
-    launches = a2a.launch_count - launches0
-    t0 = [ev[i][0].elapsed_time(ev[i][1]) for i in range(steps)]
-    t1 = [ev[i][2].elapsed_time(ev[i][3]) for i in range(steps)]
-    return t0, t1, launches, clocks, xs2
+    return e0.elapsed_time(e1), a2a.launch_count - launches0, clocks
 
 
-def bench_sweep_point(a2a, w, payload, dtype, device, flush, stream, reps):
+def timed_mode(a2a, src, dst, mode, reps, stream):
+    """Back-to-back calls of one mode between one pair of events; ms per call."""
+    for _ in range(3):
+        a2a.run(src, mode, out=dst, stream=stream)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        a2a.run(src, mode, out=dst, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def timed_flushed(a2a, src, dst, mode, flush, reps, stream):
+    """Median per-call time (ms) with a 2x-L2 write flush before every call."""
+    for _ in range(3):
+        a2a.run(src, mode, out=dst, stream=stream)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    with torch.cuda.stream(stream):
+        for i in range(reps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            a2a.run(src, mode, out=dst, stream=stream)
+            ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+
+def bench_sweep_point(a2a, w, payload, dtype, device, stream, reps):
     E = 2 if dtype == "bf16" else 4
     H, D = 8 * w, 128
     S = payload // (w * H * D * E)
-    xs = make_inputs(w, 1, S, H, D, dtype, device)
-    ys = [torch.empty((1, S * w, H // w, D), dtype=xs[0].dtype, device=device) for _ in range(w)]
-    t0, t1, _, _, _ = timed_calls(a2a, xs, ys, flush, reps, 3, stream)
+    x = make_inputs(w, 1, S, H, D, dtype, device)
+    y = [torch.empty((1, S * w, H // w, D), dtype=x[0].dtype, device=device) for _ in range(w)]
+    t0 = timed_mode(a2a, x, y, 0, reps, stream)
+    t1 = timed_mode(a2a, y, x, 1, reps, stream)
     P = w * S * H * D * E
-    del xs, ys
-    return P, statistics.median(t0), statistics.median(t1)
+    del x, y
+    return P, t0, t1
 
 
 def cpu_oracle_baseline(w, B, S, H, D, budget_s=12.0):
@@ -233,26 +263,30 @@ def run_ours(args):
     P = w * B * S * H * D * E
     a2a = UlyssesA2A(local_rank, E)
     stream = torch.cuda.Stream(device)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-    xs = make_inputs(w, B, S, H, D, "bf16", device)
-    ys = [torch.empty((B, S * w, H // w, D), dtype=torch.bfloat16, device=device) for _ in range(w)]
-    plan = a2a.plan(xs, 0, out=ys)
+    x = make_inputs(w, B, S, H, D, "bf16", device)
+    y = [torch.empty((B, S * w, H // w, D), dtype=torch.bfloat16, device=device) for _ in range(w)]
+    z = [torch.empty_like(t) for t in x]
+    # mode 1 reads its own slabs (a seeded copy of mode 0's result), not y
+    with torch.cuda.stream(stream):
+        a2a.run(x, 0, out=y, stream=stream)
+    torch.cuda.synchronize()
+    y2 = [t.clone() for t in y]
+    plan = a2a.plan(x, 0, out=y)
 
     sampler = ClockSampler(local_rank)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    t0, t1, launches, clocks, xs2 = timed_calls(a2a, xs, ys, flush, args.steps, args.warmup,
-                                                stream, sampler)
+    total_ms, launches, clocks = timed_steps(a2a, x, y, y2, z, args.steps, args.warmup, stream,
+                                             sampler)
     a2a.status(stream)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    # round trip must reproduce the input bit for bit (cheap on-device check)
+    # the round trip must reproduce the input bit for bit (y2 holds mode 0's output)
     for k in range(w):
-        if not torch.equal(xs2[k].view(torch.int16), xs[k].view(torch.int16)):
+        if not torch.equal(z[k].view(torch.int16), x[k].view(torch.int16)):
             raise SystemExit("round trip mismatch: mode1(mode0(x)) != x")
-    total_ms = sum(t0) + sum(t1)
     if dist:
         t = torch.tensor([total_ms], device=device, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -261,11 +295,7 @@ def run_ours(args):
     value = world * 2 * P * args.steps / (total_ms / 1e3) / 1e9
 
     peak, peak_src = hbm_peak()
-    m0 = statistics.mean(t0)
-    m1 = statistics.mean(t1)
-    gbs0 = P / (m0 / 1e3) / 1e9
-    gbs1 = P / (m1 / 1e3) / 1e9
-    avg_launch_ms = (m0 + m1) / 2
+    avg_launch_ms = total_ms / launches
     achieved = 2 * P / (avg_launch_ms / 1e3) / 1e9
     khash = kernel_source_hash()
     traffic, traffic_src = ncu_traffic(khash)
@@ -274,10 +304,25 @@ def run_ours(args):
         traffic_bytes = traffic.get("workloads", {}).get("w4_B1_S8192_H24_D128_bf16", {}).get(
             "dram_bytes_per_launch")
 
+    # per mode: back to back, and call by call after an L2 write flush
+    reps = max(20, min(args.steps, 400))
+    m0 = timed_mode(a2a, x, y, 0, reps, stream)
+    m1 = timed_mode(a2a, y2, z, 1, reps, stream)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    f0 = timed_flushed(a2a, x, y, 0, flush, reps, stream)
+    f1 = timed_flushed(a2a, y2, z, 1, flush, reps, stream)
+    del flush
+    gbs = lambda ms: P / (ms / 1e3) / 1e9
+    per_mode = {"mode0_gbs": round(gbs(m0), 1), "mode1_gbs": round(gbs(m1), 1),
+                "mode0_frac": round(2 * gbs(m0) / peak, 4), "mode1_frac": round(2 * gbs(m1) / peak, 4),
+                "flushed_mode0_gbs": round(gbs(f0), 1), "flushed_mode1_gbs": round(gbs(f1), 1),
+                "flushed_mode0_frac": round(2 * gbs(f0) / peak, 4),
+                "flushed_mode1_frac": round(2 * gbs(f1) / peak, 4)}
+
     # e2e: the same step through the host-buffer entry point (pinned host slabs)
     e2e = None
     if not args.no_e2e:
-        hx = [t.cpu().pin_memory() for t in xs]
+        hx = [t.cpu().pin_memory() for t in x]
         hy = [torch.empty((B, S * w, H // w, D), dtype=torch.bfloat16).pin_memory() for _ in range(w)]
         hz = [torch.empty_like(t).pin_memory() for t in hx]
         for _ in range(2):
@@ -309,10 +354,11 @@ def run_ours(args):
 
     # per-mode figures at w = 2/4/8 on a 512 MiB payload (the >= 256 MB target regime)
     w_sweep = None
-    if not args.no_sweep and rank == 0 or (not args.no_sweep and world == 1):
+    if not args.no_sweep and rank == 0:
+        del y2, z
         w_sweep = {}
         for ww in (2, 4, 8):
-            Pw, a, b = bench_sweep_point(a2a, ww, 512 << 20, "bf16", device, flush, stream,
+            Pw, a, b = bench_sweep_point(a2a, ww, 512 << 20, "bf16", device, stream,
                                          args.sweep_reps)
             w_sweep[f"w{ww}"] = {
                 "payload_bytes": Pw,
@@ -344,12 +390,13 @@ def run_ours(args):
             "w": w, "B": B, "S_local": S, "H": H, "D": D,
             "payload_bytes_per_call": P,
             "path": {1: "tma", 2: "vec"}[plan["path"]],
-            "rows_per_tile": plan["rows_per_tile"], "stages": plan["stages"], "grid": plan["grid"],
-            "l2": "flushed (2x L2 write) before every timed call, outside its events",
+            "rows_per_tile": plan["rows_per_tile"], "producers": plan["producers"],
+            "stages": plan["stages"], "chunk_units": plan["chunk_units"], "grid": plan["grid"],
+            "l2": "inputs larger than L2 (192 MiB per call vs 126 MB); no kernel reads data "
+                  "the previous kernel touched; no flush in the timed region",
             "parallelism": f"{world} independent instance(s), one per GPU",
         },
-        "per_mode": {"mode0_gbs": round(gbs0, 1), "mode1_gbs": round(gbs1, 1),
-                     "mode0_frac": round(2 * gbs0 / peak, 4), "mode1_frac": round(2 * gbs1 / peak, 4)},
+        "per_mode": per_mode,
         "roofline": {
             "bound": "hbm",
             "kernel": "ua2a_tma_kernel<0>/<1>" if plan["path"] == 1 else "ua2a_vec_kernel",
@@ -359,13 +406,14 @@ def run_ours(args):
             "frac": round(achieved / peak, 4),
             "peak_source": peak_src,
             "algorithmic_bytes_per_launch": 2 * P,
+            "avg_launch_us": round(avg_launch_ms * 1e3, 3),
             "traffic": traffic_bytes,
             "traffic_source": traffic_src,
         },
         "gpu_launches": launches,
         "e2e": e2e,
         "clocks": clocks,
-        "w_sweep_512MiB": w_sweep,
+        "w_sweep_512MiB_back_to_back": w_sweep,
         "cpu_baseline": cpu,
     }
     if rank == 0:
@@ -443,7 +491,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--sweep-reps", type=int, default=30)
+    ap.add_argument("--sweep-reps", type=int, default=50)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")

@@ -79,8 +79,15 @@ typedef struct ulysses_a2a_plan_t {
     int32_t launches;        /* kernel launches per call: 1, or B if chunked  */
     int32_t grid;            /* CTAs per launch                               */
     int32_t block;           /* threads per CTA                               */
-    int32_t stages;          /* TMA path: shared-memory ring depth            */
+    int32_t stages;          /* TMA path: shared-memory tiles per CTA (all
+                                producers together)                        */
+    int32_t lookahead;       /* TMA path: loads in flight per producer       */
+    int32_t producers;       /* TMA path: producer warps per CTA (1..8)      */
     int64_t smem_bytes;      /* dynamic shared memory per CTA                 */
+    int32_t order;           /* unit numbering: 0 = destination rank r
+                                outermost, 1 = r innermost                  */
+    int32_t chunk_units;     /* TMA path: 0 = persistent grid (static round
+                                robin); n = n consecutive units per CTA     */
 } ulysses_a2a_plan_t;
 
 /* Create a context on CUDA device `device` for elements of `elem_bytes` bytes
@@ -135,12 +142,27 @@ int ulysses_a2a_status(ulysses_a2a_ctx *ctx, void *stream);
  * with ULYSSES_A2A_ERR_UNSUPPORTED instead of silently switching. */
 int ulysses_a2a_set_path(ulysses_a2a_ctx *ctx, int path);
 
-/* Tuning overrides for later runs; 0 keeps the library's default for that
- * knob. rows_per_tile caps S_tile (1..256); ctas_per_sm sets the persistent
- * grid (1..32); stages sets the TMA ring depth (2..16). Results never depend
- * on these, only speed does. */
-int ulysses_a2a_set_tuning(ulysses_a2a_ctx *ctx, int rows_per_tile,
-                           int ctas_per_sm, int stages);
+/* Speed knobs. Results never depend on them, only speed does; every field
+ * left at its "default" value keeps the library's choice. */
+typedef struct ulysses_a2a_tuning_t {
+    int32_t rows_per_tile;  /* S_tile cap, 1..256; 0 = default                */
+    int32_t ctas_per_sm;    /* persistent TMA grid / VEC grid: CTAs per SM,
+                               1..32; 0 = default                          */
+    int32_t stages;         /* TMA: shared-memory tiles per CTA, 1..32, split
+                               evenly over the producers; 0 = default      */
+    int32_t lookahead;      /* TMA: loads in flight per producer; 0 = default */
+    int32_t producers;      /* TMA: producer warps per CTA, 1..8; 0 = default */
+    int32_t order;          /* unit numbering: 0 = destination rank r
+                               outermost, 1 = innermost; -1 = default      */
+    int32_t chunk_units;    /* TMA schedule: 0 = persistent grid (static
+                               round robin); n > 0 = n consecutive units per
+                               CTA; -1 = default (one unit per producer)   */
+    int32_t reserved;       /* must be 0                                    */
+} ulysses_a2a_tuning_t;
+
+/* Apply tuning to later runs (NULL restores every default). Values outside
+ * the ranges above are rejected with ULYSSES_A2A_ERR_INVALID. */
+int ulysses_a2a_set_tuning(ulysses_a2a_ctx *ctx, const ulysses_a2a_tuning_t *tuning);
 
 /* Kernel launches this context has issued since creation. */
 uint64_t ulysses_a2a_launch_count(const ulysses_a2a_ctx *ctx);
@@ -149,15 +171,15 @@ uint64_t ulysses_a2a_launch_count(const ulysses_a2a_ctx *ctx);
  * (except the device-residency check, which needs a GPU) and reports the path
  * and geometry it would use. Makes no CUDA call, so it runs without a GPU.
  * Pointer values are only compared and tested for alignment, never read.
- * forced_path / rows_per_tile / ctas_per_sm / stages as in the setters above;
- * num_sms = streaming multiprocessors of the target device (148 on B200).
- * On failure writes a message of at most errlen bytes into err (if non-NULL). */
+ * forced_path as in ulysses_a2a_set_path; tuning as in ulysses_a2a_set_tuning
+ * (NULL = defaults); num_sms = streaming multiprocessors of the target device
+ * (148 on B200). On failure writes a message of at most errlen bytes into err
+ * (if non-NULL). */
 int ulysses_a2a_plan(const void *const *in_slabs, void *const *out_slabs,
                      int64_t B, int64_t S_local, int64_t H, int64_t D, int w,
                      int mode, int chunked, int elem_bytes, int forced_path,
-                     int rows_per_tile, int ctas_per_sm, int stages,
-                     int num_sms, ulysses_a2a_plan_t *out, char *err,
-                     size_t errlen);
+                     const ulysses_a2a_tuning_t *tuning, int num_sms,
+                     ulysses_a2a_plan_t *out, char *err, size_t errlen);
 
 /* Allocation-free variant of ulysses_a2a_run (the pages have no counterpart:
  * this entry point exists for this library's users, not for the method).

@@ -57,8 +57,12 @@ class UlyssesA2A:
     def set_path(self, path: int) -> None:
         self._check(_lib.ulysses_a2a_set_path(self._ctx, path))
 
-    def set_tuning(self, rows_per_tile: int = 0, ctas_per_sm: int = 0, stages: int = 0) -> None:
-        self._check(_lib.ulysses_a2a_set_tuning(self._ctx, rows_per_tile, ctas_per_sm, stages))
+    def set_tuning(self, rows_per_tile: int = 0, ctas_per_sm: int = 0, stages: int = 0,
+                   **knobs) -> None:
+        """Speed knobs for later runs (see ``ulysses_a2a_tuning_t``); no argument
+        restores every default. Extra knobs: lookahead, producers, order, chunk_units."""
+        self._check(_lib.ulysses_a2a_set_tuning(self._ctx, rows_per_tile=rows_per_tile,
+                                                ctas_per_sm=ctas_per_sm, stages=stages, **knobs))
 
     @property
     def launch_count(self) -> int:
@@ -139,12 +143,13 @@ class UlyssesA2A:
         handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
         self._check(_lib.ulysses_a2a_status(self._ctx, handle))
 
-    def plan(self, xs, mode: int, chunked: bool = False, out=None) -> dict:
-        """The path and geometry a run with these tensors would use (host only)."""
+    def plan(self, xs, mode: int, chunked: bool = False, out=None, knobs=None) -> dict:
+        """The path and geometry a run with these tensors would use (host only), for the
+        default tuning or the given ``knobs`` dict."""
         w, (B, S, H, D), out = self._prepare(xs, mode, out, xs[0].device.type)
         rc, p, msg = _lib.ulysses_a2a_plan([t.data_ptr() for t in xs], [o.data_ptr() for o in out],
                                            B, S, H, D, w, mode, int(bool(chunked)),
-                                           self.elem_bytes)
+                                           self.elem_bytes, **(knobs or {}))
         if rc != _lib.OK:
             raise A2AError(rc, msg)
         return p.as_dict()

@@ -60,11 +60,42 @@ class PlanT(ctypes.Structure):
         ("grid", ctypes.c_int32),
         ("block", ctypes.c_int32),
         ("stages", ctypes.c_int32),
+        ("lookahead", ctypes.c_int32),
+        ("producers", ctypes.c_int32),
         ("smem_bytes", ctypes.c_int64),
+        ("order", ctypes.c_int32),
+        ("chunk_units", ctypes.c_int32),
     ]
 
     def as_dict(self) -> dict:
         return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+class TuningT(ctypes.Structure):
+    """Mirror of ``ulysses_a2a_tuning_t`` (speed knobs; defaults keep the library's choice)."""
+
+    _fields_ = [
+        ("rows_per_tile", ctypes.c_int32),
+        ("ctas_per_sm", ctypes.c_int32),
+        ("stages", ctypes.c_int32),
+        ("lookahead", ctypes.c_int32),
+        ("producers", ctypes.c_int32),
+        ("order", ctypes.c_int32),
+        ("chunk_units", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+    ]
+
+    DEFAULTS = dict(rows_per_tile=0, ctas_per_sm=0, stages=0, lookahead=0, producers=0,
+                    order=-1, chunk_units=-1, reserved=0)
+
+    @classmethod
+    def make(cls, **kw):
+        vals = dict(cls.DEFAULTS)
+        for k, v in kw.items():
+            if k not in vals:
+                raise TypeError(f"unknown tuning knob {k!r}")
+            vals[k] = int(v)
+        return cls(**vals)
 
 
 class A2AError(RuntimeError):
@@ -98,12 +129,12 @@ def _load() -> ctypes.CDLL:
     lib.ulysses_a2a_status.restype = c_int
     lib.ulysses_a2a_set_path.argtypes = [P, c_int]
     lib.ulysses_a2a_set_path.restype = c_int
-    lib.ulysses_a2a_set_tuning.argtypes = [P, c_int, c_int, c_int]
+    lib.ulysses_a2a_set_tuning.argtypes = [P, ctypes.POINTER(TuningT)]
     lib.ulysses_a2a_set_tuning.restype = c_int
     lib.ulysses_a2a_launch_count.argtypes = [P]
     lib.ulysses_a2a_launch_count.restype = ctypes.c_uint64
     lib.ulysses_a2a_plan.argtypes = [PP, PP, i64, i64, i64, i64, c_int, c_int, c_int, c_int,
-                                     c_int, c_int, c_int, c_int, c_int,
+                                     c_int, ctypes.POINTER(TuningT), c_int,
                                      ctypes.POINTER(PlanT), ctypes.c_char_p, ctypes.c_size_t]
     lib.ulysses_a2a_plan.restype = c_int
     lib.ulysses_a2a_run_noalloc.argtypes = [PP, PP, i64, i64, i64, i64, c_int, c_int, c_int, c_int,
@@ -158,8 +189,11 @@ def ulysses_a2a_set_path(ctx, path: int) -> int:
     return lib.ulysses_a2a_set_path(ctx, int(path))
 
 
-def ulysses_a2a_set_tuning(ctx, rows_per_tile: int = 0, ctas_per_sm: int = 0, stages: int = 0) -> int:
-    return lib.ulysses_a2a_set_tuning(ctx, int(rows_per_tile), int(ctas_per_sm), int(stages))
+def ulysses_a2a_set_tuning(ctx, **knobs) -> int:
+    """Apply TuningT knobs (rows_per_tile, ctas_per_sm, stages, lookahead, producers,
+    order, chunk_units); no knobs restores every default."""
+    t = TuningT.make(**knobs)
+    return lib.ulysses_a2a_set_tuning(ctx, ctypes.byref(t))
 
 
 def ulysses_a2a_launch_count(ctx) -> int:
@@ -178,15 +212,14 @@ def ulysses_a2a_run_noalloc(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunke
 
 
 def ulysses_a2a_plan(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, elem_bytes,
-                     forced_path=PATH_AUTO, rows_per_tile=0, ctas_per_sm=0, stages=0,
-                     num_sms=148):
+                     forced_path=PATH_AUTO, num_sms=148, **knobs):
     """Host-only planning (no CUDA call). Returns (rc, PlanT, message)."""
     plan = PlanT()
     buf = ctypes.create_string_buffer(256)
     ins = ptr_array(in_ptrs) if in_ptrs is not None else None
     outs = ptr_array(out_ptrs) if out_ptrs is not None else None
+    t = TuningT.make(**knobs)
     rc = lib.ulysses_a2a_plan(ins, outs, int(B), int(S_local), int(H), int(D), int(w), int(mode),
-                              int(chunked), int(elem_bytes), int(forced_path), int(rows_per_tile),
-                              int(ctas_per_sm), int(stages), int(num_sms), ctypes.byref(plan),
-                              buf, len(buf))
+                              int(chunked), int(elem_bytes), int(forced_path), ctypes.byref(t),
+                              int(num_sms), ctypes.byref(plan), buf, len(buf))
     return rc, plan, buf.value.decode()

@@ -50,6 +50,7 @@ struct VecParams {
   int32_t w;
   int32_t rows_per_tile;
   uint32_t units;        // w * nb * w * T
+  int32_t order;         // unit numbering: 0 = r outermost, 1 = r innermost
   FastDiv div_T;         // tiles per (r, b, j) block
   FastDiv div_w;
   FastDiv div_nb;        // planes in this launch
@@ -73,13 +74,24 @@ __global__ void __launch_bounds__(256) ua2a_vec_kernel(const __grid_constant__ V
   const int64_t strided_row = (int64_t)p.w * p.nv;  // vectors between rows s, s+1 of [B,S,H,D]
   const uint32_t step = blockDim.x * U;
   for (uint32_t u = blockIdx.x; u < p.units; u += gridDim.x) {
-    // u = ((r * nb + b_rel) * w + j) * T + t
-    const uint32_t q = fdiv(u, p.div_T);
-    const uint32_t t = u - q * p.div_T.d;
-    const uint32_t q2 = fdiv(q, p.div_w);
-    const uint32_t j = q - q2 * p.div_w.d;
-    const uint32_t r = fdiv(q2, p.div_nb);
-    const uint32_t bl = q2 - r * p.div_nb.d;
+    uint32_t t, j, r, bl;
+    if (p.order == 0) {
+      // u = ((r * nb + b_rel) * w + j) * T + t
+      const uint32_t q = fdiv(u, p.div_T);
+      t = u - q * p.div_T.d;
+      const uint32_t q2 = fdiv(q, p.div_w);
+      j = q - q2 * p.div_w.d;
+      r = fdiv(q2, p.div_nb);
+      bl = q2 - r * p.div_nb.d;
+    } else {
+      // u = ((b_rel * w + j) * T + t) * w + r
+      const uint32_t q = fdiv(u, p.div_w);
+      r = u - q * p.div_w.d;
+      const uint32_t q2 = fdiv(q, p.div_T);
+      t = q - q2 * p.div_T.d;
+      bl = fdiv(q2, p.div_w);
+      j = q2 - bl * p.div_w.d;
+    }
     const int64_t b = p.b0 + bl;
     const int64_t s0 = (int64_t)t * p.rows_per_tile;
     const int64_t rows_left = p.S_local - s0;

@@ -25,24 +25,41 @@
 
 namespace ua2a {
 
-// Bytes of one work unit the planner aims for (shared-memory stage size).
-constexpr int64_t kTileTargetBytes = 32 * 1024;
+// Bytes of one work unit the planner aims for: a shared-memory stage of the
+// TMA path, a CTA's unit of the VEC path.
+constexpr int64_t kTmaTileTargetBytes = 8 * 1024;
+constexpr int64_t kTileTargetBytes = 64 * 1024;
 // Largest TMA tile; a single row longer than this goes to the VEC path.
 constexpr int64_t kTmaMaxTileBytes = 64 * 1024;
 // Dynamic shared memory the TMA ring may use per CTA by default (of 227 KB).
 constexpr int64_t kTmaSmemBudget = 192 * 1024;
 constexpr int64_t kTmaSmemMax = 220 * 1024;
-constexpr int kTmaMaxStages = 16;
-constexpr int kTmaBlock = 32;
+constexpr int kTmaMaxStages = 32;            // all producers together
+constexpr int kTmaMaxProducers = 8;          // producer warps per CTA
+constexpr int kTmaDefaultProducers = 4;
+constexpr int kTmaStagesPerProducer = 4;     // default sub-ring depth
 constexpr int kTmaDefaultCtasPerSm = 1;
 constexpr int kTmaMaxBoxDim = 256;
 constexpr int kVecBlock = 256;
-constexpr int kVecDefaultCtasPerSm = 8;
+constexpr int kVecDefaultCtasPerSm = 16;
+// Unit numbering: 0 = destination rank outermost, 1 = innermost.
+constexpr int kDefaultOrder = 1;
+// TMA schedule: by default a grid of ceil(units / n) short-lived CTAs, each
+// taking n consecutive units, one per producer warp, with a one-tile ring per
+// producer and at most kTmaChunkSmemTarget of shared memory per CTA, so that
+// several CTAs share an SM and the hardware hands out chunks as CTAs finish
+// (no static tail imbalance). chunk_units = 0 selects a persistent grid
+// (static round robin) with deeper rings instead.
+constexpr int64_t kTmaChunkSmemTarget = 64 * 1024;
 
 struct Tuning {
   int rows_per_tile = 0;  // 0 = default
   int ctas_per_sm = 0;
   int stages = 0;
+  int lookahead = 0;      // TMA loads in flight per producer (0 = default: S - S/2)
+  int producers = 0;      // TMA producer warps per CTA (0 = default)
+  int order = -1;         // unit numbering (-1 = default)
+  int chunk_units = -1;   // TMA: units per CTA (0 = persistent grid, -1 = default)
 };
 
 inline bool mul_overflows(int64_t a, int64_t b, int64_t* out) {
@@ -79,6 +96,32 @@ inline const char* tma_blocker(const void* const* in, void* const* out, int64_t 
       return "a slab base address is not 16-byte aligned";
   }
   return nullptr;
+}
+
+// Public tuning struct -> internal knobs, with range checks (NULL = defaults).
+inline bool tuning_from(const ulysses_a2a_tuning_t* t, Tuning* out, std::string* err) {
+  *out = Tuning{};
+  if (t == nullptr) return true;
+  auto bad = [&](const char* what) {
+    if (err) *err = std::string("tuning value out of range: ") + what;
+    return false;
+  };
+  if (t->rows_per_tile < 0 || t->rows_per_tile > kTmaMaxBoxDim) return bad("rows_per_tile");
+  if (t->ctas_per_sm < 0 || t->ctas_per_sm > 32) return bad("ctas_per_sm");
+  if (t->stages < 0 || t->stages > kTmaMaxStages) return bad("stages");
+  if (t->lookahead < 0 || t->lookahead > kTmaMaxStages) return bad("lookahead");
+  if (t->producers < 0 || t->producers > kTmaMaxProducers) return bad("producers");
+  if (t->order < -1 || t->order > 1) return bad("order");
+  if (t->chunk_units < -1) return bad("chunk_units");
+  if (t->reserved != 0) return bad("reserved");
+  out->rows_per_tile = t->rows_per_tile;
+  out->ctas_per_sm = t->ctas_per_sm;
+  out->stages = t->stages;
+  out->lookahead = t->lookahead;
+  out->producers = t->producers;
+  out->order = t->order;
+  out->chunk_units = t->chunk_units;
+  return true;
 }
 
 // Validate and plan one call. Returns a ULYSSES_A2A_* status.
@@ -165,7 +208,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
   }
 
   // sequence rows per work unit
-  int64_t rows = kTileTargetBytes / row_bytes;
+  int64_t rows = (path == ULYSSES_A2A_PATH_TMA ? kTmaTileTargetBytes : kTileTargetBytes) / row_bytes;
   if (tune.rows_per_tile > 0) rows = tune.rows_per_tile;
   if (rows < 1) rows = 1;
   if (rows > kTmaMaxBoxDim) rows = kTmaMaxBoxDim;
@@ -190,27 +233,66 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
   p->units = units;
   p->payload_bytes = payload;
   p->launches = chunked ? (int32_t)(B > INT32_MAX ? INT32_MAX : B) : 1;
+  p->order = tune.order >= 0 ? (tune.order ? 1 : 0) : kDefaultOrder;
 
   if (path == ULYSSES_A2A_PATH_TMA) {
     const int64_t tile_bytes = rows * row_bytes;
     const int64_t stage_bytes = (tile_bytes + 1023) / 1024 * 1024;
-    int ctas = tune.ctas_per_sm > 0 ? tune.ctas_per_sm : kTmaDefaultCtasPerSm;
-    int64_t stages = tune.stages > 0 ? tune.stages : kTmaSmemBudget / stage_bytes;
-    if (stages > kTmaMaxStages) stages = kTmaMaxStages;
-    while (stages > 2 && stages * stage_bytes > kTmaSmemMax) --stages;
-    if (stages < 2 || stages * stage_bytes > kTmaSmemMax) {
-      // cannot hold two tiles: let the VEC path take it (or fail if forced)
+    const bool persistent = tune.chunk_units == 0;
+    const int ctas = tune.ctas_per_sm > 0 ? tune.ctas_per_sm : kTmaDefaultCtasPerSm;
+    // Producer warps per CTA, each with a sub-ring of sp stages. A requested
+    // total stage count is split evenly over the producers.
+    int np;
+    if (tune.producers > 0) {
+      np = tune.producers;
+    } else if (persistent) {
+      np = kTmaDefaultProducers;
+    } else {
+      int64_t fit = kTmaChunkSmemTarget / stage_bytes;
+      np = (int)(fit < 1 ? 1 : (fit > kTmaDefaultProducers ? kTmaDefaultProducers : fit));
+    }
+    const int min_sp = persistent ? 2 : 1;
+    int64_t sp = 0;
+    for (; np >= 1; --np) {
+      sp = tune.stages > 0 ? tune.stages / np : (persistent ? kTmaStagesPerProducer : 1);
+      const int64_t budget = (tune.stages > 0 || !persistent) ? kTmaSmemMax : kTmaSmemBudget;
+      while (sp > min_sp && np * sp * stage_bytes > budget) --sp;
+      if (sp >= min_sp && np * sp <= kTmaMaxStages && np * sp * stage_bytes <= kTmaSmemMax) break;
+    }
+    if (np < 1) {
+      // cannot hold the tiles: let the VEC path take it (or fail if forced)
       if (forced_path == ULYSSES_A2A_PATH_TMA) {
-        set_err(err, "TMA ring of two %lld-byte tiles does not fit shared memory", tile_bytes);
+        set_err(err, "TMA ring of %lld-byte tiles does not fit shared memory", tile_bytes);
         return ULYSSES_A2A_ERR_UNSUPPORTED;
       }
       p->path = path = ULYSSES_A2A_PATH_VEC;
     } else {
-      p->stages = (int32_t)stages;
-      p->smem_bytes = stages * stage_bytes;
-      p->block = kTmaBlock;
-      int64_t g = (int64_t)num_sms * ctas;
-      p->grid = (int32_t)(units < g ? units : g);
+      p->producers = np;
+      p->stages = (int32_t)(np * sp);
+      // half of each sub-ring loads ahead, the other half lets stores drain;
+      // a one-stage ring (L = S = 1) loads, stores, and waits for the store
+      // to read its stage before the next load
+      int64_t look = tune.lookahead > 0 ? tune.lookahead : sp - sp / 2;
+      if (look > sp - 1) look = sp - 1;
+      if (look < 1) look = 1;
+      p->lookahead = (int32_t)look;
+      p->smem_bytes = np * sp * stage_bytes;
+      p->block = 32 * np;
+      if (persistent) {
+        p->chunk_units = 0;
+        int64_t g = (int64_t)num_sms * ctas;
+        p->grid = (int32_t)(units < g ? units : g);
+      } else {
+        int64_t chunk = tune.chunk_units > 0 ? tune.chunk_units : np;
+        // keep the grid within the launch limit on huge problems
+        if ((units + chunk - 1) / chunk > INT32_MAX) chunk = (units + INT32_MAX - 1) / INT32_MAX;
+        if (chunk > INT32_MAX) {
+          set_err(err, "%lld units cannot be scheduled", units);
+          return ULYSSES_A2A_ERR_UNSUPPORTED;
+        }
+        p->chunk_units = (int32_t)chunk;
+        p->grid = (int32_t)((units + chunk - 1) / chunk);
+      }
       p->vec_bytes = 16;
     }
   }
@@ -236,6 +318,8 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     int64_t g = (int64_t)num_sms * ctas;
     p->vec_bytes = v;
     p->stages = 0;
+    p->lookahead = 0;
+    p->producers = 0;
     p->smem_bytes = 0;
     p->block = kVecBlock;
     p->grid = (int32_t)(units < g ? units : g);

@@ -35,6 +35,11 @@
 #include "plan.h"
 #include "ulysses_a2a.h"
 
+// L2 fetch granularity the TMA unit uses for the tensor maps (tunable at build time).
+#ifndef UA2A_L2_PROMOTION
+#define UA2A_L2_PROMOTION CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+#endif
+
 using ua2a::TmaParams;
 using ua2a::VecParams;
 
@@ -99,12 +104,6 @@ int cuda_fail(ulysses_a2a_ctx* ctx, const char* what, cudaError_t e) {
               std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")");
 }
 
-int env_int(const char* name, int dflt) {
-  const char* v = std::getenv(name);
-  if (!v || !*v) return dflt;
-  return std::atoi(v);
-}
-
 CUtensorMapDataType map_dtype(int E) {
   switch (E) {
     case 1: return CU_TENSOR_MAP_DATA_TYPE_UINT8;
@@ -125,7 +124,7 @@ int encode_strided(ulysses_a2a_ctx* ctx, CUtensorMap* m, const void* base, int64
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = ctx->encode_tiled(m, map_dtype((int)E), 4, const_cast<void*>(base), dims, strides, box,
                                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                                 UA2A_L2_PROMOTION, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(ctx, ULYSSES_A2A_ERR_CUDA, "cuTensorMapEncodeTiled (strided side) failed: " + std::to_string((int)r));
   return ULYSSES_A2A_OK;
@@ -141,7 +140,7 @@ int encode_gathered(ulysses_a2a_ctx* ctx, CUtensorMap* m, const void* base, int6
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = ctx->encode_tiled(m, map_dtype((int)E), 5, const_cast<void*>(base), dims, strides, box,
                                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                                 UA2A_L2_PROMOTION, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(ctx, ULYSSES_A2A_ERR_CUDA, "cuTensorMapEncodeTiled (gathered side) failed: " + std::to_string((int)r));
   return ULYSSES_A2A_OK;
@@ -160,7 +159,11 @@ int tma_params_for(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out
       for (int k = 0; k < w && same; ++k) same = e.in[k] == in[k] && e.out[k] == out[k];
       if (same) {
         e.stamp = ++ctx->stamp;
-        e.params.stages = pl.stages;
+        e.params.stages = pl.stages / pl.producers;
+        e.params.lookahead = pl.lookahead;
+        e.params.producers = pl.producers;
+        e.params.order = pl.order;
+        e.params.chunk_units = pl.chunk_units;
         *result = &e.params;
         return ULYSSES_A2A_OK;
       }
@@ -198,7 +201,11 @@ int tma_params_for(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out
   p.tiles_per_block = (int32_t)pl.tiles_per_block;
   p.tile_bytes = (uint32_t)(rows * pl.row_bytes);
   p.stage_bytes = (uint32_t)((p.tile_bytes + 1023u) / 1024u * 1024u);
-  p.stages = pl.stages;
+  p.stages = pl.stages / pl.producers;
+  p.lookahead = pl.lookahead;
+  p.producers = pl.producers;
+  p.order = pl.order;
+  p.chunk_units = pl.chunk_units;
   *victim = fresh;
   *result = &victim->params;
   return ULYSSES_A2A_OK;
@@ -301,6 +308,7 @@ int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, in
   p.w = w;
   p.rows_per_tile = (int32_t)pl.rows_per_tile;
   p.units = (uint32_t)pl.units;
+  p.order = pl.order;
   p.div_T = ua2a::FastDiv((uint32_t)pl.tiles_per_block);
   p.div_w = ua2a::FastDiv((uint32_t)w);
   p.div_nb = ua2a::FastDiv((uint32_t)nb);
@@ -376,10 +384,6 @@ int ulysses_a2a_create(ulysses_a2a_ctx** out, int device, int elem_bytes) {
     delete ctx;
     return ULYSSES_A2A_ERR_CUDA;
   }
-  // tuning knobs from the environment (for sweeps only; results never change)
-  ctx->tuning.rows_per_tile = env_int("ULYSSES_A2A_ROWS_PER_TILE", 0);
-  ctx->tuning.ctas_per_sm = env_int("ULYSSES_A2A_CTAS_PER_SM", 0);
-  ctx->tuning.stages = env_int("ULYSSES_A2A_STAGES", 0);
   *out = ctx;
   return ULYSSES_A2A_OK;
 }
@@ -508,14 +512,12 @@ int ulysses_a2a_set_path(ulysses_a2a_ctx* ctx, int path) {
   return ULYSSES_A2A_OK;
 }
 
-int ulysses_a2a_set_tuning(ulysses_a2a_ctx* ctx, int rows_per_tile, int ctas_per_sm, int stages) {
+int ulysses_a2a_set_tuning(ulysses_a2a_ctx* ctx, const ulysses_a2a_tuning_t* t) {
   if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
-  if (rows_per_tile < 0 || rows_per_tile > 256 || ctas_per_sm < 0 || ctas_per_sm > 32 ||
-      stages < 0 || stages == 1 || stages > ua2a::kTmaMaxStages)
-    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "tuning value out of range");
-  ctx->tuning.rows_per_tile = rows_per_tile;
-  ctx->tuning.ctas_per_sm = ctas_per_sm;
-  ctx->tuning.stages = stages;
+  ua2a::Tuning tu;
+  std::string err;
+  if (!ua2a::tuning_from(t, &tu, &err)) return fail(ctx, ULYSSES_A2A_ERR_INVALID, err);
+  ctx->tuning = tu;
   return ULYSSES_A2A_OK;
 }
 
@@ -525,15 +527,16 @@ uint64_t ulysses_a2a_launch_count(const ulysses_a2a_ctx* ctx) {
 
 int ulysses_a2a_plan(const void* const* in_slabs, void* const* out_slabs, int64_t B,
                      int64_t S_local, int64_t H, int64_t D, int w, int mode, int chunked,
-                     int elem_bytes, int forced_path, int rows_per_tile, int ctas_per_sm,
-                     int stages, int num_sms, ulysses_a2a_plan_t* out, char* err, size_t errlen) {
+                     int elem_bytes, int forced_path, const ulysses_a2a_tuning_t* tuning,
+                     int num_sms, ulysses_a2a_plan_t* out, char* err, size_t errlen) {
   ua2a::Tuning t;
-  t.rows_per_tile = rows_per_tile;
-  t.ctas_per_sm = ctas_per_sm;
-  t.stages = stages;
   std::string msg;
-  int rc = ua2a::make_plan(in_slabs, out_slabs, B, S_local, H, D, w, mode, chunked, elem_bytes,
-                           forced_path, t, num_sms, out, &msg);
+  int rc = ULYSSES_A2A_OK;
+  if (!ua2a::tuning_from(tuning, &t, &msg))
+    rc = ULYSSES_A2A_ERR_INVALID;
+  else
+    rc = ua2a::make_plan(in_slabs, out_slabs, B, S_local, H, D, w, mode, chunked, elem_bytes,
+                         forced_path, t, num_sms, out, &msg);
   if (err && errlen) {
     std::snprintf(err, errlen, "%s", rc ? msg.c_str() : "");
   }
@@ -625,7 +628,7 @@ bool noalloc_encode(CUtensorMap* m, int rank, const void* base, const cuuint64_t
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   return g_noalloc_encode(m, map_dtype(E), (cuuint32_t)rank, const_cast<void*>(base), dims, strides,
                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          UA2A_L2_PROMOTION,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -750,7 +753,11 @@ extern "C" int ulysses_a2a_run_noalloc(const void* const* in_slabs, void* const*
     p.nb = (int32_t)nb;
     p.tile_bytes = (uint32_t)(rows * pl.row_bytes);
     p.stage_bytes = (p.tile_bytes + 1023u) / 1024u * 1024u;
-    p.stages = pl.stages;
+    p.stages = pl.stages / pl.producers;
+    p.lookahead = pl.lookahead;
+    p.producers = pl.producers;
+    p.order = pl.order;
+    p.chunk_units = pl.chunk_units;
     for (int l = 0; l < pl.launches; ++l) {
       p.b0 = chunked ? l : 0;
       p.status = st.scratch + kNoAllocSlotWords * l;
@@ -774,6 +781,7 @@ extern "C" int ulysses_a2a_run_noalloc(const void* const* in_slabs, void* const*
     p.w = w;
     p.rows_per_tile = (int32_t)pl.rows_per_tile;
     p.units = (uint32_t)pl.units;
+    p.order = pl.order;
     p.div_T = ua2a::FastDiv((uint32_t)pl.tiles_per_block);
     p.div_w = ua2a::FastDiv((uint32_t)w);
     p.div_nb = ua2a::FastDiv((uint32_t)nb);

@@ -37,8 +37,8 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_plan_struct_layout_matches_header():
-    # int32 path, vec_bytes; 6 x int64; 4 x int32; int64 -> 8 + 48 + 16 + 8 = 80 bytes
-    assert ctypes.sizeof(_lib.PlanT) == 80
+    # int32 path, vec_bytes; 6 x int64; 6 x int32; int64; 2 x int32 -> 96 bytes
+    assert ctypes.sizeof(_lib.PlanT) == 96
 
 
 def fake_slabs(w, slab_bytes, base=1 << 40, align=256, gap=0):
@@ -61,21 +61,28 @@ def test_plan_cfg2_tma():
     assert rc == OK, msg
     assert p.path == PATH_TMA
     assert p.row_bytes == 6 * 128 * 2
-    assert p.rows_per_tile == 32 * 1024 // 1536       # 21 rows, ~32 KB
-    assert p.tiles_per_block == -(-8192 // 21)
-    assert p.tail_rows == 8192 % 21
+    assert p.rows_per_tile == 8 * 1024 // 1536        # 5 rows, ~8 KB tiles
+    assert p.tiles_per_block == -(-8192 // 5)
+    assert p.tail_rows == 8192 % 5 == 2
     assert p.units == 4 * 1 * 4 * p.tiles_per_block
     assert p.payload_bytes == 192 * MiB
-    assert p.launches == 1 and p.block == 32
-    assert p.grid == 148
-    assert p.stages >= 2 and p.smem_bytes <= 220 * 1024
+    assert p.launches == 1
+    # default schedule: short-lived CTAs of 4 producer warps, one 8 KB tile each
+    assert p.producers == 4 and p.block == 128 and p.stages == 4 and p.lookahead == 1
+    assert p.chunk_units == 4 and p.grid == -(-p.units // 4) == 6556
+    assert p.smem_bytes == 4 * 8 * 1024
+    assert p.order == 1
+    # the persistent schedule: one CTA per SM, 4 producers x 4-stage rings
+    rc, q, _ = plan(4, 1, 8192, 24, 128, chunk_units=0)
+    assert rc == OK and q.chunk_units == 0 and q.grid == 148
+    assert (q.producers, q.stages, q.lookahead, q.smem_bytes) == (4, 16, 2, 16 * 8 * 1024)
 
 
 def test_plan_cfg3_tail_rows():
     rc, p, _ = plan(8, 2, 4725, 40, 128)
     assert rc == OK and p.path == PATH_TMA
     assert p.row_bytes == 5 * 128 * 2
-    assert p.rows_per_tile == 25 and p.tail_rows == 0          # 4725 = 189 * 25
+    assert p.rows_per_tile == 6 and p.tail_rows == 3           # 4725 = 787 * 6 + 3
     rc, p, _ = plan(8, 2, 4725, 40, 128, rows_per_tile=32)
     assert rc == OK
     assert p.rows_per_tile == 32 and p.tail_rows == 4725 - 147 * 32 == 21
@@ -101,8 +108,8 @@ def test_plan_cfg4_chunked_launches():
 def test_plan_cfg1_small():
     rc, p, _ = plan(2, 1, 64, 4, 64)
     assert rc == OK and p.path == PATH_TMA
-    assert p.rows_per_tile == 64 and p.tail_rows == 0 and p.tiles_per_block == 1
-    assert p.units == 4 and p.grid == 4
+    assert p.rows_per_tile == 32 and p.tail_rows == 0 and p.tiles_per_block == 2
+    assert p.units == 8 and p.chunk_units == 4 and p.grid == 2
 
 
 def test_rows_never_exceed_sequence():
@@ -144,13 +151,66 @@ def test_vec_when_box_dim_too_large():
 def test_forced_vec_geometry():
     rc, p, _ = plan(4, 1, 8192, 24, 128, forced_path=PATH_VEC)
     assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 16
-    assert p.block == 256 and p.grid == min(p.units, 148 * 8)
+    assert p.rows_per_tile == 64 * 1024 // 1536
+    assert p.block == 256 and p.grid == min(p.units, 148 * 16)
+    assert p.producers == 0 and p.lookahead == 0
 
 
 def test_tuning_knobs():
-    rc, p, _ = plan(4, 1, 8192, 24, 128, rows_per_tile=16, stages=4, ctas_per_sm=2)
+    rc, p, _ = plan(4, 1, 8192, 24, 128, rows_per_tile=16, stages=4, ctas_per_sm=2,
+                    chunk_units=0)
     assert rc == OK and p.rows_per_tile == 16 and p.stages == 4 and p.grid == 296
     assert p.smem_bytes == 4 * 24 * 1024
+    rc, p, _ = plan(4, 1, 8192, 24, 128, producers=2, chunk_units=7, order=0)
+    assert rc == OK and (p.producers, p.chunk_units, p.order) == (2, 7, 0)
+    assert p.grid == -(-p.units // 7)
+
+
+@pytest.mark.parametrize("knob,value", [("rows_per_tile", 257), ("rows_per_tile", -1),
+                                        ("ctas_per_sm", 33), ("stages", 33), ("producers", 9),
+                                        ("order", 2), ("chunk_units", -2), ("lookahead", -1),
+                                        ("reserved", 1)])
+def test_tuning_out_of_range_is_rejected(knob, value):
+    rc, _, msg = plan(4, 1, 64, 8, 64, **{knob: value})
+    assert rc == ERR_INVALID and knob in msg
+
+
+def test_tuning_struct_layout():
+    assert ctypes.sizeof(_lib.TuningT) == 32
+
+
+def test_ring_split_between_producers_loads_and_stores():
+    # stages split evenly over up to 4 producer warps (sub-rings of >= 2);
+    # per producer L loads in flight, sp - L stores allowed to read their stages
+    for S, np_, sp, L in [(2, 1, 2, 1), (3, 1, 3, 2), (4, 2, 2, 1), (6, 3, 2, 1), (8, 4, 2, 1),
+                          (12, 4, 3, 2), (16, 4, 4, 2), (32, 4, 8, 4)]:
+        rc, p, _ = plan(4, 1, 8192, 24, 128, rows_per_tile=4, stages=S, chunk_units=0)
+        assert rc == OK, S
+        assert (p.producers, p.stages // p.producers, p.lookahead) == (np_, sp, L), S
+        assert p.stages == np_ * sp and p.block == 32 * np_
+        assert 1 <= p.lookahead < p.stages // p.producers
+
+
+def test_large_rows_reduce_stages_then_producers():
+    # 24 KB rows: four producers keep two 24 KB stages each (192 KB)
+    # persistent schedule
+    rc, p, _ = plan(2, 1, 16, 128, 192, chunk_units=0)
+    assert rc == OK and p.path == PATH_TMA and p.rows_per_tile == 1
+    assert p.row_bytes == 24 * 1024
+    assert (p.producers, p.stages, p.smem_bytes) == (4, 8, 192 * 1024)
+    # 32 KB rows: two stages for four producers would not fit; three producers do
+    rc, p, _ = plan(2, 1, 16, 128, 256, chunk_units=0)
+    assert rc == OK and p.row_bytes == 32 * 1024
+    assert (p.producers, p.stages, p.smem_bytes) == (3, 6, 192 * 1024)
+    # 64 KB rows: one producer with a three-stage ring
+    rc, p, _ = plan(2, 1, 8, 256, 256, chunk_units=0)
+    assert rc == OK and p.path == PATH_TMA and p.row_bytes == 64 * 1024
+    assert (p.producers, p.stages, p.lookahead, p.smem_bytes) == (1, 3, 2, 192 * 1024)
+    # default (chunked grid): at most 64 KB of tiles per CTA, one tile per producer
+    rc, p, _ = plan(2, 1, 16, 128, 192)
+    assert (p.producers, p.stages, p.chunk_units, p.smem_bytes) == (2, 2, 2, 48 * 1024)
+    rc, p, _ = plan(2, 1, 8, 256, 256)
+    assert (p.producers, p.stages, p.chunk_units, p.smem_bytes) == (1, 1, 1, 64 * 1024)
 
 
 # ---- argument validation ----------------------------------------------------
@@ -232,7 +292,7 @@ def test_null_context_handling():
     assert lib.ulysses_a2a_launch_count(None) == 0
     assert lib.ulysses_a2a_last_error(None) == b"NULL context"
     assert lib.ulysses_a2a_set_path(None, PATH_AUTO) == ERR_INVALID
-    assert lib.ulysses_a2a_set_tuning(None, 0, 0, 0) == ERR_INVALID
+    assert lib.ulysses_a2a_set_tuning(None, None) == ERR_INVALID
     arr = _lib.ptr_array([1, 2])
     assert lib.ulysses_a2a_run(None, arr, arr, 1, 1, 2, 1, 2, 0, 0, None) == ERR_INVALID
     assert lib.ulysses_a2a_run_host(None, arr, arr, 1, 1, 2, 1, 2, 0, 0, None) == ERR_INVALID

@@ -64,7 +64,7 @@ def run_case(xs_cpu, mode, *, chunked=False, path=PATH_AUTO, tuning=None, a2a=No
     a2a = a2a or UlyssesA2A(0, E)
     try:
         a2a.set_path(path)
-        a2a.set_tuning(*(tuning or (0, 0, 0)))
+        a2a.set_tuning(**(tuning or {}))
         if in_offset:
             xs = []
             for t in xs_cpu:
@@ -105,7 +105,21 @@ SHAPES = [
     (8, 1, 7, 8, 256),          # D at the TMA box limit, H/w = 1
 ]
 
-TUNINGS = [(0, 0, 0), (7, 0, 2), (16, 2, 3), (1, 1, 2)]
+# The default (short-lived CTAs, one tile per producer), then other shapes of
+# both schedules: chunked grids with deeper rings or other chunk sizes, and
+# persistent grids (chunk_units=0) with 1-4 producers and 2-4 stages each.
+TUNINGS = [
+    {},
+    dict(rows_per_tile=7, stages=2),
+    dict(rows_per_tile=5, stages=12, chunk_units=7),
+    dict(producers=1, chunk_units=3),
+    dict(producers=3, stages=3, chunk_units=5, order=0),
+    dict(rows_per_tile=16, ctas_per_sm=2, stages=3, chunk_units=0),
+    dict(rows_per_tile=1, ctas_per_sm=1, stages=2, chunk_units=0),
+    dict(rows_per_tile=2, stages=6, chunk_units=0),
+    dict(rows_per_tile=3, stages=8, chunk_units=0, order=0),
+    dict(rows_per_tile=5, ctas_per_sm=2, stages=12, chunk_units=0),
+]
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "w{}B{}S{}H{}D{}".format(*s))
@@ -123,6 +137,36 @@ def test_parity_small(shape, mode, path):
         a2a.close()
 
 
+@pytest.mark.parametrize("order", [0, 1])
+@pytest.mark.parametrize("path", [PATH_TMA, PATH_VEC], ids=["tma", "vec"])
+def test_parity_unit_orders(order, path):
+    # both numberings of the work units (destination rank outermost / innermost)
+    with UlyssesA2A(0, 2) as a2a:
+        for (w, B, S, H, D) in [(4, 2, 37, 8, 64), (8, 2, 53, 40, 128), (3, 3, 11, 6, 32)]:
+            for mode in (0, 1):
+                xs = normal_slabs(slab_shape(mode, w, B, S, H, D), w, "bf16", seed0=300 + mode)
+                for tuning in ({}, dict(rows_per_tile=7, stages=2, chunk_units=0),
+                               dict(rows_per_tile=3, stages=8)):
+                    for chunked in (False, True):
+                        run_case(xs, mode, chunked=chunked, path=path,
+                                 tuning=dict(tuning, order=order), a2a=a2a)
+
+
+@pytest.mark.parametrize("chunk_units", [1, 5, 16])
+def test_parity_chunked_grid_schedule(chunk_units):
+    # TMA grid of ceil(units / n) CTAs, each taking n consecutive units
+    for order in (0, 1):
+        with UlyssesA2A(0, 2) as a2a:
+            for (w, B, S, H, D) in [(4, 2, 37, 8, 64), (8, 1, 53, 40, 128)]:
+                for mode in (0, 1):
+                    xs = normal_slabs(slab_shape(mode, w, B, S, H, D), w, "bf16", seed0=400)
+                    for tuning in ({}, dict(rows_per_tile=7, stages=2), dict(rows_per_tile=3, stages=8),
+                                   dict(producers=2, stages=2)):
+                        run_case(xs, mode, chunked=(tuning.get("stages") == 2), path=PATH_TMA,
+                                 tuning=dict(tuning, chunk_units=chunk_units, order=order),
+                                 a2a=a2a)
+
+
 @pytest.mark.parametrize("E", [1, 2, 4, 8])
 @pytest.mark.parametrize("path", [PATH_TMA, PATH_VEC], ids=["tma", "vec"])
 def test_parity_unique_ids_every_element_size(E, path):
@@ -135,8 +179,8 @@ def test_parity_unique_ids_every_element_size(E, path):
     xs = unique_slabs((B, S, H, D), w, E)
     for mode in (0, 1):
         xin = xs if mode == 0 else oracle.ulysses_a2a(xs, 0)
-        run_case(xin, mode, path=path, tuning=(5, 0, 2))
-        run_case(xin, mode, path=path, tuning=(1, 0, 2), chunked=True)
+        run_case(xin, mode, path=path, tuning=dict(rows_per_tile=5, stages=2))
+        run_case(xin, mode, path=path, tuning=dict(rows_per_tile=1, stages=2), chunked=True)
 
 
 def test_parity_fp32_uniform():
@@ -232,8 +276,9 @@ def test_full_size_configs(name):
         run_case(y, 1, chunked=True)
     if name.startswith("cfg3"):
         # the ragged tile: 4725 = 147 * 32 + 21
-        run_case(xs, 0, tuning=(32, 0, 0))
-        run_case(y, 1, tuning=(32, 0, 0), path=PATH_VEC)
+        run_case(xs, 0, tuning=dict(rows_per_tile=32))
+        run_case(y, 1, tuning=dict(rows_per_tile=32), path=PATH_VEC)
+        run_case(xs, 0, tuning=dict(rows_per_tile=32, chunk_units=0))
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
