@@ -53,6 +53,20 @@ def env_rank():
             int(os.environ.get("WORLD_SIZE", "1")))
 
 
+def max_over_ranks(value: float, dist=None, device="cpu") -> float:
+    """The largest of every rank's `value` (the slowest rank's time); identity on one rank."""
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(world: int, bytes_per_step: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank's bytes over the slowest rank's time (GB = 1e9 B)."""
+    return world * bytes_per_step * steps / (max_ms / 1e3) / 1e9
+
+
 def hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -287,12 +301,9 @@ def run_ours(args):
     for k in range(w):
         if not torch.equal(z[k].view(torch.int16), x[k].view(torch.int16)):
             raise SystemExit("round trip mismatch: mode1(mode0(x)) != x")
-    if dist:
-        t = torch.tensor([total_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, device)
     ms_per_step = total_ms / args.steps
-    value = world * 2 * P * args.steps / (total_ms / 1e3) / 1e9
+    value = job_gbs(world, 2 * P, args.steps, total_ms)
 
     peak, peak_src = hbm_peak()
     avg_launch_ms = total_ms / launches
@@ -340,15 +351,11 @@ def run_ours(args):
             a2a.run_host(hy, 1, out=hz, stream=stream)
         eb.record(stream)
         torch.cuda.synchronize()
-        e_ms = ea.elapsed_time(eb)
-        if dist:
-            t = torch.tensor([e_ms], device=device, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(ea.elapsed_time(eb), dist, device)
         for k in range(w):
             if not torch.equal(hz[k].view(torch.int16), hx[k].view(torch.int16)):
                 raise SystemExit("host-path round trip mismatch")
-        e2e = {"value": round(world * 2 * P * e_steps / (e_ms / 1e3) / 1e9, 3), "unit": "GB/s",
+        e2e = {"value": round(job_gbs(world, 2 * P, e_steps, e_ms), 3), "unit": "GB/s",
                "h2d_bytes_per_step": 2 * P, "d2h_bytes_per_step": 2 * P,
                "steps": e_steps, "via": "ulysses_a2a_run_host, pinned host slabs"}
 

@@ -51,7 +51,8 @@ struct TmaParams {
   int32_t w;
   int32_t Hw;                                   // H / w
   int32_t rows_per_tile;                        // S_tile
-  int32_t tiles_per_block;                      // T = ceil(S_local / S_tile)
+  int32_t tiles_per_block;                      // tiles per (r, b, j) block in this launch
+  int32_t tile0;                                //   ... starting at tile tile0 (0 = whole block)
   int32_t b0;                                   // first plane of this launch
   int32_t nb;                                   // planes in this launch
   uint32_t tile_bytes;                          // full box bytes (clipped rows included)
@@ -260,7 +261,7 @@ __device__ __forceinline__ UnitCoord decode_unit(const TmaParams& p, int64_t u) 
     q /= p.w;
     c.b = p.b0 + (int)(q % p.nb);
     c.r = (int)(q / p.nb);
-    c.s0 = (int)(t * p.rows_per_tile);
+    c.s0 = (int)((p.tile0 + t) * p.rows_per_tile);
   } else {
     // destination rank innermost: u = ((b_rel * w + j) * T + t) * w + r, so w
     // consecutive units cover whole rows of the [B, S_local, H, D] side
@@ -270,7 +271,7 @@ __device__ __forceinline__ UnitCoord decode_unit(const TmaParams& p, int64_t u) 
     q /= p.tiles_per_block;
     c.j = (int)(q % p.w);
     c.b = p.b0 + (int)(q / p.w);
-    c.s0 = (int)(t * p.rows_per_tile);
+    c.s0 = (int)((p.tile0 + t) * p.rows_per_tile);
   }
   return c;
 }

@@ -51,7 +51,8 @@ struct VecParams {
   int32_t rows_per_tile;
   uint32_t units;        // w * nb * w * T
   int32_t order;         // unit numbering: 0 = r outermost, 1 = r innermost
-  FastDiv div_T;         // tiles per (r, b, j) block
+  uint32_t tile0;        // first tile of each (r, b, j) block in this launch
+  FastDiv div_T;         // tiles per (r, b, j) block in this launch
   FastDiv div_w;
   FastDiv div_nb;        // planes in this launch
   FastDiv div_nv;
@@ -93,7 +94,7 @@ __global__ void __launch_bounds__(256) ua2a_vec_kernel(const __grid_constant__ V
       j = q2 - bl * p.div_w.d;
     }
     const int64_t b = p.b0 + bl;
-    const int64_t s0 = (int64_t)t * p.rows_per_tile;
+    const int64_t s0 = (int64_t)(p.tile0 + t) * p.rows_per_tile;
     const int64_t rows_left = p.S_local - s0;
     const int64_t rows = rows_left < p.rows_per_tile ? rows_left : p.rows_per_tile;
     // strided side: row (b, s0), head group r; gathered side: row (b, j*S_local + s0)

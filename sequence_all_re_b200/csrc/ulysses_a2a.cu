@@ -46,6 +46,10 @@ using ua2a::VecParams;
 namespace {
 
 constexpr int kTmaCacheEntries = 16;
+// host-buffer entry point: sequence chunks in flight, and the payload below
+// which one chunk is used
+constexpr int64_t kHostChunks = 8;
+constexpr int64_t kHostChunkMinBytes = 8 << 20;
 
 struct TmaCacheEntry {
   bool valid = false;
@@ -75,6 +79,8 @@ struct ulysses_a2a_ctx {
   // run_host staging: one device buffer carved into 2w slabs
   void* d_stage = nullptr;
   size_t stage_bytes = 0;
+  cudaStream_t copy_stream[2] = {nullptr, nullptr};  // H2D, D2H
+  cudaEvent_t copy_events[1 + 2 * 8] = {};            // start + 2 per chunk
   PFN_cuTensorMapEncodeTiled_v12000 encode_tiled = nullptr;
   PFN_cuMemGetAddressRange_v3020 get_range = nullptr;
 };
@@ -260,11 +266,22 @@ cudaError_t launch_vec(const VecParams& p, int vec_bytes, int mode, int grid, in
   }
 }
 
+// Launch the planned kernel(s) for tiles [tile0, tile0 + ntiles) of every
+// (r, b, j) block (ntiles < 0: the whole block).
 int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, int64_t B, int64_t S,
                int64_t H, int64_t D, int w, int mode, int chunked, cudaStream_t st,
-               const ulysses_a2a_plan_t& pl) {
+               const ulysses_a2a_plan_t& pl, int64_t tile0 = 0, int64_t ntiles = -1) {
   const int64_t nb = chunked ? 1 : B;
   const int launches = chunked ? (int)B : 1;
+  const int64_t nt = ntiles < 0 ? pl.tiles_per_block : ntiles;
+  const int64_t units = (int64_t)w * nb * w * nt;
+  int grid = pl.grid;
+  if (nt != pl.tiles_per_block) {
+    if (pl.path == ULYSSES_A2A_PATH_TMA && pl.chunk_units > 0)
+      grid = (int)((units + pl.chunk_units - 1) / pl.chunk_units);
+    else if (units < grid)
+      grid = (int)units;
+  }
   if (pl.path == ULYSSES_A2A_PATH_TMA) {
     TmaParams* cached = nullptr;
     int rc = tma_params_for(ctx, in, out, B, S, H, D, w, mode, pl, &cached);
@@ -272,7 +289,9 @@ int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, in
     TmaParams p = *cached;
     p.status = ctx->d_status;
     p.nb = (int32_t)nb;
-    p.units = pl.units;
+    p.units = units;
+    p.tiles_per_block = (int32_t)nt;
+    p.tile0 = (int32_t)tile0;
     const int mi = mode ? 1 : 0;
     if (!ctx->tma_smem_set[mi] || ctx->tma_smem_set_bytes[mi] < pl.smem_bytes) {
       cudaError_t e = mode == 0 ? cudaFuncSetAttribute(ua2a::ua2a_tma_kernel<0>,
@@ -288,9 +307,9 @@ int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, in
     for (int l = 0; l < launches; ++l) {
       p.b0 = chunked ? l : 0;
       if (mode == 0)
-        ua2a::ua2a_tma_kernel<0><<<pl.grid, pl.block, (size_t)pl.smem_bytes, st>>>(p);
+        ua2a::ua2a_tma_kernel<0><<<grid, pl.block, (size_t)pl.smem_bytes, st>>>(p);
       else
-        ua2a::ua2a_tma_kernel<1><<<pl.grid, pl.block, (size_t)pl.smem_bytes, st>>>(p);
+        ua2a::ua2a_tma_kernel<1><<<grid, pl.block, (size_t)pl.smem_bytes, st>>>(p);
       cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess) return cuda_fail(ctx, "TMA kernel launch", e);
       ctx->launches++;
@@ -307,15 +326,16 @@ int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, in
   p.nv = pl.row_bytes / pl.vec_bytes;
   p.w = w;
   p.rows_per_tile = (int32_t)pl.rows_per_tile;
-  p.units = (uint32_t)pl.units;
+  p.units = (uint32_t)units;
   p.order = pl.order;
-  p.div_T = ua2a::FastDiv((uint32_t)pl.tiles_per_block);
+  p.tile0 = (uint32_t)tile0;
+  p.div_T = ua2a::FastDiv((uint32_t)nt);
   p.div_w = ua2a::FastDiv((uint32_t)w);
   p.div_nb = ua2a::FastDiv((uint32_t)nb);
   p.div_nv = ua2a::FastDiv((uint32_t)p.nv);
   for (int l = 0; l < launches; ++l) {
     p.b0 = chunked ? l : 0;
-    cudaError_t e = launch_vec(p, pl.vec_bytes, mode, pl.grid, pl.block, st);
+    cudaError_t e = launch_vec(p, pl.vec_bytes, mode, grid, pl.block, st);
     if (e != cudaSuccess) return cuda_fail(ctx, "VEC kernel launch", e);
     ctx->launches++;
   }
@@ -396,6 +416,10 @@ int ulysses_a2a_destroy(ulysses_a2a_ctx* ctx) {
     if (cudaDeviceSynchronize() != cudaSuccess) rc = ULYSSES_A2A_ERR_CUDA;
     if (ctx->d_status && cudaFree(ctx->d_status) != cudaSuccess) rc = ULYSSES_A2A_ERR_CUDA;
     if (ctx->d_stage && cudaFree(ctx->d_stage) != cudaSuccess) rc = ULYSSES_A2A_ERR_CUDA;
+    for (auto& cs : ctx->copy_stream)
+      if (cs && cudaStreamDestroy(cs) != cudaSuccess) rc = ULYSSES_A2A_ERR_CUDA;
+    for (auto& ev : ctx->copy_events)
+      if (ev && cudaEventDestroy(ev) != cudaSuccess) rc = ULYSSES_A2A_ERR_CUDA;
     cudaGetLastError();
   }
   delete ctx;  // the handle is consumed whatever the cleanup calls reported
@@ -432,13 +456,14 @@ int ulysses_a2a_run_host(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void
   if (rc) return rc;
   DeviceGuard g(ctx->device);
   if (!g.ok) return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "cannot select the context's device");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t slab_bytes = host_pl.payload_bytes / w;
   const size_t slot = ((size_t)slab_bytes + 255) / 256 * 256;
   const size_t need = slot * 2 * (size_t)w;
   if (ctx->stage_bytes < need) {
     if (ctx->d_stage) {
-      cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
-      if (e != cudaSuccess) return cuda_fail(ctx, "cudaStreamSynchronize", e);
+      cudaError_t e = cudaDeviceSynchronize();
+      if (e != cudaSuccess) return cuda_fail(ctx, "cudaDeviceSynchronize", e);
       cudaFree(ctx->d_stage);
       ctx->d_stage = nullptr;
       ctx->stage_bytes = 0;
@@ -451,6 +476,24 @@ int ulysses_a2a_run_host(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void
     }
     ctx->stage_bytes = need;
   }
+  for (int k = 0; k < 2; ++k) {
+    if (ctx->copy_stream[k] == nullptr) {
+      cudaError_t e = cudaStreamCreateWithFlags(&ctx->copy_stream[k], cudaStreamNonBlocking);
+      if (e != cudaSuccess) {
+        ctx->copy_stream[k] = nullptr;
+        return cuda_fail(ctx, "cudaStreamCreate (host-path copies)", e);
+      }
+    }
+  }
+  for (auto& ev : ctx->copy_events) {
+    if (ev == nullptr) {
+      cudaError_t e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+      if (e != cudaSuccess) {
+        ev = nullptr;
+        return cuda_fail(ctx, "cudaEventCreate (host-path copies)", e);
+      }
+    }
+  }
   std::vector<const void*> din(w);
   std::vector<void*> dout(w);
   char* base = static_cast<char*>(ctx->d_stage);
@@ -458,23 +501,77 @@ int ulysses_a2a_run_host(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void
     din[k] = base + slot * k;
     dout[k] = base + slot * (w + k);
   }
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  for (int k = 0; k < w; ++k) {
-    cudaError_t e = cudaMemcpyAsync(const_cast<void*>(din[k]), in_slabs[k], (size_t)slab_bytes,
-                                    cudaMemcpyHostToDevice, st);
-    if (e != cudaSuccess) return cuda_fail(ctx, "cudaMemcpyAsync H2D", e);
-  }
   ulysses_a2a_plan_t pl;
   rc = plan_for(ctx, din.data(), dout.data(), B, S_local, H, D, w, mode, chunked, &pl);
   if (rc) return rc;
-  rc = run_device(ctx, din.data(), dout.data(), B, S_local, H, D, w, mode, chunked, st, pl);
-  if (rc) return rc;
-  for (int k = 0; k < w; ++k) {
-    cudaError_t e = cudaMemcpyAsync(out_slabs[k], dout[k], (size_t)slab_bytes,
-                                    cudaMemcpyDeviceToHost, st);
-    if (e != cudaSuccess) return cuda_fail(ctx, "cudaMemcpyAsync D2H", e);
+
+  // Pipeline over sequence chunks: the H2D copies of chunk c+1 (copy stream 0),
+  // the kernel of chunk c (the caller's stream) and the D2H copies of chunk
+  // c-1 (copy stream 1) run at once, so PCIe carries both directions together.
+  // A chunk is a tile-aligned row range [s0, s1) of every (b, j) block; its
+  // bytes on each side are strided blocks moved by one 2-D copy per slab/plane.
+  const int64_t T = pl.tiles_per_block, rows = pl.rows_per_tile, E = ctx->elem_bytes;
+  const int64_t L = (H / w) * D;             // elements per run
+  int64_t nchunks = pl.payload_bytes < kHostChunkMinBytes ? 1 : kHostChunks;
+  if (nchunks > T) nchunks = T;
+  const int64_t tpc = (T + nchunks - 1) / nchunks;
+  nchunks = (T + tpc - 1) / tpc;
+  cudaStream_t sh = ctx->copy_stream[0], sd = ctx->copy_stream[1];
+  cudaEvent_t* ev = ctx->copy_events;  // [0]: start; [1 + 2c]: H2D done; [2 + 2c]: kernel done
+  cudaError_t e = cudaEventRecord(ev[0], st);  // copies start after earlier work on `stream`
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(sh, ev[0], 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(sd, ev[0], 0);
+  if (e != cudaSuccess) return cuda_fail(ctx, "stream ordering", e);
+  const size_t plane_s = (size_t)(S_local * H * D * E);   // [B, S, H, D] plane
+  const size_t row_s = (size_t)(H * D * E);
+  const size_t plane_g = (size_t)(w * S_local * L * E);   // [B, S*w, H/w, D] plane
+  const size_t block_g = (size_t)(S_local * L * E);       // one j block of it
+  const size_t row_g = (size_t)(L * E);
+  auto copy_rows = [&](bool h2d, int64_t s0, int64_t n, cudaStream_t cs) -> cudaError_t {
+    // mode 0 reads the [B,S,H,D] side and writes the [B,S*w,H/w,D] side;
+    // mode 1 the reverse
+    const bool strided_side = (mode == 0) == h2d;
+    for (int k = 0; k < w; ++k) {
+      const char* src_base = static_cast<const char*>(h2d ? in_slabs[k] : dout[k]);
+      char* dst_base = static_cast<char*>(h2d ? const_cast<void*>(din[k]) : out_slabs[k]);
+      cudaMemcpyKind kind = h2d ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToHost;
+      cudaError_t r;
+      if (strided_side) {
+        // rows [s0, s0+n) of every plane: B blocks of n*H*D*E bytes, plane apart
+        const size_t off = (size_t)s0 * row_s;
+        r = cudaMemcpy2DAsync(dst_base + off, plane_s, src_base + off, plane_s, (size_t)n * row_s,
+                              (size_t)B, kind, cs);
+      } else {
+        // rows [s0, s0+n) of every (b, j) block: per plane, w blocks S*L*E apart
+        r = cudaSuccess;
+        for (int64_t b = 0; b < B && r == cudaSuccess; ++b) {
+          const size_t off = b * plane_g + (size_t)s0 * row_g;
+          r = cudaMemcpy2DAsync(dst_base + off, block_g, src_base + off, block_g, (size_t)n * row_g,
+                                (size_t)w, kind, cs);
+        }
+      }
+      if (r != cudaSuccess) return r;
+    }
+    return cudaSuccess;
+  };
+  for (int64_t c = 0; c < nchunks; ++c) {
+    const int64_t t0 = c * tpc;
+    const int64_t nt = (t0 + tpc <= T) ? tpc : T - t0;
+    const int64_t s0 = t0 * rows;
+    const int64_t s1 = (t0 + nt) * rows < S_local ? (t0 + nt) * rows : S_local;
+    e = copy_rows(true, s0, s1 - s0, sh);
+    if (e == cudaSuccess) e = cudaEventRecord(ev[1 + 2 * c], sh);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev[1 + 2 * c], 0);
+    if (e != cudaSuccess) return cuda_fail(ctx, "host-path H2D copy", e);
+    rc = run_device(ctx, din.data(), dout.data(), B, S_local, H, D, w, mode, chunked, st, pl, t0, nt);
+    if (rc) return rc;
+    e = cudaEventRecord(ev[2 + 2 * c], st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(sd, ev[2 + 2 * c], 0);
+    if (e == cudaSuccess) e = copy_rows(false, s0, s1 - s0, sd);
+    if (e != cudaSuccess) return cuda_fail(ctx, "host-path D2H copy", e);
   }
-  cudaError_t e = cudaStreamSynchronize(st);
+  e = cudaStreamSynchronize(sd);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(ctx, "cudaStreamSynchronize", e);
   return ULYSSES_A2A_OK;
 }
@@ -750,6 +847,7 @@ extern "C" int ulysses_a2a_run_noalloc(const void* const* in_slabs, void* const*
     p.Hw = (int32_t)Hw;
     p.rows_per_tile = (int32_t)rows;
     p.tiles_per_block = (int32_t)pl.tiles_per_block;
+    p.tile0 = 0;
     p.nb = (int32_t)nb;
     p.tile_bytes = (uint32_t)(rows * pl.row_bytes);
     p.stage_bytes = (p.tile_bytes + 1023u) / 1024u * 1024u;

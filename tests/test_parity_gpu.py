@@ -317,6 +317,28 @@ def test_run_host_matches_oracle():
             assert torch.equal(bits(out[k]), bits(want[k]))
 
 
+@pytest.mark.parametrize("path", [PATH_TMA, PATH_VEC], ids=["tma", "vec"])
+def test_run_host_pipelined_chunks(path):
+    # >= 8 MB of payload: the host path overlaps H2D, kernel and D2H over 8
+    # sequence chunks; S_local = 1000 leaves a ragged last tile and chunk
+    w, B, S, H, D = 4, 2, 1000, 8, 128
+    with UlyssesA2A(0, 2) as a2a:
+        a2a.set_path(path)
+        for mode in (0, 1):
+            xs = [t.pin_memory() for t in
+                  normal_slabs(slab_shape(mode, w, B, S, H, D), w, "bf16", seed0=23 + mode)]
+            want = oracle.ulysses_a2a(xs, mode)
+            for chunked in (False, True):
+                for knobs in ({}, dict(rows_per_tile=7), dict(chunk_units=0, rows_per_tile=13)):
+                    a2a.set_tuning(**knobs)
+                    n0 = a2a.launch_count
+                    out = a2a.run_host(xs, mode, chunked=chunked)
+                    assert a2a.launch_count - n0 > (B if chunked else 1)   # several chunks
+                    for k in range(w):
+                        assert torch.equal(bits(out[k]), bits(want[k])), (mode, chunked, knobs)
+        a2a.status()
+
+
 # ---- argument errors on a live device: nothing is launched ------------------
 
 def test_errors_launch_nothing():
@@ -390,3 +412,43 @@ def test_status_is_clean_and_destroy_is_idempotent_on_null():
     a2a.close()
     a2a.close()
     assert _lib.lib.ulysses_a2a_destroy(None) == _lib.OK
+
+
+# ---- the autograd pairing: backward of mode m is mode 1-m -------------------
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_autograd_backward_is_the_inverse_mode(mode, dtype):
+    from sequence_all_re_b200.autograd import all_to_all_4d
+
+    w, B, S, H, D = 4, 2, 29, 8, 64
+    E = 2 if dtype == "bf16" else 4
+    xs = normal_slabs(slab_shape(mode, w, B, S, H, D), w, dtype, seed0=500)
+    # upstream gradient: one seeded weight tensor per output slab
+    cs = normal_slabs(slab_shape(1 - mode, w, B, S, H, D), w, dtype, seed0=600)
+    with UlyssesA2A(0, E) as a2a:
+        xd = [t.cuda().requires_grad_(True) for t in xs]
+        ys = all_to_all_4d(a2a, xd, mode, chunked=(mode == 1))
+        loss = sum((y.float() * c.cuda().float()).sum() for y, c in zip(ys, cs))
+        loss.backward()
+        a2a.status()
+        want_y = oracle.ulysses_a2a(xs, mode)
+        want_g = oracle.ulysses_a2a(cs, 1 - mode)     # P^-1 applied to the weights
+        for k in range(w):
+            assert torch.equal(bits(ys[k].detach().cpu()), bits(want_y[k]))
+            assert torch.equal(bits(xd[k].grad.cpu()), bits(want_g[k]))
+
+
+def test_autograd_unused_outputs_get_zero_gradient():
+    from sequence_all_re_b200.autograd import all_to_all_4d
+
+    w, B, S, H, D = 2, 1, 16, 4, 64
+    xs = normal_slabs((B, S, H, D), w, "fp32", seed0=7)
+    with UlyssesA2A(0, 4) as a2a:
+        xd = [t.cuda().requires_grad_(True) for t in xs]
+        ys = all_to_all_4d(a2a, xd, 0)
+        ys[1].sum().backward()          # only rank 1's output is used
+        ones_then_zero = [torch.zeros_like(ys[0]).cpu(), torch.ones_like(ys[1]).cpu()]
+        want = oracle.ulysses_a2a(ones_then_zero, 1)
+        for k in range(w):
+            assert torch.equal(xd[k].grad.cpu(), want[k])
