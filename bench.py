@@ -236,6 +236,72 @@ def bench_sweep_point(a2a, w, payload, dtype, device, stream, reps):
     return P, t0, t1
 
 
+def graph_ms_per_call(a2a, src, dst, mode, calls, reps, stream):
+    """Device time per call of `calls` back-to-back calls captured in one CUDA graph."""
+    with torch.cuda.stream(stream):
+        a2a.run(src, mode, out=dst, stream=stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(calls):
+            a2a.run(src, mode, out=dst, stream=stream)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    # replay() launches on the current stream: make it the timed stream
+    with torch.cuda.stream(stream):
+        g.replay()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (reps * calls)
+    del g
+    return ms
+
+
+def bandwidth_sweep(device, peak):
+    """Payload 128 KiB .. 2 GiB (doubling), w = 2/4/8, H = 8w, D = 128, B = 1, bf16 and
+    fp32 U[-1,1), both modes; device time per call from CUDA-graph replays."""
+    from sequence_all_re_b200 import UlyssesA2A
+
+    stream = torch.cuda.Stream(device)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    rows = []
+    for dtype, E in (("bf16", 2), ("fp32", 4)):
+        a2a = UlyssesA2A(device.index or 0, E)
+        for w in (2, 4, 8):
+            H, D = 8 * w, 128
+            for k in range(17, 32):
+                P = 1 << k
+                S = P // (w * H * D * E)
+                if S < 1:
+                    rows.append({"dtype": dtype, "w": w, "payload_bytes": P, "S_local": None,
+                                 "note": "n/a: one sequence row across all ranks exceeds the payload"})
+                    continue
+                dt = torch.bfloat16 if E == 2 else torch.float32
+                x = []
+                for r in range(w):
+                    gen = torch.Generator(device=device)
+                    gen.manual_seed(1234 + r)
+                    x.append((torch.rand((1, S, H, D), generator=gen, device=device) * 2 - 1).to(dt))
+                y = [torch.empty((1, S * w, H // w, D), dtype=dt, device=device) for _ in range(w)]
+                calls = max(1, min(64, (256 << 20) // P))
+                reps = max(3, min(50, (8 << 30) // (P * calls)))
+                t0 = graph_ms_per_call(a2a, x, y, 0, calls, reps, stream)
+                t1 = graph_ms_per_call(a2a, y, x, 1, calls, reps, stream)
+                g0, g1 = P / (t0 / 1e3) / 1e9, P / (t1 / 1e3) / 1e9
+                rows.append({"dtype": dtype, "w": w, "payload_bytes": P, "S_local": S,
+                             "mode0_gbs": round(g0, 1), "mode1_gbs": round(g1, 1),
+                             "mode0_frac": round(2 * g0 / peak, 4),
+                             "mode1_frac": round(2 * g1 / peak, 4),
+                             "l2_assisted": 2 * P <= l2})
+                del x, y
+        a2a.close()
+    return rows
+
+
 def cpu_oracle_baseline(w, B, S, H, D, budget_s=12.0):
     """The oracle, as it stands, on the host: full workload steps until ~budget_s."""
     import oracle
@@ -375,6 +441,10 @@ def run_ours(args):
                 "mode1_frac": round(2 * Pw / (b / 1e3) / 1e9 / peak, 4),
             }
 
+    sweep = None
+    if args.sweep and rank == 0:
+        sweep = bandwidth_sweep(device, peak)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_baseline(w, B, S, H, D, budget_s=args.cpu_budget)
@@ -423,6 +493,8 @@ def run_ours(args):
         "w_sweep_512MiB_back_to_back": w_sweep,
         "cpu_baseline": cpu,
     }
+    if sweep is not None:
+        line["bandwidth_sweep"] = sweep
     if rank == 0:
         print(json.dumps(line), flush=True)
     a2a.close()
@@ -503,6 +575,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="also run the 128 KiB..2 GiB bandwidth sweep (w=2/4/8, bf16/fp32)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("note: warm-up raised to 3 steps", file=sys.stderr)

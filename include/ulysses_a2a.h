@@ -88,7 +88,28 @@ typedef struct ulysses_a2a_plan_t {
                                 outermost, 1 = r innermost                  */
     int32_t chunk_units;     /* TMA path: 0 = persistent grid (static round
                                 robin); n = n consecutive units per CTA     */
+    int64_t row_pitch;       /* elements between rows of the [B,S_local,H,D]
+                                side (H*D when dense)                       */
 } ulysses_a2a_plan_t;
+
+/* One call's arguments, for ulysses_a2a_run_ex / ulysses_a2a_plan_ex. Same
+ * meaning as the ulysses_a2a_run parameters, plus row_pitch: the number of
+ * elements between consecutive (b, s) rows of the [B, S_local, H, D] side (the
+ * inputs in mode 0, the outputs in mode 1), whose planes are then
+ * S_local*row_pitch elements apart; 0 means dense (H*D). A pitch > H*D lets
+ * mode 0 read q, k or v in place from a packed [B, S_local, 3, H, D] projection
+ * output (row_pitch = 3*H*D, slab pointers offset by 0, H*D or 2*H*D
+ * elements), and lets mode 1 write into such a packed buffer; elements between
+ * H*D and row_pitch are neither read nor written. The other side is always
+ * dense. */
+typedef struct ulysses_a2a_desc_t {
+    const void *const *in_slabs;
+    void *const *out_slabs;
+    int64_t B, S_local, H, D;
+    int32_t w, mode, chunked;
+    int32_t reserved;        /* must be 0 */
+    int64_t row_pitch;
+} ulysses_a2a_desc_t;
 
 /* Create a context on CUDA device `device` for elements of `elem_bytes` bytes
  * (1, 2, 4 or 8; bf16 = 2, fp32 = 4). On success *out holds a new context that
@@ -118,6 +139,10 @@ int ulysses_a2a_run(ulysses_a2a_ctx *ctx, const void *const *in_slabs,
                     void *const *out_slabs, int64_t B, int64_t S_local,
                     int64_t H, int64_t D, int w, int mode, int chunked,
                     void *stream);
+
+/* ulysses_a2a_run with the arguments in a descriptor (adds row_pitch). */
+int ulysses_a2a_run_ex(ulysses_a2a_ctx *ctx, const ulysses_a2a_desc_t *desc,
+                       void *stream);
 
 /* Same operation on HOST slabs (pageable or pinned): copies every input to
  * context-owned device buffers, runs the re-layout on `stream`, copies every
@@ -214,6 +239,12 @@ int ulysses_a2a_run_noalloc(const void *const *in_slabs, void *const *out_slabs,
                             int64_t B, int64_t S_local, int64_t H, int64_t D,
                             int w, int mode, int chunked, int elem_bytes,
                             void *stream, int wait, char *err, size_t errlen);
+
+/* ulysses_a2a_plan for a descriptor (adds row_pitch). */
+int ulysses_a2a_plan_ex(const ulysses_a2a_desc_t *desc, int elem_bytes,
+                        int forced_path, const ulysses_a2a_tuning_t *tuning,
+                        int num_sms, ulysses_a2a_plan_t *out, char *err,
+                        size_t errlen);
 
 #ifdef __cplusplus
 } /* extern "C" */

@@ -50,6 +50,11 @@ def load_library(path: str) -> ctypes.CDLL:
         fn.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_void_p),
                        ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                        ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    fn = lib.oracle_ulysses_a2a_pitched
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_void_p),
+                   ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                   ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64]
     return lib
 
 
@@ -114,3 +119,37 @@ def ulysses_a2a(inputs, mode: int, chunked: bool = False, lib: ctypes.CDLL | Non
     if rc != 0:
         raise ValueError(f"oracle rejected the arguments (rc={rc})")
     return outs
+
+
+def ulysses_a2a_pitched(bufs, mode: int, w: int, B: int, S_local: int, H: int, D: int,
+                        row_pitch: int, offset: int = 0, out_bufs=None,
+                        lib: ctypes.CDLL | None = None):
+    """The re-layout with a row pitch on the [B, S_local, H, D] side.
+
+    ``bufs``: w 1-D CPU tensors (any dtype) holding the input slabs; in mode 0
+    each is a pitched buffer read from element ``offset`` on (for example a
+    packed QKV projection output, offset selecting q, k or v), in mode 1 each is
+    a dense [B, S_local*w, H//w, D] slab. ``out_bufs``: w 1-D CPU tensors
+    receiving the output (mode 0: dense; mode 1: pitched, written from
+    ``offset`` on, gap elements untouched); allocated and 0xFF-filled if None.
+    Returns the output buffers.
+    """
+    lib = lib or _get_lib()
+    dt = bufs[0].dtype
+    E = bufs[0].element_size()
+    if out_bufs is None:
+        n = (B * S_local * H * D) if mode == 0 else ((B * S_local - 1) * row_pitch + H * D + offset)
+        out_bufs = []
+        for _ in range(w):
+            o = torch.empty(n, dtype=dt)
+            o.view(torch.uint8).fill_(0xFF)
+            out_bufs.append(o)
+    in_off = offset if mode == 0 else 0
+    out_off = offset if mode == 1 else 0
+    in_arr = (ctypes.c_void_p * w)(*[t.data_ptr() + in_off * E for t in bufs])
+    out_arr = (ctypes.c_void_p * w)(*[t.data_ptr() + out_off * E for t in out_bufs])
+    rc = lib.oracle_ulysses_a2a_pitched(in_arr, out_arr, B, S_local, H, D, w, int(mode), E,
+                                        int(row_pitch))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the arguments (rc={rc})")
+    return out_bufs

@@ -90,6 +90,45 @@ int oracle_ulysses_a2a(const void *const *in, void *const *out, int64_t B,
     return 0;
 }
 
+/* Same map with the [B, S_local, H, D] side laid out with a row pitch: the
+ * element (b, s, h, d) of that side sits at ((b*S_local + s)*row_pitch + h*D + d)
+ * (row_pitch >= H*D elements; the gathered side stays dense). This is the
+ * layout of, e.g., q inside a packed [B, S_local, 3, H, D] projection output
+ * (row_pitch = 3*H*D). Elements in the gap between H*D and row_pitch are
+ * neither read nor written. */
+int oracle_ulysses_a2a_pitched(const void *const *in, void *const *out,
+                               int64_t B, int64_t S_local, int64_t H, int64_t D,
+                               int w, int mode, int elem_bytes, int64_t row_pitch)
+{
+    if (bad_args(in, out, B, S_local, H, D, w, mode, elem_bytes)) return -1;
+    if (row_pitch < H * D) return -1;
+    const int64_t Hw = H / w;
+    const int64_t S_global = S_local * w;
+    const int64_t E = elem_bytes;
+    for (int r = 0; r < w; ++r)
+        for (int64_t b = 0; b < B; ++b)
+            for (int j = 0; j < w; ++j)
+                for (int64_t s = 0; s < S_local; ++s)
+                    for (int64_t hp = 0; hp < Hw; ++hp)
+                        for (int64_t d = 0; d < D; ++d) {
+                            /* pitched side: rank j's row (b, s), head r*Hw + h' */
+                            int64_t a = (b * S_local + s) * row_pitch
+                                        + ((int64_t)r * Hw + hp) * D + d;
+                            int64_t c = at4(b, (int64_t)j * S_local + s, hp, d,
+                                            S_global, Hw, D);
+                            if (mode == 0) {
+                                const char *src = (const char *)in[j] + a * E;
+                                char *dst = (char *)out[r] + c * E;
+                                memcpy(dst, src, (size_t)E);
+                            } else {
+                                const char *src = (const char *)in[r] + c * E;
+                                char *dst = (char *)out[j] + a * E;
+                                memcpy(dst, src, (size_t)E);
+                            }
+                        }
+    return 0;
+}
+
 /* The chunked variant: one call per plane, each on B = 1 plane views. */
 int oracle_ulysses_a2a_chunked(const void *const *in, void *const *out,
                                int64_t B, int64_t S_local, int64_t H, int64_t D,

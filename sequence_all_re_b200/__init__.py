@@ -76,7 +76,28 @@ class UlyssesA2A:
             raise A2AError(rc, self.last_error())
 
     # ------------------------------------------------------------- the op
-    def _prepare(self, xs, mode, out, device_type):
+    @staticmethod
+    def _row_pitch(ts, allow_pitch):
+        """Row pitch (elements) shared by [B, S, H, D] tensors: 0 when contiguous,
+        else p for views whose strides are (S*p, p, D, 1) with p >= H*D (for
+        example q, k or v of a packed [B, S, 3, H, D] projection output)."""
+        if all(t.is_contiguous() for t in ts):
+            return 0
+        if not allow_pitch:
+            raise ValueError("rank slabs must be contiguous")
+        B, S, H, D = ts[0].shape
+        pitch = None
+        for t in ts:
+            st = t.stride()
+            p = st[1]
+            ok = st[3] == 1 and (H == 1 or st[2] == D) and p >= H * D and (B == 1 or st[0] == S * p)
+            if not ok or (pitch is not None and p != pitch):
+                raise ValueError("a [B, S, H, D] slab must be contiguous or a view with strides "
+                                 "(S*p, p, D, 1), p >= H*D, shared by all slabs")
+            pitch = p
+        return pitch
+
+    def _prepare(self, xs, mode, out, device_type, allow_pitch=False):
         w = len(xs)
         if w < 1:
             raise ValueError("need at least one rank slab")
@@ -88,8 +109,6 @@ class UlyssesA2A:
                 raise ValueError("rank slabs must share shape and dtype")
             if t.element_size() != self.elem_bytes:
                 raise ValueError(f"context handles {self.elem_bytes}-byte elements")
-            if not t.is_contiguous():
-                raise ValueError("rank slabs must be contiguous")
             if t.device.type != device_type:
                 raise ValueError(f"rank slabs must be on {device_type}")
         if mode not in (0, 1):
@@ -105,22 +124,31 @@ class UlyssesA2A:
             if len(out) != w:
                 raise ValueError("need one output per rank")
             for o in out:
-                if tuple(o.shape) != oshape or o.dtype != xs[0].dtype or not o.is_contiguous():
-                    raise ValueError(f"outputs must be contiguous {oshape} {xs[0].dtype}")
+                if tuple(o.shape) != oshape or o.dtype != xs[0].dtype:
+                    raise ValueError(f"outputs must be {oshape} {xs[0].dtype}")
+        # the [B, S, H, D] side (inputs in mode 0, outputs in mode 1) may be pitched
+        strided, dense = (xs, out) if mode == 0 else (out, xs)
+        pitch = self._row_pitch(strided, allow_pitch)
+        if not all(t.is_contiguous() for t in dense):
+            raise ValueError("the [B, S_local*w, H/w, D] slabs must be contiguous")
+        self._last_pitch = pitch
         return w, (B, S, H, D), out
 
     def run(self, xs, mode: int, chunked: bool = False, out=None, stream=None):
         """Re-layout device slabs ``xs`` (list of w tensors); returns the w outputs.
 
-        Asynchronous on ``stream`` (default: torch's current stream on the device).
+        The [B, S_local, H, D] side (``xs`` in mode 0, ``out`` in mode 1) may be
+        a row-pitched view, e.g. ``qkv[:, :, 0]`` of a packed [B, S, 3, H, D]
+        projection output: it is read or written in place. Asynchronous on
+        ``stream`` (default: torch's current stream on the device).
         """
-        w, (B, S, H, D), out = self._prepare(xs, mode, out, "cuda")
+        w, (B, S, H, D), out = self._prepare(xs, mode, out, "cuda", allow_pitch=True)
         if stream is None:
             stream = torch.cuda.current_stream(self.device)
         handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
-        rc = _lib.ulysses_a2a_run(self._ctx, [t.data_ptr() for t in xs],
-                                  [o.data_ptr() for o in out], B, S, H, D, w, mode,
-                                  int(bool(chunked)), handle)
+        rc = _lib.ulysses_a2a_run_ex(self._ctx, [t.data_ptr() for t in xs],
+                                     [o.data_ptr() for o in out], B, S, H, D, w, mode,
+                                     int(bool(chunked)), self._last_pitch, handle)
         self._check(rc)
         return out
 
@@ -146,10 +174,11 @@ class UlyssesA2A:
     def plan(self, xs, mode: int, chunked: bool = False, out=None, knobs=None) -> dict:
         """The path and geometry a run with these tensors would use (host only), for the
         default tuning or the given ``knobs`` dict."""
-        w, (B, S, H, D), out = self._prepare(xs, mode, out, xs[0].device.type)
-        rc, p, msg = _lib.ulysses_a2a_plan([t.data_ptr() for t in xs], [o.data_ptr() for o in out],
-                                           B, S, H, D, w, mode, int(bool(chunked)),
-                                           self.elem_bytes, **(knobs or {}))
+        w, (B, S, H, D), out = self._prepare(xs, mode, out, xs[0].device.type, allow_pitch=True)
+        rc, p, msg = _lib.ulysses_a2a_plan_ex([t.data_ptr() for t in xs],
+                                              [o.data_ptr() for o in out], B, S, H, D, w, mode,
+                                              int(bool(chunked)), self.elem_bytes,
+                                              row_pitch=self._last_pitch, **(knobs or {}))
         if rc != _lib.OK:
             raise A2AError(rc, msg)
         return p.as_dict()

@@ -41,6 +41,8 @@ EXPORTED = (
     "ulysses_a2a_launch_count",
     "ulysses_a2a_plan",
     "ulysses_a2a_run_noalloc",
+    "ulysses_a2a_run_ex",
+    "ulysses_a2a_plan_ex",
 )
 
 
@@ -65,6 +67,7 @@ class PlanT(ctypes.Structure):
         ("smem_bytes", ctypes.c_int64),
         ("order", ctypes.c_int32),
         ("chunk_units", ctypes.c_int32),
+        ("row_pitch", ctypes.c_int64),
     ]
 
     def as_dict(self) -> dict:
@@ -96,6 +99,35 @@ class TuningT(ctypes.Structure):
                 raise TypeError(f"unknown tuning knob {k!r}")
             vals[k] = int(v)
         return cls(**vals)
+
+
+class DescT(ctypes.Structure):
+    """Mirror of ``ulysses_a2a_desc_t``."""
+
+    _fields_ = [
+        ("in_slabs", ctypes.POINTER(ctypes.c_void_p)),
+        ("out_slabs", ctypes.POINTER(ctypes.c_void_p)),
+        ("B", ctypes.c_int64),
+        ("S_local", ctypes.c_int64),
+        ("H", ctypes.c_int64),
+        ("D", ctypes.c_int64),
+        ("w", ctypes.c_int32),
+        ("mode", ctypes.c_int32),
+        ("chunked", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("row_pitch", ctypes.c_int64),
+    ]
+
+
+def make_desc(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, row_pitch=0):
+    """A DescT plus the pointer arrays it references (keep both alive together)."""
+    ins = ptr_array(in_ptrs) if in_ptrs is not None else None
+    outs = ptr_array(out_ptrs) if out_ptrs is not None else None
+    d = DescT(ctypes.cast(ins, ctypes.POINTER(ctypes.c_void_p)) if ins is not None else None,
+              ctypes.cast(outs, ctypes.POINTER(ctypes.c_void_p)) if outs is not None else None,
+              int(B), int(S_local), int(H), int(D), int(w), int(mode), int(chunked), 0,
+              int(row_pitch))
+    return d, (ins, outs)
 
 
 class A2AError(RuntimeError):
@@ -140,6 +172,12 @@ def _load() -> ctypes.CDLL:
     lib.ulysses_a2a_run_noalloc.argtypes = [PP, PP, i64, i64, i64, i64, c_int, c_int, c_int, c_int,
                                             P, c_int, ctypes.c_char_p, ctypes.c_size_t]
     lib.ulysses_a2a_run_noalloc.restype = c_int
+    lib.ulysses_a2a_run_ex.argtypes = [P, ctypes.POINTER(DescT), P]
+    lib.ulysses_a2a_run_ex.restype = c_int
+    lib.ulysses_a2a_plan_ex.argtypes = [ctypes.POINTER(DescT), c_int, c_int, ctypes.POINTER(TuningT),
+                                        c_int, ctypes.POINTER(PlanT), ctypes.c_char_p,
+                                        ctypes.c_size_t]
+    lib.ulysses_a2a_plan_ex.restype = c_int
     return lib
 
 
@@ -222,4 +260,22 @@ def ulysses_a2a_plan(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, elem
     rc = lib.ulysses_a2a_plan(ins, outs, int(B), int(S_local), int(H), int(D), int(w), int(mode),
                               int(chunked), int(elem_bytes), int(forced_path), ctypes.byref(t),
                               int(num_sms), ctypes.byref(plan), buf, len(buf))
+    return rc, plan, buf.value.decode()
+
+
+def ulysses_a2a_run_ex(ctx, in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, row_pitch,
+                       stream) -> int:
+    d, keep = make_desc(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, row_pitch)
+    return lib.ulysses_a2a_run_ex(ctx, ctypes.byref(d), ctypes.c_void_p(int(stream)))
+
+
+def ulysses_a2a_plan_ex(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, elem_bytes,
+                        row_pitch=0, forced_path=PATH_AUTO, num_sms=148, **knobs):
+    """Host-only planning of a descriptor (no CUDA call). Returns (rc, PlanT, message)."""
+    d, keep = make_desc(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, row_pitch)
+    plan = PlanT()
+    buf = ctypes.create_string_buffer(256)
+    t = TuningT.make(**knobs)
+    rc = lib.ulysses_a2a_plan_ex(ctypes.byref(d), int(elem_bytes), int(forced_path),
+                                 ctypes.byref(t), int(num_sms), ctypes.byref(plan), buf, len(buf))
     return rc, plan, buf.value.decode()

@@ -47,6 +47,7 @@ struct VecParams {
   int64_t S_local;
   int64_t b0;            // first plane of this launch
   int64_t nv;            // vectors per run: L*E / V
+  int64_t srow;          // vectors between rows (b, s), (b, s+1) of the [B,S,H,D] side
   int32_t w;
   int32_t rows_per_tile;
   uint32_t units;        // w * nb * w * T
@@ -72,7 +73,7 @@ __device__ __forceinline__ void st_stream(unsigned char* p, unsigned char v) { _
 template <typename V, int MODE, int U>
 __global__ void __launch_bounds__(256) ua2a_vec_kernel(const __grid_constant__ VecParams p) {
   const uint32_t nv = (uint32_t)p.nv;
-  const int64_t strided_row = (int64_t)p.w * p.nv;  // vectors between rows s, s+1 of [B,S,H,D]
+  const int64_t strided_row = p.srow;  // vectors between rows s, s+1 of [B,S,H,D] (pitch)
   const uint32_t step = blockDim.x * U;
   for (uint32_t u = blockIdx.x; u < p.units; u += gridDim.x) {
     uint32_t t, j, r, bl;

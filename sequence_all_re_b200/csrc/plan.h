@@ -81,15 +81,16 @@ inline bool overlaps(uintptr_t a, uintptr_t a_end, uintptr_t b, uintptr_t b_end)
 // Why the TMA path cannot take a shape (nullptr if it can).
 inline const char* tma_blocker(const void* const* in, void* const* out, int64_t B,
                                int64_t S, int64_t H, int64_t D, int w, int E,
-                               int64_t row_bytes) {
+                               int64_t row_bytes, int64_t pitch) {
   const int64_t Hw = H / w;
+  if ((pitch * E) % 16 != 0) return "the row pitch is not a multiple of 16 bytes";
   if (w > ULYSSES_A2A_MAX_W_TMA) return "w exceeds the TMA path's rank limit";
   if (D > kTmaMaxBoxDim || Hw > kTmaMaxBoxDim) return "D or H/w exceeds a TMA box dimension (256)";
   if ((D * E) % 16 != 0) return "D*elem_bytes is not a multiple of 16 bytes";
   if (row_bytes > kTmaMaxTileBytes) return "one row run exceeds the TMA tile limit";
   if (S > INT32_MAX || B > INT32_MAX) return "S_local or B exceeds a TMA coordinate";
   // global strides must stay below 2^40 bytes: the largest is one plane
-  if (S * H * D * E >= (int64_t(1) << 40)) return "plane stride exceeds the TMA stride limit";
+  if (S * pitch * E >= (int64_t(1) << 40)) return "plane stride exceeds the TMA stride limit";
   for (int k = 0; k < w; ++k) {
     if ((reinterpret_cast<uintptr_t>(in[k]) & 15u) != 0 ||
         (reinterpret_cast<uintptr_t>(out[k]) & 15u) != 0)
@@ -125,10 +126,12 @@ inline bool tuning_from(const ulysses_a2a_tuning_t* t, Tuning* out, std::string*
 }
 
 // Validate and plan one call. Returns a ULYSSES_A2A_* status.
+// row_pitch: elements between consecutive (b, s) rows of the [B, S, H, D]
+// side (0 = dense, H*D); that side's planes are S*row_pitch elements apart.
 inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t S,
                      int64_t H, int64_t D, int w, int mode, int chunked, int E,
                      int forced_path, const Tuning& tune, int num_sms,
-                     ulysses_a2a_plan_t* p, std::string* err) {
+                     ulysses_a2a_plan_t* p, std::string* err, int64_t row_pitch = 0) {
   if (p == nullptr) { set_err(err, "plan output is NULL"); return ULYSSES_A2A_ERR_INVALID; }
   *p = ulysses_a2a_plan_t{};
   if (in == nullptr || out == nullptr) {
@@ -157,33 +160,49 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
   if (num_sms < 1) { set_err(err, "num_sms must be >= 1"); return ULYSSES_A2A_ERR_INVALID; }
 
   // sizes, overflow-checked
-  int64_t plane_elems, slab_elems, slab_bytes, payload, tmp;
+  int64_t plane_elems, slab_elems, slab_bytes, payload, tmp, HD;
   if (mul_overflows(S, H, &tmp) || mul_overflows(tmp, D, &plane_elems) ||
       mul_overflows(plane_elems, B, &slab_elems) || mul_overflows(slab_elems, E, &slab_bytes) ||
-      mul_overflows(slab_bytes, (int64_t)w, &payload) || payload > (int64_t(1) << 56)) {
+      mul_overflows(slab_bytes, (int64_t)w, &payload) || payload > (int64_t(1) << 56) ||
+      mul_overflows(H, D, &HD)) {
     set_err(err, "slab sizes overflow");
     return ULYSSES_A2A_ERR_INVALID;
   }
+  const int64_t pitch = row_pitch == 0 ? HD : row_pitch;
+  if (pitch < HD) {
+    set_err(err, "row pitch %lld is smaller than H*D = %lld", pitch, HD);
+    return ULYSSES_A2A_ERR_INVALID;
+  }
+  // bytes spanned by one slab of the [B, S, H, D] side (gaps included)
+  int64_t strided_bytes;
+  if (mul_overflows(B * S - 1, pitch, &tmp) || mul_overflows(tmp + HD, (int64_t)E, &strided_bytes) ||
+      strided_bytes > (int64_t(1) << 56)) {
+    set_err(err, "pitched slab extent overflows");
+    return ULYSSES_A2A_ERR_INVALID;
+  }
+  const int64_t in_bytes = mode == 0 ? strided_bytes : slab_bytes;
+  const int64_t out_bytes = mode == 0 ? slab_bytes : strided_bytes;
   for (int k = 0; k < w; ++k) {
     if (in[k] == nullptr || out[k] == nullptr) {
       set_err(err, "slab pointer %lld is NULL", k);
       return ULYSSES_A2A_ERR_INVALID;
     }
   }
-  // No output may overlap an input or another output (inputs may alias each other).
+  // No output may overlap an input or another output (inputs may alias each
+  // other). A pitched slab counts with its whole extent, gaps included.
   for (int k = 0; k < w; ++k) {
     const uintptr_t o = reinterpret_cast<uintptr_t>(out[k]);
-    const uintptr_t oe = o + (uintptr_t)slab_bytes;
+    const uintptr_t oe = o + (uintptr_t)out_bytes;
     if (oe < o) { set_err(err, "output slab %lld wraps the address space", k); return ULYSSES_A2A_ERR_INVALID; }
     for (int m = 0; m < w; ++m) {
       const uintptr_t i = reinterpret_cast<uintptr_t>(in[m]);
-      if (overlaps(o, oe, i, i + (uintptr_t)slab_bytes)) {
+      if (overlaps(o, oe, i, i + (uintptr_t)in_bytes)) {
         set_err(err, "output slab %lld overlaps input slab %lld", k, m);
         return ULYSSES_A2A_ERR_OVERLAP;
       }
       if (m != k) {
         const uintptr_t q = reinterpret_cast<uintptr_t>(out[m]);
-        if (overlaps(o, oe, q, q + (uintptr_t)slab_bytes)) {
+        if (overlaps(o, oe, q, q + (uintptr_t)out_bytes)) {
           set_err(err, "output slab %lld overlaps output slab %lld", k, m);
           return ULYSSES_A2A_ERR_OVERLAP;
         }
@@ -193,7 +212,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
 
   const int64_t Hw = H / w;
   const int64_t row_bytes = Hw * D * E;  // one contiguous run, L*E
-  const char* blocker = tma_blocker(in, out, B, S, H, D, w, E, row_bytes);
+  const char* blocker = tma_blocker(in, out, B, S, H, D, w, E, row_bytes, pitch);
   int path;
   if (forced_path == ULYSSES_A2A_PATH_TMA) {
     if (blocker) {
@@ -233,6 +252,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
   p->units = units;
   p->payload_bytes = payload;
   p->launches = chunked ? (int32_t)(B > INT32_MAX ? INT32_MAX : B) : 1;
+  p->row_pitch = pitch;
   p->order = tune.order >= 0 ? (tune.order ? 1 : 0) : kDefaultOrder;
 
   if (path == ULYSSES_A2A_PATH_TMA) {
@@ -299,7 +319,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
   if (path == ULYSSES_A2A_PATH_VEC) {
     int v = 16;
     while (v > 1) {
-      bool ok = (row_bytes % v) == 0;
+      bool ok = (row_bytes % v) == 0 && ((pitch * E) % v) == 0;
       for (int k = 0; k < w && ok; ++k)
         ok = (reinterpret_cast<uintptr_t>(in[k]) % v) == 0 &&
              (reinterpret_cast<uintptr_t>(out[k]) % v) == 0;

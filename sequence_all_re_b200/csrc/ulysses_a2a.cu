@@ -55,7 +55,7 @@ struct TmaCacheEntry {
   bool valid = false;
   uint64_t stamp = 0;
   int mode = 0, w = 0;
-  int64_t B = 0, S = 0, H = 0, D = 0, rows = 0;
+  int64_t B = 0, S = 0, H = 0, D = 0, rows = 0, pitch = 0;
   const void* in[ULYSSES_A2A_MAX_W_TMA] = {};
   void* out[ULYSSES_A2A_MAX_W_TMA] = {};
   TmaParams params;  // tensor maps + geometry (b0/nb/status filled per launch)
@@ -122,10 +122,10 @@ CUtensorMapDataType map_dtype(int E) {
 // Tensor maps of one strided-side slab [B, S, H, D] and one gathered-side slab
 // [B, S*w, H/w, D] (viewed as [B, w, S, H/w, D] so rows stop at S per block).
 int encode_strided(ulysses_a2a_ctx* ctx, CUtensorMap* m, const void* base, int64_t B, int64_t S,
-                   int64_t H, int64_t D, int64_t Hw, int64_t rows) {
+                   int64_t H, int64_t D, int64_t Hw, int64_t rows, int64_t pitch) {
   const int64_t E = ctx->elem_bytes;
   cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
-  cuuint64_t strides[3] = {(cuuint64_t)(D * E), (cuuint64_t)(H * D * E), (cuuint64_t)(S * H * D * E)};
+  cuuint64_t strides[3] = {(cuuint64_t)(D * E), (cuuint64_t)(pitch * E), (cuuint64_t)(S * pitch * E)};
   cuuint32_t box[4] = {(cuuint32_t)D, (cuuint32_t)Hw, (cuuint32_t)rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = ctx->encode_tiled(m, map_dtype((int)E), 4, const_cast<void*>(base), dims, strides, box,
@@ -157,10 +157,11 @@ int tma_params_for(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out
                    int64_t S, int64_t H, int64_t D, int w, int mode, const ulysses_a2a_plan_t& pl,
                    TmaParams** result) {
   const int64_t rows = pl.rows_per_tile;
+  const int64_t pitch = pl.row_pitch;
   TmaCacheEntry* victim = &ctx->tma_cache[0];
   for (auto& e : ctx->tma_cache) {
     if (e.valid && e.mode == mode && e.w == w && e.B == B && e.S == S && e.H == H && e.D == D &&
-        e.rows == rows) {
+        e.rows == rows && e.pitch == pitch) {
       bool same = true;
       for (int k = 0; k < w && same; ++k) same = e.in[k] == in[k] && e.out[k] == out[k];
       if (same) {
@@ -183,7 +184,7 @@ int tma_params_for(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out
   for (int k = 0; k < w; ++k) {
     const void* strided = mode == 0 ? in[k] : out[k];
     const void* gathered = mode == 0 ? out[k] : in[k];
-    int rc = encode_strided(ctx, &fresh.params.strided[k], strided, B, S, H, D, Hw, rows);
+    int rc = encode_strided(ctx, &fresh.params.strided[k], strided, B, S, H, D, Hw, rows, pitch);
     if (rc) return rc;
     rc = encode_gathered(ctx, &fresh.params.gathered[k], gathered, B, S, Hw, D, w, rows);
     if (rc) return rc;
@@ -199,6 +200,7 @@ int tma_params_for(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out
   fresh.H = H;
   fresh.D = D;
   fresh.rows = rows;
+  fresh.pitch = pitch;
   TmaParams& p = fresh.params;
   p.status = ctx->d_status;
   p.w = w;
@@ -324,6 +326,7 @@ int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, in
   }
   p.S_local = S;
   p.nv = pl.row_bytes / pl.vec_bytes;
+  p.srow = pl.row_pitch * ctx->elem_bytes / pl.vec_bytes;
   p.w = w;
   p.rows_per_tile = (int32_t)pl.rows_per_tile;
   p.units = (uint32_t)units;
@@ -343,10 +346,11 @@ int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, in
 }
 
 int plan_for(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, int64_t B, int64_t S,
-             int64_t H, int64_t D, int w, int mode, int chunked, ulysses_a2a_plan_t* pl) {
+             int64_t H, int64_t D, int w, int mode, int chunked, ulysses_a2a_plan_t* pl,
+             int64_t row_pitch = 0) {
   std::string err;
   int rc = ua2a::make_plan(in, out, B, S, H, D, w, mode, chunked, ctx->elem_bytes, ctx->forced_path,
-                           ctx->tuning, ctx->num_sms, pl, &err);
+                           ctx->tuning, ctx->num_sms, pl, &err, row_pitch);
   if (rc) return fail(ctx, rc, err);
   return ULYSSES_A2A_OK;
 }
@@ -426,23 +430,45 @@ int ulysses_a2a_destroy(ulysses_a2a_ctx* ctx) {
   return rc;
 }
 
-int ulysses_a2a_run(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void* const* out_slabs,
-                    int64_t B, int64_t S_local, int64_t H, int64_t D, int w, int mode, int chunked,
-                    void* stream) {
+int ulysses_a2a_run_ex(ulysses_a2a_ctx* ctx, const ulysses_a2a_desc_t* d, void* stream) {
   if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
   ctx->last_error.clear();
+  if (d == nullptr) return fail(ctx, ULYSSES_A2A_ERR_INVALID, "descriptor is NULL");
+  if (d->reserved != 0 || d->row_pitch < 0)
+    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "descriptor: reserved must be 0, row_pitch >= 0");
   ulysses_a2a_plan_t pl;
-  int rc = plan_for(ctx, in_slabs, out_slabs, B, S_local, H, D, w, mode, chunked, &pl);
+  int rc = plan_for(ctx, d->in_slabs, d->out_slabs, d->B, d->S_local, d->H, d->D, d->w, d->mode,
+                    d->chunked, &pl, d->row_pitch);
   if (rc) return rc;
   DeviceGuard g(ctx->device);
   if (!g.ok) return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "cannot select the context's device");
-  const int64_t slab_bytes = pl.payload_bytes / w;
-  rc = check_residency(ctx, in_slabs, w, slab_bytes, "input");
+  const int64_t dense_bytes = pl.payload_bytes / d->w;
+  const int64_t strided_bytes = ((d->B * d->S_local - 1) * pl.row_pitch + d->H * d->D) *
+                                (int64_t)ctx->elem_bytes;
+  rc = check_residency(ctx, d->in_slabs, d->w, d->mode == 0 ? strided_bytes : dense_bytes, "input");
   if (rc) return rc;
-  rc = check_residency(ctx, reinterpret_cast<const void* const*>(out_slabs), w, slab_bytes, "output");
+  rc = check_residency(ctx, reinterpret_cast<const void* const*>(d->out_slabs), d->w,
+                       d->mode == 0 ? dense_bytes : strided_bytes, "output");
   if (rc) return rc;
-  return run_device(ctx, in_slabs, out_slabs, B, S_local, H, D, w, mode, chunked,
-                    static_cast<cudaStream_t>(stream), pl);
+  return run_device(ctx, d->in_slabs, d->out_slabs, d->B, d->S_local, d->H, d->D, d->w, d->mode,
+                    d->chunked, static_cast<cudaStream_t>(stream), pl);
+}
+
+int ulysses_a2a_run(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void* const* out_slabs,
+                    int64_t B, int64_t S_local, int64_t H, int64_t D, int w, int mode, int chunked,
+                    void* stream) {
+  ulysses_a2a_desc_t d{};
+  d.in_slabs = in_slabs;
+  d.out_slabs = out_slabs;
+  d.B = B;
+  d.S_local = S_local;
+  d.H = H;
+  d.D = D;
+  d.w = w;
+  d.mode = mode;
+  d.chunked = chunked;
+  d.row_pitch = 0;
+  return ulysses_a2a_run_ex(ctx, &d, stream);
 }
 
 int ulysses_a2a_run_host(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void* const* out_slabs,
@@ -620,6 +646,28 @@ int ulysses_a2a_set_tuning(ulysses_a2a_ctx* ctx, const ulysses_a2a_tuning_t* t) 
 
 uint64_t ulysses_a2a_launch_count(const ulysses_a2a_ctx* ctx) {
   return ctx ? ctx->launches : 0;
+}
+
+int ulysses_a2a_plan_ex(const ulysses_a2a_desc_t* d, int elem_bytes, int forced_path,
+                        const ulysses_a2a_tuning_t* tuning, int num_sms, ulysses_a2a_plan_t* out,
+                        char* err, size_t errlen) {
+  ua2a::Tuning t;
+  std::string msg;
+  int rc = ULYSSES_A2A_OK;
+  if (d == nullptr) {
+    msg = "descriptor is NULL";
+    rc = ULYSSES_A2A_ERR_INVALID;
+  } else if (d->reserved != 0 || d->row_pitch < 0) {
+    msg = "descriptor: reserved must be 0, row_pitch >= 0";
+    rc = ULYSSES_A2A_ERR_INVALID;
+  } else if (!ua2a::tuning_from(tuning, &t, &msg)) {
+    rc = ULYSSES_A2A_ERR_INVALID;
+  } else {
+    rc = ua2a::make_plan(d->in_slabs, d->out_slabs, d->B, d->S_local, d->H, d->D, d->w, d->mode,
+                         d->chunked, elem_bytes, forced_path, t, num_sms, out, &msg, d->row_pitch);
+  }
+  if (err && errlen) std::snprintf(err, errlen, "%s", rc ? msg.c_str() : "");
+  return rc;
 }
 
 int ulysses_a2a_plan(const void* const* in_slabs, void* const* out_slabs, int64_t B,
@@ -876,6 +924,7 @@ extern "C" int ulysses_a2a_run_noalloc(const void* const* in_slabs, void* const*
     }
     p.S_local = S_local;
     p.nv = pl.row_bytes / pl.vec_bytes;
+    p.srow = pl.row_pitch * elem_bytes / pl.vec_bytes;
     p.w = w;
     p.rows_per_tile = (int32_t)pl.rows_per_tile;
     p.units = (uint32_t)pl.units;

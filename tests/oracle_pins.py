@@ -207,6 +207,68 @@ def pin_bits_not_values(run):
         assert torch.equal(y[r].view(torch.int32), want[r]), "bit pattern changed"
 
 
+def _pitched_run_default(run):
+    """The pitched oracle bound to the same library build as `run` (see oracle_pins users)."""
+    return getattr(run, "pitched", None)
+
+
+def pin_pitched_packed_qkv(run):
+    """q, k, v read in place from a packed [B, S, 3, H, D] buffer (row pitch 3*H*D) give
+    the same result as the dense oracle on torch's own q/k/v slices."""
+    pitched = _pitched_run_default(run)
+    if pitched is None:
+        return
+    for (w, B, S, H, D) in [(2, 1, 3, 4, 2), (4, 2, 5, 8, 3), (3, 2, 4, 6, 2)]:
+        packed = unique_slabs((B, S, 3, H, D), w, 4)
+        for c in range(3):
+            dense_in = [t[:, :, c].contiguous() for t in packed]
+            want = run(dense_in, 0, False)
+            got = pitched([t.reshape(-1) for t in packed], 0, w, B, S, H, D, 3 * H * D,
+                          offset=c * H * D)
+            for r in range(w):
+                assert torch.equal(got[r].reshape(want[r].shape), want[r]), f"pitched mode 0 c={c}"
+
+
+def pin_pitched_mode1_writes_only_its_slot(run):
+    """Mode 1 into slot c of packed [B, S, 3, H, D] outputs: that slot equals the dense
+    oracle's output, the other two slots keep their poison bytes."""
+    pitched = _pitched_run_default(run)
+    if pitched is None:
+        return
+    w, B, S, H, D = 4, 2, 3, 8, 2
+    ys = unique_slabs((B, S * w, H // w, D), w, 4)
+    want = run(ys, 1, False)
+    for c in range(3):
+        outs = [torch.full((B * S * 3 * H * D,), -1, dtype=torch.int32) for _ in range(w)]
+        pitched([t.reshape(-1) for t in ys], 1, w, B, S, H, D, 3 * H * D, offset=c * H * D,
+                out_bufs=outs)
+        for j in range(w):
+            v = outs[j].view(B, S, 3, H, D)
+            assert torch.equal(v[:, :, c], want[j]), f"pitched mode 1 slot {c}"
+            for other in range(3):
+                if other != c:
+                    assert bool((v[:, :, other] == -1).all()), "a gap element was written"
+
+
+def pin_pitched_hand_table(run):
+    """w=2, B=1, S_local=2, H=2, D=1, row pitch 3: rows are (head 0, head 1, gap).
+    Derived by hand as in hand_w2_B1_S2_H2_D1.txt: rank r keeps head r."""
+    pitched = _pitched_run_default(run)
+    if pitched is None:
+        return
+    # x0 = [a0 a1 g | a2 a3 g], x1 = [b0 b1 g | b2 b3 g], g = gap
+    a0, a1, a2, a3, b0, b1, b2, b3, g = 1, 2, 3, 4, 5, 6, 7, 8, 99
+    x = [torch.tensor([a0, a1, g, a2, a3, g], dtype=torch.int32),
+         torch.tensor([b0, b1, g, b2, b3, g], dtype=torch.int32)]
+    out = pitched(x, 0, 2, 1, 2, 2, 1, 3)
+    assert out[0].tolist() == [a0, a2, b0, b2]
+    assert out[1].tolist() == [a1, a3, b1, b3]
+    back = pitched(out, 1, 2, 1, 2, 2, 1, 3,
+                   out_bufs=[torch.full((6,), 0, dtype=torch.int32) for _ in range(2)])
+    assert back[0].tolist() == [a0, a1, 0, a2, a3, 0]
+    assert back[1].tolist() == [b0, b1, 0, b2, b3, 0]
+
+
 ALL_PINS = [
     pin_hand_tables,
     pin_identity_w1,
@@ -216,4 +278,7 @@ ALL_PINS = [
     pin_rank_tagged_bf16_width,
     pin_chunked_equals_unchunked,
     pin_bits_not_values,
+    pin_pitched_packed_qkv,
+    pin_pitched_mode1_writes_only_its_slot,
+    pin_pitched_hand_table,
 ]

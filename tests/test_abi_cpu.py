@@ -37,8 +37,10 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_plan_struct_layout_matches_header():
-    # int32 path, vec_bytes; 6 x int64; 6 x int32; int64; 2 x int32 -> 96 bytes
-    assert ctypes.sizeof(_lib.PlanT) == 96
+    # int32 path, vec_bytes; 6 x int64; 6 x int32; int64; 2 x int32; int64 -> 104 bytes
+    assert ctypes.sizeof(_lib.PlanT) == 104
+    # two pointers, 4 x int64, 4 x int32, int64 -> 72 bytes
+    assert ctypes.sizeof(_lib.DescT) == 72
 
 
 def fake_slabs(w, slab_bytes, base=1 << 40, align=256, gap=0):
@@ -303,3 +305,49 @@ def test_create_rejects_bad_element_size_before_touching_cuda():
     h = ctypes.c_void_p()
     assert _lib.lib.ulysses_a2a_create(ctypes.byref(h), 0, 3) == ERR_INVALID
     assert _lib.lib.ulysses_a2a_create(None, 0, 2) == ERR_INVALID
+
+
+# ---- row pitch on the [B, S, H, D] side (packed QKV layouts) -----------------
+
+def plan_ex(w, B, S, H, D, pitch, mode=0, E=2, base=1 << 40, **kw):
+    ext = ((B * S - 1) * pitch + H * D) * E
+    dense = B * S * H * D * E
+    step = (max(ext, dense) + 4095) // 4096 * 4096
+    ins = [base + k * step for k in range(w)]
+    outs = [base + (w + k) * step for k in range(w)]
+    return _lib.ulysses_a2a_plan_ex(ins, outs, B, S, H, D, w, mode, 0, E, row_pitch=pitch, **kw)
+
+
+def test_pitch_defaults_to_dense_and_is_reported():
+    rc, p, _ = plan_ex(4, 1, 64, 8, 64, 0)
+    assert rc == OK and p.row_pitch == 8 * 64
+    rc, p, _ = plan_ex(4, 1, 64, 8, 64, 3 * 8 * 64)
+    assert rc == OK and p.row_pitch == 3 * 8 * 64 and p.path == PATH_TMA
+
+
+def test_pitch_smaller_than_a_row_is_rejected():
+    rc, _, msg = plan_ex(4, 1, 64, 8, 64, 8 * 64 - 1)
+    assert rc == ERR_INVALID and "pitch" in msg
+
+
+def test_pitch_alignment_selects_the_vector_width():
+    # pitch * E = (512 + 4) * 2 bytes: 8-byte aligned rows only
+    rc, p, _ = plan_ex(4, 1, 64, 8, 64, 8 * 64 + 4)
+    assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 8
+    rc, _, msg = plan_ex(4, 1, 64, 8, 64, 8 * 64 + 4, forced_path=PATH_TMA)
+    assert rc == ERR_UNSUPPORTED and "pitch" in msg
+
+
+def test_pitched_extent_counts_for_overlap():
+    # mode 1 writes pitched outputs: a second output placed inside the first
+    # one's gaps still overlaps its extent
+    w, B, S, H, D, E = 2, 1, 4, 4, 8, 2
+    pitch = 3 * H * D
+    ins = [1 << 40, (1 << 40) + (1 << 20)]
+    outs = [(1 << 41), (1 << 41) + H * D * E]          # interleaved like k next to q
+    rc, _, msg = _lib.ulysses_a2a_plan_ex(ins, outs, B, S, H, D, w, 1, 0, E, row_pitch=pitch)
+    assert rc == ERR_OVERLAP
+    # the same pointers as *inputs* of mode 0 may alias (q, k, v of one buffer)
+    rc, _, _ = _lib.ulysses_a2a_plan_ex(outs, [1 << 42, (1 << 42) + (1 << 20)], B, S, H, D, w, 0,
+                                        0, E, row_pitch=pitch)
+    assert rc == OK

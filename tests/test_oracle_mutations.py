@@ -57,6 +57,14 @@ MUTATIONS = {
     "chunked_plane_stride": (
         "const int64_t plane = S_local * H * D;",
         "const int64_t plane = S_local * D * w;"),
+    # pitched side indexed as if dense (row pitch ignored)
+    "pitch_ignored": (
+        "int64_t a = (b * S_local + s) * row_pitch",
+        "int64_t a = (b * S_local + s) * (H * D)"),
+    # pitched side: head group taken from the source rank
+    "pitched_head_group": (
+        "+ ((int64_t)r * Hw + hp) * D + d;",
+        "+ ((int64_t)j * Hw + hp) * D + d;"),
     # mode 1 copies the wrong way round (reads the destination layout's offset)
     "mode1_swapped_offsets": (
         "const char *src = (const char *)in[r] + c * E;",
@@ -67,6 +75,11 @@ MUTATIONS = {
 def _run_all_pins(lib):
     def run(xs, mode, chunked):
         return oracle.ulysses_a2a(xs, mode, chunked, lib=lib)
+
+    def pitched(*a, **k):
+        return oracle.ulysses_a2a_pitched(*a, lib=lib, **k)
+
+    run.pitched = pitched
     failed = []
     for pin in ALL_PINS:
         try:
@@ -76,13 +89,32 @@ def _run_all_pins(lib):
     return failed
 
 
+# the same edits applied to the second copy of a loop (the pitched function)
+MUTATIONS.update({
+    "pitched_drops_last_row": (
+        "for (int64_t s = 0; s < S_local; ++s)",
+        "for (int64_t s = 0; s < S_local - 1; ++s)", 1),
+    "pitched_partial_element": (
+        "memcpy(dst, src, (size_t)E);\n                            } else {",
+        "memcpy(dst, src, (size_t)1);\n                            } else {", 1),
+})
+
+
+def _apply(text, old, new, nth=0):
+    """Replace the nth occurrence (0-based) of `old` in `text`."""
+    at = -1
+    for _ in range(nth + 1):
+        at = text.find(old, at + 1)
+        assert at >= 0, "mutation anchor not found"
+    return text[:at] + new + text[at + len(old):]
+
+
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_mutation_is_caught(name, tmp_path):
-    old, new = MUTATIONS[name]
+    old, new, *nth = MUTATIONS[name]
     text = open(SRC).read()
-    assert text.count(old) == 1, f"mutation anchor for {name} not found exactly once"
     mutated = tmp_path / "mutated.c"
-    mutated.write_text(text.replace(old, new))
+    mutated.write_text(_apply(text, old, new, nth[0] if nth else 0))
     so = oracle.build(force=True, src=str(mutated), out=str(tmp_path / f"lib_{name}.so"),
                       extra=("-Wno-unused-variable", "-Wno-error"))
     lib = oracle.load_library(so)

@@ -11,6 +11,9 @@ def _run(xs, mode, chunked):
     return oracle.ulysses_a2a(xs, mode, chunked)
 
 
+_run.pitched = oracle.ulysses_a2a_pitched
+
+
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
 def test_pin(pin):
     pin(_run)

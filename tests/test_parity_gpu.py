@@ -452,3 +452,114 @@ def test_autograd_unused_outputs_get_zero_gradient():
         want = oracle.ulysses_a2a(ones_then_zero, 1)
         for k in range(w):
             assert torch.equal(xd[k].grad.cpu(), want[k])
+
+
+# ---- CUDA graph capture of the C-ABI call -----------------------------------
+
+def test_run_captures_into_a_cuda_graph():
+    w, B, S, H, D = 4, 2, 37, 8, 64
+    xs = normal_slabs((B, S, H, D), w, "bf16", seed0=31)
+    want = oracle.ulysses_a2a(xs, 0)
+    back = oracle.ulysses_a2a(want, 1)
+    with UlyssesA2A(0, 2) as a2a:
+        xd = [t.cuda() for t in xs]
+        yd = [torch.empty(B, S * w, H // w, D, dtype=torch.bfloat16, device="cuda") for _ in range(w)]
+        zd = [torch.empty_like(t) for t in xd]
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):                 # warm-up outside capture
+            a2a.run(xd, 0, out=yd, stream=s)
+            a2a.run(yd, 1, out=zd, stream=s, chunked=True)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            a2a.run(xd, 0, out=yd)
+            a2a.run(yd, 1, out=zd, chunked=True)
+        for t in yd + zd:
+            t.view(torch.int16).fill_(-1)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        a2a.status()
+        for k in range(w):
+            assert torch.equal(bits(yd[k].cpu()), bits(want[k]))
+            assert torch.equal(bits(zd[k].cpu()), bits(back[k]))
+        del g
+
+
+# ---- row-pitched [B, S, H, D] side: packed QKV projection layouts -----------
+
+@pytest.mark.parametrize("path", [PATH_TMA, PATH_VEC], ids=["tma", "vec"])
+def test_packed_qkv_mode0_reads_in_place(path):
+    w, B, S, H, D = 4, 2, 37, 8, 64
+    packed_cpu = normal_slabs((B, S, 3, H, D), w, "bf16", seed0=700)
+    flat = [t.reshape(-1) for t in packed_cpu]
+    with UlyssesA2A(0, 2) as a2a:
+        a2a.set_path(path)
+        packed = [t.cuda() for t in packed_cpu]
+        for c in range(3):                                # q, k, v
+            want = oracle.ulysses_a2a_pitched(flat, 0, w, B, S, H, D, 3 * H * D, offset=c * H * D)
+            views = [t[:, :, c] for t in packed]          # strides (S*3HD, 3HD, D, 1)
+            assert views[0].stride() == (S * 3 * H * D, 3 * H * D, D, 1)
+            for chunked in (False, True):
+                for knobs in ({}, dict(rows_per_tile=5, chunk_units=0)):
+                    a2a.set_tuning(**knobs)
+                    assert a2a.plan(views, 0, knobs=knobs)["row_pitch"] == 3 * H * D
+                    out = a2a.run(views, 0, chunked=chunked)
+                    for r in range(w):
+                        assert torch.equal(bits(out[r].cpu()).reshape(-1), bits(want[r])), (c, r)
+        a2a.status()
+
+
+@pytest.mark.parametrize("path", [PATH_TMA, PATH_VEC], ids=["tma", "vec"])
+def test_mode1_writes_into_packed_slots(path):
+    w, B, S, H, D = 4, 2, 29, 8, 64
+    with UlyssesA2A(0, 2) as a2a:
+        a2a.set_path(path)
+        ys = [normal_slabs((B, S * w, H // w, D), w, "bf16", seed0=710 + c) for c in range(3)]
+        packed = [torch.empty((B, S, 3, H, D), dtype=torch.bfloat16, device="cuda")
+                  for _ in range(w)]
+        for t in packed:
+            t.view(torch.int16).fill_(-1)
+        # write only slot 1 (k) first: slots 0 and 2 keep their poison
+        a2a.run([y.cuda() for y in ys[1]], 1, out=[t[:, :, 1] for t in packed])
+        torch.cuda.synchronize()
+        want1 = oracle.ulysses_a2a(ys[1], 1)
+        for j in range(w):
+            got = packed[j].cpu()
+            assert torch.equal(bits(got[:, :, 1].contiguous()), bits(want1[j]))
+            assert bool((got[:, :, 0].view(torch.int16) == -1).all())
+            assert bool((got[:, :, 2].view(torch.int16) == -1).all())
+        for c in (0, 2):
+            a2a.run([y.cuda() for y in ys[c]], 1, out=[t[:, :, c] for t in packed], chunked=True)
+        a2a.status()
+        for c in range(3):
+            want = oracle.ulysses_a2a(ys[c], 1)
+            for j in range(w):
+                assert torch.equal(bits(packed[j][:, :, c].cpu().contiguous()), bits(want[j]))
+
+
+def test_odd_row_pitch_uses_narrower_vectors():
+    # rows of H*D + 4 bf16 elements: 8-byte aligned only, so the VEC path with
+    # 8-byte vectors; the 4 trailing elements of every row stay untouched
+    w, B, S, H, D = 2, 2, 19, 4, 32
+    pitch = H * D + 4
+    bufs_cpu = normal_slabs((B * S * pitch,), w, "bf16", seed0=720)
+    want = oracle.ulysses_a2a_pitched(bufs_cpu, 0, w, B, S, H, D, pitch)
+    with UlyssesA2A(0, 2) as a2a:
+        bufs = [t.cuda() for t in bufs_cpu]
+        views = [t.as_strided((B, S, H, D), (S * pitch, pitch, D, 1)) for t in bufs]
+        p = a2a.plan(views, 0)
+        assert p["path"] == PATH_VEC and p["vec_bytes"] == 8 and p["row_pitch"] == pitch
+        out = a2a.run(views, 0)
+        for r in range(w):
+            assert torch.equal(bits(out[r].cpu()).reshape(-1), bits(want[r]))
+        # and back: mode 1 into the pitched buffers leaves the gaps alone
+        dst = [torch.full_like(t, float("nan")) for t in bufs]
+        a2a.run(out, 1, out=[t.as_strided((B, S, H, D), (S * pitch, pitch, D, 1)) for t in dst])
+        a2a.status()
+        for j in range(w):
+            got = dst[j].cpu().view(B * S, pitch)
+            src = bufs_cpu[j].view(B * S, pitch)
+            assert torch.equal(bits(got[:, :H * D].contiguous()), bits(src[:, :H * D].contiguous()))
+            assert bool(torch.isnan(got[:, H * D:].float()).all())
