@@ -62,6 +62,7 @@ extern "C" {
 #define ULYSSES_A2A_PATH_VEC  2  /* 16/8/4/2/1-byte LDG/STG copy               */
 
 #define ULYSSES_A2A_MAX_W     64 /* largest rank count any path accepts        */
+#define ULYSSES_A2A_CHUNKED_WINDOW 2 /* chunked = 2: per plane via a window   */
 #define ULYSSES_A2A_MAX_W_TMA 8  /* largest rank count of the TMA path         */
 
 typedef struct ulysses_a2a_ctx ulysses_a2a_ctx; /* opaque */
@@ -131,8 +132,13 @@ int ulysses_a2a_destroy(ulysses_a2a_ctx *ctx);
  *   mode      : 0 (scatter heads, gather sequence) or 1 (the inverse).
  *   chunked   : 0 = one launch over all B planes; 1 = the per-plane variant:
  *               one launch per plane b on the one-plane views, in stream
- *               order, so plane b is complete before plane b+1 starts. Same
- *               bytes either way.
+ *               order, so plane b is complete before plane b+1 starts;
+ *               2 = the per-plane variant through a staging window: plane b
+ *               of every input slab is first copied into a context-owned
+ *               device window (grown on demand, reused plane after plane),
+ *               then re-laid out from the window into plane b of the outputs
+ *               (twice the memory traffic of 0 and 1). Same bytes in the
+ *               outputs whichever is chosen.
  *   stream    : a cudaStream_t (NULL = legacy default stream).
  * Asynchronous on `stream`; no host synchronisation and no allocation. */
 int ulysses_a2a_run(ulysses_a2a_ctx *ctx, const void *const *in_slabs,
@@ -161,6 +167,16 @@ const char *ulysses_a2a_last_error(const ulysses_a2a_ctx *ctx);
  * Returns ULYSSES_A2A_ERR_TIMEOUT if any kernel launched by this context gave
  * up a bounded wait since the last check, else ULYSSES_A2A_OK. */
 int ulysses_a2a_status(ulysses_a2a_ctx *ctx, void *stream);
+
+/* Failure-path self-test: launches on `stream` a one-thread kernel that waits
+ * on an mbarrier nothing ever arrives on, through the same bounded wait the
+ * copy kernel uses, but limited to limit_us microseconds (1..2 000 000); on
+ * expiry it records the timeout in the context's status words exactly as the
+ * copy kernel would. The next ulysses_a2a_status then returns
+ * ULYSSES_A2A_ERR_TIMEOUT, and the context stays usable. Nothing but the
+ * status words is touched. */
+int ulysses_a2a_selftest_wait_timeout(ulysses_a2a_ctx *ctx, uint32_t limit_us,
+                                      void *stream);
 
 /* Force a copy path (ULYSSES_A2A_PATH_*) for later runs; AUTO restores the
  * default choice. A forced path that cannot express a shape makes run fail

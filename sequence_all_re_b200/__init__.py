@@ -8,7 +8,8 @@ device_communicators/ulysses_a2a, ``run_armed``):
   becomes ``[B, S_local*w, H//w, D]`` with
   ``out_r[b, j*S_local+s, h', d] = x_j[b, s, r*(H//w)+h', d]``;
 * mode 1 is the exact inverse;
-* ``chunked=True`` runs one launch per batch plane, in stream order.
+* ``chunked=True`` runs one launch per batch plane, in stream order;
+  ``chunked=2`` stages each plane through a context-owned window first.
 
 The work happens in ``libulysses_a2a.so`` (hand-written CUDA for sm_100a,
 C ABI in ``include/ulysses_a2a.h``). This package only marshals tensors into
@@ -148,7 +149,7 @@ class UlyssesA2A:
         handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
         rc = _lib.ulysses_a2a_run_ex(self._ctx, [t.data_ptr() for t in xs],
                                      [o.data_ptr() for o in out], B, S, H, D, w, mode,
-                                     int(bool(chunked)), self._last_pitch, handle)
+                                     int(chunked), self._last_pitch, handle)
         self._check(rc)
         return out
 
@@ -160,7 +161,7 @@ class UlyssesA2A:
         handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
         rc = _lib.ulysses_a2a_run_host(self._ctx, [t.data_ptr() for t in xs],
                                        [o.data_ptr() for o in out], B, S, H, D, w, mode,
-                                       int(bool(chunked)), handle)
+                                       int(chunked), handle)
         self._check(rc)
         return out
 
@@ -177,7 +178,7 @@ class UlyssesA2A:
         w, (B, S, H, D), out = self._prepare(xs, mode, out, xs[0].device.type, allow_pitch=True)
         rc, p, msg = _lib.ulysses_a2a_plan_ex([t.data_ptr() for t in xs],
                                               [o.data_ptr() for o in out], B, S, H, D, w, mode,
-                                              int(bool(chunked)), self.elem_bytes,
+                                              int(chunked), self.elem_bytes,
                                               row_pitch=self._last_pitch, **(knobs or {}))
         if rc != _lib.OK:
             raise A2AError(rc, msg)

@@ -43,6 +43,7 @@ EXPORTED = (
     "ulysses_a2a_run_noalloc",
     "ulysses_a2a_run_ex",
     "ulysses_a2a_plan_ex",
+    "ulysses_a2a_selftest_wait_timeout",
 )
 
 
@@ -139,7 +140,7 @@ class A2AError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is not built; run `python -m sequence_all_re_b200.build` "
+            f"{LIB_PATH} is not built; run `python sequence_all_re_b200/build.py` "
             "(the CUDA library is required: there is no fallback path)")
     lib = ctypes.CDLL(LIB_PATH)
     P = ctypes.c_void_p
@@ -178,6 +179,8 @@ def _load() -> ctypes.CDLL:
                                         c_int, ctypes.POINTER(PlanT), ctypes.c_char_p,
                                         ctypes.c_size_t]
     lib.ulysses_a2a_plan_ex.restype = c_int
+    lib.ulysses_a2a_selftest_wait_timeout.argtypes = [P, ctypes.c_uint32, P]
+    lib.ulysses_a2a_selftest_wait_timeout.restype = c_int
     return lib
 
 

@@ -1,6 +1,6 @@
 """Build libulysses_a2a.so in-tree with nvcc for sm_100a.
 
-Usage: ``python -m sequence_all_re_b200.build [--force] [--ptxas-info]``.
+Usage: ``python sequence_all_re_b200/build.py [--force] [--ptxas-info]``.
 The library is linked against the static CUDA runtime and reaches the driver
 API through ``cudaGetDriverEntryPointByVersion``, so it loads (and exports its
 symbols) on a machine without a GPU driver; only its compute calls need one.

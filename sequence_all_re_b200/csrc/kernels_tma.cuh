@@ -96,13 +96,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete, for at most
-// kWaitLimitNs (checked every 256 polls) and at most 2^30 polls.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+// limit_ns of %globaltimer (checked every 256 polls) and at most 2^30 polls.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t it = 1; it < (1u << 30); ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
+    if ((it & 255u) == 0 && global_ns() - t0 > limit_ns) return false;
   }
   return false;
 }
@@ -374,6 +375,24 @@ __global__ void __launch_bounds__(32 * kTmaMaxProducers, 1)
     }
   }
   bulk_wait_all();
+}
+
+// Self-test of the failure path: one thread initialises an mbarrier that
+// nothing ever arrives on, waits for it through mbar_wait_bounded with a short
+// limit, and records the expiry in the status words exactly as the copy
+// kernel does. No memory other than the status words is touched.
+__global__ void __launch_bounds__(32, 1)
+    ua2a_wait_selftest_kernel(unsigned int* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_addr(&bar);
+  mbar_init(b, 1);
+  fence_barrier_init();
+  if (!mbar_wait_bounded(b, 0, limit_ns)) {
+    atomicOr(status, kStatusWaitTimeout);
+    atomicExch(status + 1, (unsigned)blockIdx.x + 1u);
+    atomicExch(status + 2, 0u);
+  }
 }
 
 }  // namespace ua2a

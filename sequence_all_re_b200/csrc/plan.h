@@ -147,7 +147,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     return ULYSSES_A2A_ERR_INVALID;
   }
   if (mode != 0 && mode != 1) { set_err(err, "mode=%lld not 0 or 1", mode); return ULYSSES_A2A_ERR_INVALID; }
-  if (chunked != 0 && chunked != 1) { set_err(err, "chunked=%lld not 0 or 1", chunked); return ULYSSES_A2A_ERR_INVALID; }
+  if (chunked < 0 || chunked > 2) { set_err(err, "chunked=%lld not 0, 1 or 2", chunked); return ULYSSES_A2A_ERR_INVALID; }
   if (B < 1 || S < 1 || H < 1 || D < 1) {
     set_err(err, "sizes must be >= 1 (B, S_local, H, D)");
     return ULYSSES_A2A_ERR_INVALID;

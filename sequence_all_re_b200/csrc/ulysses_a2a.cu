@@ -80,6 +80,9 @@ struct ulysses_a2a_ctx {
   void* d_stage = nullptr;
   size_t stage_bytes = 0;
   cudaStream_t copy_stream[2] = {nullptr, nullptr};  // H2D, D2H
+  // chunked = 2: the staging window (one plane of every input slab)
+  void* d_window = nullptr;
+  size_t window_bytes = 0;
   cudaEvent_t copy_events[1 + 2 * 8] = {};            // start + 2 per chunk
   PFN_cuTensorMapEncodeTiled_v12000 encode_tiled = nullptr;
   PFN_cuMemGetAddressRange_v3020 get_range = nullptr;
@@ -318,8 +321,7 @@ int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, in
     }
     return ULYSSES_A2A_OK;
   }
-  VecParams p;
-  std::memset(&p, 0, sizeof(p));
+  VecParams p{};
   for (int k = 0; k < w; ++k) {
     p.in[k] = static_cast<const char*>(in[k]);
     p.out[k] = static_cast<char*>(out[k]);
@@ -420,6 +422,7 @@ int ulysses_a2a_destroy(ulysses_a2a_ctx* ctx) {
     if (cudaDeviceSynchronize() != cudaSuccess) rc = ULYSSES_A2A_ERR_CUDA;
     if (ctx->d_status && cudaFree(ctx->d_status) != cudaSuccess) rc = ULYSSES_A2A_ERR_CUDA;
     if (ctx->d_stage && cudaFree(ctx->d_stage) != cudaSuccess) rc = ULYSSES_A2A_ERR_CUDA;
+    if (ctx->d_window && cudaFree(ctx->d_window) != cudaSuccess) rc = ULYSSES_A2A_ERR_CUDA;
     for (auto& cs : ctx->copy_stream)
       if (cs && cudaStreamDestroy(cs) != cudaSuccess) rc = ULYSSES_A2A_ERR_CUDA;
     for (auto& ev : ctx->copy_events)
@@ -429,6 +432,72 @@ int ulysses_a2a_destroy(ulysses_a2a_ctx* ctx) {
   delete ctx;  // the handle is consumed whatever the cleanup calls reported
   return rc;
 }
+
+namespace {
+
+// chunked = 2: per plane, publish every rank's input plane into the window
+// (the page's registered window, reused plane after plane: each copy finishes
+// in stream order before the next plane overwrites it), then re-lay it out
+// from the window into that plane of the outputs.
+int run_windowed(ulysses_a2a_ctx* ctx, const ulysses_a2a_desc_t* d, const ulysses_a2a_plan_t& pl,
+                 cudaStream_t st) {
+  const int w = d->w;
+  const int64_t E = ctx->elem_bytes;
+  const int64_t HD = d->H * d->D;
+  const size_t plane = (size_t)(d->S_local * HD * E);        // one dense plane of one slab
+  const size_t slot = (plane + 255) / 256 * 256;
+  const size_t need = slot * (size_t)w;
+  if (ctx->window_bytes < need) {                              // grow on demand
+    cudaError_t e;
+    if (ctx->d_window) {
+      e = cudaStreamSynchronize(st);
+      if (e != cudaSuccess) return cuda_fail(ctx, "cudaStreamSynchronize (window grow)", e);
+      cudaFree(ctx->d_window);
+      ctx->d_window = nullptr;
+      ctx->window_bytes = 0;
+      for (auto& c : ctx->tma_cache) c.valid = false;       // maps may point into it
+    }
+    e = cudaMalloc(&ctx->d_window, need);
+    if (e != cudaSuccess) {
+      ctx->d_window = nullptr;
+      return cuda_fail(ctx, "cudaMalloc (staging window)", e);
+    }
+    ctx->window_bytes = need;
+  }
+  std::vector<const void*> win(w);
+  std::vector<void*> outb(w);
+  char* wbase = static_cast<char*>(ctx->d_window);
+  for (int k = 0; k < w; ++k) win[k] = wbase + slot * k;
+  const int64_t pitch = pl.row_pitch;
+  for (int64_t b = 0; b < d->B; ++b) {
+    for (int k = 0; k < w; ++k) {
+      cudaError_t e;
+      if (d->mode == 0) {   // pitched [B, S, H, D] input plane -> dense window slot
+        const char* src = static_cast<const char*>(d->in_slabs[k]) + (size_t)(b * d->S_local * pitch * E);
+        if (pitch == HD)
+          e = cudaMemcpyAsync(const_cast<void*>(win[k]), src, plane, cudaMemcpyDeviceToDevice, st);
+        else
+          e = cudaMemcpy2DAsync(const_cast<void*>(win[k]), (size_t)(HD * E), src, (size_t)(pitch * E),
+                                (size_t)(HD * E), (size_t)d->S_local, cudaMemcpyDeviceToDevice, st);
+        outb[k] = static_cast<char*>(d->out_slabs[k]) + plane * b;
+      } else {              // dense [B, S*w, H/w, D] input plane -> window slot
+        const char* src = static_cast<const char*>(d->in_slabs[k]) + plane * b;
+        e = cudaMemcpyAsync(const_cast<void*>(win[k]), src, plane, cudaMemcpyDeviceToDevice, st);
+        outb[k] = static_cast<char*>(d->out_slabs[k]) + (size_t)(b * d->S_local * pitch * E);
+      }
+      if (e != cudaSuccess) return cuda_fail(ctx, "cudaMemcpyAsync (publish into the window)", e);
+    }
+    ulysses_a2a_plan_t pb;
+    int rc = plan_for(ctx, win.data(), outb.data(), 1, d->S_local, d->H, d->D, w, d->mode, 0, &pb,
+                      d->mode == 1 ? pitch : 0);
+    if (rc) return rc;
+    rc = run_device(ctx, win.data(), outb.data(), 1, d->S_local, d->H, d->D, w, d->mode, 0, st, pb);
+    if (rc) return rc;
+  }
+  return ULYSSES_A2A_OK;
+}
+
+}  // namespace
 
 int ulysses_a2a_run_ex(ulysses_a2a_ctx* ctx, const ulysses_a2a_desc_t* d, void* stream) {
   if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
@@ -450,6 +519,8 @@ int ulysses_a2a_run_ex(ulysses_a2a_ctx* ctx, const ulysses_a2a_desc_t* d, void* 
   rc = check_residency(ctx, reinterpret_cast<const void* const*>(d->out_slabs), d->w,
                        d->mode == 0 ? dense_bytes : strided_bytes, "output");
   if (rc) return rc;
+  if (d->chunked == ULYSSES_A2A_CHUNKED_WINDOW)
+    return run_windowed(ctx, d, pl, static_cast<cudaStream_t>(stream));
   return run_device(ctx, d->in_slabs, d->out_slabs, d->B, d->S_local, d->H, d->D, d->w, d->mode,
                     d->chunked, static_cast<cudaStream_t>(stream), pl);
 }
@@ -477,6 +548,9 @@ int ulysses_a2a_run_host(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void
   if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
   ctx->last_error.clear();
   // validate the host pointers (overlap, sizes) before touching the device
+  if (chunked == ULYSSES_A2A_CHUNKED_WINDOW)
+    return fail(ctx, ULYSSES_A2A_ERR_UNSUPPORTED,
+                "the host-buffer path stages through its own buffers: chunked must be 0 or 1");
   ulysses_a2a_plan_t host_pl;
   int rc = plan_for(ctx, in_slabs, out_slabs, B, S_local, H, D, w, mode, chunked, &host_pl);
   if (rc) return rc;
@@ -625,6 +699,20 @@ int ulysses_a2a_status(ulysses_a2a_ctx* ctx, void* stream) {
                 h[1] ? h[1] - 1 : 0u, h[2],
                 (h[0] & ua2a::kStatusDrainTimeout) ? "; draining also timed out" : "");
   return fail(ctx, ULYSSES_A2A_ERR_TIMEOUT, buf);
+}
+
+int ulysses_a2a_selftest_wait_timeout(ulysses_a2a_ctx* ctx, uint32_t limit_us, void* stream) {
+  if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
+  if (limit_us < 1 || limit_us > 2000000)
+    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "limit_us must be in [1, 2000000]");
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "cannot select the context's device");
+  ua2a::ua2a_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      ctx->d_status, (uint64_t)limit_us * 1000ull);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(ctx, "self-test kernel launch", e);
+  ctx->launches++;
+  return ULYSSES_A2A_OK;
 }
 
 int ulysses_a2a_set_path(ulysses_a2a_ctx* ctx, int path) {
@@ -800,6 +888,9 @@ extern "C" int ulysses_a2a_run_noalloc(const void* const* in_slabs, void* const*
   });
   if (g_noalloc_encode == nullptr)
     return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  if (chunked == ULYSSES_A2A_CHUNKED_WINDOW)
+    return noalloc_report(err, errlen, ULYSSES_A2A_ERR_UNSUPPORTED,
+                          "chunked = 2 needs a staging window; use chunked 0 or 1 here");
 
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) {
@@ -916,8 +1007,7 @@ extern "C" int ulysses_a2a_run_noalloc(const void* const* in_slabs, void* const*
         return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "TMA kernel launch failed (plane %lld)", l);
     }
   } else {
-    VecParams p;
-    std::memset(&p, 0, sizeof(p));
+    VecParams p{};
     for (int k = 0; k < w; ++k) {
       p.in[k] = static_cast<const char*>(in_slabs[k]);
       p.out[k] = static_cast<char*>(out_slabs[k]);

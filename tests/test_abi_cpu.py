@@ -107,6 +107,13 @@ def test_plan_cfg4_chunked_launches():
     assert p.payload_bytes == q.payload_bytes == 1 << 30
 
 
+def test_plan_windowed_chunked_variant():
+    rc, p, _ = plan(4, 4, 16384, 32, 64, chunked=2)
+    assert rc == OK and p.launches == 4
+    rc, q, _ = plan(4, 4, 16384, 32, 64, chunked=1)
+    assert p.units == q.units
+
+
 def test_plan_cfg1_small():
     rc, p, _ = plan(2, 1, 64, 4, 64)
     assert rc == OK and p.path == PATH_TMA
@@ -226,6 +233,7 @@ def test_large_rows_reduce_stages_then_producers():
     (dict(w=65, B=1, S=4, H=65, D=8), ERR_INVALID),
     (dict(w=2, B=1, S=4, H=4, D=8, mode=2), ERR_INVALID),
     (dict(w=2, B=1, S=4, H=4, D=8, chunked=3), ERR_INVALID),
+    (dict(w=2, B=1, S=4, H=4, D=8, chunked=-1), ERR_INVALID),
     (dict(w=2, B=1, S=4, H=4, D=8, E=3), ERR_INVALID),
 ])
 def test_rejects_bad_arguments(args, code):

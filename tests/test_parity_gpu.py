@@ -563,3 +563,62 @@ def test_odd_row_pitch_uses_narrower_vectors():
             src = bufs_cpu[j].view(B * S, pitch)
             assert torch.equal(bits(got[:, :H * D].contiguous()), bits(src[:, :H * D].contiguous()))
             assert bool(torch.isnan(got[:, H * D:].float()).all())
+
+
+# ---- failure detection: a bounded wait that expires ---------------------------
+
+def test_bounded_wait_expiry_is_reported_and_context_survives():
+    # the self-test kernel waits on an mbarrier nothing arrives on (50 ms limit)
+    from sequence_all_re_b200 import _lib as L
+
+    with UlyssesA2A(0, 2) as a2a:
+        a2a.status()                                       # clean to start with
+        stream = torch.cuda.current_stream()
+        rc = L.lib.ulysses_a2a_selftest_wait_timeout(a2a._ctx, 50000, stream.cuda_stream)
+        assert rc == L.OK
+        with pytest.raises(A2AError) as e:
+            a2a.status()
+        assert e.value.code == L.ERR_TIMEOUT and "gave up" in a2a.last_error()
+        a2a.status()                                       # reading it cleared it
+        # the context and the device still work
+        run_case(normal_slabs((1, 16, 4, 64), 2, "bf16", seed0=3), 0, a2a=a2a)
+        rc = L.lib.ulysses_a2a_selftest_wait_timeout(a2a._ctx, 0, stream.cuda_stream)
+        assert rc == L.ERR_INVALID
+
+
+# ---- chunked = 2: per plane through the context's staging window -------------
+
+@pytest.mark.parametrize("path", [PATH_TMA, PATH_VEC], ids=["tma", "vec"])
+def test_windowed_chunked_variant(path):
+    with UlyssesA2A(0, 2) as a2a:
+        a2a.set_path(path)
+        # small first, then larger planes: the window grows on demand
+        for (w, B, S, H, D) in [(2, 2, 9, 4, 64), (4, 3, 37, 8, 64), (8, 2, 53, 40, 128)]:
+            for mode in (0, 1):
+                xs = normal_slabs(slab_shape(mode, w, B, S, H, D), w, "bf16", seed0=800 + mode)
+                run_case(xs, mode, chunked=2, path=path, a2a=a2a)
+        # packed QKV input read through the window
+        w, B, S, H, D = 4, 2, 21, 8, 64
+        packed_cpu = normal_slabs((B, S, 3, H, D), w, "bf16", seed0=810)
+        want = oracle.ulysses_a2a_pitched([t.reshape(-1) for t in packed_cpu], 0, w, B, S, H, D,
+                                          3 * H * D, offset=H * D)
+        packed = [t.cuda() for t in packed_cpu]
+        out = a2a.run([t[:, :, 1] for t in packed], 0, chunked=2)
+        for r in range(w):
+            assert torch.equal(bits(out[r].cpu()).reshape(-1), bits(want[r]))
+        a2a.status()
+
+
+def test_windowed_variant_is_refused_where_no_window_exists():
+    w, B, S, H, D = 2, 2, 8, 4, 64
+    xs = normal_slabs((B, S, H, D), w, "bf16")
+    with UlyssesA2A(0, 2) as a2a:
+        with pytest.raises(A2AError) as e:
+            a2a.run_host(xs, 0, chunked=2)
+        assert e.value.code == _lib.ERR_UNSUPPORTED
+    xd = [t.cuda() for t in xs]
+    yd = [torch.empty(B, S * w, H // w, D, dtype=torch.bfloat16, device="cuda") for _ in range(w)]
+    rc, msg = _lib.ulysses_a2a_run_noalloc([t.data_ptr() for t in xd], [t.data_ptr() for t in yd],
+                                           B, S, H, D, w, 0, 2, 2,
+                                           torch.cuda.current_stream().cuda_stream)
+    assert rc == _lib.ERR_UNSUPPORTED and "window" in msg
