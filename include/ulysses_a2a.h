@@ -198,7 +198,9 @@ typedef struct ulysses_a2a_tuning_t {
     int32_t chunk_units;    /* TMA schedule: 0 = persistent grid (static
                                round robin); n > 0 = n consecutive units per
                                CTA; -1 = default (one unit per producer)   */
-    int32_t reserved;       /* must be 0                                    */
+    int32_t host_chunks;    /* host-buffer entry point: sequence chunks its
+                               copies and kernels are pipelined over, 1..64;
+                               0 = default                                */
 } ulysses_a2a_tuning_t;
 
 /* Apply tuning to later runs (NULL restores every default). Values outside

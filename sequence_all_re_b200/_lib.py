@@ -86,11 +86,11 @@ class TuningT(ctypes.Structure):
         ("producers", ctypes.c_int32),
         ("order", ctypes.c_int32),
         ("chunk_units", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("host_chunks", ctypes.c_int32),
     ]
 
     DEFAULTS = dict(rows_per_tile=0, ctas_per_sm=0, stages=0, lookahead=0, producers=0,
-                    order=-1, chunk_units=-1, reserved=0)
+                    order=-1, chunk_units=-1, host_chunks=0)
 
     @classmethod
     def make(cls, **kw):

@@ -44,6 +44,11 @@ constexpr int kVecBlock = 256;
 constexpr int kVecDefaultCtasPerSm = 16;
 // Unit numbering: 0 = destination rank outermost, 1 = innermost.
 constexpr int kDefaultOrder = 1;
+// Host-buffer entry point: sequence chunks its H2D copies, kernels and D2H
+// copies are pipelined over (payloads below kHostChunkMinBytes use one).
+constexpr int kHostMaxChunks = 64;
+constexpr int kHostDefaultChunks = 8;
+constexpr int64_t kHostChunkMinBytes = 8 << 20;
 // TMA schedule: by default a grid of ceil(units / n) short-lived CTAs, each
 // taking n consecutive units, one per producer warp, with a one-tile ring per
 // producer and at most kTmaChunkSmemTarget of shared memory per CTA, so that
@@ -60,6 +65,7 @@ struct Tuning {
   int producers = 0;      // TMA producer warps per CTA (0 = default)
   int order = -1;         // unit numbering (-1 = default)
   int chunk_units = -1;   // TMA: units per CTA (0 = persistent grid, -1 = default)
+  int host_chunks = 0;    // host-buffer path pipeline depth (0 = default)
 };
 
 inline bool mul_overflows(int64_t a, int64_t b, int64_t* out) {
@@ -114,7 +120,7 @@ inline bool tuning_from(const ulysses_a2a_tuning_t* t, Tuning* out, std::string*
   if (t->producers < 0 || t->producers > kTmaMaxProducers) return bad("producers");
   if (t->order < -1 || t->order > 1) return bad("order");
   if (t->chunk_units < -1) return bad("chunk_units");
-  if (t->reserved != 0) return bad("reserved");
+  if (t->host_chunks < 0 || t->host_chunks > kHostMaxChunks) return bad("host_chunks");
   out->rows_per_tile = t->rows_per_tile;
   out->ctas_per_sm = t->ctas_per_sm;
   out->stages = t->stages;
@@ -122,6 +128,7 @@ inline bool tuning_from(const ulysses_a2a_tuning_t* t, Tuning* out, std::string*
   out->producers = t->producers;
   out->order = t->order;
   out->chunk_units = t->chunk_units;
+  out->host_chunks = t->host_chunks;
   return true;
 }
 

@@ -46,10 +46,7 @@ using ua2a::VecParams;
 namespace {
 
 constexpr int kTmaCacheEntries = 16;
-// host-buffer entry point: sequence chunks in flight, and the payload below
-// which one chunk is used
-constexpr int64_t kHostChunks = 8;
-constexpr int64_t kHostChunkMinBytes = 8 << 20;
+
 
 struct TmaCacheEntry {
   bool valid = false;
@@ -83,7 +80,7 @@ struct ulysses_a2a_ctx {
   // chunked = 2: the staging window (one plane of every input slab)
   void* d_window = nullptr;
   size_t window_bytes = 0;
-  cudaEvent_t copy_events[1 + 2 * 8] = {};            // start + 2 per chunk
+  std::vector<cudaEvent_t> copy_events;              // start + 2 per chunk
   PFN_cuTensorMapEncodeTiled_v12000 encode_tiled = nullptr;
   PFN_cuMemGetAddressRange_v3020 get_range = nullptr;
 };
@@ -585,14 +582,11 @@ int ulysses_a2a_run_host(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void
       }
     }
   }
-  for (auto& ev : ctx->copy_events) {
-    if (ev == nullptr) {
-      cudaError_t e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
-      if (e != cudaSuccess) {
-        ev = nullptr;
-        return cuda_fail(ctx, "cudaEventCreate (host-path copies)", e);
-      }
-    }
+  while (ctx->copy_events.size() < (size_t)(1 + 2 * ua2a::kHostMaxChunks)) {
+    cudaEvent_t ev = nullptr;
+    cudaError_t e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(ctx, "cudaEventCreate (host-path copies)", e);
+    ctx->copy_events.push_back(ev);
   }
   std::vector<const void*> din(w);
   std::vector<void*> dout(w);
@@ -612,12 +606,15 @@ int ulysses_a2a_run_host(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void
   // bytes on each side are strided blocks moved by one 2-D copy per slab/plane.
   const int64_t T = pl.tiles_per_block, rows = pl.rows_per_tile, E = ctx->elem_bytes;
   const int64_t L = (H / w) * D;             // elements per run
-  int64_t nchunks = pl.payload_bytes < kHostChunkMinBytes ? 1 : kHostChunks;
+  // Chunk boundaries (in tiles): equal chunks. (Shorter first and last chunks,
+  // to shrink the pipeline's fill and drain, measured no better.)
+  int64_t nchunks = ctx->tuning.host_chunks > 0 ? ctx->tuning.host_chunks : ua2a::kHostDefaultChunks;
+  if (pl.payload_bytes < ua2a::kHostChunkMinBytes) nchunks = 1;
   if (nchunks > T) nchunks = T;
-  const int64_t tpc = (T + nchunks - 1) / nchunks;
-  nchunks = (T + tpc - 1) / tpc;
+  std::vector<int64_t> bounds;  // chunk c covers tiles [bounds[c], bounds[c+1])
+  for (int64_t c = 0; c <= nchunks; ++c) bounds.push_back(T * c / nchunks);
   cudaStream_t sh = ctx->copy_stream[0], sd = ctx->copy_stream[1];
-  cudaEvent_t* ev = ctx->copy_events;  // [0]: start; [1 + 2c]: H2D done; [2 + 2c]: kernel done
+  cudaEvent_t* ev = ctx->copy_events.data();  // [0]: start; [1 + 2c]: H2D; [2 + 2c]: kernel
   cudaError_t e = cudaEventRecord(ev[0], st);  // copies start after earlier work on `stream`
   if (e == cudaSuccess) e = cudaStreamWaitEvent(sh, ev[0], 0);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(sd, ev[0], 0);
@@ -655,8 +652,9 @@ int ulysses_a2a_run_host(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void
     return cudaSuccess;
   };
   for (int64_t c = 0; c < nchunks; ++c) {
-    const int64_t t0 = c * tpc;
-    const int64_t nt = (t0 + tpc <= T) ? tpc : T - t0;
+    const int64_t t0 = bounds[c];
+    const int64_t nt = bounds[c + 1] - t0;
+    if (nt <= 0) continue;
     const int64_t s0 = t0 * rows;
     const int64_t s1 = (t0 + nt) * rows < S_local ? (t0 + nt) * rows : S_local;
     e = copy_rows(true, s0, s1 - s0, sh);

@@ -178,7 +178,7 @@ def test_tuning_knobs():
 @pytest.mark.parametrize("knob,value", [("rows_per_tile", 257), ("rows_per_tile", -1),
                                         ("ctas_per_sm", 33), ("stages", 33), ("producers", 9),
                                         ("order", 2), ("chunk_units", -2), ("lookahead", -1),
-                                        ("reserved", 1)])
+                                        ("host_chunks", 65), ("host_chunks", -1)])
 def test_tuning_out_of_range_is_rejected(knob, value):
     rc, _, msg = plan(4, 1, 64, 8, 64, **{knob: value})
     assert rc == ERR_INVALID and knob in msg
