@@ -622,3 +622,68 @@ def test_windowed_variant_is_refused_where_no_window_exists():
                                            B, S, H, D, w, 0, 2, 2,
                                            torch.cuda.current_stream().cuda_stream)
     assert rc == _lib.ERR_UNSUPPORTED and "window" in msg
+
+
+# ---- randomized coverage ------------------------------------------------------
+
+def test_randomized_shapes_layouts_and_knobs():
+    """150 seeded random cases: w in 1..16, ragged S_local, odd D, element sizes
+    1/2/4/8, both modes, chunked 0/1/2, random row pitches on the [B,S,H,D] side
+    (gap bytes must survive), random tuning and both paths; bit-exact against
+    the oracle every time."""
+    import random
+
+    rng = random.Random(20241202)
+    INT = {1: torch.uint8, 2: torch.int16, 4: torch.int32, 8: torch.int64}
+    ctxs = {E: UlyssesA2A(0, E) for E in (1, 2, 4, 8)}
+    try:
+        for case in range(150):
+            w = rng.choice([1, 2, 3, 4, 5, 8, 12, 16])
+            B, S = rng.randint(1, 3), rng.randint(1, 70)
+            H = w * rng.randint(1, 4)
+            D = rng.choice([1, 3, 8, 16, 24, 64, 128, 200, 256])
+            E = rng.choice([1, 2, 4, 8])
+            mode, chunked = rng.randint(0, 1), rng.choice([0, 0, 1, 2])
+            pitch = H * D + rng.choice([0, 0, 0, rng.randint(1, 40), 8 * rng.randint(1, 6)])
+            knobs = {}
+            if rng.random() < 0.6:
+                knobs = dict(rows_per_tile=rng.randint(0, 9), stages=rng.choice([0, 2, 3, 4, 8, 12]),
+                             chunk_units=rng.choice([-1, 0, 1, 3, 7]), order=rng.choice([-1, 0, 1]),
+                             producers=rng.choice([0, 1, 2, 3, 4, 8]))
+            path = rng.choice([PATH_AUTO, PATH_AUTO, PATH_VEC])
+            a2a = ctxs[E]
+            a2a.set_path(path)
+            a2a.set_tuning(**knobs)
+            dt = INT[E]
+            n_pitched = (B * S - 1) * pitch + H * D
+            n_dense = B * S * H * D
+            seed = 9000 + case
+            if mode == 0:
+                bufs = [t.view(dt) for t in random_byte_slabs((n_pitched * E,), w, seed0=seed)]
+                want = oracle.ulysses_a2a_pitched(bufs, 0, w, B, S, H, D, pitch)
+                dev = [t.cuda() for t in bufs]
+                xs = [t.as_strided((B, S, H, D), (S * pitch, pitch, D, 1)) for t in dev]
+                out = [torch.empty(B, S * w, H // w, D, dtype=dt, device="cuda") for _ in range(w)]
+                for o in out:
+                    o.view(torch.uint8).fill_(0xFF)
+                a2a.run(xs, 0, chunked=chunked, out=out)
+                got = [o.cpu().reshape(-1) for o in out]
+            else:
+                ins = [t.view(dt) for t in random_byte_slabs((n_dense * E,), w, seed0=seed)]
+                poison = [torch.full((n_pitched * E,), 0xA5, dtype=torch.uint8).view(dt)
+                          for _ in range(w)]
+                want = oracle.ulysses_a2a_pitched(ins, 1, w, B, S, H, D, pitch,
+                                                  out_bufs=[p.clone() for p in poison])
+                xs = [t.cuda().view(B, S * w, H // w, D) for t in ins]
+                dst = [p.cuda() for p in poison]
+                out = [t.as_strided((B, S, H, D), (S * pitch, pitch, D, 1)) for t in dst]
+                a2a.run(xs, 1, chunked=chunked, out=out)
+                got = [t.cpu() for t in dst]
+            a2a.status()
+            for k in range(w):
+                assert torch.equal(got[k], want[k].reshape(-1)), (
+                    f"case {case}: w={w} B={B} S={S} H={H} D={D} E={E} mode={mode} "
+                    f"chunked={chunked} pitch={pitch} path={path} knobs={knobs} rank={k}")
+    finally:
+        for c in ctxs.values():
+            c.close()
