@@ -42,7 +42,24 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "payload GB/s and % of HBM roofline (2x bytes) per mode at w=2/4/8, 1xB200"
-WORKLOAD = dict(w=4, B=1, S_local=8192, H=24, D=128, dtype="bf16")
+# The benchmark configurations (bf16, N(0,1) values); cfg2 is the default workload.
+WORKLOADS = {
+    "cfg1": dict(w=2, B=1, S_local=64, H=4, D=64),
+    "cfg2": dict(w=4, B=1, S_local=8192, H=24, D=128),
+    "cfg3": dict(w=8, B=2, S_local=4725, H=40, D=128),
+    "cfg4": dict(w=4, B=4, S_local=16384, H=32, D=64),
+}
+WORKLOAD = WORKLOADS["cfg2"]
+
+
+def workload_key(w, B, S, H, D, path):
+    return f"{path}:w{w}_B{B}_S{S}_H{H}_D{D}_bf16"
+
+
+def workload_name(w, B, S, H, D, chunked):
+    how = {0: "", 1: ", chunked per plane", 2: ", chunked through the staging window"}[chunked]
+    return (f"ulysses_a2a w={w} B={B} S_local={S} H={H} D={D} bf16, step = mode 0 + mode 1"
+            f"{how}")
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 2 * 126 * 1024 * 1024 + (4 << 20)
 
@@ -168,13 +185,13 @@ def make_inputs(w, B, S, H, D, dtype, device, seed0=1234):
     return xs
 
 
-def timed_steps(a2a, x, y, y2, z, steps, warmup, stream, sampler=None):
+def timed_steps(a2a, x, y, y2, z, steps, warmup, stream, sampler=None, chunked=0):
     """K back-to-back steps (mode 0: x -> y, mode 1: y2 -> z) between one pair of events.
 
     Returns (total ms, launches of our kernels in the timed region, clocks)."""
     for _ in range(warmup):
-        a2a.run(x, 0, out=y, stream=stream)
-        a2a.run(y2, 1, out=z, stream=stream)
+        a2a.run(x, 0, out=y, stream=stream, chunked=chunked)
+        a2a.run(y2, 1, out=z, stream=stream, chunked=chunked)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -183,33 +200,33 @@ def timed_steps(a2a, x, y, y2, z, steps, warmup, stream, sampler=None):
         sampler.start()
     e0.record(stream)
     for _ in range(steps):
-        a2a.run(x, 0, out=y, stream=stream)
-        a2a.run(y2, 1, out=z, stream=stream)
+        a2a.run(x, 0, out=y, stream=stream, chunked=chunked)
+        a2a.run(y2, 1, out=z, stream=stream, chunked=chunked)
     e1.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
     return e0.elapsed_time(e1), a2a.launch_count - launches0, clocks
 
 
-def timed_mode(a2a, src, dst, mode, reps, stream):
+def timed_mode(a2a, src, dst, mode, reps, stream, chunked=0):
     """Back-to-back calls of one mode between one pair of events; ms per call."""
     for _ in range(3):
-        a2a.run(src, mode, out=dst, stream=stream)
+        a2a.run(src, mode, out=dst, stream=stream, chunked=chunked)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(reps):
-        a2a.run(src, mode, out=dst, stream=stream)
+        a2a.run(src, mode, out=dst, stream=stream, chunked=chunked)
     e1.record(stream)
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / reps
 
 
-def timed_flushed(a2a, src, dst, mode, flush, reps, stream):
+def timed_flushed(a2a, src, dst, mode, flush, reps, stream, chunked=0):
     """Median per-call time (ms) with a 2x-L2 write flush before every call."""
     for _ in range(3):
-        a2a.run(src, mode, out=dst, stream=stream)
+        a2a.run(src, mode, out=dst, stream=stream, chunked=chunked)
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(reps)]
@@ -217,7 +234,7 @@ def timed_flushed(a2a, src, dst, mode, flush, reps, stream):
         for i in range(reps):
             flush.fill_(i & 0xFF)
             ev[i][0].record(stream)
-            a2a.run(src, mode, out=dst, stream=stream)
+            a2a.run(src, mode, out=dst, stream=stream, chunked=chunked)
             ev[i][1].record(stream)
     torch.cuda.synchronize()
     return statistics.median(a.elapsed_time(b) for a, b in ev)
@@ -338,10 +355,13 @@ def run_ours(args):
 
     from sequence_all_re_b200 import UlyssesA2A
 
-    w, B, S, H, D = (WORKLOAD[k] for k in ("w", "B", "S_local", "H", "D"))
+    wl = WORKLOADS[args.workload]
+    w, B, S, H, D = (wl[k] for k in ("w", "B", "S_local", "H", "D"))
     E = 2
     P = w * B * S * H * D * E
     a2a = UlyssesA2A(local_rank, E)
+    a2a.set_path({"auto": 0, "tma": 1, "vec": 2}[args.path])
+    chunked = args.chunked
     stream = torch.cuda.Stream(device)
     x = make_inputs(w, B, S, H, D, "bf16", device)
     y = [torch.empty((B, S * w, H // w, D), dtype=torch.bfloat16, device=device) for _ in range(w)]
@@ -351,14 +371,14 @@ def run_ours(args):
         a2a.run(x, 0, out=y, stream=stream)
     torch.cuda.synchronize()
     y2 = [t.clone() for t in y]
-    plan = a2a.plan(x, 0, out=y)
+    plan = a2a.plan(x, 0, chunked=chunked, out=y)
 
     sampler = ClockSampler(local_rank)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     total_ms, launches, clocks = timed_steps(a2a, x, y, y2, z, args.steps, args.warmup, stream,
-                                             sampler)
+                                             sampler, chunked)
     a2a.status(stream)
     torch.cuda.synchronize()
     if dist:
@@ -373,21 +393,24 @@ def run_ours(args):
 
     peak, peak_src = hbm_peak()
     avg_launch_ms = total_ms / launches
-    achieved = 2 * P / (avg_launch_ms / 1e3) / 1e9
+    bytes_per_launch = 2 * P * 2 * args.steps // launches       # 2 calls of 2P per step
+    achieved = bytes_per_launch / (avg_launch_ms / 1e3) / 1e9
     khash = kernel_source_hash()
     traffic, traffic_src = ncu_traffic(khash)
     traffic_bytes = None
     if traffic:
-        traffic_bytes = traffic.get("workloads", {}).get("w4_B1_S8192_H24_D128_bf16", {}).get(
-            "dram_bytes_per_launch")
+        key = workload_key(w, B, S, H, D, {1: "tma", 2: "vec"}[plan["path"]])
+        traffic_bytes = traffic.get("workloads", {}).get(key, {}).get("dram_bytes_per_launch")
+        if traffic_bytes is None:
+            traffic_src = "no ncu capture of this kernel and workload"
 
     # per mode: back to back, and call by call after an L2 write flush
     reps = max(20, min(args.steps, 400))
-    m0 = timed_mode(a2a, x, y, 0, reps, stream)
-    m1 = timed_mode(a2a, y2, z, 1, reps, stream)
+    m0 = timed_mode(a2a, x, y, 0, reps, stream, chunked)
+    m1 = timed_mode(a2a, y2, z, 1, reps, stream, chunked)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-    f0 = timed_flushed(a2a, x, y, 0, flush, reps, stream)
-    f1 = timed_flushed(a2a, y2, z, 1, flush, reps, stream)
+    f0 = timed_flushed(a2a, x, y, 0, flush, reps, stream, chunked)
+    f1 = timed_flushed(a2a, y2, z, 1, flush, reps, stream, chunked)
     del flush
     gbs = lambda ms: P / (ms / 1e3) / 1e9
     per_mode = {"mode0_gbs": round(gbs(m0), 1), "mode1_gbs": round(gbs(m1), 1),
@@ -463,14 +486,17 @@ def run_ours(args):
         "dtype": "bf16",
         "data": "synthetic",
         "config": {
-            "workload": "ulysses_a2a w=4 B=1 S_local=8192 H=24 D=128 bf16, step = mode 0 + mode 1",
+            "workload": workload_name(w, B, S, H, D, chunked),
+            "name": args.workload,
             "w": w, "B": B, "S_local": S, "H": H, "D": D,
             "payload_bytes_per_call": P,
             "path": {1: "tma", 2: "vec"}[plan["path"]],
             "rows_per_tile": plan["rows_per_tile"], "producers": plan["producers"],
             "stages": plan["stages"], "chunk_units": plan["chunk_units"], "grid": plan["grid"],
-            "l2": "inputs larger than L2 (192 MiB per call vs 126 MB); no kernel reads data "
-                  "the previous kernel touched; no flush in the timed region",
+            "l2": (f"inputs larger than L2 ({P / 2**20:.0f} MiB per call vs 126 MB); no kernel "
+                   "reads data the previous kernel touched; no flush in the timed region")
+                  if P > 126 * 2**20 else
+                  "L2-assisted: the inputs fit in L2 (below 126 MB); no flush",
             "parallelism": f"{world} independent instance(s), one per GPU",
         },
         "per_mode": per_mode,
@@ -482,10 +508,13 @@ def run_ours(args):
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
             "peak_source": peak_src,
-            "algorithmic_bytes_per_launch": 2 * P,
+            "algorithmic_bytes_per_launch": bytes_per_launch,
             "avg_launch_us": round(avg_launch_ms * 1e3, 3),
             "traffic": traffic_bytes,
             "traffic_source": traffic_src,
+            **({"note": "chunked = 2 also copies every plane into the staging window: the "
+                        "bytes actually moved are twice the algorithmic bytes"}
+               if chunked == 2 else {}),
         },
         "gpu_launches": launches,
         "e2e": e2e,
@@ -511,7 +540,8 @@ def run_reference(args):
     import oracle
     from synth import normal_slabs
 
-    w, B, S, H, D = (WORKLOAD[k] for k in ("w", "B", "S_local", "H", "D"))
+    wl = WORKLOADS[args.workload]
+    w, B, S, H, D = (wl[k] for k in ("w", "B", "S_local", "H", "D"))
     E = 2
     # size each step's sample so warmup + steps finish in about two minutes
     probe_S = 256
@@ -551,9 +581,8 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "ulysses_a2a w=4 B=1 S_local=8192 H=24 D=128 bf16, "
-                               "step = mode 0 + mode 1", "w": w, "B": B, "S_local": S, "H": H,
-                   "D": D},
+        "config": {"workload": workload_name(w, B, S, H, D, 0), "name": args.workload,
+                   "w": w, "B": B, "S_local": S, "H": H, "D": D},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -575,6 +604,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="cfg2",
+                    help="benchmark configuration (default cfg2: w=4, S_local=8192, H=24, D=128)")
+    ap.add_argument("--path", choices=["auto", "tma", "vec"], default="auto")
+    ap.add_argument("--chunked", type=int, choices=[0, 1, 2], default=0)
     ap.add_argument("--sweep", action="store_true",
                     help="also run the 128 KiB..2 GiB bandwidth sweep (w=2/4/8, bf16/fp32)")
     args = ap.parse_args()
