@@ -91,7 +91,7 @@ def hbm_peak():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs: torch copy, 1 Gi bf16)"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier measurement on this pool)"
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s copy bandwidth, an earlier B200 measurement)"
 
 
 def kernel_source_hash():

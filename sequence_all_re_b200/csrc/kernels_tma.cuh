@@ -130,6 +130,22 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 #define UA2A_CACHE_HINT 0
 #endif
 
+// Programmatic dependent launch (launch attribute + griddepcontrol); 0 turns
+// it off at build time, for measurement.
+#ifndef UA2A_PDL
+#define UA2A_PDL 1
+#endif
+
+// Let the next grid in the stream begin launching, then wait until every grid
+// this one depends on has finished and its memory operations are visible.
+// Both are no-ops for a grid launched without the programmatic attribute.
+__device__ __forceinline__ void pdl_launch_then_wait() {
+#if UA2A_PDL
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
+}
+
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t pol = 0;
 #if UA2A_CACHE_HINT
@@ -312,6 +328,9 @@ __global__ void __launch_bounds__(32 * kTmaMaxProducers, 1)
   for (int s = 0; s < S; ++s) mbar_init(bar0 + 8u * s, 1);
   fence_barrier_init();
   fence_proxy_async_smem();
+  // the previous kernel in the stream may still be running: wait for it
+  // before touching global memory (programmatic dependent launch)
+  pdl_launch_then_wait();
 
   auto unit_of = [&](int64_t m) { return first + (k + m * NP) * G; };
   auto issue_load = [&](int64_t m) {

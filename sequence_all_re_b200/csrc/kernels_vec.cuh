@@ -20,6 +20,11 @@
 
 #include "ulysses_a2a.h"
 
+// Programmatic dependent launch (see kernels_tma.cuh); 0 turns it off.
+#ifndef UA2A_PDL
+#define UA2A_PDL 1
+#endif
+
 namespace ua2a {
 
 // Division by a run-time invariant divisor d (1 <= d < 2^31) for dividends
@@ -72,6 +77,12 @@ __device__ __forceinline__ void st_stream(unsigned char* p, unsigned char v) { _
 
 template <typename V, int MODE, int U>
 __global__ void __launch_bounds__(256) ua2a_vec_kernel(const __grid_constant__ VecParams p) {
+#if UA2A_PDL
+  // programmatic dependent launch: start the next grid's launch, then wait for
+  // the previous one to finish before touching global memory
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
   const uint32_t nv = (uint32_t)p.nv;
   const int64_t strided_row = p.srow;  // vectors between rows s, s+1 of [B,S,H,D] (pitch)
   const uint32_t step = blockDim.x * U;

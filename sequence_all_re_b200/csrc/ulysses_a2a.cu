@@ -248,13 +248,40 @@ int check_residency(ulysses_a2a_ctx* ctx, const void* const* ptrs, int w, int64_
   return ULYSSES_A2A_OK;
 }
 
+// Launch with programmatic stream serialization (the kernels start with
+// griddepcontrol.wait, so a dependent launch cannot overtake its producer).
+template <typename Kernel, typename Params>
+cudaError_t launch_pdl(Kernel kernel, int grid, int block, size_t smem, cudaStream_t st,
+                       const Params& p) {
+#if UA2A_PDL
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, p);
+  if (e != cudaSuccess) return e;
+#else
+  kernel<<<grid, block, smem, st>>>(p);
+#endif
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tma(int mode, int grid, int block, size_t smem, cudaStream_t st,
+                       const TmaParams& p) {
+  return mode == 0 ? launch_pdl(ua2a::ua2a_tma_kernel<0>, grid, block, smem, st, p)
+                   : launch_pdl(ua2a::ua2a_tma_kernel<1>, grid, block, smem, st, p);
+}
+
 template <typename V>
 cudaError_t launch_vec_t(const VecParams& p, int mode, int grid, int block, cudaStream_t st) {
-  if (mode == 0)
-    ua2a::ua2a_vec_kernel<V, 0, 4><<<grid, block, 0, st>>>(p);
-  else
-    ua2a::ua2a_vec_kernel<V, 1, 4><<<grid, block, 0, st>>>(p);
-  return cudaGetLastError();
+  return mode == 0 ? launch_pdl(ua2a::ua2a_vec_kernel<V, 0, 4>, grid, block, 0, st, p)
+                   : launch_pdl(ua2a::ua2a_vec_kernel<V, 1, 4>, grid, block, 0, st, p);
 }
 
 cudaError_t launch_vec(const VecParams& p, int vec_bytes, int mode, int grid, int block,
@@ -308,10 +335,8 @@ int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, in
     }
     for (int l = 0; l < launches; ++l) {
       p.b0 = chunked ? l : 0;
-      if (mode == 0)
-        ua2a::ua2a_tma_kernel<0><<<grid, pl.block, (size_t)pl.smem_bytes, st>>>(p);
-      else
-        ua2a::ua2a_tma_kernel<1><<<grid, pl.block, (size_t)pl.smem_bytes, st>>>(p);
+      cudaError_t le = launch_tma(mode, grid, pl.block, (size_t)pl.smem_bytes, st, p);
+      if (le != cudaSuccess) return cuda_fail(ctx, "TMA kernel launch", le);
       cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess) return cuda_fail(ctx, "TMA kernel launch", e);
       ctx->launches++;
@@ -996,11 +1021,7 @@ extern "C" int ulysses_a2a_run_noalloc(const void* const* in_slabs, void* const*
     for (int l = 0; l < pl.launches; ++l) {
       p.b0 = chunked ? l : 0;
       p.status = st.scratch + kNoAllocSlotWords * l;
-      if (mode == 0)
-        ua2a::ua2a_tma_kernel<0><<<pl.grid, pl.block, (size_t)pl.smem_bytes, st_>>>(p);
-      else
-        ua2a::ua2a_tma_kernel<1><<<pl.grid, pl.block, (size_t)pl.smem_bytes, st_>>>(p);
-      e = cudaGetLastError();
+      e = launch_tma(mode, pl.grid, pl.block, (size_t)pl.smem_bytes, st_, p);
       if (e != cudaSuccess)
         return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "TMA kernel launch failed (plane %lld)", l);
     }
