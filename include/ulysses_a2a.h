@@ -28,6 +28,15 @@
  * ulysses_a2a_run_host is used) device staging buffers that grow on demand.
  * Nothing returned by this API ever aliases caller memory.
  *
+ * Launches: every kernel is launched with programmatic stream serialization
+ * (programmatic dependent launch) and waits for the previous grid in the
+ * stream (griddepcontrol.wait) before it touches memory, so it is safe after
+ * any producer. It also signals its dependents early: a kernel the caller
+ * launches next on the same stream WITH programmatic stream serialization
+ * must call cudaGridDependencySynchronize() before reading these outputs, as
+ * the CUDA programming model requires of such kernels. Kernels launched
+ * without that attribute, copies and events see the usual stream order.
+ *
  * Errors: every entry point returns an int status (ULYSSES_A2A_OK = 0). All
  * arguments are checked on the host BEFORE anything is launched; a rejected
  * call launches nothing, leaves the outputs untouched and the context usable,
