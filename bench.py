@@ -94,13 +94,24 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback (6.65 TB/s copy bandwidth, an earlier B200 measurement)"
 
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source with comments removed and whitespace collapsed."""
+    import re
+
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash():
+    """Hash of the library's code (comments and layout ignored): ncu counters
+    taken on one hash stay valid until the code itself changes."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sequence_all_re_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode())
-            h.update(f.read())
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -20,12 +20,24 @@
 // hardware: the load zero-fills the rows beyond the plane and the store skips
 // them. No multicast is used anywhere.
 //
-// One elected thread in each of `producers` warps per CTA drives its own ring
-// of `stages` shared-memory tiles over every producers-th unit this CTA owns
-// (u = blockIdx.x + i*gridDim.x, a static round-robin persistent schedule),
-// keeping `lookahead` loads and up to stages - lookahead stores in flight. Every mbarrier wait is bounded in time; on expiry the
-// kernel records the failure in the context's status word, waits (bounded)
-// for its own copies still in flight and returns.
+// Strided-side maps take the row pitch as their sequence stride, so a slab
+// may sit inside wider rows (q, k or v of a packed projection output).
+//
+// Schedule: one elected thread in each of `producers` warps per CTA drives its
+// own ring of `stages` shared-memory tiles over every producers-th unit this
+// CTA owns, keeping `lookahead` loads and up to stages - lookahead stores in
+// flight (TMA operations issued by one thread complete roughly one at a time,
+// so several producers keep enough in flight). A CTA owns either a chunk of
+// `chunk_units` consecutive units (the default: short-lived CTAs, several per
+// SM, handed out by the hardware as SMs free up) or, with chunk_units = 0,
+// units blockIdx.x + i*gridDim.x of a persistent grid. Units are numbered with
+// the destination rank innermost or outermost (`order`). Launches use
+// programmatic dependent launch: each CTA waits for the previous grid before
+// touching global memory.
+//
+// Every mbarrier wait is bounded in time; on expiry the kernel records the
+// failure in the context's status word, waits (bounded) for its own copies
+// still in flight and returns.
 #pragma once
 
 #include <cuda.h>
@@ -320,7 +332,7 @@ __global__ void __launch_bounds__(32 * kTmaMaxProducers, 1)
   if (first >= p.units || k >= NP) return;
   const int64_t n = n_cta > k ? (n_cta - k + NP - 1) / NP : 0;
   const int S = p.stages;      // stages of this producer's sub-ring
-  const int L = p.lookahead;   // its loads in flight, 1 <= L < S
+  const int L = p.lookahead;   // its loads in flight, 1 <= L < S (L = S = 1 allowed)
   const uint32_t smem0 = smem_addr(smem) + (uint32_t)(k * S) * p.stage_bytes;
   const uint32_t bar0 = smem_addr(full) + 8u * (uint32_t)(k * S);
 
