@@ -687,3 +687,26 @@ def test_randomized_shapes_layouts_and_knobs():
     finally:
         for c in ctxs.values():
             c.close()
+
+
+def test_two_contexts_on_two_streams_concurrently():
+    # independent contexts and streams: results must not interfere
+    w, B, S, H, D = 4, 2, 300, 8, 128
+    xa = normal_slabs((B, S, H, D), w, "bf16", seed0=901)
+    xb = normal_slabs((B, S * w, H // w, D), w, "bf16", seed0=902)
+    wa, wb = oracle.ulysses_a2a(xa, 0), oracle.ulysses_a2a(xb, 1)
+    sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
+    with UlyssesA2A(0, 2) as c1, UlyssesA2A(0, 2) as c2:
+        c2.set_path(PATH_VEC)
+        da, db = [t.cuda() for t in xa], [t.cuda() for t in xb]
+        ya = [torch.empty(B, S * w, H // w, D, dtype=torch.bfloat16, device="cuda") for _ in range(w)]
+        yb = [torch.empty(B, S, H, D, dtype=torch.bfloat16, device="cuda") for _ in range(w)]
+        torch.cuda.synchronize()
+        for _ in range(20):
+            c1.run(da, 0, out=ya, stream=sa)
+            c2.run(db, 1, out=yb, stream=sb, chunked=True)
+        c1.status(sa)
+        c2.status(sb)
+        for k in range(w):
+            assert torch.equal(bits(ya[k].cpu()), bits(wa[k]))
+            assert torch.equal(bits(yb[k].cpu()), bits(wb[k]))
