@@ -112,8 +112,8 @@ def ulysses_a2a(inputs, mode: int, chunked: bool = False, lib: ctypes.CDLL | Non
         o = torch.empty(out_shape, dtype=dt)
         o.view(torch.uint8).fill_(0xFF) if o.numel() else None
         outs.append(o)
-    in_arr = (ctypes.c_void_p * w)(*[t.data_ptr() for t in ins])
-    out_arr = (ctypes.c_void_p * w)(*[t.data_ptr() for t in outs])
+    in_arr = (ctypes.c_void_p * w)(*[t.data_ptr() or None for t in ins])
+    out_arr = (ctypes.c_void_p * w)(*[t.data_ptr() or None for t in outs])
     fn = lib.oracle_ulysses_a2a_chunked if chunked else lib.oracle_ulysses_a2a
     rc = fn(in_arr, out_arr, B, S_local, H, D, w, int(mode), ins[0].element_size())
     if rc != 0:

@@ -26,22 +26,26 @@
  * Elements are copied as raw bytes (elem_bytes each): no arithmetic touches a
  * value, so NaN payloads and signed zeros survive unchanged.
  *
- * Return codes: 0 = done; -1 = bad argument (null pointer, non-positive size,
- * H not divisible by w, unsupported mode or element size).
+ * Return codes: 0 = done; -1 = bad argument (null pointer for a non-empty
+ * slab, negative size, H not divisible by w, unsupported mode or element
+ * size). Zero sizes are an empty re-layout: done, nothing touched.
  */
 #include <stdint.h>
 #include <string.h>
 
+/* A size of 0 makes the index set empty: nothing is read or written, and
+ * the slab pointers may then be NULL. */
 static int bad_args(const void *const *in, void *const *out, int64_t B,
                     int64_t S_local, int64_t H, int64_t D, int w, int mode,
                     int elem_bytes)
 {
     if (in == NULL || out == NULL) return 1;
-    if (w < 1 || B < 1 || S_local < 1 || H < 1 || D < 1) return 1;
+    if (w < 1 || B < 0 || S_local < 0 || H < 0 || D < 0) return 1;
     if (H % w != 0) return 1;
     if (mode != 0 && mode != 1) return 1;
     if (elem_bytes < 1) return 1;
-    for (int k = 0; k < w; ++k)
+    const int empty = (B == 0 || S_local == 0 || H == 0 || D == 0);
+    for (int k = 0; k < w && !empty; ++k)
         if (in[k] == NULL || out[k] == NULL) return 1;
     return 0;
 }

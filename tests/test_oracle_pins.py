@@ -62,5 +62,20 @@ def test_rejects_bad_arguments():
     a = (ctypes.c_void_p * 2)(good[0].data_ptr(), good[1].data_ptr())
     b = (ctypes.c_void_p * 2)(good[2].data_ptr(), good[3].data_ptr())
     assert lib.oracle_ulysses_a2a(a, b, 1, 1, 2, 1, 2, 2, 4) == -1    # mode 2
-    assert lib.oracle_ulysses_a2a(a, b, 0, 1, 2, 1, 2, 0, 4) == -1    # B = 0
+    assert lib.oracle_ulysses_a2a(a, b, -1, 1, 2, 1, 2, 0, 4) == -1   # B < 0
     assert lib.oracle_ulysses_a2a(a, b, 1, 1, 2, 1, 2, 0, 4) == 0
+
+
+def test_empty_index_sets_are_a_no_op():
+    # the definition over an empty index set moves nothing; NULL slabs allowed
+    import ctypes
+    lib = oracle._get_lib()
+    nul = (ctypes.c_void_p * 2)(None, None)
+    for (B, S, H, D) in [(0, 3, 4, 2), (2, 0, 4, 2), (2, 3, 0, 2), (2, 3, 4, 0)]:
+        assert lib.oracle_ulysses_a2a(nul, nul, B, S, H, D, 2, 0, 2) == 0
+        assert lib.oracle_ulysses_a2a_chunked(nul, nul, B, S, H, D, 2, 1, 2) == 0
+        x = [torch.zeros(B, S, H, D) for _ in range(2)]
+        y = oracle.ulysses_a2a(x, 0)
+        assert all(tuple(t.shape) == (B, S * 2, H // 2, D) for t in y)
+    # a zero size does not hide a non-empty slab's NULL pointer
+    assert lib.oracle_ulysses_a2a(nul, nul, 1, 1, 2, 1, 2, 0, 2) == -1
