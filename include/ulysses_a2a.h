@@ -136,7 +136,9 @@ int ulysses_a2a_destroy(ulysses_a2a_ctx *ctx);
  *   in_slabs  : host array of w device pointers, the input slab of each rank.
  *   out_slabs : host array of w device pointers, caller-allocated outputs. No
  *               output may overlap any input or any other output.
- *   B, S_local, H, D : mode-0-local sizes, all >= 1, H % w == 0.
+ *   B, S_local, H, D : mode-0-local sizes, all >= 0, H % w == 0. If any is
+ *               0 the re-layout is empty: the call returns ULYSSES_A2A_OK
+ *               without launching anything (slab pointers may be NULL).
  *   w         : rank count, 1 <= w <= ULYSSES_A2A_MAX_W (w = 1 is a copy).
  *   mode      : 0 (scatter heads, gather sequence) or 1 (the inverse).
  *   chunked   : 0 = one launch over all B planes; 1 = the per-plane variant:

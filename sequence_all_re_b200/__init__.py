@@ -152,8 +152,8 @@ class UlyssesA2A:
         if stream is None:
             stream = torch.cuda.current_stream(self.device)
         handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
-        rc = _lib.ulysses_a2a_run_ex(self._ctx, [t.data_ptr() for t in xs],
-                                     [o.data_ptr() for o in out], B, S, H, D, w, mode,
+        rc = _lib.ulysses_a2a_run_ex(self._ctx, [t.data_ptr() or 0 for t in xs],
+                                     [o.data_ptr() or 0 for o in out], B, S, H, D, w, mode,
                                      int(chunked), self._last_pitch, handle)
         self._check(rc)
         return out

@@ -188,7 +188,7 @@ lib = _load()
 
 
 def ptr_array(ptrs) -> ctypes.Array:
-    return (ctypes.c_void_p * len(ptrs))(*[int(p) for p in ptrs])
+    return (ctypes.c_void_p * len(ptrs))(*[int(p) or None for p in ptrs])
 
 
 # ---- same-named thin wrappers -------------------------------------------------

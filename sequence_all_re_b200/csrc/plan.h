@@ -155,11 +155,22 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
   }
   if (mode != 0 && mode != 1) { set_err(err, "mode=%lld not 0 or 1", mode); return ULYSSES_A2A_ERR_INVALID; }
   if (chunked < 0 || chunked > 2) { set_err(err, "chunked=%lld not 0, 1 or 2", chunked); return ULYSSES_A2A_ERR_INVALID; }
-  if (B < 1 || S < 1 || H < 1 || D < 1) {
-    set_err(err, "sizes must be >= 1 (B, S_local, H, D)");
+  if (B < 0 || S < 0 || H < 0 || D < 0) {
+    set_err(err, "sizes must be >= 0 (B, S_local, H, D)");
     return ULYSSES_A2A_ERR_INVALID;
   }
   if (H % w != 0) { set_err(err, "H=%lld not divisible by w=%lld", H, w); return ULYSSES_A2A_ERR_INVALID; }
+  if (B == 0 || S == 0 || H == 0 || D == 0) {
+    // an empty re-layout: nothing to read or write, nothing to launch (slab
+    // pointers may be NULL)
+    if (forced_path < ULYSSES_A2A_PATH_AUTO || forced_path > ULYSSES_A2A_PATH_VEC) {
+      set_err(err, "unknown path %lld", forced_path);
+      return ULYSSES_A2A_ERR_INVALID;
+    }
+    p->path = forced_path == ULYSSES_A2A_PATH_AUTO ? ULYSSES_A2A_PATH_VEC : forced_path;
+    p->row_pitch = row_pitch > 0 ? row_pitch : H * D;
+    return ULYSSES_A2A_OK;
+  }
   if (forced_path < ULYSSES_A2A_PATH_AUTO || forced_path > ULYSSES_A2A_PATH_VEC) {
     set_err(err, "unknown path %lld", forced_path);
     return ULYSSES_A2A_ERR_INVALID;

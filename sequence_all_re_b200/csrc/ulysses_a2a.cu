@@ -531,6 +531,7 @@ int ulysses_a2a_run_ex(ulysses_a2a_ctx* ctx, const ulysses_a2a_desc_t* d, void* 
   int rc = plan_for(ctx, d->in_slabs, d->out_slabs, d->B, d->S_local, d->H, d->D, d->w, d->mode,
                     d->chunked, &pl, d->row_pitch);
   if (rc) return rc;
+  if (pl.units == 0) return ULYSSES_A2A_OK;  // empty: nothing to do
   DeviceGuard g(ctx->device);
   if (!g.ok) return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "cannot select the context's device");
   const int64_t dense_bytes = pl.payload_bytes / d->w;
@@ -576,6 +577,7 @@ int ulysses_a2a_run_host(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void
   ulysses_a2a_plan_t host_pl;
   int rc = plan_for(ctx, in_slabs, out_slabs, B, S_local, H, D, w, mode, chunked, &host_pl);
   if (rc) return rc;
+  if (host_pl.units == 0) return ULYSSES_A2A_OK;  // empty: nothing to do
   DeviceGuard g(ctx->device);
   if (!g.ok) return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "cannot select the context's device");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -938,6 +940,7 @@ extern "C" int ulysses_a2a_run_noalloc(const void* const* in_slabs, void* const*
     if (err && errlen) std::snprintf(err, errlen, "%s", msg.c_str());
     return rc;
   }
+  if (pl.units == 0) return ULYSSES_A2A_OK;  // empty: nothing to do
   const int slots = pl.launches;
   if (slots > kNoAllocSlots)
     return noalloc_report(err, errlen, ULYSSES_A2A_ERR_UNSUPPORTED,

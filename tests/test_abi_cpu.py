@@ -226,9 +226,9 @@ def test_large_rows_reduce_stages_then_producers():
 
 @pytest.mark.parametrize("args,code", [
     (dict(w=2, B=1, S=4, H=3, D=8), ERR_INVALID),        # H % w
-    (dict(w=2, B=0, S=4, H=4, D=8), ERR_INVALID),
-    (dict(w=2, B=1, S=0, H=4, D=8), ERR_INVALID),
-    (dict(w=2, B=1, S=4, H=4, D=0), ERR_INVALID),
+    (dict(w=2, B=-1, S=4, H=4, D=8), ERR_INVALID),
+    (dict(w=2, B=1, S=-3, H=4, D=8), ERR_INVALID),
+    (dict(w=2, B=1, S=4, H=4, D=-1), ERR_INVALID),
     (dict(w=0, B=1, S=4, H=4, D=8), ERR_INVALID),
     (dict(w=65, B=1, S=4, H=65, D=8), ERR_INVALID),
     (dict(w=2, B=1, S=4, H=4, D=8, mode=2), ERR_INVALID),
@@ -245,6 +245,17 @@ def test_rejects_bad_arguments(args, code):
     rc, _, msg = ulysses_a2a_plan(ins[:max(w, 0)] or [0], outs[:max(w, 0)] or [0], B, S, H, D, w,
                                   mode, chunked, E)
     assert rc == code and msg
+
+
+@pytest.mark.parametrize("B,S,H,D", [(0, 4, 4, 8), (1, 0, 4, 8), (1, 4, 0, 8), (1, 4, 4, 0)])
+def test_empty_relayout_is_a_no_op_plan(B, S, H, D):
+    # any zero size: nothing to move, nothing to launch, NULL slabs accepted
+    for chunked in (0, 1, 2):
+        rc, p, msg = ulysses_a2a_plan([0, 0], [0, 0], B, S, H, D, 2, 0, chunked, 2)
+        assert rc == OK, msg
+        assert p.units == 0 and p.launches == 0 and p.payload_bytes == 0
+    rc, _, _ = ulysses_a2a_plan([0, 0], [0, 0], B, S, 3, D, 2, 0, 0, 2)   # H % w still checked
+    assert rc == ERR_INVALID
 
 
 def test_rejects_size_overflow():

@@ -710,3 +710,57 @@ def test_two_contexts_on_two_streams_concurrently():
         for k in range(w):
             assert torch.equal(bits(ya[k].cpu()), bits(wa[k]))
             assert torch.equal(bits(yb[k].cpu()), bits(wb[k]))
+
+
+# ---- edge sizes: empty, maximum rank count, box limits, a 2 GiB payload -------
+
+def test_empty_relayouts_launch_nothing():
+    with UlyssesA2A(0, 2) as a2a:
+        for shape, mode in [((0, 8, 4, 64), 0), ((2, 0, 4, 64), 0), ((2, 8, 4, 0), 0),
+                            ((2, 0, 2, 64), 1)]:
+            xs = [torch.empty(shape, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+            for chunked in (0, 1, 2):
+                n0 = a2a.launch_count
+                ys = a2a.run(xs, mode, chunked=chunked)
+                assert a2a.launch_count == n0
+                assert all(y.numel() == 0 for y in ys)
+                assert tuple(ys[0].shape) == oracle.output_shape(shape, mode, 2)
+            hs = a2a.run_host([x.cpu() for x in xs], mode)
+            assert all(h.numel() == 0 for h in hs)
+        a2a.status()
+    rc, msg = _lib.ulysses_a2a_run_noalloc([0, 0], [0, 0], 0, 8, 4, 64, 2, 0, 0, 2,
+                                           torch.cuda.current_stream().cuda_stream)
+    assert rc == _lib.OK, msg
+
+
+def test_maximum_rank_count():
+    w, B, S, H, D = 64, 1, 3, 64, 16            # ULYSSES_A2A_MAX_W ranks
+    for mode in (0, 1):
+        xs = unique_slabs(slab_shape(mode, w, B, S, H, D), w, 4)
+        run_case(xs, mode)
+        run_case(xs, mode, chunked=2)
+
+
+def test_tma_box_and_tile_limits():
+    # H/w = 128 heads x D = 256 bf16: one 64 KB row per tile, the largest TMA tile
+    w, B, S, H, D = 2, 2, 5, 256, 256
+    with UlyssesA2A(0, 2) as a2a:
+        xs = normal_slabs((B, S, H, D), w, "bf16", seed0=950)
+        p = a2a.plan([t.cuda() for t in xs], 0)
+        assert p["path"] == PATH_TMA and p["rows_per_tile"] == 1 and p["row_bytes"] == 64 * 1024
+        for mode, x in ((0, xs), (1, oracle.ulysses_a2a(xs, 0))):
+            run_case(x, mode, a2a=a2a, path=PATH_TMA)
+            run_case(x, mode, a2a=a2a, path=PATH_TMA, tuning=dict(chunk_units=0))
+    # rows just over the tile limit go to the VEC path
+    w, B, S, H, D = 2, 1, 3, 264, 256
+    xs = normal_slabs((B, S, H, D), w, "bf16", seed0=951)
+    run_case(xs, 0)
+
+
+def test_two_gib_payload_full_compare():
+    # w = 8, H = 64, D = 128, S_local = 16384: 2 GiB of bf16 per call
+    w, B, S, H, D = 8, 1, 16384, 64, 128
+    xs = uniform_slabs((B, S, H, D), w, "bf16", seed0=960)
+    y = run_case(xs, 0)
+    del xs
+    run_case(y, 1)
