@@ -103,12 +103,17 @@ def _code_only(text: str) -> str:
     return " ".join(text.split())
 
 
+KERNEL_FILES = ("kernels_tma.cuh", "kernels_vec.cuh")
+LAUNCH_FIELDS = ("path", "rows_per_tile", "producers", "stages", "lookahead", "chunk_units",
+                 "order", "grid", "block", "smem_bytes", "vec_bytes")
+
+
 def kernel_source_hash():
-    """Hash of the library's code (comments and layout ignored): ncu counters
-    taken on one hash stay valid until the code itself changes."""
+    """Hash of the kernels' device code (comments and layout ignored): ncu
+    counters taken on one hash stay valid until that code changes."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sequence_all_re_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_FILES:
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode())
             h.update(_code_only(f.read()).encode())
@@ -411,9 +416,14 @@ def run_ours(args):
     traffic_bytes = None
     if traffic:
         key = workload_key(w, B, S, H, D, {1: "tma", 2: "vec"}[plan["path"]])
-        traffic_bytes = traffic.get("workloads", {}).get(key, {}).get("dram_bytes_per_launch")
-        if traffic_bytes is None:
+        entry = traffic.get("workloads", {}).get(key, {})
+        launch = entry.get("launch", {})
+        if not entry:
             traffic_src = "no ncu capture of this kernel and workload"
+        elif chunked or any(launch.get(f) != plan[f] for f in LAUNCH_FIELDS):
+            traffic_src = "the capture was taken with another launch shape"
+        else:
+            traffic_bytes = entry.get("dram_bytes_per_launch")
 
     # per mode: back to back, and call by call after an L2 write flush
     reps = max(20, min(args.steps, 400))
