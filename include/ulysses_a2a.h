@@ -275,6 +275,94 @@ int ulysses_a2a_plan_ex(const ulysses_a2a_desc_t *desc, int elem_bytes,
                         int num_sms, ulysses_a2a_plan_t *out, char *err,
                         size_t errlen);
 
+/* ---- multi-GPU exchange through published windows ----------------------
+ *
+ * One process per GPU, w ranks. Each rank owns a device window that every
+ * other rank maps (CUDA IPC, or directly when the ranks share a process), in
+ * the manner of the FastVideo API docs' ulysses_a2a communicator: a window
+ * built once and reused call after call and plane after plane (`run_armed`,
+ * chunked branch), rebuilt when a call needs more bytes (`try_all_to_all_4D`,
+ * window grow), and torn down collectively (`close`). The pypto-lib pull
+ * request "pipeline HCA AllToAll into O-A" publishes each rank's output into a
+ * distributed window and has consumers load from it after a handshake; the
+ * exchange here follows the same order:
+ *
+ *   1. ulysses_a2a_peer_publish: copy this rank's input slab (or one plane of
+ *      it) into this rank's window, dense;
+ *   2. a barrier: every rank's publish is complete;
+ *   3. ulysses_a2a_peer_pull: one kernel reads this rank's share out of every
+ *      rank's window (peer loads over NVLink) and writes this rank's output
+ *      slab, with the same element map as ulysses_a2a_run, of which it is the
+ *      launch restricted to output slab `rank`;
+ *   4. a barrier: every rank's pull is complete, so the windows may be
+ *      published into again.
+ *
+ * The barriers are the caller's (a stream-ordered collective such as a
+ * one-element NCCL all-reduce on the same stream, or a stream synchronise plus
+ * a host barrier): this library launches no kernel that waits for another GPU.
+ * Chunked calls pass one-plane views (B = 1) and repeat 1-4 per plane.
+ * Sizes are mode-0-local as everywhere in this header; in mode 0 rank k's
+ * input is x_k [B, S_local, H, D] (row pitch allowed) and its output out_k
+ * [B, S_local*w, H/w, D]; in mode 1 the input is [B, S_local*w, H/w, D] and
+ * the output [B, S_local, H, D] (row pitch allowed). A window must hold one
+ * input slab of the largest call: B*S_local*H*D*elem_bytes bytes. The output
+ * never aliases a window.
+ */
+typedef struct ulysses_a2a_peer ulysses_a2a_peer; /* opaque */
+
+#define ULYSSES_A2A_PEER_HANDLE_BYTES 128 /* size of one exchanged record */
+
+/* Allocate this rank's window (window_bytes >= 1, on ctx's device) and write
+ * its exchange record, ULYSSES_A2A_PEER_HANDLE_BYTES bytes, into handle_out.
+ * The caller gathers every rank's record, in rank order, to every rank (for
+ * example with an all-gather) and passes them to ulysses_a2a_peer_open. The
+ * peer object uses ctx (element size, device, status) and must be destroyed
+ * before it. 1 <= world <= ULYSSES_A2A_MAX_W, 0 <= rank < world. */
+int ulysses_a2a_peer_create(ulysses_a2a_ctx *ctx, int rank, int world,
+                            size_t window_bytes, ulysses_a2a_peer **out,
+                            void *handle_out);
+
+/* Map every other rank's window. handles: world records in rank order, as
+ * written by each rank's ulysses_a2a_peer_create. Records must agree on
+ * world, element size and window size, and record k must come from rank k;
+ * a record from this same process is used directly (its device gets peer
+ * access if it differs from ctx's), any other is opened with CUDA IPC.
+ * Fails without mapping anything if a record is malformed. */
+int ulysses_a2a_peer_open(ulysses_a2a_peer *peer, const void *handles);
+
+/* Step 1: copy this rank's input slab into its own window (asynchronous on
+ * stream). mode 0: in_local is [B, S_local, H, D] with row_pitch (0 = dense,
+ * else >= H*D elements between rows, as in ulysses_a2a_desc_t); mode 1:
+ * in_local is [B, S_local*w, H/w, D] dense and row_pitch must be 0. The
+ * window receives the dense slab. */
+int ulysses_a2a_peer_publish(ulysses_a2a_peer *peer, const void *in_local,
+                             int64_t B, int64_t S_local, int64_t H, int64_t D,
+                             int mode, int64_t row_pitch, void *stream);
+
+/* Step 3: write this rank's output slab from every rank's published window
+ * (asynchronous on stream; VEC kernel, peer loads). out_local is on ctx's
+ * device, caller-owned, and overlaps no window. mode 0: out_local is
+ * [B, S_local*w, H/w, D] dense, row_pitch must be 0; mode 1: out_local is
+ * [B, S_local, H, D] with row_pitch (0 = dense). Requires
+ * ulysses_a2a_peer_open to have succeeded. */
+int ulysses_a2a_peer_pull(ulysses_a2a_peer *peer, void *out_local, int64_t B,
+                          int64_t S_local, int64_t H, int64_t D, int mode,
+                          int64_t row_pitch, void *stream);
+
+/* Base address of rank k's window as this process sees it (NULL if k is out
+ * of range or not mapped yet), and the window size in bytes. */
+void *ulysses_a2a_peer_window(const ulysses_a2a_peer *peer, int rank);
+size_t ulysses_a2a_peer_window_bytes(const ulysses_a2a_peer *peer);
+
+/* Unmap the other ranks' windows (synchronising ctx's device first); the own
+ * window stays. Call it on every rank, then barrier, then destroy: a window
+ * must not be freed while a peer still maps it. Idempotent. */
+int ulysses_a2a_peer_close(ulysses_a2a_peer *peer);
+
+/* Close (if not done) and free the own window; consumes the handle even when
+ * a CUDA call reports an error. NULL is accepted. */
+int ulysses_a2a_peer_destroy(ulysses_a2a_peer *peer);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif

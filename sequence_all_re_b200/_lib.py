@@ -44,7 +44,17 @@ EXPORTED = (
     "ulysses_a2a_run_ex",
     "ulysses_a2a_plan_ex",
     "ulysses_a2a_selftest_wait_timeout",
+    "ulysses_a2a_peer_create",
+    "ulysses_a2a_peer_open",
+    "ulysses_a2a_peer_publish",
+    "ulysses_a2a_peer_pull",
+    "ulysses_a2a_peer_window",
+    "ulysses_a2a_peer_window_bytes",
+    "ulysses_a2a_peer_close",
+    "ulysses_a2a_peer_destroy",
 )
+
+PEER_HANDLE_BYTES = 128
 
 
 class PlanT(ctypes.Structure):
@@ -181,6 +191,22 @@ def _load() -> ctypes.CDLL:
     lib.ulysses_a2a_plan_ex.restype = c_int
     lib.ulysses_a2a_selftest_wait_timeout.argtypes = [P, ctypes.c_uint32, P]
     lib.ulysses_a2a_selftest_wait_timeout.restype = c_int
+    lib.ulysses_a2a_peer_create.argtypes = [P, c_int, c_int, ctypes.c_size_t, ctypes.POINTER(P), P]
+    lib.ulysses_a2a_peer_create.restype = c_int
+    lib.ulysses_a2a_peer_open.argtypes = [P, P]
+    lib.ulysses_a2a_peer_open.restype = c_int
+    lib.ulysses_a2a_peer_publish.argtypes = [P, P, i64, i64, i64, i64, c_int, i64, P]
+    lib.ulysses_a2a_peer_publish.restype = c_int
+    lib.ulysses_a2a_peer_pull.argtypes = [P, P, i64, i64, i64, i64, c_int, i64, P]
+    lib.ulysses_a2a_peer_pull.restype = c_int
+    lib.ulysses_a2a_peer_window.argtypes = [P, c_int]
+    lib.ulysses_a2a_peer_window.restype = P
+    lib.ulysses_a2a_peer_window_bytes.argtypes = [P]
+    lib.ulysses_a2a_peer_window_bytes.restype = ctypes.c_size_t
+    lib.ulysses_a2a_peer_close.argtypes = [P]
+    lib.ulysses_a2a_peer_close.restype = c_int
+    lib.ulysses_a2a_peer_destroy.argtypes = [P]
+    lib.ulysses_a2a_peer_destroy.restype = c_int
     return lib
 
 
@@ -282,3 +308,49 @@ def ulysses_a2a_plan_ex(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, e
     rc = lib.ulysses_a2a_plan_ex(ctypes.byref(d), int(elem_bytes), int(forced_path),
                                  ctypes.byref(t), int(num_sms), ctypes.byref(plan), buf, len(buf))
     return rc, plan, buf.value.decode()
+
+
+# ---- multi-GPU exchange through published windows ------------------------------
+
+def ulysses_a2a_peer_create(ctx, rank: int, world: int, window_bytes: int):
+    """Returns (rc, peer handle, the rank's exchange record as bytes)."""
+    h = ctypes.c_void_p()
+    rec = ctypes.create_string_buffer(PEER_HANDLE_BYTES)
+    rc = lib.ulysses_a2a_peer_create(ctx, int(rank), int(world), int(window_bytes),
+                                     ctypes.byref(h), rec)
+    return rc, h, rec.raw
+
+
+def ulysses_a2a_peer_open(peer, records) -> int:
+    """records: every rank's exchange record (bytes), in rank order."""
+    blob = b"".join(bytes(r) for r in records)
+    buf = ctypes.create_string_buffer(blob, len(blob))
+    return lib.ulysses_a2a_peer_open(peer, buf)
+
+
+def ulysses_a2a_peer_publish(peer, in_ptr, B, S_local, H, D, mode, row_pitch, stream) -> int:
+    return lib.ulysses_a2a_peer_publish(peer, ctypes.c_void_p(int(in_ptr) or None), int(B),
+                                        int(S_local), int(H), int(D), int(mode), int(row_pitch),
+                                        ctypes.c_void_p(int(stream)))
+
+
+def ulysses_a2a_peer_pull(peer, out_ptr, B, S_local, H, D, mode, row_pitch, stream) -> int:
+    return lib.ulysses_a2a_peer_pull(peer, ctypes.c_void_p(int(out_ptr) or None), int(B),
+                                     int(S_local), int(H), int(D), int(mode), int(row_pitch),
+                                     ctypes.c_void_p(int(stream)))
+
+
+def ulysses_a2a_peer_window(peer, rank: int) -> int:
+    return int(lib.ulysses_a2a_peer_window(peer, int(rank)) or 0)
+
+
+def ulysses_a2a_peer_window_bytes(peer) -> int:
+    return int(lib.ulysses_a2a_peer_window_bytes(peer))
+
+
+def ulysses_a2a_peer_close(peer) -> int:
+    return lib.ulysses_a2a_peer_close(peer)
+
+
+def ulysses_a2a_peer_destroy(peer) -> int:
+    return lib.ulysses_a2a_peer_destroy(peer)

@@ -14,6 +14,10 @@
 // time: up to S_tile rows of one (r, b, j) block, the last tile of a block
 // holding only the S_local % S_tile remaining rows (ceil-div tiling, clamped
 // row count). Each thread keeps U vectors in flight before storing them.
+//
+// A launch may cover every output slab or only one (r in [r0, r0 + nr) and
+// j in [j0, j0 + nj)): one rank's share of a multi-GPU exchange writes its own
+// output slab and reads every rank's published input through peer mappings.
 #pragma once
 
 #include <cstdint>
@@ -55,11 +59,13 @@ struct VecParams {
   int64_t srow;          // vectors between rows (b, s), (b, s+1) of the [B,S,H,D] side
   int32_t w;
   int32_t rows_per_tile;
-  uint32_t units;        // w * nb * w * T
+  uint32_t units;        // nr * nb * nj * T
   int32_t order;         // unit numbering: 0 = r outermost, 1 = r innermost
   uint32_t tile0;        // first tile of each (r, b, j) block in this launch
+  uint32_t r0, j0;       // first r and first j this launch covers
   FastDiv div_T;         // tiles per (r, b, j) block in this launch
-  FastDiv div_w;
+  FastDiv div_nr;        // r values covered (w, or 1 for one output slab)
+  FastDiv div_nj;        // j values covered
   FastDiv div_nb;        // planes in this launch
   FastDiv div_nv;
 };
@@ -89,22 +95,24 @@ __global__ void __launch_bounds__(256) ua2a_vec_kernel(const __grid_constant__ V
   for (uint32_t u = blockIdx.x; u < p.units; u += gridDim.x) {
     uint32_t t, j, r, bl;
     if (p.order == 0) {
-      // u = ((r * nb + b_rel) * w + j) * T + t
+      // u = ((r_rel * nb + b_rel) * nj + j_rel) * T + t
       const uint32_t q = fdiv(u, p.div_T);
       t = u - q * p.div_T.d;
-      const uint32_t q2 = fdiv(q, p.div_w);
-      j = q - q2 * p.div_w.d;
+      const uint32_t q2 = fdiv(q, p.div_nj);
+      j = q - q2 * p.div_nj.d;
       r = fdiv(q2, p.div_nb);
       bl = q2 - r * p.div_nb.d;
     } else {
-      // u = ((b_rel * w + j) * T + t) * w + r
-      const uint32_t q = fdiv(u, p.div_w);
-      r = u - q * p.div_w.d;
+      // u = ((b_rel * nj + j_rel) * T + t) * nr + r_rel
+      const uint32_t q = fdiv(u, p.div_nr);
+      r = u - q * p.div_nr.d;
       const uint32_t q2 = fdiv(q, p.div_T);
       t = q - q2 * p.div_T.d;
-      bl = fdiv(q2, p.div_w);
-      j = q2 - bl * p.div_w.d;
+      bl = fdiv(q2, p.div_nj);
+      j = q2 - bl * p.div_nj.d;
     }
+    r += p.r0;
+    j += p.j0;
     const int64_t b = p.b0 + bl;
     const int64_t s0 = (int64_t)(p.tile0 + t) * p.rows_per_tile;
     const int64_t rows_left = p.S_local - s0;

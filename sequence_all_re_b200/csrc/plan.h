@@ -135,10 +135,14 @@ inline bool tuning_from(const ulysses_a2a_tuning_t* t, Tuning* out, std::string*
 // Validate and plan one call. Returns a ULYSSES_A2A_* status.
 // row_pitch: elements between consecutive (b, s) rows of the [B, S, H, D]
 // side (0 = dense, H*D); that side's planes are S*row_pitch elements apart.
+// only_out >= 0: the call writes output slab only_out alone (VEC path); the
+// other out[] entries are neither checked nor used, and units counts that
+// slab's blocks only.
 inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t S,
                      int64_t H, int64_t D, int w, int mode, int chunked, int E,
                      int forced_path, const Tuning& tune, int num_sms,
-                     ulysses_a2a_plan_t* p, std::string* err, int64_t row_pitch = 0) {
+                     ulysses_a2a_plan_t* p, std::string* err, int64_t row_pitch = 0,
+                     int only_out = -1) {
   if (p == nullptr) { set_err(err, "plan output is NULL"); return ULYSSES_A2A_ERR_INVALID; }
   *p = ulysses_a2a_plan_t{};
   if (in == nullptr || out == nullptr) {
@@ -154,6 +158,10 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     return ULYSSES_A2A_ERR_INVALID;
   }
   if (mode != 0 && mode != 1) { set_err(err, "mode=%lld not 0 or 1", mode); return ULYSSES_A2A_ERR_INVALID; }
+  if (only_out >= w || (only_out >= 0 && forced_path != ULYSSES_A2A_PATH_VEC)) {
+    set_err(err, "one-output plan: slab %lld of %lld, VEC path required", only_out, w);
+    return ULYSSES_A2A_ERR_INVALID;
+  }
   if (chunked < 0 || chunked > 2) { set_err(err, "chunked=%lld not 0, 1 or 2", chunked); return ULYSSES_A2A_ERR_INVALID; }
   if (B < 0 || S < 0 || H < 0 || D < 0) {
     set_err(err, "sizes must be >= 0 (B, S_local, H, D)");
@@ -200,8 +208,9 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
   }
   const int64_t in_bytes = mode == 0 ? strided_bytes : slab_bytes;
   const int64_t out_bytes = mode == 0 ? slab_bytes : strided_bytes;
+  auto used_out = [&](int k) { return only_out < 0 || k == only_out; };
   for (int k = 0; k < w; ++k) {
-    if (in[k] == nullptr || out[k] == nullptr) {
+    if (in[k] == nullptr || (used_out(k) && out[k] == nullptr)) {
       set_err(err, "slab pointer %lld is NULL", k);
       return ULYSSES_A2A_ERR_INVALID;
     }
@@ -209,6 +218,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
   // No output may overlap an input or another output (inputs may alias each
   // other). A pitched slab counts with its whole extent, gaps included.
   for (int k = 0; k < w; ++k) {
+    if (!used_out(k)) continue;
     const uintptr_t o = reinterpret_cast<uintptr_t>(out[k]);
     const uintptr_t oe = o + (uintptr_t)out_bytes;
     if (oe < o) { set_err(err, "output slab %lld wraps the address space", k); return ULYSSES_A2A_ERR_INVALID; }
@@ -218,7 +228,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
         set_err(err, "output slab %lld overlaps input slab %lld", k, m);
         return ULYSSES_A2A_ERR_OVERLAP;
       }
-      if (m != k) {
+      if (m != k && used_out(m)) {
         const uintptr_t q = reinterpret_cast<uintptr_t>(out[m]);
         if (overlaps(o, oe, q, q + (uintptr_t)out_bytes)) {
           set_err(err, "output slab %lld overlaps output slab %lld", k, m);
@@ -230,7 +240,8 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
 
   const int64_t Hw = H / w;
   const int64_t row_bytes = Hw * D * E;  // one contiguous run, L*E
-  const char* blocker = tma_blocker(in, out, B, S, H, D, w, E, row_bytes, pitch);
+  const char* blocker = only_out >= 0 ? "one-output launches use the VEC path"
+                                      : tma_blocker(in, out, B, S, H, D, w, E, row_bytes, pitch);
   int path;
   if (forced_path == ULYSSES_A2A_PATH_TMA) {
     if (blocker) {
@@ -256,8 +267,9 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
 
   const int64_t T = (S + rows - 1) / rows;  // ceil-div: the ragged last tile is a unit too
   const int64_t nb = chunked ? 1 : B;
+  const int64_t blocks_wide = only_out >= 0 ? (int64_t)w : (int64_t)w * w;
   int64_t units;
-  if (mul_overflows((int64_t)w * w, nb, &tmp) || mul_overflows(tmp, T, &units)) {
+  if (mul_overflows(blocks_wide, nb, &tmp) || mul_overflows(tmp, T, &units)) {
     set_err(err, "unit count overflows");
     return ULYSSES_A2A_ERR_INVALID;
   }
@@ -268,7 +280,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
   p->tiles_per_block = T;
   p->tail_rows = S % rows;
   p->units = units;
-  p->payload_bytes = payload;
+  p->payload_bytes = only_out >= 0 ? slab_bytes : payload;
   p->launches = chunked ? (int32_t)(B > INT32_MAX ? INT32_MAX : B) : 1;
   p->row_pitch = pitch;
   p->order = tune.order >= 0 ? (tune.order ? 1 : 0) : kDefaultOrder;
@@ -340,7 +352,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
       bool ok = (row_bytes % v) == 0 && ((pitch * E) % v) == 0;
       for (int k = 0; k < w && ok; ++k)
         ok = (reinterpret_cast<uintptr_t>(in[k]) % v) == 0 &&
-             (reinterpret_cast<uintptr_t>(out[k]) % v) == 0;
+             (!used_out(k) || (reinterpret_cast<uintptr_t>(out[k]) % v) == 0);
       if (ok) break;
       v >>= 1;
     }

@@ -1,0 +1,280 @@
+"""Multi-GPU Ulysses all-to-all: one process per GPU, exchange through windows.
+
+Each rank holds its own sequence shard ``x_rank`` ([B, S_local, H, D]) on its
+own GPU; mode 0 gives every rank ``[B, S_local*w, H//w, D]`` (its head group,
+whole sequence), mode 1 undoes it, with the element map of the single-GPU
+re-layout (``UlyssesA2A``), of which rank k's part is the output slab k.
+
+The communicator follows the FastVideo API docs' ulysses_a2a helper:
+
+* a device window per rank, built once (``_build``) and reused call after
+  call; a call that needs more bytes closes and rebuilds it (window grow in
+  ``try_all_to_all_4D``);
+* ``chunked=True`` runs the exchange plane by plane on one-plane views, each
+  plane complete before the next reuses the window (``run_armed``);
+* the result owns its storage and never aliases the window;
+* teardown is collective (``close``): synchronise, agree, release.
+
+One exchange (per call, or per plane when chunked), as in the pypto-lib pull
+request "pipeline HCA AllToAll into O-A", which publishes into a distributed
+window and has consumers load from it after a handshake:
+barrier -> publish (own input into own window) -> barrier -> pull (one kernel
+reads this rank's share out of every window over NVLink and writes the local
+output). The barriers are collectives of the process group on the caller's
+stream (NCCL: a one-element all-reduce, stream ordered, no host wait) or, for
+host-only backends such as gloo, a stream synchronise plus a group barrier.
+No kernel waits for another GPU.
+
+Every copy runs in ``libulysses_a2a.so`` (``ulysses_a2a_peer_*``); this module
+only sequences the calls and the group's collectives.
+"""
+
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import UlyssesA2A, _lib, mode0_local_tuple, output_shape
+from ._lib import A2AError
+
+__all__ = ["PeerExchange", "NativePeer"]
+
+
+class NativePeer:
+    """The C ABI's peer object for one rank (marshalling only)."""
+
+    def __init__(self, device, elem_bytes: int):
+        self.a2a = UlyssesA2A(device, elem_bytes)
+        self.device = self.a2a.device
+        self.elem_bytes = self.a2a.elem_bytes
+        self._peer = None
+
+    def _check(self, rc):
+        if rc != _lib.OK:
+            raise A2AError(rc, self.a2a.last_error())
+
+    def create(self, rank: int, world: int, nbytes: int) -> bytes:
+        if self._peer is not None:
+            raise RuntimeError("window already built")
+        rc, h, rec = _lib.ulysses_a2a_peer_create(self.a2a._ctx, rank, world, nbytes)
+        self._check(rc)
+        self._peer = h
+        return rec
+
+    def open(self, records) -> None:
+        self._check(_lib.ulysses_a2a_peer_open(self._peer, records))
+
+    def publish(self, x, B, S, H, D, mode, row_pitch, stream) -> None:
+        self._check(_lib.ulysses_a2a_peer_publish(self._peer, x.data_ptr(), B, S, H, D, mode,
+                                                  row_pitch, stream.cuda_stream))
+
+    def pull(self, out, B, S, H, D, mode, row_pitch, stream) -> None:
+        self._check(_lib.ulysses_a2a_peer_pull(self._peer, out.data_ptr(), B, S, H, D, mode,
+                                               row_pitch, stream.cuda_stream))
+
+    def window(self, rank: int) -> int:
+        return _lib.ulysses_a2a_peer_window(self._peer, rank) if self._peer is not None else 0
+
+    def unmap(self) -> None:
+        if self._peer is not None:
+            self._check(_lib.ulysses_a2a_peer_close(self._peer))
+
+    def release(self) -> None:
+        if self._peer is not None:
+            h, self._peer = self._peer, None
+            rc = _lib.ulysses_a2a_peer_destroy(h)
+            if rc != _lib.OK:
+                raise A2AError(rc, "peer_destroy reported a CUDA error (the handle is released)")
+
+    @property
+    def launch_count(self) -> int:
+        return self.a2a.launch_count
+
+    def current_stream(self):
+        return torch.cuda.current_stream(self.device)
+
+    def synchronize(self) -> None:
+        torch.cuda.synchronize(self.device)
+
+    def close(self) -> None:
+        self.release()
+        self.a2a.close()
+
+
+class PeerExchange:
+    """This rank's side of the multi-GPU Ulysses all-to-all over ``group``."""
+
+    def __init__(self, group=None, device=None, elem_bytes: int = 2, barrier: str = "auto",
+                 native=None):
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+        if native is None:
+            native = NativePeer(torch.cuda.current_device() if device is None else device,
+                                elem_bytes)
+        self.native = native
+        self.device = self.native.device
+        self.elem_bytes = int(elem_bytes)
+        if barrier == "auto":
+            barrier = "stream" if dist.get_backend(group) == "nccl" else "host"
+        if barrier not in ("stream", "host"):
+            raise ValueError("barrier must be 'auto', 'stream' or 'host'")
+        self.barrier_kind = barrier
+        self._flag = (torch.zeros(1, dtype=torch.int32, device=self.device)
+                      if barrier == "stream" else None)
+        self._nbytes = 0
+        self._armed = False
+        self._agreed = set()           # call signatures every rank has confirmed
+        self.disabled_reason = None
+
+    # ---------------------------------------------------------- group helpers
+    def _gather(self, obj):
+        out = [None] * self.world
+        dist.all_gather_object(out, obj, group=self.group)
+        return out
+
+    def _agree(self, ok: bool) -> bool:
+        return all(self._gather(bool(ok)))
+
+    def _barrier(self, stream) -> None:
+        if self.barrier_kind == "stream":
+            with torch.cuda.stream(stream):
+                dist.all_reduce(self._flag, group=self.group)
+        else:
+            stream.synchronize()
+            dist.barrier(group=self.group)
+
+    def _disable(self, reason: str) -> None:
+        self.disabled_reason = reason
+
+    # --------------------------------------------------------------- lifecycle
+    def build(self, nbytes: int) -> bool:
+        """Collectively allocate every rank's window (``nbytes`` each) and map
+        the peers' windows. Returns whether every rank succeeded."""
+        rec, ok = None, True
+        try:
+            rec = self.native.create(self.rank, self.world, int(nbytes))
+        except (A2AError, RuntimeError):
+            ok = False
+        recs = self._gather(rec if ok else None)
+        if any(r is None for r in recs):
+            self._release_after_failure()
+            return False
+        try:
+            self.native.open(recs)
+        except A2AError:
+            ok = False
+        if not self._agree(ok):
+            # every rank unmaps and waits for the others before freeing
+            self._teardown_mapped()
+            return False
+        self._nbytes = int(nbytes)
+        self._armed = True
+        return True
+
+    def _release_after_failure(self) -> None:
+        try:
+            self.native.release()
+        except A2AError:
+            pass
+        self._nbytes = 0
+        self._armed = False
+
+    def _teardown_mapped(self) -> bool:
+        ok = True
+        try:
+            self.native.unmap()
+        except A2AError:
+            ok = False
+        dist.barrier(group=self.group)          # no peer maps our window any more
+        try:
+            self.native.release()
+        except A2AError:
+            ok = False
+        self._nbytes = 0
+        self._armed = False
+        return ok
+
+    def close(self) -> bool:
+        """Collective teardown of the windows; returns whether every rank completed it."""
+        all_armed = self._agree(self._armed)
+        all_unarmed = self._agree(not self._armed)
+        if all_unarmed:
+            return True
+        if not all_armed:
+            self._release_after_failure()
+            self._disable("ranks disagreed on whether a window was built during teardown")
+            return False
+        sync_ok = True
+        try:
+            self.native.synchronize()
+        except RuntimeError:
+            sync_ok = False
+        if not self._agree(sync_ok):
+            self._disable("a peer rank could not synchronize before window teardown")
+            return False
+        return self._agree(self._teardown_mapped())
+
+    def shutdown(self) -> None:
+        """close() and release the library context (collective)."""
+        self.close()
+        self.native.close()
+
+    # -------------------------------------------------------------------- the op
+    def all_to_all_4d(self, x: torch.Tensor, mode: int, chunked: bool = False, out=None,
+                      stream=None) -> torch.Tensor:
+        """Exchange this rank's slab ``x``; returns this rank's output slab.
+
+        mode 0: ``x`` is [B, S_local, H, D] (contiguous, or a row-pitched view
+        such as q of a packed [B, S, 3, H, D] buffer) -> [B, S_local*w, H//w, D].
+        mode 1: ``x`` is [B, S_local*w, H//w, D] -> [B, S_local, H, D] (``out``
+        may be a row-pitched view). Every rank calls it with the same shape,
+        mode and chunking.
+        """
+        if self.disabled_reason is not None:
+            raise RuntimeError(f"peer exchange disabled: {self.disabled_reason}")
+        if mode not in (0, 1):
+            raise ValueError("mode must be 0 or 1")
+        if x.dim() != 4 or x.device != self.device or x.element_size() != self.elem_bytes:
+            raise ValueError(f"x must be a 4D tensor of {self.elem_bytes}-byte elements on "
+                             f"{self.device}")
+        w = self.world
+        if (mode == 0 and x.shape[2] % w) or (mode == 1 and x.shape[1] % w):
+            raise ValueError("H (mode 0) or S_global (mode 1) must be divisible by the world size")
+        B, S, H, D = mode0_local_tuple(tuple(x.shape), mode, w)
+        oshape = output_shape(tuple(x.shape), mode, w)
+        if out is None:
+            out = torch.empty(oshape, dtype=x.dtype, device=x.device)
+        elif tuple(out.shape) != oshape or out.dtype != x.dtype or out.device != x.device:
+            raise ValueError(f"out must be {oshape} {x.dtype} on {x.device}")
+        strided, dense = (x, out) if mode == 0 else (out, x)
+        pitch = UlyssesA2A._row_pitch([strided], allow_pitch=True)
+        if not dense.is_contiguous():
+            raise ValueError("the [B, S_local*w, H/w, D] slab must be contiguous")
+        if B * S * H * D == 0:
+            return out
+        planes = B if chunked else 1
+        need = (1 if chunked else B) * S * H * D * self.elem_bytes
+        sig = (mode, bool(chunked), B, S, H, D, x.dtype)
+        if sig not in self._agreed:
+            sigs = self._gather(sig)
+            if any(s != sig for s in sigs):
+                raise ValueError(f"ranks called the exchange with different arguments: {sigs}")
+            self._agreed.add(sig)
+        if need > self._nbytes:
+            if self._armed and not self.close():
+                raise RuntimeError("window teardown before growing failed")
+            if not self.build(need):
+                self._disable("a rank could not build its window")
+                raise RuntimeError("peer exchange: window build failed on some rank")
+        if stream is None:
+            stream = self.native.current_stream()
+        nb = 1 if chunked else B
+        for b in range(planes):
+            xv = x[b:b + 1] if chunked else x
+            ov = out[b:b + 1] if chunked else out
+            self._barrier(stream)    # every rank is done reading the windows
+            self.native.publish(xv, nb, S, H, D, mode, pitch if mode == 0 else 0, stream)
+            self._barrier(stream)    # every window holds this plane
+            self.native.pull(ov, nb, S, H, D, mode, pitch if mode == 1 else 0, stream)
+        return out

@@ -1,0 +1,208 @@
+"""Host logic of PeerExchange on CPU: gloo, world size 2, no GPU.
+
+The native peer object is replaced by a stand-in whose windows are POSIX
+shared memory and whose pull assembles the rank's output from the other
+process's window with tensor slicing. What is under test is the sequencing
+that PeerExchange owns: the record exchange, the barrier before every publish
+and before every pull, window growth (collective close + rebuild), the
+agreement on call signatures, and collective teardown. Delays make a missing
+barrier visible. Rank 1 publishes late, so rank 0, pulling without the
+barrier before the pull, would read rank 1's window before it is written; rank
+1 also pulls late, so rank 0, publishing its next call without the barrier
+before the publish, would overwrite its window while rank 1 still reads it.
+Expected values come from the oracle.
+"""
+
+import os
+import time
+from datetime import timedelta
+from multiprocessing import shared_memory
+
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+class _HostStream:
+    def synchronize(self):
+        pass
+
+
+class ShmNative:
+    """Stand-in for sequence_all_re_b200.peer.NativePeer with host windows."""
+
+    def __init__(self, rank, publish_delay=0.0, pull_delay=0.0, fail_create=False):
+        self.device = torch.device("cpu")
+        self.elem_bytes = 2
+        self.rank = rank
+        self.world = None
+        self.own = None
+        self.peers = {}
+        self.log = []
+        self.publish_delay = publish_delay
+        self.pull_delay = pull_delay
+        self.fail_create = fail_create
+        self.launch_count = 0
+
+    def create(self, rank, world, nbytes):
+        if self.fail_create:
+            raise RuntimeError("window allocation failed (injected)")
+        self.world = world
+        self.own = shared_memory.SharedMemory(create=True, size=nbytes)
+        self.log.append(("create", nbytes))
+        return self.own.name
+
+    def open(self, records):
+        for k, name in enumerate(records):
+            if k != self.rank:
+                self.peers[k] = shared_memory.SharedMemory(name=name)
+        self.log.append(("open",))
+
+    def _win(self, k, dtype, shape):
+        shm = self.own if k == self.rank else self.peers[k]
+        n = 1
+        for v in shape:
+            n *= v
+        return torch.frombuffer(shm.buf, dtype=dtype, count=n).view(shape)
+
+    def publish(self, x, B, S, H, D, mode, row_pitch, stream):
+        time.sleep(self.publish_delay)
+        w = self.world
+        shape = (B, S, H, D) if mode == 0 else (B, S * w, H // w, D)
+        self._win(self.rank, x.dtype, shape).copy_(x)
+        self.log.append("publish")
+
+    def pull(self, out, B, S, H, D, mode, row_pitch, stream):
+        time.sleep(self.pull_delay)
+        w, k = self.world, self.rank
+        Hw = H // w
+        if mode == 0:
+            o = out.view(B, w, S, Hw, D)
+            for j in range(w):
+                o[:, j] = self._win(j, out.dtype, (B, S, H, D))[:, :, k * Hw:(k + 1) * Hw]
+        else:
+            for r in range(w):
+                out[:, :, r * Hw:(r + 1) * Hw] = self._win(r, out.dtype,
+                                                           (B, S * w, Hw, D))[:, k * S:(k + 1) * S]
+        self.log.append("pull")
+
+    def unmap(self):
+        for shm in self.peers.values():
+            shm.close()
+        self.peers.clear()
+        self.log.append(("unmap",))
+
+    def release(self):
+        if self.own is not None:
+            self.own.close()
+            self.own.unlink()
+            self.own = None
+            self.log.append(("release",))
+
+    def current_stream(self):
+        return _HostStream()
+
+    def synchronize(self):
+        pass
+
+    def close(self):
+        self.release()
+
+
+def _worker(rank, world, port, scenario, q):
+    import oracle
+    from sequence_all_re_b200.peer import PeerExchange
+    from synth import normal_slabs, uniform_slabs
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    rep = {"rank": rank, "ok": [], "errors": []}
+    try:
+        if scenario == "exchange":
+            # rank 0 never waits; rank 1 publishes late and pulls late
+            native = ShmNative(rank, publish_delay=0.05 if rank == 1 else 0.0,
+                               pull_delay=0.2 if rank == 1 else 0.0)
+            ex = PeerExchange(native=native, elem_bytes=2)
+            calls = [((2, 5, 4, 8), 0, False, normal_slabs),
+                     ((2, 5, 4, 8), 0, False, uniform_slabs),   # same size: windows reused
+                     ((2, 5, 4, 8), 1, True, normal_slabs),
+                     ((1, 16, 8, 8), 0, False, uniform_slabs)]  # larger: grow
+            for shape, mode, chunked, gen in calls:
+                xs = gen(shape, world, "bf16")
+                if mode == 0:
+                    x, want = xs[rank], oracle.ulysses_a2a(xs, 0)[rank]
+                else:
+                    x, want = oracle.ulysses_a2a(xs, 0)[rank], xs[rank]
+                got = ex.all_to_all_4d(x, mode, chunked=chunked)
+                rep["ok"].append(torch.equal(got.view(torch.int16), want.view(torch.int16)))
+            rep["closed"] = ex.close()
+            rep["log"] = native.log
+        elif scenario == "fail_build":
+            native = ShmNative(rank, fail_create=(rank == 1))
+            ex = PeerExchange(native=native, elem_bytes=2)
+            try:
+                ex.all_to_all_4d(torch.zeros(1, 4, 2, 8, dtype=torch.bfloat16), 0)
+            except RuntimeError as e:
+                rep["errors"].append(str(e))
+            rep["disabled"] = ex.disabled_reason
+            rep["closed"] = ex.close()
+            rep["log"] = native.log
+        elif scenario == "mismatch":
+            ex = PeerExchange(native=ShmNative(rank), elem_bytes=2)
+            S = 4 if rank == 0 else 6
+            try:
+                ex.all_to_all_4d(torch.zeros(1, S, 2, 8, dtype=torch.bfloat16), 0)
+            except ValueError as e:
+                rep["errors"].append(str(e))
+            rep["closed"] = ex.close()
+    except Exception as e:
+        rep["errors"].append("unexpected: " + repr(e))
+    finally:
+        q.put(rep)
+        dist.destroy_process_group()
+
+
+def _run(scenario, port_offset):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 32000 + port_offset + os.getpid() % 500
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, scenario, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    reps = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    return sorted(reps, key=lambda r: r["rank"])
+
+
+def test_exchange_sequence_barriers_and_growth():
+    for rep in _run("exchange", 0):
+        assert rep["errors"] == [], rep
+        assert rep["ok"] == [True] * 4, rep
+        assert rep["closed"] is True
+        log = rep["log"]
+        creates = [e[1] for e in log if isinstance(e, tuple) and e[0] == "create"]
+        # 2*5*4*8*2 bytes for the first three calls (one plane when chunked fits),
+        # then the larger slab after a collective close
+        assert creates == [2 * 5 * 4 * 8 * 2, 16 * 8 * 8 * 2]
+        ops = [e for e in log if isinstance(e, str)]
+        # one publish + one pull per exchange, per plane when chunked
+        assert ops == ["publish", "pull"] * (1 + 1 + 2 + 1)
+        assert log.index(("unmap",)) < log.index(("release",))
+
+
+def test_failed_window_build_disables_every_rank():
+    reps = _run("fail_build", 100)
+    for rep in reps:
+        assert len(rep["errors"]) == 1 and "window build failed" in rep["errors"][0], rep
+        assert rep["disabled"] is not None
+        assert rep["closed"] is True             # nothing left armed anywhere
+    # the rank whose allocation worked released its window again
+    assert ("release",) in reps[0]["log"]
+
+
+def test_ranks_with_different_arguments_all_raise():
+    for rep in _run("mismatch", 200):
+        assert len(rep["errors"]) == 1 and "different arguments" in rep["errors"][0], rep
+        assert rep["closed"] is True
