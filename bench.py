@@ -103,34 +103,38 @@ def _code_only(text: str) -> str:
     return " ".join(text.split())
 
 
-KERNEL_FILES = ("kernels_tma.cuh", "kernels_vec.cuh")
+KERNEL_FILES = {"tma": "kernels_tma.cuh", "vec": "kernels_vec.cuh"}
 LAUNCH_FIELDS = ("path", "rows_per_tile", "producers", "stages", "lookahead", "chunk_units",
                  "order", "grid", "block", "smem_bytes", "vec_bytes")
 
 
-def kernel_source_hash():
-    """Hash of the kernels' device code (comments and layout ignored): ncu
-    counters taken on one hash stay valid until that code changes."""
+def kernel_source_hash(path):
+    """Hash of one kernel file's device code (comments and layout ignored):
+    ncu counters taken on one hash stay valid until that code changes."""
+    name = KERNEL_FILES[path]
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "sequence_all_re_b200", "csrc")
-    for name in KERNEL_FILES:
-        with open(os.path.join(csrc, name), encoding="utf-8") as f:
-            h.update(name.encode())
-            h.update(_code_only(f.read()).encode())
+    with open(os.path.join(ROOT, "sequence_all_re_b200", "csrc", name), encoding="utf-8") as f:
+        h.update(name.encode())
+        h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_hash):
-    """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+def ncu_traffic(key, plan, chunked):
+    """DRAM bytes per launch from the committed ncu summary, while the capture
+    matches this kernel's code and this launch shape; else (None, why)."""
     try:
-        with open(path) as f:
-            d = json.load(f)
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            entry = json.load(f).get("workloads", {}).get(key)
     except Exception:
         return None, "no ncu traffic summary"
-    if d.get("kernel_source_hash") != kernel_hash:
+    if not entry:
+        return None, "no ncu capture of this kernel and workload"
+    if entry.get("kernel_hash") != kernel_source_hash(key.split(":")[0]):
         return None, "kernel changed since the ncu counters were taken"
-    return d, "ncu"
+    launch = entry.get("launch", {})
+    if chunked or any(launch.get(f) != plan[f] for f in LAUNCH_FIELDS):
+        return None, "the capture was taken with another launch shape"
+    return entry.get("dram_bytes_per_launch"), "ncu"
 
 
 class ClockSampler:
@@ -411,19 +415,8 @@ def run_ours(args):
     avg_launch_ms = total_ms / launches
     bytes_per_launch = 2 * P * 2 * args.steps // launches       # 2 calls of 2P per step
     achieved = bytes_per_launch / (avg_launch_ms / 1e3) / 1e9
-    khash = kernel_source_hash()
-    traffic, traffic_src = ncu_traffic(khash)
-    traffic_bytes = None
-    if traffic:
-        key = workload_key(w, B, S, H, D, {1: "tma", 2: "vec"}[plan["path"]])
-        entry = traffic.get("workloads", {}).get(key, {})
-        launch = entry.get("launch", {})
-        if not entry:
-            traffic_src = "no ncu capture of this kernel and workload"
-        elif chunked or any(launch.get(f) != plan[f] for f in LAUNCH_FIELDS):
-            traffic_src = "the capture was taken with another launch shape"
-        else:
-            traffic_bytes = entry.get("dram_bytes_per_launch")
+    key = workload_key(w, B, S, H, D, {1: "tma", 2: "vec"}[plan["path"]])
+    traffic_bytes, traffic_src = ncu_traffic(key, plan, chunked)
 
     # per mode: back to back, and call by call after an L2 write flush
     reps = max(20, min(args.steps, 400))
