@@ -547,6 +547,124 @@ def run_ours(args):
 
 
 # ---------------------------------------------------------------- reference arm
+def run_peer_one_gpu(args):
+    """The multi-GPU exchange's kernels with the w ranks as contexts on one GPU.
+
+    Each step is, for mode 0 and then mode 1: every rank publishes its slab into
+    its window, then every rank pulls its output slab from all windows (stream
+    order stands in for the barriers). On one GPU the pulls' "peer" loads are
+    local, so this times the two kernels against HBM, not NVLink.
+    """
+    from sequence_all_re_b200 import UlyssesA2A, _lib
+
+    if args.gpus != 1:
+        raise SystemExit("--peer-one-gpu runs on one GPU")
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    wl = WORKLOADS[args.workload]
+    w, B, S, H, D = (wl[k] for k in ("w", "B", "S_local", "H", "D"))
+    E = 2
+    slab = B * S * H * D * E
+    P = w * slab
+    ctxs = [UlyssesA2A(0, E) for _ in range(w)]
+    peers, recs = [], []
+    for k in range(w):
+        rc, h, rec = _lib.ulysses_a2a_peer_create(ctxs[k]._ctx, k, w, slab)
+        if rc != _lib.OK:
+            raise SystemExit("peer_create: " + ctxs[k].last_error())
+        peers.append(h)
+        recs.append(rec)
+    for k in range(w):
+        if _lib.ulysses_a2a_peer_open(peers[k], recs) != _lib.OK:
+            raise SystemExit("peer_open: " + ctxs[k].last_error())
+    x = make_inputs(w, B, S, H, D, "bf16", device)
+    y = [torch.empty((B, S * w, H // w, D), dtype=torch.bfloat16, device=device) for _ in range(w)]
+    z = [torch.empty_like(t) for t in x]
+    stream = torch.cuda.Stream(device)
+    st = stream.cuda_stream
+
+    def publish(src, mode):
+        for k in range(w):
+            if _lib.ulysses_a2a_peer_publish(peers[k], src[k].data_ptr(), B, S, H, D, mode, 0,
+                                             st) != _lib.OK:
+                raise SystemExit("peer_publish: " + ctxs[k].last_error())
+
+    def pull(dst, mode):
+        for k in range(w):
+            if _lib.ulysses_a2a_peer_pull(peers[k], dst[k].data_ptr(), B, S, H, D, mode, 0,
+                                          st) != _lib.OK:
+                raise SystemExit("peer_pull: " + ctxs[k].last_error())
+
+    def step():
+        publish(x, 0)
+        pull(y, 0)
+        publish(y, 1)
+        pull(z, 1)
+
+    def timed(fn, reps):
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                fn()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b.record(stream)
+            b.synchronize()
+        return a.elapsed_time(b) / reps
+
+    steps = min(args.steps, 500)
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.synchronize()
+    if not all(torch.equal(z[k], x[k]) for k in range(w)):
+        raise SystemExit("round trip mismatch through the peer windows")
+    n0 = sum(c.launch_count for c in ctxs)
+    sampler = ClockSampler(0)
+    sampler.start()
+    ms_step = timed(step, steps)
+    clocks = sampler.stop()
+    launches = sum(c.launch_count for c in ctxs) - n0
+    ms_pub = timed(lambda: publish(x, 0), steps)
+    ms_pull0 = timed(lambda: pull(y, 0), steps)
+    ms_pull1 = timed(lambda: pull(z, 1), steps)
+    peak, peak_src = hbm_peak()
+
+    def roof(ms_group):
+        # w launches per group, each reading and writing one slab
+        us = ms_group * 1e3 / w
+        ach = 2 * slab / (us / 1e6) / 1e9
+        return {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(ach / peak, 4), "avg_launch_us": round(us, 3),
+                "algorithmic_bytes_per_launch": 2 * slab}
+
+    line = {
+        "metric": "Ulysses all-to-all payload throughput through the peer-window exchange "
+                  "(w ranks as contexts on one GPU)",
+        "value": round(2 * P / (ms_step / 1e3) / 1e9, 1), "unit": "GB/s", "n_gpus": 1,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_name(w, B, S, H, D, 0) + "; publish + pull per rank",
+                   "l2": "inputs larger than L2 (back to back)"},
+        "gpu_launches": launches,
+        "kernels": {"publish (one-rank re-layout into the own window)": roof(ms_pub),
+                    "pull mode 0 (VEC, one output slab)": roof(ms_pull0),
+                    "pull mode 1 (VEC, one output slab)": roof(ms_pull1)},
+        "peak_source": peak_src,
+        "clocks": clocks,
+        "note": "each step moves every byte twice (publish + pull) per mode; value counts "
+                "the payload 2P once per mode, as the main bench line does",
+    }
+    for h in peers:
+        _lib.ulysses_a2a_peer_close(h)
+    for h in peers:
+        _lib.ulysses_a2a_peer_destroy(h)
+    for c in ctxs:
+        c.close()
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args):
     rank, _, world = env_rank()
     if rank != 0:
@@ -624,12 +742,17 @@ def main():
     ap.add_argument("--chunked", type=int, choices=[0, 1, 2], default=0)
     ap.add_argument("--sweep", action="store_true",
                     help="also run the 128 KiB..2 GiB bandwidth sweep (w=2/4/8, bf16/fp32)")
+    ap.add_argument("--peer-one-gpu", action="store_true",
+                    help="time the multi-GPU exchange's publish and pull kernels with the w "
+                         "ranks as contexts on one GPU (prints its own line)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("note: warm-up raised to 3 steps", file=sys.stderr)
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.peer_one_gpu:
+        run_peer_one_gpu(args)
     else:
         run_ours(args)
 

@@ -81,8 +81,13 @@ __device__ __forceinline__ void st_stream(unsigned int* p, unsigned int v) { __s
 __device__ __forceinline__ void st_stream(unsigned short* p, unsigned short v) { __stcs(p, v); }
 __device__ __forceinline__ void st_stream(unsigned char* p, unsigned char v) { __stcs(p, v); }
 
+// 256-thread CTAs, at least 6 resident per SM: caps the kernel at 40
+// registers, so every variant runs at 75% occupancy.
+constexpr int kVecMinBlocksPerSm = 6;
+
 template <typename V, int MODE, int U>
-__global__ void __launch_bounds__(256) ua2a_vec_kernel(const __grid_constant__ VecParams p) {
+__global__ void __launch_bounds__(256, kVecMinBlocksPerSm)
+    ua2a_vec_kernel(const __grid_constant__ VecParams p) {
 #if UA2A_PDL
   // programmatic dependent launch: start the next grid's launch, then wait for
   // the previous one to finish before touching global memory

@@ -42,6 +42,12 @@ constexpr int kTmaDefaultCtasPerSm = 1;
 constexpr int kTmaMaxBoxDim = 256;
 constexpr int kVecBlock = 256;
 constexpr int kVecDefaultCtasPerSm = 16;
+// CTAs of the VEC kernel resident per SM (its launch bound). A launch with
+// fewer than kVecMinWaves waves of units gets smaller units, kVecTargetWaves
+// waves' worth, so the last wave does not leave most SMs idle.
+constexpr int kVecResidentCtasPerSm = 6;
+constexpr int kVecMinWaves = 3;
+constexpr int kVecTargetWaves = 4;
 // Unit numbering: 0 = destination rank outermost, 1 = innermost.
 constexpr int kDefaultOrder = 1;
 // Host-buffer entry point: sequence chunks its H2D copies, kernels and D2H
@@ -265,7 +271,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
   }
   if (rows > S) rows = S;
 
-  const int64_t T = (S + rows - 1) / rows;  // ceil-div: the ragged last tile is a unit too
+  int64_t T = (S + rows - 1) / rows;  // ceil-div: the ragged last tile is a unit too
   const int64_t nb = chunked ? 1 : B;
   const int64_t blocks_wide = only_out >= 0 ? (int64_t)w : (int64_t)w * w;
   int64_t units;
@@ -347,6 +353,23 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     }
   }
   if (path == ULYSSES_A2A_PATH_VEC) {
+    if (tune.rows_per_tile <= 0) {
+      const int64_t slots = (int64_t)num_sms * kVecResidentCtasPerSm;
+      if (units < kVecMinWaves * slots) {
+        const int64_t blocks = units / T;       // (r, b, j) blocks in this launch
+        int64_t r2 = blocks * S / (kVecTargetWaves * slots);
+        if (r2 < 1) r2 = 1;
+        if (r2 < rows) {
+          rows = r2;
+          T = (S + rows - 1) / rows;
+          units = blocks * T;
+          p->rows_per_tile = rows;
+          p->tiles_per_block = T;
+          p->tail_rows = S % rows;
+          p->units = units;
+        }
+      }
+    }
     int v = 16;
     while (v > 1) {
       bool ok = (row_bytes % v) == 0 && ((pitch * E) % v) == 0;

@@ -47,6 +47,9 @@
 using ua2a::TmaParams;
 using ua2a::VecParams;
 
+static_assert(ua2a::kVecResidentCtasPerSm == ua2a::kVecMinBlocksPerSm,
+              "the planner's VEC residency must match the kernel's launch bound");
+
 namespace {
 
 constexpr int kTmaCacheEntries = 16;

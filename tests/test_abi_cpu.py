@@ -160,9 +160,25 @@ def test_vec_when_box_dim_too_large():
 def test_forced_vec_geometry():
     rc, p, _ = plan(4, 1, 8192, 24, 128, forced_path=PATH_VEC)
     assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 16
-    assert p.rows_per_tile == 64 * 1024 // 1536
+    # 16 blocks x 196 tiles = 3136 units: more than 3 waves of 148 x 6 resident CTAs
+    assert p.rows_per_tile == 64 * 1024 // 1536 == 42 and p.units == 3136
     assert p.block == 256 and p.grid == min(p.units, 148 * 16)
     assert p.producers == 0 and p.lookahead == 0
+
+
+def test_vec_units_shrink_below_three_waves():
+    # w=2: 64 KB units would be 4 blocks x 391 tiles = 1564 units, under 3 waves of
+    # 888 resident CTAs; the planner takes 4 waves' worth: 4 * 8192 // 3552 = 9 rows
+    rc, p, _ = plan(2, 1, 8192, 24, 128, forced_path=PATH_VEC)
+    assert rc == OK and p.rows_per_tile == 9 and p.tiles_per_block == -(-8192 // 9)
+    assert p.units == 4 * p.tiles_per_block == 3644 and p.tail_rows == 8192 % 9
+    assert p.grid == 148 * 16
+    # an explicit tile size is kept as given
+    rc, p, _ = plan(2, 1, 8192, 24, 128, forced_path=PATH_VEC, rows_per_tile=21)
+    assert rc == OK and p.rows_per_tile == 21 and p.units == 4 * 391
+    # a tiny problem goes down to one row per unit
+    rc, p, _ = plan(2, 1, 64, 4, 64, forced_path=PATH_VEC)
+    assert rc == OK and p.rows_per_tile == 1 and p.units == 4 * 64
 
 
 def test_tuning_knobs():
