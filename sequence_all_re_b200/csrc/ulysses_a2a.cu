@@ -860,10 +860,14 @@ uint64_t process_nonce() {
   static std::once_flag once;
   static uint64_t nonce = 0;
   std::call_once(once, [] {
-    std::random_device rd;
-    uint64_t v = ((uint64_t)rd() << 32) ^ (uint64_t)rd();
-    v ^= (uint64_t)std::chrono::steady_clock::now().time_since_epoch().count();
+    uint64_t v = (uint64_t)std::chrono::steady_clock::now().time_since_epoch().count();
     v ^= (uint64_t)getpid() << 17;
+    v ^= (uint64_t)(uintptr_t)&nonce;
+    try {  // no exception may leave the C ABI
+      std::random_device rd;
+      v ^= ((uint64_t)rd() << 32) ^ (uint64_t)rd();
+    } catch (...) {
+    }
     nonce = v ? v : 1;
   });
   return nonce;

@@ -1,7 +1,8 @@
 /*
  * Plain-C user of libulysses_a2a.so (no Python, no torch): allocates rank
  * slabs with cudaMalloc, runs both modes through ulysses_a2a_run, runs the
- * host-buffer entry point, checks the error codes of a few rejected calls, and
+ * host-buffer entry point, checks the error codes of a few rejected calls, runs
+ * the multi-GPU exchange entry points with its ranks in this process, and
  * compares every output byte with the CPU oracle (libulysses_oracle.so, test
  * infrastructure). Exit status 0 = all checks passed.
  */
@@ -81,6 +82,44 @@ int main(void) {
               ULYSSES_A2A_ERR_DEVICE, "host pointer accepted as device memory");
     CHECK(ulysses_a2a_launch_count(ctx) == launches, "a rejected call launched work");
     CHECK(strlen(ulysses_a2a_last_error(ctx)) > 0, "no error message");
+
+    /* the multi-GPU exchange with its W ranks in this process: one context and
+       window per rank, records handed over in memory; every publish, then every
+       pull, on the default stream (stream order stands in for the barriers) */
+    {
+        ulysses_a2a_ctx *rctx[W];
+        ulysses_a2a_peer *peer[W];
+        unsigned char rec[W][ULYSSES_A2A_PEER_HANDLE_BYTES];
+        for (int k = 0; k < W; ++k) {
+            CHECK(ulysses_a2a_create(&rctx[k], 0, E) == ULYSSES_A2A_OK, "create (rank)");
+            CHECK(ulysses_a2a_peer_create(rctx[k], k, W, bytes, &peer[k], rec[k]) ==
+                      ULYSSES_A2A_OK, ulysses_a2a_last_error(rctx[k]));
+        }
+        for (int k = 0; k < W; ++k)
+            CHECK(ulysses_a2a_peer_open(peer[k], rec) == ULYSSES_A2A_OK,
+                  ulysses_a2a_last_error(rctx[k]));
+        CHECK(ulysses_a2a_peer_window_bytes(peer[0]) == bytes, "window size");
+        for (int k = 0; k < W; ++k) {
+            CHECK(cudaMemcpy(din[k], hin[k], bytes, cudaMemcpyHostToDevice) == cudaSuccess, "H2D");
+            CHECK(cudaMemset(dout[k], 0xFF, bytes) == cudaSuccess, "poison");
+        }
+        for (int k = 0; k < W; ++k)
+            CHECK(ulysses_a2a_peer_publish(peer[k], din[k], B, S, H, D, 0, 0, NULL) ==
+                      ULYSSES_A2A_OK, ulysses_a2a_last_error(rctx[k]));
+        for (int k = 0; k < W; ++k)
+            CHECK(ulysses_a2a_peer_pull(peer[k], dout[k], B, S, H, D, 0, 0, NULL) ==
+                      ULYSSES_A2A_OK, ulysses_a2a_last_error(rctx[k]));
+        for (int k = 0; k < W; ++k) {
+            CHECK(cudaMemcpy(hout[k], dout[k], bytes, cudaMemcpyDeviceToHost) == cudaSuccess, "D2H");
+            CHECK(memcmp(hout[k], want[k], bytes) == 0, "peer exchange differs from the oracle");
+        }
+        for (int k = 0; k < W; ++k) CHECK(ulysses_a2a_peer_close(peer[k]) == ULYSSES_A2A_OK, "close");
+        for (int k = 0; k < W; ++k) {
+            CHECK(ulysses_a2a_peer_destroy(peer[k]) == ULYSSES_A2A_OK, "peer destroy");
+            CHECK(ulysses_a2a_destroy(rctx[k]) == ULYSSES_A2A_OK, "destroy (rank)");
+        }
+        CHECK(ulysses_a2a_peer_destroy(NULL) == ULYSSES_A2A_OK, "peer destroy(NULL)");
+    }
 
     CHECK(ulysses_a2a_destroy(ctx) == ULYSSES_A2A_OK, "destroy");
     CHECK(ulysses_a2a_destroy(NULL) == ULYSSES_A2A_OK, "destroy(NULL)");
