@@ -64,6 +64,9 @@ extern "C" {
 #define ULYSSES_A2A_ERR_UNSUPPORTED 5  /* forced path cannot express the shape  */
 #define ULYSSES_A2A_ERR_NOMEM       6  /* host or device allocation failed      */
 #define ULYSSES_A2A_ERR_TIMEOUT     7  /* a kernel's bounded wait gave up       */
+#define ULYSSES_A2A_ERR_INTERNAL    8  /* an unexpected host-side failure inside
+                                          the library (no exception ever leaves
+                                          an entry point)                       */
 
 /* ---- copy paths ------------------------------------------------------- */
 #define ULYSSES_A2A_PATH_AUTO 0  /* TMA when the shape allows it, else VEC     */

@@ -21,6 +21,7 @@ ERR_CUDA = 4
 ERR_UNSUPPORTED = 5
 ERR_NOMEM = 6
 ERR_TIMEOUT = 7
+ERR_INTERNAL = 8
 
 PATH_AUTO = 0
 PATH_TMA = 1

@@ -400,7 +400,7 @@ int plan_for(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, int6
 
 extern "C" {
 
-int ulysses_a2a_create(ulysses_a2a_ctx** out, int device, int elem_bytes) {
+static int ua2a_impl_create(ulysses_a2a_ctx** out, int device, int elem_bytes) {
   if (out == nullptr) return ULYSSES_A2A_ERR_INVALID;
   *out = nullptr;
   if (!(elem_bytes == 1 || elem_bytes == 2 || elem_bytes == 4 || elem_bytes == 8))
@@ -453,7 +453,7 @@ int ulysses_a2a_create(ulysses_a2a_ctx** out, int device, int elem_bytes) {
   return ULYSSES_A2A_OK;
 }
 
-int ulysses_a2a_destroy(ulysses_a2a_ctx* ctx) {
+static int ua2a_impl_destroy(ulysses_a2a_ctx* ctx) {
   if (ctx == nullptr) return ULYSSES_A2A_OK;
   int rc = ULYSSES_A2A_OK;
   {
@@ -538,7 +538,7 @@ int run_windowed(ulysses_a2a_ctx* ctx, const ulysses_a2a_desc_t* d, const ulysse
 
 }  // namespace
 
-int ulysses_a2a_run_ex(ulysses_a2a_ctx* ctx, const ulysses_a2a_desc_t* d, void* stream) {
+static int ua2a_impl_run_ex(ulysses_a2a_ctx* ctx, const ulysses_a2a_desc_t* d, void* stream) {
   if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
   ctx->last_error.clear();
   if (d == nullptr) return fail(ctx, ULYSSES_A2A_ERR_INVALID, "descriptor is NULL");
@@ -565,7 +565,7 @@ int ulysses_a2a_run_ex(ulysses_a2a_ctx* ctx, const ulysses_a2a_desc_t* d, void* 
                     d->chunked, static_cast<cudaStream_t>(stream), pl);
 }
 
-int ulysses_a2a_run(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void* const* out_slabs,
+static int ua2a_impl_run(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void* const* out_slabs,
                     int64_t B, int64_t S_local, int64_t H, int64_t D, int w, int mode, int chunked,
                     void* stream) {
   ulysses_a2a_desc_t d{};
@@ -582,7 +582,7 @@ int ulysses_a2a_run(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void* con
   return ulysses_a2a_run_ex(ctx, &d, stream);
 }
 
-int ulysses_a2a_run_host(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void* const* out_slabs,
+static int ua2a_impl_run_host(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void* const* out_slabs,
                          int64_t B, int64_t S_local, int64_t H, int64_t D, int w, int mode,
                          int chunked, void* stream) {
   if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
@@ -723,7 +723,7 @@ const char* ulysses_a2a_last_error(const ulysses_a2a_ctx* ctx) {
   return ctx->last_error.c_str();
 }
 
-int ulysses_a2a_status(ulysses_a2a_ctx* ctx, void* stream) {
+static int ua2a_impl_status(ulysses_a2a_ctx* ctx, void* stream) {
   if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
   DeviceGuard g(ctx->device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -743,7 +743,7 @@ int ulysses_a2a_status(ulysses_a2a_ctx* ctx, void* stream) {
   return fail(ctx, ULYSSES_A2A_ERR_TIMEOUT, buf);
 }
 
-int ulysses_a2a_selftest_wait_timeout(ulysses_a2a_ctx* ctx, uint32_t limit_us, void* stream) {
+static int ua2a_impl_selftest_wait_timeout(ulysses_a2a_ctx* ctx, uint32_t limit_us, void* stream) {
   if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
   if (limit_us < 1 || limit_us > 2000000)
     return fail(ctx, ULYSSES_A2A_ERR_INVALID, "limit_us must be in [1, 2000000]");
@@ -757,7 +757,7 @@ int ulysses_a2a_selftest_wait_timeout(ulysses_a2a_ctx* ctx, uint32_t limit_us, v
   return ULYSSES_A2A_OK;
 }
 
-int ulysses_a2a_set_path(ulysses_a2a_ctx* ctx, int path) {
+static int ua2a_impl_set_path(ulysses_a2a_ctx* ctx, int path) {
   if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
   if (path < ULYSSES_A2A_PATH_AUTO || path > ULYSSES_A2A_PATH_VEC)
     return fail(ctx, ULYSSES_A2A_ERR_INVALID, "unknown path");
@@ -765,7 +765,7 @@ int ulysses_a2a_set_path(ulysses_a2a_ctx* ctx, int path) {
   return ULYSSES_A2A_OK;
 }
 
-int ulysses_a2a_set_tuning(ulysses_a2a_ctx* ctx, const ulysses_a2a_tuning_t* t) {
+static int ua2a_impl_set_tuning(ulysses_a2a_ctx* ctx, const ulysses_a2a_tuning_t* t) {
   if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
   ua2a::Tuning tu;
   std::string err;
@@ -778,7 +778,7 @@ uint64_t ulysses_a2a_launch_count(const ulysses_a2a_ctx* ctx) {
   return ctx ? ctx->launches : 0;
 }
 
-int ulysses_a2a_plan_ex(const ulysses_a2a_desc_t* d, int elem_bytes, int forced_path,
+static int ua2a_impl_plan_ex(const ulysses_a2a_desc_t* d, int elem_bytes, int forced_path,
                         const ulysses_a2a_tuning_t* tuning, int num_sms, ulysses_a2a_plan_t* out,
                         char* err, size_t errlen) {
   ua2a::Tuning t;
@@ -800,7 +800,7 @@ int ulysses_a2a_plan_ex(const ulysses_a2a_desc_t* d, int elem_bytes, int forced_
   return rc;
 }
 
-int ulysses_a2a_plan(const void* const* in_slabs, void* const* out_slabs, int64_t B,
+static int ua2a_impl_plan(const void* const* in_slabs, void* const* out_slabs, int64_t B,
                      int64_t S_local, int64_t H, int64_t D, int w, int mode, int chunked,
                      int elem_bytes, int forced_path, const ulysses_a2a_tuning_t* tuning,
                      int num_sms, ulysses_a2a_plan_t* out, char* err, size_t errlen) {
@@ -904,7 +904,7 @@ void peer_unmap(ulysses_a2a_peer* p, int* rc) {
 
 extern "C" {
 
-int ulysses_a2a_peer_create(ulysses_a2a_ctx* ctx, int rank, int world, size_t window_bytes,
+static int ua2a_impl_peer_create(ulysses_a2a_ctx* ctx, int rank, int world, size_t window_bytes,
                             ulysses_a2a_peer** out, void* handle_out) {
   if (out) *out = nullptr;
   if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
@@ -951,7 +951,7 @@ int ulysses_a2a_peer_create(ulysses_a2a_ctx* ctx, int rank, int world, size_t wi
   return ULYSSES_A2A_OK;
 }
 
-int ulysses_a2a_peer_open(ulysses_a2a_peer* p, const void* handles) {
+static int ua2a_impl_peer_open(ulysses_a2a_peer* p, const void* handles) {
   if (p == nullptr) return ULYSSES_A2A_ERR_INVALID;
   ulysses_a2a_ctx* ctx = p->ctx;
   ctx->last_error.clear();
@@ -1021,7 +1021,7 @@ int ulysses_a2a_peer_open(ulysses_a2a_peer* p, const void* handles) {
   return ULYSSES_A2A_OK;
 }
 
-int ulysses_a2a_peer_publish(ulysses_a2a_peer* p, const void* in_local, int64_t B, int64_t S_local,
+static int ua2a_impl_peer_publish(ulysses_a2a_peer* p, const void* in_local, int64_t B, int64_t S_local,
                              int64_t H, int64_t D, int mode, int64_t row_pitch, void* stream) {
   if (p == nullptr) return ULYSSES_A2A_ERR_INVALID;
   ulysses_a2a_ctx* ctx = p->ctx;
@@ -1055,7 +1055,7 @@ int ulysses_a2a_peer_publish(ulysses_a2a_peer* p, const void* in_local, int64_t 
   return run_device(ctx, in, out, B, S1, H1, D, 1, 0, 0, static_cast<cudaStream_t>(stream), pl);
 }
 
-int ulysses_a2a_peer_pull(ulysses_a2a_peer* p, void* out_local, int64_t B, int64_t S_local, int64_t H,
+static int ua2a_impl_peer_pull(ulysses_a2a_peer* p, void* out_local, int64_t B, int64_t S_local, int64_t H,
                           int64_t D, int mode, int64_t row_pitch, void* stream) {
   if (p == nullptr) return ULYSSES_A2A_ERR_INVALID;
   ulysses_a2a_ctx* ctx = p->ctx;
@@ -1097,7 +1097,7 @@ size_t ulysses_a2a_peer_window_bytes(const ulysses_a2a_peer* p) {
   return p ? p->window_bytes : 0;
 }
 
-int ulysses_a2a_peer_close(ulysses_a2a_peer* p) {
+static int ua2a_impl_peer_close(ulysses_a2a_peer* p) {
   if (p == nullptr) return ULYSSES_A2A_ERR_INVALID;
   if (!p->open) return ULYSSES_A2A_OK;
   int rc = ULYSSES_A2A_OK;
@@ -1110,7 +1110,7 @@ int ulysses_a2a_peer_close(ulysses_a2a_peer* p) {
   return rc;
 }
 
-int ulysses_a2a_peer_destroy(ulysses_a2a_peer* p) {
+static int ua2a_impl_peer_destroy(ulysses_a2a_peer* p) {
   if (p == nullptr) return ULYSSES_A2A_OK;
   int rc = ulysses_a2a_peer_close(p);
   {
@@ -1215,7 +1215,7 @@ bool noalloc_encode(CUtensorMap* m, int rank, const void* base, const cuuint64_t
 
 }  // namespace
 
-extern "C" int ulysses_a2a_run_noalloc(const void* const* in_slabs, void* const* out_slabs,
+static int ua2a_impl_run_noalloc(const void* const* in_slabs, void* const* out_slabs,
                                        int64_t B, int64_t S_local, int64_t H, int64_t D, int w,
                                        int mode, int chunked, int elem_bytes, void* stream,
                                        int wait, char* err, size_t errlen) {
@@ -1392,3 +1392,124 @@ extern "C" int ulysses_a2a_run_noalloc(const void* const* in_slabs, void* const*
   }
   return ULYSSES_A2A_OK;
 }
+
+// ---------------------------------------------------------------------------
+// The exported entry points: no exception may cross the C ABI. A failed host
+// allocation inside the library becomes ULYSSES_A2A_ERR_NOMEM, any other
+// exception ULYSSES_A2A_ERR_INTERNAL.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+template <typename F>
+int no_throw(F&& f) noexcept {
+  try {
+    return f();
+  } catch (const std::bad_alloc&) {
+    return ULYSSES_A2A_ERR_NOMEM;
+  } catch (...) {
+    return ULYSSES_A2A_ERR_INTERNAL;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int ulysses_a2a_create(ulysses_a2a_ctx** out, int device, int elem_bytes) {
+  return no_throw([&] { return ua2a_impl_create(out, device, elem_bytes); });
+}
+
+int ulysses_a2a_destroy(ulysses_a2a_ctx* ctx) {
+  return no_throw([&] { return ua2a_impl_destroy(ctx); });
+}
+
+int ulysses_a2a_run_ex(ulysses_a2a_ctx* ctx, const ulysses_a2a_desc_t* d, void* stream) {
+  return no_throw([&] { return ua2a_impl_run_ex(ctx, d, stream); });
+}
+
+int ulysses_a2a_run(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void* const* out_slabs,
+                    int64_t B, int64_t S_local, int64_t H, int64_t D, int w, int mode, int chunked,
+                    void* stream) {
+  return no_throw([&] { return ua2a_impl_run(ctx, in_slabs, out_slabs, B, S_local, H, D, w, mode,
+                                             chunked, stream); });
+}
+
+int ulysses_a2a_run_host(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void* const* out_slabs,
+                         int64_t B, int64_t S_local, int64_t H, int64_t D, int w, int mode,
+                         int chunked, void* stream) {
+  return no_throw([&] { return ua2a_impl_run_host(ctx, in_slabs, out_slabs, B, S_local, H, D, w,
+                                                  mode, chunked, stream); });
+}
+
+int ulysses_a2a_status(ulysses_a2a_ctx* ctx, void* stream) {
+  return no_throw([&] { return ua2a_impl_status(ctx, stream); });
+}
+
+int ulysses_a2a_selftest_wait_timeout(ulysses_a2a_ctx* ctx, uint32_t limit_us, void* stream) {
+  return no_throw([&] { return ua2a_impl_selftest_wait_timeout(ctx, limit_us, stream); });
+}
+
+int ulysses_a2a_set_path(ulysses_a2a_ctx* ctx, int path) {
+  return no_throw([&] { return ua2a_impl_set_path(ctx, path); });
+}
+
+int ulysses_a2a_set_tuning(ulysses_a2a_ctx* ctx, const ulysses_a2a_tuning_t* t) {
+  return no_throw([&] { return ua2a_impl_set_tuning(ctx, t); });
+}
+
+int ulysses_a2a_plan_ex(const ulysses_a2a_desc_t* d, int elem_bytes, int forced_path,
+                        const ulysses_a2a_tuning_t* tuning, int num_sms, ulysses_a2a_plan_t* out,
+                        char* err, size_t errlen) {
+  return no_throw([&] { return ua2a_impl_plan_ex(d, elem_bytes, forced_path, tuning, num_sms, out,
+                                                 err, errlen); });
+}
+
+int ulysses_a2a_plan(const void* const* in_slabs, void* const* out_slabs, int64_t B,
+                     int64_t S_local, int64_t H, int64_t D, int w, int mode, int chunked,
+                     int elem_bytes, int forced_path, const ulysses_a2a_tuning_t* tuning,
+                     int num_sms, ulysses_a2a_plan_t* out, char* err, size_t errlen) {
+  return no_throw([&] { return ua2a_impl_plan(in_slabs, out_slabs, B, S_local, H, D, w, mode,
+                                              chunked, elem_bytes, forced_path, tuning, num_sms,
+                                              out, err, errlen); });
+}
+
+int ulysses_a2a_peer_create(ulysses_a2a_ctx* ctx, int rank, int world, size_t window_bytes,
+                            ulysses_a2a_peer** out, void* handle_out) {
+  return no_throw([&] { return ua2a_impl_peer_create(ctx, rank, world, window_bytes, out,
+                                                     handle_out); });
+}
+
+int ulysses_a2a_peer_open(ulysses_a2a_peer* p, const void* handles) {
+  return no_throw([&] { return ua2a_impl_peer_open(p, handles); });
+}
+
+int ulysses_a2a_peer_publish(ulysses_a2a_peer* p, const void* in_local, int64_t B, int64_t S_local,
+                             int64_t H, int64_t D, int mode, int64_t row_pitch, void* stream) {
+  return no_throw([&] { return ua2a_impl_peer_publish(p, in_local, B, S_local, H, D, mode,
+                                                      row_pitch, stream); });
+}
+
+int ulysses_a2a_peer_pull(ulysses_a2a_peer* p, void* out_local, int64_t B, int64_t S_local,
+                          int64_t H, int64_t D, int mode, int64_t row_pitch, void* stream) {
+  return no_throw([&] { return ua2a_impl_peer_pull(p, out_local, B, S_local, H, D, mode, row_pitch,
+                                                   stream); });
+}
+
+int ulysses_a2a_peer_close(ulysses_a2a_peer* p) {
+  return no_throw([&] { return ua2a_impl_peer_close(p); });
+}
+
+int ulysses_a2a_peer_destroy(ulysses_a2a_peer* p) {
+  return no_throw([&] { return ua2a_impl_peer_destroy(p); });
+}
+
+int ulysses_a2a_run_noalloc(const void* const* in_slabs, void* const* out_slabs, int64_t B,
+                            int64_t S_local, int64_t H, int64_t D, int w, int mode, int chunked,
+                            int elem_bytes, void* stream, int wait, char* err, size_t errlen) {
+  return no_throw([&] { return ua2a_impl_run_noalloc(in_slabs, out_slabs, B, S_local, H, D, w, mode,
+                                                     chunked, elem_bytes, stream, wait, err,
+                                                     errlen); });
+}
+
+}  // extern "C"
