@@ -201,8 +201,9 @@ int ulysses_a2a_set_path(ulysses_a2a_ctx *ctx, int path);
  * left at its "default" value keeps the library's choice. */
 typedef struct ulysses_a2a_tuning_t {
     int32_t rows_per_tile;  /* S_tile cap, 1..256; 0 = default                */
-    int32_t ctas_per_sm;    /* persistent TMA grid / VEC grid: CTAs per SM,
-                               1..32; 0 = default                          */
+    int32_t ctas_per_sm;    /* persistent TMA grid / grid-stride VEC grid:
+                               CTAs per SM, 1..32; 0 = default (VEC: one
+                               CTA per unit)                              */
     int32_t stages;         /* TMA: shared-memory tiles per CTA, 1..32, split
                                evenly over the producers; 0 = default      */
     int32_t lookahead;      /* TMA: loads in flight per producer; 0 = default */

@@ -160,25 +160,24 @@ def test_vec_when_box_dim_too_large():
 def test_forced_vec_geometry():
     rc, p, _ = plan(4, 1, 8192, 24, 128, forced_path=PATH_VEC)
     assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 16
-    # 16 blocks x 196 tiles = 3136 units: more than 3 waves of 148 x 6 resident CTAs
-    assert p.rows_per_tile == 64 * 1024 // 1536 == 42 and p.units == 3136
-    assert p.block == 256 and p.grid == min(p.units, 148 * 16)
+    # 12 KB units of 8 rows x 1536 B: 16 blocks x 1024 tiles, one CTA per unit
+    assert p.rows_per_tile == 12 * 1024 // 1536 == 8 and p.units == 16 * 1024
+    assert p.block == 256 and p.grid == p.units
     assert p.producers == 0 and p.lookahead == 0
 
 
-def test_vec_units_shrink_below_three_waves():
-    # w=2: 64 KB units would be 4 blocks x 391 tiles = 1564 units, under 3 waves of
-    # 888 resident CTAs; the planner takes 4 waves' worth: 4 * 8192 // 3552 = 9 rows
-    rc, p, _ = plan(2, 1, 8192, 24, 128, forced_path=PATH_VEC)
-    assert rc == OK and p.rows_per_tile == 9 and p.tiles_per_block == -(-8192 // 9)
-    assert p.units == 4 * p.tiles_per_block == 3644 and p.tail_rows == 8192 % 9
-    assert p.grid == 148 * 16
-    # an explicit tile size is kept as given
-    rc, p, _ = plan(2, 1, 8192, 24, 128, forced_path=PATH_VEC, rows_per_tile=21)
-    assert rc == OK and p.rows_per_tile == 21 and p.units == 4 * 391
-    # a tiny problem goes down to one row per unit
-    rc, p, _ = plan(2, 1, 64, 4, 64, forced_path=PATH_VEC)
-    assert rc == OK and p.rows_per_tile == 1 and p.units == 4 * 64
+def test_vec_grid_one_cta_per_unit_unless_set():
+    rc, p, _ = plan(8, 2, 4725, 40, 128, forced_path=PATH_VEC)      # 1280 B rows
+    assert rc == OK and p.rows_per_tile == 9 and p.tail_rows == 4725 % 9
+    assert p.units == 8 * 2 * 8 * 525 and p.grid == p.units
+    # a row longer than the target makes one-row units
+    rc, p, _ = plan(1, 1, 100, 64, 128, forced_path=PATH_VEC)       # 16 KB rows
+    assert rc == OK and p.rows_per_tile == 1 and p.units == 100 and p.grid == 100
+    # ctas_per_sm selects a grid-stride grid; rows_per_tile is kept as given
+    rc, p, _ = plan(2, 1, 8192, 24, 128, forced_path=PATH_VEC, rows_per_tile=21, ctas_per_sm=16)
+    assert rc == OK and p.rows_per_tile == 21 and p.units == 4 * 391 and p.grid == 1564
+    rc, p, _ = plan(8, 2, 4725, 40, 128, forced_path=PATH_VEC, ctas_per_sm=4)
+    assert rc == OK and p.grid == 148 * 4
 
 
 def test_tuning_knobs():
