@@ -35,6 +35,15 @@ constexpr int64_t kTmaMaxTileBytes = 64 * 1024;
 // Dynamic shared memory the TMA ring may use per CTA by default (of 227 KB).
 constexpr int64_t kTmaSmemBudget = 192 * 1024;
 constexpr int64_t kTmaSmemMax = 220 * 1024;
+// B200 (sm_100): shared memory an SM can give its resident CTAs, and the part
+// of it the driver reserves per CTA.
+constexpr int64_t kSmemPerSm = 228 * 1024;
+constexpr int64_t kSmemReservedPerCta = 1024;
+// Chunk schedule default: one producer warp and one unit per CTA, with the
+// CTAs resident on an SM capped so that about this many tile bytes are in
+// flight per SM (measured on B200: ~90-110 KB beats both the uncapped ~190 KB
+// and 60-80 KB by 1-15 %).
+constexpr int64_t kTmaInflightPerSm = 100 * 1024;
 constexpr int kTmaMaxStages = 32;            // all producers together
 constexpr int kTmaMaxProducers = 8;          // producer warps per CTA
 constexpr int kTmaDefaultProducers = 4;
@@ -55,11 +64,10 @@ constexpr int kHostDefaultChunks = 8;
 constexpr int64_t kHostChunkMinBytes = 8 << 20;
 // TMA schedule: by default a grid of ceil(units / n) short-lived CTAs, each
 // taking n consecutive units, one per producer warp, with a one-tile ring per
-// producer and at most kTmaChunkSmemTarget of shared memory per CTA, so that
-// several CTAs share an SM and the hardware hands out chunks as CTAs finish
-// (no static tail imbalance). chunk_units = 0 selects a persistent grid
-// (static round robin) with deeper rings instead.
-constexpr int64_t kTmaChunkSmemTarget = 64 * 1024;
+// producer (default: one producer, n = 1). The hardware hands CTAs to SMs as
+// they finish, so there is no static tail imbalance, and the residency cap
+// (kTmaInflightPerSm) sets how many share an SM. chunk_units = 0 selects a
+// persistent grid (static round robin) with deeper rings instead.
 
 struct Tuning {
   int rows_per_tile = 0;  // 0 = default
@@ -302,8 +310,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     } else if (persistent) {
       np = kTmaDefaultProducers;
     } else {
-      int64_t fit = kTmaChunkSmemTarget / stage_bytes;
-      np = (int)(fit < 1 ? 1 : (fit > kTmaDefaultProducers ? kTmaDefaultProducers : fit));
+      np = 1;
     }
     const int min_sp = persistent ? 2 : 1;
     int64_t sp = 0;
@@ -346,6 +353,20 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
         }
         p->chunk_units = (int32_t)chunk;
         p->grid = (int32_t)((units + chunk - 1) / chunk);
+        // Residency cap: reserve enough shared memory per CTA that at most
+        // `cap` CTAs fit on an SM, which bounds the bytes in flight per SM.
+        int64_t cap = tune.ctas_per_sm;
+        if (cap <= 0) {
+          const int64_t per_cta_inflight = np * tile_bytes;
+          cap = (kTmaInflightPerSm + per_cta_inflight / 2) / per_cta_inflight;
+          if (cap < 1) cap = 1;
+          if (cap > 32) cap = 32;
+        }
+        {
+          int64_t per_cta = (kSmemPerSm / cap - kSmemReservedPerCta) / 1024 * 1024;
+          if (per_cta > kTmaSmemMax) per_cta = kTmaSmemMax;
+          if (per_cta > p->smem_bytes) p->smem_bytes = per_cta;
+        }
       }
       p->vec_bytes = 16;
     }

@@ -69,11 +69,21 @@ def test_plan_cfg2_tma():
     assert p.units == 4 * 1 * 4 * p.tiles_per_block
     assert p.payload_bytes == 192 * MiB
     assert p.launches == 1
-    # default schedule: short-lived CTAs of 4 producer warps, one 8 KB tile each
-    assert p.producers == 4 and p.block == 128 and p.stages == 4 and p.lookahead == 1
-    assert p.chunk_units == 4 and p.grid == -(-p.units // 4) == 6556
-    assert p.smem_bytes == 4 * 8 * 1024
+    # default schedule: one short-lived single-warp CTA per 7.5 KB tile, at most
+    # round(100 KB / 7.5 KB) = 13 resident per SM: 228 KB / 13 - 1 KB reserved,
+    # rounded down to 1 KB = 16 KB of shared memory each
+    assert p.producers == 1 and p.block == 32 and p.stages == 1 and p.lookahead == 1
+    assert p.chunk_units == 1 and p.grid == p.units == 26224
+    assert p.smem_bytes == 16 * 1024
+    assert (228 * 1024) // (p.smem_bytes + 1024) == 13
     assert p.order == 1
+    # the residency cap is the ctas_per_sm knob: 12 CTAs -> 18 KB each
+    rc, q, _ = plan(4, 1, 8192, 24, 128, ctas_per_sm=12)
+    assert rc == OK and q.smem_bytes == 18 * 1024 and (228 * 1024) // (q.smem_bytes + 1024) == 12
+    # four producers per CTA: the cap drops to round(100 / 30) = 3 CTAs per SM
+    rc, q, _ = plan(4, 1, 8192, 24, 128, producers=4, chunk_units=4)
+    assert rc == OK and q.block == 128 and q.grid == -(-q.units // 4)
+    assert q.smem_bytes == (228 * 1024 // 3 - 1024) // 1024 * 1024
     # the persistent schedule: one CTA per SM, 4 producers x 4-stage rings
     rc, q, _ = plan(4, 1, 8192, 24, 128, chunk_units=0)
     assert rc == OK and q.chunk_units == 0 and q.grid == 148
@@ -118,7 +128,7 @@ def test_plan_cfg1_small():
     rc, p, _ = plan(2, 1, 64, 4, 64)
     assert rc == OK and p.path == PATH_TMA
     assert p.rows_per_tile == 32 and p.tail_rows == 0 and p.tiles_per_block == 2
-    assert p.units == 8 and p.chunk_units == 4 and p.grid == 2
+    assert p.units == 8 and p.chunk_units == 1 and p.grid == 8
 
 
 def test_rows_never_exceed_sequence():
@@ -230,11 +240,17 @@ def test_large_rows_reduce_stages_then_producers():
     rc, p, _ = plan(2, 1, 8, 256, 256, chunk_units=0)
     assert rc == OK and p.path == PATH_TMA and p.row_bytes == 64 * 1024
     assert (p.producers, p.stages, p.lookahead, p.smem_bytes) == (1, 3, 2, 192 * 1024)
-    # default (chunked grid): at most 64 KB of tiles per CTA, one tile per producer
+    # default (chunked grid): one producer, one tile; the residency cap reserves
+    # shared memory for round(100 KB / tile) CTAs per SM (24 KB tiles: 4 CTAs)
     rc, p, _ = plan(2, 1, 16, 128, 192)
-    assert (p.producers, p.stages, p.chunk_units, p.smem_bytes) == (2, 2, 2, 48 * 1024)
+    assert (p.producers, p.stages, p.chunk_units) == (1, 1, 1)
+    assert p.smem_bytes == (228 * 1024 // 4 - 1024) // 1024 * 1024
+    # 64 KB tiles: cap round(100 / 64) = 2 CTAs per SM (113 KB each)
     rc, p, _ = plan(2, 1, 8, 256, 256)
-    assert (p.producers, p.stages, p.chunk_units, p.smem_bytes) == (1, 1, 1, 64 * 1024)
+    assert (p.producers, p.stages, p.chunk_units, p.smem_bytes) == (1, 1, 1, 113 * 1024)
+    # a tile larger than the cap's share keeps its own size (cap 1 is 220 KB max)
+    rc, p, _ = plan(2, 1, 8, 256, 256, ctas_per_sm=8)
+    assert p.smem_bytes == 64 * 1024
 
 
 # ---- argument validation ----------------------------------------------------
