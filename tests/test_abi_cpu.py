@@ -30,6 +30,23 @@ def test_header_declares_expected_entry_points():
     assert sorted(names) == sorted(_lib.EXPORTED)
 
 
+def test_header_constants_match_the_binding():
+    text = open(HEADER).read()
+    defines = {m.group(1): int(m.group(2))
+               for m in re.finditer(r"#define\s+ULYSSES_A2A_(\w+)\s+(\d+)", text)}
+    binding = {"OK": _lib.OK, "ERR_INVALID": _lib.ERR_INVALID, "ERR_OVERLAP": _lib.ERR_OVERLAP,
+               "ERR_DEVICE": _lib.ERR_DEVICE, "ERR_CUDA": _lib.ERR_CUDA,
+               "ERR_UNSUPPORTED": _lib.ERR_UNSUPPORTED, "ERR_NOMEM": _lib.ERR_NOMEM,
+               "ERR_TIMEOUT": _lib.ERR_TIMEOUT, "ERR_INTERNAL": _lib.ERR_INTERNAL,
+               "PATH_AUTO": _lib.PATH_AUTO, "PATH_TMA": _lib.PATH_TMA, "PATH_VEC": _lib.PATH_VEC,
+               "MAX_W": _lib.MAX_W, "MAX_W_TMA": _lib.MAX_W_TMA,
+               "PEER_HANDLE_BYTES": _lib.PEER_HANDLE_BYTES}
+    for name, value in binding.items():
+        assert defines[name] == value, name
+    # every status code the header defines is mirrored
+    assert {k for k in defines if k == "OK" or k.startswith("ERR_")} <= set(binding)
+
+
 def test_library_exports_every_declared_symbol():
     lib = ctypes.CDLL(_lib.LIB_PATH)
     for name in declared_functions():
