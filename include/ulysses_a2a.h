@@ -201,9 +201,13 @@ int ulysses_a2a_set_path(ulysses_a2a_ctx *ctx, int path);
  * left at its "default" value keeps the library's choice. */
 typedef struct ulysses_a2a_tuning_t {
     int32_t rows_per_tile;  /* S_tile cap, 1..256; 0 = default                */
-    int32_t ctas_per_sm;    /* persistent TMA grid / grid-stride VEC grid:
-                               CTAs per SM, 1..32; 0 = default (VEC: one
-                               CTA per unit)                              */
+    int32_t ctas_per_sm;    /* CTAs per SM, 1..32; 0 = default. TMA
+                               chunk schedule: a cap on resident CTAs per
+                               SM, enforced by reserving shared memory
+                               (default: about 100 KB of tiles in flight
+                               per SM); persistent TMA grid: its size;
+                               VEC: a grid-stride grid of this many per SM
+                               (default: one CTA per unit)                */
     int32_t stages;         /* TMA: shared-memory tiles per CTA, 1..32, split
                                evenly over the producers; 0 = default      */
     int32_t lookahead;      /* TMA: loads in flight per producer; 0 = default */
@@ -212,7 +216,8 @@ typedef struct ulysses_a2a_tuning_t {
                                outermost, 1 = innermost; -1 = default      */
     int32_t chunk_units;    /* TMA schedule: 0 = persistent grid (static
                                round robin); n > 0 = n consecutive units per
-                               CTA; -1 = default (one unit per producer)   */
+                               CTA; -1 = default (one unit per producer;
+                               one producer by default)                   */
     int32_t host_chunks;    /* host-buffer entry point: sequence chunks its
                                copies and kernels are pipelined over, 1..64;
                                0 = default                                */

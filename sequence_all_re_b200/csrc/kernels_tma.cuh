@@ -26,10 +26,10 @@
 // Schedule: one elected thread in each of `producers` warps per CTA drives its
 // own ring of `stages` shared-memory tiles over every producers-th unit this
 // CTA owns, keeping `lookahead` loads and up to stages - lookahead stores in
-// flight (TMA operations issued by one thread complete roughly one at a time,
-// so several producers keep enough in flight). A CTA owns either a chunk of
-// `chunk_units` consecutive units (the default: short-lived CTAs, several per
-// SM, handed out by the hardware as SMs free up) or, with chunk_units = 0,
+// flight. A CTA owns either a chunk of `chunk_units` consecutive units (the
+// default, with one producer and one unit per CTA: short-lived single-warp
+// CTAs handed out by the hardware as SMs free up, their residency per SM
+// capped by the shared memory the planner reserves) or, with chunk_units = 0,
 // units blockIdx.x + i*gridDim.x of a persistent grid. Units are numbered with
 // the destination rank innermost or outermost (`order`). Launches use
 // programmatic dependent launch: each CTA waits for the previous grid before
