@@ -105,11 +105,14 @@ SHAPES = [
     (8, 1, 7, 8, 256),          # D at the TMA box limit, H/w = 1
 ]
 
-# The default (short-lived CTAs, one tile per producer), then other shapes of
-# both schedules: chunked grids with deeper rings or other chunk sizes, and
-# persistent grids (chunk_units=0) with 1-4 producers and 2-4 stages each.
+# The default (short-lived single-warp CTAs, one tile each, residency capped),
+# other residency caps, then other shapes of both schedules: chunked grids
+# with deeper rings or other chunk sizes, and persistent grids
+# (chunk_units=0) with 1-4 producers and 2-4 stages each.
 TUNINGS = [
     {},
+    dict(ctas_per_sm=4),                          # residency cap: 56 KB reserved per CTA
+    dict(producers=2, chunk_units=2, ctas_per_sm=7),
     dict(rows_per_tile=7, stages=2),
     dict(rows_per_tile=5, stages=12, chunk_units=7),
     dict(producers=1, chunk_units=3),
