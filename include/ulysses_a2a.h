@@ -126,7 +126,12 @@ typedef struct ulysses_a2a_desc_t {
 
 /* Create a context on CUDA device `device` for elements of `elem_bytes` bytes
  * (1, 2, 4 or 8; bf16 = 2, fp32 = 4). On success *out holds a new context that
- * ulysses_a2a_destroy must release. Allocates a few bytes of device memory. */
+ * ulysses_a2a_destroy must release. Allocates a few bytes of device memory.
+ * For testing, two environment variables set the context's initial knobs
+ * (ulysses_a2a_set_path / ulysses_a2a_set_tuning override them later):
+ * ULYSSES_A2A_FORCE_PATH = auto | tma | vec, and ULYSSES_A2A_CTAS_PER_SM =
+ * 1..32 (the ctas_per_sm knob). A malformed value makes creation fail with
+ * ULYSSES_A2A_ERR_INVALID. */
 int ulysses_a2a_create(ulysses_a2a_ctx **out, int device, int elem_bytes);
 
 /* Release a context. NULL is accepted. Always consumes the handle, even when a
@@ -226,6 +231,13 @@ typedef struct ulysses_a2a_tuning_t {
 /* Apply tuning to later runs (NULL restores every default). Values outside
  * the ranges above are rejected with ULYSSES_A2A_ERR_INVALID. */
 int ulysses_a2a_set_tuning(ulysses_a2a_ctx *ctx, const ulysses_a2a_tuning_t *tuning);
+
+/* The context's current forced path (ULYSSES_A2A_PATH_*) and tuning, as set
+ * by the environment at creation, ulysses_a2a_set_path and
+ * ulysses_a2a_set_tuning (default fields keep their "default" values). Either
+ * output may be NULL. */
+int ulysses_a2a_get_settings(const ulysses_a2a_ctx *ctx, int32_t *path,
+                             ulysses_a2a_tuning_t *tuning);
 
 /* Kernel launches this context has issued since creation. */
 uint64_t ulysses_a2a_launch_count(const ulysses_a2a_ctx *ctx);

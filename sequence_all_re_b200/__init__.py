@@ -53,13 +53,10 @@ class UlyssesA2A:
         self.device = dev
         self.elem_bytes = int(elem_bytes)
         self._ctx = _lib.ulysses_a2a_create(dev.index or 0, self.elem_bytes)
-        self._path = _lib.PATH_AUTO      # mirrors of the context's settings, for plan()
-        self._knobs = {}
 
     # ------------------------------------------------------------------ knobs
     def set_path(self, path: int) -> None:
         self._check(_lib.ulysses_a2a_set_path(self._ctx, path))
-        self._path = int(path)
 
     def set_tuning(self, rows_per_tile: int = 0, ctas_per_sm: int = 0, stages: int = 0,
                    **knobs) -> None:
@@ -67,8 +64,12 @@ class UlyssesA2A:
         restores every default. Extra knobs: lookahead, producers, order, chunk_units."""
         self._check(_lib.ulysses_a2a_set_tuning(self._ctx, rows_per_tile=rows_per_tile,
                                                 ctas_per_sm=ctas_per_sm, stages=stages, **knobs))
-        self._knobs = dict(rows_per_tile=rows_per_tile, ctas_per_sm=ctas_per_sm, stages=stages,
-                           **knobs)
+
+    def settings(self):
+        """(forced path, tuning knobs) of this context, as the library holds them."""
+        rc, path, knobs = _lib.ulysses_a2a_get_settings(self._ctx)
+        self._check(rc)
+        return path, knobs
 
     @property
     def launch_count(self) -> int:
@@ -181,11 +182,12 @@ class UlyssesA2A:
         """The path and geometry a run with these tensors would use (host only), with
         this context's forced path and tuning, or the given ``knobs`` dict instead."""
         w, (B, S, H, D), out = self._prepare(xs, mode, out, xs[0].device.type, allow_pitch=True)
+        path, current = self.settings()
         rc, p, msg = _lib.ulysses_a2a_plan_ex([t.data_ptr() for t in xs],
                                               [o.data_ptr() for o in out], B, S, H, D, w, mode,
                                               int(chunked), self.elem_bytes,
-                                              row_pitch=self._last_pitch, forced_path=self._path,
-                                              **(self._knobs if knobs is None else knobs))
+                                              row_pitch=self._last_pitch, forced_path=path,
+                                              **(current if knobs is None else knobs))
         if rc != _lib.OK:
             raise A2AError(rc, msg)
         return p.as_dict()

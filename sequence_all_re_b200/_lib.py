@@ -45,6 +45,7 @@ EXPORTED = (
     "ulysses_a2a_run_ex",
     "ulysses_a2a_plan_ex",
     "ulysses_a2a_selftest_wait_timeout",
+    "ulysses_a2a_get_settings",
     "ulysses_a2a_peer_create",
     "ulysses_a2a_peer_open",
     "ulysses_a2a_peer_publish",
@@ -192,6 +193,9 @@ def _load() -> ctypes.CDLL:
     lib.ulysses_a2a_plan_ex.restype = c_int
     lib.ulysses_a2a_selftest_wait_timeout.argtypes = [P, ctypes.c_uint32, P]
     lib.ulysses_a2a_selftest_wait_timeout.restype = c_int
+    lib.ulysses_a2a_get_settings.argtypes = [P, ctypes.POINTER(ctypes.c_int32),
+                                             ctypes.POINTER(TuningT)]
+    lib.ulysses_a2a_get_settings.restype = c_int
     lib.ulysses_a2a_peer_create.argtypes = [P, c_int, c_int, ctypes.c_size_t, ctypes.POINTER(P), P]
     lib.ulysses_a2a_peer_create.restype = c_int
     lib.ulysses_a2a_peer_open.argtypes = [P, P]
@@ -262,6 +266,14 @@ def ulysses_a2a_set_tuning(ctx, **knobs) -> int:
     order, chunk_units); no knobs restores every default."""
     t = TuningT.make(**knobs)
     return lib.ulysses_a2a_set_tuning(ctx, ctypes.byref(t))
+
+
+def ulysses_a2a_get_settings(ctx):
+    """Returns (rc, forced path, dict of tuning knobs)."""
+    path = ctypes.c_int32()
+    t = TuningT()
+    rc = lib.ulysses_a2a_get_settings(ctx, ctypes.byref(path), ctypes.byref(t))
+    return rc, path.value, {name: getattr(t, name) for name, _ in TuningT._fields_}
 
 
 def ulysses_a2a_launch_count(ctx) -> int:

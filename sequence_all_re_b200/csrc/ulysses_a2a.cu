@@ -396,6 +396,27 @@ int plan_for(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, int6
   return ULYSSES_A2A_OK;
 }
 
+// Test-only configuration read when a context is created; set_path and
+// set_tuning override it afterwards. ULYSSES_A2A_FORCE_PATH = auto | tma | vec
+// forces a copy path, ULYSSES_A2A_CTAS_PER_SM = 1..32 sets the ctas_per_sm
+// knob. Returns false on a malformed value (creation then fails).
+bool env_config(int* path, int* ctas) {
+  if (const char* v = std::getenv("ULYSSES_A2A_FORCE_PATH")) {
+    const std::string s(v);
+    if (s == "auto" || s.empty()) *path = ULYSSES_A2A_PATH_AUTO;
+    else if (s == "tma") *path = ULYSSES_A2A_PATH_TMA;
+    else if (s == "vec") *path = ULYSSES_A2A_PATH_VEC;
+    else return false;
+  }
+  if (const char* v = std::getenv("ULYSSES_A2A_CTAS_PER_SM")) {
+    char* end = nullptr;
+    const long n = std::strtol(v, &end, 10);
+    if (end == v || *end != '\0' || n < 1 || n > 32) return false;
+    *ctas = (int)n;
+  }
+  return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -405,6 +426,8 @@ static int ua2a_impl_create(ulysses_a2a_ctx** out, int device, int elem_bytes) {
   *out = nullptr;
   if (!(elem_bytes == 1 || elem_bytes == 2 || elem_bytes == 4 || elem_bytes == 8))
     return ULYSSES_A2A_ERR_INVALID;
+  int env_path = ULYSSES_A2A_PATH_AUTO, env_ctas = 0;
+  if (!env_config(&env_path, &env_ctas)) return ULYSSES_A2A_ERR_INVALID;
   int count = 0;
   if (cudaGetDeviceCount(&count) != cudaSuccess || device < 0 || device >= count) {
     cudaGetLastError();
@@ -414,6 +437,8 @@ static int ua2a_impl_create(ulysses_a2a_ctx** out, int device, int elem_bytes) {
   if (!ctx) return ULYSSES_A2A_ERR_NOMEM;
   ctx->device = device;
   ctx->elem_bytes = elem_bytes;
+  ctx->forced_path = env_path;
+  ctx->tuning.ctas_per_sm = env_ctas;
   DeviceGuard g(device);
   if (!g.ok) {
     delete ctx;
@@ -771,6 +796,24 @@ static int ua2a_impl_set_tuning(ulysses_a2a_ctx* ctx, const ulysses_a2a_tuning_t
   std::string err;
   if (!ua2a::tuning_from(t, &tu, &err)) return fail(ctx, ULYSSES_A2A_ERR_INVALID, err);
   ctx->tuning = tu;
+  return ULYSSES_A2A_OK;
+}
+
+static int ua2a_impl_get_settings(const ulysses_a2a_ctx* ctx, int32_t* path,
+                                  ulysses_a2a_tuning_t* t) {
+  if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
+  if (path) *path = ctx->forced_path;
+  if (t) {
+    const ua2a::Tuning& u = ctx->tuning;
+    t->rows_per_tile = u.rows_per_tile;
+    t->ctas_per_sm = u.ctas_per_sm;
+    t->stages = u.stages;
+    t->lookahead = u.lookahead;
+    t->producers = u.producers;
+    t->order = u.order;
+    t->chunk_units = u.chunk_units;
+    t->host_chunks = u.host_chunks;
+  }
   return ULYSSES_A2A_OK;
 }
 
@@ -1472,6 +1515,10 @@ int ulysses_a2a_plan(const void* const* in_slabs, void* const* out_slabs, int64_
   return no_throw([&] { return ua2a_impl_plan(in_slabs, out_slabs, B, S_local, H, D, w, mode,
                                               chunked, elem_bytes, forced_path, tuning, num_sms,
                                               out, err, errlen); });
+}
+
+int ulysses_a2a_get_settings(const ulysses_a2a_ctx* ctx, int32_t* path, ulysses_a2a_tuning_t* t) {
+  return no_throw([&] { return ua2a_impl_get_settings(ctx, path, t); });
 }
 
 int ulysses_a2a_peer_create(ulysses_a2a_ctx* ctx, int rank, int world, size_t window_bytes,

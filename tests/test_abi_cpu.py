@@ -418,3 +418,32 @@ def test_pitched_extent_counts_for_overlap():
     rc, _, _ = _lib.ulysses_a2a_plan_ex(outs, [1 << 42, (1 << 42) + (1 << 20)], B, S, H, D, w, 0,
                                         0, E, row_pitch=pitch)
     assert rc == OK
+
+
+# ---- test-only environment overrides at context creation ----------------------
+
+@pytest.mark.parametrize("name,value", [("ULYSSES_A2A_FORCE_PATH", "fast"),
+                                        ("ULYSSES_A2A_CTAS_PER_SM", "0"),
+                                        ("ULYSSES_A2A_CTAS_PER_SM", "33"),
+                                        ("ULYSSES_A2A_CTAS_PER_SM", "8x")])
+def test_malformed_environment_override_fails_creation(monkeypatch, name, value):
+    monkeypatch.setenv(name, value)
+    h = ctypes.c_void_p()
+    # checked before the device is touched, so this holds without a GPU too
+    assert _lib.lib.ulysses_a2a_create(ctypes.byref(h), 0, 2) == ERR_INVALID
+    assert not h.value
+
+
+def test_valid_environment_override_is_accepted(monkeypatch):
+    monkeypatch.setenv("ULYSSES_A2A_FORCE_PATH", "vec")
+    monkeypatch.setenv("ULYSSES_A2A_CTAS_PER_SM", "8")
+    h = ctypes.c_void_p()
+    rc = _lib.lib.ulysses_a2a_create(ctypes.byref(h), 0, 2)
+    assert rc != ERR_INVALID               # OK on a GPU, ERR_DEVICE without one
+    if rc == OK:
+        assert _lib.ulysses_a2a_get_settings(h)[:2] == (OK, PATH_VEC)
+        _lib.ulysses_a2a_destroy(h)
+
+
+def test_get_settings_rejects_null_context():
+    assert _lib.lib.ulysses_a2a_get_settings(None, None, None) == ERR_INVALID

@@ -767,3 +767,23 @@ def test_two_gib_payload_full_compare():
     y = run_case(xs, 0)
     del xs
     run_case(y, 1)
+
+
+def test_environment_overrides_set_the_initial_knobs(monkeypatch):
+    monkeypatch.setenv("ULYSSES_A2A_FORCE_PATH", "vec")
+    monkeypatch.setenv("ULYSSES_A2A_CTAS_PER_SM", "8")
+    with UlyssesA2A(0, 2) as a2a:
+        monkeypatch.delenv("ULYSSES_A2A_FORCE_PATH")
+        monkeypatch.delenv("ULYSSES_A2A_CTAS_PER_SM")
+        path, knobs = a2a.settings()
+        assert path == PATH_VEC and knobs["ctas_per_sm"] == 8
+        xs = normal_slabs((1, 96, 8, 64), 4, "bf16")
+        out = run_case(xs, 0, a2a=a2a, path=PATH_VEC, tuning={"ctas_per_sm": 8})
+        p = a2a.plan([t.cuda() for t in xs], 0)
+        assert p["path"] == PATH_VEC and p["grid"] <= 148 * 8
+        # the API overrides the environment
+        a2a.set_path(PATH_AUTO)
+        a2a.set_tuning()
+        assert a2a.settings() == (PATH_AUTO, dict(_lib.TuningT.DEFAULTS))
+        assert a2a.plan([t.cuda() for t in xs], 0)["path"] == PATH_TMA
+        del out
