@@ -355,7 +355,11 @@ int ulysses_a2a_peer_open(ulysses_a2a_peer *peer, const void *handles);
  * stream). mode 0: in_local is [B, S_local, H, D] with row_pitch (0 = dense,
  * else >= H*D elements between rows, as in ulysses_a2a_desc_t); mode 1:
  * in_local is [B, S_local*w, H/w, D] dense and row_pitch must be 0. The
- * window receives the dense slab. */
+ * window receives the dense slab. If in_local is this rank's own window
+ * (ulysses_a2a_peer_window(peer, rank)) holding the dense slab, the slab was
+ * written in place and nothing is copied or launched (zero-copy publish: the
+ * producer of the slab writes into the window directly, after the barrier of
+ * step 4 of the previous exchange). */
 int ulysses_a2a_peer_publish(ulysses_a2a_peer *peer, const void *in_local,
                              int64_t B, int64_t S_local, int64_t H, int64_t D,
                              int mode, int64_t row_pitch, void *stream);

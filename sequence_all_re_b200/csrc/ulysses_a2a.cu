@@ -1080,6 +1080,16 @@ static int ua2a_impl_peer_publish(ulysses_a2a_peer* p, const void* in_local, int
   // pitch); mode 1 copies [B, S*w, H/w, D]
   const int64_t S1 = mode == 0 ? S_local : S_local * w;
   const int64_t H1 = mode == 0 ? H : H / w;
+  if (in_local == p->own && (row_pitch == 0 || row_pitch == H1 * D)) {
+    // the slab was written into the window in place: nothing to copy
+    int64_t bytes = 0;
+    if (ua2a::mul_overflows(B, S1, &bytes) || ua2a::mul_overflows(bytes, H1, &bytes) ||
+        ua2a::mul_overflows(bytes, D, &bytes) ||
+        ua2a::mul_overflows(bytes, (int64_t)ctx->elem_bytes, &bytes) ||
+        (uint64_t)bytes > (uint64_t)p->window_bytes)
+      return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_publish: the slab exceeds the window");
+    return ULYSSES_A2A_OK;
+  }
   const void* in[1] = {in_local};
   void* out[1] = {p->own};
   ulysses_a2a_plan_t pl;

@@ -20,7 +20,9 @@ request "pipeline HCA AllToAll into O-A", which publishes into a distributed
 window and has consumers load from it after a handshake:
 barrier -> publish (own input into own window) -> barrier -> pull (one kernel
 reads this rank's share out of every window over NVLink and writes the local
-output). The barriers are collectives of the process group on the caller's
+output). With ``input_buffer()`` the producer of the slab writes it into the
+window itself (that pull request's publishing workers), and the first barrier
+and the publish copy drop out. The barriers are collectives of the process group on the caller's
 stream (NCCL: a one-element all-reduce, stream ordered, no host wait) or, for
 host-only backends such as gloo, a stream synchronise plus a group barrier.
 No kernel waits for another GPU.
@@ -38,6 +40,15 @@ from . import UlyssesA2A, _lib, mode0_local_tuple, output_shape
 from ._lib import A2AError
 
 __all__ = ["PeerExchange", "NativePeer"]
+
+
+class _DeviceBytes:
+    """n bytes of device memory at ptr, exposed through the CUDA array interface
+    (so torch can view the window without copying it)."""
+
+    def __init__(self, ptr: int, n: int):
+        self.__cuda_array_interface__ = {"data": (int(ptr), False), "shape": (int(n),),
+                                         "typestr": "|u1", "version": 2, "strides": None}
 
 
 class NativePeer:
@@ -59,6 +70,8 @@ class NativePeer:
         rc, h, rec = _lib.ulysses_a2a_peer_create(self.a2a._ctx, rank, world, nbytes)
         self._check(rc)
         self._peer = h
+        self._rank = rank
+        self._nbytes = int(nbytes)
         return rec
 
     def open(self, records) -> None:
@@ -74,6 +87,17 @@ class NativePeer:
 
     def window(self, rank: int) -> int:
         return _lib.ulysses_a2a_peer_window(self._peer, rank) if self._peer is not None else 0
+
+    def window_tensor(self, shape, dtype) -> torch.Tensor:
+        """This rank's window as a dense tensor (no copy; valid until the window
+        is released)."""
+        n = torch.empty((), dtype=dtype).element_size()
+        for v in shape:
+            n *= int(v)
+        if self._peer is None or n > self._nbytes:
+            raise ValueError("the window is not built or is smaller than the tensor")
+        raw = torch.as_tensor(_DeviceBytes(self.window(self._rank), n), device=self.device)
+        return raw.view(dtype).view(tuple(shape))
 
     def unmap(self) -> None:
         if self._peer is not None:
@@ -125,6 +149,7 @@ class PeerExchange:
         self._nbytes = 0
         self._armed = False
         self._agreed = set()           # call signatures every rank has confirmed
+        self._in_place = None          # window address handed out by input_buffer()
         self.disabled_reason = None
 
     # ---------------------------------------------------------- group helpers
@@ -221,6 +246,49 @@ class PeerExchange:
         self.native.close()
 
     # -------------------------------------------------------------------- the op
+    def _agree_signature(self, sig) -> None:
+        if sig not in self._agreed:
+            sigs = self._gather(sig)
+            if any(s != sig for s in sigs):
+                raise ValueError(f"ranks called the exchange with different arguments: {sigs}")
+            self._agreed.add(sig)
+
+    def _ensure_window(self, need: int) -> None:
+        if need > self._nbytes:
+            if self._armed and not self.close():
+                raise RuntimeError("window teardown before growing failed")
+            if not self.build(need):
+                self._disable("a rank could not build its window")
+                raise RuntimeError("peer exchange: window build failed on some rank")
+
+    def input_buffer(self, shape, dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+        """This rank's window as a dense tensor of ``shape``, for an in-place input.
+
+        Collective: every rank calls it with the same shape. It takes the
+        barrier after which no rank reads the windows any more, so the caller
+        may write its slab straight into the returned tensor (for example as
+        the output of the projection that produces it) and then pass that
+        tensor to ``all_to_all_4d`` with ``chunked=False``, which skips the
+        publish copy and its barrier. The tensor is valid until the window is
+        rebuilt or closed.
+        """
+        if self.disabled_reason is not None:
+            raise RuntimeError(f"peer exchange disabled: {self.disabled_reason}")
+        shape = tuple(int(v) for v in shape)
+        if len(shape) != 4 or torch.empty((), dtype=dtype).element_size() != self.elem_bytes:
+            raise ValueError(f"a 4D shape of {self.elem_bytes}-byte elements is required")
+        need = self.elem_bytes
+        for v in shape:
+            need *= v
+        self._agree_signature(("input_buffer", shape, dtype))
+        self._ensure_window(need)
+        if stream is None:
+            stream = self.native.current_stream()
+        self._barrier(stream)         # every rank is done reading the windows
+        t = self.native.window_tensor(shape, dtype)
+        self._in_place = t.data_ptr()
+        return t
+
     def all_to_all_4d(self, x: torch.Tensor, mode: int, chunked: bool = False, out=None,
                       stream=None) -> torch.Tensor:
         """Exchange this rank's slab ``x``; returns this rank's output slab.
@@ -255,20 +323,20 @@ class PeerExchange:
             return out
         planes = B if chunked else 1
         need = (1 if chunked else B) * S * H * D * self.elem_bytes
-        sig = (mode, bool(chunked), B, S, H, D, x.dtype)
-        if sig not in self._agreed:
-            sigs = self._gather(sig)
-            if any(s != sig for s in sigs):
-                raise ValueError(f"ranks called the exchange with different arguments: {sigs}")
-            self._agreed.add(sig)
-        if need > self._nbytes:
-            if self._armed and not self.close():
-                raise RuntimeError("window teardown before growing failed")
-            if not self.build(need):
-                self._disable("a rank could not build its window")
-                raise RuntimeError("peer exchange: window build failed on some rank")
+        in_place = self._armed and x.data_ptr() == self.native.window(self.rank)
+        self._agree_signature((mode, bool(chunked), B, S, H, D, x.dtype, in_place))
         if stream is None:
             stream = self.native.current_stream()
+        if in_place:
+            # the slab was written into the window after input_buffer()'s barrier
+            if chunked or not x.is_contiguous() or self._in_place != x.data_ptr():
+                raise ValueError("an input in the window must come from input_buffer() and be "
+                                 "exchanged whole (chunked=False)")
+            self._in_place = None
+            self._barrier(stream)    # every window holds its slab
+            self.native.pull(out, B, S, H, D, mode, pitch if mode == 1 else 0, stream)
+            return out
+        self._ensure_window(need)
         nb = 1 if chunked else B
         for b in range(planes):
             xv = x[b:b + 1] if chunked else x

@@ -65,6 +65,18 @@ class ShmNative:
             n *= v
         return torch.frombuffer(shm.buf, dtype=dtype, count=n).view(shape)
 
+    def window(self, rank):
+        shm = self.own if rank == self.rank else self.peers.get(rank)
+        if shm is None:
+            return 0
+        return torch.frombuffer(shm.buf, dtype=torch.uint8, count=1).data_ptr()
+
+    def window_tensor(self, shape, dtype):
+        n = 1
+        for v in shape:
+            n *= v
+        return torch.frombuffer(self.own.buf, dtype=dtype, count=n).view(shape)
+
     def publish(self, x, B, S, H, D, mode, row_pitch, stream):
         time.sleep(self.publish_delay)
         w = self.world
@@ -137,6 +149,31 @@ def _worker(rank, world, port, scenario, q):
                 rep["ok"].append(torch.equal(got.view(torch.int16), want.view(torch.int16)))
             rep["closed"] = ex.close()
             rep["log"] = native.log
+        elif scenario == "in_place":
+            # rank 1 writes its slab late and pulls late: without the barrier in
+            # input_buffer() rank 0 would overwrite its window while rank 1 still
+            # reads it; without the one before the pull, rank 0 would read rank
+            # 1's window before the slab is in it
+            native = ShmNative(rank, pull_delay=0.2 if rank == 1 else 0.0)
+            ex = PeerExchange(native=native, elem_bytes=2)
+            shape = (2, 5, 4, 8)
+            for it in range(3):
+                xs = normal_slabs(shape, world, "bf16", seed0=1000 + 10 * it)
+                buf = ex.input_buffer(shape, torch.bfloat16)
+                if rank == 1:
+                    time.sleep(0.05)
+                buf.copy_(xs[rank])
+                got = ex.all_to_all_4d(buf, 0)
+                del buf
+                want = oracle.ulysses_a2a(xs, 0)[rank]
+                rep["ok"].append(torch.equal(got.view(torch.int16), want.view(torch.int16)))
+            # an ordinary call still works after in-place ones
+            xs = normal_slabs(shape, world, "bf16", seed0=2000)
+            got = ex.all_to_all_4d(xs[rank].clone(), 0)
+            rep["ok"].append(torch.equal(got.view(torch.int16),
+                                         oracle.ulysses_a2a(xs, 0)[rank].view(torch.int16)))
+            rep["closed"] = ex.close()
+            rep["log"] = native.log
         elif scenario == "fail_build":
             native = ShmNative(rank, fail_create=(rank == 1))
             ex = PeerExchange(native=native, elem_bytes=2)
@@ -190,6 +227,16 @@ def test_exchange_sequence_barriers_and_growth():
         # one publish + one pull per exchange, per plane when chunked
         assert ops == ["publish", "pull"] * (1 + 1 + 2 + 1)
         assert log.index(("unmap",)) < log.index(("release",))
+
+
+def test_in_place_input_skips_the_publish():
+    for rep in _run("in_place", 300):
+        assert rep["errors"] == [], rep
+        assert rep["ok"] == [True] * 4, rep
+        assert rep["closed"] is True
+        ops = [e for e in rep["log"] if isinstance(e, str)]
+        # three in-place exchanges pull without publishing, then one ordinary one
+        assert ops == ["pull"] * 3 + ["publish", "pull"]
 
 
 def test_failed_window_build_disables_every_rank():

@@ -264,3 +264,36 @@ def test_peer_errors_launch_nothing():
             assert torch.equal(bits(outs[k].cpu()), bits(want[k]))
     finally:
         ranks.close()
+
+
+def test_publishing_the_own_window_copies_nothing():
+    """Zero-copy publish: a slab already in the rank's own window is left in place."""
+    w, B, S, H, D = 4, 2, 33, 8, 64
+    xs_cpu = normal_slabs((B, S, H, D), w, "bf16")
+    ranks = LocalRanks(w, 2, slab_bytes((B, S, H, D), 2)).open()
+    try:
+        stream = torch.cuda.current_stream().cuda_stream
+        xs = [t.cuda() for t in xs_cpu]
+        for k in range(w):      # an ordinary publish puts each slab into its window
+            assert _lib.ulysses_a2a_peer_publish(ranks.peers[k], xs[k].data_ptr(), B, S, H, D, 0, 0,
+                                                 stream) == _lib.OK
+        n0 = ranks.launches()
+        for k in range(w):
+            own = _lib.ulysses_a2a_peer_window(ranks.peers[k], k)
+            assert _lib.ulysses_a2a_peer_publish(ranks.peers[k], own, B, S, H, D, 0, 0,
+                                                 stream) == _lib.OK
+            # the window as a pitched source is not in place: it overlaps the window
+            assert _lib.ulysses_a2a_peer_publish(ranks.peers[k], own, B, S, H, D, 0, 2 * H * D,
+                                                 stream) == _lib.ERR_OVERLAP
+        assert ranks.launches() == n0
+        want = oracle.ulysses_a2a(xs_cpu, 0)
+        g = Guarded(tuple(want[0].shape), torch.bfloat16, w)
+        for k in range(w):
+            assert _lib.ulysses_a2a_peer_pull(ranks.peers[k], g.slabs[k].data_ptr(), B, S, H, D, 0,
+                                              0, stream) == _lib.OK
+        torch.cuda.synchronize()
+        for k in range(w):
+            assert torch.equal(bits(g.slabs[k].cpu()), bits(want[k]))
+        g.check_guards()
+    finally:
+        ranks.close()

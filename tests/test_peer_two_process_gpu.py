@@ -48,6 +48,19 @@ def _worker(rank, world, port, q):
             report["ok"].append(torch.equal(y.cpu().view(torch.int16), want_y.view(torch.int16)) and
                                 torch.equal(z.cpu().view(torch.int16), xs[rank].view(torch.int16)))
             report["grew"].append(ex._nbytes)
+        # in place: the slab is written straight into this rank's window
+        shape = (1, 512, 16, 128)
+        xs = normal_slabs(shape, world, "bf16", seed0=4321)
+        n0 = ex.native.launch_count
+        buf = ex.input_buffer(shape, torch.bfloat16)
+        assert buf.data_ptr() == ex.native.window(rank)
+        buf.copy_(xs[rank].cuda())
+        y = ex.all_to_all_4d(buf, 0)
+        del buf
+        torch.cuda.synchronize()
+        report["in_place_ok"] = torch.equal(y.cpu().view(torch.int16),
+                                            oracle.ulysses_a2a(xs, 0)[rank].view(torch.int16))
+        report["in_place_launches"] = ex.native.launch_count - n0
         report["closed"] = ex.close()
         report["launches"] = ex.native.launch_count
         ex.native.close()
@@ -80,5 +93,7 @@ def test_two_processes_exchange_through_ipc_windows():
         # windows: one plane when chunked, the whole slab otherwise; grown once
         # for the large case, never shrunk
         assert rep["grew"] == [2 * 37 * 8 * 64 * 2] * 2 + [512 * 16 * 128 * 2] * 2
-        # publish + pull per exchange (per plane when chunked), two exchanges per case
-        assert rep["launches"] == 2 * 2 * (1 + 2 + 1 + 3)
+        # publish + pull per exchange (per plane when chunked), two exchanges per case,
+        # then one in-place exchange: a pull and nothing else
+        assert rep["in_place_ok"] is True and rep["in_place_launches"] == 1
+        assert rep["launches"] == 2 * 2 * (1 + 2 + 1 + 3) + 1
