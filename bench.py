@@ -648,6 +648,9 @@ def run_peer_one_gpu(args):
         "config": {"workload": workload_name(w, B, S, H, D, 0) + "; publish + pull per rank",
                    "l2": "inputs larger than L2 (back to back)"},
         "gpu_launches": launches,
+        # inputs written into the windows in place (PeerExchange.input_buffer):
+        # the step is the two pull groups alone, timed above
+        "in_place_value": round(2 * P / ((ms_pull0 + ms_pull1) / 1e3) / 1e9, 1),
         "kernels": {"publish (one-rank re-layout into the own window)": roof(ms_pub),
                     "pull mode 0 (VEC, one output slab)": roof(ms_pull0),
                     "pull mode 1 (VEC, one output slab)": roof(ms_pull1)},
