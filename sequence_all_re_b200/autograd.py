@@ -4,7 +4,10 @@
 The re-layout is a permutation of elements, y = P x, so the gradient of the
 input is the inverse permutation of the output gradient: dL/dx = P^-1 dL/dy.
 Mode 1 is the inverse of mode 0, so the backward of a mode-m call is a
-mode-(1-m) call on the output gradients, run by the same CUDA kernels.
+mode-(1-m) call on the output gradients, run by the same CUDA kernels. This
+holds for the single-GPU re-layout of all w slabs (`all_to_all_4d`) and for
+one rank's side of the cross-GPU exchange (`peer_all_to_all_4d`), whose
+backward is itself an exchange and so is collective like the forward.
 """
 
 from __future__ import annotations
@@ -39,3 +42,26 @@ class UlyssesAllToAll4D(torch.autograd.Function):
 def all_to_all_4d(a2a: UlyssesA2A, xs, mode: int, chunked: bool = False) -> list:
     """Differentiable re-layout of the w slabs `xs` (see UlyssesA2A.run)."""
     return list(UlyssesAllToAll4D.apply(a2a, int(mode), bool(chunked), *xs))
+
+
+class PeerAllToAll4D(torch.autograd.Function):
+    """forward: this rank's mode-`mode` exchange; backward: the inverse-mode exchange
+    of the output gradient (every rank runs it, in the same order)."""
+
+    @staticmethod
+    def forward(ctx, ex, mode: int, chunked: bool, x):
+        ctx.ex = ex
+        ctx.mode = int(mode)
+        ctx.chunked = bool(chunked)
+        return ex.all_to_all_4d(x.detach(), ctx.mode, chunked=ctx.chunked)
+
+    @staticmethod
+    def backward(ctx, grad):
+        g = ctx.ex.all_to_all_4d(grad.contiguous(), 1 - ctx.mode, chunked=ctx.chunked)
+        return None, None, None, g
+
+
+def peer_all_to_all_4d(ex, x, mode: int, chunked: bool = False):
+    """Differentiable cross-GPU exchange of this rank's slab `x` (see
+    sequence_all_re_b200.peer.PeerExchange.all_to_all_4d)."""
+    return PeerAllToAll4D.apply(ex, int(mode), bool(chunked), x)

@@ -174,6 +174,21 @@ def _worker(rank, world, port, scenario, q):
                                          oracle.ulysses_a2a(xs, 0)[rank].view(torch.int16)))
             rep["closed"] = ex.close()
             rep["log"] = native.log
+        elif scenario == "autograd":
+            from sequence_all_re_b200.autograd import peer_all_to_all_4d
+            ex = PeerExchange(native=ShmNative(rank), elem_bytes=2)
+            shape = (2, 5, 4, 8)
+            xs = normal_slabs(shape, world, "bf16")
+            gys = uniform_slabs((2, 5 * world, 4 // world, 8), world, "bf16", seed0=77)
+            x = xs[rank].clone().requires_grad_()
+            y = peer_all_to_all_4d(ex, x, 0)
+            y.backward(gys[rank])
+            # forward: mode 0 of the rank slabs; backward: mode 1 of the gradients
+            rep["ok"].append(torch.equal(y.detach().view(torch.int16),
+                                         oracle.ulysses_a2a(xs, 0)[rank].view(torch.int16)))
+            rep["ok"].append(torch.equal(x.grad.view(torch.int16),
+                                         oracle.ulysses_a2a(gys, 1)[rank].view(torch.int16)))
+            rep["closed"] = ex.close()
         elif scenario == "fail_build":
             native = ShmNative(rank, fail_create=(rank == 1))
             ex = PeerExchange(native=native, elem_bytes=2)
@@ -237,6 +252,13 @@ def test_in_place_input_skips_the_publish():
         ops = [e for e in rep["log"] if isinstance(e, str)]
         # three in-place exchanges pull without publishing, then one ordinary one
         assert ops == ["pull"] * 3 + ["publish", "pull"]
+
+
+def test_autograd_backward_is_the_inverse_exchange():
+    for rep in _run("autograd", 400):
+        assert rep["errors"] == [], rep
+        assert rep["ok"] == [True, True], rep
+        assert rep["closed"] is True
 
 
 def test_failed_window_build_disables_every_rank():

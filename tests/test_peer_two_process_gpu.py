@@ -61,8 +61,21 @@ def _worker(rank, world, port, q):
         report["in_place_ok"] = torch.equal(y.cpu().view(torch.int16),
                                             oracle.ulysses_a2a(xs, 0)[rank].view(torch.int16))
         report["in_place_launches"] = ex.native.launch_count - n0
+        # autograd: the backward of a mode-0 exchange is the mode-1 exchange
+        from sequence_all_re_b200.autograd import peer_all_to_all_4d
+        from synth import uniform_slabs
+        shape = (2, 37, 8, 64)
+        xs = normal_slabs(shape, world, "bf16", seed0=99)
+        gys = uniform_slabs((2, 37 * world, 8 // world, 64), world, "bf16", seed0=7)
+        x = xs[rank].cuda().requires_grad_()
+        y = peer_all_to_all_4d(ex, x, 0)
+        y.backward(gys[rank].cuda())
+        torch.cuda.synchronize()
+        report["grad_ok"] = torch.equal(x.grad.cpu().view(torch.int16),
+                                        oracle.ulysses_a2a(gys, 1)[rank].view(torch.int16))
+        n1 = ex.native.launch_count
         report["closed"] = ex.close()
-        report["launches"] = ex.native.launch_count
+        report["launches"] = n1
         ex.native.close()
     except Exception as e:  # reported to the parent, which fails the test
         report["error"] = repr(e)
@@ -96,4 +109,6 @@ def test_two_processes_exchange_through_ipc_windows():
         # publish + pull per exchange (per plane when chunked), two exchanges per case,
         # then one in-place exchange: a pull and nothing else
         assert rep["in_place_ok"] is True and rep["in_place_launches"] == 1
-        assert rep["launches"] == 2 * 2 * (1 + 2 + 1 + 3) + 1
+        assert rep["grad_ok"] is True
+        # ... and a forward + backward exchange of publish + pull each
+        assert rep["launches"] == 2 * 2 * (1 + 2 + 1 + 3) + 1 + 2 * 2
