@@ -546,7 +546,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-# ---------------------------------------------------------------- reference arm
+# ------------------------------------------- cross-GPU exchange kernels, one GPU
 def run_peer_one_gpu(args):
     """The multi-GPU exchange's kernels with the w ranks as contexts on one GPU.
 
@@ -668,6 +668,7 @@ def run_peer_one_gpu(args):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- reference arm
 def run_reference(args):
     rank, _, world = env_rank()
     if rank != 0:
