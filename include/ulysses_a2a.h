@@ -106,21 +106,33 @@ typedef struct ulysses_a2a_plan_t {
 } ulysses_a2a_plan_t;
 
 /* One call's arguments, for ulysses_a2a_run_ex / ulysses_a2a_plan_ex. Same
- * meaning as the ulysses_a2a_run parameters, plus row_pitch: the number of
- * elements between consecutive (b, s) rows of the [B, S_local, H, D] side (the
- * inputs in mode 0, the outputs in mode 1), whose planes are then
- * S_local*row_pitch elements apart; 0 means dense (H*D). A pitch > H*D lets
- * mode 0 read q, k or v in place from a packed [B, S_local, 3, H, D] projection
- * output (row_pitch = 3*H*D, slab pointers offset by 0, H*D or 2*H*D
- * elements), and lets mode 1 write into such a packed buffer; elements between
- * H*D and row_pitch are neither read nor written. The other side is always
- * dense. */
+ * meaning as the ulysses_a2a_run parameters, plus:
+ *
+ * row_pitch: the number of elements between consecutive (b, s) rows of the
+ * [B, S_local, H, D] side (the inputs in mode 0, the outputs in mode 1), whose
+ * planes are then S_local*row_pitch elements apart; 0 means dense. A pitch
+ * > H*D lets mode 0 read q, k or v in place from a packed [B, S_local, 3, H, D]
+ * projection output (row_pitch = 3*H*D, slab pointers offset by 0, H*D or
+ * 2*H*D elements), and lets mode 1 write into such a packed buffer; elements
+ * between H*D and row_pitch are neither read nor written. The other side is
+ * always dense.
+ *
+ * ntensors: 0 or 1 for one tensor per rank. T > 1 re-lays out T tensors packed
+ * along the head dimension in one launch (for example q, k and v of a
+ * [B, S_local, 3, H, D] projection output): the [B, S_local, T, H, D] side has
+ * w slabs (rows of T*H*D elements, or row_pitch), the other side T*w dense
+ * [B, S_local*w, H/w, D] slabs ordered tensor-major, slab t*w + r being
+ * tensor t's slab of rank r:
+ *   mode 0: out[t*w + r][b, j*S_local + s, h', d] = in[j][b, s, t, r*(H/w) + h', d]
+ *   mode 1: out[j][b, s, t, r*(H/w) + h', d]     = in[t*w + r][b, j*S_local + s, h', d]
+ * Equal to T separate calls on the row-pitched views of each tensor. Needs
+ * T*w <= ULYSSES_A2A_MAX_W and chunked 0 or 1; uses the VEC path. */
 typedef struct ulysses_a2a_desc_t {
     const void *const *in_slabs;
     void *const *out_slabs;
     int64_t B, S_local, H, D;
     int32_t w, mode, chunked;
-    int32_t reserved;        /* must be 0 */
+    int32_t ntensors;        /* 0 or 1: one tensor; T > 1: head-packed tensors */
     int64_t row_pitch;
 } ulysses_a2a_desc_t;
 

@@ -159,6 +159,61 @@ class UlyssesA2A:
         self._check(rc)
         return out
 
+    def run_packed(self, xs, mode: int, chunked: bool = False, out=None, stream=None):
+        """Re-layout T tensors packed along the head dimension in one launch.
+
+        mode 0: ``xs`` is w contiguous tensors [B, S_local, T, H, D] (for example
+        a packed q/k/v projection output per rank); returns T lists of w
+        tensors [B, S_local*w, H//w, D] (list t holds tensor t of every rank).
+        mode 1: ``xs`` is T lists of w tensors [B, S_local*w, H//w, D]; returns
+        w tensors [B, S_local, T, H, D]. Same bytes as T calls of ``run`` on
+        the per-tensor views; one kernel launch (VEC path).
+        """
+        if mode not in (0, 1):
+            raise ValueError("mode must be 0 or 1")
+        if mode == 0:
+            w = len(xs)
+            if w < 1 or xs[0].dim() != 5:
+                raise ValueError("mode 0 takes w tensors [B, S_local, T, H, D]")
+            B, S, T, H, D = (int(v) for v in xs[0].shape)
+            if H % w:
+                raise ValueError("H must be divisible by w")
+            ins = list(xs)
+            shape_out = (B, S * w, H // w, D)
+            if out is None:
+                out = [[torch.empty(shape_out, dtype=xs[0].dtype, device=xs[0].device)
+                        for _ in range(w)] for _ in range(T)]
+            flat_out = [o for per_t in out for o in per_t]
+            checks = [(t, (B, S, T, H, D)) for t in ins] + [(o, shape_out) for o in flat_out]
+        else:
+            T = len(xs)
+            w = len(xs[0]) if T else 0
+            if T < 1 or w < 1 or xs[0][0].dim() != 4:
+                raise ValueError("mode 1 takes T lists of w tensors [B, S_local*w, H/w, D]")
+            B, Sg, Hw, D = (int(v) for v in xs[0][0].shape)
+            if Sg % w:
+                raise ValueError("S_local*w must be divisible by w")
+            S, H = Sg // w, Hw * w
+            ins = [x for per_t in xs for x in per_t]
+            if out is None:
+                out = [torch.empty((B, S, T, H, D), dtype=ins[0].dtype, device=ins[0].device)
+                       for _ in range(w)]
+            flat_out = list(out)
+            checks = [(t, (B, Sg, Hw, D)) for t in ins] + [(o, (B, S, T, H, D)) for o in flat_out]
+        for t, shape in checks:
+            if (tuple(t.shape) != shape or t.dtype != ins[0].dtype or t.device.type != "cuda"
+                    or not t.is_contiguous() or t.element_size() != self.elem_bytes):
+                raise ValueError(f"every slab must be a contiguous {shape} CUDA tensor of "
+                                 f"{self.elem_bytes}-byte elements")
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        rc = _lib.ulysses_a2a_run_ex(self._ctx, [t.data_ptr() or 0 for t in ins],
+                                     [o.data_ptr() or 0 for o in flat_out], B, S, H, D, w, mode,
+                                     int(chunked), 0, handle, ntensors=T)
+        self._check(rc)
+        return out
+
     def run_host(self, xs, mode: int, chunked: bool = False, out=None, stream=None):
         """Same op on host slabs: H2D copies, the kernel, D2H copies; returns when done."""
         w, (B, S, H, D), out = self._prepare(xs, mode, out, "cpu")

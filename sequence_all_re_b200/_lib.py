@@ -127,19 +127,19 @@ class DescT(ctypes.Structure):
         ("w", ctypes.c_int32),
         ("mode", ctypes.c_int32),
         ("chunked", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("ntensors", ctypes.c_int32),
         ("row_pitch", ctypes.c_int64),
     ]
 
 
-def make_desc(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, row_pitch=0):
+def make_desc(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, row_pitch=0, ntensors=0):
     """A DescT plus the pointer arrays it references (keep both alive together)."""
     ins = ptr_array(in_ptrs) if in_ptrs is not None else None
     outs = ptr_array(out_ptrs) if out_ptrs is not None else None
     d = DescT(ctypes.cast(ins, ctypes.POINTER(ctypes.c_void_p)) if ins is not None else None,
               ctypes.cast(outs, ctypes.POINTER(ctypes.c_void_p)) if outs is not None else None,
-              int(B), int(S_local), int(H), int(D), int(w), int(mode), int(chunked), 0,
-              int(row_pitch))
+              int(B), int(S_local), int(H), int(D), int(w), int(mode), int(chunked),
+              int(ntensors), int(row_pitch))
     return d, (ins, outs)
 
 
@@ -306,15 +306,16 @@ def ulysses_a2a_plan(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, elem
 
 
 def ulysses_a2a_run_ex(ctx, in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, row_pitch,
-                       stream) -> int:
-    d, keep = make_desc(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, row_pitch)
+                       stream, ntensors=0) -> int:
+    d, keep = make_desc(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, row_pitch, ntensors)
     return lib.ulysses_a2a_run_ex(ctx, ctypes.byref(d), ctypes.c_void_p(int(stream)))
 
 
 def ulysses_a2a_plan_ex(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, elem_bytes,
-                        row_pitch=0, forced_path=PATH_AUTO, num_sms=148, **knobs):
+                        row_pitch=0, forced_path=PATH_AUTO, num_sms=148, ntensors=0, **knobs):
     """Host-only planning of a descriptor (no CUDA call). Returns (rc, PlanT, message)."""
-    d, keep = make_desc(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, row_pitch)
+    d, keep = make_desc(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, row_pitch,
+                        ntensors)
     plan = PlanT()
     buf = ctypes.create_string_buffer(256)
     t = TuningT.make(**knobs)

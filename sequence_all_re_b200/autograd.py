@@ -44,6 +44,36 @@ def all_to_all_4d(a2a: UlyssesA2A, xs, mode: int, chunked: bool = False) -> list
     return list(UlyssesAllToAll4D.apply(a2a, int(mode), bool(chunked), *xs))
 
 
+class UlyssesAllToAll4DPacked(torch.autograd.Function):
+    """forward: mode 0 of w head-packed [B, S, T, H, D] slabs (one launch);
+    backward: the packed mode 1 of the T*w output gradients."""
+
+    @staticmethod
+    def forward(ctx, a2a: UlyssesA2A, chunked: bool, *xs):
+        ctx.a2a = a2a
+        ctx.chunked = bool(chunked)
+        ctx.w = len(xs)
+        outs = a2a.run_packed(list(xs), 0, chunked=ctx.chunked)
+        ctx.T = len(outs)
+        return tuple(o for per_t in outs for o in per_t)
+
+    @staticmethod
+    def backward(ctx, *grads):
+        ref = next(g for g in grads if g is not None)
+        gs = [(g if g is not None else torch.zeros_like(ref)).contiguous() for g in grads]
+        per_t = [gs[t * ctx.w:(t + 1) * ctx.w] for t in range(ctx.T)]
+        gin = ctx.a2a.run_packed(per_t, 1, chunked=ctx.chunked)
+        return (None, None, *gin)
+
+
+def all_to_all_4d_packed(a2a: UlyssesA2A, xs, chunked: bool = False) -> list:
+    """Differentiable mode-0 re-layout of w head-packed slabs [B, S, T, H, D];
+    returns T lists of w slabs (see UlyssesA2A.run_packed)."""
+    outs = UlyssesAllToAll4DPacked.apply(a2a, bool(chunked), *xs)
+    w = len(xs)
+    return [list(outs[t * w:(t + 1) * w]) for t in range(len(outs) // w)]
+
+
 class PeerAllToAll4D(torch.autograd.Function):
     """forward: this rank's mode-`mode` exchange; backward: the inverse-mode exchange
     of the output gradient (every rank runs it, in the same order)."""

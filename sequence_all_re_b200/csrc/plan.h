@@ -150,11 +150,15 @@ inline bool tuning_from(const ulysses_a2a_tuning_t* t, Tuning* out, std::string*
 // only_out >= 0: the call writes output slab only_out alone (VEC path); the
 // other out[] entries are neither checked nor used, and units counts that
 // slab's blocks only.
+// ntensors = T > 1: T tensors packed along the head dimension of the
+// [B, S, H, D] side ([B, S, T, H, D], rows of T*H*D elements), re-laid out in
+// one launch (VEC path). That side then has w slabs and the other T*w, tensor-
+// major: slab t*w + r is tensor t's [B, S*w, H/w, D] slab of rank r.
 inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t S,
                      int64_t H, int64_t D, int w, int mode, int chunked, int E,
                      int forced_path, const Tuning& tune, int num_sms,
                      ulysses_a2a_plan_t* p, std::string* err, int64_t row_pitch = 0,
-                     int only_out = -1) {
+                     int only_out = -1, int ntensors = 1) {
   if (p == nullptr) { set_err(err, "plan output is NULL"); return ULYSSES_A2A_ERR_INVALID; }
   *p = ulysses_a2a_plan_t{};
   if (in == nullptr || out == nullptr) {
@@ -174,6 +178,15 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     set_err(err, "one-output plan: slab %lld of %lld, VEC path required", only_out, w);
     return ULYSSES_A2A_ERR_INVALID;
   }
+  if (ntensors < 1 || (int64_t)ntensors * w > ULYSSES_A2A_MAX_W || (ntensors > 1 && only_out >= 0)) {
+    set_err(err, "ntensors=%lld: need 1 <= ntensors and ntensors*w <= %lld", ntensors,
+            ULYSSES_A2A_MAX_W);
+    return ULYSSES_A2A_ERR_INVALID;
+  }
+  if (ntensors > 1 && chunked == 2) {
+    set_err(err, "packed tensors are not staged through the window (chunked must be 0 or 1)");
+    return ULYSSES_A2A_ERR_UNSUPPORTED;
+  }
   if (chunked < 0 || chunked > 2) { set_err(err, "chunked=%lld not 0, 1 or 2", chunked); return ULYSSES_A2A_ERR_INVALID; }
   if (B < 0 || S < 0 || H < 0 || D < 0) {
     set_err(err, "sizes must be >= 0 (B, S_local, H, D)");
@@ -188,7 +201,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
       return ULYSSES_A2A_ERR_INVALID;
     }
     p->path = forced_path == ULYSSES_A2A_PATH_AUTO ? ULYSSES_A2A_PATH_VEC : forced_path;
-    p->row_pitch = row_pitch > 0 ? row_pitch : H * D;
+    p->row_pitch = row_pitch > 0 ? row_pitch : (int64_t)ntensors * H * D;
     return ULYSSES_A2A_OK;
   }
   if (forced_path < ULYSSES_A2A_PATH_AUTO || forced_path > ULYSSES_A2A_PATH_VEC) {
@@ -198,48 +211,60 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
   if (num_sms < 1) { set_err(err, "num_sms must be >= 1"); return ULYSSES_A2A_ERR_INVALID; }
 
   // sizes, overflow-checked
-  int64_t plane_elems, slab_elems, slab_bytes, payload, tmp, HD;
+  int64_t plane_elems, slab_elems, slab_bytes, payload, tmp, HD, HDp;
   if (mul_overflows(S, H, &tmp) || mul_overflows(tmp, D, &plane_elems) ||
       mul_overflows(plane_elems, B, &slab_elems) || mul_overflows(slab_elems, E, &slab_bytes) ||
-      mul_overflows(slab_bytes, (int64_t)w, &payload) || payload > (int64_t(1) << 56) ||
-      mul_overflows(H, D, &HD)) {
+      mul_overflows(slab_bytes, (int64_t)w * ntensors, &payload) || payload > (int64_t(1) << 56) ||
+      mul_overflows(H, D, &HD) || mul_overflows(HD, (int64_t)ntensors, &HDp)) {
     set_err(err, "slab sizes overflow");
     return ULYSSES_A2A_ERR_INVALID;
   }
-  const int64_t pitch = row_pitch == 0 ? HD : row_pitch;
-  if (pitch < HD) {
-    set_err(err, "row pitch %lld is smaller than H*D = %lld", pitch, HD);
+  // HDp: elements of one (b, s) row of the [B, S, (T,) H, D] side
+  const int64_t pitch = row_pitch == 0 ? HDp : row_pitch;
+  if (pitch < HDp) {
+    set_err(err, "row pitch %lld is smaller than a row (%lld elements)", pitch, HDp);
     return ULYSSES_A2A_ERR_INVALID;
   }
   // bytes spanned by one slab of the [B, S, H, D] side (gaps included)
   int64_t strided_bytes;
-  if (mul_overflows(B * S - 1, pitch, &tmp) || mul_overflows(tmp + HD, (int64_t)E, &strided_bytes) ||
+  if (mul_overflows(B * S - 1, pitch, &tmp) || mul_overflows(tmp + HDp, (int64_t)E, &strided_bytes) ||
       strided_bytes > (int64_t(1) << 56)) {
     set_err(err, "pitched slab extent overflows");
     return ULYSSES_A2A_ERR_INVALID;
   }
   const int64_t in_bytes = mode == 0 ? strided_bytes : slab_bytes;
   const int64_t out_bytes = mode == 0 ? slab_bytes : strided_bytes;
+  // slab counts: w on the [B, S, (T,) H, D] side, T*w on the gathered side
+  const int nin = mode == 0 ? w : w * ntensors;
+  const int nout = mode == 0 ? w * ntensors : w;
   auto used_out = [&](int k) { return only_out < 0 || k == only_out; };
-  for (int k = 0; k < w; ++k) {
-    if (in[k] == nullptr || (used_out(k) && out[k] == nullptr)) {
-      set_err(err, "slab pointer %lld is NULL", k);
+  for (int k = 0; k < nin; ++k) {
+    if (in[k] == nullptr) {
+      set_err(err, "input slab pointer %lld is NULL", k);
+      return ULYSSES_A2A_ERR_INVALID;
+    }
+  }
+  for (int k = 0; k < nout; ++k) {
+    if (used_out(k) && out[k] == nullptr) {
+      set_err(err, "output slab pointer %lld is NULL", k);
       return ULYSSES_A2A_ERR_INVALID;
     }
   }
   // No output may overlap an input or another output (inputs may alias each
   // other). A pitched slab counts with its whole extent, gaps included.
-  for (int k = 0; k < w; ++k) {
+  for (int k = 0; k < nout; ++k) {
     if (!used_out(k)) continue;
     const uintptr_t o = reinterpret_cast<uintptr_t>(out[k]);
     const uintptr_t oe = o + (uintptr_t)out_bytes;
     if (oe < o) { set_err(err, "output slab %lld wraps the address space", k); return ULYSSES_A2A_ERR_INVALID; }
-    for (int m = 0; m < w; ++m) {
+    for (int m = 0; m < nin; ++m) {
       const uintptr_t i = reinterpret_cast<uintptr_t>(in[m]);
       if (overlaps(o, oe, i, i + (uintptr_t)in_bytes)) {
         set_err(err, "output slab %lld overlaps input slab %lld", k, m);
         return ULYSSES_A2A_ERR_OVERLAP;
       }
+    }
+    for (int m = 0; m < nout; ++m) {
       if (m != k && used_out(m)) {
         const uintptr_t q = reinterpret_cast<uintptr_t>(out[m]);
         if (overlaps(o, oe, q, q + (uintptr_t)out_bytes)) {
@@ -252,8 +277,9 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
 
   const int64_t Hw = H / w;
   const int64_t row_bytes = Hw * D * E;  // one contiguous run, L*E
-  const char* blocker = only_out >= 0 ? "one-output launches use the VEC path"
-                                      : tma_blocker(in, out, B, S, H, D, w, E, row_bytes, pitch);
+  const char* blocker = only_out >= 0   ? "one-output launches use the VEC path"
+                        : ntensors > 1 ? "packed launches use the VEC path"
+                                       : tma_blocker(in, out, B, S, H, D, w, E, row_bytes, pitch);
   int path;
   if (forced_path == ULYSSES_A2A_PATH_TMA) {
     if (blocker) {
@@ -279,7 +305,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
 
   const int64_t T = (S + rows - 1) / rows;  // ceil-div: the ragged last tile is a unit too
   const int64_t nb = chunked ? 1 : B;
-  const int64_t blocks_wide = only_out >= 0 ? (int64_t)w : (int64_t)w * w;
+  const int64_t blocks_wide = only_out >= 0 ? (int64_t)w : (int64_t)w * w * ntensors;
   int64_t units;
   if (mul_overflows(blocks_wide, nb, &tmp) || mul_overflows(tmp, T, &units)) {
     set_err(err, "unit count overflows");
@@ -375,9 +401,9 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     int v = 16;
     while (v > 1) {
       bool ok = (row_bytes % v) == 0 && ((pitch * E) % v) == 0;
-      for (int k = 0; k < w && ok; ++k)
-        ok = (reinterpret_cast<uintptr_t>(in[k]) % v) == 0 &&
-             (!used_out(k) || (reinterpret_cast<uintptr_t>(out[k]) % v) == 0);
+      for (int k = 0; k < nin && ok; ++k) ok = (reinterpret_cast<uintptr_t>(in[k]) % v) == 0;
+      for (int k = 0; k < nout && ok; ++k)
+        ok = !used_out(k) || (reinterpret_cast<uintptr_t>(out[k]) % v) == 0;
       if (ok) break;
       v >>= 1;
     }

@@ -305,19 +305,20 @@ cudaError_t launch_vec(const VecParams& p, int vec_bytes, int mode, int grid, in
 // Launch the planned kernel(s) for tiles [tile0, tile0 + ntiles) of every
 // (r, b, j) block (ntiles < 0: the whole block). only_out >= 0 (VEC path
 // only) restricts the launch to the blocks of output slab only_out: r fixed in
-// mode 0, j fixed in mode 1.
+// mode 0, j fixed in mode 1. ntensors > 1 (VEC path only): head-packed
+// tensors, r ranging over ntensors*w head groups.
 int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, int64_t B, int64_t S,
                int64_t H, int64_t D, int w, int mode, int chunked, cudaStream_t st,
                const ulysses_a2a_plan_t& pl, int64_t tile0 = 0, int64_t ntiles = -1,
-               int only_out = -1) {
+               int only_out = -1, int ntensors = 1) {
   const int64_t nb = chunked ? 1 : B;
   const int launches = chunked ? (int)B : 1;
   const int64_t nt = ntiles < 0 ? pl.tiles_per_block : ntiles;
-  const int nr = (only_out >= 0 && mode == 0) ? 1 : w;
+  const int nr = (only_out >= 0 && mode == 0) ? 1 : w * ntensors;
   const int nj = (only_out >= 0 && mode == 1) ? 1 : w;
   const int64_t units = (int64_t)nr * nb * nj * nt;
-  if (only_out >= 0 && pl.path != ULYSSES_A2A_PATH_VEC)
-    return fail(ctx, ULYSSES_A2A_ERR_UNSUPPORTED, "one-output launches use the VEC path");
+  if ((only_out >= 0 || ntensors > 1) && pl.path != ULYSSES_A2A_PATH_VEC)
+    return fail(ctx, ULYSSES_A2A_ERR_UNSUPPORTED, "one-output and packed launches use the VEC path");
   int grid = pl.grid;
   if (nt != pl.tiles_per_block) {
     if (pl.path == ULYSSES_A2A_PATH_TMA && pl.chunk_units > 0)
@@ -358,10 +359,10 @@ int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, in
     return ULYSSES_A2A_OK;
   }
   VecParams p{};
-  for (int k = 0; k < w; ++k) {
-    p.in[k] = static_cast<const char*>(in[k]);
-    p.out[k] = static_cast<char*>(out[k]);
-  }
+  const int nin = mode == 0 ? w : w * ntensors;
+  const int nout = mode == 0 ? w * ntensors : w;
+  for (int k = 0; k < nin; ++k) p.in[k] = static_cast<const char*>(in[k]);
+  for (int k = 0; k < nout; ++k) p.out[k] = static_cast<char*>(out[k]);
   p.S_local = S;
   p.nv = pl.row_bytes / pl.vec_bytes;
   p.srow = pl.row_pitch * ctx->elem_bytes / pl.vec_bytes;
@@ -388,10 +389,10 @@ int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, in
 
 int plan_for(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, int64_t B, int64_t S,
              int64_t H, int64_t D, int w, int mode, int chunked, ulysses_a2a_plan_t* pl,
-             int64_t row_pitch = 0) {
+             int64_t row_pitch = 0, int ntensors = 1) {
   std::string err;
   int rc = ua2a::make_plan(in, out, B, S, H, D, w, mode, chunked, ctx->elem_bytes, ctx->forced_path,
-                           ctx->tuning, ctx->num_sms, pl, &err, row_pitch);
+                           ctx->tuning, ctx->num_sms, pl, &err, row_pitch, -1, ntensors);
   if (rc) return fail(ctx, rc, err);
   return ULYSSES_A2A_OK;
 }
@@ -567,27 +568,31 @@ static int ua2a_impl_run_ex(ulysses_a2a_ctx* ctx, const ulysses_a2a_desc_t* d, v
   if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
   ctx->last_error.clear();
   if (d == nullptr) return fail(ctx, ULYSSES_A2A_ERR_INVALID, "descriptor is NULL");
-  if (d->reserved != 0 || d->row_pitch < 0)
-    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "descriptor: reserved must be 0, row_pitch >= 0");
+  if (d->ntensors < 0 || d->row_pitch < 0)
+    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "descriptor: ntensors and row_pitch must be >= 0");
+  const int T = d->ntensors > 1 ? d->ntensors : 1;
   ulysses_a2a_plan_t pl;
   int rc = plan_for(ctx, d->in_slabs, d->out_slabs, d->B, d->S_local, d->H, d->D, d->w, d->mode,
-                    d->chunked, &pl, d->row_pitch);
+                    d->chunked, &pl, d->row_pitch, T);
   if (rc) return rc;
   if (pl.units == 0) return ULYSSES_A2A_OK;  // empty: nothing to do
   DeviceGuard g(ctx->device);
   if (!g.ok) return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "cannot select the context's device");
-  const int64_t dense_bytes = pl.payload_bytes / d->w;
-  const int64_t strided_bytes = ((d->B * d->S_local - 1) * pl.row_pitch + d->H * d->D) *
+  // one [B, S*w, H/w, D] slab, and one (pitched, T-packed) [B, S, (T,) H, D] slab
+  const int64_t dense_bytes = pl.payload_bytes / ((int64_t)d->w * T);
+  const int64_t strided_bytes = ((d->B * d->S_local - 1) * pl.row_pitch + (int64_t)T * d->H * d->D) *
                                 (int64_t)ctx->elem_bytes;
-  rc = check_residency(ctx, d->in_slabs, d->w, d->mode == 0 ? strided_bytes : dense_bytes, "input");
+  const int nin = d->mode == 0 ? d->w : d->w * T;
+  const int nout = d->mode == 0 ? d->w * T : d->w;
+  rc = check_residency(ctx, d->in_slabs, nin, d->mode == 0 ? strided_bytes : dense_bytes, "input");
   if (rc) return rc;
-  rc = check_residency(ctx, reinterpret_cast<const void* const*>(d->out_slabs), d->w,
+  rc = check_residency(ctx, reinterpret_cast<const void* const*>(d->out_slabs), nout,
                        d->mode == 0 ? dense_bytes : strided_bytes, "output");
   if (rc) return rc;
   if (d->chunked == ULYSSES_A2A_CHUNKED_WINDOW)
     return run_windowed(ctx, d, pl, static_cast<cudaStream_t>(stream));
   return run_device(ctx, d->in_slabs, d->out_slabs, d->B, d->S_local, d->H, d->D, d->w, d->mode,
-                    d->chunked, static_cast<cudaStream_t>(stream), pl);
+                    d->chunked, static_cast<cudaStream_t>(stream), pl, 0, -1, -1, T);
 }
 
 static int ua2a_impl_run(ulysses_a2a_ctx* ctx, const void* const* in_slabs, void* const* out_slabs,
@@ -830,14 +835,15 @@ static int ua2a_impl_plan_ex(const ulysses_a2a_desc_t* d, int elem_bytes, int fo
   if (d == nullptr) {
     msg = "descriptor is NULL";
     rc = ULYSSES_A2A_ERR_INVALID;
-  } else if (d->reserved != 0 || d->row_pitch < 0) {
-    msg = "descriptor: reserved must be 0, row_pitch >= 0";
+  } else if (d->ntensors < 0 || d->row_pitch < 0) {
+    msg = "descriptor: ntensors and row_pitch must be >= 0";
     rc = ULYSSES_A2A_ERR_INVALID;
   } else if (!ua2a::tuning_from(tuning, &t, &msg)) {
     rc = ULYSSES_A2A_ERR_INVALID;
   } else {
     rc = ua2a::make_plan(d->in_slabs, d->out_slabs, d->B, d->S_local, d->H, d->D, d->w, d->mode,
-                         d->chunked, elem_bytes, forced_path, t, num_sms, out, &msg, d->row_pitch);
+                         d->chunked, elem_bytes, forced_path, t, num_sms, out, &msg, d->row_pitch,
+                         -1, d->ntensors > 1 ? d->ntensors : 1);
   }
   if (err && errlen) std::snprintf(err, errlen, "%s", rc ? msg.c_str() : "");
   return rc;

@@ -447,3 +447,49 @@ def test_valid_environment_override_is_accepted(monkeypatch):
 
 def test_get_settings_rejects_null_context():
     assert _lib.lib.ulysses_a2a_get_settings(None, None, None) == ERR_INVALID
+
+
+# ---- head-packed tensors in one launch (ntensors) -----------------------------
+
+def packed_plan(T, w, B, S, H, D, mode=0, chunked=0, E=2, **kw):
+    P = B * S * H * D * E
+    strided = [(1 << 40) + k * (1 << 32) for k in range(w)]
+    # the gathered side has max(T, 1) * w slabs (ntensors 0 means one tensor)
+    gathered = [(1 << 44) + k * (1 << 32) for k in range(max(T, 1) * w)]
+    ins, outs = (strided, gathered) if mode == 0 else (gathered, strided)
+    return _lib.ulysses_a2a_plan_ex(ins, outs, B, S, H, D, w, mode, chunked, E, ntensors=T, **kw)
+
+
+def test_packed_plan_geometry():
+    rc, p, msg = packed_plan(3, 4, 2, 8192, 24, 128)
+    assert rc == OK, msg
+    assert p.path == PATH_VEC and p.row_bytes == 6 * 128 * 2
+    assert p.row_pitch == 3 * 24 * 128                    # one packed row holds q, k and v
+    assert p.units == 3 * 4 * 4 * 2 * p.tiles_per_block    # T*w head groups x w blocks x planes
+    assert p.payload_bytes == 3 * 4 * 2 * 8192 * 24 * 128 * 2
+    # ntensors 0 and 1 both mean one tensor, and plan exactly as before
+    rc0, p0, _ = packed_plan(0, 4, 2, 8192, 24, 128)
+    rc1, p1, _ = packed_plan(1, 4, 2, 8192, 24, 128)
+    rcp, pp, _ = plan(4, 2, 8192, 24, 128)
+    assert rc0 == rc1 == rcp == OK and p0.as_dict() == p1.as_dict() == pp.as_dict()
+
+
+def test_packed_plan_validation():
+    assert packed_plan(17, 4, 1, 64, 8, 64)[0] == ERR_INVALID        # T*w > 64
+    assert packed_plan(-1, 4, 1, 64, 8, 64)[0] == ERR_INVALID
+    assert packed_plan(3, 4, 1, 64, 8, 64, chunked=2)[0] == ERR_UNSUPPORTED
+    rc, _, msg = packed_plan(3, 4, 1, 64, 8, 64, forced_path=PATH_TMA)
+    assert rc == ERR_UNSUPPORTED and "packed" in msg
+    # two gathered slabs of different tensors overlapping
+    w, T, B, S, H, D = 2, 3, 1, 64, 4, 64
+    slab = B * S * H * D * 2
+    strided = [(1 << 40) + k * (1 << 32) for k in range(w)]
+    gathered = [(1 << 44) + k * (1 << 32) for k in range(T * w)]
+    gathered[5] = gathered[1] + slab // 2
+    rc, _, msg = _lib.ulysses_a2a_plan_ex(strided, gathered, B, S, H, D, w, 0, 0, 2, ntensors=T)
+    assert rc == ERR_OVERLAP
+    # a NULL among the T*w mode-1 inputs
+    gathered = [(1 << 44) + k * (1 << 32) for k in range(T * w)]
+    gathered[4] = 0
+    rc, _, msg = _lib.ulysses_a2a_plan_ex(gathered, strided, B, S, H, D, w, 1, 0, 2, ntensors=T)
+    assert rc == ERR_INVALID and "NULL" in msg

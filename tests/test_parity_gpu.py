@@ -787,3 +787,60 @@ def test_environment_overrides_set_the_initial_knobs(monkeypatch):
         assert a2a.settings() == (PATH_AUTO, dict(_lib.TuningT.DEFAULTS))
         assert a2a.plan([t.cuda() for t in xs], 0)["path"] == PATH_TMA
         del out
+
+
+# ---- head-packed tensors in one launch ---------------------------------------
+
+PACKED = [
+    # (T, w, B, S_local, H, D)
+    (3, 4, 2, 37, 8, 64),       # q, k, v; ragged S_local
+    (2, 2, 1, 100, 4, 128),
+    (3, 8, 1, 53, 40, 128),     # cfg3's head geometry
+    (3, 4, 2, 19, 4, 13),       # odd D: narrow vectors
+    (1, 4, 1, 64, 8, 64),       # T = 1: the plain re-layout
+]
+
+
+@pytest.mark.parametrize("case", PACKED, ids=lambda c: "T{}w{}B{}S{}H{}D{}".format(*c))
+@pytest.mark.parametrize("chunked", [False, True], ids=["whole", "per_plane"])
+def test_packed_tensors_in_one_launch(case, chunked):
+    T, w, B, S, H, D = case
+    packed_cpu = normal_slabs((B, S, T, H, D), w, "bf16", seed0=900 + T)
+    flat = [t.reshape(-1) for t in packed_cpu]
+    with UlyssesA2A(0, 2) as a2a:
+        packed = [t.cuda() for t in packed_cpu]
+        n0 = a2a.launch_count
+        outs = a2a.run_packed(packed, 0, chunked=chunked)
+        assert a2a.launch_count - n0 == (B if chunked else 1)
+        for t in range(T):
+            # tensor t of the packed slabs: a row-pitched view, T*H*D between rows
+            want = oracle.ulysses_a2a_pitched(flat, 0, w, B, S, H, D, T * H * D, offset=t * H * D)
+            for r in range(w):
+                assert torch.equal(bits(outs[t][r].cpu()).reshape(-1), bits(want[r])), (t, r)
+        # mode 1 back into poisoned packed buffers, one launch (per plane when chunked)
+        back = [torch.full((B, S, T, H, D), -1, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+                for _ in range(w)]
+        n1 = a2a.launch_count
+        a2a.run_packed(outs, 1, chunked=chunked, out=back)
+        a2a.status()
+        assert a2a.launch_count - n1 == (B if chunked else 1)
+        for j in range(w):
+            assert torch.equal(bits(back[j].cpu()), bits(packed_cpu[j])), j
+
+
+def test_packed_autograd_backward_is_packed_mode1():
+    from sequence_all_re_b200.autograd import all_to_all_4d_packed
+
+    T, w, B, S, H, D = 3, 4, 1, 45, 8, 64
+    packed_cpu = normal_slabs((B, S, T, H, D), w, "bf16", seed0=950)
+    gys = [uniform_slabs((B, S * w, H // w, D), w, "bf16", seed0=960 + t) for t in range(T)]
+    with UlyssesA2A(0, 2) as a2a:
+        xs = [t.cuda().requires_grad_() for t in packed_cpu]
+        outs = all_to_all_4d_packed(a2a, xs)
+        torch.autograd.backward([o for per_t in outs for o in per_t],
+                                [g.cuda() for per_t in gys for g in per_t])
+        # the gradient of packed slab j: tensor t's mode-1 result in slot t
+        for t in range(T):
+            want = oracle.ulysses_a2a(gys[t], 1)
+            for j in range(w):
+                assert torch.equal(bits(xs[j].grad[:, :, t].cpu().contiguous()), bits(want[j]))
