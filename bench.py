@@ -42,14 +42,19 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "payload GB/s and % of HBM roofline (2x bytes) per mode at w=2/4/8, 1xB200"
-# The benchmark configurations (bf16, N(0,1) values); cfg2 is the default workload.
+# The benchmark workloads (bf16, N(0,1) values), named by their sizes:
+#   w2_S64_H4_D64          a tiny round trip (B = 1);
+#   w4_S8192_H24_D128      the default, 192 MiB per call (B = 1);
+#   w8_B2_S4725_H40_D128   a ragged sequence tail (4725 = 787 x 6 + 3), 774 MB;
+#   w4_B4_S16384_H32_D64   four planes, for the chunked per-plane variant, 1 GiB.
+DEFAULT_WORKLOAD = "w4_S8192_H24_D128"
 WORKLOADS = {
-    "cfg1": dict(w=2, B=1, S_local=64, H=4, D=64),
-    "cfg2": dict(w=4, B=1, S_local=8192, H=24, D=128),
-    "cfg3": dict(w=8, B=2, S_local=4725, H=40, D=128),
-    "cfg4": dict(w=4, B=4, S_local=16384, H=32, D=64),
+    "w2_S64_H4_D64": dict(w=2, B=1, S_local=64, H=4, D=64),
+    "w4_S8192_H24_D128": dict(w=4, B=1, S_local=8192, H=24, D=128),
+    "w8_B2_S4725_H40_D128": dict(w=8, B=2, S_local=4725, H=40, D=128),
+    "w4_B4_S16384_H32_D64": dict(w=4, B=4, S_local=16384, H=32, D=64),
 }
-WORKLOAD = WORKLOADS["cfg2"]
+WORKLOAD = WORKLOADS[DEFAULT_WORKLOAD]
 
 
 def workload_key(w, B, S, H, D, path):
@@ -740,8 +745,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="cfg2",
-                    help="benchmark configuration (default cfg2: w=4, S_local=8192, H=24, D=128)")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD,
+                    help="benchmark workload, named by its sizes (default %(default)s)")
     ap.add_argument("--path", choices=["auto", "tma", "vec"], default="auto")
     ap.add_argument("--chunked", type=int, choices=[0, 1, 2], default=0)
     ap.add_argument("--sweep", action="store_true",

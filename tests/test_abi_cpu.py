@@ -75,7 +75,7 @@ def plan(w, B, S, H, D, mode=0, chunked=0, E=2, **kw):
 
 # ---- geometry at the benchmark configurations -------------------------------
 
-def test_plan_cfg2_tma():
+def test_plan_default_workload_tma():
     rc, p, msg = plan(4, 1, 8192, 24, 128)
     assert rc == OK, msg
     assert p.path == PATH_TMA
@@ -107,7 +107,7 @@ def test_plan_cfg2_tma():
     assert (q.producers, q.stages, q.lookahead, q.smem_bytes) == (4, 16, 2, 16 * 8 * 1024)
 
 
-def test_plan_cfg3_tail_rows():
+def test_plan_ragged_tail_rows():
     rc, p, _ = plan(8, 2, 4725, 40, 128)
     assert rc == OK and p.path == PATH_TMA
     assert p.row_bytes == 5 * 128 * 2
@@ -124,7 +124,7 @@ def test_plan_cfg3_tail_rows():
     assert rc == OK and p.rows_per_tile == 64 and p.tail_rows == 53
 
 
-def test_plan_cfg4_chunked_launches():
+def test_plan_four_planes_chunked_launches():
     rc, p, _ = plan(4, 4, 16384, 32, 64, chunked=1)
     assert rc == OK and p.path == PATH_TMA
     assert p.launches == 4
@@ -141,7 +141,7 @@ def test_plan_windowed_chunked_variant():
     assert p.units == q.units
 
 
-def test_plan_cfg1_small():
+def test_plan_tiny_workload():
     rc, p, _ = plan(2, 1, 64, 4, 64)
     assert rc == OK and p.path == PATH_TMA
     assert p.rows_per_tile == 32 and p.tail_rows == 0 and p.tiles_per_block == 2

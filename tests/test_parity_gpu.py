@@ -99,7 +99,7 @@ SHAPES = [
     (2, 1, 64, 4, 64),          # the small oracle-size case
     (2, 3, 37, 4, 64),          # ragged S_local, several planes
     (4, 2, 100, 8, 128),
-    (8, 2, 53, 40, 128),        # cfg3's head geometry, short sequence
+    (8, 2, 53, 40, 128),        # the ragged-tail workload's heads, short sequence
     (3, 2, 29, 6, 32),          # odd rank count
     (1, 2, 33, 4, 64),          # w = 1: identity copy
     (8, 1, 7, 8, 256),          # D at the TMA box limit, H/w = 1
@@ -261,10 +261,10 @@ def test_shapes_tma_cannot_express_use_vec():
 # ---- the benchmark's configurations at full size (default launch config) ----
 
 FULL = {
-    "cfg1_w2_S64": (2, 1, 64, 4, 64),
-    "cfg2_w4_S8192": (4, 1, 8192, 24, 128),
-    "cfg3_w8_S4725": (8, 2, 4725, 40, 128),
-    "cfg4_w4_B4_S16384": (4, 4, 16384, 32, 64),
+    "w2_S64_H4_D64": (2, 1, 64, 4, 64),
+    "w4_S8192_H24_D128": (4, 1, 8192, 24, 128),
+    "w8_B2_S4725_H40_D128": (8, 2, 4725, 40, 128),
+    "w4_B4_S16384_H32_D64": (4, 4, 16384, 32, 64),
 }
 
 
@@ -277,7 +277,7 @@ def test_full_size_configs(name):
     if B > 1:
         run_case(xs, 0, chunked=True)
         run_case(y, 1, chunked=True)
-    if name.startswith("cfg3"):
+    if name.startswith("w8_B2_S4725"):
         # the ragged tile: 4725 = 147 * 32 + 21
         run_case(xs, 0, tuning=dict(rows_per_tile=32))
         run_case(y, 1, tuning=dict(rows_per_tile=32), path=PATH_VEC)
@@ -795,7 +795,7 @@ PACKED = [
     # (T, w, B, S_local, H, D)
     (3, 4, 2, 37, 8, 64),       # q, k, v; ragged S_local
     (2, 2, 1, 100, 4, 128),
-    (3, 8, 1, 53, 40, 128),     # cfg3's head geometry
+    (3, 8, 1, 53, 40, 128),     # the ragged-tail workload's heads
     (3, 4, 2, 19, 4, 13),       # odd D: narrow vectors
     (1, 4, 1, 64, 8, 64),       # T = 1: the plain re-layout
 ]
