@@ -673,6 +673,79 @@ def run_peer_one_gpu(args):
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------- head-packed q, k, v in one launch
+def run_packed(args):
+    """q, k and v of the chosen workload's shape, packed [B, S_local, 3, H, D] per
+    rank: one packed launch (run_packed) against three launches on the
+    row-pitched per-tensor views (run), back to back."""
+    from sequence_all_re_b200 import UlyssesA2A
+
+    if args.gpus != 1:
+        raise SystemExit("--packed runs on one GPU")
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    wl = WORKLOADS[args.workload]
+    w, B, S, H, D = (wl[k] for k in ("w", "B", "S_local", "H", "D"))
+    T, E = 3, 2
+    P = T * w * B * S * H * D * E
+    a2a = UlyssesA2A(0, E)
+    stream = torch.cuda.Stream(device)
+    g = torch.Generator(device=device)
+    g.manual_seed(1234)
+    packed = [torch.randn((B, S, T, H, D), generator=g, device=device).to(torch.bfloat16)
+              for _ in range(w)]
+    outs = [[torch.empty((B, S * w, H // w, D), dtype=torch.bfloat16, device=device)
+             for _ in range(w)] for _ in range(T)]
+    ref = [[torch.empty_like(o) for o in per_t] for per_t in outs]
+
+    def one():
+        a2a.run_packed(packed, 0, out=outs, stream=stream)
+
+    def three():
+        for t in range(T):
+            a2a.run([x[:, :, t] for x in packed], 0, out=ref[t], stream=stream)
+
+    def timed(fn, reps):
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                fn()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+            e1.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    reps = min(args.steps, 500)
+    n0 = a2a.launch_count
+    ms_one = timed(one, reps)
+    launches = a2a.launch_count - n0
+    ms_three = timed(three, reps)
+    torch.cuda.synchronize()
+    if not all(torch.equal(outs[t][r], ref[t][r]) for t in range(T) for r in range(w)):
+        raise SystemExit("packed launch differs from the per-tensor launches")
+    peak, peak_src = hbm_peak()
+    line = {
+        "metric": "q, k, v Ulysses re-layout (mode 0) payload throughput: one packed launch",
+        "value": round(P / (ms_one / 1e3) / 1e9, 1), "unit": "GB/s", "n_gpus": 1,
+        "steps": reps, "warmup": args.warmup, "ms_per_step": round(ms_one, 4),
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"q, k, v packed [B, S_local, 3, H, D]: w={w} B={B} "
+                               f"S_local={S} H={H} D={D} bf16, mode 0",
+                   "l2": "inputs larger than L2 (back to back)"},
+        "gpu_launches": launches,
+        "frac_of_copy": round(2 * P / (ms_one / 1e3) / 1e9 / peak, 4),
+        "three_launches": {"ms": round(ms_three, 4),
+                           "value": round(P / (ms_three / 1e3) / 1e9, 1),
+                           "frac_of_copy": round(2 * P / (ms_three / 1e3) / 1e9 / peak, 4)},
+        "peak_source": peak_src,
+    }
+    a2a.close()
+    print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------- reference arm
 def run_reference(args):
     rank, _, world = env_rank()
@@ -751,6 +824,9 @@ def main():
     ap.add_argument("--chunked", type=int, choices=[0, 1, 2], default=0)
     ap.add_argument("--sweep", action="store_true",
                     help="also run the 128 KiB..2 GiB bandwidth sweep (w=2/4/8, bf16/fp32)")
+    ap.add_argument("--packed", action="store_true",
+                    help="time q, k, v in one packed launch against three per-tensor launches "
+                         "(prints its own line)")
     ap.add_argument("--peer-one-gpu", action="store_true",
                     help="time the multi-GPU exchange's publish and pull kernels with the w "
                          "ranks as contexts on one GPU (prints its own line)")
@@ -762,6 +838,8 @@ def main():
         run_reference(args)
     elif args.peer_one_gpu:
         run_peer_one_gpu(args)
+    elif args.packed:
+        run_packed(args)
     else:
         run_ours(args)
 
