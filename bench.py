@@ -626,11 +626,14 @@ def run_peer_one_gpu(args):
     if not all(torch.equal(z[k], x[k]) for k in range(w)):
         raise SystemExit("round trip mismatch through the peer windows")
     n0 = sum(c.launch_count for c in ctxs)
+    with torch.cuda.stream(stream):
+        step()
+    per_step = sum(c.launch_count for c in ctxs) - n0      # kernel launches of one step
     sampler = ClockSampler(0)
     sampler.start()
     ms_step = timed(step, steps)
     clocks = sampler.stop()
-    launches = sum(c.launch_count for c in ctxs) - n0
+    launches = per_step * steps
     ms_pub = timed(lambda: publish(x, 0), steps)
     ms_pull0 = timed(lambda: pull(y, 0), steps)
     ms_pull1 = timed(lambda: pull(z, 1), steps)
