@@ -844,3 +844,38 @@ def test_packed_autograd_backward_is_packed_mode1():
             want = oracle.ulysses_a2a(gys[t], 1)
             for j in range(w):
                 assert torch.equal(bits(xs[j].grad[:, :, t].cpu().contiguous()), bits(want[j]))
+
+
+def test_randomized_packed_launches():
+    """Seeded random head-packed launches: T, w, shapes, element size, chunking."""
+    import random
+
+    rng = random.Random(4242)
+    with UlyssesA2A(0, 2) as a2, UlyssesA2A(0, 4) as a4, UlyssesA2A(0, 1) as a1:
+        ctx_of = {1: a1, 2: a2, 4: a4}
+        for case in range(40):
+            E = rng.choice([1, 2, 4])
+            w = rng.choice([1, 2, 3, 4, 8])
+            T = rng.randint(1, min(4, 64 // w))
+            Hw = rng.choice([1, 2, 3, 5])
+            H, B = Hw * w, rng.randint(1, 3)
+            S = rng.randint(1, 70)
+            D = rng.choice([1, 7, 16, 33, 64])
+            chunked = rng.random() < 0.5
+            dtype = {1: torch.uint8, 2: torch.int16, 4: torch.int32}[E]
+            packed_cpu = random_byte_slabs((B, S, T, H, D * E), w, seed0=5000 + case)
+            packed_cpu = [t.view(dtype).reshape(B, S, T, H, D) for t in packed_cpu]
+            a2a = ctx_of[E]
+            packed = [t.cuda() for t in packed_cpu]
+            outs = a2a.run_packed(packed, 0, chunked=chunked)
+            flat = [t.reshape(-1) for t in packed_cpu]
+            for t in range(T):
+                want = oracle.ulysses_a2a_pitched(flat, 0, w, B, S, H, D, T * H * D,
+                                                  offset=t * H * D)
+                for r in range(w):
+                    assert torch.equal(outs[t][r].cpu().reshape(-1), want[r]), (case, t, r)
+            back = a2a.run_packed(outs, 1, chunked=not chunked)
+            for j in range(w):
+                assert torch.equal(back[j].cpu(), packed_cpu[j]), (case, j)
+        for a in (a1, a2, a4):
+            a.status()
