@@ -46,7 +46,7 @@ def build(force: bool = False, ptxas_info: bool = False, out: str = LIB) -> str:
         return out
     cmd = [nvcc(), *ARCH, "-lineinfo", "-O3", "-std=c++17", "-shared",
            "-Xcompiler", "-fPIC,-O2,-Wall", "-I", INCLUDE, "-I", CSRC,
-           "-o", out, os.path.join(CSRC, "ulysses_a2a.cu")]
+           "-o", out, *sorted(glob.glob(os.path.join(CSRC, "*.cu")))]
     if ptxas_info:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)

@@ -412,6 +412,9 @@ __global__ void __launch_bounds__(32 * kTmaMaxProducers, 1)
 // nothing ever arrives on, waits for it through mbar_wait_bounded with a short
 // limit, and records the expiry in the status words exactly as the copy
 // kernel does. No memory other than the status words is touched.
+// (A template, like the copy kernels, so that it is instantiated only in the
+// translation unit that launches it.)
+template <int kUnused = 0>
 __global__ void __launch_bounds__(32, 1)
     ua2a_wait_selftest_kernel(unsigned int* status, uint64_t limit_ns) {
   __shared__ __align__(8) uint64_t bar;

@@ -1,4 +1,5 @@
-// ulysses_a2a.cu - C ABI of the B200 Ulysses 4D all-to-all re-layout.
+// ulysses_a2a.cu - C ABI of the B200 Ulysses 4D all-to-all re-layout: the
+// context, the single-GPU entry points and every kernel launch.
 //
 // Implements include/ulysses_a2a.h. The operation and its argument convention
 // follow the FastVideo API docs, fastvideo.distributed.device_communicators
@@ -16,33 +17,16 @@
 // shape), the device status word of the bounded waits, and the device staging
 // buffers of the host-buffer entry point (grown on demand, like the page's
 // window `_build`/grow).
-#include <cuda.h>
-#include <cuda_runtime.h>
-#include <cudaTypedefs.h>
-
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
-#include <chrono>
 #include <cstring>
 #include <functional>
 #include <mutex>
-#include <new>
-#include <random>
 #include <string>
 #include <vector>
 
-#include <unistd.h>
-
-#include "kernels_tma.cuh"
-#include "kernels_vec.cuh"
-#include "plan.h"
-#include "ulysses_a2a.h"
-
-// L2 fetch granularity the TMA unit uses for the tensor maps (tunable at build time).
-#ifndef UA2A_L2_PROMOTION
-#define UA2A_L2_PROMOTION CU_TENSOR_MAP_L2_PROMOTION_L2_256B
-#endif
+#include "internal.h"
 
 using ua2a::TmaParams;
 using ua2a::VecParams;
@@ -50,62 +34,8 @@ using ua2a::VecParams;
 static_assert(ua2a::kVecResidentCtasPerSm == ua2a::kVecMinBlocksPerSm,
               "the planner's VEC residency must match the kernel's launch bound");
 
-namespace {
+namespace ua2a {
 
-constexpr int kTmaCacheEntries = 16;
-
-
-struct TmaCacheEntry {
-  bool valid = false;
-  uint64_t stamp = 0;
-  int mode = 0, w = 0;
-  int64_t B = 0, S = 0, H = 0, D = 0, rows = 0, pitch = 0;
-  const void* in[ULYSSES_A2A_MAX_W_TMA] = {};
-  void* out[ULYSSES_A2A_MAX_W_TMA] = {};
-  TmaParams params;  // tensor maps + geometry (b0/nb/status filled per launch)
-};
-
-}  // namespace
-
-struct ulysses_a2a_ctx {
-  int device = 0;
-  int elem_bytes = 2;
-  int num_sms = 148;
-  int forced_path = ULYSSES_A2A_PATH_AUTO;
-  ua2a::Tuning tuning;
-  unsigned int* d_status = nullptr;  // 4 words, see kernels_tma.cuh
-  std::string last_error;
-  uint64_t launches = 0;
-  uint64_t stamp = 0;
-  TmaCacheEntry tma_cache[kTmaCacheEntries];
-  bool tma_smem_set[2] = {false, false};
-  int64_t tma_smem_set_bytes[2] = {0, 0};
-  // run_host staging: one device buffer carved into 2w slabs
-  void* d_stage = nullptr;
-  size_t stage_bytes = 0;
-  cudaStream_t copy_stream[2] = {nullptr, nullptr};  // H2D, D2H
-  // chunked = 2: the staging window (one plane of every input slab)
-  void* d_window = nullptr;
-  size_t window_bytes = 0;
-  std::vector<cudaEvent_t> copy_events;              // start + 2 per chunk
-  PFN_cuTensorMapEncodeTiled_v12000 encode_tiled = nullptr;
-  PFN_cuMemGetAddressRange_v3020 get_range = nullptr;
-};
-
-namespace {
-
-// Switch to the context's device for the lifetime of the guard.
-struct DeviceGuard {
-  int prev = -1;
-  bool ok = false;
-  explicit DeviceGuard(int dev) {
-    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
-    ok = cudaSetDevice(dev) == cudaSuccess;
-  }
-  ~DeviceGuard() {
-    if (prev >= 0) cudaSetDevice(prev);
-  }
-};
 
 int fail(ulysses_a2a_ctx* ctx, int code, const std::string& msg) {
   if (ctx) ctx->last_error = msg;
@@ -302,15 +232,11 @@ cudaError_t launch_vec(const VecParams& p, int vec_bytes, int mode, int grid, in
   }
 }
 
-// Launch the planned kernel(s) for tiles [tile0, tile0 + ntiles) of every
-// (r, b, j) block (ntiles < 0: the whole block). only_out >= 0 (VEC path
-// only) restricts the launch to the blocks of output slab only_out: r fixed in
-// mode 0, j fixed in mode 1. ntensors > 1 (VEC path only): head-packed
-// tensors, r ranging over ntensors*w head groups.
+// run_device: see internal.h.
 int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, int64_t B, int64_t S,
                int64_t H, int64_t D, int w, int mode, int chunked, cudaStream_t st,
-               const ulysses_a2a_plan_t& pl, int64_t tile0 = 0, int64_t ntiles = -1,
-               int only_out = -1, int ntensors = 1) {
+               const ulysses_a2a_plan_t& pl, int64_t tile0, int64_t ntiles, int only_out,
+               int ntensors) {
   const int64_t nb = chunked ? 1 : B;
   const int launches = chunked ? (int)B : 1;
   const int64_t nt = ntiles < 0 ? pl.tiles_per_block : ntiles;
@@ -389,7 +315,7 @@ int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, in
 
 int plan_for(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, int64_t B, int64_t S,
              int64_t H, int64_t D, int w, int mode, int chunked, ulysses_a2a_plan_t* pl,
-             int64_t row_pitch = 0, int ntensors = 1) {
+             int64_t row_pitch, int ntensors) {
   std::string err;
   int rc = ua2a::make_plan(in, out, B, S, H, D, w, mode, chunked, ctx->elem_bytes, ctx->forced_path,
                            ctx->tuning, ctx->num_sms, pl, &err, row_pitch, -1, ntensors);
@@ -418,7 +344,22 @@ bool env_config(int* path, int* ctas) {
   return true;
 }
 
-}  // namespace
+}  // namespace ua2a
+
+namespace ua2a {
+
+cudaError_t tma_allow_max_smem() {
+  cudaError_t e = cudaFuncSetAttribute(ua2a_tma_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kTmaSmemMax);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(ua2a_tma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kTmaSmemMax);
+  return e;
+}
+
+}  // namespace ua2a
+
+using namespace ua2a;
 
 extern "C" {
 
@@ -779,7 +720,7 @@ static int ua2a_impl_selftest_wait_timeout(ulysses_a2a_ctx* ctx, uint32_t limit_
     return fail(ctx, ULYSSES_A2A_ERR_INVALID, "limit_us must be in [1, 2000000]");
   DeviceGuard g(ctx->device);
   if (!g.ok) return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "cannot select the context's device");
-  ua2a::ua2a_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+  ua2a::ua2a_wait_selftest_kernel<0><<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       ctx->d_status, (uint64_t)limit_us * 1000ull);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(ctx, "self-test kernel launch", e);
@@ -869,609 +810,6 @@ static int ua2a_impl_plan(const void* const* in_slabs, void* const* out_slabs, i
 
 }  // extern "C"
 
-// ---------------------------------------------------------------------------
-// Multi-GPU exchange through published windows (ulysses_a2a_peer_*).
-//
-// Each rank owns one device window that the other ranks map: CUDA IPC between
-// processes, the plain address inside one process. A call publishes the local
-// input slab into the own window (a w = 1 re-layout, i.e. a copy that drops any
-// row pitch), and after the caller's barrier pulls this rank's output slab out
-// of all w windows with the VEC kernel restricted to that one output slab, so
-// the bytes crossing NVLink are read by the GPU that needs them and written to
-// its own memory. The barriers are left to the caller: no kernel here waits on
-// another GPU.
-// ---------------------------------------------------------------------------
-
-namespace {
-
-constexpr uint32_t kPeerMagic = 0x50324155u;  // "UA2P"
-constexpr uint32_t kPeerVersion = 1;
-
-// The record one rank hands to the others (ULYSSES_A2A_PEER_HANDLE_BYTES).
-struct PeerRecord {
-  uint32_t magic;
-  uint32_t version;
-  uint64_t process_nonce;  // random per process: with pid, tells "same process"
-  int32_t rank;
-  int32_t world;
-  int32_t device;          // owner's device ordinal (meaningful in its process)
-  int32_t elem_bytes;
-  uint64_t window_bytes;
-  uint64_t base;           // owner's window address (used in the same process)
-  uint64_t pid;
-  cudaIpcMemHandle_t ipc;  // 64 bytes; valid if ipc_ok
-  int32_t ipc_ok;
-  int32_t pad;
-};
-static_assert(sizeof(PeerRecord) == ULYSSES_A2A_PEER_HANDLE_BYTES, "peer record size");
-
-uint64_t process_nonce() {
-  static std::once_flag once;
-  static uint64_t nonce = 0;
-  std::call_once(once, [] {
-    uint64_t v = (uint64_t)std::chrono::steady_clock::now().time_since_epoch().count();
-    v ^= (uint64_t)getpid() << 17;
-    v ^= (uint64_t)(uintptr_t)&nonce;
-    try {  // no exception may leave the C ABI
-      std::random_device rd;
-      v ^= ((uint64_t)rd() << 32) ^ (uint64_t)rd();
-    } catch (...) {
-    }
-    nonce = v ? v : 1;
-  });
-  return nonce;
-}
-
-}  // namespace
-
-struct ulysses_a2a_peer {
-  ulysses_a2a_ctx* ctx = nullptr;
-  int rank = 0, world = 1;
-  size_t window_bytes = 0;
-  void* own = nullptr;
-  std::vector<void*> bases;        // window of rank k as mapped here
-  std::vector<char> ipc_opened;    // 1 where cudaIpcOpenMemHandle made the mapping
-  bool open = false;
-};
-
-namespace {
-
-void peer_unmap(ulysses_a2a_peer* p, int* rc) {
-  for (int k = 0; k < p->world; ++k) {
-    if (k == p->rank) continue;
-    if (p->ipc_opened[k] && p->bases[k] && cudaIpcCloseMemHandle(p->bases[k]) != cudaSuccess) {
-      cudaGetLastError();
-      if (rc) *rc = ULYSSES_A2A_ERR_CUDA;
-    }
-    p->ipc_opened[k] = 0;
-    p->bases[k] = nullptr;
-  }
-  p->open = false;
-}
-
-}  // namespace
-
-extern "C" {
-
-static int ua2a_impl_peer_create(ulysses_a2a_ctx* ctx, int rank, int world, size_t window_bytes,
-                            ulysses_a2a_peer** out, void* handle_out) {
-  if (out) *out = nullptr;
-  if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
-  ctx->last_error.clear();
-  if (out == nullptr || handle_out == nullptr)
-    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_create: out or handle_out is NULL");
-  if (world < 1 || world > ULYSSES_A2A_MAX_W || rank < 0 || rank >= world)
-    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_create: need 1 <= world <= 64, 0 <= rank < world");
-  if (window_bytes < 1) return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_create: window_bytes must be >= 1");
-  DeviceGuard g(ctx->device);
-  if (!g.ok) return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "cannot select the context's device");
-  ulysses_a2a_peer* p = new (std::nothrow) ulysses_a2a_peer();
-  if (!p) return fail(ctx, ULYSSES_A2A_ERR_NOMEM, "peer_create: host allocation failed");
-  p->ctx = ctx;
-  p->rank = rank;
-  p->world = world;
-  p->window_bytes = window_bytes;
-  p->bases.assign(world, nullptr);
-  p->ipc_opened.assign(world, 0);
-  cudaError_t e = cudaMalloc(&p->own, window_bytes);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    delete p;
-    return fail(ctx, ULYSSES_A2A_ERR_NOMEM, "peer_create: cudaMalloc of the window failed");
-  }
-  p->bases[rank] = p->own;
-  PeerRecord r;
-  std::memset(&r, 0, sizeof(r));
-  r.magic = kPeerMagic;
-  r.version = kPeerVersion;
-  r.process_nonce = process_nonce();
-  r.rank = rank;
-  r.world = world;
-  r.device = ctx->device;
-  r.elem_bytes = ctx->elem_bytes;
-  r.window_bytes = window_bytes;
-  r.base = (uint64_t)(uintptr_t)p->own;
-  r.pid = (uint64_t)getpid();
-  // a window that cannot be exported still serves ranks in this process
-  r.ipc_ok = cudaIpcGetMemHandle(&r.ipc, p->own) == cudaSuccess ? 1 : 0;
-  if (!r.ipc_ok) cudaGetLastError();
-  std::memcpy(handle_out, &r, sizeof(r));
-  *out = p;
-  return ULYSSES_A2A_OK;
-}
-
-static int ua2a_impl_peer_open(ulysses_a2a_peer* p, const void* handles) {
-  if (p == nullptr) return ULYSSES_A2A_ERR_INVALID;
-  ulysses_a2a_ctx* ctx = p->ctx;
-  ctx->last_error.clear();
-  if (handles == nullptr) return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_open: handles is NULL");
-  if (p->open) return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_open: already open");
-  std::vector<PeerRecord> recs(p->world);
-  std::memcpy(recs.data(), handles, sizeof(PeerRecord) * (size_t)p->world);
-  const uint64_t nonce = process_nonce();
-  const uint64_t pid = (uint64_t)getpid();
-  // check every record before mapping anything
-  for (int k = 0; k < p->world; ++k) {
-    const PeerRecord& r = recs[k];
-    const std::string who = "peer_open: record " + std::to_string(k);
-    if (r.magic != kPeerMagic || r.version != kPeerVersion)
-      return fail(ctx, ULYSSES_A2A_ERR_INVALID, who + " is not a peer record of this library version");
-    if (r.rank != k || r.world != p->world)
-      return fail(ctx, ULYSSES_A2A_ERR_INVALID, who + " carries rank " + std::to_string(r.rank) +
-                                                    " of world " + std::to_string(r.world));
-    if (r.elem_bytes != ctx->elem_bytes || r.window_bytes != (uint64_t)p->window_bytes)
-      return fail(ctx, ULYSSES_A2A_ERR_INVALID, who + ": element size or window size differs");
-    const bool local = r.process_nonce == nonce && r.pid == pid;
-    if (k == p->rank && !(local && r.base == (uint64_t)(uintptr_t)p->own))
-      return fail(ctx, ULYSSES_A2A_ERR_INVALID, who + " is not this peer's own record");
-    if (k != p->rank && !local && !r.ipc_ok)
-      return fail(ctx, ULYSSES_A2A_ERR_DEVICE, who + ": its window could not be exported (CUDA IPC)");
-  }
-  DeviceGuard g(ctx->device);
-  if (!g.ok) return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "cannot select the context's device");
-  for (int k = 0; k < p->world; ++k) {
-    if (k == p->rank) continue;
-    const PeerRecord& r = recs[k];
-    const bool local = r.process_nonce == nonce && r.pid == pid;
-    cudaError_t e = cudaSuccess;
-    if (local) {
-      if (r.device != ctx->device) {
-        int can = 0;
-        e = cudaDeviceCanAccessPeer(&can, ctx->device, r.device);
-        if (e == cudaSuccess && !can) {
-          peer_unmap(p, nullptr);
-          return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "peer_open: device " + std::to_string(ctx->device) +
-                                                       " cannot access device " + std::to_string(r.device));
-        }
-        if (e == cudaSuccess) {
-          e = cudaDeviceEnablePeerAccess(r.device, 0);
-          if (e == cudaErrorPeerAccessAlreadyEnabled) {
-            cudaGetLastError();
-            e = cudaSuccess;
-          }
-        }
-      }
-      if (e == cudaSuccess) p->bases[k] = reinterpret_cast<void*>((uintptr_t)r.base);
-    } else {
-      void* ptr = nullptr;
-      e = cudaIpcOpenMemHandle(&ptr, r.ipc, cudaIpcMemLazyEnablePeerAccess);
-      if (e == cudaSuccess) {
-        p->bases[k] = ptr;
-        p->ipc_opened[k] = 1;
-      }
-    }
-    if (e != cudaSuccess) {
-      cudaGetLastError();
-      peer_unmap(p, nullptr);
-      return cuda_fail(ctx, ("peer_open: mapping the window of rank " + std::to_string(k)).c_str(), e);
-    }
-  }
-  p->open = true;
-  return ULYSSES_A2A_OK;
-}
-
-static int ua2a_impl_peer_publish(ulysses_a2a_peer* p, const void* in_local, int64_t B, int64_t S_local,
-                             int64_t H, int64_t D, int mode, int64_t row_pitch, void* stream) {
-  if (p == nullptr) return ULYSSES_A2A_ERR_INVALID;
-  ulysses_a2a_ctx* ctx = p->ctx;
-  ctx->last_error.clear();
-  const int w = p->world;
-  if (mode != 0 && mode != 1) return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_publish: mode must be 0 or 1");
-  if (B < 0 || S_local < 0 || H < 0 || D < 0 || row_pitch < 0)
-    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_publish: sizes and row_pitch must be >= 0");
-  if (H % w != 0) return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_publish: H not divisible by the world size");
-  if (mode == 1 && row_pitch != 0)
-    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_publish: a mode-1 input is dense (row_pitch 0)");
-  // the copy, as a one-rank re-layout: mode 0 keeps [B, S, H, D] (dropping the
-  // pitch); mode 1 copies [B, S*w, H/w, D]
-  const int64_t S1 = mode == 0 ? S_local : S_local * w;
-  const int64_t H1 = mode == 0 ? H : H / w;
-  if (in_local == p->own && (row_pitch == 0 || row_pitch == H1 * D)) {
-    // the slab was written into the window in place: nothing to copy
-    int64_t bytes = 0;
-    if (ua2a::mul_overflows(B, S1, &bytes) || ua2a::mul_overflows(bytes, H1, &bytes) ||
-        ua2a::mul_overflows(bytes, D, &bytes) ||
-        ua2a::mul_overflows(bytes, (int64_t)ctx->elem_bytes, &bytes) ||
-        (uint64_t)bytes > (uint64_t)p->window_bytes)
-      return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_publish: the slab exceeds the window");
-    return ULYSSES_A2A_OK;
-  }
-  const void* in[1] = {in_local};
-  void* out[1] = {p->own};
-  ulysses_a2a_plan_t pl;
-  int rc = plan_for(ctx, in, out, B, S1, H1, D, 1, 0, 0, &pl, row_pitch);
-  if (rc) return rc;
-  if (pl.units == 0) return ULYSSES_A2A_OK;
-  if ((uint64_t)pl.payload_bytes > (uint64_t)p->window_bytes)
-    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_publish: the slab (" + std::to_string(pl.payload_bytes) +
-                                                  " bytes) exceeds the window (" +
-                                                  std::to_string(p->window_bytes) + " bytes)");
-  DeviceGuard g(ctx->device);
-  if (!g.ok) return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "cannot select the context's device");
-  const int64_t in_bytes = ((B * S1 - 1) * pl.row_pitch + H1 * D) * (int64_t)ctx->elem_bytes;
-  rc = check_residency(ctx, in, 1, in_bytes, "input");
-  if (rc) return rc;
-  return run_device(ctx, in, out, B, S1, H1, D, 1, 0, 0, static_cast<cudaStream_t>(stream), pl);
-}
-
-static int ua2a_impl_peer_pull(ulysses_a2a_peer* p, void* out_local, int64_t B, int64_t S_local, int64_t H,
-                          int64_t D, int mode, int64_t row_pitch, void* stream) {
-  if (p == nullptr) return ULYSSES_A2A_ERR_INVALID;
-  ulysses_a2a_ctx* ctx = p->ctx;
-  ctx->last_error.clear();
-  if (!p->open) return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_pull: the peer windows are not open");
-  const int w = p->world;
-  if (mode == 0 && row_pitch != 0)
-    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_pull: a mode-0 output is dense (row_pitch 0)");
-  std::vector<void*> outs(w, nullptr);
-  outs[p->rank] = out_local;
-  std::string err;
-  ulysses_a2a_plan_t pl;
-  int rc = ua2a::make_plan(p->bases.data(), outs.data(), B, S_local, H, D, w, mode, 0, ctx->elem_bytes,
-                           ULYSSES_A2A_PATH_VEC, ctx->tuning, ctx->num_sms, &pl, &err, row_pitch,
-                           p->rank);
-  if (rc) return fail(ctx, rc, "peer_pull: " + err);
-  if (pl.units == 0) return ULYSSES_A2A_OK;
-  if ((uint64_t)pl.payload_bytes > (uint64_t)p->window_bytes)
-    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_pull: the slab (" + std::to_string(pl.payload_bytes) +
-                                                  " bytes) exceeds the windows (" +
-                                                  std::to_string(p->window_bytes) + " bytes)");
-  DeviceGuard g(ctx->device);
-  if (!g.ok) return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "cannot select the context's device");
-  const int64_t out_bytes = mode == 0 ? pl.payload_bytes
-                                      : ((B * S_local - 1) * pl.row_pitch + H * D) * (int64_t)ctx->elem_bytes;
-  const void* o[1] = {out_local};
-  rc = check_residency(ctx, o, 1, out_bytes, "output");
-  if (rc) return rc;
-  return run_device(ctx, p->bases.data(), outs.data(), B, S_local, H, D, w, mode, 0,
-                    static_cast<cudaStream_t>(stream), pl, 0, -1, p->rank);
-}
-
-void* ulysses_a2a_peer_window(const ulysses_a2a_peer* p, int rank) {
-  if (p == nullptr || rank < 0 || rank >= p->world) return nullptr;
-  return p->bases[rank];
-}
-
-size_t ulysses_a2a_peer_window_bytes(const ulysses_a2a_peer* p) {
-  return p ? p->window_bytes : 0;
-}
-
-static int ua2a_impl_peer_close(ulysses_a2a_peer* p) {
-  if (p == nullptr) return ULYSSES_A2A_ERR_INVALID;
-  if (!p->open) return ULYSSES_A2A_OK;
-  int rc = ULYSSES_A2A_OK;
-  DeviceGuard g(p->ctx->device);
-  if (cudaDeviceSynchronize() != cudaSuccess) {
-    cudaGetLastError();
-    rc = ULYSSES_A2A_ERR_CUDA;
-  }
-  peer_unmap(p, &rc);
-  return rc;
-}
-
-static int ua2a_impl_peer_destroy(ulysses_a2a_peer* p) {
-  if (p == nullptr) return ULYSSES_A2A_OK;
-  int rc = ulysses_a2a_peer_close(p);
-  {
-    DeviceGuard g(p->ctx->device);
-    if (p->own && cudaFree(p->own) != cudaSuccess) {
-      cudaGetLastError();
-      rc = ULYSSES_A2A_ERR_CUDA;
-    }
-  }
-  delete p;  // consumed whatever the cleanup calls reported
-  return rc;
-}
-
-}  // extern "C"
-
-// ---------------------------------------------------------------------------
-// Allocation-free entry point (ulysses_a2a_run_noalloc).
-//
-// For callers that may not allocate device memory themselves: a process whose
-// device memory is owned by another allocator under a fixed budget, or a host
-// thread running where a cudaMalloc/cudaFree (which can synchronise the device)
-// is not allowed. ulysses_a2a_create allocates the TMA kernel's status records;
-// this entry point runs the same kernels with those records in a file-scope
-// static device array instead, and needs no context.
-//
-// The array is modest and fixed: kNoAllocSlots records of 16 bytes (1 KiB),
-// one record per kernel launch of a call (a chunked call launches once per
-// plane), held by every GPU that loads this library until the process exits.
-// Every call shares it and it keeps the last call's contents: each call clears
-// the records it uses, on its stream, before launching, so two calls whose work
-// overlaps on the GPU (different streams, or different host threads) race on it.
-// ---------------------------------------------------------------------------
-
-namespace {
-constexpr int kNoAllocSlots = 64;
-constexpr int kNoAllocSlotWords = 4;
-constexpr int kNoAllocMaxDevices = 64;
-}  // namespace
-
-static __device__ __align__(256) unsigned int ua2a_noalloc_scratch[kNoAllocSlots * kNoAllocSlotWords];
-
-namespace {
-
-struct NoAllocDevice {
-  std::once_flag once;
-  int rc = ULYSSES_A2A_OK;
-  char why[96] = {0};
-  unsigned int* scratch = nullptr;  // this device's address of ua2a_noalloc_scratch
-  int num_sms = 0;
-};
-
-NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
-std::once_flag g_noalloc_driver_once;
-PFN_cuTensorMapEncodeTiled_v12000 g_noalloc_encode = nullptr;
-PFN_cuMemGetAddressRange_v3020 g_noalloc_range = nullptr;
-
-int noalloc_report(char* err, size_t errlen, int rc, const char* fmt, long long a = 0,
-                   long long b = 0) {
-  if (err && errlen) std::snprintf(err, errlen, fmt, a, b);
-  return rc;
-}
-
-// Once per device, with that device current: resolve the array's device address
-// (the symbol itself is only a host-side stand-in) and set the kernels' shared
-// memory limit.
-void noalloc_setup(NoAllocDevice& st, int dev) {
-  cudaDeviceProp prop;
-  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess || prop.major < 10) {
-    cudaGetLastError();
-    st.rc = ULYSSES_A2A_ERR_DEVICE;
-    std::snprintf(st.why, sizeof(st.why), "device %d is not an sm_100 GPU", dev);
-    return;
-  }
-  st.num_sms = prop.multiProcessorCount;
-  void* addr = nullptr;
-  cudaError_t e = cudaGetSymbolAddress(&addr, ua2a_noalloc_scratch);
-  if (e != cudaSuccess || addr == nullptr) {
-    cudaGetLastError();
-    st.rc = ULYSSES_A2A_ERR_CUDA;
-    std::snprintf(st.why, sizeof(st.why), "cudaGetSymbolAddress failed: %s", cudaGetErrorName(e));
-    return;
-  }
-  st.scratch = static_cast<unsigned int*>(addr);
-  if (cudaFuncSetAttribute(ua2a::ua2a_tma_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)ua2a::kTmaSmemMax) != cudaSuccess ||
-      cudaFuncSetAttribute(ua2a::ua2a_tma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)ua2a::kTmaSmemMax) != cudaSuccess) {
-    cudaGetLastError();
-    st.rc = ULYSSES_A2A_ERR_CUDA;
-    std::snprintf(st.why, sizeof(st.why), "cudaFuncSetAttribute failed");
-  }
-}
-
-bool noalloc_encode(CUtensorMap* m, int rank, const void* base, const cuuint64_t* dims,
-                    const cuuint64_t* strides, const cuuint32_t* box, int E) {
-  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  return g_noalloc_encode(m, map_dtype(E), (cuuint32_t)rank, const_cast<void*>(base), dims, strides,
-                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                          UA2A_L2_PROMOTION,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-}  // namespace
-
-static int ua2a_impl_run_noalloc(const void* const* in_slabs, void* const* out_slabs,
-                                       int64_t B, int64_t S_local, int64_t H, int64_t D, int w,
-                                       int mode, int chunked, int elem_bytes, void* stream,
-                                       int wait, char* err, size_t errlen) {
-  if (err && errlen) err[0] = '\0';
-  std::call_once(g_noalloc_driver_once, [] {
-    cudaDriverEntryPointQueryResult q;
-    void* fn = nullptr;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      g_noalloc_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    fn = nullptr;
-    if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &fn, 12000, cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      g_noalloc_range = reinterpret_cast<PFN_cuMemGetAddressRange_v3020>(fn);
-    cudaGetLastError();
-  });
-  if (g_noalloc_encode == nullptr)
-    return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  if (chunked == ULYSSES_A2A_CHUNKED_WINDOW)
-    return noalloc_report(err, errlen, ULYSSES_A2A_ERR_UNSUPPORTED,
-                          "chunked = 2 needs a staging window; use chunked 0 or 1 here");
-
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) {
-    cudaGetLastError();
-    return noalloc_report(err, errlen, ULYSSES_A2A_ERR_DEVICE, "no usable current CUDA device");
-  }
-  NoAllocDevice& st = g_noalloc_dev[dev];
-  std::call_once(st.once, noalloc_setup, std::ref(st), dev);
-  if (st.rc != ULYSSES_A2A_OK) {
-    if (err && errlen) std::snprintf(err, errlen, "%s", st.why);
-    return st.rc;
-  }
-
-  // the same checks as ulysses_a2a_run, before anything is launched
-  ulysses_a2a_plan_t pl;
-  int rc = ua2a::make_plan(in_slabs, out_slabs, B, S_local, H, D, w, mode, chunked, elem_bytes,
-                           ULYSSES_A2A_PATH_AUTO, ua2a::Tuning{}, st.num_sms, &pl, nullptr);
-  if (rc != ULYSSES_A2A_OK) {
-    std::string msg;
-    ua2a::make_plan(in_slabs, out_slabs, B, S_local, H, D, w, mode, chunked, elem_bytes,
-                    ULYSSES_A2A_PATH_AUTO, ua2a::Tuning{}, st.num_sms, &pl, &msg);
-    if (err && errlen) std::snprintf(err, errlen, "%s", msg.c_str());
-    return rc;
-  }
-  if (pl.units == 0) return ULYSSES_A2A_OK;  // empty: nothing to do
-  const int slots = pl.launches;
-  if (slots > kNoAllocSlots)
-    return noalloc_report(err, errlen, ULYSSES_A2A_ERR_UNSUPPORTED,
-                          "chunked call over %lld planes needs %lld status records; the static "
-                          "scratch holds 64 (1 KiB): split the call or use ulysses_a2a_run",
-                          (long long)slots, (long long)slots);
-  const int64_t slab_bytes = pl.payload_bytes / w;
-  for (int side = 0; side < 2; ++side) {
-    for (int k = 0; k < w; ++k) {
-      const void* p = side == 0 ? in_slabs[k] : out_slabs[k];
-      cudaPointerAttributes a;
-      if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
-        cudaGetLastError();
-        if (err && errlen)
-          std::snprintf(err, errlen, "%s slab %d is not a CUDA pointer", side ? "output" : "input", k);
-        return ULYSSES_A2A_ERR_DEVICE;
-      }
-      if (!(a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) || a.device != dev) {
-        if (err && errlen)
-          std::snprintf(err, errlen, "%s slab %d is not device memory of the current device %d",
-                        side ? "output" : "input", k, dev);
-        return ULYSSES_A2A_ERR_DEVICE;
-      }
-      if (g_noalloc_range && a.type == cudaMemoryTypeDevice) {
-        CUdeviceptr base = 0;
-        size_t size = 0;
-        if (g_noalloc_range(&base, &size, (CUdeviceptr)(uintptr_t)p) == CUDA_SUCCESS &&
-            (uintptr_t)p + (uintptr_t)slab_bytes > (uintptr_t)base + size) {
-          if (err && errlen)
-            std::snprintf(err, errlen, "%s slab %d runs past the end of its allocation",
-                          side ? "output" : "input", k);
-          return ULYSSES_A2A_ERR_DEVICE;
-        }
-      }
-    }
-  }
-
-  cudaStream_t st_ = static_cast<cudaStream_t>(stream);
-  // the records of this call start at zero (the array keeps the previous call's)
-  cudaError_t e = cudaMemsetAsync(st.scratch, 0, sizeof(unsigned int) * kNoAllocSlotWords * slots, st_);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "cudaMemsetAsync of the status records failed");
-  }
-  const int64_t nb = chunked ? 1 : B;
-  if (pl.path == ULYSSES_A2A_PATH_TMA) {
-    TmaParams p;
-    std::memset(&p, 0, sizeof(p));
-    const int64_t E = elem_bytes, Hw = H / w, rows = pl.rows_per_tile;
-    for (int k = 0; k < w; ++k) {
-      const void* strided = mode == 0 ? in_slabs[k] : out_slabs[k];
-      const void* gathered = mode == 0 ? out_slabs[k] : in_slabs[k];
-      const cuuint64_t sd[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S_local, (cuuint64_t)B};
-      const cuuint64_t ss[3] = {(cuuint64_t)(D * E), (cuuint64_t)(H * D * E),
-                                (cuuint64_t)(S_local * H * D * E)};
-      const cuuint32_t sb[4] = {(cuuint32_t)D, (cuuint32_t)Hw, (cuuint32_t)rows, 1};
-      const cuuint64_t gd[5] = {(cuuint64_t)D, (cuuint64_t)Hw, (cuuint64_t)S_local, (cuuint64_t)w,
-                                (cuuint64_t)B};
-      const cuuint64_t gs[4] = {(cuuint64_t)(D * E), (cuuint64_t)(Hw * D * E),
-                                (cuuint64_t)(S_local * Hw * D * E),
-                                (cuuint64_t)(w * S_local * Hw * D * E)};
-      const cuuint32_t gb[5] = {(cuuint32_t)D, (cuuint32_t)Hw, (cuuint32_t)rows, 1, 1};
-      if (!noalloc_encode(&p.strided[k], 4, strided, sd, ss, sb, elem_bytes) ||
-          !noalloc_encode(&p.gathered[k], 5, gathered, gd, gs, gb, elem_bytes))
-        return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "cuTensorMapEncodeTiled failed for slab %lld", k);
-    }
-    p.units = pl.units;
-    p.w = w;
-    p.Hw = (int32_t)Hw;
-    p.rows_per_tile = (int32_t)rows;
-    p.tiles_per_block = (int32_t)pl.tiles_per_block;
-    p.tile0 = 0;
-    p.nb = (int32_t)nb;
-    p.tile_bytes = (uint32_t)(rows * pl.row_bytes);
-    p.stage_bytes = (p.tile_bytes + 1023u) / 1024u * 1024u;
-    p.stages = pl.stages / pl.producers;
-    p.lookahead = pl.lookahead;
-    p.producers = pl.producers;
-    p.order = pl.order;
-    p.chunk_units = pl.chunk_units;
-    for (int l = 0; l < pl.launches; ++l) {
-      p.b0 = chunked ? l : 0;
-      p.status = st.scratch + kNoAllocSlotWords * l;
-      e = launch_tma(mode, pl.grid, pl.block, (size_t)pl.smem_bytes, st_, p);
-      if (e != cudaSuccess)
-        return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "TMA kernel launch failed (plane %lld)", l);
-    }
-  } else {
-    VecParams p{};
-    for (int k = 0; k < w; ++k) {
-      p.in[k] = static_cast<const char*>(in_slabs[k]);
-      p.out[k] = static_cast<char*>(out_slabs[k]);
-    }
-    p.S_local = S_local;
-    p.nv = pl.row_bytes / pl.vec_bytes;
-    p.srow = pl.row_pitch * elem_bytes / pl.vec_bytes;
-    p.w = w;
-    p.rows_per_tile = (int32_t)pl.rows_per_tile;
-    p.units = (uint32_t)pl.units;
-    p.order = pl.order;
-    p.div_T = ua2a::FastDiv((uint32_t)pl.tiles_per_block);
-    p.div_nr = ua2a::FastDiv((uint32_t)w);
-    p.div_nj = ua2a::FastDiv((uint32_t)w);
-    p.div_nb = ua2a::FastDiv((uint32_t)nb);
-    p.div_nv = ua2a::FastDiv((uint32_t)p.nv);
-    for (int l = 0; l < pl.launches; ++l) {
-      p.b0 = chunked ? l : 0;
-      e = launch_vec(p, pl.vec_bytes, mode, pl.grid, pl.block, st_);
-      if (e != cudaSuccess)
-        return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "VEC kernel launch failed (plane %lld)", l);
-    }
-  }
-  if (!wait) return ULYSSES_A2A_OK;
-  e = cudaStreamSynchronize(st_);
-  if (e != cudaSuccess)
-    return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "cudaStreamSynchronize failed");
-  unsigned int h[kNoAllocSlots * kNoAllocSlotWords];
-  e = cudaMemcpy(h, st.scratch, sizeof(unsigned int) * kNoAllocSlotWords * slots, cudaMemcpyDeviceToHost);
-  if (e != cudaSuccess)
-    return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "reading the status records failed");
-  for (int l = 0; l < slots; ++l) {
-    if (h[kNoAllocSlotWords * l] != 0)
-      return noalloc_report(err, errlen, ULYSSES_A2A_ERR_TIMEOUT,
-                            "a TMA wait gave up in launch %lld (flags 0x%llx)", l,
-                            h[kNoAllocSlotWords * l]);
-  }
-  return ULYSSES_A2A_OK;
-}
-
-// ---------------------------------------------------------------------------
-// The exported entry points: no exception may cross the C ABI. A failed host
-// allocation inside the library becomes ULYSSES_A2A_ERR_NOMEM, any other
-// exception ULYSSES_A2A_ERR_INTERNAL.
-// ---------------------------------------------------------------------------
-
-namespace {
-
-template <typename F>
-int no_throw(F&& f) noexcept {
-  try {
-    return f();
-  } catch (const std::bad_alloc&) {
-    return ULYSSES_A2A_ERR_NOMEM;
-  } catch (...) {
-    return ULYSSES_A2A_ERR_INTERNAL;
-  }
-}
-
-}  // namespace
 
 extern "C" {
 
@@ -1535,44 +873,6 @@ int ulysses_a2a_plan(const void* const* in_slabs, void* const* out_slabs, int64_
 
 int ulysses_a2a_get_settings(const ulysses_a2a_ctx* ctx, int32_t* path, ulysses_a2a_tuning_t* t) {
   return no_throw([&] { return ua2a_impl_get_settings(ctx, path, t); });
-}
-
-int ulysses_a2a_peer_create(ulysses_a2a_ctx* ctx, int rank, int world, size_t window_bytes,
-                            ulysses_a2a_peer** out, void* handle_out) {
-  return no_throw([&] { return ua2a_impl_peer_create(ctx, rank, world, window_bytes, out,
-                                                     handle_out); });
-}
-
-int ulysses_a2a_peer_open(ulysses_a2a_peer* p, const void* handles) {
-  return no_throw([&] { return ua2a_impl_peer_open(p, handles); });
-}
-
-int ulysses_a2a_peer_publish(ulysses_a2a_peer* p, const void* in_local, int64_t B, int64_t S_local,
-                             int64_t H, int64_t D, int mode, int64_t row_pitch, void* stream) {
-  return no_throw([&] { return ua2a_impl_peer_publish(p, in_local, B, S_local, H, D, mode,
-                                                      row_pitch, stream); });
-}
-
-int ulysses_a2a_peer_pull(ulysses_a2a_peer* p, void* out_local, int64_t B, int64_t S_local,
-                          int64_t H, int64_t D, int mode, int64_t row_pitch, void* stream) {
-  return no_throw([&] { return ua2a_impl_peer_pull(p, out_local, B, S_local, H, D, mode, row_pitch,
-                                                   stream); });
-}
-
-int ulysses_a2a_peer_close(ulysses_a2a_peer* p) {
-  return no_throw([&] { return ua2a_impl_peer_close(p); });
-}
-
-int ulysses_a2a_peer_destroy(ulysses_a2a_peer* p) {
-  return no_throw([&] { return ua2a_impl_peer_destroy(p); });
-}
-
-int ulysses_a2a_run_noalloc(const void* const* in_slabs, void* const* out_slabs, int64_t B,
-                            int64_t S_local, int64_t H, int64_t D, int w, int mode, int chunked,
-                            int elem_bytes, void* stream, int wait, char* err, size_t errlen) {
-  return no_throw([&] { return ua2a_impl_run_noalloc(in_slabs, out_slabs, B, S_local, H, D, w, mode,
-                                                     chunked, elem_bytes, stream, wait, err,
-                                                     errlen); });
 }
 
 }  // extern "C"
