@@ -2,7 +2,8 @@
  * Plain-C user of libulysses_a2a.so (no Python, no torch): allocates rank
  * slabs with cudaMalloc, runs both modes through ulysses_a2a_run, runs the
  * host-buffer entry point, checks the error codes of a few rejected calls, runs
- * the multi-GPU exchange entry points with its ranks in this process, and
+ * the multi-GPU exchange entry points with its ranks in this process, runs a
+ * head-packed launch (three tensors, one call of ulysses_a2a_run_ex), and
  * compares every output byte with the CPU oracle (libulysses_oracle.so, test
  * infrastructure). Exit status 0 = all checks passed.
  */
@@ -17,6 +18,9 @@
 int oracle_ulysses_a2a(const void *const *in, void *const *out, int64_t B,
                        int64_t S_local, int64_t H, int64_t D, int w, int mode,
                        int elem_bytes);
+int oracle_ulysses_a2a_pitched(const void *const *in, void *const *out,
+                               int64_t B, int64_t S_local, int64_t H, int64_t D,
+                               int w, int mode, int elem_bytes, int64_t row_pitch);
 
 #define W 4
 #define CHECK(cond, msg)                                             \
@@ -119,6 +123,52 @@ int main(void) {
             CHECK(ulysses_a2a_destroy(rctx[k]) == ULYSSES_A2A_OK, "destroy (rank)");
         }
         CHECK(ulysses_a2a_peer_destroy(NULL) == ULYSSES_A2A_OK, "peer destroy(NULL)");
+    }
+
+    /* three head-packed tensors in one launch: in[j] is [B, S, 3, H, D], out[t*W + r]
+       tensor t's [B, S*W, H/W, D] slab of rank r; the oracle runs once per tensor
+       on the row-pitched views (pitch 3*H*D, offset t*H*D) */
+    {
+        enum { T = 3 };
+        const size_t pn = n * T, pbytes = pn * E;
+        uint16_t *hp[W], *hq[T * W], *wq[T * W];
+        void *dp[W], *dq[T * W];
+        for (int k = 0; k < W; ++k) {
+            hp[k] = malloc(pbytes);
+            for (size_t i = 0; i < pn; ++i) hp[k][i] = (uint16_t)(k * 7919u + i * 40503u);
+            CHECK(cudaMalloc(&dp[k], pbytes) == cudaSuccess, "cudaMalloc packed");
+            CHECK(cudaMemcpy(dp[k], hp[k], pbytes, cudaMemcpyHostToDevice) == cudaSuccess, "H2D");
+        }
+        for (int k = 0; k < T * W; ++k) {
+            hq[k] = malloc(bytes);
+            wq[k] = malloc(bytes);
+            CHECK(cudaMalloc(&dq[k], bytes) == cudaSuccess, "cudaMalloc gathered");
+        }
+        for (int t = 0; t < T; ++t) {
+            const void *views[W];
+            void *wants[W];
+            for (int k = 0; k < W; ++k) {
+                views[k] = hp[k] + (size_t)t * H * D;
+                wants[k] = wq[t * W + k];
+            }
+            CHECK(oracle_ulysses_a2a_pitched(views, wants, B, S, H, D, W, 0, E, T * H * D) == 0,
+                  "pitched oracle");
+        }
+        ulysses_a2a_desc_t d;
+        memset(&d, 0, sizeof(d));
+        d.in_slabs = (const void *const *)dp;
+        d.out_slabs = dq;
+        d.B = B; d.S_local = S; d.H = H; d.D = D;
+        d.w = W; d.mode = 0; d.chunked = 0; d.ntensors = T; d.row_pitch = 0;
+        const uint64_t l0 = ulysses_a2a_launch_count(ctx);
+        CHECK(ulysses_a2a_run_ex(ctx, &d, NULL) == ULYSSES_A2A_OK, ulysses_a2a_last_error(ctx));
+        CHECK(ulysses_a2a_launch_count(ctx) == l0 + 1, "packed call is one launch");
+        for (int k = 0; k < T * W; ++k) {
+            CHECK(cudaMemcpy(hq[k], dq[k], bytes, cudaMemcpyDeviceToHost) == cudaSuccess, "D2H");
+            CHECK(memcmp(hq[k], wq[k], bytes) == 0, "packed launch differs from the oracle");
+        }
+        for (int k = 0; k < W; ++k) { cudaFree(dp[k]); free(hp[k]); }
+        for (int k = 0; k < T * W; ++k) { cudaFree(dq[k]); free(hq[k]); free(wq[k]); }
     }
 
     CHECK(ulysses_a2a_destroy(ctx) == ULYSSES_A2A_OK, "destroy");
