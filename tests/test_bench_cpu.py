@@ -1,0 +1,56 @@
+"""bench.py host logic without a GPU: the ncu traffic lookup and the workload table."""
+
+import json
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from sequence_all_re_b200 import _lib  # noqa: E402
+
+
+def plan_dict(w, B, S, H, D, path=_lib.PATH_AUTO):
+    step = (B * S * H * D * 2 + 4095) // 4096 * 4096
+    ins = [(1 << 40) + k * step for k in range(w)]
+    outs = [(1 << 40) + (w + k) * step for k in range(w)]
+    rc, p, msg = _lib.ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, 2, forced_path=path)
+    assert rc == _lib.OK, msg
+    return p.as_dict()
+
+
+def test_committed_captures_match_the_current_kernels_and_plans():
+    traffic = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))["workloads"]
+    for key, entry in traffic.items():
+        path, shape = key.split(":")
+        w, B, S, H, D = (int(part[1:]) for part in shape.split("_")[:5])
+        p = plan_dict(w, B, S, H, D, _lib.PATH_TMA if path == "tma" else _lib.PATH_VEC)
+        got, why = bench.ncu_traffic(key, p, 0)
+        assert why == "ncu", (key, why)
+        assert got == entry["dram_bytes_per_launch"]
+        # DRAM reads of a launch cover the payload (no re-reads beyond a few per mille)
+        payload = w * B * S * H * D * 2
+        for m in ("mode0", "mode1"):
+            assert 0.999 * payload <= entry[m]["dram_read"] <= 1.002 * payload, (key, m)
+
+
+def test_traffic_is_withheld_when_the_launch_differs():
+    wl = bench.WORKLOADS[bench.DEFAULT_WORKLOAD]
+    key = bench.workload_key(wl["w"], wl["B"], wl["S_local"], wl["H"], wl["D"], "tma")
+    p = plan_dict(wl["w"], wl["B"], wl["S_local"], wl["H"], wl["D"])
+    assert bench.ncu_traffic(key, p, 0)[1] == "ncu"
+    assert bench.ncu_traffic(key, dict(p, grid=p["grid"] + 1), 0) == (
+        None, "the capture was taken with another launch shape")
+    assert bench.ncu_traffic(key, p, 1)[0] is None                 # chunked launches
+    assert bench.ncu_traffic("tma:w3_B1_S7_H3_D8_bf16", p, 0) == (
+        None, "no ncu capture of this kernel and workload")
+
+
+def test_workload_table_names_each_workload_by_its_sizes():
+    for name, wl in bench.WORKLOADS.items():
+        parts = {p[0]: int(p[1:]) for p in name.split("_")}
+        assert parts["w"] == wl["w"] and parts["S"] == wl["S_local"]
+        assert parts["H"] == wl["H"] and parts["D"] == wl["D"]
+        assert parts.get("B", 1) == wl["B"]
+    assert bench.DEFAULT_WORKLOAD in bench.WORKLOADS
