@@ -363,28 +363,36 @@ int ulysses_a2a_peer_create(ulysses_a2a_ctx *ctx, int rank, int world,
  * Fails without mapping anything if a record is malformed. */
 int ulysses_a2a_peer_open(ulysses_a2a_peer *peer, const void *handles);
 
-/* Step 1: copy this rank's input slab into its own window (asynchronous on
- * stream). mode 0: in_local is [B, S_local, H, D] with row_pitch (0 = dense,
- * else >= H*D elements between rows, as in ulysses_a2a_desc_t); mode 1:
- * in_local is [B, S_local*w, H/w, D] dense and row_pitch must be 0. The
- * window receives the dense slab. If in_local is this rank's own window
- * (ulysses_a2a_peer_window(peer, rank)) holding the dense slab, the slab was
- * written in place and nothing is copied or launched (zero-copy publish: the
- * producer of the slab writes into the window directly, after the barrier of
- * step 4 of the previous exchange). */
+/* Step 1: copy this rank's input slab into its own window, from byte
+ * window_offset on (asynchronous on stream). mode 0: in_local is
+ * [B, S_local, H, D] with row_pitch (0 = dense, else >= H*D elements between
+ * rows, as in ulysses_a2a_desc_t); mode 1: in_local is [B, S_local*w, H/w, D]
+ * dense and row_pitch must be 0. The window receives the dense slab.
+ * window_offset is a multiple of the element size, and the slab must fit in
+ * the window after it. Several slabs can share a window at different offsets
+ * (for example the T tensors of a head-packed exchange).
+ * If in_local is the window itself at that offset holding the dense slab, the
+ * slab was written in place and nothing is copied or launched (zero-copy
+ * publish: the producer of the slab writes into the window directly, after
+ * the barrier of step 4 of the previous exchange). */
 int ulysses_a2a_peer_publish(ulysses_a2a_peer *peer, const void *in_local,
                              int64_t B, int64_t S_local, int64_t H, int64_t D,
-                             int mode, int64_t row_pitch, void *stream);
+                             int mode, int64_t row_pitch, size_t window_offset,
+                             void *stream);
 
-/* Step 3: write this rank's output slab from every rank's published window
- * (asynchronous on stream; VEC kernel, peer loads). out_local is on ctx's
- * device, caller-owned, and overlaps no window. mode 0: out_local is
- * [B, S_local*w, H/w, D] dense, row_pitch must be 0; mode 1: out_local is
- * [B, S_local, H, D] with row_pitch (0 = dense). Requires
- * ulysses_a2a_peer_open to have succeeded. */
+/* Step 3: write this rank's output slab from every rank's published window,
+ * each read from byte window_offset on (asynchronous on stream; VEC kernel,
+ * peer loads). out_local is on ctx's device, caller-owned, and overlaps no
+ * window. row_pitch belongs to the [B, S_local, H, D] side: in mode 0 that is
+ * the windows (read with that pitch: e.g. tensor t of a head-packed slab
+ * published whole, with row_pitch = T*H*D and window_offset = t*H*D*elem_bytes)
+ * and out_local is [B, S_local*w, H/w, D] dense; in mode 1 it is out_local,
+ * [B, S_local, H, D] with row_pitch (0 = dense), and the windows hold dense
+ * [B, S_local*w, H/w, D] slabs. Requires ulysses_a2a_peer_open to have
+ * succeeded. */
 int ulysses_a2a_peer_pull(ulysses_a2a_peer *peer, void *out_local, int64_t B,
                           int64_t S_local, int64_t H, int64_t D, int mode,
-                          int64_t row_pitch, void *stream);
+                          int64_t row_pitch, size_t window_offset, void *stream);
 
 /* Base address of rank k's window as this process sees it (NULL if k is out
  * of range or not mapped yet), and the window size in bytes. */

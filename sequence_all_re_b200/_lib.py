@@ -200,9 +200,9 @@ def _load() -> ctypes.CDLL:
     lib.ulysses_a2a_peer_create.restype = c_int
     lib.ulysses_a2a_peer_open.argtypes = [P, P]
     lib.ulysses_a2a_peer_open.restype = c_int
-    lib.ulysses_a2a_peer_publish.argtypes = [P, P, i64, i64, i64, i64, c_int, i64, P]
+    lib.ulysses_a2a_peer_publish.argtypes = [P, P, i64, i64, i64, i64, c_int, i64, ctypes.c_size_t, P]
     lib.ulysses_a2a_peer_publish.restype = c_int
-    lib.ulysses_a2a_peer_pull.argtypes = [P, P, i64, i64, i64, i64, c_int, i64, P]
+    lib.ulysses_a2a_peer_pull.argtypes = [P, P, i64, i64, i64, i64, c_int, i64, ctypes.c_size_t, P]
     lib.ulysses_a2a_peer_pull.restype = c_int
     lib.ulysses_a2a_peer_window.argtypes = [P, c_int]
     lib.ulysses_a2a_peer_window.restype = P
@@ -342,16 +342,18 @@ def ulysses_a2a_peer_open(peer, records) -> int:
     return lib.ulysses_a2a_peer_open(peer, buf)
 
 
-def ulysses_a2a_peer_publish(peer, in_ptr, B, S_local, H, D, mode, row_pitch, stream) -> int:
+def ulysses_a2a_peer_publish(peer, in_ptr, B, S_local, H, D, mode, row_pitch, stream,
+                             window_offset=0) -> int:
     return lib.ulysses_a2a_peer_publish(peer, ctypes.c_void_p(int(in_ptr) or None), int(B),
                                         int(S_local), int(H), int(D), int(mode), int(row_pitch),
-                                        ctypes.c_void_p(int(stream)))
+                                        int(window_offset), ctypes.c_void_p(int(stream)))
 
 
-def ulysses_a2a_peer_pull(peer, out_ptr, B, S_local, H, D, mode, row_pitch, stream) -> int:
+def ulysses_a2a_peer_pull(peer, out_ptr, B, S_local, H, D, mode, row_pitch, stream,
+                          window_offset=0) -> int:
     return lib.ulysses_a2a_peer_pull(peer, ctypes.c_void_p(int(out_ptr) or None), int(B),
                                      int(S_local), int(H), int(D), int(mode), int(row_pitch),
-                                     ctypes.c_void_p(int(stream)))
+                                     int(window_offset), ctypes.c_void_p(int(stream)))
 
 
 def ulysses_a2a_peer_window(peer, rank: int) -> int:

@@ -215,8 +215,18 @@ static int ua2a_impl_peer_open(ulysses_a2a_peer* p, const void* handles) {
   return ULYSSES_A2A_OK;
 }
 
-static int ua2a_impl_peer_publish(ulysses_a2a_peer* p, const void* in_local, int64_t B, int64_t S_local,
-                             int64_t H, int64_t D, int mode, int64_t row_pitch, void* stream) {
+// A byte offset into the windows: a multiple of the element size, inside them.
+static int check_window_offset(ulysses_a2a_peer* p, size_t window_offset, const char* who) {
+  if (window_offset % (size_t)p->ctx->elem_bytes != 0 || window_offset > p->window_bytes)
+    return fail(p->ctx, ULYSSES_A2A_ERR_INVALID,
+                std::string(who) + ": window_offset must be a multiple of the element size "
+                                   "inside the window");
+  return ULYSSES_A2A_OK;
+}
+
+static int ua2a_impl_peer_publish(ulysses_a2a_peer* p, const void* in_local, int64_t B,
+                                  int64_t S_local, int64_t H, int64_t D, int mode,
+                                  int64_t row_pitch, size_t window_offset, void* stream) {
   if (p == nullptr) return ULYSSES_A2A_ERR_INVALID;
   ulysses_a2a_ctx* ctx = p->ctx;
   ctx->last_error.clear();
@@ -227,30 +237,33 @@ static int ua2a_impl_peer_publish(ulysses_a2a_peer* p, const void* in_local, int
   if (H % w != 0) return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_publish: H not divisible by the world size");
   if (mode == 1 && row_pitch != 0)
     return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_publish: a mode-1 input is dense (row_pitch 0)");
+  int rc = check_window_offset(p, window_offset, "peer_publish");
+  if (rc) return rc;
+  const size_t room = p->window_bytes - window_offset;
+  void* dst = static_cast<char*>(p->own) + window_offset;
   // the copy, as a one-rank re-layout: mode 0 keeps [B, S, H, D] (dropping the
   // pitch); mode 1 copies [B, S*w, H/w, D]
   const int64_t S1 = mode == 0 ? S_local : S_local * w;
   const int64_t H1 = mode == 0 ? H : H / w;
-  if (in_local == p->own && (row_pitch == 0 || row_pitch == H1 * D)) {
+  if (in_local == dst && (row_pitch == 0 || row_pitch == H1 * D)) {
     // the slab was written into the window in place: nothing to copy
     int64_t bytes = 0;
     if (ua2a::mul_overflows(B, S1, &bytes) || ua2a::mul_overflows(bytes, H1, &bytes) ||
         ua2a::mul_overflows(bytes, D, &bytes) ||
-        ua2a::mul_overflows(bytes, (int64_t)ctx->elem_bytes, &bytes) ||
-        (uint64_t)bytes > (uint64_t)p->window_bytes)
+        ua2a::mul_overflows(bytes, (int64_t)ctx->elem_bytes, &bytes) || (uint64_t)bytes > room)
       return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_publish: the slab exceeds the window");
     return ULYSSES_A2A_OK;
   }
   const void* in[1] = {in_local};
-  void* out[1] = {p->own};
+  void* out[1] = {dst};
   ulysses_a2a_plan_t pl;
-  int rc = plan_for(ctx, in, out, B, S1, H1, D, 1, 0, 0, &pl, row_pitch);
+  rc = plan_for(ctx, in, out, B, S1, H1, D, 1, 0, 0, &pl, row_pitch);
   if (rc) return rc;
   if (pl.units == 0) return ULYSSES_A2A_OK;
-  if ((uint64_t)pl.payload_bytes > (uint64_t)p->window_bytes)
+  if ((uint64_t)pl.payload_bytes > room)
     return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_publish: the slab (" + std::to_string(pl.payload_bytes) +
-                                                  " bytes) exceeds the window (" +
-                                                  std::to_string(p->window_bytes) + " bytes)");
+                                                  " bytes) exceeds the window (" + std::to_string(room) +
+                                                  " bytes from the offset)");
   DeviceGuard g(ctx->device);
   if (!g.ok) return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "cannot select the context's device");
   const int64_t in_bytes = ((B * S1 - 1) * pl.row_pitch + H1 * D) * (int64_t)ctx->elem_bytes;
@@ -259,36 +272,42 @@ static int ua2a_impl_peer_publish(ulysses_a2a_peer* p, const void* in_local, int
   return run_device(ctx, in, out, B, S1, H1, D, 1, 0, 0, static_cast<cudaStream_t>(stream), pl);
 }
 
-static int ua2a_impl_peer_pull(ulysses_a2a_peer* p, void* out_local, int64_t B, int64_t S_local, int64_t H,
-                          int64_t D, int mode, int64_t row_pitch, void* stream) {
+static int ua2a_impl_peer_pull(ulysses_a2a_peer* p, void* out_local, int64_t B, int64_t S_local,
+                               int64_t H, int64_t D, int mode, int64_t row_pitch,
+                               size_t window_offset, void* stream) {
   if (p == nullptr) return ULYSSES_A2A_ERR_INVALID;
   ulysses_a2a_ctx* ctx = p->ctx;
   ctx->last_error.clear();
   if (!p->open) return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_pull: the peer windows are not open");
   const int w = p->world;
-  if (mode == 0 && row_pitch != 0)
-    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_pull: a mode-0 output is dense (row_pitch 0)");
+  int rc = check_window_offset(p, window_offset, "peer_pull");
+  if (rc) return rc;
+  // every rank's window, read from the offset on
+  std::vector<const void*> ins(w);
+  for (int k = 0; k < w; ++k) ins[k] = static_cast<const char*>(p->bases[k]) + window_offset;
   std::vector<void*> outs(w, nullptr);
   outs[p->rank] = out_local;
   std::string err;
   ulysses_a2a_plan_t pl;
-  int rc = ua2a::make_plan(p->bases.data(), outs.data(), B, S_local, H, D, w, mode, 0, ctx->elem_bytes,
-                           ULYSSES_A2A_PATH_VEC, ctx->tuning, ctx->num_sms, &pl, &err, row_pitch,
-                           p->rank);
+  // row_pitch belongs to the [B, S, H, D] side: the windows in mode 0, the output in mode 1
+  rc = ua2a::make_plan(ins.data(), outs.data(), B, S_local, H, D, w, mode, 0, ctx->elem_bytes,
+                       ULYSSES_A2A_PATH_VEC, ctx->tuning, ctx->num_sms, &pl, &err, row_pitch, p->rank);
   if (rc) return fail(ctx, rc, "peer_pull: " + err);
   if (pl.units == 0) return ULYSSES_A2A_OK;
-  if ((uint64_t)pl.payload_bytes > (uint64_t)p->window_bytes)
-    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_pull: the slab (" + std::to_string(pl.payload_bytes) +
+  const int64_t strided_bytes = ((B * S_local - 1) * pl.row_pitch + H * D) * (int64_t)ctx->elem_bytes;
+  const int64_t window_side = mode == 0 ? strided_bytes : pl.payload_bytes;
+  if ((uint64_t)window_side > (uint64_t)(p->window_bytes - window_offset))
+    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_pull: the slab (" + std::to_string(window_side) +
                                                   " bytes) exceeds the windows (" +
-                                                  std::to_string(p->window_bytes) + " bytes)");
+                                                  std::to_string(p->window_bytes - window_offset) +
+                                                  " bytes from the offset)");
   DeviceGuard g(ctx->device);
   if (!g.ok) return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "cannot select the context's device");
-  const int64_t out_bytes = mode == 0 ? pl.payload_bytes
-                                      : ((B * S_local - 1) * pl.row_pitch + H * D) * (int64_t)ctx->elem_bytes;
+  const int64_t out_bytes = mode == 0 ? pl.payload_bytes : strided_bytes;
   const void* o[1] = {out_local};
   rc = check_residency(ctx, o, 1, out_bytes, "output");
   if (rc) return rc;
-  return run_device(ctx, p->bases.data(), outs.data(), B, S_local, H, D, w, mode, 0,
+  return run_device(ctx, ins.data(), outs.data(), B, S_local, H, D, w, mode, 0,
                     static_cast<cudaStream_t>(stream), pl, 0, -1, p->rank);
 }
 
@@ -343,15 +362,21 @@ int ulysses_a2a_peer_open(ulysses_a2a_peer* p, const void* handles) {
 }
 
 int ulysses_a2a_peer_publish(ulysses_a2a_peer* p, const void* in_local, int64_t B, int64_t S_local,
-                             int64_t H, int64_t D, int mode, int64_t row_pitch, void* stream) {
-  return no_throw([&] { return ua2a_impl_peer_publish(p, in_local, B, S_local, H, D, mode,
-                                                      row_pitch, stream); });
+                             int64_t H, int64_t D, int mode, int64_t row_pitch,
+                             size_t window_offset, void* stream) {
+  return no_throw([&] {
+    return ua2a_impl_peer_publish(p, in_local, B, S_local, H, D, mode, row_pitch, window_offset,
+                                  stream);
+  });
 }
 
 int ulysses_a2a_peer_pull(ulysses_a2a_peer* p, void* out_local, int64_t B, int64_t S_local,
-                          int64_t H, int64_t D, int mode, int64_t row_pitch, void* stream) {
-  return no_throw([&] { return ua2a_impl_peer_pull(p, out_local, B, S_local, H, D, mode, row_pitch,
-                                                   stream); });
+                          int64_t H, int64_t D, int mode, int64_t row_pitch, size_t window_offset,
+                          void* stream) {
+  return no_throw([&] {
+    return ua2a_impl_peer_pull(p, out_local, B, S_local, H, D, mode, row_pitch, window_offset,
+                               stream);
+  });
 }
 
 int ulysses_a2a_peer_close(ulysses_a2a_peer* p) {

@@ -77,13 +77,13 @@ class NativePeer:
     def open(self, records) -> None:
         self._check(_lib.ulysses_a2a_peer_open(self._peer, records))
 
-    def publish(self, x, B, S, H, D, mode, row_pitch, stream) -> None:
+    def publish(self, x, B, S, H, D, mode, row_pitch, stream, window_offset=0) -> None:
         self._check(_lib.ulysses_a2a_peer_publish(self._peer, x.data_ptr(), B, S, H, D, mode,
-                                                  row_pitch, stream.cuda_stream))
+                                                  row_pitch, stream.cuda_stream, window_offset))
 
-    def pull(self, out, B, S, H, D, mode, row_pitch, stream) -> None:
+    def pull(self, out, B, S, H, D, mode, row_pitch, stream, window_offset=0) -> None:
         self._check(_lib.ulysses_a2a_peer_pull(self._peer, out.data_ptr(), B, S, H, D, mode,
-                                               row_pitch, stream.cuda_stream))
+                                               row_pitch, stream.cuda_stream, window_offset))
 
     def window(self, rank: int) -> int:
         return _lib.ulysses_a2a_peer_window(self._peer, rank) if self._peer is not None else 0
@@ -288,6 +288,75 @@ class PeerExchange:
         t = self.native.window_tensor(shape, dtype)
         self._in_place = t.data_ptr()
         return t
+
+    def all_to_all_4d_packed(self, x, mode: int, out=None, stream=None):
+        """Exchange T tensors packed along the head dimension with one barrier pair.
+
+        mode 0: ``x`` is this rank's contiguous [B, S_local, T, H, D] slab (for
+        example its packed q/k/v projection output); returns T tensors
+        [B, S_local*w, H//w, D]. It is published whole, and each tensor is
+        pulled from the windows at its head offset with row pitch T*H*D.
+        mode 1: ``x`` is a list of T tensors [B, S_local*w, H//w, D]; returns
+        the packed [B, S_local, T, H, D] slab (``out`` may be given). The T
+        slabs share the window at consecutive offsets, and each is pulled
+        into its slot of the packed output.
+        Same bytes as T calls of ``all_to_all_4d``; 2 barriers instead of 2T.
+        """
+        if self.disabled_reason is not None:
+            raise RuntimeError(f"peer exchange disabled: {self.disabled_reason}")
+        if mode not in (0, 1):
+            raise ValueError("mode must be 0 or 1")
+        w, E = self.world, self.elem_bytes
+        if mode == 0:
+            if x.dim() != 5 or not x.is_contiguous():
+                raise ValueError("mode 0 takes a contiguous [B, S_local, T, H, D] slab")
+            B, S, T, H, D = (int(v) for v in x.shape)
+            srcs = [x]
+            dtype, device = x.dtype, x.device
+        else:
+            T = len(x)
+            if T < 1 or x[0].dim() != 4:
+                raise ValueError("mode 1 takes a list of T tensors [B, S_local*w, H/w, D]")
+            B, Sg, Hw, D = (int(v) for v in x[0].shape)
+            S, H = Sg // w, Hw * w
+            srcs = list(x)
+            dtype, device = x[0].dtype, x[0].device
+            if Sg % w or any(tuple(t.shape) != (B, Sg, Hw, D) or not t.is_contiguous()
+                             for t in srcs):
+                raise ValueError("the T tensors must be contiguous [B, S_local*w, H/w, D]")
+        if H % w:
+            raise ValueError("H must be divisible by the world size")
+        if any(t.device != self.device or t.element_size() != E for t in srcs):
+            raise ValueError(f"tensors must hold {E}-byte elements on {self.device}")
+        slab = B * S * H * D * E                     # one tensor's slab, either layout
+        if mode == 0:
+            outs = out if out is not None else [
+                torch.empty((B, S * w, H // w, D), dtype=dtype, device=device) for _ in range(T)]
+        else:
+            outs = out if out is not None else torch.empty((B, S, T, H, D), dtype=dtype,
+                                                           device=device)
+        if slab == 0:
+            return outs
+        self._agree_signature(("packed", mode, T, B, S, H, D, dtype))
+        self._ensure_window(T * slab)
+        if stream is None:
+            stream = self.native.current_stream()
+        self._barrier(stream)        # every rank is done reading the windows
+        if mode == 0:
+            # the packed rows published whole: T*H heads of D
+            self.native.publish(x, B, S, T * H, D, 0, 0, stream)
+        else:
+            for t in range(T):
+                self.native.publish(srcs[t], B, S, H, D, 1, 0, stream, window_offset=t * slab)
+        self._barrier(stream)        # every window holds its slabs
+        for t in range(T):
+            if mode == 0:
+                self.native.pull(outs[t], B, S, H, D, 0, T * H * D, stream,
+                                 window_offset=t * H * D * E)
+            else:
+                self.native.pull(outs[:, :, t], B, S, H, D, 1, T * H * D, stream,
+                                 window_offset=t * slab)
+        return outs
 
     def all_to_all_4d(self, x: torch.Tensor, mode: int, chunked: bool = False, out=None,
                       stream=None) -> torch.Tensor:

@@ -108,10 +108,10 @@ int main(void) {
             CHECK(cudaMemset(dout[k], 0xFF, bytes) == cudaSuccess, "poison");
         }
         for (int k = 0; k < W; ++k)
-            CHECK(ulysses_a2a_peer_publish(peer[k], din[k], B, S, H, D, 0, 0, NULL) ==
+            CHECK(ulysses_a2a_peer_publish(peer[k], din[k], B, S, H, D, 0, 0, 0, NULL) ==
                       ULYSSES_A2A_OK, ulysses_a2a_last_error(rctx[k]));
         for (int k = 0; k < W; ++k)
-            CHECK(ulysses_a2a_peer_pull(peer[k], dout[k], B, S, H, D, 0, 0, NULL) ==
+            CHECK(ulysses_a2a_peer_pull(peer[k], dout[k], B, S, H, D, 0, 0, 0, NULL) ==
                       ULYSSES_A2A_OK, ulysses_a2a_last_error(rctx[k]));
         for (int k = 0; k < W; ++k) {
             CHECK(cudaMemcpy(hout[k], dout[k], bytes, cudaMemcpyDeviceToHost) == cudaSuccess, "D2H");

@@ -58,12 +58,19 @@ class ShmNative:
                 self.peers[k] = shared_memory.SharedMemory(name=name)
         self.log.append(("open",))
 
-    def _win(self, k, dtype, shape):
+    def _win(self, k, dtype, shape, offset_bytes=0, strides=None):
+        """Rank k's window as a tensor of `shape` from byte offset_bytes on
+        (dense, or with the given element strides)."""
         shm = self.own if k == self.rank else self.peers[k]
-        n = 1
-        for v in shape:
-            n *= v
-        return torch.frombuffer(shm.buf, dtype=dtype, count=n).view(shape)
+        esz = torch.empty((), dtype=dtype).element_size()
+        whole = torch.frombuffer(shm.buf, dtype=dtype, count=shm.size // esz)
+        if strides is None:
+            strides = []
+            acc = 1
+            for v in reversed(shape):
+                strides.insert(0, acc)
+                acc *= v
+        return whole.as_strided(tuple(shape), tuple(strides), offset_bytes // esz)
 
     def window(self, rank):
         shm = self.own if rank == self.rank else self.peers.get(rank)
@@ -77,25 +84,28 @@ class ShmNative:
             n *= v
         return torch.frombuffer(self.own.buf, dtype=dtype, count=n).view(shape)
 
-    def publish(self, x, B, S, H, D, mode, row_pitch, stream):
+    def publish(self, x, B, S, H, D, mode, row_pitch, stream, window_offset=0):
         time.sleep(self.publish_delay)
         w = self.world
         shape = (B, S, H, D) if mode == 0 else (B, S * w, H // w, D)
-        self._win(self.rank, x.dtype, shape).copy_(x)
+        src = x if tuple(x.shape) == shape else x.reshape(shape)   # a packed slab: T*H heads
+        self._win(self.rank, x.dtype, shape, window_offset).copy_(src)
         self.log.append("publish")
 
-    def pull(self, out, B, S, H, D, mode, row_pitch, stream):
+    def pull(self, out, B, S, H, D, mode, row_pitch, stream, window_offset=0):
         time.sleep(self.pull_delay)
         w, k = self.world, self.rank
         Hw = H // w
         if mode == 0:
+            p = row_pitch or H * D                 # the windows' row pitch
             o = out.view(B, w, S, Hw, D)
             for j in range(w):
-                o[:, j] = self._win(j, out.dtype, (B, S, H, D))[:, :, k * Hw:(k + 1) * Hw]
+                win = self._win(j, out.dtype, (B, S, H, D), window_offset, (S * p, p, D, 1))
+                o[:, j] = win[:, :, k * Hw:(k + 1) * Hw]
         else:
             for r in range(w):
-                out[:, :, r * Hw:(r + 1) * Hw] = self._win(r, out.dtype,
-                                                           (B, S * w, Hw, D))[:, k * S:(k + 1) * S]
+                win = self._win(r, out.dtype, (B, S * w, Hw, D), window_offset)
+                out[:, :, r * Hw:(r + 1) * Hw] = win[:, k * S:(k + 1) * S]
         self.log.append("pull")
 
     def unmap(self):
@@ -189,6 +199,25 @@ def _worker(rank, world, port, scenario, q):
             rep["ok"].append(torch.equal(x.grad.view(torch.int16),
                                          oracle.ulysses_a2a(gys, 1)[rank].view(torch.int16)))
             rep["closed"] = ex.close()
+        elif scenario == "packed":
+            # q, k, v packed per rank: one publish and T pulls in mode 0; T publishes
+            # at window offsets and T pulls into the packed slots in mode 1
+            native = ShmNative(rank, publish_delay=0.05 if rank == 1 else 0.0,
+                               pull_delay=0.2 if rank == 1 else 0.0)
+            ex = PeerExchange(native=native, elem_bytes=2)
+            T, B, S, H, D = 3, 2, 5, 4, 8
+            packed = normal_slabs((B, S, T, H, D), world, "bf16", seed0=600)
+            flat = [t.reshape(-1) for t in packed]
+            outs = ex.all_to_all_4d_packed(packed[rank], 0)
+            for t in range(T):
+                want = oracle.ulysses_a2a_pitched(flat, 0, world, B, S, H, D, T * H * D,
+                                                  offset=t * H * D)[rank]
+                rep["ok"].append(torch.equal(outs[t].reshape(-1).view(torch.int16),
+                                             want.view(torch.int16)))
+            back = ex.all_to_all_4d_packed(outs, 1)
+            rep["ok"].append(torch.equal(back.view(torch.int16), packed[rank].view(torch.int16)))
+            rep["closed"] = ex.close()
+            rep["log"] = native.log
         elif scenario == "fail_build":
             native = ShmNative(rank, fail_create=(rank == 1))
             ex = PeerExchange(native=native, elem_bytes=2)
@@ -259,6 +288,15 @@ def test_autograd_backward_is_the_inverse_exchange():
         assert rep["errors"] == [], rep
         assert rep["ok"] == [True, True], rep
         assert rep["closed"] is True
+
+
+def test_packed_exchange_uses_one_barrier_pair():
+    for rep in _run("packed", 500):
+        assert rep["errors"] == [], rep
+        assert rep["ok"] == [True] * 4, rep
+        assert rep["closed"] is True
+        ops = [e for e in rep["log"] if isinstance(e, str)]
+        assert ops == ["publish"] + ["pull"] * 3 + ["publish"] * 3 + ["pull"] * 3
 
 
 def test_failed_window_build_disables_every_rank():

@@ -297,3 +297,65 @@ def test_publishing_the_own_window_copies_nothing():
         g.check_guards()
     finally:
         ranks.close()
+
+
+def test_packed_exchange_through_window_offsets():
+    """q, k, v packed per rank: one publish of the packed slab and a pull per tensor
+    (windows read with row pitch T*H*D at the tensor's head offset); back in mode 1
+    with the T slabs at consecutive window offsets, pulled into the packed slots."""
+    T, w, B, S, H, D = 3, 4, 2, 37, 8, 64
+    E = 2
+    slab = B * S * H * D * E
+    packed_cpu = normal_slabs((B, S, T, H, D), w, "bf16", seed0=880)
+    flat = [t.reshape(-1) for t in packed_cpu]
+    ranks = LocalRanks(w, E, T * slab).open()
+    try:
+        stream = torch.cuda.current_stream().cuda_stream
+        packed = [t.cuda() for t in packed_cpu]
+        n0 = ranks.launches()
+        for k in range(w):
+            assert _lib.ulysses_a2a_peer_publish(ranks.peers[k], packed[k].data_ptr(), B, S, T * H,
+                                                 D, 0, 0, stream) == _lib.OK
+        outs = [[torch.empty(B, S * w, H // w, D, dtype=torch.bfloat16, device="cuda")
+                 for _ in range(T)] for _ in range(w)]
+        for k in range(w):
+            for t in range(T):
+                rc = _lib.ulysses_a2a_peer_pull(ranks.peers[k], outs[k][t].data_ptr(), B, S, H, D, 0,
+                                                T * H * D, stream, window_offset=t * H * D * E)
+                assert rc == _lib.OK, ranks.ctxs[k].last_error()
+        torch.cuda.synchronize()
+        assert ranks.launches() - n0 == w + w * T
+        for t in range(T):
+            want = oracle.ulysses_a2a_pitched(flat, 0, w, B, S, H, D, T * H * D, offset=t * H * D)
+            for k in range(w):
+                assert torch.equal(bits(outs[k][t].cpu()).reshape(-1), bits(want[k])), (t, k)
+        # mode 1: rank k's T slabs at window offsets t*slab, pulled into packed slots
+        for k in range(w):
+            for t in range(T):
+                assert _lib.ulysses_a2a_peer_publish(ranks.peers[k], outs[k][t].data_ptr(), B, S, H,
+                                                     D, 1, 0, stream, window_offset=t * slab) == _lib.OK
+        back = [torch.full((B, S, T, H, D), -1, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+                for _ in range(w)]
+        for k in range(w):
+            for t in range(T):
+                rc = _lib.ulysses_a2a_peer_pull(ranks.peers[k], back[k][:, :, t].data_ptr(), B, S, H,
+                                                D, 1, T * H * D, stream, window_offset=t * slab)
+                assert rc == _lib.OK, ranks.ctxs[k].last_error()
+        torch.cuda.synchronize()
+        for k in range(w):
+            assert torch.equal(bits(back[k].cpu()), bits(packed_cpu[k])), k
+        # offsets: not a multiple of the element size, past the window, or leaving too
+        # little room for the slab
+        p0 = ranks.peers[0]
+        n1 = ranks.launches()
+        assert _lib.ulysses_a2a_peer_publish(p0, packed[0].data_ptr(), B, S, H, D, 0, T * H * D,
+                                             stream, window_offset=1) == _lib.ERR_INVALID
+        assert _lib.ulysses_a2a_peer_pull(p0, outs[0][0].data_ptr(), B, S, H, D, 0, T * H * D,
+                                          stream, window_offset=T * slab + 2) == _lib.ERR_INVALID
+        assert _lib.ulysses_a2a_peer_publish(p0, outs[0][0].data_ptr(), B, S, H, D, 1, 0, stream,
+                                             window_offset=T * slab - slab // 2) == _lib.ERR_INVALID
+        assert _lib.ulysses_a2a_peer_pull(p0, outs[0][0].data_ptr(), B, S, H, D, 0, T * H * D,
+                                          stream, window_offset=T * H * D * E) == _lib.ERR_INVALID
+        assert ranks.launches() == n1
+    finally:
+        ranks.close()

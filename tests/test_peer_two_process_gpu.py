@@ -61,6 +61,22 @@ def _worker(rank, world, port, q):
         report["in_place_ok"] = torch.equal(y.cpu().view(torch.int16),
                                             oracle.ulysses_a2a(xs, 0)[rank].view(torch.int16))
         report["in_place_launches"] = ex.native.launch_count - n0
+        # q, k, v packed: one barrier pair per direction
+        T = 3
+        shape = (2, 37, T, 8, 64)
+        packed = normal_slabs(shape, world, "bf16", seed0=555)
+        flat = [t.reshape(-1) for t in packed]
+        outs = ex.all_to_all_4d_packed(packed[rank].cuda(), 0)
+        ok = True
+        for t in range(T):
+            want = oracle.ulysses_a2a_pitched(flat, 0, world, 2, 37, 8, 64, T * 8 * 64,
+                                              offset=t * 8 * 64)[rank]
+            ok = ok and torch.equal(outs[t].cpu().reshape(-1).view(torch.int16),
+                                    want.view(torch.int16))
+        back = ex.all_to_all_4d_packed(outs, 1)
+        torch.cuda.synchronize()
+        report["packed_ok"] = ok and torch.equal(back.cpu().view(torch.int16),
+                                                 packed[rank].view(torch.int16))
         # autograd: the backward of a mode-0 exchange is the mode-1 exchange
         from sequence_all_re_b200.autograd import peer_all_to_all_4d
         from synth import uniform_slabs
@@ -109,6 +125,7 @@ def test_two_processes_exchange_through_ipc_windows():
         # publish + pull per exchange (per plane when chunked), two exchanges per case,
         # then one in-place exchange: a pull and nothing else
         assert rep["in_place_ok"] is True and rep["in_place_launches"] == 1
-        assert rep["grad_ok"] is True
-        # ... and a forward + backward exchange of publish + pull each
-        assert rep["launches"] == 2 * 2 * (1 + 2 + 1 + 3) + 1 + 2 * 2
+        assert rep["grad_ok"] is True and rep["packed_ok"] is True
+        # ... a packed exchange each way (1 + 3 then 3 + 3 launches), and a forward +
+        # backward exchange of publish + pull each
+        assert rep["launches"] == 2 * 2 * (1 + 2 + 1 + 3) + 1 + (1 + 3) + (3 + 3) + 2 * 2
