@@ -493,3 +493,33 @@ def test_packed_plan_validation():
     gathered[4] = 0
     rc, _, msg = _lib.ulysses_a2a_plan_ex(gathered, strided, B, S, H, D, w, 1, 0, 2, ntensors=T)
     assert rc == ERR_INVALID and "NULL" in msg
+
+
+@pytest.mark.parametrize("compiler,std", [("gcc", "c99"), ("gcc", "c11"), ("g++", "c++11"),
+                                          ("g++", "c++17")])
+def test_header_compiles_standalone(tmp_path, compiler, std):
+    """The public header is self-contained C (and C++): it compiles on its own,
+    pedantically, with every warning an error, and sizeof the ABI structs
+    agrees with the Python mirrors."""
+    import shutil
+    import subprocess
+
+    if shutil.which(compiler) is None:
+        pytest.skip(f"{compiler} not available")
+    ext = "c" if compiler == "gcc" else "cpp"
+    src = tmp_path / f"hdr.{ext}"
+    src.write_text(
+        '#include "ulysses_a2a.h"\n'
+        "#include <stdio.h>\n"
+        "int main(void) {\n"
+        '  printf("%d %d %d %d\\n", (int)sizeof(ulysses_a2a_plan_t),\n'
+        "         (int)sizeof(ulysses_a2a_tuning_t), (int)sizeof(ulysses_a2a_desc_t),\n"
+        "         ULYSSES_A2A_PEER_HANDLE_BYTES);\n"
+        "  return 0;\n"
+        "}\n")
+    exe = tmp_path / "hdr"
+    subprocess.run([compiler, f"-std={std}", "-pedantic", "-Wall", "-Wextra", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert [int(v) for v in out] == [ctypes.sizeof(_lib.PlanT), ctypes.sizeof(_lib.TuningT),
+                                     ctypes.sizeof(_lib.DescT), _lib.PEER_HANDLE_BYTES]
