@@ -523,3 +523,55 @@ def test_header_compiles_standalone(tmp_path, compiler, std):
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
     assert [int(v) for v in out] == [ctypes.sizeof(_lib.PlanT), ctypes.sizeof(_lib.TuningT),
                                      ctypes.sizeof(_lib.DescT), _lib.PEER_HANDLE_BYTES]
+
+
+# ---- planner invariants over random shapes (property test) -------------------
+
+from hypothesis import given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@settings(max_examples=300, deadline=None)
+@given(w=st.sampled_from([1, 2, 3, 4, 8, 16]), hw=st.integers(1, 6), B=st.integers(1, 4),
+       S=st.integers(1, 5000), D=st.sampled_from([1, 3, 8, 13, 64, 128, 256]),
+       E=st.sampled_from([1, 2, 4, 8]), mode=st.sampled_from([0, 1]),
+       chunked=st.sampled_from([0, 1]), path=st.sampled_from([PATH_AUTO, PATH_VEC]),
+       rows=st.sampled_from([0, 0, 1, 7, 64]), ntensors=st.sampled_from([1, 1, 2, 3]))
+def test_planner_invariants(w, hw, B, S, D, E, mode, chunked, path, rows, ntensors):
+    H = hw * w
+    if ntensors * w > 64:
+        return
+    slab = B * S * H * D * E
+    step = (slab * ntensors + 4095) // 4096 * 4096
+    strided = [(1 << 40) + k * step for k in range(w)]
+    gathered = [(1 << 44) + k * step for k in range(ntensors * w)]
+    ins, outs = (strided, gathered) if mode == 0 else (gathered, strided)
+    rc, p, msg = _lib.ulysses_a2a_plan_ex(ins, outs, B, S, H, D, w, mode, chunked, E,
+                                          forced_path=path, ntensors=ntensors,
+                                          rows_per_tile=rows)
+    assert rc == OK, msg
+    nb = 1 if chunked else B
+    # tiles cover every sequence row exactly once per (r, b, j) block
+    assert 1 <= p.rows_per_tile <= min(S, 256)
+    assert p.tiles_per_block == -(-S // p.rows_per_tile)
+    assert p.tail_rows == S % p.rows_per_tile
+    assert p.units == ntensors * w * w * nb * p.tiles_per_block
+    assert p.payload_bytes == ntensors * w * slab
+    assert p.launches == (B if chunked else 1)
+    assert p.row_bytes == hw * D * E and p.row_pitch == ntensors * H * D
+    if rows:
+        assert p.rows_per_tile == min(rows, S)
+    if p.path == PATH_TMA:
+        assert path == PATH_AUTO and ntensors == 1
+        assert (D * E) % 16 == 0 and w <= 8 and D <= 256 and hw <= 256
+        assert p.rows_per_tile * p.row_bytes <= 64 * 1024
+        assert 32 <= p.block == 32 * p.producers <= 256
+        assert p.smem_bytes <= 220 * 1024
+        assert p.grid == -(-p.units // p.chunk_units)
+    else:
+        assert p.path == PATH_VEC
+        v = p.vec_bytes
+        assert v in (1, 2, 4, 8, 16) and p.row_bytes % v == 0 and (p.row_pitch * E) % v == 0
+        # the widest width the run length and the pitch allow (pointers are 4 KiB aligned)
+        assert v == 16 or (p.row_bytes % (2 * v) or (p.row_pitch * E) % (2 * v))
+        assert p.grid == p.units and p.block == 256
