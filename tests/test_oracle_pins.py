@@ -4,7 +4,7 @@ import pytest
 import torch
 
 import oracle
-from oracle_pins import ALL_PINS, load_table, table_names
+from oracle_pins import ALL_PINS, load_table, permute_formulation, table_names
 
 
 def _run(xs, mode, chunked):
@@ -79,3 +79,32 @@ def test_empty_index_sets_are_a_no_op():
         assert all(tuple(t.shape) == (B, S * 2, H // 2, D) for t in y)
     # a zero size does not hide a non-empty slab's NULL pointer
     assert lib.oracle_ulysses_a2a(nul, nul, 1, 1, 2, 1, 2, 0, 2) == -1
+
+
+# ---- the same facts over random small shapes (property test) ------------------
+
+from hypothesis import given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@settings(max_examples=200, deadline=None, derandomize=True, database=None)
+@given(w=st.integers(1, 6), hw=st.integers(1, 4), B=st.integers(1, 3), S=st.integers(1, 9),
+       D=st.integers(1, 9), E=st.sampled_from([1, 2, 4, 8]), seed=st.integers(0, 2**31 - 1))
+def test_oracle_properties_on_random_shapes(w, hw, B, S, D, E, seed):
+    """mode 1 undoes mode 0, the maps agree with the independent permute
+    formulation, and chunked equals unchunked, on random small shapes."""
+    H = hw * w
+    dt = {1: torch.uint8, 2: torch.int16, 4: torch.int32, 8: torch.int64}[E]
+    g = torch.Generator().manual_seed(seed)
+    xs = [torch.randint(0, 100, (B, S, H, D), generator=g, dtype=torch.int64).to(dt)
+          for _ in range(w)]
+    y = oracle.ulysses_a2a(xs, 0)
+    want = permute_formulation(xs, 0, w)
+    for r in range(w):
+        assert torch.equal(y[r], want[r])
+    z = oracle.ulysses_a2a(y, 1)
+    for j in range(w):
+        assert torch.equal(z[j], xs[j])
+    yc = oracle.ulysses_a2a(xs, 0, chunked=True)
+    for r in range(w):
+        assert torch.equal(yc[r], y[r])
