@@ -8,8 +8,6 @@ another. Outputs are poisoned and guarded as in test_parity_gpu.py; expected
 values come from the oracle only.
 """
 
-import ctypes
-
 import pytest
 import torch
 
@@ -250,11 +248,9 @@ def test_peer_errors_launch_nothing():
         assert _lib.ulysses_a2a_peer_pull(p0, 0, B, 0, H, D, 0, 0, stream) == _lib.OK
         assert ranks.launches() == n0
         # bad arguments to create
-        h = ctypes.c_void_p()
         assert _lib.ulysses_a2a_peer_create(c0._ctx, 2, 2, nbytes)[0] == _lib.ERR_INVALID
         assert _lib.ulysses_a2a_peer_create(c0._ctx, 0, 65, nbytes)[0] == _lib.ERR_INVALID
         assert _lib.ulysses_a2a_peer_create(c0._ctx, 0, 2, 0)[0] == _lib.ERR_INVALID
-        del h
         # the context still runs a correct exchange after every rejection
         xs_cpu = normal_slabs((B, S, H, D), w, "bf16")
         want = oracle.ulysses_a2a(xs_cpu, 0)
