@@ -22,11 +22,15 @@
  * is [B, S_local, H, D] and each out_slabs[r] is [B, S_local*w, H/w, D]; in
  * mode 1 the roles are swapped. (B, S_local, H, D) are ALWAYS passed in
  * mode-0-local terms, whichever the mode, as the page's native op receives them.
+ * ulysses_a2a_run_ex adds row-pitched slabs and head-packed tensors (several
+ * tensors in one launch); the ulysses_a2a_peer_* functions run the same map
+ * across GPUs, one process per GPU.
  *
  * Ownership: the caller owns every slab and the stream. The context owns a tiny
  * device status word, a cache of TMA descriptors, and (only if
- * ulysses_a2a_run_host is used) device staging buffers that grow on demand.
- * Nothing returned by this API ever aliases caller memory.
+ * ulysses_a2a_run_host is used) device staging buffers that grow on demand; a
+ * peer object owns its rank's window. Nothing returned by this API ever aliases
+ * caller memory.
  *
  * Launches: every kernel is launched with programmatic stream serialization
  * (programmatic dependent launch) and waits for the previous grid in the
