@@ -110,6 +110,12 @@ class NativePeer:
             if rc != _lib.OK:
                 raise A2AError(rc, "peer_destroy reported a CUDA error (the handle is released)")
 
+    def abandon(self) -> None:
+        """Forget the peer object without unmapping or freeing its window: the
+        memory stays allocated until the process exits (for a teardown the
+        ranks could not agree on)."""
+        self._peer = None
+
     @property
     def launch_count(self) -> int:
         return self.a2a.launch_count
@@ -227,7 +233,12 @@ class PeerExchange:
         if all_unarmed:
             return True
         if not all_armed:
-            self._release_after_failure()
+            # An armed/unarmed split cannot be torn down safely: a peer may still
+            # map this window. Leave it allocated until the process exits, as the
+            # FastVideo communicator does, and disable the exchange.
+            self.native.abandon()
+            self._nbytes = 0
+            self._armed = False
             self._disable("ranks disagreed on whether a window was built during teardown")
             return False
         sync_ok = True

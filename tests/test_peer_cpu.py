@@ -121,6 +121,11 @@ class ShmNative:
             self.own = None
             self.log.append(("release",))
 
+    def abandon(self):
+        self.log.append(("abandon",))
+        self.own = None            # left to the process's exit, never unlinked here
+        self.peers = {}
+
     def current_stream(self):
         return _HostStream()
 
@@ -218,6 +223,20 @@ def _worker(rank, world, port, scenario, q):
             rep["ok"].append(torch.equal(back.view(torch.int16), packed[rank].view(torch.int16)))
             rep["closed"] = ex.close()
             rep["log"] = native.log
+        elif scenario == "split_close":
+            # rank 1 believes its window is gone while rank 0's is armed
+            native = ShmNative(rank)
+            ex = PeerExchange(native=native, elem_bytes=2)
+            ex.all_to_all_4d(normal_slabs((1, 4, 2, 8), world, "bf16")[rank], 0)
+            if rank == 1:
+                ex._armed = False
+            rep["closed"] = ex.close()
+            rep["disabled"] = ex.disabled_reason
+            rep["log"] = native.log
+            try:
+                ex.all_to_all_4d(torch.zeros(1, 4, 2, 8, dtype=torch.bfloat16), 0)
+            except RuntimeError as e:
+                rep["errors"].append(str(e))
         elif scenario == "fail_build":
             native = ShmNative(rank, fail_create=(rank == 1))
             ex = PeerExchange(native=native, elem_bytes=2)
@@ -297,6 +316,15 @@ def test_packed_exchange_uses_one_barrier_pair():
         assert rep["closed"] is True
         ops = [e for e in rep["log"] if isinstance(e, str)]
         assert ops == ["publish"] + ["pull"] * 3 + ["publish"] * 3 + ["pull"] * 3
+
+
+def test_split_teardown_leaks_instead_of_freeing():
+    for rep in _run("split_close", 600):
+        assert rep["closed"] is False and "disagreed" in rep["disabled"], rep
+        # the armed rank leaves its window to the process exit: no unmap, no release
+        if rep["rank"] == 0:
+            assert ("abandon",) in rep["log"] and ("release",) not in rep["log"], rep["log"]
+        assert len(rep["errors"]) == 1 and "disabled" in rep["errors"][0], rep
 
 
 def test_failed_window_build_disables_every_rank():
