@@ -751,6 +751,94 @@ def run_packed(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------- cross-GPU exchange arms (torchrun, N > 1)
+def nccl_all_to_all_4d(x, mode, group=None):
+    """The comparison arm: the same element map as a library all-to-all.
+
+    mode 0: this rank's x [B, S_local, H, D] -> [B, S_local*w, H/w, D]; mode 1
+    the inverse. Head group r is packed contiguous for rank r, exchanged with
+    torch.distributed.all_to_all_single, and the received blocks are laid out
+    rank-major. Plain torch ops and one collective: a baseline, not this
+    library's path."""
+    import torch.distributed as dist
+
+    w = dist.get_world_size(group)
+    if mode == 0:
+        B, S, H, D = x.shape
+        send = x.reshape(B, S, w, H // w, D).permute(2, 0, 1, 3, 4).contiguous()   # [r, b, s, h', d]
+        recv = torch.empty_like(send)                                               # [j, b, s, h', d]
+        dist.all_to_all_single(recv, send, group=group)
+        return recv.permute(1, 0, 2, 3, 4).reshape(B, w * S, H // w, D)
+    B, Sg, Hw, D = x.shape
+    S = Sg // w
+    send = x.reshape(B, w, S, Hw, D).permute(1, 0, 2, 3, 4).contiguous()           # [j, b, s, h', d]
+    recv = torch.empty_like(send)                                                   # [r, b, s, h', d]
+    dist.all_to_all_single(recv, send, group=group)
+    return recv.permute(1, 2, 0, 3, 4).reshape(B, S, w * Hw, D)
+
+
+def run_exchange(args):
+    """Time the Ulysses all-to-all across the GPUs of a torchrun job: each rank
+    holds one rank slab of the workload (w = the number of GPUs); a step is
+    mode 0 then mode 1. --exchange nccl times the library all-to-all above,
+    --exchange peer this library's PeerExchange (windows, peer loads)."""
+    import datetime
+    import torch.distributed as dist
+
+    rank, local_rank, world = env_rank()
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist.init_process_group("nccl", device_id=device, timeout=datetime.timedelta(seconds=120))
+    wl = WORKLOADS[args.workload]
+    B, S, H, D = (wl[k] for k in ("B", "S_local", "H", "D"))
+    if H % world:
+        raise SystemExit(f"H={H} is not divisible by {world} GPUs")
+    x = make_inputs(1, B, S, H, D, "bf16", device, seed0=1234 + rank)[0]
+    ex = None
+    if args.exchange == "peer":
+        from sequence_all_re_b200.peer import PeerExchange
+        ex = PeerExchange(device=local_rank, elem_bytes=2)
+
+        def step():
+            return ex.all_to_all_4d(ex.all_to_all_4d(x, 0), 1)
+    else:
+        def step():
+            return nccl_all_to_all_4d(nccl_all_to_all_4d(x, 0), 1)
+
+    stream = torch.cuda.current_stream(device)
+    for _ in range(args.warmup):
+        z = step()
+    if not torch.equal(z, x):
+        raise SystemExit("round trip mismatch across GPUs")
+    steps = min(args.steps, 200)
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
+    slab = B * S * H * D * 2
+    if rank == 0:
+        print(json.dumps({
+            "metric": "Ulysses all-to-all across GPUs: payload GB/s per step (mode 0 + mode 1)",
+            "value": round(job_gbs(world, 2 * slab, steps, ms), 1), "unit": "GB/s",
+            "n_gpus": world, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": round(ms / steps, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "exchange": args.exchange,
+            "config": {"workload": f"one rank slab per GPU, w = {world}: B={B} S_local={S} H={H} "
+                                   f"D={D} bf16", "parallelism": f"ulysses sp{world}"}}),
+            flush=True)
+    if ex is not None:
+        ex.shutdown()
+    dist.barrier()
+    dist.destroy_process_group()
+
+
 # ---------------------------------------------------------------- reference arm
 def run_reference(args):
     rank, _, world = env_rank()
@@ -829,6 +917,10 @@ def main():
     ap.add_argument("--chunked", type=int, choices=[0, 1, 2], default=0)
     ap.add_argument("--sweep", action="store_true",
                     help="also run the 128 KiB..2 GiB bandwidth sweep (w=2/4/8, bf16/fp32)")
+    ap.add_argument("--exchange", choices=["nccl", "peer"], default=None,
+                    help="multi-GPU Ulysses exchange (one rank slab per GPU, under torchrun): "
+                         "nccl = a library all-to-all baseline, peer = this library's "
+                         "PeerExchange (prints its own line)")
     ap.add_argument("--packed", action="store_true",
                     help="time q, k, v in one packed launch against three per-tensor launches "
                          "(prints its own line)")
@@ -841,6 +933,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.exchange:
+        run_exchange(args)
     elif args.peer_one_gpu:
         run_peer_one_gpu(args)
     elif args.packed:

@@ -79,3 +79,37 @@ def test_reference_arm_rank0_prints_one_line():
     assert d["unit"] == "GB/s" and d["higher_is_better"] is True and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+
+
+def _exchange_worker(rank, world, port, out_q):
+    import oracle
+    from synth import normal_slabs
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        res = []
+        for (B, S, H, D) in ((2, 5, 4, 8), (1, 7, 6, 3)):
+            xs = normal_slabs((B, S, H, D), world, "fp32", seed0=40)
+            y = bench.nccl_all_to_all_4d(xs[rank], 0)
+            z = bench.nccl_all_to_all_4d(y, 1)
+            res.append(torch.equal(y, oracle.ulysses_a2a(xs, 0)[rank]) and torch.equal(z, xs[rank]))
+        out_q.put((rank, res))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_library_all_to_all_comparison_arm_matches_the_oracle_gloo():
+    """bench.py --exchange nccl's all-to-all arm, run here over gloo on CPU
+    tensors: the same element map as the oracle, and mode 1 undoes mode 0."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 33500 + os.getpid() % 500
+    procs = [ctx.Process(target=_exchange_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = sorted(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert got == [(0, [True, True]), (1, [True, True])]
