@@ -22,6 +22,15 @@ nothing is exchanged); `value` = payload of all ranks / the slowest rank's time
 
 `--impl reference` times the CPU oracle (the plain nested-loop definition) on
 the host cores, on a bounded sample of the same workload, as a baseline only.
+
+Other modes, each printing its own line:
+  --sweep          adds the 128 KiB..2 GiB bandwidth sweep (w = 2/4/8, bf16/fp32);
+  --packed         q, k, v in one head-packed launch vs three per-tensor launches;
+  --peer-one-gpu   the cross-GPU exchange's publish and pull kernels, with the
+                   ranks as contexts on one GPU;
+  --exchange X     the Ulysses all-to-all across the GPUs of a torchrun job (one
+                   rank slab per GPU): X = nccl (a library all-to-all baseline)
+                   or peer (PeerExchange).
 """
 
 from __future__ import annotations
