@@ -30,7 +30,9 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "ulysses_oracle.c")
 _LIB = os.path.join(_HERE, "libulysses_oracle.so")
+_LIB_OMP = os.path.join(_HERE, "libulysses_oracle_omp.so")
 _lib = None
+_lib_omp = None
 
 
 def build(force: bool = False, src: str = _SRC, out: str = _LIB, extra=()) -> str:
@@ -40,6 +42,29 @@ def build(force: bool = False, src: str = _SRC, out: str = _LIB, extra=()) -> st
                *extra, "-o", out, src]
         subprocess.run(cmd, check=True)
     return out
+
+
+def build_omp(force: bool = False) -> str:
+    """The same source built with OpenMP: the outer (r, b) loops run on every
+    host core (same results, element order of the copies aside)."""
+    return build(force, _SRC, _LIB_OMP, extra=("-fopenmp",))
+
+
+def omp_lib() -> ctypes.CDLL:
+    """The OpenMP build, loaded once."""
+    global _lib_omp
+    if _lib_omp is None:
+        _lib_omp = load_library(build_omp())
+    return _lib_omp
+
+
+def omp_threads() -> int:
+    """Threads the OpenMP build uses (OMP_NUM_THREADS, else the cores this
+    process may run on)."""
+    v = os.environ.get("OMP_NUM_THREADS", "").split(",")[0].strip()
+    if v.isdigit() and int(v) > 0:
+        return int(v)
+    return len(os.sched_getaffinity(0))
 
 
 def load_library(path: str) -> ctypes.CDLL:

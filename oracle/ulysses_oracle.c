@@ -26,12 +26,26 @@
  * Elements are copied as raw bytes (elem_bytes each): no arithmetic touches a
  * value, so NaN payloads and signed zeros survive unchanged.
  *
+ * Two builds of this one file: the plain single-threaded one, and an OpenMP
+ * one (gcc -fopenmp) that splits the outermost (r, b) loop pair over the host
+ * cores. Each (r, b) iteration writes its own disjoint part of the outputs
+ * (mode 0: plane b of out_r; mode 1: head group r of plane b of every out_j),
+ * so the split changes only the order in which elements are copied, never a
+ * result. Without -fopenmp the pragmas are compiled out.
+ *
  * Return codes: 0 = done; -1 = bad argument (null pointer for a non-empty
  * slab, negative size, H not divisible by w, unsupported mode or element
  * size). Zero sizes are an empty re-layout: done, nothing touched.
  */
 #include <stdint.h>
 #include <string.h>
+
+/* The (r, b) loop pair is split over threads in the OpenMP build only. */
+#ifdef _OPENMP
+#define OUTER_LOOPS_PARALLEL _Pragma("omp parallel for collapse(2) schedule(static)")
+#else
+#define OUTER_LOOPS_PARALLEL
+#endif
 
 /* A size of 0 makes the index set empty: nothing is read or written, and
  * the slab pointers may then be NULL. */
@@ -66,7 +80,8 @@ int oracle_ulysses_a2a(const void *const *in, void *const *out, int64_t B,
     const int64_t S_global = S_local * w;
     const int64_t E = elem_bytes;
 
-    for (int r = 0; r < w; ++r)
+    OUTER_LOOPS_PARALLEL
+    for (int64_t r = 0; r < w; ++r)
         for (int64_t b = 0; b < B; ++b)
             for (int j = 0; j < w; ++j)
                 for (int64_t s = 0; s < S_local; ++s)
@@ -74,7 +89,7 @@ int oracle_ulysses_a2a(const void *const *in, void *const *out, int64_t B,
                         for (int64_t d = 0; d < D; ++d) {
                             /* the two sides of the same correspondence */
                             /* A: rank j's sequence shard, all H heads    */
-                            int64_t a = at4(b, s, (int64_t)r * Hw + hp, d,
+                            int64_t a = at4(b, s, r * Hw + hp, d,
                                             S_local, H, D);
                             /* C: rank r's head group, whole sequence    */
                             int64_t c = at4(b, (int64_t)j * S_local + s, hp, d,
@@ -109,7 +124,8 @@ int oracle_ulysses_a2a_pitched(const void *const *in, void *const *out,
     const int64_t Hw = H / w;
     const int64_t S_global = S_local * w;
     const int64_t E = elem_bytes;
-    for (int r = 0; r < w; ++r)
+    OUTER_LOOPS_PARALLEL
+    for (int64_t r = 0; r < w; ++r)
         for (int64_t b = 0; b < B; ++b)
             for (int j = 0; j < w; ++j)
                 for (int64_t s = 0; s < S_local; ++s)
@@ -117,7 +133,7 @@ int oracle_ulysses_a2a_pitched(const void *const *in, void *const *out,
                         for (int64_t d = 0; d < D; ++d) {
                             /* pitched side: rank j's row (b, s), head r*Hw + h' */
                             int64_t a = (b * S_local + s) * row_pitch
-                                        + ((int64_t)r * Hw + hp) * D + d;
+                                        + (r * Hw + hp) * D + d;
                             int64_t c = at4(b, (int64_t)j * S_local + s, hp, d,
                                             S_global, Hw, D);
                             if (mode == 0) {

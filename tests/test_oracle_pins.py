@@ -7,22 +7,47 @@ import oracle
 from oracle_pins import ALL_PINS, load_table, permute_formulation, table_names
 
 
-def _run(xs, mode, chunked):
-    return oracle.ulysses_a2a(xs, mode, chunked)
+def _bound(lib_of):
+    """The oracle bound to one build of its C library: the plain single-threaded
+    one, or the OpenMP one that splits the outer (r, b) loops over the cores."""
+    def run(xs, mode, chunked):
+        return oracle.ulysses_a2a(xs, mode, chunked, lib=lib_of())
+
+    def pitched(*args, **kw):
+        return oracle.ulysses_a2a_pitched(*args, lib=lib_of(), **kw)
+
+    run.pitched = pitched
+    return run
 
 
-_run.pitched = oracle.ulysses_a2a_pitched
+_run = _bound(oracle._get_lib)
+BUILDS = {"plain": _run, "openmp": _bound(oracle.omp_lib)}
 
 
+@pytest.mark.parametrize("build", sorted(BUILDS))
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
-def test_pin(pin):
-    pin(_run)
+def test_pin(pin, build):
+    pin(BUILDS[build])
 
 
+@pytest.mark.parametrize("build", sorted(BUILDS))
 @pytest.mark.parametrize("E", [1, 2, 4, 8])
-def test_hand_tables_every_element_size(E):
+def test_hand_tables_every_element_size(E, build):
     from oracle_pins import pin_hand_tables
-    pin_hand_tables(_run, elem_bytes=E)
+    pin_hand_tables(BUILDS[build], elem_bytes=E)
+
+
+def test_openmp_build_uses_several_threads_and_matches_on_a_larger_shape():
+    # the split over (r, b) must not change a byte, also with more (r, b)
+    # pairs than threads and a ragged plane count
+    from synth import unique_slabs
+    xs = unique_slabs((5, 33, 12, 7), 6, 4)
+    y_plain = oracle.ulysses_a2a(xs, 0)
+    y_omp = oracle.ulysses_a2a(xs, 0, lib=oracle.omp_lib())
+    assert all(torch.equal(a, b) for a, b in zip(y_plain, y_omp))
+    back = oracle.ulysses_a2a(y_omp, 1, lib=oracle.omp_lib())
+    assert all(torch.equal(a, b) for a, b in zip(back, xs))
+    assert oracle.omp_threads() >= 1
 
 
 def test_tables_are_well_formed():
