@@ -4,27 +4,50 @@
 One step = one pass of the whole hot path over one batch of synthetic input:
 mode 0 (scatter heads, gather sequence) on the w input slabs, then mode 1 (the
 inverse) on its result, each through the C ABI (host checks, descriptor table,
-tile scheduler, copy kernel). Workload: w=4, B=1, S_local=8192, H=24, D=128,
-bf16, N(0,1) values (payload P = 192 MiB per call).
+tile scheduler, copy kernel). Headline workload: w=8, B=2, S_local=4725 (a
+ragged last tile), H=40, D=128, bf16, N(0,1) values: a payload P of 774.1 MB
+per call.
 
 Metric: payload GB/s (P per call / device time, 1 GB = 1e9 B) and the fraction
-of the measured HBM copy bandwidth, counting 2P bytes moved per call. The K
-steps run back to back between two CUDA events on the launching stream. Every
-input (192 MiB per call) is larger than the 126 MB L2, and mode 1 reads its own
-input slabs rather than mode 0's fresh output, so no kernel reads what the
-kernel before it touched. As a cross-check, each mode is also timed call by
-call after a 2x-L2 write flush (per-call events, ~2 us resolution).
+of the HBM roofline counting 2P bytes moved per call, against the measured copy
+bandwidth of this B200 (MEASURED_PEAKS.json) and against the nominal 8 TB/s of
+B200 HBM3e. The K steps run back to back between two CUDA events on the
+launching stream; every call's input (774 MB) is larger than the 126 MB L2 and
+mode 1 reads its own input slabs rather than mode 0's fresh output, so no kernel
+reads what the kernel before it touched.
+
+The same line carries, on one GPU:
+  per_mode        each mode of the headline workload, back to back (>= 1 s each);
+  isolated_call   one call at a time after an L2 flush that READS a buffer twice
+                  the L2 (leaving only clean lines), for the headline workload
+                  and w4_S8192_H24_D128: median device time per call;
+  workloads       w4_S8192_H24_D128 per mode, and w4_B4_S16384_H32_D64 unchunked,
+                  chunked per plane and chunked through the staging window;
+  sweep           payloads of 1 MiB, 64 MiB, 512 MiB and 2 GiB at w = 2/4/8
+                  (H = 8w, D = 128, B = 1), bf16 and fp32 U[-1,1), both modes;
+                  the 512 MiB bf16 points (w_sweep_512MiB) run >= 1 s per mode;
+  vec_shapes      shapes only the vector path takes: 200-byte and 6/12-byte
+                  rows, slab bases 8 and 2 bytes off a 16-byte boundary, w = 16;
+  e2e             the step through the host-buffer entry point (pinned slabs);
+  cpu_baseline    the CPU oracle on a sample of the headline workload: the
+                  OpenMP build on every host core, and the single-threaded one.
+Each timed section carries its own clock record (SM MHz sampled every ~2 ms by
+NVML during that section, and the clock-event reasons seen).
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own independent
-instance of the workload (the w logical ranks all live in one GPU's memory, so
-nothing is exchanged); `value` = payload of all ranks / the slowest rank's time
-("weak" scaling). The only collective is the max-over-ranks of the timings.
+instance of the headline workload (the w logical ranks all live in one GPU's
+memory), and `value` = payload of all ranks / the slowest rank's time ("weak"
+scaling). The line then adds the Ulysses all-to-all ACROSS the GPUs (w = the
+number of GPUs, one rank slab of the headline's per-rank shape per GPU):
+exchange_peer_gbs (this library's PeerExchange: windows, peer loads) and
+exchange_nccl_gbs (a library all-to-all baseline), with the barrier share of a
+PeerExchange step.
 
 `--impl reference` times the CPU oracle (the plain nested-loop definition) on
 the host cores, on a bounded sample of the same workload, as a baseline only.
 
 Other modes, each printing its own line:
-  --sweep          adds the 128 KiB..2 GiB bandwidth sweep (w = 2/4/8, bf16/fp32);
+  --sweep          the full 128 KiB..2 GiB bandwidth sweep (w = 2/4/8, bf16/fp32);
   --packed         q, k, v in one head-packed launch vs three per-tensor launches;
   --peer-one-gpu   the cross-GPU exchange's publish and pull kernels, with the
                    ranks as contexts on one GPU;
@@ -38,10 +61,12 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 import torch
@@ -53,10 +78,11 @@ if ROOT not in sys.path:
 METRIC = "payload GB/s and % of HBM roofline (2x bytes) per mode at w=2/4/8, 1xB200"
 # The benchmark workloads (bf16, N(0,1) values), named by their sizes:
 #   w2_S64_H4_D64          a tiny round trip (B = 1);
-#   w4_S8192_H24_D128      the default, 192 MiB per call (B = 1);
-#   w8_B2_S4725_H40_D128   a ragged sequence tail (4725 = 787 x 6 + 3), 774 MB;
+#   w4_S8192_H24_D128      192 MiB per call (B = 1);
+#   w8_B2_S4725_H40_D128   the default: w = 8, a ragged sequence tail
+#                          (4725 = 787 x 6 + 3), 774 MB per call;
 #   w4_B4_S16384_H32_D64   four planes, for the chunked per-plane variant, 1 GiB.
-DEFAULT_WORKLOAD = "w4_S8192_H24_D128"
+DEFAULT_WORKLOAD = "w8_B2_S4725_H40_D128"
 WORKLOADS = {
     "w2_S64_H4_D64": dict(w=2, B=1, S_local=64, H=4, D=64),
     "w4_S8192_H24_D128": dict(w=4, B=1, S_local=8192, H=24, D=128),
@@ -64,6 +90,16 @@ WORKLOADS = {
     "w4_B4_S16384_H32_D64": dict(w=4, B=4, S_local=16384, H=32, D=64),
 }
 WORKLOAD = WORKLOADS[DEFAULT_WORKLOAD]
+# Shapes only the vector path takes (bf16 unless noted): name -> (w, B, S, H, D,
+# element bytes, byte offset of every slab base from a 16-byte boundary).
+VEC_SHAPES = {
+    "rows200B_w8_S41943_H8_D100": (8, 1, 41943, 8, 100, 2, 0),     # 200-byte runs
+    "rows12B_w4_S1398101_H4_D3_fp32": (4, 1, 1398101, 4, 3, 4, 0),  # 12-byte runs
+    "rows6B_w4_S2796202_H4_D3": (4, 1, 2796202, 4, 3, 2, 0),        # 6-byte runs
+    "base8_w4_S8192_H24_D128": (4, 1, 8192, 24, 128, 2, 8),         # bases 8 B off
+    "base2_w4_S8192_H24_D128": (4, 1, 8192, 24, 128, 2, 2),         # bases 2 B off
+    "w16_S4096_H32_D128": (16, 1, 4096, 32, 128, 2, 0),             # w above the TMA limit
+}
 
 
 def workload_key(w, B, S, H, D, path):
@@ -74,8 +110,11 @@ def workload_name(w, B, S, H, D, chunked):
     how = {0: "", 1: ", chunked per plane", 2: ", chunked through the staging window"}[chunked]
     return (f"ulysses_a2a w={w} B={B} S_local={S} H={H} D={D} bf16, step = mode 0 + mode 1"
             f"{how}")
+
+
 FALLBACK_HBM_GBS = 6650.0
-L2_FLUSH_BYTES = 2 * 126 * 1024 * 1024 + (4 << 20)
+NOMINAL_HBM_GBS = 8000.0        # B200 HBM3e, nominal
+L2_BYTES = 126 * 1024 * 1024
 
 
 # ---------------------------------------------------------------- helpers
@@ -106,6 +145,14 @@ def hbm_peak():
         return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs: torch copy, 1 Gi bf16)"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback (6.65 TB/s copy bandwidth, an earlier B200 measurement)"
+
+
+def fracs(payload_bytes: int, ms: float, peak: float) -> dict:
+    """Payload GB/s of one call of `ms`, and 2 x payload against the measured and
+    the nominal HBM bandwidth."""
+    gbs = payload_bytes / (ms / 1e3) / 1e9
+    return {"gbs": round(gbs, 1), "frac": round(2 * gbs / peak, 4),
+            "frac_nominal": round(2 * gbs / NOMINAL_HBM_GBS, 4)}
 
 
 def _code_only(text: str) -> str:
@@ -152,77 +199,132 @@ def ncu_traffic(key, plan, chunked):
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    """SM clock and clock-event reasons of one GPU, sampled every ~2 ms by a
+    background thread for as long as it runs (NVML; nvidia-smi every 100 ms
+    when NVML is unavailable). `window(t0, t1)` summarises the samples taken
+    between two time.perf_counter() stamps, i.e. during one timed region."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits that matter for a bandwidth number
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+    SMI_FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index):
-        self.proc = None
-        self.lines = []
+    def __init__(self, device_index, period_s=0.002):
+        self.period = period_s
+        self.samples = []            # (t, sm_mhz, reason names)
+        self.source = None
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._proc = None
         try:
             p = torch.cuda.get_device_properties(device_index)
             self.bus = "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
         except Exception:
             self.bus = None
 
-    def start(self):
-        if self.bus is None:
-            return
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self.bus, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except Exception:
-            self.proc = None
+    def _nvml_loop(self, nv, h):
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except Exception:
+                break
+            names = tuple(n for b, n in self.REASONS.items() if bits & b)
+            self.samples.append((time.perf_counter(), float(mhz), names))
+            time.sleep(self.period)
 
-    def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except Exception:
-            self.proc.kill()
-            out = ""
-        sms, maxes, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
+    def _smi_loop(self):
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in self._proc.stdout:
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 6:
                 continue
             try:
-                sms.append(float(parts[1]))
-                maxes.append(float(parts[2]))
+                mhz, mx = float(parts[0]), float(parts[1])
             except ValueError:
                 continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        if not sms:
+            self.max_mhz = mx
+            act = tuple(n for n, v in zip(names, parts[2:6]) if v.lower() == "active")
+            self.samples.append((time.perf_counter(), mhz, act))
+
+    def start(self):
+        if self.bus is None:
+            return self
+        try:
+            import pynvml as nv
+
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByPciBusId(self.bus)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.source = "nvml"
+            self._thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+        except Exception:
+            try:
+                self._proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", self.bus, f"--query-gpu={self.SMI_FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.source = "nvidia-smi"
+                self._thread = threading.Thread(target=self._smi_loop, daemon=True)
+            except Exception:
+                return self
+        self._thread.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self._proc is not None:
+            self._proc.terminate()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
+
+    def window(self, t0, t1):
+        """Median SM MHz and the reasons seen between t0 and t1 (None if no sample)."""
+        sel = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not sel:
             return None
-        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes),
-                "samples": len(sms), "reasons": sorted(reasons)}
+        reasons = sorted({n for s in sel for n in s[2]})
+        return {"sm_mhz": statistics.median(s[1] for s in sel), "sm_max_mhz": self.max_mhz,
+                "samples": len(sel), "reasons": reasons, "source": self.source}
 
 
 # ---------------------------------------------------------------- our arm
-def make_inputs(w, B, S, H, D, dtype, device, seed0=1234):
-    """Seeded N(0,1) slabs drawn on the device generator (values do not affect timing)."""
+def make_inputs(w, B, S, H, D, dtype, device, seed0=1234, offset_bytes=0):
+    """Seeded N(0,1) slabs drawn on the device generator (values do not affect
+    timing); with offset_bytes each slab starts that many bytes past the start
+    of its own allocation (a base off the 16-byte boundary)."""
     dt = {"bf16": torch.bfloat16, "fp32": torch.float32}[dtype]
     xs = []
     for k in range(w):
         g = torch.Generator(device=device)
         g.manual_seed(seed0 + k)
-        xs.append(torch.randn((B, S, H, D), generator=g, device=device, dtype=torch.float32).to(dt))
+        v = torch.randn((B, S, H, D), generator=g, device=device, dtype=torch.float32).to(dt)
+        if offset_bytes:
+            n = v.numel() * v.element_size()
+            raw = torch.empty(n + offset_bytes, dtype=torch.uint8, device=device)
+            t = raw[offset_bytes:].view(dt).view(B, S, H, D)
+            t.copy_(v)
+            v = t
+        xs.append(v)
     return xs
 
 
-def timed_steps(a2a, x, y, y2, z, steps, warmup, stream, sampler=None, chunked=0):
+def empty_slabs(w, shape, dt, device, offset_bytes=0):
+    if not offset_bytes:
+        return [torch.empty(shape, dtype=dt, device=device) for _ in range(w)]
+    E = torch.empty((), dtype=dt).element_size()
+    n = math.prod(shape) * E
+    return [torch.empty(n + offset_bytes, dtype=torch.uint8, device=device)[offset_bytes:]
+            .view(dt).view(shape) for _ in range(w)]
+
+
+def timed_steps(a2a, x, y, y2, z, steps, warmup, stream, chunked=0):
     """K back-to-back steps (mode 0: x -> y, mode 1: y2 -> z) between one pair of events.
 
-    Returns (total ms, launches of our kernels in the timed region, clocks)."""
+    Returns (total ms, launches of our kernels in the timed region, t0, t1)."""
     for _ in range(warmup):
         a2a.run(x, 0, out=y, stream=stream, chunked=chunked)
         a2a.run(y2, 1, out=z, stream=stream, chunked=chunked)
@@ -230,61 +332,43 @@ def timed_steps(a2a, x, y, y2, z, steps, warmup, stream, sampler=None, chunked=0
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     launches0 = a2a.launch_count
-    if sampler:
-        sampler.start()
+    t0 = time.perf_counter()
     e0.record(stream)
     for _ in range(steps):
         a2a.run(x, 0, out=y, stream=stream, chunked=chunked)
         a2a.run(y2, 1, out=z, stream=stream, chunked=chunked)
     e1.record(stream)
     torch.cuda.synchronize()
-    clocks = sampler.stop() if sampler else None
-    return e0.elapsed_time(e1), a2a.launch_count - launches0, clocks
+    t1 = time.perf_counter()
+    return e0.elapsed_time(e1), a2a.launch_count - launches0, t0, t1
 
 
-def timed_mode(a2a, src, dst, mode, reps, stream, chunked=0):
-    """Back-to-back calls of one mode between one pair of events; ms per call."""
-    for _ in range(3):
-        a2a.run(src, mode, out=dst, stream=stream, chunked=chunked)
+def timed_loop(fn, stream, min_seconds, sampler=None, warmup=3):
+    """Back-to-back calls of fn (each enqueues one call on `stream`) for at least
+    min_seconds of device time, between one pair of events.
+
+    Returns (ms per call, calls timed, clock record of the timed region)."""
+    for _ in range(warmup):
+        fn()
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(reps):
-        a2a.run(src, mode, out=dst, stream=stream, chunked=chunked)
+    for _ in range(3):
+        fn()
     e1.record(stream)
     torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / reps
-
-
-def timed_flushed(a2a, src, dst, mode, flush, reps, stream, chunked=0):
-    """Median per-call time (ms) with a 2x-L2 write flush before every call."""
-    for _ in range(3):
-        a2a.run(src, mode, out=dst, stream=stream, chunked=chunked)
+    per = max(e0.elapsed_time(e1) / 3, 1e-3)
+    reps = max(3, int(math.ceil(min_seconds * 1e3 / per)))
+    t0 = time.perf_counter()
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
     torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(reps)]
-    with torch.cuda.stream(stream):
-        for i in range(reps):
-            flush.fill_(i & 0xFF)
-            ev[i][0].record(stream)
-            a2a.run(src, mode, out=dst, stream=stream, chunked=chunked)
-            ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    return statistics.median(a.elapsed_time(b) for a, b in ev)
-
-
-def bench_sweep_point(a2a, w, payload, dtype, device, stream, reps):
-    E = 2 if dtype == "bf16" else 4
-    H, D = 8 * w, 128
-    S = payload // (w * H * D * E)
-    x = make_inputs(w, 1, S, H, D, dtype, device)
-    y = [torch.empty((1, S * w, H // w, D), dtype=x[0].dtype, device=device) for _ in range(w)]
-    t0 = timed_mode(a2a, x, y, 0, reps, stream)
-    t1 = timed_mode(a2a, y, x, 1, reps, stream)
-    P = w * S * H * D * E
-    del x, y
-    return P, t0, t1
+    t1 = time.perf_counter()
+    clocks = sampler.window(t0, t1) if sampler else None
+    return e0.elapsed_time(e1) / reps, reps, clocks
 
 
 def graph_ms_per_call(a2a, src, dst, mode, calls, reps, stream):
@@ -312,19 +396,41 @@ def graph_ms_per_call(a2a, src, dst, mode, calls, reps, stream):
     return ms
 
 
-def bandwidth_sweep(device, peak):
-    """Payload 128 KiB .. 2 GiB (doubling), w = 2/4/8, H = 8w, D = 128, B = 1, bf16 and
-    fp32 U[-1,1), both modes; device time per call from CUDA-graph replays."""
+def isolated_call(a2a, src, dst, mode, stream, reps, flush, acc, sampler=None):
+    """Median device time (ms) of one call at a time, each after an L2 flush that
+    reads `flush` (twice the L2): the flush leaves only clean lines in L2, so no
+    write-back of earlier data falls inside the timed call."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps + 2)]
+    with torch.cuda.stream(stream):
+        t0 = time.perf_counter()
+        for a, b in ev:
+            acc.add_(flush.sum())
+            a.record(stream)
+            a2a.run(src, mode, out=dst, stream=stream)
+            b.record(stream)
+        torch.cuda.synchronize()
+        t1 = time.perf_counter()
+    times = [a.elapsed_time(b) for a, b in ev[2:]]
+    return statistics.median(times), min(times), sampler.window(t0, t1) if sampler else None
+
+
+def bandwidth_sweep(device, peak, payload_exps=range(17, 32), dtypes=(("bf16", 2), ("fp32", 4)),
+                    ws=(2, 4, 8), sampler=None, long_payload=None, long_seconds=1.0):
+    """Payloads 2^e bytes (e in payload_exps), w = 2/4/8, H = 8w, D = 128, B = 1,
+    U[-1,1) values, both modes. Payloads under 64 MiB: device time per call from
+    CUDA-graph replays of back-to-back calls; larger: back-to-back loops of at
+    least 0.25 s (long_seconds for the long_payload bf16 points)."""
     from sequence_all_re_b200 import UlyssesA2A
 
     stream = torch.cuda.Stream(device)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     rows = []
-    for dtype, E in (("bf16", 2), ("fp32", 4)):
+    for dtype, E in dtypes:
         a2a = UlyssesA2A(device.index or 0, E)
-        for w in (2, 4, 8):
+        for w in ws:
             H, D = 8 * w, 128
-            for k in range(17, 32):
+            for k in payload_exps:
                 P = 1 << k
                 S = P // (w * H * D * E)
                 if S < 1:
@@ -338,41 +444,161 @@ def bandwidth_sweep(device, peak):
                     gen.manual_seed(1234 + r)
                     x.append((torch.rand((1, S, H, D), generator=gen, device=device) * 2 - 1).to(dt))
                 y = [torch.empty((1, S * w, H // w, D), dtype=dt, device=device) for _ in range(w)]
-                calls = max(1, min(64, (256 << 20) // P))
-                reps = max(3, min(50, (8 << 30) // (P * calls)))
-                t0 = graph_ms_per_call(a2a, x, y, 0, calls, reps, stream)
-                t1 = graph_ms_per_call(a2a, y, x, 1, calls, reps, stream)
-                g0, g1 = P / (t0 / 1e3) / 1e9, P / (t1 / 1e3) / 1e9
-                rows.append({"dtype": dtype, "w": w, "payload_bytes": P, "S_local": S,
-                             "mode0_gbs": round(g0, 1), "mode1_gbs": round(g1, 1),
-                             "mode0_frac": round(2 * g0 / peak, 4),
-                             "mode1_frac": round(2 * g1 / peak, 4),
-                             "l2_assisted": 2 * P <= l2})
+                row = {"dtype": dtype, "w": w, "payload_bytes": P, "S_local": S,
+                       "l2_assisted": 2 * P <= l2}
+                for mode, (src, dst) in ((0, (x, y)), (1, (y, x))):
+                    if P < (64 << 20):
+                        calls = max(1, min(64, (256 << 20) // P))
+                        reps = max(3, min(50, (8 << 30) // (P * calls)))
+                        ms = graph_ms_per_call(a2a, src, dst, mode, calls, reps, stream)
+                        clk = None
+                    else:
+                        secs = long_seconds if (P == long_payload and dtype == "bf16") else 0.25
+                        ms, _, clk = timed_loop(
+                            lambda: a2a.run(src, mode, out=dst, stream=stream), stream, secs,
+                            sampler)
+                    f = fracs(P, ms, peak)
+                    row[f"mode{mode}_gbs"] = f["gbs"]
+                    row[f"mode{mode}_frac"] = f["frac"]
+                    row[f"mode{mode}_frac_nominal"] = f["frac_nominal"]
+                    if clk:
+                        row[f"mode{mode}_clocks"] = clk
+                rows.append(row)
                 del x, y
         a2a.close()
+    torch.cuda.empty_cache()
     return rows
 
 
+def per_mode_block(a2a, ins, outs, back, P, stream, peak, sampler, seconds, chunked=0):
+    """Mode 0 (ins -> outs) and mode 1 (outs -> back), each back to back for at
+    least `seconds`: payload GB/s, fractions and the clock record per mode."""
+    res = {}
+    for mode, (src, dst) in ((0, (ins, outs)), (1, (outs, back))):
+        ms, reps, clk = timed_loop(
+            lambda: a2a.run(src, mode, out=dst, stream=stream, chunked=chunked), stream,
+            seconds, sampler)
+        res[f"mode{mode}"] = dict(fracs(P, ms, peak), us_per_call=round(ms * 1e3, 2), calls=reps,
+                                  clocks=clk)
+    return res
+
+
+def vec_shape_block(device, peak, sampler, seconds=0.5):
+    """The VEC-only shapes: each mode back to back; plan, GB/s and fractions."""
+    from sequence_all_re_b200 import UlyssesA2A
+
+    stream = torch.cuda.Stream(device)
+    out = {}
+    for name, (w, B, S, H, D, E, off) in VEC_SHAPES.items():
+        dt = {2: "bf16", 4: "fp32"}[E]
+        a2a = UlyssesA2A(device.index or 0, E)
+        x = make_inputs(w, B, S, H, D, dt, device, offset_bytes=off)
+        y = empty_slabs(w, (B, S * w, H // w, D), x[0].dtype, device, off)
+        z = empty_slabs(w, (B, S, H, D), x[0].dtype, device, off)
+        p = a2a.plan(x, 0, out=y)
+        P = w * B * S * H * D * E
+        res = per_mode_block(a2a, x, y, z, P, stream, peak, sampler, seconds)
+        torch.cuda.synchronize()
+        if not all(torch.equal(z[k], x[k]) for k in range(w)):
+            raise SystemExit(f"vector-path shape {name}: round trip mismatch")
+        out[name] = {"payload_bytes": P, "path": {1: "tma", 2: "vec"}[p["path"]],
+                     "vec_bytes": p["vec_bytes"], "row_bytes": p["row_bytes"],
+                     "base_offset_bytes": off, **res}
+        a2a.close()
+        del x, y, z
+        torch.cuda.empty_cache()
+    return out
+
+
 def cpu_oracle_baseline(w, B, S, H, D, budget_s=12.0):
-    """The oracle, as it stands, on the host: full workload steps until ~budget_s."""
+    """The oracle, as it stands, on the host cores: the OpenMP build (the outer
+    (r, b) loops over every core) and the single-threaded build, each on whole
+    mode 0 + mode 1 steps of a sample of the workload for about budget_s / 2."""
     import oracle
     from synth import normal_slabs
 
-    xs = normal_slabs((B, S, H, D), w, "bf16")
-    done = 0
-    t_start = time.perf_counter()
-    while True:
-        y = oracle.ulysses_a2a(xs, 0)
-        oracle.ulysses_a2a(y, 1)
-        done += 1
-        if time.perf_counter() - t_start > budget_s:
-            break
-    el = time.perf_counter() - t_start
-    P = w * B * S * H * D * 2
-    return {"value": round(2 * P * done / el / 1e9, 4), "unit": "GB/s", "cores": 1,
-            "kind": "oracle",
-            "sample": f"{done} full steps (mode 0 + mode 1 on w={w},B={B},S_local={S},H={H},"
-                      f"D={D} bf16) in {el:.1f} s, single-threaded C nested loops"}
+    E = 2
+    cores_on_box = os.cpu_count() or 1
+    threads = oracle.omp_threads()
+    res = {}
+    for kind, lib in (("openmp", oracle.omp_lib()), ("single", oracle._get_lib())):
+        # size the sample from a small probe: about 1 s per step
+        probe_S = min(S, 64)
+        xs = normal_slabs((B, probe_S, H, D), w, "bf16")
+        t = time.perf_counter()
+        oracle.ulysses_a2a(oracle.ulysses_a2a(xs, 0, lib=lib), 1, lib=lib)
+        per_row = (time.perf_counter() - t) / probe_S
+        S_sample = int(max(1, min(S, 1.0 / max(per_row, 1e-9))))
+        xs = normal_slabs((B, S_sample, H, D), w, "bf16")
+        done, t_start = 0, time.perf_counter()
+        while True:
+            oracle.ulysses_a2a(oracle.ulysses_a2a(xs, 0, lib=lib), 1, lib=lib)
+            done += 1
+            if time.perf_counter() - t_start > budget_s / 2:
+                break
+        el = time.perf_counter() - t_start
+        P = w * B * S_sample * H * D * E
+        res[kind] = {"value": round(2 * P * done / el / 1e9, 4), "threads": threads if kind == "openmp" else 1,
+                     "sample": f"{done} steps (mode 0 + mode 1) on S_local={S_sample} of {S} rows "
+                               f"(w={w},B={B},H={H},D={D} bf16) in {el:.1f} s"}
+    return {"value": res["openmp"]["value"], "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "threads": threads, "cores_on_box": cores_on_box,
+            "sample": "OpenMP build, outer (r, b) loops over every core: " + res["openmp"]["sample"],
+            "single_thread": {"value": res["single"]["value"], "unit": "GB/s", "cores": 1,
+                              "sample": res["single"]["sample"]}}
+
+
+def exchange_arms(dist, device, rank, world, steps, warmup, wl):
+    """The Ulysses all-to-all across the job's GPUs (w = world, one rank slab of
+    the workload's per-rank shape per GPU), a step being mode 0 then mode 1:
+    this library's PeerExchange and a library all-to-all (NCCL) baseline. Every
+    rank takes the same steps in the same order; times are the max over ranks."""
+    from sequence_all_re_b200.peer import PeerExchange
+
+    B, S, H, D = (wl[k] for k in ("B", "S_local", "H", "D"))
+    if H % world:
+        return {"skipped": f"H={H} is not divisible by {world} GPUs"}
+    x = make_inputs(1, B, S, H, D, "bf16", device, seed0=1234 + rank)[0]
+    slab = B * S * H * D * 2
+    stream = torch.cuda.current_stream(device)
+    res = {"workload": f"one rank slab per GPU, w = {world}: B={B} S_local={S} H={H} D={D} bf16",
+           "steps": steps}
+
+    def timed(step):
+        for _ in range(warmup):
+            z = step()
+        torch.cuda.synchronize()
+        if not torch.equal(z, x):
+            raise SystemExit("round trip mismatch across GPUs")
+        dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1), dist, device) / steps
+
+    ex = PeerExchange(device=device.index, elem_bytes=2)
+    ms = timed(lambda: ex.all_to_all_4d(ex.all_to_all_4d(x, 0), 1))
+    # the barrier alone (a one-element all-reduce on the stream), 4 per step
+    nb = 50
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(nb):
+        ex._barrier(stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    bar_ms = max_over_ranks(e0.elapsed_time(e1), dist, device) / nb
+    ex.shutdown()
+    res["peer"] = {"ms_per_step": round(ms, 4), "gbs": round(job_gbs(world, 2 * slab, 1, ms), 1),
+                   "barrier_us": round(bar_ms * 1e3, 2), "barriers_per_step": 4,
+                   "barrier_share": round(4 * bar_ms / ms, 4)}
+    ms = timed(lambda: nccl_all_to_all_4d(nccl_all_to_all_4d(x, 0), 1))
+    res["nccl"] = {"ms_per_step": round(ms, 4), "gbs": round(job_gbs(world, 2 * slab, 1, ms), 1)}
+    return res
 
 
 def run_ours(args):
@@ -389,6 +615,7 @@ def run_ours(args):
 
     from sequence_all_re_b200 import UlyssesA2A
 
+    sampler = ClockSampler(local_rank).start()
     wl = WORKLOADS[args.workload]
     w, B, S, H, D = (wl[k] for k in ("w", "B", "S_local", "H", "D"))
     E = 2
@@ -407,12 +634,12 @@ def run_ours(args):
     y2 = [t.clone() for t in y]
     plan = a2a.plan(x, 0, chunked=chunked, out=y)
 
-    sampler = ClockSampler(local_rank)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    total_ms, launches, clocks = timed_steps(a2a, x, y, y2, z, args.steps, args.warmup, stream,
-                                             sampler, chunked)
+    total_ms, launches, t0, t1 = timed_steps(a2a, x, y, y2, z, args.steps, args.warmup, stream,
+                                             chunked)
+    clocks = sampler.window(t0, t1)
     a2a.status(stream)
     torch.cuda.synchronize()
     if dist:
@@ -432,20 +659,61 @@ def run_ours(args):
     key = workload_key(w, B, S, H, D, {1: "tma", 2: "vec"}[plan["path"]])
     traffic_bytes, traffic_src = ncu_traffic(key, plan, chunked)
 
-    # per mode: back to back, and call by call after an L2 write flush
-    reps = max(20, min(args.steps, 400))
-    m0 = timed_mode(a2a, x, y, 0, reps, stream, chunked)
-    m1 = timed_mode(a2a, y2, z, 1, reps, stream, chunked)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-    f0 = timed_flushed(a2a, x, y, 0, flush, reps, stream, chunked)
-    f1 = timed_flushed(a2a, y2, z, 1, flush, reps, stream, chunked)
-    del flush
-    gbs = lambda ms: P / (ms / 1e3) / 1e9
-    per_mode = {"mode0_gbs": round(gbs(m0), 1), "mode1_gbs": round(gbs(m1), 1),
-                "mode0_frac": round(2 * gbs(m0) / peak, 4), "mode1_frac": round(2 * gbs(m1) / peak, 4),
-                "flushed_mode0_gbs": round(gbs(f0), 1), "flushed_mode1_gbs": round(gbs(f1), 1),
-                "flushed_mode0_frac": round(2 * gbs(f0) / peak, 4),
-                "flushed_mode1_frac": round(2 * gbs(f1) / peak, 4)}
+    extras = {}
+    if world == 1 and not args.no_extras:
+        # each mode of the headline workload, back to back for >= 1 s
+        extras["per_mode"] = per_mode_block(a2a, x, y2, z, P, stream, peak, sampler, 1.0, chunked)
+        # one call at a time after a clean L2 flush
+        flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.int32, device=device)
+        acc = torch.zeros((), dtype=torch.int64, device=device)
+        iso = {args.workload: {}}
+        for mode, (src, dst) in ((0, (x, y)), (1, (y, z))):
+            med, mn, clk = isolated_call(a2a, src, dst, mode, stream, 40, flush, acc, sampler)
+            iso[args.workload][f"mode{mode}"] = dict(fracs(P, med, peak),
+                                                     us_median=round(med * 1e3, 2),
+                                                     us_min=round(mn * 1e3, 2), clocks=clk)
+        del y2, z
+        torch.cuda.empty_cache()
+        # the other single-GPU workloads
+        wls = {}
+        for name, variants in (("w4_S8192_H24_D128", ((0, 1.0),)),
+                               ("w4_B4_S16384_H32_D64", ((0, 0.5), (1, 0.5), (2, 0.5)))):
+            v = WORKLOADS[name]
+            ww, BB, SS, HH, DD = (v[k] for k in ("w", "B", "S_local", "H", "D"))
+            PP = ww * BB * SS * HH * DD * E
+            xa = make_inputs(ww, BB, SS, HH, DD, "bf16", device)
+            ya = [torch.empty((BB, SS * ww, HH // ww, DD), dtype=torch.bfloat16, device=device)
+                  for _ in range(ww)]
+            za = [torch.empty_like(t) for t in xa]
+            entry = {"payload_bytes": PP}
+            for ch, secs in variants:
+                entry[{0: "unchunked", 1: "chunked_per_plane", 2: "chunked_window"}[ch]] = \
+                    per_mode_block(a2a, xa, ya, za, PP, stream, peak, sampler, secs, ch)
+            torch.cuda.synchronize()
+            if not all(torch.equal(za[k], xa[k]) for k in range(ww)):
+                raise SystemExit(f"{name}: round trip mismatch")
+            if name == "w4_S8192_H24_D128":
+                iso[name] = {}
+                for mode, (src, dst) in ((0, (xa, ya)), (1, (ya, za))):
+                    med, mn, clk = isolated_call(a2a, src, dst, mode, stream, 40, flush, acc,
+                                                 sampler)
+                    iso[name][f"mode{mode}"] = dict(fracs(PP, med, peak),
+                                                    us_median=round(med * 1e3, 2),
+                                                    us_min=round(mn * 1e3, 2), clocks=clk)
+            wls[name] = entry
+            del xa, ya, za
+            torch.cuda.empty_cache()
+        del flush
+        extras["isolated_call"] = iso
+        extras["workloads"] = wls
+        # compact bandwidth sweep: 1 MiB, 64 MiB, 512 MiB, 2 GiB
+        sweep = bandwidth_sweep(device, peak, payload_exps=(20, 26, 29, 31), sampler=sampler,
+                                long_payload=512 << 20, long_seconds=1.0)
+        extras["sweep"] = sweep
+        extras["w_sweep_512MiB"] = {
+            f"w{r['w']}": {k: r[k] for k in r if k.startswith("mode") or k == "payload_bytes"}
+            for r in sweep if r["dtype"] == "bf16" and r["payload_bytes"] == 512 << 20}
+        extras["vec_shapes"] = vec_shape_block(device, peak, sampler)
 
     # e2e: the same step through the host-buffer entry point (pinned host slabs)
     e2e = None
@@ -462,40 +730,34 @@ def run_ours(args):
         torch.cuda.synchronize()
         ea = torch.cuda.Event(enable_timing=True)
         eb = torch.cuda.Event(enable_timing=True)
+        ta = time.perf_counter()
         ea.record(stream)
         for _ in range(e_steps):
             a2a.run_host(hx, 0, out=hy, stream=stream)
             a2a.run_host(hy, 1, out=hz, stream=stream)
         eb.record(stream)
         torch.cuda.synchronize()
+        tb = time.perf_counter()
         e_ms = max_over_ranks(ea.elapsed_time(eb), dist, device)
         for k in range(w):
             if not torch.equal(hz[k].view(torch.int16), hx[k].view(torch.int16)):
                 raise SystemExit("host-path round trip mismatch")
         e2e = {"value": round(job_gbs(world, 2 * P, e_steps, e_ms), 3), "unit": "GB/s",
                "h2d_bytes_per_step": 2 * P, "d2h_bytes_per_step": 2 * P,
-               "steps": e_steps, "via": "ulysses_a2a_run_host, pinned host slabs"}
+               "steps": e_steps, "via": "ulysses_a2a_run_host, pinned host slabs",
+               "clocks": sampler.window(ta, tb)}
+        del hx, hy, hz
 
-    # per-mode figures at w = 2/4/8 on a 512 MiB payload (the >= 256 MB target regime)
-    w_sweep = None
-    if not args.no_sweep and rank == 0:
-        del y2, z
-        w_sweep = {}
-        for ww in (2, 4, 8):
-            Pw, a, b = bench_sweep_point(a2a, ww, 512 << 20, "bf16", device, stream,
-                                         args.sweep_reps)
-            w_sweep[f"w{ww}"] = {
-                "payload_bytes": Pw,
-                "mode0_gbs": round(Pw / (a / 1e3) / 1e9, 1),
-                "mode1_gbs": round(Pw / (b / 1e3) / 1e9, 1),
-                "mode0_frac": round(2 * Pw / (a / 1e3) / 1e9 / peak, 4),
-                "mode1_frac": round(2 * Pw / (b / 1e3) / 1e9 / peak, 4),
-            }
+    exchange = None
+    if world > 1 and not args.no_exchange:
+        exchange = exchange_arms(dist, device, rank, world, min(args.steps, 200),
+                                 max(3, args.warmup), wl)
 
-    sweep = None
+    full_sweep = None
     if args.sweep and rank == 0:
-        sweep = bandwidth_sweep(device, peak)
+        full_sweep = bandwidth_sweep(device, peak, sampler=sampler)
 
+    sampler.stop()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_baseline(w, B, S, H, D, budget_s=args.cpu_budget)
@@ -523,11 +785,10 @@ def run_ours(args):
             "stages": plan["stages"], "chunk_units": plan["chunk_units"], "grid": plan["grid"],
             "l2": (f"inputs larger than L2 ({P / 2**20:.0f} MiB per call vs 126 MB); no kernel "
                    "reads data the previous kernel touched; no flush in the timed region")
-                  if P > 126 * 2**20 else
+                  if P > L2_BYTES else
                   "L2-assisted: the inputs fit in L2 (below 126 MB); no flush",
             "parallelism": f"{world} independent instance(s), one per GPU",
         },
-        "per_mode": per_mode,
         "roofline": {
             "bound": "hbm",
             "kernel": "ua2a_tma_kernel<0>/<1>" if plan["path"] == 1 else "ua2a_vec_kernel",
@@ -535,6 +796,7 @@ def run_ours(args):
             "peak": peak,
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
+            "frac_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
             "peak_source": peak_src,
             "algorithmic_bytes_per_launch": bytes_per_launch,
             "avg_launch_us": round(avg_launch_ms * 1e3, 3),
@@ -547,11 +809,15 @@ def run_ours(args):
         "gpu_launches": launches,
         "e2e": e2e,
         "clocks": clocks,
-        "w_sweep_512MiB_back_to_back": w_sweep,
+        **extras,
         "cpu_baseline": cpu,
     }
-    if sweep is not None:
-        line["bandwidth_sweep"] = sweep
+    if exchange is not None:
+        line["exchange_peer_gbs"] = exchange.get("peer", {}).get("gbs")
+        line["exchange_nccl_gbs"] = exchange.get("nccl", {}).get("gbs")
+        line["exchange"] = exchange
+    if full_sweep is not None:
+        line["bandwidth_sweep"] = full_sweep
     if rank == 0:
         print(json.dumps(line), flush=True)
     a2a.close()
@@ -853,8 +1119,14 @@ def run_exchange(args):
     dist.destroy_process_group()
 
 
+
+
 # ---------------------------------------------------------------- reference arm
 def run_reference(args):
+    """The CPU oracle, as it stands, on the host cores: the OpenMP build over
+    every core, each step mode 0 + mode 1 on a sample of the workload sized so
+    that warm-up and timed steps end in about two minutes; the single-threaded
+    build is timed on a short sample beside it."""
     rank, _, world = env_rank()
     if rank != 0:
         return
@@ -864,30 +1136,43 @@ def run_reference(args):
     wl = WORKLOADS[args.workload]
     w, B, S, H, D = (wl[k] for k in ("w", "B", "S_local", "H", "D"))
     E = 2
-    # size each step's sample so warmup + steps finish in about two minutes
-    probe_S = 256
-    xs = normal_slabs((B, probe_S, H, D), w, "bf16")
-    t = time.perf_counter()
-    y = oracle.ulysses_a2a(xs, 0)
-    oracle.ulysses_a2a(y, 1)
-    per_row = (time.perf_counter() - t) / probe_S
-    budget = 120.0 / max(1, args.steps + args.warmup)
-    S_sample = int(max(1, min(S, budget / max(per_row, 1e-9))))
+    lib = oracle.omp_lib()
+    threads = oracle.omp_threads()
+
+    def step(xs, which):
+        return oracle.ulysses_a2a(oracle.ulysses_a2a(xs, 0, lib=which), 1, lib=which)
+
+    def per_row(which):
+        probe_S = min(S, 64)
+        xs = normal_slabs((B, probe_S, H, D), w, "bf16")
+        t = time.perf_counter()
+        step(xs, which)
+        return (time.perf_counter() - t) / probe_S
+
+    budget = min(4.0, 120.0 / max(1, args.steps + args.warmup))
+    S_sample = int(max(1, min(S, budget / max(per_row(lib), 1e-9))))
     xs = normal_slabs((B, S_sample, H, D), w, "bf16")
     for _ in range(args.warmup):
-        y = oracle.ulysses_a2a(xs, 0)
-        oracle.ulysses_a2a(y, 1)
+        step(xs, lib)
     times = []
     for _ in range(args.steps):
         t = time.perf_counter()
-        y = oracle.ulysses_a2a(xs, 0)
-        oracle.ulysses_a2a(y, 1)
+        step(xs, lib)
         times.append(time.perf_counter() - t)
     P = w * B * S_sample * H * D * E
     total = sum(times)
     value = 2 * P * args.steps / total / 1e9
+    # the single-threaded build, on a sample of about 4 s
+    single = oracle._get_lib()
+    S1 = int(max(1, min(S, 4.0 / max(per_row(single), 1e-9))))
+    xs1 = normal_slabs((B, S1, H, D), w, "bf16")
+    t = time.perf_counter()
+    step(xs1, single)
+    t1 = time.perf_counter() - t
+    single_value = 2 * (w * B * S1 * H * D * E) / t1 / 1e9
     sample = (f"each step: mode 0 + mode 1 on S_local={S_sample} of {S} rows "
-              f"(w={w},B={B},H={H},D={D} bf16), single-threaded C nested loops")
+              f"(w={w},B={B},H={H},D={D} bf16), OpenMP build of the C nested loops, outer "
+              f"(r, b) loops over {threads} threads")
     line = {
         "impl": "reference",
         "metric": METRIC,
@@ -904,8 +1189,12 @@ def run_reference(args):
         "data": "synthetic",
         "config": {"workload": workload_name(w, B, S, H, D, 0), "name": args.workload,
                    "w": w, "B": B, "S_local": S, "H": H, "D": D},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "sample": sample, "threads": threads,
+                         "cores_on_box": os.cpu_count() or 1,
+                         "single_thread": {"value": round(single_value, 4), "unit": "GB/s",
+                                           "cores": 1,
+                                           "sample": f"one step on S_local={S1} of {S} rows"}},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "note": "ms_per_step is scaled from the sample to the full workload",
@@ -916,21 +1205,25 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--sweep-reps", type=int, default=50)
-    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--cpu-budget", type=float, default=16.0,
+                    help="seconds of CPU oracle timing, split over its two builds")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="only the headline step (no per-mode, isolated-call, other-workload, "
+                         "sweep or vector-shape sections)")
+    ap.add_argument("--no-exchange", action="store_true",
+                    help="with N > 1 GPUs, skip the cross-GPU exchange arms")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD,
                     help="benchmark workload, named by its sizes (default %(default)s)")
     ap.add_argument("--path", choices=["auto", "tma", "vec"], default="auto")
     ap.add_argument("--chunked", type=int, choices=[0, 1, 2], default=0)
     ap.add_argument("--sweep", action="store_true",
-                    help="also run the 128 KiB..2 GiB bandwidth sweep (w=2/4/8, bf16/fp32)")
+                    help="also run the full 128 KiB..2 GiB bandwidth sweep (w=2/4/8, bf16/fp32)")
     ap.add_argument("--exchange", choices=["nccl", "peer"], default=None,
                     help="multi-GPU Ulysses exchange (one rank slab per GPU, under torchrun): "
                          "nccl = a library all-to-all baseline, peer = this library's "

@@ -27,10 +27,11 @@
  * across GPUs, one process per GPU.
  *
  * Ownership: the caller owns every slab and the stream. The context owns a tiny
- * device status word, a cache of TMA descriptors, and (only if
- * ulysses_a2a_run_host is used) device staging buffers that grow on demand; a
- * peer object owns its rank's window. Nothing returned by this API ever aliases
- * caller memory.
+ * device status word, a cache of TMA descriptors, and two device buffers that
+ * exist only once they are used and then grow on demand: the staging window of
+ * chunked = 2 calls (one plane of every input slab) and the staging buffers of
+ * ulysses_a2a_run_host. A peer object owns its rank's window. Nothing returned
+ * by this API ever aliases caller memory.
  *
  * Launches: every kernel is launched with programmatic stream serialization
  * (programmatic dependent launch) and waits for the previous grid in the
@@ -175,7 +176,12 @@ int ulysses_a2a_destroy(ulysses_a2a_ctx *ctx);
  *               (twice the memory traffic of 0 and 1). Same bytes in the
  *               outputs whichever is chosen.
  *   stream    : a cudaStream_t (NULL = legacy default stream).
- * Asynchronous on `stream`; no host synchronisation and no allocation. */
+ * With chunked = 0 or 1 the call is asynchronous on `stream`: it neither
+ * synchronises the host nor allocates device memory. With chunked = 2, a call
+ * whose planes need a larger window than the context holds first synchronises
+ * `stream`, frees the old window and allocates a larger one (cudaMalloc), then
+ * queues its work; calls whose planes fit the current window neither allocate
+ * nor synchronise. */
 int ulysses_a2a_run(ulysses_a2a_ctx *ctx, const void *const *in_slabs,
                     void *const *out_slabs, int64_t B, int64_t S_local,
                     int64_t H, int64_t D, int w, int mode, int chunked,
@@ -281,26 +287,31 @@ int ulysses_a2a_plan(const void *const *in_slabs, void *const *out_slabs,
  * synchronise the whole device) is not allowed. ulysses_a2a_create allocates
  * the TMA kernel's status records; this call needs no context and allocates
  * nothing: it keeps those records in a file-scope static device array of 64
- * records x 16 bytes (1 KiB), one record per kernel launch, which every GPU
- * that loads the library holds until the process exits.
+ * records x 16 bytes (1 KiB), one record per TMA kernel launch, which every
+ * GPU that loads the library holds until the process exits. (The vector-path
+ * kernel has no bounded wait and uses no record.)
  *
  * Arguments and layout as ulysses_a2a_run, plus elem_bytes (1, 2, 4 or 8). It
  * runs on the CURRENT CUDA device, which must hold every slab. The caller still
  * owns all inputs and outputs.
- *   wait = 0 : return once the work is queued on `stream`.
+ *   wait = 0 : return once the work is queued on `stream`. Nothing reads
+ *              the status records of such a call, so a bounded wait that
+ *              gave up in it is never reported (the next call clears them).
  *   wait = 1 : also synchronise `stream` and check the status records;
  *              returns ULYSSES_A2A_ERR_TIMEOUT if a kernel gave up a wait.
  *   err      : optional buffer (errlen bytes) for a message on failure.
- * Limit: a chunked call launches once per plane and needs one record per
- * plane, so chunked calls over more than 64 planes are rejected with
- * ULYSSES_A2A_ERR_UNSUPPORTED and a message (unchunked calls need one record).
+ * Limit: a chunked call on the TMA path launches once per plane and needs one
+ * record per plane, so such calls over more than 64 planes are rejected with
+ * ULYSSES_A2A_ERR_UNSUPPORTED and a message (unchunked calls need one record,
+ * vector-path calls none).
  *
  * The first call on a device also does a one-time set-up for that device
  * (resolving the array's device address and the kernels' shared-memory limit);
- * make that first call before any stream capture. Every call shares the array
- * and the array keeps the last call's contents: each call clears the records
- * it uses, on `stream`, before its kernels run, so calls whose work overlaps
- * on the GPU (other streams, other host threads) race on the records. */
+ * make that first call before any stream capture. A set-up that fails is not
+ * remembered: the next call on that device tries it again. Every call shares
+ * the array and the array keeps the last call's contents: each call clears the
+ * records it uses, on `stream`, before its kernels run, so calls whose work
+ * overlaps on the GPU (other streams, other host threads) race on the records. */
 int ulysses_a2a_run_noalloc(const void *const *in_slabs, void *const *out_slabs,
                             int64_t B, int64_t S_local, int64_t H, int64_t D,
                             int w, int mode, int chunked, int elem_bytes,

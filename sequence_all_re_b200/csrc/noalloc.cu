@@ -23,8 +23,9 @@ using ua2a::VecParams;
 // static device array instead, and needs no context.
 //
 // The array is modest and fixed: kNoAllocSlots records of 16 bytes (1 KiB),
-// one record per kernel launch of a call (a chunked call launches once per
-// plane), held by every GPU that loads this library until the process exits.
+// one record per TMA kernel launch of a call (a chunked call launches once per
+// plane; the VEC kernel has no bounded wait and uses none), held by every GPU
+// that loads this library until the process exits.
 // Every call shares it and it keeps the last call's contents: each call clears
 // the records it uses, on its stream, before launching, so two calls whose work
 // overlaps on the GPU (different streams, or different host threads) race on it.
@@ -41,9 +42,8 @@ static __device__ __align__(256) unsigned int ua2a_noalloc_scratch[kNoAllocSlots
 namespace {
 
 struct NoAllocDevice {
-  std::once_flag once;
-  int rc = ULYSSES_A2A_OK;
-  char why[96] = {0};
+  std::mutex mu;
+  bool ready = false;               // set-up done and succeeded on this device
   unsigned int* scratch = nullptr;  // this device's address of ua2a_noalloc_scratch
   int num_sms = 0;
 };
@@ -59,32 +59,37 @@ int noalloc_report(char* err, size_t errlen, int rc, const char* fmt, long long 
   return rc;
 }
 
-// Once per device, with that device current: resolve the array's device address
+// Per device, with that device current: resolve the array's device address
 // (the symbol itself is only a host-side stand-in) and set the kernels' shared
-// memory limit.
-void noalloc_setup(NoAllocDevice& st, int dev) {
+// memory limit. Only a successful set-up is remembered; after a failure (for
+// example a cudaFuncSetAttribute refused during a stream capture) the next
+// call on that device tries again.
+int noalloc_setup(NoAllocDevice& st, int dev, char* err, size_t errlen) {
+  std::lock_guard<std::mutex> lock(st.mu);
+  if (st.ready) return ULYSSES_A2A_OK;
   cudaDeviceProp prop;
   if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess || prop.major < 10) {
     cudaGetLastError();
-    st.rc = ULYSSES_A2A_ERR_DEVICE;
-    std::snprintf(st.why, sizeof(st.why), "device %d is not an sm_100 GPU", dev);
-    return;
+    return noalloc_report(err, errlen, ULYSSES_A2A_ERR_DEVICE, "device %lld is not an sm_100 GPU",
+                          dev);
   }
-  st.num_sms = prop.multiProcessorCount;
   void* addr = nullptr;
   cudaError_t e = cudaGetSymbolAddress(&addr, ua2a_noalloc_scratch);
   if (e != cudaSuccess || addr == nullptr) {
     cudaGetLastError();
-    st.rc = ULYSSES_A2A_ERR_CUDA;
-    std::snprintf(st.why, sizeof(st.why), "cudaGetSymbolAddress failed: %s", cudaGetErrorName(e));
-    return;
+    if (err && errlen)
+      std::snprintf(err, errlen, "cudaGetSymbolAddress failed: %s", cudaGetErrorName(e));
+    return ULYSSES_A2A_ERR_CUDA;
   }
-  st.scratch = static_cast<unsigned int*>(addr);
   if (tma_allow_max_smem() != cudaSuccess) {
     cudaGetLastError();
-    st.rc = ULYSSES_A2A_ERR_CUDA;
-    std::snprintf(st.why, sizeof(st.why), "cudaFuncSetAttribute failed");
+    return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA,
+                          "cudaFuncSetAttribute failed (set-up is retried on the next call)");
   }
+  st.num_sms = prop.multiProcessorCount;
+  st.scratch = static_cast<unsigned int*>(addr);
+  st.ready = true;
+  return ULYSSES_A2A_OK;
 }
 
 bool noalloc_encode(CUtensorMap* m, int rank, const void* base, const cuuint64_t* dims,
@@ -129,11 +134,8 @@ static int ua2a_impl_run_noalloc(const void* const* in_slabs, void* const* out_s
     return noalloc_report(err, errlen, ULYSSES_A2A_ERR_DEVICE, "no usable current CUDA device");
   }
   NoAllocDevice& st = g_noalloc_dev[dev];
-  std::call_once(st.once, noalloc_setup, std::ref(st), dev);
-  if (st.rc != ULYSSES_A2A_OK) {
-    if (err && errlen) std::snprintf(err, errlen, "%s", st.why);
-    return st.rc;
-  }
+  const int setup_rc = noalloc_setup(st, dev, err, errlen);
+  if (setup_rc != ULYSSES_A2A_OK) return setup_rc;
 
   // the same checks as ulysses_a2a_run, before anything is launched
   ulysses_a2a_plan_t pl;
@@ -147,7 +149,10 @@ static int ua2a_impl_run_noalloc(const void* const* in_slabs, void* const* out_s
     return rc;
   }
   if (pl.units == 0) return ULYSSES_A2A_OK;  // empty: nothing to do
-  const int slots = pl.launches;
+  // Only the TMA kernel writes status records (one per launch); the VEC kernel
+  // has no bounded wait and needs none.
+  const bool tma = pl.path == ULYSSES_A2A_PATH_TMA;
+  const int slots = tma ? pl.launches : 0;
   if (slots > kNoAllocSlots)
     return noalloc_report(err, errlen, ULYSSES_A2A_ERR_UNSUPPORTED,
                           "chunked call over %lld planes needs %lld status records; the static "
@@ -185,14 +190,18 @@ static int ua2a_impl_run_noalloc(const void* const* in_slabs, void* const* out_s
   }
 
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);
-  // the records of this call start at zero (the array keeps the previous call's)
-  cudaError_t e = cudaMemsetAsync(st.scratch, 0, sizeof(unsigned int) * kNoAllocSlotWords * slots, st_);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "cudaMemsetAsync of the status records failed");
+  cudaError_t e = cudaSuccess;
+  if (slots > 0) {
+    // the records of this call start at zero (the array keeps the previous call's)
+    e = cudaMemsetAsync(st.scratch, 0, sizeof(unsigned int) * kNoAllocSlotWords * slots, st_);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA,
+                            "cudaMemsetAsync of the status records failed");
+    }
   }
   const int64_t nb = chunked ? 1 : B;
-  if (pl.path == ULYSSES_A2A_PATH_TMA) {
+  if (tma) {
     TmaParams p;
     std::memset(&p, 0, sizeof(p));
     const int64_t E = elem_bytes, Hw = H / w, rows = pl.rows_per_tile;
@@ -263,6 +272,7 @@ static int ua2a_impl_run_noalloc(const void* const* in_slabs, void* const* out_s
   e = cudaStreamSynchronize(st_);
   if (e != cudaSuccess)
     return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "cudaStreamSynchronize failed");
+  if (slots == 0) return ULYSSES_A2A_OK;
   unsigned int h[kNoAllocSlots * kNoAllocSlotWords];
   e = cudaMemcpy(h, st.scratch, sizeof(unsigned int) * kNoAllocSlotWords * slots, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess)

@@ -54,3 +54,29 @@ def test_workload_table_names_each_workload_by_its_sizes():
         assert parts["H"] == wl["H"] and parts["D"] == wl["D"]
         assert parts.get("B", 1) == wl["B"]
     assert bench.DEFAULT_WORKLOAD in bench.WORKLOADS
+
+
+def test_clock_windows_cover_only_their_timed_region():
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.samples = [(1.0, 1965.0, ()), (2.0, 1800.0, ("sw_power_cap",)), (3.0, 1965.0, ()),
+                 (4.0, 900.0, ("hw_slowdown",))]
+    s.max_mhz, s.source = 1965.0, "nvml"
+    w = s.window(1.5, 3.5)
+    assert w == {"sm_mhz": 1882.5, "sm_max_mhz": 1965.0, "samples": 2,
+                 "reasons": ["sw_power_cap"], "source": "nvml"}
+    assert s.window(4.5, 5.0) is None
+    assert s.window(0.0, 9.0)["reasons"] == ["hw_slowdown", "sw_power_cap"]
+
+
+def test_fractions_count_twice_the_payload():
+    # 1 GB of payload in 1 ms: 1000 GB/s of payload, 2000 GB/s of traffic
+    f = bench.fracs(10**9, 1.0, 4000.0)
+    assert f == {"gbs": 1000.0, "frac": 0.5, "frac_nominal": 0.25}
+
+
+def test_vector_shapes_are_named_by_their_sizes_and_leave_the_tma_path():
+    for name, (w, B, S, H, D, E, off) in bench.VEC_SHAPES.items():
+        assert f"w{w}_" in name and f"S{S}_" in name and f"H{H}_" in name and f"D{D}" in name
+        row = (H // w) * D * E
+        tma_blocked = row % 16 != 0 or off % 16 != 0 or w > 8
+        assert tma_blocked, name

@@ -4,17 +4,19 @@ Some callers cannot allocate device memory (their process's device memory is
 owned by another allocator under a fixed budget, or they run where cudaMalloc
 is not allowed). For them the library offers one entry point that allocates
 nothing: it keeps the copy kernel's status records in a static device array.
-These tests call it through the C ABI and check that its output equals the
-regular entry point's (bit for bit, the tolerance every test here uses) on two
-calls in a row, and that it rejects a chunked call needing more status records
-than the array holds. This file is named so pytest collects it last; it also
-passes when run alone in a fresh process (its first call does the one-time
-per-device set-up).
+These tests call it through the C ABI, on two calls in a row, and check every
+output byte against the CPU oracle's element map and against the regular entry
+point's output (bit for bit, the tolerance every test here uses). They also
+check that it rejects a TMA-path chunked call needing more status records than
+the array holds, while a vector-path chunked call over as many planes needs no
+record and runs. This file is named so pytest collects it last; it also passes
+when run alone in a fresh process (its first call does the per-device set-up).
 """
 
 import pytest
 import torch
 
+import oracle
 from sequence_all_re_b200 import UlyssesA2A, _lib
 from synth import normal_slabs, slab_shape, uniform_slabs
 
@@ -23,13 +25,36 @@ pytestmark = pytest.mark.gpu
 INT_OF = {2: torch.int16, 4: torch.int32}
 
 CASES = [
-    # (w, B, S_local, H, D, dtype, chunked)  -- TMA path unless noted
-    (4, 1, 8192, 24, 128, "bf16", 0),
-    (8, 2, 4725, 40, 128, "bf16", 1),
-    (2, 3, 37, 4, 64, "bf16", 1),
-    (4, 2, 45, 8, 128, "fp32", 0),
-    (2, 2, 17, 4, 3, "bf16", 0),      # 12-byte runs: the vector path
+    # (w, B, S_local, H, D, dtype, chunked, base offset in bytes); path noted
+    (4, 1, 8192, 24, 128, "bf16", 0, 0),    # TMA
+    (8, 2, 4725, 40, 128, "bf16", 1, 0),    # TMA, chunked, ragged tail
+    (2, 3, 37, 4, 64, "bf16", 1, 0),        # TMA, chunked
+    (4, 2, 45, 8, 128, "fp32", 0, 0),       # TMA, fp32
+    (2, 2, 17, 4, 3, "bf16", 0, 0),         # VEC: 12-byte runs
+    (2, 3, 17, 4, 3, "bf16", 1, 0),         # VEC, chunked
+    (4, 2, 33, 8, 64, "bf16", 0, 2),        # VEC: slab bases 2 bytes off 16
+    (4, 2, 33, 8, 64, "bf16", 1, 8),        # VEC, chunked, bases 8 bytes off 16
 ]
+
+
+def _device_slabs(cpu_slabs, offset):
+    """Copies of the CPU slabs on the GPU, each starting `offset` bytes into its
+    own allocation (a base address off the 16-byte boundary when offset > 0)."""
+    out = []
+    for t in cpu_slabs:
+        n = t.numel() * t.element_size()
+        raw = torch.empty(n + offset, dtype=torch.uint8, device="cuda")
+        d = raw[offset:].view(t.dtype).view(t.shape)
+        d.copy_(t)
+        out.append(d)
+    return out
+
+
+def _poisoned(shape, dtype, w, offset):
+    outs = _device_slabs([torch.empty(shape, dtype=dtype) for _ in range(w)], offset)
+    for o in outs:
+        o.view(torch.uint8).fill_(0xFF)
+    return outs
 
 
 def _noalloc(xs, outs, shape, mode, chunked, E, stream):
@@ -39,27 +64,32 @@ def _noalloc(xs, outs, shape, mode, chunked, E, stream):
                                         wait=1)
 
 
-@pytest.mark.parametrize("case", CASES, ids=lambda c: "w{}B{}S{}H{}D{}_{}_c{}".format(*c))
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "w{}B{}S{}H{}D{}_{}_c{}_off{}".format(*c))
 @pytest.mark.parametrize("mode", [0, 1])
-def test_noalloc_matches_run_on_two_calls_in_a_row(case, mode):
-    w, B, S, H, D, dtype, chunked = case
+def test_noalloc_matches_the_oracle_and_run_on_two_calls_in_a_row(case, mode):
+    w, B, S, H, D, dtype, chunked, off = case
     E = 2 if dtype == "bf16" else 4
     torch.cuda.set_device(0)
     stream = torch.cuda.current_stream()
     make = normal_slabs if dtype == "bf16" else uniform_slabs
     in_shape = slab_shape(mode, w, B, S, H, D)
     out_shape = slab_shape(1 - mode, w, B, S, H, D)
-    first = [t.cuda() for t in make(in_shape, w, dtype, seed0=40 + mode)]
-    second = [t.cuda() for t in make(in_shape, w, dtype, seed0=60 + mode)]
+    cpu1 = make(in_shape, w, dtype, seed0=40 + mode)
+    cpu2 = make(in_shape, w, dtype, seed0=60 + mode)
+    first, second = _device_slabs(cpu1, off), _device_slabs(cpu2, off)
+    plan = UlyssesA2A(0, E).plan(first, mode, chunked=bool(chunked))
+    assert plan["path"] == (_lib.PATH_VEC if (D * E) % 16 or off else _lib.PATH_TMA)
 
-    # expected outputs from the regular entry point
+    # expected outputs: the CPU oracle, and the regular entry point
+    oracle1 = oracle.ulysses_a2a(cpu1, mode)
+    oracle2 = oracle.ulysses_a2a(cpu2, mode)
     with UlyssesA2A(0, E) as a2a:
-        want1 = a2a.run(first, mode, chunked=bool(chunked))
-        want2 = a2a.run(second, mode, chunked=bool(chunked))
+        run1 = a2a.run(first, mode, chunked=bool(chunked))
+        run2 = a2a.run(second, mode, chunked=bool(chunked))
         a2a.status()
 
-    out1 = [torch.full(out_shape, float("nan"), dtype=first[0].dtype, device="cuda") for _ in range(w)]
-    out2 = [torch.full(out_shape, float("nan"), dtype=first[0].dtype, device="cuda") for _ in range(w)]
+    out1 = _poisoned(out_shape, first[0].dtype, w, off)
+    out2 = _poisoned(out_shape, first[0].dtype, w, off)
     torch.cuda.synchronize()
     rc, msg = _noalloc(first, out1, (w, B, S, H, D), mode, chunked, E, stream)
     assert rc == _lib.OK, msg
@@ -73,12 +103,15 @@ def test_noalloc_matches_run_on_two_calls_in_a_row(case, mode):
     assert torch.cuda.memory_allocated() == torch_before
     dt = INT_OF[E]
     for k in range(w):
-        assert torch.equal(out1[k].view(dt), want1[k].view(dt)), f"first call, rank {k}"
-        assert torch.equal(out2[k].view(dt), want2[k].view(dt)), f"second call, rank {k}"
+        got1, got2 = out1[k].cpu().view(dt), out2[k].cpu().view(dt)
+        assert torch.equal(got1, oracle1[k].view(dt)), f"first call vs oracle, rank {k}"
+        assert torch.equal(got2, oracle2[k].view(dt)), f"second call vs oracle, rank {k}"
+        assert torch.equal(got1, run1[k].cpu().view(dt)), f"first call vs run, rank {k}"
+        assert torch.equal(got2, run2[k].cpu().view(dt)), f"second call vs run, rank {k}"
 
 
-def test_noalloc_rejects_more_planes_than_status_records():
-    w, B, S, H, D = 2, 65, 2, 2, 8        # a chunked call over 65 planes needs 65 records
+def test_noalloc_rejects_more_tma_planes_than_status_records():
+    w, B, S, H, D = 2, 65, 2, 2, 8        # 16-byte runs: TMA, one record per plane
     stream = torch.cuda.current_stream()
     xs = [t.cuda() for t in normal_slabs((B, S, H, D), w, "bf16")]
     outs = [torch.zeros((B, S * w, H // w, D), dtype=torch.bfloat16, device="cuda") for _ in range(w)]
@@ -90,6 +123,21 @@ def test_noalloc_rejects_more_planes_than_status_records():
     # the same data unchunked needs one record and is accepted
     rc, msg = _noalloc(xs, outs, (w, B, S, H, D), 0, 0, 2, stream)
     assert rc == _lib.OK, msg
+    want = oracle.ulysses_a2a([t.cpu() for t in xs], 0)
+    assert all(torch.equal(o.cpu().view(torch.int16), e.view(torch.int16)) for o, e in zip(outs, want))
+
+
+def test_noalloc_chunked_vector_path_needs_no_status_record():
+    w, B, S, H, D = 2, 65, 3, 2, 3        # 6-byte runs: VEC path, 65 launches, no record
+    stream = torch.cuda.current_stream()
+    cpu = normal_slabs((B, S, H, D), w, "bf16", seed0=90)
+    xs = [t.cuda() for t in cpu]
+    outs = [torch.full((B, S * w, H // w, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+            for _ in range(w)]
+    rc, msg = _noalloc(xs, outs, (w, B, S, H, D), 0, 1, 2, stream)
+    assert rc == _lib.OK, msg
+    want = oracle.ulysses_a2a(cpu, 0)
+    assert all(torch.equal(o.cpu().view(torch.int16), e.view(torch.int16)) for o, e in zip(outs, want))
 
 
 def test_noalloc_rejects_bad_arguments_with_a_message():
