@@ -102,14 +102,24 @@ VEC_SHAPES = {
 }
 
 
-def workload_key(w, B, S, H, D, path):
-    return f"{path}:w{w}_B{B}_S{S}_H{H}_D{D}_bf16"
+# Every workload --workload accepts: the table above, and the vector-path shapes
+# (element size and base offset as listed there).
+ALL_WORKLOADS = {**{n: dict(v, E=2, off=0) for n, v in WORKLOADS.items()},
+                 **{n: dict(w=v[0], B=v[1], S_local=v[2], H=v[3], D=v[4], E=v[5], off=v[6])
+                    for n, v in VEC_SHAPES.items()}}
+DTYPE_OF = {2: "bf16", 4: "fp32"}
+INT_OF = {2: torch.int16, 4: torch.int32}
 
 
-def workload_name(w, B, S, H, D, chunked):
+def workload_key(w, B, S, H, D, path, E=2, off=0):
+    return f"{path}:w{w}_B{B}_S{S}_H{H}_D{D}_{DTYPE_OF[E]}" + (f"_base{off}" if off else "")
+
+
+def workload_name(w, B, S, H, D, chunked, E=2, off=0):
     how = {0: "", 1: ", chunked per plane", 2: ", chunked through the staging window"}[chunked]
-    return (f"ulysses_a2a w={w} B={B} S_local={S} H={H} D={D} bf16, step = mode 0 + mode 1"
-            f"{how}")
+    base = f", slab bases {off} bytes past a 16-byte boundary" if off else ""
+    return (f"ulysses_a2a w={w} B={B} S_local={S} H={H} D={D} {DTYPE_OF[E]}{base}, "
+            f"step = mode 0 + mode 1{how}")
 
 
 FALLBACK_HBM_GBS = 6650.0
@@ -164,7 +174,8 @@ def _code_only(text: str) -> str:
     return " ".join(text.split())
 
 
-KERNEL_FILES = {"tma": "kernels_tma.cuh", "vec": "kernels_vec.cuh"}
+KERNEL_FILES = {"tma": "kernels_tma.cuh", "vec": "kernels_vec.cuh", "staged": "kernels_stage.cuh"}
+PATH_NAMES = {1: "tma", 2: "vec", 3: "staged"}
 LAUNCH_FIELDS = ("path", "rows_per_tile", "producers", "stages", "lookahead", "chunk_units",
                  "order", "grid", "block", "smem_bytes", "vec_bytes")
 
@@ -484,7 +495,9 @@ def per_mode_block(a2a, ins, outs, back, P, stream, peak, sampler, seconds, chun
 
 
 def vec_shape_block(device, peak, sampler, seconds=0.5):
-    """The VEC-only shapes: each mode back to back; plan, GB/s and fractions."""
+    """The shapes TMA cannot take: each mode back to back, on the path AUTO picks
+    (the staged path where 16-byte vectors cannot be used directly) and on the
+    vector path forced; plan, GB/s and fractions."""
     from sequence_all_re_b200 import UlyssesA2A
 
     stream = torch.cuda.Stream(device)
@@ -501,35 +514,47 @@ def vec_shape_block(device, peak, sampler, seconds=0.5):
         torch.cuda.synchronize()
         if not all(torch.equal(z[k], x[k]) for k in range(w)):
             raise SystemExit(f"vector-path shape {name}: round trip mismatch")
-        out[name] = {"payload_bytes": P, "path": {1: "tma", 2: "vec"}[p["path"]],
+        out[name] = {"payload_bytes": P, "path": PATH_NAMES[p["path"]],
                      "vec_bytes": p["vec_bytes"], "row_bytes": p["row_bytes"],
                      "base_offset_bytes": off, **res}
+        if p["path"] != 2:
+            a2a.set_path(2)
+            pv = a2a.plan(x, 0, out=y)
+            for t in z:
+                t.zero_()
+            forced = per_mode_block(a2a, x, y, z, P, stream, peak, sampler, seconds)
+            torch.cuda.synchronize()
+            if not all(torch.equal(z[k], x[k]) for k in range(w)):
+                raise SystemExit(f"vector-path shape {name}: round trip mismatch (VEC forced)")
+            out[name]["vec_forced"] = {"vec_bytes": pv["vec_bytes"],
+                                       **{m: {k: v for k, v in forced[m].items() if k != "clocks"}
+                                          for m in forced}}
         a2a.close()
         del x, y, z
         torch.cuda.empty_cache()
     return out
 
 
-def cpu_oracle_baseline(w, B, S, H, D, budget_s=12.0):
+def cpu_oracle_baseline(w, B, S, H, D, budget_s=12.0, E=2):
     """The oracle, as it stands, on the host cores: the OpenMP build (the outer
     (r, b) loops over every core) and the single-threaded build, each on whole
     mode 0 + mode 1 steps of a sample of the workload for about budget_s / 2."""
     import oracle
     from synth import normal_slabs
 
-    E = 2
+    dt = DTYPE_OF[E]
     cores_on_box = os.cpu_count() or 1
     threads = oracle.omp_threads()
     res = {}
     for kind, lib in (("openmp", oracle.omp_lib()), ("single", oracle._get_lib())):
         # size the sample from a small probe: about 1 s per step
         probe_S = min(S, 64)
-        xs = normal_slabs((B, probe_S, H, D), w, "bf16")
+        xs = normal_slabs((B, probe_S, H, D), w, dt)
         t = time.perf_counter()
         oracle.ulysses_a2a(oracle.ulysses_a2a(xs, 0, lib=lib), 1, lib=lib)
         per_row = (time.perf_counter() - t) / probe_S
         S_sample = int(max(1, min(S, 1.0 / max(per_row, 1e-9))))
-        xs = normal_slabs((B, S_sample, H, D), w, "bf16")
+        xs = normal_slabs((B, S_sample, H, D), w, dt)
         done, t_start = 0, time.perf_counter()
         while True:
             oracle.ulysses_a2a(oracle.ulysses_a2a(xs, 0, lib=lib), 1, lib=lib)
@@ -540,7 +565,7 @@ def cpu_oracle_baseline(w, B, S, H, D, budget_s=12.0):
         P = w * B * S_sample * H * D * E
         res[kind] = {"value": round(2 * P * done / el / 1e9, 4), "threads": threads if kind == "openmp" else 1,
                      "sample": f"{done} steps (mode 0 + mode 1) on S_local={S_sample} of {S} rows "
-                               f"(w={w},B={B},H={H},D={D} bf16) in {el:.1f} s"}
+                               f"(w={w},B={B},H={H},D={D} {dt}) in {el:.1f} s"}
     return {"value": res["openmp"]["value"], "unit": "GB/s", "cores": threads, "kind": "oracle",
             "threads": threads, "cores_on_box": cores_on_box,
             "sample": "OpenMP build, outer (r, b) loops over every core: " + res["openmp"]["sample"],
@@ -616,22 +641,23 @@ def run_ours(args):
     from sequence_all_re_b200 import UlyssesA2A
 
     sampler = ClockSampler(local_rank).start()
-    wl = WORKLOADS[args.workload]
-    w, B, S, H, D = (wl[k] for k in ("w", "B", "S_local", "H", "D"))
-    E = 2
+    wl = ALL_WORKLOADS[args.workload]
+    w, B, S, H, D, E, off = (wl[k] for k in ("w", "B", "S_local", "H", "D", "E", "off"))
     P = w * B * S * H * D * E
     a2a = UlyssesA2A(local_rank, E)
-    a2a.set_path({"auto": 0, "tma": 1, "vec": 2}[args.path])
+    a2a.set_path({"auto": 0, "tma": 1, "vec": 2, "staged": 3}[args.path])
     chunked = args.chunked
     stream = torch.cuda.Stream(device)
-    x = make_inputs(w, B, S, H, D, "bf16", device)
-    y = [torch.empty((B, S * w, H // w, D), dtype=torch.bfloat16, device=device) for _ in range(w)]
-    z = [torch.empty_like(t) for t in x]
+    x = make_inputs(w, B, S, H, D, DTYPE_OF[E], device, offset_bytes=off)
+    y = empty_slabs(w, (B, S * w, H // w, D), x[0].dtype, device, off)
+    z = empty_slabs(w, (B, S, H, D), x[0].dtype, device, off)
     # mode 1 reads its own slabs (a seeded copy of mode 0's result), not y
     with torch.cuda.stream(stream):
         a2a.run(x, 0, out=y, stream=stream)
     torch.cuda.synchronize()
-    y2 = [t.clone() for t in y]
+    y2 = empty_slabs(w, (B, S * w, H // w, D), x[0].dtype, device, off)
+    for a, b in zip(y2, y):
+        a.copy_(b)
     plan = a2a.plan(x, 0, chunked=chunked, out=y)
 
     if dist:
@@ -646,7 +672,7 @@ def run_ours(args):
         dist.barrier()
     # the round trip must reproduce the input bit for bit (y2 holds mode 0's output)
     for k in range(w):
-        if not torch.equal(z[k].view(torch.int16), x[k].view(torch.int16)):
+        if not torch.equal(z[k].view(INT_OF[E]), x[k].view(INT_OF[E])):
             raise SystemExit("round trip mismatch: mode1(mode0(x)) != x")
     total_ms = max_over_ranks(total_ms, dist, device)
     ms_per_step = total_ms / args.steps
@@ -656,11 +682,11 @@ def run_ours(args):
     avg_launch_ms = total_ms / launches
     bytes_per_launch = 2 * P * 2 * args.steps // launches       # 2 calls of 2P per step
     achieved = bytes_per_launch / (avg_launch_ms / 1e3) / 1e9
-    key = workload_key(w, B, S, H, D, {1: "tma", 2: "vec"}[plan["path"]])
+    key = workload_key(w, B, S, H, D, PATH_NAMES[plan["path"]], E, off)
     traffic_bytes, traffic_src = ncu_traffic(key, plan, chunked)
 
     extras = {}
-    if world == 1 and not args.no_extras:
+    if world == 1 and not args.no_extras and args.workload in WORKLOADS:
         # each mode of the headline workload, back to back for >= 1 s
         extras["per_mode"] = per_mode_block(a2a, x, y2, z, P, stream, peak, sampler, 1.0, chunked)
         # one call at a time after a clean L2 flush
@@ -719,7 +745,7 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         hx = [t.cpu().pin_memory() for t in x]
-        hy = [torch.empty((B, S * w, H // w, D), dtype=torch.bfloat16).pin_memory() for _ in range(w)]
+        hy = [torch.empty((B, S * w, H // w, D), dtype=x[0].dtype).pin_memory() for _ in range(w)]
         hz = [torch.empty_like(t).pin_memory() for t in hx]
         for _ in range(2):
             a2a.run_host(hx, 0, out=hy, stream=stream)
@@ -740,7 +766,7 @@ def run_ours(args):
         tb = time.perf_counter()
         e_ms = max_over_ranks(ea.elapsed_time(eb), dist, device)
         for k in range(w):
-            if not torch.equal(hz[k].view(torch.int16), hx[k].view(torch.int16)):
+            if not torch.equal(hz[k].view(INT_OF[E]), hx[k].view(INT_OF[E])):
                 raise SystemExit("host-path round trip mismatch")
         e2e = {"value": round(job_gbs(world, 2 * P, e_steps, e_ms), 3), "unit": "GB/s",
                "h2d_bytes_per_step": 2 * P, "d2h_bytes_per_step": 2 * P,
@@ -760,7 +786,7 @@ def run_ours(args):
     sampler.stop()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_oracle_baseline(w, B, S, H, D, budget_s=args.cpu_budget)
+        cpu = cpu_oracle_baseline(w, B, S, H, D, budget_s=args.cpu_budget, E=E)
 
     line = {
         "metric": METRIC,
@@ -773,14 +799,14 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": DTYPE_OF[E],
         "data": "synthetic",
         "config": {
-            "workload": workload_name(w, B, S, H, D, chunked),
+            "workload": workload_name(w, B, S, H, D, chunked, E, off),
             "name": args.workload,
             "w": w, "B": B, "S_local": S, "H": H, "D": D,
             "payload_bytes_per_call": P,
-            "path": {1: "tma", 2: "vec"}[plan["path"]],
+            "path": PATH_NAMES[plan["path"]],
             "rows_per_tile": plan["rows_per_tile"], "producers": plan["producers"],
             "stages": plan["stages"], "chunk_units": plan["chunk_units"], "grid": plan["grid"],
             "l2": (f"inputs larger than L2 ({P / 2**20:.0f} MiB per call vs 126 MB); no kernel "
@@ -791,7 +817,8 @@ def run_ours(args):
         },
         "roofline": {
             "bound": "hbm",
-            "kernel": "ua2a_tma_kernel<0>/<1>" if plan["path"] == 1 else "ua2a_vec_kernel",
+            "kernel": {1: "ua2a_tma_kernel<0>/<1>", 2: "ua2a_vec_kernel",
+                       3: "ua2a_stage_kernel"}[plan["path"]],
             "achieved": round(achieved, 1),
             "peak": peak,
             "unit": "GB/s",
@@ -1133,9 +1160,9 @@ def run_reference(args):
     import oracle
     from synth import normal_slabs
 
-    wl = WORKLOADS[args.workload]
-    w, B, S, H, D = (wl[k] for k in ("w", "B", "S_local", "H", "D"))
-    E = 2
+    wl = ALL_WORKLOADS[args.workload]
+    w, B, S, H, D, E = (wl[k] for k in ("w", "B", "S_local", "H", "D", "E"))
+    dt = DTYPE_OF[E]
     lib = oracle.omp_lib()
     threads = oracle.omp_threads()
 
@@ -1144,14 +1171,14 @@ def run_reference(args):
 
     def per_row(which):
         probe_S = min(S, 64)
-        xs = normal_slabs((B, probe_S, H, D), w, "bf16")
+        xs = normal_slabs((B, probe_S, H, D), w, dt)
         t = time.perf_counter()
         step(xs, which)
         return (time.perf_counter() - t) / probe_S
 
     budget = min(4.0, 120.0 / max(1, args.steps + args.warmup))
     S_sample = int(max(1, min(S, budget / max(per_row(lib), 1e-9))))
-    xs = normal_slabs((B, S_sample, H, D), w, "bf16")
+    xs = normal_slabs((B, S_sample, H, D), w, dt)
     for _ in range(args.warmup):
         step(xs, lib)
     times = []
@@ -1165,13 +1192,13 @@ def run_reference(args):
     # the single-threaded build, on a sample of about 4 s
     single = oracle._get_lib()
     S1 = int(max(1, min(S, 4.0 / max(per_row(single), 1e-9))))
-    xs1 = normal_slabs((B, S1, H, D), w, "bf16")
+    xs1 = normal_slabs((B, S1, H, D), w, dt)
     t = time.perf_counter()
     step(xs1, single)
     t1 = time.perf_counter() - t
     single_value = 2 * (w * B * S1 * H * D * E) / t1 / 1e9
     sample = (f"each step: mode 0 + mode 1 on S_local={S_sample} of {S} rows "
-              f"(w={w},B={B},H={H},D={D} bf16), OpenMP build of the C nested loops, outer "
+              f"(w={w},B={B},H={H},D={D} {dt}), OpenMP build of the C nested loops, outer "
               f"(r, b) loops over {threads} threads")
     line = {
         "impl": "reference",
@@ -1185,9 +1212,9 @@ def run_reference(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": dt,
         "data": "synthetic",
-        "config": {"workload": workload_name(w, B, S, H, D, 0), "name": args.workload,
+        "config": {"workload": workload_name(w, B, S, H, D, 0, E, wl["off"]), "name": args.workload,
                    "w": w, "B": B, "S_local": S, "H": H, "D": D},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
                          "kind": "oracle", "sample": sample, "threads": threads,
@@ -1218,9 +1245,9 @@ def main():
     ap.add_argument("--no-exchange", action="store_true",
                     help="with N > 1 GPUs, skip the cross-GPU exchange arms")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD,
+    ap.add_argument("--workload", choices=sorted(ALL_WORKLOADS), default=DEFAULT_WORKLOAD,
                     help="benchmark workload, named by its sizes (default %(default)s)")
-    ap.add_argument("--path", choices=["auto", "tma", "vec"], default="auto")
+    ap.add_argument("--path", choices=["auto", "tma", "vec", "staged"], default="auto")
     ap.add_argument("--chunked", type=int, choices=[0, 1, 2], default=0)
     ap.add_argument("--sweep", action="store_true",
                     help="also run the full 128 KiB..2 GiB bandwidth sweep (w=2/4/8, bf16/fp32)")

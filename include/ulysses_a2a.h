@@ -74,9 +74,13 @@ extern "C" {
                                           an entry point)                       */
 
 /* ---- copy paths ------------------------------------------------------- */
-#define ULYSSES_A2A_PATH_AUTO 0  /* TMA when the shape allows it, else VEC     */
+#define ULYSSES_A2A_PATH_AUTO 0  /* TMA when the shape allows it; else VEC, or
+                                    STAGED when VEC could only use vectors
+                                    narrower than 16 bytes                   */
 #define ULYSSES_A2A_PATH_TMA  1  /* cp.async.bulk.tensor load -> smem -> store */
 #define ULYSSES_A2A_PATH_VEC  2  /* 16/8/4/2/1-byte LDG/STG copy               */
+#define ULYSSES_A2A_PATH_STAGED 3 /* 16-byte LDG/STG, re-aligned in shared
+                                    memory: runs or bases off 16 bytes     */
 
 #define ULYSSES_A2A_MAX_W     64 /* largest rank count any path accepts        */
 #define ULYSSES_A2A_CHUNKED_WINDOW 2 /* chunked = 2: per plane via a window   */
@@ -86,13 +90,17 @@ typedef struct ulysses_a2a_ctx ulysses_a2a_ctx; /* opaque */
 
 /* Geometry and path the library picks for one call (see ulysses_a2a_plan). */
 typedef struct ulysses_a2a_plan_t {
-    int32_t path;            /* ULYSSES_A2A_PATH_TMA or _VEC                  */
-    int32_t vec_bytes;       /* VEC path: bytes per load/store (16..1)        */
+    int32_t path;            /* ULYSSES_A2A_PATH_TMA, _VEC or _STAGED         */
+    int32_t vec_bytes;       /* VEC path: bytes per load/store (16..1);
+                                STAGED: bytes per piece re-aligned in shared
+                                memory (global accesses are 16 bytes)       */
     int64_t row_bytes;       /* one contiguous run: (H/w)*D*elem_bytes        */
     int64_t rows_per_tile;   /* S_tile: sequence rows per work unit           */
     int64_t tiles_per_block; /* ceil(S_local / S_tile)                        */
     int64_t tail_rows;       /* S_local % S_tile (0 = no ragged tile)         */
-    int64_t units;           /* work units per launch: w * B_launch * w * T   */
+    int64_t units;           /* work units per launch: w * B_launch * w * T
+                                (STAGED: w * B_launch * T, each unit moving
+                                every head group of its rows)              */
     int64_t payload_bytes;   /* sum of input slab bytes = w*B*S_local*H*D*E   */
     int32_t launches;        /* kernel launches per call: 1, or B if chunked  */
     int32_t grid;            /* CTAs per launch                               */
@@ -408,6 +416,26 @@ int ulysses_a2a_peer_publish(ulysses_a2a_peer *peer, const void *in_local,
 int ulysses_a2a_peer_pull(ulysses_a2a_peer *peer, void *out_local, int64_t B,
                           int64_t S_local, int64_t H, int64_t D, int mode,
                           int64_t row_pitch, size_t window_offset, void *stream);
+
+/* Step 3 for T tensors packed along the head dimension (for example q, k and
+ * v of a packed projection output), in ONE kernel launch for all T (the
+ * launch of ulysses_a2a_run_ex with ntensors = T, restricted to this rank's
+ * outputs). 1 <= ntensors, ntensors * world <= ULYSSES_A2A_MAX_W.
+ *   mode 0: every window holds its rank's packed [B, S_local, T, H, D] slab,
+ *           dense, from byte window_offset on (published with T*H heads);
+ *           out_local holds T device pointers, out_local[t] receiving this
+ *           rank's dense [B, S_local*w, H/w, D] slab of tensor t.
+ *   mode 1: every window holds T dense [B, S_local*w, H/w, D] slabs, tensor
+ *           t's at byte window_offset + t*B*S_local*H*D*elem_bytes;
+ *           out_local[0] receives this rank's dense packed [B, S_local, T, H,
+ *           D] slab.
+ * Same bytes as T calls of ulysses_a2a_peer_pull with row pitch T*H*D and
+ * the matching window offsets. Asynchronous on stream; VEC kernel, peer
+ * loads; no output overlaps a window. */
+int ulysses_a2a_peer_pull_packed(ulysses_a2a_peer *peer, void *const *out_local,
+                                 int ntensors, int64_t B, int64_t S_local,
+                                 int64_t H, int64_t D, int mode,
+                                 size_t window_offset, void *stream);
 
 /* Base address of rank k's window as this process sees it (NULL if k is out
  * of range or not mapped yet), and the window size in bytes. */

@@ -22,10 +22,10 @@ from __future__ import annotations
 import torch
 
 from . import _lib
-from ._lib import A2AError, PATH_AUTO, PATH_TMA, PATH_VEC  # noqa: F401
+from ._lib import A2AError, PATH_AUTO, PATH_STAGED, PATH_TMA, PATH_VEC  # noqa: F401
 
 __all__ = ["UlyssesA2A", "A2AError", "output_shape", "mode0_local_tuple",
-           "PATH_AUTO", "PATH_TMA", "PATH_VEC"]
+           "PATH_AUTO", "PATH_TMA", "PATH_VEC", "PATH_STAGED"]
 
 
 def output_shape(in_shape, mode: int, w: int) -> tuple:

@@ -26,6 +26,7 @@ ERR_INTERNAL = 8
 PATH_AUTO = 0
 PATH_TMA = 1
 PATH_VEC = 2
+PATH_STAGED = 3
 
 MAX_W = 64
 MAX_W_TMA = 8
@@ -50,6 +51,7 @@ EXPORTED = (
     "ulysses_a2a_peer_open",
     "ulysses_a2a_peer_publish",
     "ulysses_a2a_peer_pull",
+    "ulysses_a2a_peer_pull_packed",
     "ulysses_a2a_peer_window",
     "ulysses_a2a_peer_window_bytes",
     "ulysses_a2a_peer_close",
@@ -204,6 +206,9 @@ def _load() -> ctypes.CDLL:
     lib.ulysses_a2a_peer_publish.restype = c_int
     lib.ulysses_a2a_peer_pull.argtypes = [P, P, i64, i64, i64, i64, c_int, i64, ctypes.c_size_t, P]
     lib.ulysses_a2a_peer_pull.restype = c_int
+    lib.ulysses_a2a_peer_pull_packed.argtypes = [P, PP, c_int, i64, i64, i64, i64, c_int,
+                                                 ctypes.c_size_t, P]
+    lib.ulysses_a2a_peer_pull_packed.restype = c_int
     lib.ulysses_a2a_peer_window.argtypes = [P, c_int]
     lib.ulysses_a2a_peer_window.restype = P
     lib.ulysses_a2a_peer_window_bytes.argtypes = [P]
@@ -354,6 +359,15 @@ def ulysses_a2a_peer_pull(peer, out_ptr, B, S_local, H, D, mode, row_pitch, stre
     return lib.ulysses_a2a_peer_pull(peer, ctypes.c_void_p(int(out_ptr) or None), int(B),
                                      int(S_local), int(H), int(D), int(mode), int(row_pitch),
                                      int(window_offset), ctypes.c_void_p(int(stream)))
+
+
+def ulysses_a2a_peer_pull_packed(peer, out_ptrs, ntensors, B, S_local, H, D, mode, stream,
+                                 window_offset=0) -> int:
+    """One launch for T head-packed tensors: out_ptrs holds T output pointers in
+    mode 0, the one packed output in mode 1."""
+    return lib.ulysses_a2a_peer_pull_packed(peer, ptr_array(out_ptrs), int(ntensors), int(B),
+                                            int(S_local), int(H), int(D), int(mode),
+                                            int(window_offset), ctypes.c_void_p(int(stream)))
 
 
 def ulysses_a2a_peer_window(peer, rank: int) -> int:

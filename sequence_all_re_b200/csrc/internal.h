@@ -15,6 +15,7 @@
 #include <string>
 #include <vector>
 
+#include "kernels_stage.cuh"
 #include "kernels_tma.cuh"
 #include "kernels_vec.cuh"
 #include "plan.h"
@@ -55,6 +56,7 @@ struct ulysses_a2a_ctx {
   uint64_t stamp = 0;
   ua2a::TmaCacheEntry tma_cache[ua2a::kTmaCacheEntries];
   bool tma_smem_set[2] = {false, false};
+  bool stage_smem_set = false;
   int64_t tma_smem_set_bytes[2] = {0, 0};
   // run_host staging: one device buffer carved into 2w slabs
   void* d_stage = nullptr;
@@ -98,6 +100,14 @@ cudaError_t launch_tma(int mode, int grid, int block, size_t smem, cudaStream_t 
                        const TmaParams& p);
 cudaError_t launch_vec(const VecParams& p, int vec_bytes, int mode, int grid, int block,
                        cudaStream_t st);
+cudaError_t launch_stage(const StageParams& p, int piece_bytes, int mode, int grid, int block,
+                         size_t smem, cudaStream_t st);
+// Let every staged kernel use up to kStageSmemMax of dynamic shared memory.
+cudaError_t stage_allow_max_smem();
+// Staged-kernel parameters for a plan (slab pointers, tile0 and b0 left for
+// the caller): nt tiles per (b, j) block, `units` units in the launch.
+StageParams stage_params(int64_t S, int w, int ntensors, int E, const ulysses_a2a_plan_t& pl,
+                         int64_t nt, int64_t units);
 // Let both TMA kernels use up to kTmaSmemMax of dynamic shared memory (on the
 // current device; the attribute belongs to the instantiations launched above).
 cudaError_t tma_allow_max_smem();

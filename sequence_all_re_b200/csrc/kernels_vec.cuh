@@ -15,9 +15,11 @@
 // holding only the S_local % S_tile remaining rows (ceil-div tiling, clamped
 // row count). Each thread keeps U vectors in flight before storing them.
 //
-// A launch may cover every output slab or only one (r in [r0, r0 + nr) and
-// j in [j0, j0 + nj)): one rank's share of a multi-GPU exchange writes its own
-// output slab and reads every rank's published input through peer mappings.
+// A launch may cover every output slab or only one rank's: r in
+// {r0 + k*r_stride : k < nr} and j in [j0, j0 + nj). One rank's share of a
+// multi-GPU exchange writes its own output slab (one per tensor when T
+// tensors are head-packed: head groups t*w + rank, r_stride = w) and reads
+// every rank's published input through peer mappings.
 #pragma once
 
 #include <cstdint>
@@ -63,6 +65,8 @@ struct VecParams {
   int32_t order;         // unit numbering: 0 = r outermost, 1 = r innermost
   uint32_t tile0;        // first tile of each (r, b, j) block in this launch
   uint32_t r0, j0;       // first r and first j this launch covers
+  uint32_t r_stride;     // head groups between consecutive r of the launch (1, or w to
+                         // take one rank's group of each of T head-packed tensors)
   FastDiv div_T;         // tiles per (r, b, j) block in this launch
   FastDiv div_nr;        // r values covered (w, or 1 for one output slab)
   FastDiv div_nj;        // j values covered
@@ -75,11 +79,17 @@ __device__ __forceinline__ uint2 ld_stream(const uint2* p) { return __ldcs(p); }
 __device__ __forceinline__ unsigned int ld_stream(const unsigned int* p) { return __ldcs(p); }
 __device__ __forceinline__ unsigned short ld_stream(const unsigned short* p) { return __ldcs(p); }
 __device__ __forceinline__ unsigned char ld_stream(const unsigned char* p) { return __ldcs(p); }
+__device__ __forceinline__ unsigned long long ld_stream(const unsigned long long* p) {
+  return __ldcs(p);
+}
 __device__ __forceinline__ void st_stream(uint4* p, uint4 v) { __stcs(p, v); }
 __device__ __forceinline__ void st_stream(uint2* p, uint2 v) { __stcs(p, v); }
 __device__ __forceinline__ void st_stream(unsigned int* p, unsigned int v) { __stcs(p, v); }
 __device__ __forceinline__ void st_stream(unsigned short* p, unsigned short v) { __stcs(p, v); }
 __device__ __forceinline__ void st_stream(unsigned char* p, unsigned char v) { __stcs(p, v); }
+__device__ __forceinline__ void st_stream(unsigned long long* p, unsigned long long v) {
+  __stcs(p, v);
+}
 
 // 256-thread CTAs, at least 6 resident per SM: caps the kernel at 40
 // registers, so every variant runs at 75% occupancy.
@@ -116,7 +126,7 @@ __global__ void __launch_bounds__(256, kVecMinBlocksPerSm)
       bl = fdiv(q2, p.div_nj);
       j = q2 - bl * p.div_nj.d;
     }
-    r += p.r0;
+    r = p.r0 + r * p.r_stride;
     j += p.j0;
     const int64_t b = p.b0 + bl;
     const int64_t s0 = (int64_t)(p.tile0 + t) * p.rows_per_tile;

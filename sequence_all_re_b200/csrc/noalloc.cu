@@ -9,6 +9,7 @@
 #include "internal.h"
 
 using namespace ua2a;
+using ua2a::StageParams;
 using ua2a::TmaParams;
 using ua2a::VecParams;
 
@@ -81,7 +82,7 @@ int noalloc_setup(NoAllocDevice& st, int dev, char* err, size_t errlen) {
       std::snprintf(err, errlen, "cudaGetSymbolAddress failed: %s", cudaGetErrorName(e));
     return ULYSSES_A2A_ERR_CUDA;
   }
-  if (tma_allow_max_smem() != cudaSuccess) {
+  if (tma_allow_max_smem() != cudaSuccess || stage_allow_max_smem() != cudaSuccess) {
     cudaGetLastError();
     return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA,
                           "cudaFuncSetAttribute failed (set-up is retried on the next call)");
@@ -243,6 +244,18 @@ static int ua2a_impl_run_noalloc(const void* const* in_slabs, void* const* out_s
       if (e != cudaSuccess)
         return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "TMA kernel launch failed (plane %lld)", l);
     }
+  } else if (pl.path == ULYSSES_A2A_PATH_STAGED) {
+    StageParams p = stage_params(S_local, w, 1, elem_bytes, pl, pl.tiles_per_block, pl.units);
+    for (int k = 0; k < w; ++k) {
+      p.in[k] = static_cast<const char*>(in_slabs[k]);
+      p.out[k] = static_cast<char*>(out_slabs[k]);
+    }
+    for (int l = 0; l < pl.launches; ++l) {
+      p.b0 = chunked ? l : 0;
+      e = launch_stage(p, pl.vec_bytes, mode, pl.grid, pl.block, (size_t)pl.smem_bytes, st_);
+      if (e != cudaSuccess)
+        return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "staged kernel launch failed (plane %lld)", l);
+    }
   } else {
     VecParams p{};
     for (int k = 0; k < w; ++k) {
@@ -250,6 +263,7 @@ static int ua2a_impl_run_noalloc(const void* const* in_slabs, void* const* out_s
       p.out[k] = static_cast<char*>(out_slabs[k]);
     }
     p.S_local = S_local;
+    p.r_stride = 1;
     p.nv = pl.row_bytes / pl.vec_bytes;
     p.srow = pl.row_pitch * elem_bytes / pl.vec_bytes;
     p.w = w;

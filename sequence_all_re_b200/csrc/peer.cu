@@ -311,6 +311,69 @@ static int ua2a_impl_peer_pull(ulysses_a2a_peer* p, void* out_local, int64_t B, 
                     static_cast<cudaStream_t>(stream), pl, 0, -1, p->rank);
 }
 
+static int ua2a_impl_peer_pull_packed(ulysses_a2a_peer* p, void* const* out_local, int ntensors,
+                                      int64_t B, int64_t S_local, int64_t H, int64_t D, int mode,
+                                      size_t window_offset, void* stream) {
+  if (p == nullptr) return ULYSSES_A2A_ERR_INVALID;
+  ulysses_a2a_ctx* ctx = p->ctx;
+  ctx->last_error.clear();
+  if (!p->open) return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_pull_packed: the peer windows are not open");
+  const int w = p->world;
+  const int T = ntensors;
+  if (out_local == nullptr || T < 1 || (int64_t)T * w > ULYSSES_A2A_MAX_W)
+    return fail(ctx, ULYSSES_A2A_ERR_INVALID,
+                "peer_pull_packed: need an output array and 1 <= ntensors, ntensors * world <= 64");
+  if (mode != 0 && mode != 1) return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_pull_packed: mode must be 0 or 1");
+  if (B < 0 || S_local < 0 || H < 0 || D < 0)
+    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_pull_packed: sizes must be >= 0");
+  int rc = check_window_offset(p, window_offset, "peer_pull_packed");
+  if (rc) return rc;
+  int64_t slab = 0;  // one tensor's slab of one rank, either layout
+  if (ua2a::mul_overflows(B, S_local, &slab) || ua2a::mul_overflows(slab, H, &slab) ||
+      ua2a::mul_overflows(slab, D, &slab) || ua2a::mul_overflows(slab, (int64_t)ctx->elem_bytes, &slab) ||
+      slab > (int64_t(1) << 56))
+    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_pull_packed: slab sizes overflow");
+  // Mode 0: every window holds a packed [B, S, T, H, D] slab (rows of T*H*D
+  // elements), tensor t's heads at element t*H*D of each row; this rank's
+  // output slab of tensor t is out[t*w + rank]. Mode 1: every window holds T
+  // dense [B, S*w, H/w, D] slabs, tensor t at byte t*slab, i.e. input slab
+  // t*w + r of the packed launch; this rank's packed output is out[rank].
+  std::vector<const void*> ins(mode == 0 ? w : (size_t)T * w);
+  std::vector<void*> outs(mode == 0 ? (size_t)T * w : w, nullptr);
+  for (int k = 0; k < w; ++k) {
+    const char* base = static_cast<const char*>(p->bases[k]) + window_offset;
+    if (mode == 0)
+      ins[k] = base;
+    else
+      for (int t = 0; t < T; ++t) ins[(size_t)t * w + k] = base + (size_t)t * (size_t)slab;
+  }
+  if (mode == 0)
+    for (int t = 0; t < T; ++t) outs[(size_t)t * w + p->rank] = out_local[t];
+  else
+    outs[p->rank] = out_local[0];
+  std::string err;
+  ulysses_a2a_plan_t pl;
+  rc = ua2a::make_plan(ins.data(), outs.data(), B, S_local, H, D, w, mode, 0, ctx->elem_bytes,
+                       ULYSSES_A2A_PATH_VEC, ctx->tuning, ctx->num_sms, &pl, &err, 0, p->rank, T);
+  if (rc) return fail(ctx, rc, "peer_pull_packed: " + err);
+  if (pl.units == 0) return ULYSSES_A2A_OK;
+  if ((uint64_t)slab * (uint64_t)T > (uint64_t)(p->window_bytes - window_offset))
+    return fail(ctx, ULYSSES_A2A_ERR_INVALID, "peer_pull_packed: the " + std::to_string(T) +
+                                                  " slabs exceed the windows from the offset");
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return fail(ctx, ULYSSES_A2A_ERR_DEVICE, "cannot select the context's device");
+  if (mode == 0) {
+    std::vector<const void*> o(out_local, out_local + T);
+    rc = check_residency(ctx, o.data(), T, slab, "output");
+  } else {
+    const void* o[1] = {out_local[0]};
+    rc = check_residency(ctx, o, 1, slab * T, "output");
+  }
+  if (rc) return rc;
+  return run_device(ctx, ins.data(), outs.data(), B, S_local, H, D, w, mode, 0,
+                    static_cast<cudaStream_t>(stream), pl, 0, -1, p->rank, T);
+}
+
 void* ulysses_a2a_peer_window(const ulysses_a2a_peer* p, int rank) {
   if (p == nullptr || rank < 0 || rank >= p->world) return nullptr;
   return p->bases[rank];
@@ -377,6 +440,13 @@ int ulysses_a2a_peer_pull(ulysses_a2a_peer* p, void* out_local, int64_t B, int64
     return ua2a_impl_peer_pull(p, out_local, B, S_local, H, D, mode, row_pitch, window_offset,
                                stream);
   });
+}
+
+int ulysses_a2a_peer_pull_packed(ulysses_a2a_peer* peer, void* const* out_local, int ntensors,
+                                 int64_t B, int64_t S_local, int64_t H, int64_t D, int mode,
+                                 size_t window_offset, void* stream) {
+  return no_throw([&] { return ua2a_impl_peer_pull_packed(peer, out_local, ntensors, B, S_local, H, D,
+                                                          mode, window_offset, stream); });
 }
 
 int ulysses_a2a_peer_close(ulysses_a2a_peer* p) {

@@ -55,6 +55,11 @@ constexpr int kVecBlock = 256;
 // VEC grid has one CTA per unit, and the hardware hands CTAs to SMs as they
 // free up, so no SM is left with a tail of units.
 constexpr int kVecResidentCtasPerSm = 6;
+// Re-aligning (staged) path: strided-side bytes per work unit, the shared
+// memory one CTA may use, and its threads.
+constexpr int64_t kStageTileTargetBytes = 16 * 1024;
+constexpr int64_t kStageSmemMax = 96 * 1024;
+constexpr int kStageBlock = 256;
 // Unit numbering: 0 = destination rank outermost, 1 = innermost.
 constexpr int kDefaultOrder = 1;
 // Host-buffer entry point: sequence chunks its H2D copies, kernels and D2H
@@ -117,6 +122,41 @@ inline const char* tma_blocker(const void* const* in, void* const* out, int64_t 
   return nullptr;
 }
 
+// Geometry of the re-aligning (staged) path for runs of R bytes, ng head
+// groups per strided row (HDE = ng * R bytes) and S_local rows: the rows per
+// unit (about kStageTileTargetBytes of strided-side bytes, or rows_cap when
+// set), the 16-byte chunks scanned per strided row (Cs) and per gathered range
+// (Cg), and the shared memory of a CTA: ng regions of RS bytes (RS = 16*Cg
+// rounded to an odd number of 16-byte chunks, so that consecutive regions
+// start in different shared-memory banks) and ng 4-byte region offsets.
+// Returns false if not even one row fits kStageSmemMax.
+struct StageGeometry {
+  int64_t rows = 0, tiles = 0, Cs = 0, Cg = 0, RS = 0, smem_bytes = 0;
+};
+
+inline bool stage_geometry(int64_t R, int64_t ng, int64_t S, int rows_cap, StageGeometry* g) {
+  const int64_t HDE = ng * R;
+  if (R < 1 || ng < 1 || S < 1 || HDE >= (int64_t(1) << 30)) return false;
+  int64_t rows = rows_cap > 0 ? rows_cap : kStageTileTargetBytes / HDE;
+  if (rows < 1) rows = 1;
+  if (rows > S) rows = S;
+  for (; rows >= 1; rows = rows > 1 ? rows / 2 : 0) {
+    const int64_t Cg = (rows * R + 30) / 16;
+    const int64_t RS = 16 * (Cg % 2 ? Cg : Cg + 1);
+    const int64_t smem = ng * RS + 4 * ng;
+    if (smem <= kStageSmemMax && rows * HDE < (int64_t(1) << 30)) {
+      g->rows = rows;
+      g->tiles = (S + rows - 1) / rows;
+      g->Cs = (HDE + 30) / 16;
+      g->Cg = Cg;
+      g->RS = RS;
+      g->smem_bytes = (smem + 15) / 16 * 16;
+      return true;
+    }
+  }
+  return false;
+}
+
 // Public tuning struct -> internal knobs, with range checks (NULL = defaults).
 inline bool tuning_from(const ulysses_a2a_tuning_t* t, Tuning* out, std::string* err) {
   *out = Tuning{};
@@ -147,9 +187,10 @@ inline bool tuning_from(const ulysses_a2a_tuning_t* t, Tuning* out, std::string*
 // Validate and plan one call. Returns a ULYSSES_A2A_* status.
 // row_pitch: elements between consecutive (b, s) rows of the [B, S, H, D]
 // side (0 = dense, H*D); that side's planes are S*row_pitch elements apart.
-// only_out >= 0: the call writes output slab only_out alone (VEC path); the
-// other out[] entries are neither checked nor used, and units counts that
-// slab's blocks only.
+// only_out >= 0: the call writes the output slab(s) of rank only_out alone
+// (VEC path): slab only_out, or with ntensors = T > 1 in mode 0 the T slabs
+// t*w + only_out; the other out[] entries are neither checked nor used, and
+// units counts those slabs' blocks only.
 // ntensors = T > 1: T tensors packed along the head dimension of the
 // [B, S, H, D] side ([B, S, T, H, D], rows of T*H*D elements), re-laid out in
 // one launch (VEC path). That side then has w slabs and the other T*w, tensor-
@@ -178,7 +219,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     set_err(err, "one-output plan: slab %lld of %lld, VEC path required", only_out, w);
     return ULYSSES_A2A_ERR_INVALID;
   }
-  if (ntensors < 1 || (int64_t)ntensors * w > ULYSSES_A2A_MAX_W || (ntensors > 1 && only_out >= 0)) {
+  if (ntensors < 1 || (int64_t)ntensors * w > ULYSSES_A2A_MAX_W) {
     set_err(err, "ntensors=%lld: need 1 <= ntensors and ntensors*w <= %lld", ntensors,
             ULYSSES_A2A_MAX_W);
     return ULYSSES_A2A_ERR_INVALID;
@@ -196,7 +237,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
   if (B == 0 || S == 0 || H == 0 || D == 0) {
     // an empty re-layout: nothing to read or write, nothing to launch (slab
     // pointers may be NULL)
-    if (forced_path < ULYSSES_A2A_PATH_AUTO || forced_path > ULYSSES_A2A_PATH_VEC) {
+    if (forced_path < ULYSSES_A2A_PATH_AUTO || forced_path > ULYSSES_A2A_PATH_STAGED) {
       set_err(err, "unknown path %lld", forced_path);
       return ULYSSES_A2A_ERR_INVALID;
     }
@@ -204,7 +245,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     p->row_pitch = row_pitch > 0 ? row_pitch : (int64_t)ntensors * H * D;
     return ULYSSES_A2A_OK;
   }
-  if (forced_path < ULYSSES_A2A_PATH_AUTO || forced_path > ULYSSES_A2A_PATH_VEC) {
+  if (forced_path < ULYSSES_A2A_PATH_AUTO || forced_path > ULYSSES_A2A_PATH_STAGED) {
     set_err(err, "unknown path %lld", forced_path);
     return ULYSSES_A2A_ERR_INVALID;
   }
@@ -237,7 +278,10 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
   // slab counts: w on the [B, S, (T,) H, D] side, T*w on the gathered side
   const int nin = mode == 0 ? w : w * ntensors;
   const int nout = mode == 0 ? w * ntensors : w;
-  auto used_out = [&](int k) { return only_out < 0 || k == only_out; };
+  // outputs this call writes: all, or rank only_out's (one per tensor in mode 0)
+  auto used_out = [&](int k) {
+    return only_out < 0 || (mode == 0 ? k % w == only_out : k == only_out);
+  };
   for (int k = 0; k < nin; ++k) {
     if (in[k] == nullptr) {
       set_err(err, "input slab pointer %lld is NULL", k);
@@ -287,8 +331,8 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
       return ULYSSES_A2A_ERR_UNSUPPORTED;
     }
     path = ULYSSES_A2A_PATH_TMA;
-  } else if (forced_path == ULYSSES_A2A_PATH_VEC) {
-    path = ULYSSES_A2A_PATH_VEC;
+  } else if (forced_path == ULYSSES_A2A_PATH_VEC || forced_path == ULYSSES_A2A_PATH_STAGED) {
+    path = ULYSSES_A2A_PATH_VEC;  // the staged path is decided with the vector width below
   } else {
     path = blocker ? ULYSSES_A2A_PATH_VEC : ULYSSES_A2A_PATH_TMA;
   }
@@ -305,7 +349,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
 
   const int64_t T = (S + rows - 1) / rows;  // ceil-div: the ragged last tile is a unit too
   const int64_t nb = chunked ? 1 : B;
-  const int64_t blocks_wide = only_out >= 0 ? (int64_t)w : (int64_t)w * w * ntensors;
+  const int64_t blocks_wide = (only_out >= 0 ? (int64_t)w : (int64_t)w * w) * ntensors;
   int64_t units;
   if (mul_overflows(blocks_wide, nb, &tmp) || mul_overflows(tmp, T, &units)) {
     set_err(err, "unit count overflows");
@@ -318,7 +362,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
   p->tiles_per_block = T;
   p->tail_rows = S % rows;
   p->units = units;
-  p->payload_bytes = only_out >= 0 ? slab_bytes : payload;
+  p->payload_bytes = only_out >= 0 ? slab_bytes * ntensors : payload;
   p->launches = chunked ? (int32_t)(B > INT32_MAX ? INT32_MAX : B) : 1;
   p->row_pitch = pitch;
   p->order = tune.order >= 0 ? (tune.order ? 1 : 0) : kDefaultOrder;
@@ -425,6 +469,35 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     p->smem_bytes = 0;
     p->block = kVecBlock;
     p->grid = (int32_t)(units < g ? units : g);
+
+    // The re-aligning path takes what the vector path could only move in
+    // pieces narrower than 16 bytes (or what it is forced onto), except
+    // one-output launches.
+    const bool forced_stage = forced_path == ULYSSES_A2A_PATH_STAGED;
+    if (forced_stage || (forced_path == ULYSSES_A2A_PATH_AUTO && v < 16 && only_out < 0)) {
+      StageGeometry sg;
+      if (stage_geometry(row_bytes, (int64_t)w * ntensors, S, tune.rows_per_tile, &sg)) {
+        const int64_t nbl = chunked ? 1 : B;
+        int64_t su;
+        if (mul_overflows((int64_t)w * nbl, sg.tiles, &su) || su >= (int64_t(1) << 31)) {
+          set_err(err, "%lld staged work units exceed the 2^31 limit", su);
+          return ULYSSES_A2A_ERR_UNSUPPORTED;
+        }
+        const int64_t sgrid = tune.ctas_per_sm > 0 ? (int64_t)num_sms * tune.ctas_per_sm : su;
+        p->path = ULYSSES_A2A_PATH_STAGED;
+        p->rows_per_tile = sg.rows;
+        p->tiles_per_block = sg.tiles;
+        p->tail_rows = S % sg.rows;
+        p->units = su;
+        p->smem_bytes = sg.smem_bytes;
+        p->block = kStageBlock;
+        p->grid = (int32_t)(su < sgrid ? su : sgrid);
+      } else if (forced_stage) {
+        set_err(err, "staged path forced but one row of %lld bytes does not fit its shared memory",
+                row_bytes * w * ntensors);
+        return ULYSSES_A2A_ERR_UNSUPPORTED;
+      }
+    }
   }
   return ULYSSES_A2A_OK;
 }

@@ -28,6 +28,7 @@
 
 #include "internal.h"
 
+using ua2a::StageParams;
 using ua2a::TmaParams;
 using ua2a::VecParams;
 
@@ -232,6 +233,69 @@ cudaError_t launch_vec(const VecParams& p, int vec_bytes, int mode, int grid, in
   }
 }
 
+template <int G>
+cudaError_t launch_stage_t(const StageParams& p, int mode, int grid, int block, size_t smem,
+                           cudaStream_t st) {
+  return mode == 0 ? launch_pdl(ua2a::ua2a_stage_kernel<G, 0>, grid, block, smem, st, p)
+                   : launch_pdl(ua2a::ua2a_stage_kernel<G, 1>, grid, block, smem, st, p);
+}
+
+cudaError_t launch_stage(const StageParams& p, int piece_bytes, int mode, int grid, int block,
+                         size_t smem, cudaStream_t st) {
+  switch (piece_bytes) {
+    case 16: return launch_stage_t<16>(p, mode, grid, block, smem, st);
+    case 8: return launch_stage_t<8>(p, mode, grid, block, smem, st);
+    case 4: return launch_stage_t<4>(p, mode, grid, block, smem, st);
+    case 2: return launch_stage_t<2>(p, mode, grid, block, smem, st);
+    default: return launch_stage_t<1>(p, mode, grid, block, smem, st);
+  }
+}
+
+template <int G>
+cudaError_t stage_allow_t() {
+  cudaError_t e = cudaFuncSetAttribute(ua2a::ua2a_stage_kernel<G, 0>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)ua2a::kStageSmemMax);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(ua2a::ua2a_stage_kernel<G, 1>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ua2a::kStageSmemMax);
+  return e;
+}
+
+cudaError_t stage_allow_max_smem() {
+  cudaError_t e = stage_allow_t<16>();
+  if (e == cudaSuccess) e = stage_allow_t<8>();
+  if (e == cudaSuccess) e = stage_allow_t<4>();
+  if (e == cudaSuccess) e = stage_allow_t<2>();
+  if (e == cudaSuccess) e = stage_allow_t<1>();
+  return e;
+}
+
+StageParams stage_params(int64_t S, int w, int ntensors, int E, const ulysses_a2a_plan_t& pl,
+                         int64_t nt, int64_t units) {
+  StageParams p{};
+  p.S_local = S;
+  p.P = pl.row_pitch * E;
+  p.R = (int32_t)pl.row_bytes;
+  p.ng = w * ntensors;
+  p.HDE = (int32_t)(pl.row_bytes * p.ng);
+  p.w = w;
+  p.rows_per_tile = (int32_t)pl.rows_per_tile;
+  p.units = (uint32_t)units;
+  StageGeometry sg;
+  stage_geometry(pl.row_bytes, p.ng, S, (int)pl.rows_per_tile, &sg);
+  p.RS = (int32_t)sg.RS;
+  p.Cs = (int32_t)sg.Cs;
+  p.Cg = (int32_t)sg.Cg;
+  p.div_T = ua2a::FastDiv((uint32_t)nt);
+  p.div_w = ua2a::FastDiv((uint32_t)w);
+  p.div_R = ua2a::FastDiv((uint32_t)p.R);
+  p.div_ng = ua2a::FastDiv((uint32_t)p.ng);
+  p.div_Cs = ua2a::FastDiv((uint32_t)p.Cs);
+  p.div_Cg = ua2a::FastDiv((uint32_t)p.Cg);
+  return p;
+}
+
 // run_device: see internal.h.
 int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, int64_t B, int64_t S,
                int64_t H, int64_t D, int w, int mode, int chunked, cudaStream_t st,
@@ -240,17 +304,43 @@ int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, in
   const int64_t nb = chunked ? 1 : B;
   const int launches = chunked ? (int)B : 1;
   const int64_t nt = ntiles < 0 ? pl.tiles_per_block : ntiles;
-  const int nr = (only_out >= 0 && mode == 0) ? 1 : w * ntensors;
+  // a one-output launch covers rank only_out's head group of each tensor
+  // (mode 0) or its sequence block j (mode 1)
+  const int nr = (only_out >= 0 && mode == 0) ? ntensors : w * ntensors;
   const int nj = (only_out >= 0 && mode == 1) ? 1 : w;
-  const int64_t units = (int64_t)nr * nb * nj * nt;
-  if ((only_out >= 0 || ntensors > 1) && pl.path != ULYSSES_A2A_PATH_VEC)
-    return fail(ctx, ULYSSES_A2A_ERR_UNSUPPORTED, "one-output and packed launches use the VEC path");
+  const bool staged = pl.path == ULYSSES_A2A_PATH_STAGED;
+  // staged units cover every head group of their rows
+  const int64_t units = staged ? (int64_t)nb * nj * nt : (int64_t)nr * nb * nj * nt;
+  if (only_out >= 0 && pl.path != ULYSSES_A2A_PATH_VEC)
+    return fail(ctx, ULYSSES_A2A_ERR_UNSUPPORTED, "one-output launches use the VEC path");
+  if (ntensors > 1 && pl.path == ULYSSES_A2A_PATH_TMA)
+    return fail(ctx, ULYSSES_A2A_ERR_UNSUPPORTED, "packed launches use the VEC or staged path");
   int grid = pl.grid;
   if (nt != pl.tiles_per_block) {
     if (pl.path == ULYSSES_A2A_PATH_TMA && pl.chunk_units > 0)
       grid = (int)((units + pl.chunk_units - 1) / pl.chunk_units);
     else if (units < grid)
       grid = (int)units;
+  }
+  if (staged) {
+    StageParams p = stage_params(S, w, ntensors, ctx->elem_bytes, pl, nt, units);
+    const int nin = mode == 0 ? w : w * ntensors;
+    const int nout = mode == 0 ? w * ntensors : w;
+    for (int k = 0; k < nin; ++k) p.in[k] = static_cast<const char*>(in[k]);
+    for (int k = 0; k < nout; ++k) p.out[k] = static_cast<char*>(out[k]);
+    p.tile0 = (uint32_t)tile0;
+    if (!ctx->stage_smem_set) {
+      cudaError_t e = stage_allow_max_smem();
+      if (e != cudaSuccess) return cuda_fail(ctx, "cudaFuncSetAttribute (staged kernels)", e);
+      ctx->stage_smem_set = true;
+    }
+    for (int l = 0; l < launches; ++l) {
+      p.b0 = chunked ? l : 0;
+      cudaError_t e = launch_stage(p, pl.vec_bytes, mode, grid, pl.block, (size_t)pl.smem_bytes, st);
+      if (e != cudaSuccess) return cuda_fail(ctx, "staged kernel launch", e);
+      ctx->launches++;
+    }
+    return ULYSSES_A2A_OK;
   }
   if (pl.path == ULYSSES_A2A_PATH_TMA) {
     TmaParams* cached = nullptr;
@@ -298,6 +388,7 @@ int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, in
   p.order = pl.order;
   p.tile0 = (uint32_t)tile0;
   p.r0 = (only_out >= 0 && mode == 0) ? (uint32_t)only_out : 0u;
+  p.r_stride = (only_out >= 0 && mode == 0) ? (uint32_t)w : 1u;
   p.j0 = (only_out >= 0 && mode == 1) ? (uint32_t)only_out : 0u;
   p.div_T = ua2a::FastDiv((uint32_t)nt);
   p.div_nr = ua2a::FastDiv((uint32_t)nr);
@@ -333,6 +424,7 @@ bool env_config(int* path, int* ctas) {
     if (s == "auto" || s.empty()) *path = ULYSSES_A2A_PATH_AUTO;
     else if (s == "tma") *path = ULYSSES_A2A_PATH_TMA;
     else if (s == "vec") *path = ULYSSES_A2A_PATH_VEC;
+    else if (s == "staged") *path = ULYSSES_A2A_PATH_STAGED;
     else return false;
   }
   if (const char* v = std::getenv("ULYSSES_A2A_CTAS_PER_SM")) {
@@ -730,7 +822,7 @@ static int ua2a_impl_selftest_wait_timeout(ulysses_a2a_ctx* ctx, uint32_t limit_
 
 static int ua2a_impl_set_path(ulysses_a2a_ctx* ctx, int path) {
   if (ctx == nullptr) return ULYSSES_A2A_ERR_INVALID;
-  if (path < ULYSSES_A2A_PATH_AUTO || path > ULYSSES_A2A_PATH_VEC)
+  if (path < ULYSSES_A2A_PATH_AUTO || path > ULYSSES_A2A_PATH_STAGED)
     return fail(ctx, ULYSSES_A2A_ERR_INVALID, "unknown path");
   ctx->forced_path = path;
   return ULYSSES_A2A_OK;

@@ -85,6 +85,13 @@ class NativePeer:
         self._check(_lib.ulysses_a2a_peer_pull(self._peer, out.data_ptr(), B, S, H, D, mode,
                                                row_pitch, stream.cuda_stream, window_offset))
 
+    def pull_packed(self, outs, T, B, S, H, D, mode, stream, window_offset=0) -> None:
+        """One launch for T head-packed tensors: ``outs`` is T tensors (mode 0)
+        or the one packed [B, S, T, H, D] output (mode 1)."""
+        ptrs = [t.data_ptr() for t in outs] if mode == 0 else [outs.data_ptr()]
+        self._check(_lib.ulysses_a2a_peer_pull_packed(self._peer, ptrs, T, B, S, H, D, mode,
+                                                      stream.cuda_stream, window_offset))
+
     def window(self, rank: int) -> int:
         return _lib.ulysses_a2a_peer_window(self._peer, rank) if self._peer is not None else 0
 
@@ -311,7 +318,8 @@ class PeerExchange:
         the packed [B, S_local, T, H, D] slab (``out`` may be given). The T
         slabs share the window at consecutive offsets, and each is pulled
         into its slot of the packed output.
-        Same bytes as T calls of ``all_to_all_4d``; 2 barriers instead of 2T.
+        Same bytes as T calls of ``all_to_all_4d``; 2 barriers instead of 2T,
+        and one pull launch for all T tensors.
         """
         if self.disabled_reason is not None:
             raise RuntimeError(f"peer exchange disabled: {self.disabled_reason}")
@@ -360,13 +368,9 @@ class PeerExchange:
             for t in range(T):
                 self.native.publish(srcs[t], B, S, H, D, 1, 0, stream, window_offset=t * slab)
         self._barrier(stream)        # every window holds its slabs
-        for t in range(T):
-            if mode == 0:
-                self.native.pull(outs[t], B, S, H, D, 0, T * H * D, stream,
-                                 window_offset=t * H * D * E)
-            else:
-                self.native.pull(outs[:, :, t], B, S, H, D, 1, T * H * D, stream,
-                                 window_offset=t * slab)
+        if mode == 1 and not outs.is_contiguous():
+            raise ValueError("the packed output must be contiguous")
+        self.native.pull_packed(outs, T, B, S, H, D, mode, stream)
         return outs
 
     def all_to_all_4d(self, x: torch.Tensor, mode: int, chunked: bool = False, out=None,

@@ -9,7 +9,7 @@ import pytest
 
 from sequence_all_re_b200 import _lib
 from sequence_all_re_b200._lib import (ERR_INVALID, ERR_OVERLAP, ERR_UNSUPPORTED, OK, PATH_AUTO,
-                                       PATH_TMA, PATH_VEC, ulysses_a2a_plan)
+                                       PATH_STAGED, PATH_TMA, PATH_VEC, ulysses_a2a_plan)
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "ulysses_a2a.h")
@@ -39,6 +39,7 @@ def test_header_constants_match_the_binding():
                "ERR_UNSUPPORTED": _lib.ERR_UNSUPPORTED, "ERR_NOMEM": _lib.ERR_NOMEM,
                "ERR_TIMEOUT": _lib.ERR_TIMEOUT, "ERR_INTERNAL": _lib.ERR_INTERNAL,
                "PATH_AUTO": _lib.PATH_AUTO, "PATH_TMA": _lib.PATH_TMA, "PATH_VEC": _lib.PATH_VEC,
+               "PATH_STAGED": _lib.PATH_STAGED,
                "MAX_W": _lib.MAX_W, "MAX_W_TMA": _lib.MAX_W_TMA,
                "PEER_HANDLE_BYTES": _lib.PEER_HANDLE_BYTES}
     for name, value in binding.items():
@@ -155,11 +156,39 @@ def test_rows_never_exceed_sequence():
 
 # ---- path selection --------------------------------------------------------
 
-def test_vec_when_feature_bytes_not_16_aligned():
+def test_runs_off_16_bytes_take_the_staged_path():
+    # AUTO re-aligns in shared memory (16-byte global accesses, pieces of the
+    # width the run allows); the vector path, when forced, uses that width
     rc, p, _ = plan(2, 1, 16, 4, 3)             # D*E = 6 bytes
-    assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 4   # run = 2*3*2 = 12 B
+    assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 4   # run = 2*3*2 = 12 B
+    rc, p, _ = plan(2, 1, 16, 4, 3, forced_path=PATH_VEC)
+    assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 4
     rc, p, _ = plan(2, 1, 16, 2, 5, E=1)        # run = 5 B
+    assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 1
+    rc, p, _ = plan(2, 1, 16, 2, 5, E=1, forced_path=PATH_VEC)
     assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 1
+
+
+def test_staged_geometry():
+    # 200-byte runs, 8 head groups of 1600-byte rows: units of 10 rows (16 KB),
+    # one per (b, j, tile) covering every head group
+    rc, p, _ = plan(8, 2, 4725, 8, 100)
+    assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 8
+    assert p.rows_per_tile == 16 * 1024 // 1600 == 10 and p.tail_rows == 4725 % 10
+    assert p.units == 8 * 2 * p.tiles_per_block and p.grid == p.units and p.block == 256
+    cg = (10 * 200 + 30) // 16
+    assert p.smem_bytes == (8 * 16 * (cg if cg % 2 else cg + 1) + 4 * 8 + 15) // 16 * 16
+    # chunked: one plane per launch
+    rc, p, _ = plan(8, 2, 4725, 8, 100, chunked=1)
+    assert rc == OK and p.units == 8 * p.tiles_per_block and p.launches == 2
+    # forced on an aligned shape, the pieces are 16 bytes
+    rc, p, _ = plan(4, 1, 8192, 24, 128, forced_path=PATH_STAGED)
+    assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 16
+    # a row too long for the shared memory stays on the vector path
+    rc, p, _ = plan(4, 1, 16, 4 * 8, 512, E=8)  # 8 groups x 32 KB runs (E = 8, D = 512)
+    assert rc == OK and p.path == PATH_VEC
+    rc, _, msg = plan(4, 1, 16, 4 * 8, 512, E=8, forced_path=PATH_STAGED)
+    assert rc == ERR_UNSUPPORTED and "shared memory" in msg
 
 
 def test_vec_when_misaligned_pointer():
@@ -167,6 +196,8 @@ def test_vec_when_misaligned_pointer():
     ins, outs = fake_slabs(w, B * S * H * D * E)
     outs[1] += 8
     rc, p, _ = ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E)
+    assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 8
+    rc, p, _ = ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E, forced_path=PATH_VEC)
     assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 8
     rc, p, msg = ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E, forced_path=PATH_TMA)
     assert rc == ERR_UNSUPPORTED and "aligned" in msg
@@ -400,6 +431,8 @@ def test_pitch_smaller_than_a_row_is_rejected():
 def test_pitch_alignment_selects_the_vector_width():
     # pitch * E = (512 + 4) * 2 bytes: 8-byte aligned rows only
     rc, p, _ = plan_ex(4, 1, 64, 8, 64, 8 * 64 + 4)
+    assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 8
+    rc, p, _ = plan_ex(4, 1, 64, 8, 64, 8 * 64 + 4, forced_path=PATH_VEC)
     assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 8
     rc, _, msg = plan_ex(4, 1, 64, 8, 64, 8 * 64 + 4, forced_path=PATH_TMA)
     assert rc == ERR_UNSUPPORTED and "pitch" in msg
@@ -531,11 +564,20 @@ from hypothesis import given, settings  # noqa: E402
 from hypothesis import strategies as st  # noqa: E402
 
 
+def _one_row_fits_stage(R, ng):
+    """Whether one strided row fits the staged path's 96 KB of shared memory:
+    ng regions of (R + 30) // 16 chunks, rounded to an odd count, plus ng
+    4-byte region offsets."""
+    cg = (R + 30) // 16
+    return ng * 16 * (cg if cg % 2 else cg + 1) + 4 * ng <= 96 * 1024
+
+
 @settings(max_examples=300, deadline=None, derandomize=True, database=None)
 @given(w=st.sampled_from([1, 2, 3, 4, 8, 16]), hw=st.integers(1, 6), B=st.integers(1, 4),
        S=st.integers(1, 5000), D=st.sampled_from([1, 3, 8, 13, 64, 128, 256]),
        E=st.sampled_from([1, 2, 4, 8]), mode=st.sampled_from([0, 1]),
-       chunked=st.sampled_from([0, 1]), path=st.sampled_from([PATH_AUTO, PATH_VEC]),
+       chunked=st.sampled_from([0, 1]),
+       path=st.sampled_from([PATH_AUTO, PATH_VEC, PATH_STAGED]),
        rows=st.sampled_from([0, 0, 1, 7, 64]), ntensors=st.sampled_from([1, 1, 2, 3]))
 def test_planner_invariants(w, hw, B, S, D, E, mode, chunked, path, rows, ntensors):
     H = hw * w
@@ -549,8 +591,27 @@ def test_planner_invariants(w, hw, B, S, D, E, mode, chunked, path, rows, ntenso
     rc, p, msg = _lib.ulysses_a2a_plan_ex(ins, outs, B, S, H, D, w, mode, chunked, E,
                                           forced_path=path, ntensors=ntensors,
                                           rows_per_tile=rows)
+    if path == PATH_STAGED and rc == ERR_UNSUPPORTED:
+        assert "shared memory" in msg       # one strided row does not fit
+        assert not _one_row_fits_stage(hw * D * E, ntensors * w)
+        return
     assert rc == OK, msg
     nb = 1 if chunked else B
+    if p.path == PATH_STAGED:
+        # one unit per (b, j, tile), every head group of its rows; pieces of the
+        # widest width the run and the pitch allow; shared memory within 96 KB
+        assert path in (PATH_AUTO, PATH_STAGED)
+        hde = ntensors * hw * w * D * E
+        assert 1 <= p.rows_per_tile <= S and p.tiles_per_block == -(-S // p.rows_per_tile)
+        assert p.rows_per_tile == 1 or p.rows_per_tile * hde <= 16 * 1024 or rows
+        assert p.units == w * nb * p.tiles_per_block and p.grid == p.units
+        assert p.block == 256 and p.smem_bytes <= 96 * 1024
+        v = p.vec_bytes
+        assert p.row_bytes % v == 0 and (p.row_pitch * E) % v == 0
+        assert v == 16 or (p.row_bytes % (2 * v) or (p.row_pitch * E) % (2 * v))
+        if path == PATH_AUTO:
+            assert v < 16
+        return
     # tiles cover every sequence row exactly once per (r, b, j) block
     assert 1 <= p.rows_per_tile <= min(S, 256)
     assert p.tiles_per_block == -(-S // p.rows_per_tile)
@@ -574,6 +635,8 @@ def test_planner_invariants(w, hw, B, S, D, E, mode, chunked, path, rows, ntenso
         assert p.path == PATH_VEC
         v = p.vec_bytes
         assert v in (1, 2, 4, 8, 16) and p.row_bytes % v == 0 and (p.row_pitch * E) % v == 0
+        # AUTO leaves narrower vectors to the staged path unless a row is too long
+        assert path == PATH_VEC or v == 16 or not _one_row_fits_stage(hw * D * E, ntensors * w)
         # the widest width the run length and the pitch allow (pointers are 4 KiB aligned)
         assert v == 16 or (p.row_bytes % (2 * v) or (p.row_pitch * E) % (2 * v))
         assert p.grid == p.units and p.block == 256

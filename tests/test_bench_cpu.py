@@ -25,7 +25,8 @@ def test_committed_captures_match_the_current_kernels_and_plans():
     for key, entry in traffic.items():
         path, shape = key.split(":")
         w, B, S, H, D = (int(part[1:]) for part in shape.split("_")[:5])
-        p = plan_dict(w, B, S, H, D, _lib.PATH_TMA if path == "tma" else _lib.PATH_VEC)
+        p = plan_dict(w, B, S, H, D, {"tma": _lib.PATH_TMA, "vec": _lib.PATH_VEC,
+                                      "staged": _lib.PATH_STAGED}[path])
         got, why = bench.ncu_traffic(key, p, 0)
         assert why == "ncu", (key, why)
         assert got == entry["dram_bytes_per_launch"]

@@ -27,7 +27,7 @@ MUTATIONS = {
         "char *dst = (char *)out[r] + a * E;"),
     # the head group taken from the strided side follows j instead of r
     "head_group_index": (
-        "int64_t a = at4(b, s, (int64_t)r * Hw + hp, d,",
+        "int64_t a = at4(b, s, r * Hw + hp, d,",
         "int64_t a = at4(b, s, (int64_t)j * Hw + hp, d,"),
     # the gathered sequence block follows r instead of j
     "sequence_block_index": (
@@ -63,7 +63,7 @@ MUTATIONS = {
         "int64_t a = (b * S_local + s) * (H * D)"),
     # pitched side: head group taken from the source rank
     "pitched_head_group": (
-        "+ ((int64_t)r * Hw + hp) * D + d;",
+        "+ (r * Hw + hp) * D + d;",
         "+ ((int64_t)j * Hw + hp) * D + d;"),
     # mode 1 copies the wrong way round (reads the destination layout's offset)
     "mode1_swapped_offsets": (

@@ -11,7 +11,8 @@ import pytest
 import torch
 
 import oracle
-from sequence_all_re_b200 import A2AError, PATH_AUTO, PATH_TMA, PATH_VEC, UlyssesA2A, _lib
+from sequence_all_re_b200 import (A2AError, PATH_AUTO, PATH_STAGED, PATH_TMA, PATH_VEC, UlyssesA2A,
+                                  _lib)
 from synth import (normal_slabs, random_byte_slabs, rank_tagged_slabs, slab_shape, uniform_slabs,
                    unique_slabs)
 
@@ -227,7 +228,10 @@ def test_nan_payloads_and_signed_zero_survive():
 # ---- alignment: misaligned slabs take the narrower vector path --------------
 
 @pytest.mark.parametrize("offset,vec", [(8, 8), (4, 4), (2, 2), (1, 1)])
-def test_misaligned_pointers_select_narrower_vectors(offset, vec):
+def test_misaligned_pointers_select_narrower_pieces(offset, vec):
+    # a base off the 16-byte boundary: AUTO re-aligns through shared memory in
+    # pieces of the alignment the bases allow; the vector path, when forced,
+    # uses vectors of that width
     w, B, S, H, D = 2, 2, 21, 4, 64
     E = 2 if offset % 2 == 0 else 1
     if E == 2:
@@ -238,18 +242,28 @@ def test_misaligned_pointers_select_narrower_vectors(offset, vec):
         xd = [t.cuda() for t in xs]
         g = Guarded(oracle.output_shape(tuple(xs[0].shape), 0, w), xs[0].dtype, w, offset=offset)
         plan = a2a.plan(xd, 0, out=g.slabs)
+        assert plan["path"] == PATH_STAGED and plan["vec_bytes"] == vec
+        a2a.set_path(PATH_VEC)
+        plan = a2a.plan(xd, 0, out=g.slabs)
         assert plan["path"] == PATH_VEC and plan["vec_bytes"] == vec
-    run_case(xs, 0, out_offset=offset)
-    run_case(xs, 0, in_offset=offset)
+    for path in (PATH_AUTO, PATH_VEC):
+        for chunked in (False, True):
+            run_case(xs, 0, out_offset=offset, path=path, chunked=chunked)
+            run_case(xs, 0, in_offset=offset, path=path, chunked=chunked)
+            ys = oracle.ulysses_a2a(xs, 0)
+            run_case(ys, 1, out_offset=offset, path=path, chunked=chunked)
+            run_case(ys, 1, in_offset=offset, path=path, chunked=chunked)
 
 
 def test_shapes_tma_cannot_express_use_vec():
-    # D*E = 6 bytes: rows of 12 bytes, VEC path with 4-byte vectors
+    # D*E = 6 bytes: rows of 12 bytes; AUTO re-aligns them (staged path, 4-byte
+    # pieces), and the VEC path with 4-byte vectors gives the same bytes
     w, B, S, H, D = 2, 2, 17, 4, 3
     for mode in (0, 1):
         xs = normal_slabs(slab_shape(mode, w, B, S, H, D), w, "bf16", seed0=1)
-        run_case(xs, mode)
-        run_case(xs, mode, chunked=True)
+        for path in (PATH_AUTO, PATH_VEC):
+            run_case(xs, mode, path=path)
+            run_case(xs, mode, chunked=True, path=path)
     # w = 16 exceeds the TMA descriptor table
     w, B, S, H, D = 16, 1, 9, 16, 64
     xs = normal_slabs((B, S, H, D), w, "bf16", seed0=2)
@@ -542,18 +556,22 @@ def test_mode1_writes_into_packed_slots(path):
                 assert torch.equal(bits(packed[j][:, :, c].cpu().contiguous()), bits(want[j]))
 
 
-def test_odd_row_pitch_uses_narrower_vectors():
-    # rows of H*D + 4 bf16 elements: 8-byte aligned only, so the VEC path with
-    # 8-byte vectors; the 4 trailing elements of every row stay untouched
+@pytest.mark.parametrize("path", [PATH_AUTO, PATH_VEC], ids=["auto", "vec"])
+def test_odd_row_pitch_uses_narrower_pieces(path):
+    # rows of H*D + 4 bf16 elements: 8-byte aligned only, so 8-byte pieces
+    # (staged, AUTO) or 8-byte vectors (VEC); the 4 trailing elements of every
+    # row stay untouched
     w, B, S, H, D = 2, 2, 19, 4, 32
     pitch = H * D + 4
     bufs_cpu = normal_slabs((B * S * pitch,), w, "bf16", seed0=720)
     want = oracle.ulysses_a2a_pitched(bufs_cpu, 0, w, B, S, H, D, pitch)
     with UlyssesA2A(0, 2) as a2a:
+        a2a.set_path(path)
         bufs = [t.cuda() for t in bufs_cpu]
         views = [t.as_strided((B, S, H, D), (S * pitch, pitch, D, 1)) for t in bufs]
         p = a2a.plan(views, 0)
-        assert p["path"] == PATH_VEC and p["vec_bytes"] == 8 and p["row_pitch"] == pitch
+        assert p["path"] == (PATH_STAGED if path == PATH_AUTO else PATH_VEC)
+        assert p["vec_bytes"] == 8 and p["row_pitch"] == pitch
         out = a2a.run(views, 0)
         for r in range(w):
             assert torch.equal(bits(out[r].cpu()).reshape(-1), bits(want[r]))
@@ -653,7 +671,9 @@ def test_randomized_shapes_layouts_and_knobs():
                 knobs = dict(rows_per_tile=rng.randint(0, 9), stages=rng.choice([0, 2, 3, 4, 8, 12]),
                              chunk_units=rng.choice([-1, 0, 1, 3, 7]), order=rng.choice([-1, 0, 1]),
                              producers=rng.choice([0, 1, 2, 3, 4, 8]))
-            path = rng.choice([PATH_AUTO, PATH_AUTO, PATH_VEC])
+            path = rng.choice([PATH_AUTO, PATH_AUTO, PATH_VEC, PATH_STAGED])
+            if path == PATH_STAGED and H * D * E > 90 * 1024:
+                path = PATH_AUTO            # one row would not fit the staged path's shared memory
             a2a = ctxs[E]
             a2a.set_path(path)
             a2a.set_tuning(**knobs)

@@ -108,6 +108,25 @@ class ShmNative:
                 out[:, :, r * Hw:(r + 1) * Hw] = win[:, k * S:(k + 1) * S]
         self.log.append("pull")
 
+    def pull_packed(self, outs, T, B, S, H, D, mode, stream, window_offset=0):
+        """The T tensors of a head-packed exchange at once (one native launch)."""
+        time.sleep(self.pull_delay)
+        w, k = self.world, self.rank
+        Hw = H // w
+        slab_bytes = B * S * H * D * self.elem_bytes
+        if mode == 0:
+            for t in range(T):
+                o = outs[t].view(B, w, S, Hw, D)
+                for j in range(w):
+                    win = self._win(j, o.dtype, (B, S, T, H, D), window_offset)
+                    o[:, j] = win[:, :, t, k * Hw:(k + 1) * Hw]
+        else:
+            for t in range(T):
+                for r in range(w):
+                    win = self._win(r, outs.dtype, (B, S * w, Hw, D), window_offset + t * slab_bytes)
+                    outs[:, :, t, r * Hw:(r + 1) * Hw] = win[:, k * S:(k + 1) * S]
+        self.log.append("pull")
+
     def unmap(self):
         for shm in self.peers.values():
             shm.close()
@@ -205,8 +224,8 @@ def _worker(rank, world, port, scenario, q):
                                          oracle.ulysses_a2a(gys, 1)[rank].view(torch.int16)))
             rep["closed"] = ex.close()
         elif scenario == "packed":
-            # q, k, v packed per rank: one publish and T pulls in mode 0; T publishes
-            # at window offsets and T pulls into the packed slots in mode 1
+            # q, k, v packed per rank: one publish and one pull in mode 0; T
+            # publishes at window offsets and one pull into the packed slots in mode 1
             native = ShmNative(rank, publish_delay=0.05 if rank == 1 else 0.0,
                                pull_delay=0.2 if rank == 1 else 0.0)
             ex = PeerExchange(native=native, elem_bytes=2)
@@ -309,13 +328,14 @@ def test_autograd_backward_is_the_inverse_exchange():
         assert rep["closed"] is True
 
 
-def test_packed_exchange_uses_one_barrier_pair():
+def test_packed_exchange_uses_one_barrier_pair_and_one_pull():
     for rep in _run("packed", 500):
         assert rep["errors"] == [], rep
         assert rep["ok"] == [True] * 4, rep
         assert rep["closed"] is True
         ops = [e for e in rep["log"] if isinstance(e, str)]
-        assert ops == ["publish"] + ["pull"] * 3 + ["publish"] * 3 + ["pull"] * 3
+        # one pull (one native launch) for the three tensors in each mode
+        assert ops == ["publish", "pull"] + ["publish"] * 3 + ["pull"]
 
 
 def test_split_teardown_leaks_instead_of_freeing():

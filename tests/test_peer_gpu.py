@@ -355,3 +355,63 @@ def test_packed_exchange_through_window_offsets():
         assert ranks.launches() == n1
     finally:
         ranks.close()
+
+
+def test_packed_exchange_pulls_every_tensor_in_one_launch():
+    """ulysses_a2a_peer_pull_packed: mode 0 pulls rank k's head group of all T
+    tensors from the packed windows in one launch; mode 1 pulls the T gathered
+    slabs (at window offsets t*slab) into rank k's packed slab in one launch.
+    Same bytes as T pitched oracle calls; ragged S_local and odd D (narrow
+    vectors) included."""
+    E = 2
+    for (T, w, B, S, H, D) in ((3, 4, 2, 37, 8, 64), (2, 2, 1, 19, 4, 13), (3, 8, 1, 11, 40, 128)):
+        slab = B * S * H * D * E
+        packed_cpu = normal_slabs((B, S, T, H, D), w, "bf16", seed0=890 + T + w)
+        flat = [t.reshape(-1) for t in packed_cpu]
+        ranks = LocalRanks(w, E, T * slab).open()
+        try:
+            stream = torch.cuda.current_stream().cuda_stream
+            packed = [t.cuda() for t in packed_cpu]
+            for k in range(w):
+                assert _lib.ulysses_a2a_peer_publish(ranks.peers[k], packed[k].data_ptr(), B, S,
+                                                     T * H, D, 0, 0, stream) == _lib.OK
+            outs = [[torch.full((B, S * w, H // w, D), -1, dtype=torch.int16, device="cuda")
+                     .view(torch.bfloat16) for _ in range(T)] for _ in range(w)]
+            n0 = ranks.launches()
+            for k in range(w):
+                rc = _lib.ulysses_a2a_peer_pull_packed(ranks.peers[k],
+                                                       [o.data_ptr() for o in outs[k]], T, B, S,
+                                                       H, D, 0, stream)
+                assert rc == _lib.OK, ranks.ctxs[k].last_error()
+            torch.cuda.synchronize()
+            assert ranks.launches() - n0 == w            # one launch per rank for all T
+            for t in range(T):
+                want = oracle.ulysses_a2a_pitched(flat, 0, w, B, S, H, D, T * H * D,
+                                                  offset=t * H * D)
+                for k in range(w):
+                    assert torch.equal(bits(outs[k][t].cpu()).reshape(-1), bits(want[k])), (t, k)
+            for k in range(w):
+                for t in range(T):
+                    assert _lib.ulysses_a2a_peer_publish(ranks.peers[k], outs[k][t].data_ptr(), B,
+                                                         S, H, D, 1, 0, stream,
+                                                         window_offset=t * slab) == _lib.OK
+            back = [torch.full((B, S, T, H, D), -1, dtype=torch.int16, device="cuda")
+                    .view(torch.bfloat16) for _ in range(w)]
+            n1 = ranks.launches()
+            for k in range(w):
+                rc = _lib.ulysses_a2a_peer_pull_packed(ranks.peers[k], [back[k].data_ptr()], T, B,
+                                                       S, H, D, 1, stream)
+                assert rc == _lib.OK, ranks.ctxs[k].last_error()
+            torch.cuda.synchronize()
+            assert ranks.launches() - n1 == w
+            for k in range(w):
+                assert torch.equal(bits(back[k].cpu()), bits(packed_cpu[k])), k
+            # too many tensors for the windows, or T * w above the limit: rejected, nothing launched
+            n2 = ranks.launches()
+            assert _lib.ulysses_a2a_peer_pull_packed(ranks.peers[0], [back[0].data_ptr()], T + 1, B,
+                                                     S, H, D, 1, stream) == _lib.ERR_INVALID
+            assert _lib.ulysses_a2a_peer_pull_packed(ranks.peers[0], [back[0].data_ptr()], 65, B,
+                                                     S, H, D, 1, stream) == _lib.ERR_INVALID
+            assert ranks.launches() == n2
+        finally:
+            ranks.close()
