@@ -51,6 +51,8 @@ Other modes, each printing its own line:
   --packed         q, k, v in one head-packed launch vs three per-tensor launches;
   --peer-one-gpu   the cross-GPU exchange's publish and pull kernels, with the
                    ranks as contexts on one GPU;
+  --tuning-sweep   the schedule knobs one at a time (the measurements behind the
+                   default schedule);
   --exchange X     the Ulysses all-to-all across the GPUs of a torchrun job (one
                    rank slab per GPU): X = nccl (a library all-to-all baseline)
                    or peer (PeerExchange).
@@ -573,11 +575,14 @@ def cpu_oracle_baseline(w, B, S, H, D, budget_s=12.0, E=2):
                               "sample": res["single"]["sample"]}}
 
 
-def exchange_arms(dist, device, rank, world, steps, warmup, wl):
+def exchange_arms(dist, device, rank, world, steps, warmup, wl, native=None):
     """The Ulysses all-to-all across the job's GPUs (w = world, one rank slab of
     the workload's per-rank shape per GPU), a step being mode 0 then mode 1:
     this library's PeerExchange and a library all-to-all (NCCL) baseline. Every
-    rank takes the same steps in the same order; times are the max over ranks."""
+    rank takes the same steps in the same order; times are the max over ranks,
+    from CUDA events on the launching stream (host timing between barriers when
+    the group runs on CPU tensors, as the tests do; `native` then stands in for
+    the peer object)."""
     from sequence_all_re_b200.peer import PeerExchange
 
     B, S, H, D = (wl[k] for k in ("B", "S_local", "H", "D"))
@@ -585,38 +590,48 @@ def exchange_arms(dist, device, rank, world, steps, warmup, wl):
         return {"skipped": f"H={H} is not divisible by {world} GPUs"}
     x = make_inputs(1, B, S, H, D, "bf16", device, seed0=1234 + rank)[0]
     slab = B * S * H * D * 2
-    stream = torch.cuda.current_stream(device)
+    cuda = device.type == "cuda"
+    stream = torch.cuda.current_stream(device) if cuda else None
     res = {"workload": f"one rank slab per GPU, w = {world}: B={B} S_local={S} H={H} D={D} bf16",
            "steps": steps}
+
+    def sync():
+        if cuda:
+            torch.cuda.synchronize()
+
+    def clock_ms(fn, n):
+        """ms for n back-to-back calls of fn, the slowest rank's."""
+        dist.barrier()
+        sync()
+        if cuda:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n):
+                fn()
+            e1.record(stream)
+            sync()
+            ms = e0.elapsed_time(e1)
+        else:
+            t0 = time.perf_counter()
+            for _ in range(n):
+                fn()
+            ms = (time.perf_counter() - t0) * 1e3
+        return max_over_ranks(ms, dist, device)
 
     def timed(step):
         for _ in range(warmup):
             z = step()
-        torch.cuda.synchronize()
+        sync()
         if not torch.equal(z, x):
             raise SystemExit("round trip mismatch across GPUs")
-        dist.barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(steps):
-            step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        return max_over_ranks(e0.elapsed_time(e1), dist, device) / steps
+        return clock_ms(step, steps) / steps
 
-    ex = PeerExchange(device=device.index, elem_bytes=2)
+    ex = (PeerExchange(device=device.index, elem_bytes=2) if native is None
+          else PeerExchange(native=native, elem_bytes=2))
     ms = timed(lambda: ex.all_to_all_4d(ex.all_to_all_4d(x, 0), 1))
-    # the barrier alone (a one-element all-reduce on the stream), 4 per step
+    # the barrier alone (on NCCL a one-element all-reduce on the stream), 4 per step
     nb = 50
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(nb):
-        ex._barrier(stream)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    bar_ms = max_over_ranks(e0.elapsed_time(e1), dist, device) / nb
+    bar_ms = clock_ms(lambda: ex._barrier(ex.native.current_stream()), nb) / nb
     ex.shutdown()
     res["peer"] = {"ms_per_step": round(ms, 4), "gbs": round(job_gbs(world, 2 * slab, 1, ms), 1),
                    "barrier_us": round(bar_ms * 1e3, 2), "barriers_per_step": 4,
@@ -624,6 +639,13 @@ def exchange_arms(dist, device, rank, world, steps, warmup, wl):
     ms = timed(lambda: nccl_all_to_all_4d(nccl_all_to_all_4d(x, 0), 1))
     res["nccl"] = {"ms_per_step": round(ms, 4), "gbs": round(job_gbs(world, 2 * slab, 1, ms), 1)}
     return res
+
+
+def exchange_keys(exchange):
+    """The bench line's cross-GPU keys from exchange_arms' result."""
+    return {"exchange_peer_gbs": exchange.get("peer", {}).get("gbs"),
+            "exchange_nccl_gbs": exchange.get("nccl", {}).get("gbs"),
+            "exchange": exchange}
 
 
 def run_ours(args):
@@ -733,12 +755,13 @@ def run_ours(args):
         extras["isolated_call"] = iso
         extras["workloads"] = wls
         # compact bandwidth sweep: 1 MiB, 64 MiB, 512 MiB, 2 GiB
-        sweep = bandwidth_sweep(device, peak, payload_exps=(20, 26, 29, 31), sampler=sampler,
-                                long_payload=512 << 20, long_seconds=1.0)
-        extras["sweep"] = sweep
-        extras["w_sweep_512MiB"] = {
-            f"w{r['w']}": {k: r[k] for k in r if k.startswith("mode") or k == "payload_bytes"}
-            for r in sweep if r["dtype"] == "bf16" and r["payload_bytes"] == 512 << 20}
+        if not args.no_sweep:
+            sweep = bandwidth_sweep(device, peak, payload_exps=(20, 26, 29, 31), sampler=sampler,
+                                    long_payload=512 << 20, long_seconds=1.0)
+            extras["sweep"] = sweep
+            extras["w_sweep_512MiB"] = {
+                f"w{r['w']}": {k: r[k] for k in r if k.startswith("mode") or k == "payload_bytes"}
+                for r in sweep if r["dtype"] == "bf16" and r["payload_bytes"] == 512 << 20}
         extras["vec_shapes"] = vec_shape_block(device, peak, sampler)
 
     # e2e: the same step through the host-buffer entry point (pinned host slabs)
@@ -840,9 +863,7 @@ def run_ours(args):
         "cpu_baseline": cpu,
     }
     if exchange is not None:
-        line["exchange_peer_gbs"] = exchange.get("peer", {}).get("gbs")
-        line["exchange_nccl_gbs"] = exchange.get("nccl", {}).get("gbs")
-        line["exchange"] = exchange
+        line.update(exchange_keys(exchange))
     if full_sweep is not None:
         line["bandwidth_sweep"] = full_sweep
     if rank == 0:
@@ -1148,6 +1169,74 @@ def run_exchange(args):
 
 
 
+# ------------------------------------------------------------ schedule sweep
+TUNING_SWEEP = [
+    # (label, path, knobs): the default schedule, then one knob changed at a time
+    ("default", "auto", {}),
+    ("persistent grid, 4 producers x 4 stages", "tma", dict(chunk_units=0)),
+    ("persistent grid, 1 producer x 4 stages", "tma", dict(chunk_units=0, producers=1, stages=4)),
+    ("persistent grid, 8 producers x 2 stages", "tma", dict(chunk_units=0, producers=8, stages=16)),
+    ("destination rank outermost", "tma", dict(order=0)),
+    ("residency cap 8 CTAs/SM", "tma", dict(ctas_per_sm=8)),
+    ("residency cap 11 CTAs/SM", "tma", dict(ctas_per_sm=11)),
+    ("residency cap 16 CTAs/SM", "tma", dict(ctas_per_sm=16)),
+    ("residency cap 20 CTAs/SM", "tma", dict(ctas_per_sm=20)),
+    ("2 producers per CTA, cap 7", "tma", dict(producers=2, chunk_units=2, ctas_per_sm=7)),
+    ("12 KB tiles (8 rows of 1.5 KB), cap 9", "tma", dict(rows_per_tile=8, ctas_per_sm=9)),
+    ("vector path, 12 KB units", "vec", {}),
+    ("vector path, grid-stride 16 CTAs/SM", "vec", dict(ctas_per_sm=16)),
+    ("vector path, 4 KB units", "vec", dict(rows_per_tile=3)),
+]
+
+
+def run_tuning_sweep(args):
+    """Each schedule of TUNING_SWEEP on w4_S8192_H24_D128 and the headline
+    workload, both modes back to back (>= 0.5 s each): the measurements behind
+    the default schedule, re-run from one command."""
+    from sequence_all_re_b200 import UlyssesA2A
+
+    if args.gpus != 1:
+        raise SystemExit("--tuning-sweep runs on one GPU")
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    peak, peak_src = hbm_peak()
+    sampler = ClockSampler(0).start()
+    stream = torch.cuda.Stream(device)
+    res = {}
+    for name in ("w4_S8192_H24_D128", DEFAULT_WORKLOAD):
+        v = WORKLOADS[name]
+        w, B, S, H, D = (v[k] for k in ("w", "B", "S_local", "H", "D"))
+        P = w * B * S * H * D * 2
+        x = make_inputs(w, B, S, H, D, "bf16", device)
+        y = [torch.empty((B, S * w, H // w, D), dtype=torch.bfloat16, device=device)
+             for _ in range(w)]
+        z = [torch.empty_like(t) for t in x]
+        a2a = UlyssesA2A(0, 2)
+        rows = []
+        for label, path, knobs in TUNING_SWEEP:
+            a2a.set_path({"auto": 0, "tma": 1, "vec": 2}[path])
+            a2a.set_tuning(**knobs)
+            p = a2a.plan(x, 0, out=y)
+            pm = per_mode_block(a2a, x, y, z, P, stream, peak, sampler, 0.5)
+            rows.append({"schedule": label, "knobs": knobs, "path": PATH_NAMES[p["path"]],
+                         "grid": p["grid"], "block": p["block"], "rows_per_tile": p["rows_per_tile"],
+                         "smem_bytes": p["smem_bytes"],
+                         "mode0_frac": pm["mode0"]["frac"], "mode1_frac": pm["mode1"]["frac"],
+                         "sm_mhz": (pm["mode0"]["clocks"] or {}).get("sm_mhz"),
+                         "reasons": (pm["mode0"]["clocks"] or {}).get("reasons")})
+        torch.cuda.synchronize()
+        if not all(torch.equal(z[k], x[k]) for k in range(w)):
+            raise SystemExit(f"{name}: round trip mismatch")
+        res[name] = rows
+        a2a.close()
+        del x, y, z
+        torch.cuda.empty_cache()
+    sampler.stop()
+    print(json.dumps({"metric": "fraction of the measured copy bandwidth per schedule, "
+                                "back to back, 2 x payload per call",
+                      "peak": peak, "peak_source": peak_src, "workloads": res}), flush=True)
+
+
 # ---------------------------------------------------------------- reference arm
 def run_reference(args):
     """The CPU oracle, as it stands, on the host cores: the OpenMP build over
@@ -1242,6 +1331,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true",
                     help="only the headline step (no per-mode, isolated-call, other-workload, "
                          "sweep or vector-shape sections)")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the compact bandwidth sweep of the extra sections")
     ap.add_argument("--no-exchange", action="store_true",
                     help="with N > 1 GPUs, skip the cross-GPU exchange arms")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -1258,6 +1349,9 @@ def main():
     ap.add_argument("--packed", action="store_true",
                     help="time q, k, v in one packed launch against three per-tensor launches "
                          "(prints its own line)")
+    ap.add_argument("--tuning-sweep", action="store_true",
+                    help="time the schedule knobs one at a time on two workloads (prints its "
+                         "own line)")
     ap.add_argument("--peer-one-gpu", action="store_true",
                     help="time the multi-GPU exchange's publish and pull kernels with the w "
                          "ranks as contexts on one GPU (prints its own line)")
@@ -1273,6 +1367,8 @@ def main():
         run_peer_one_gpu(args)
     elif args.packed:
         run_packed(args)
+    elif args.tuning_sweep:
+        run_tuning_sweep(args)
     else:
         run_ours(args)
 

@@ -175,9 +175,14 @@ def test_staged_geometry():
     rc, p, _ = plan(8, 2, 4725, 8, 100)
     assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 8
     assert p.rows_per_tile == 16 * 1024 // 1600 == 10 and p.tail_rows == 4725 % 10
-    assert p.units == 8 * 2 * p.tiles_per_block and p.grid == p.units and p.block == 256
+    # a persistent grid of 4 CTAs per SM (148 SMs), each taking every 592nd unit
+    assert p.units == 8 * 2 * p.tiles_per_block and p.grid == 148 * 4 and p.block == 256
     cg = (10 * 200 + 30) // 16
-    assert p.smem_bytes == (8 * 16 * (cg if cg % 2 else cg + 1) + 4 * 8 + 15) // 16 * 16
+    assert p.smem_bytes == (8 * 16 * (cg if cg % 2 else cg + 1) + 8 * 8 + 15) // 16 * 16
+    # a unit's in-side is held in registers: at most 1024 16-byte chunks per side
+    assert (10 * 1600 + 30) // 16 <= 1024 and 8 * cg <= 1024
+    rc, p, _ = plan(4, 1, 8192, 24, 128, forced_path=PATH_STAGED, rows_per_tile=8)
+    assert rc == OK and p.rows_per_tile == 2        # (2 * 6144 + 30) // 16 = 769 chunks
     # chunked: one plane per launch
     rc, p, _ = plan(8, 2, 4725, 8, 100, chunked=1)
     assert rc == OK and p.units == 8 * p.tiles_per_block and p.launches == 2
@@ -565,11 +570,12 @@ from hypothesis import strategies as st  # noqa: E402
 
 
 def _one_row_fits_stage(R, ng):
-    """Whether one strided row fits the staged path's 96 KB of shared memory:
-    ng regions of (R + 30) // 16 chunks, rounded to an odd count, plus ng
-    4-byte region offsets."""
+    """Whether one strided row fits the staged path: at most 1024 16-byte
+    chunks per side, and 96 KB of shared memory for ng regions of (R + 30) // 16
+    chunks, rounded to an odd count, plus two arrays of ng 4-byte offsets."""
     cg = (R + 30) // 16
-    return ng * 16 * (cg if cg % 2 else cg + 1) + 4 * ng <= 96 * 1024
+    return (ng * 16 * (cg if cg % 2 else cg + 1) + 8 * ng <= 96 * 1024
+            and (ng * R + 30) // 16 <= 1024 and ng * cg <= 1024)
 
 
 @settings(max_examples=300, deadline=None, derandomize=True, database=None)
@@ -604,8 +610,12 @@ def test_planner_invariants(w, hw, B, S, D, E, mode, chunked, path, rows, ntenso
         hde = ntensors * hw * w * D * E
         assert 1 <= p.rows_per_tile <= S and p.tiles_per_block == -(-S // p.rows_per_tile)
         assert p.rows_per_tile == 1 or p.rows_per_tile * hde <= 16 * 1024 or rows
-        assert p.units == w * nb * p.tiles_per_block and p.grid == p.units
+        assert p.units == w * nb * p.tiles_per_block and p.grid == min(p.units, 148 * 4)
         assert p.block == 256 and p.smem_bytes <= 96 * 1024
+        cg = (p.rows_per_tile * p.row_bytes + 30) // 16
+        strided = ((p.rows_per_tile * hde + 30) // 16 if p.row_pitch * E == hde
+                   else p.rows_per_tile * ((hde + 30) // 16))
+        assert strided <= 1024 and ntensors * w * cg <= 1024
         v = p.vec_bytes
         assert p.row_bytes % v == 0 and (p.row_pitch * E) % v == 0
         assert v == 16 or (p.row_bytes % (2 * v) or (p.row_pitch * E) % (2 * v))

@@ -113,3 +113,48 @@ def test_library_all_to_all_comparison_arm_matches_the_oracle_gloo():
         p.join(timeout=60)
         assert p.exitcode == 0
     assert got == [(0, [True, True]), (1, [True, True])]
+
+
+def _bench_exchange_worker(rank, world, port, out_q):
+    from test_peer_cpu import ShmNative
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        wl = dict(w=world, B=1, S_local=6, H=4, D=8)
+        res = bench.exchange_arms(dist, torch.device("cpu"), rank, world, steps=3, warmup=1, wl=wl,
+                                  native=ShmNative(rank))
+        out_q.put((rank, bench.exchange_keys(res)))
+    except BaseException as e:          # report, so the parent does not wait for nothing
+        out_q.put((rank, repr(e)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_multi_gpu_bench_line_carries_both_exchange_arms_gloo():
+    """bench.py's multi-GPU exchange section (run_ours with N > 1 ranks) on CPU
+    gloo ranks, with host windows standing in for the peer object: the round
+    trip holds on every rank (checked inside), and the line gets
+    exchange_peer_gbs, exchange_nccl_gbs and the barrier share."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 34100 + os.getpid() % 500
+    procs = [ctx.Process(target=_bench_exchange_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=240) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank in (0, 1):
+        keys = got[rank]
+        assert isinstance(keys, dict), keys
+        ex = keys["exchange"]
+        # a few-KB slab on CPU: GB/s rounds to ~0, the step times are what count
+        assert keys["exchange_peer_gbs"] == ex["peer"]["gbs"] >= 0
+        assert keys["exchange_nccl_gbs"] == ex["nccl"]["gbs"] >= 0
+        assert ex["peer"]["ms_per_step"] > 0 and ex["nccl"]["ms_per_step"] > 0
+        assert ex["peer"]["barriers_per_step"] == 4 and 0 < ex["peer"]["barrier_share"]
+        assert ex["steps"] == 3 and "w = 2" in ex["workload"]
+    # both ranks report the same (max-over-ranks) times
+    assert got[0]["exchange"]["peer"]["ms_per_step"] == got[1]["exchange"]["peer"]["ms_per_step"]

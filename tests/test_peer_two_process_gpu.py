@@ -126,6 +126,6 @@ def test_two_processes_exchange_through_ipc_windows():
         # then one in-place exchange: a pull and nothing else
         assert rep["in_place_ok"] is True and rep["in_place_launches"] == 1
         assert rep["grad_ok"] is True and rep["packed_ok"] is True
-        # ... a packed exchange each way (1 + 3 then 3 + 3 launches), and a forward +
+        # ... a packed exchange each way (1 + 1 then 3 + 1 launches: one pull for all three tensors), and a forward +
         # backward exchange of publish + pull each
-        assert rep["launches"] == 2 * 2 * (1 + 2 + 1 + 3) + 1 + (1 + 3) + (3 + 3) + 2 * 2
+        assert rep["launches"] == 2 * 2 * (1 + 2 + 1 + 3) + 1 + (1 + 1) + (3 + 1) + 2 * 2

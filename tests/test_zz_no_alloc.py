@@ -8,8 +8,8 @@ These tests call it through the C ABI, on two calls in a row, and check every
 output byte against the CPU oracle's element map and against the regular entry
 point's output (bit for bit, the tolerance every test here uses). They also
 check that it rejects a TMA-path chunked call needing more status records than
-the array holds, while a vector-path chunked call over as many planes needs no
-record and runs. This file is named so pytest collects it last; it also passes
+the array holds, while a staged- or vector-path chunked call over as many
+planes needs no record and runs. This file is named so pytest collects it last; it also passes
 when run alone in a fresh process (its first call does the per-device set-up).
 """
 
@@ -24,16 +24,19 @@ pytestmark = pytest.mark.gpu
 
 INT_OF = {2: torch.int16, 4: torch.int32}
 
+TMA, VEC, STAGED = _lib.PATH_TMA, _lib.PATH_VEC, _lib.PATH_STAGED
 CASES = [
-    # (w, B, S_local, H, D, dtype, chunked, base offset in bytes); path noted
-    (4, 1, 8192, 24, 128, "bf16", 0, 0),    # TMA
-    (8, 2, 4725, 40, 128, "bf16", 1, 0),    # TMA, chunked, ragged tail
-    (2, 3, 37, 4, 64, "bf16", 1, 0),        # TMA, chunked
-    (4, 2, 45, 8, 128, "fp32", 0, 0),       # TMA, fp32
-    (2, 2, 17, 4, 3, "bf16", 0, 0),         # VEC: 12-byte runs
-    (2, 3, 17, 4, 3, "bf16", 1, 0),         # VEC, chunked
-    (4, 2, 33, 8, 64, "bf16", 0, 2),        # VEC: slab bases 2 bytes off 16
-    (4, 2, 33, 8, 64, "bf16", 1, 8),        # VEC, chunked, bases 8 bytes off 16
+    # (w, B, S_local, H, D, dtype, chunked, base offset in bytes, the path AUTO takes)
+    (4, 1, 8192, 24, 128, "bf16", 0, 0, TMA),
+    (8, 2, 4725, 40, 128, "bf16", 1, 0, TMA),     # chunked, ragged tail
+    (2, 3, 37, 4, 64, "bf16", 1, 0, TMA),         # chunked
+    (4, 2, 45, 8, 128, "fp32", 0, 0, TMA),        # fp32
+    (16, 2, 19, 16, 64, "bf16", 0, 0, VEC),       # w = 16: the vector path
+    (16, 3, 19, 16, 64, "bf16", 1, 0, VEC),       # the vector path, chunked
+    (2, 2, 17, 4, 3, "bf16", 0, 0, STAGED),       # 12-byte runs: re-aligned in shared memory
+    (2, 3, 17, 4, 3, "bf16", 1, 0, STAGED),       # chunked
+    (4, 2, 33, 8, 64, "bf16", 0, 2, STAGED),      # slab bases 2 bytes off 16
+    (4, 2, 33, 8, 64, "bf16", 1, 8, STAGED),      # chunked, bases 8 bytes off 16
 ]
 
 
@@ -67,7 +70,7 @@ def _noalloc(xs, outs, shape, mode, chunked, E, stream):
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "w{}B{}S{}H{}D{}_{}_c{}_off{}".format(*c))
 @pytest.mark.parametrize("mode", [0, 1])
 def test_noalloc_matches_the_oracle_and_run_on_two_calls_in_a_row(case, mode):
-    w, B, S, H, D, dtype, chunked, off = case
+    w, B, S, H, D, dtype, chunked, off, path = case
     E = 2 if dtype == "bf16" else 4
     torch.cuda.set_device(0)
     stream = torch.cuda.current_stream()
@@ -78,7 +81,7 @@ def test_noalloc_matches_the_oracle_and_run_on_two_calls_in_a_row(case, mode):
     cpu2 = make(in_shape, w, dtype, seed0=60 + mode)
     first, second = _device_slabs(cpu1, off), _device_slabs(cpu2, off)
     plan = UlyssesA2A(0, E).plan(first, mode, chunked=bool(chunked))
-    assert plan["path"] == (_lib.PATH_VEC if (D * E) % 16 or off else _lib.PATH_TMA)
+    assert plan["path"] == path
 
     # expected outputs: the CPU oracle, and the regular entry point
     oracle1 = oracle.ulysses_a2a(cpu1, mode)
@@ -127,8 +130,11 @@ def test_noalloc_rejects_more_tma_planes_than_status_records():
     assert all(torch.equal(o.cpu().view(torch.int16), e.view(torch.int16)) for o, e in zip(outs, want))
 
 
-def test_noalloc_chunked_vector_path_needs_no_status_record():
-    w, B, S, H, D = 2, 65, 3, 2, 3        # 6-byte runs: VEC path, 65 launches, no record
+@pytest.mark.parametrize("shape", [(2, 65, 3, 2, 3), (16, 65, 3, 16, 64)],
+                         ids=["staged_6B_runs", "vec_w16"])
+def test_noalloc_chunked_non_tma_paths_need_no_status_record(shape):
+    # 65 planes, 65 launches: the staged and vector kernels keep no status record
+    w, B, S, H, D = shape
     stream = torch.cuda.current_stream()
     cpu = normal_slabs((B, S, H, D), w, "bf16", seed0=90)
     xs = [t.cuda() for t in cpu]
