@@ -519,18 +519,21 @@ def vec_shape_block(device, peak, sampler, seconds=0.5):
         out[name] = {"payload_bytes": P, "path": PATH_NAMES[p["path"]],
                      "vec_bytes": p["vec_bytes"], "row_bytes": p["row_bytes"],
                      "base_offset_bytes": off, **res}
-        if p["path"] != 2:
-            a2a.set_path(2)
-            pv = a2a.plan(x, 0, out=y)
+        # the other of the two paths, forced: the vector kernel where AUTO
+        # re-aligns, the staged kernel where AUTO moves narrow vectors
+        other = {3: 2, 2: 3 if p["vec_bytes"] < 16 else None}.get(p["path"])
+        if other is not None:
+            a2a.set_path(other)
+            po = a2a.plan(x, 0, out=y)
             for t in z:
                 t.zero_()
             forced = per_mode_block(a2a, x, y, z, P, stream, peak, sampler, seconds)
             torch.cuda.synchronize()
             if not all(torch.equal(z[k], x[k]) for k in range(w)):
-                raise SystemExit(f"vector-path shape {name}: round trip mismatch (VEC forced)")
-            out[name]["vec_forced"] = {"vec_bytes": pv["vec_bytes"],
-                                       **{m: {k: v for k, v in forced[m].items() if k != "clocks"}
-                                          for m in forced}}
+                raise SystemExit(f"shape {name}: round trip mismatch ({PATH_NAMES[other]} forced)")
+            out[name][f"{PATH_NAMES[other]}_forced"] = {
+                "vec_bytes": po["vec_bytes"],
+                **{m: {k: v for k, v in forced[m].items() if k != "clocks"} for m in forced}}
         a2a.close()
         del x, y, z
         torch.cuda.empty_cache()

@@ -27,8 +27,8 @@
 //     split into (or assembled from) G-byte pieces at their places in the
 //     regions, where G (1..16) is the largest power of two dividing R, P and
 //     every slab base address, so that every piece is G-aligned on both sides.
-// Mode 0: strided rows -> registers -> regions -> gathered ranges.
-// Mode 1: gathered ranges -> registers -> regions -> strided rows.
+// Mode 0: strided rows -> regions (phase A), regions -> gathered ranges (B).
+// Mode 1: gathered ranges -> regions (phase A), regions -> strided rows (B).
 // Global bytes outside the unit are never read or written: a partial chunk
 // moves only its valid G-byte pieces.
 #pragma once
@@ -183,243 +183,178 @@ __device__ __forceinline__ uint4 strided_pieces_full(unsigned char* sm, const in
   return c.v;
 }
 
-// Threads per CTA, 16-byte chunks of a unit's in-side (the side read from
-// global memory first) each thread holds, and CTAs per SM the launch bound
-// keeps resident. The planner keeps every unit's in-side within
-// kStageThreads * kStageChunksPerThread chunks.
-constexpr int kStageThreads = 256;
-constexpr int kStageChunksPerThread = 4;
+// Loads in flight per thread before they are placed in shared memory.
+constexpr int kStageUnroll = 4;
+// 256-thread CTAs; at least 4 resident per SM.
 constexpr int kStageMinBlocksPerSm = 4;
 
-// One unit's geometry.
-struct StageUnit {
-  int64_t goff;        // byte offset of the unit's range in every gathered slab
-  const char* srow0;   // first strided row of the unit (strided slab j)
-  int32_t L;           // bytes of each gathered range
-  int32_t seg_len;     // bytes of a strided segment
-  int32_t nS;          // strided chunks scanned
-  int32_t nG;          // gathered chunks scanned (ng * Cg)
-  bool dense;          // one strided segment (P == HDE) or one per row
-};
-
-template <int MODE>
-__device__ __forceinline__ StageUnit stage_unit(const StageParams& p, uint32_t u) {
-  // u = (b_rel * w + j) * T + t
-  const uint32_t q = fdiv(u, p.div_T);
-  const uint32_t t = u - q * p.div_T.d;
-  const uint32_t bl = fdiv(q, p.div_w);
-  const uint32_t j = q - bl * p.div_w.d;
-  const int64_t b = p.b0 + bl;
-  const int64_t s0 = (int64_t)(p.tile0 + t) * p.rows_per_tile;
-  const int64_t left = p.S_local - s0;
-  const int32_t rows = (int32_t)(left < p.rows_per_tile ? left : p.rows_per_tile);
-  StageUnit su;
-  su.goff = ((b * p.w + j) * p.S_local + s0) * (int64_t)p.R;
-  su.srow0 = (MODE == 0 ? p.in[j] : p.out[j]) + (b * p.S_local + s0) * p.P;
-  su.L = rows * p.R;
-  su.dense = p.P == (int64_t)p.HDE;
-  su.seg_len = su.dense ? rows * p.HDE : p.HDE;
-  su.nS = su.dense
-              ? (int32_t)(((reinterpret_cast<uintptr_t>(su.srow0) & 15u) + su.seg_len + 15) >> 4)
-              : rows * p.Cs;
-  su.nG = p.ng * p.Cg;
-  return su;
-}
-
-// Strided chunk e of a unit: its aligned global address h, the offset o0 of
-// its byte 0 from the start of its segment (which begins at unit row i0), and
-// its valid bytes [x0, x1).
-struct StridedChunk {
-  const char* h;
-  int32_t o0, i0;
-  int x0, x1;
-};
-
-__device__ __forceinline__ StridedChunk strided_chunk(const StageParams& p, const StageUnit& su,
-                                                      int32_t e) {
-  StridedChunk c;
-  const uint32_t i = su.dense ? 0u : fdiv((uint32_t)e, p.div_Cs);
-  const int32_t k = su.dense ? e : e - (int32_t)i * p.Cs;
-  const char* a = su.srow0 + (int64_t)i * p.P;
-  c.o0 = 16 * k - (int32_t)(reinterpret_cast<uintptr_t>(a) & 15u);
-  c.h = a + c.o0;
-  c.i0 = (int32_t)i;
-  c.x0 = c.o0 < 0 ? -c.o0 : 0;
-  c.x1 = su.seg_len - c.o0 < 16 ? su.seg_len - c.o0 : 16;
-  return c;
-}
-
-// Gathered chunk e of a unit: head group g, its aligned global address h in
-// gathered slab g, its shared-memory slot (the region mirrors the range's
-// alignment, so the chunk sits whole at region offset 16c) and valid bytes.
-struct GatheredChunk {
-  const char* h;
-  int32_t slot;
-  int x0, x1;
-};
-
-template <int MODE>
-__device__ __forceinline__ GatheredChunk gathered_chunk(const StageParams& p, const StageUnit& su,
-                                                        int32_t e) {
-  GatheredChunk c;
-  const uint32_t g = fdiv((uint32_t)e, p.div_Cg);
-  const int32_t k = e - (int32_t)g * p.Cg;
-  const char* base = (MODE == 0 ? p.out[g] : p.in[g]) + su.goff;
-  const int32_t o0 = 16 * k - (int32_t)(reinterpret_cast<uintptr_t>(base) & 15u);
-  c.h = base + o0;
-  c.slot = (int32_t)g * p.RS + 16 * k;
-  c.x0 = o0 < 0 ? -o0 : 0;
-  c.x1 = su.L - o0 < 16 ? su.L - o0 : 16;
-  return c;
-}
-
-template <int MODE>
-__device__ __forceinline__ void stage_region_bases(const StageParams& p, const StageUnit& su,
-                                                   int32_t* rbase) {
-  for (int g = threadIdx.x; g < p.ng; g += blockDim.x) {
-    const char* ga = (MODE == 0 ? p.out[g] : p.in[g]) + su.goff;
-    rbase[g] = g * p.RS + (int32_t)(reinterpret_cast<uintptr_t>(ga) & 15u);
-  }
-}
-
-// Issue the loads of a unit's in-side (mode 0: the strided chunks; mode 1: the
-// gathered chunks) into this thread's registers.
 template <int G, int MODE>
-__device__ __forceinline__ void stage_load(const StageParams& p, const StageUnit& su,
-                                           uint4 (&v)[kStageChunksPerThread]) {
-#pragma unroll
-  for (int k = 0; k < kStageChunksPerThread; ++k) {
-    const int32_t e = (int32_t)threadIdx.x + k * kStageThreads;
-    if (MODE == 0) {
-      if (e < su.nS) {
-        const StridedChunk c = strided_chunk(p, su, e);
-        if (c.x0 == 0 && c.x1 == 16)
-          v[k] = ld_stream(reinterpret_cast<const uint4*>(c.h));
-        else if (c.x0 < c.x1)
-          v[k] = load_pieces<G>(c.h, c.x0, c.x1);
-      }
-    } else {
-      if (e < su.nG) {
-        const GatheredChunk c = gathered_chunk<MODE>(p, su, e);
-        if (c.x0 == 0 && c.x1 == 16)
-          v[k] = ld_stream(reinterpret_cast<const uint4*>(c.h));
-        else if (c.x0 < c.x1)
-          v[k] = load_pieces<G>(c.h, c.x0, c.x1);
-      }
-    }
-  }
-}
-
-// Place the loaded in-side into the regions.
-template <int G, int MODE>
-__device__ __forceinline__ void stage_place(unsigned char* sm, const int32_t* rbase,
-                                            const StageParams& p, const StageUnit& su,
-                                            const uint4 (&v)[kStageChunksPerThread]) {
-#pragma unroll
-  for (int k = 0; k < kStageChunksPerThread; ++k) {
-    const int32_t e = (int32_t)threadIdx.x + k * kStageThreads;
-    if (MODE == 0) {
-      if (e < su.nS) {
-        const StridedChunk c = strided_chunk(p, su, e);
-        if (c.x0 == 0 && c.x1 == 16 && p.R >= 16)
-          strided_pieces_full<G, true>(sm, rbase, p, v[k], c.o0, c.i0);
-        else if (c.x0 < c.x1)
-          strided_pieces<G, true>(sm, rbase, p, v[k], c.x0, c.x1, c.o0, c.i0);
-      }
-    } else {
-      if (e < su.nG) {
-        const GatheredChunk c = gathered_chunk<MODE>(p, su, e);
-        unsigned char* slot = sm + c.slot;
-        if (c.x0 == 0 && c.x1 == 16) {
-          *reinterpret_cast<uint4*>(slot) = v[k];
-        } else if (c.x0 < c.x1) {
-          Chunk16<G> cv;
-          cv.v = v[k];
-#pragma unroll
-          for (int m = 0; m < 16 / G; ++m)
-            if (m * G >= c.x0 && m * G < c.x1)
-              *reinterpret_cast<typename PieceOf<G>::type*>(slot + m * G) = cv.e[m];
-        }
-      }
-    }
-  }
-}
-
-// Write the unit's out-side from the regions (mode 0: the gathered ranges,
-// aligned; mode 1: the strided rows, assembled from pieces).
-template <int G, int MODE>
-__device__ __forceinline__ void stage_store(unsigned char* sm, const int32_t* rbase,
-                                            const StageParams& p, const StageUnit& su) {
-  if (MODE == 0) {
-    for (int32_t e = threadIdx.x; e < su.nG; e += kStageThreads) {
-      const GatheredChunk c = gathered_chunk<MODE>(p, su, e);
-      if (c.x0 >= c.x1) continue;
-      const uint4 v = *reinterpret_cast<const uint4*>(sm + c.slot);
-      char* h = const_cast<char*>(c.h);
-      if (c.x0 == 0 && c.x1 == 16)
-        st_stream(reinterpret_cast<uint4*>(h), v);
-      else
-        store_pieces<G>(h, v, c.x0, c.x1);
-    }
-  } else {
-    for (int32_t e = threadIdx.x; e < su.nS; e += kStageThreads) {
-      const StridedChunk c = strided_chunk(p, su, e);
-      if (c.x0 >= c.x1) continue;
-      char* h = const_cast<char*>(c.h);
-      if (c.x0 == 0 && c.x1 == 16) {
-        const uint4 v = p.R >= 16
-                            ? strided_pieces_full<G, false>(sm, rbase, p, make_uint4(0, 0, 0, 0),
-                                                            c.o0, c.i0)
-                            : strided_pieces<G, false>(sm, rbase, p, make_uint4(0, 0, 0, 0), 0,
-                                                       16, c.o0, c.i0);
-        st_stream(reinterpret_cast<uint4*>(h), v);
-      } else {
-        const uint4 v = strided_pieces<G, false>(sm, rbase, p, make_uint4(0, 0, 0, 0), c.x0,
-                                                 c.x1, c.o0, c.i0);
-        store_pieces<G>(h, v, c.x0, c.x1);
-      }
-    }
-  }
-}
-
-// A persistent grid: CTA k takes units k, k + gridDim.x, ... and keeps the
-// next unit's loads in flight while it writes the current unit out:
-//   place(u) | barrier | load(u + G), store(u) | barrier
-// The region offsets are double-buffered, so two barriers per unit suffice.
-template <int G, int MODE>
-__global__ void __launch_bounds__(kStageThreads, kStageMinBlocksPerSm)
+__global__ void __launch_bounds__(256, kStageMinBlocksPerSm)
     ua2a_stage_kernel(const __grid_constant__ StageParams p) {
   extern __shared__ __align__(16) unsigned char sm[];
-  int32_t* rbase2 = reinterpret_cast<int32_t*>(sm + (size_t)p.ng * p.RS);  // 2 x ng offsets
+  int32_t* rbase = reinterpret_cast<int32_t*>(sm + (size_t)p.ng * p.RS);
 #if UA2A_PDL
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
 #endif
-  uint32_t u = blockIdx.x;
-  if (u >= p.units) return;
-  int cur = 0;
-  StageUnit su = stage_unit<MODE>(p, u);
-  uint4 v[kStageChunksPerThread];
-  stage_region_bases<MODE>(p, su, rbase2);
-  stage_load<G, MODE>(p, su, v);
-  __syncthreads();
-  for (;;) {
-    const int32_t* rbase = rbase2 + cur * p.ng;
-    stage_place<G, MODE>(sm, rbase, p, su, v);
-    __syncthreads();  // the regions hold unit u
-    const uint32_t un = u + gridDim.x;
-    StageUnit sn = su;
-    if (un < p.units) {
-      sn = stage_unit<MODE>(p, un);
-      stage_region_bases<MODE>(p, sn, rbase2 + (cur ^ 1) * p.ng);
-      stage_load<G, MODE>(p, sn, v);
+  const int32_t R = p.R;
+  for (uint32_t u = blockIdx.x; u < p.units; u += gridDim.x) {
+    // u = (b_rel * w + j) * T + t
+    const uint32_t q = fdiv(u, p.div_T);
+    const uint32_t t = u - q * p.div_T.d;
+    const uint32_t bl = fdiv(q, p.div_w);
+    const uint32_t j = q - bl * p.div_w.d;
+    const int64_t b = p.b0 + bl;
+    const int64_t s0 = (int64_t)(p.tile0 + t) * p.rows_per_tile;
+    const int64_t left = p.S_local - s0;
+    const int32_t rows = (int32_t)(left < p.rows_per_tile ? left : p.rows_per_tile);
+    const int32_t L = rows * R;  // bytes of each gathered range of this unit
+    // byte offset of the unit's range in every gathered slab, and of its first
+    // row in strided slab j
+    const int64_t goff = ((b * p.w + j) * p.S_local + s0) * (int64_t)R;
+    const int64_t soff = (b * p.S_local + s0) * p.P;
+    const char* srow0 = (MODE == 0 ? p.in[j] : p.out[j]) + soff;
+    // Strided segments: the unit's rows are one contiguous segment when the
+    // slab is dense (P == HDE), else one segment per row.
+    const bool dense = p.P == (int64_t)p.HDE;
+    const int32_t seg_len = dense ? rows * p.HDE : p.HDE;
+    const int32_t nS = dense ? (int32_t)(((reinterpret_cast<uintptr_t>(srow0) & 15u) + seg_len + 15) >> 4)
+                             : rows * p.Cs;
+
+    for (int g = threadIdx.x; g < p.ng; g += blockDim.x) {
+      const char* ga = (MODE == 0 ? p.out[g] : p.in[g]) + goff;
+      rbase[g] = g * p.RS + (int32_t)(reinterpret_cast<uintptr_t>(ga) & 15u);
     }
-    stage_store<G, MODE>(sm, rbase, p, su);
-    __syncthreads();  // unit u is out of the regions; the next offsets are visible
-    if (un >= p.units) break;
-    u = un;
-    su = sn;
-    cur ^= 1;
+    __syncthreads();
+
+    if (MODE == 0) {
+      // phase A: strided rows -> regions, kStageUnroll loads in flight per thread
+      const int32_t nA = nS;
+      for (int32_t e0 = threadIdx.x; e0 < nA; e0 += blockDim.x * kStageUnroll) {
+        uint4 v[kStageUnroll];
+#pragma unroll
+        for (int k = 0; k < kStageUnroll; ++k) {
+          const int32_t e = e0 + k * (int32_t)blockDim.x;
+          if (e < nA) {
+            const uint32_t i = dense ? 0u : fdiv((uint32_t)e, p.div_Cs);
+            const int32_t c = dense ? e : e - (int32_t)i * p.Cs;
+            const char* a = srow0 + (int64_t)i * p.P;
+            const int32_t o0 = 16 * c - (int32_t)(reinterpret_cast<uintptr_t>(a) & 15u);
+            const int x0 = o0 < 0 ? -o0 : 0;
+            const int x1 = seg_len - o0 < 16 ? seg_len - o0 : 16;
+            if (x0 == 0 && x1 == 16)
+              v[k] = ld_stream(reinterpret_cast<const uint4*>(a + o0));
+            else if (x0 < x1)
+              v[k] = load_pieces<G>(a + o0, x0, x1);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kStageUnroll; ++k) {
+          const int32_t e = e0 + k * (int32_t)blockDim.x;
+          if (e < nA) {
+            const uint32_t i = dense ? 0u : fdiv((uint32_t)e, p.div_Cs);
+            const int32_t c = dense ? e : e - (int32_t)i * p.Cs;
+            const char* a = srow0 + (int64_t)i * p.P;
+            const int32_t o0 = 16 * c - (int32_t)(reinterpret_cast<uintptr_t>(a) & 15u);
+            const int x0 = o0 < 0 ? -o0 : 0;
+            const int x1 = seg_len - o0 < 16 ? seg_len - o0 : 16;
+            if (x0 == 0 && x1 == 16 && p.R >= 16)
+              strided_pieces_full<G, true>(sm, rbase, p, v[k], o0, (int32_t)i);
+            else if (x0 < x1)
+              strided_pieces<G, true>(sm, rbase, p, v[k], x0, x1, o0, (int32_t)i);
+          }
+        }
+      }
+      __syncthreads();
+      // phase B: regions -> gathered ranges (aligned in both)
+      const int32_t nB = p.ng * p.Cg;
+      for (int32_t e = threadIdx.x; e < nB; e += blockDim.x) {
+        const uint32_t g = fdiv((uint32_t)e, p.div_Cg);
+        const int32_t c = e - (int32_t)g * p.Cg;
+        char* d = p.out[g] + goff;
+        const int32_t o0 = 16 * c - (int32_t)(reinterpret_cast<uintptr_t>(d) & 15u);
+        const int x0 = o0 < 0 ? -o0 : 0;
+        const int x1 = L - o0 < 16 ? L - o0 : 16;
+        if (x0 >= x1) continue;
+        const uint4 v = *reinterpret_cast<const uint4*>(sm + (int32_t)g * p.RS + 16 * c);
+        if (x0 == 0 && x1 == 16)
+          st_stream(reinterpret_cast<uint4*>(d + o0), v);
+        else
+          store_pieces<G>(d + o0, v, x0, x1);
+      }
+    } else {
+      // phase A: gathered ranges -> regions, kStageUnroll loads in flight per thread
+      const int32_t nA = p.ng * p.Cg;
+      for (int32_t e0 = threadIdx.x; e0 < nA; e0 += blockDim.x * kStageUnroll) {
+        uint4 v[kStageUnroll];
+#pragma unroll
+        for (int k = 0; k < kStageUnroll; ++k) {
+          const int32_t e = e0 + k * (int32_t)blockDim.x;
+          if (e < nA) {
+            const uint32_t g = fdiv((uint32_t)e, p.div_Cg);
+            const int32_t c = e - (int32_t)g * p.Cg;
+            const char* s = p.in[g] + goff;
+            const int32_t o0 = 16 * c - (int32_t)(reinterpret_cast<uintptr_t>(s) & 15u);
+            const int x0 = o0 < 0 ? -o0 : 0;
+            const int x1 = L - o0 < 16 ? L - o0 : 16;
+            if (x0 == 0 && x1 == 16)
+              v[k] = ld_stream(reinterpret_cast<const uint4*>(s + o0));
+            else if (x0 < x1)
+              v[k] = load_pieces<G>(s + o0, x0, x1);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kStageUnroll; ++k) {
+          const int32_t e = e0 + k * (int32_t)blockDim.x;
+          if (e < nA) {
+            const uint32_t g = fdiv((uint32_t)e, p.div_Cg);
+            const int32_t c = e - (int32_t)g * p.Cg;
+            const char* s = p.in[g] + goff;
+            const int32_t o0 = 16 * c - (int32_t)(reinterpret_cast<uintptr_t>(s) & 15u);
+            const int x0 = o0 < 0 ? -o0 : 0;
+            const int x1 = L - o0 < 16 ? L - o0 : 16;
+            // the region mirrors the range's alignment, so chunk c sits whole
+            // at region offset 16c; a partial chunk fills only its valid pieces
+            unsigned char* slot = sm + (int32_t)g * p.RS + 16 * c;
+            if (x0 == 0 && x1 == 16) {
+              *reinterpret_cast<uint4*>(slot) = v[k];
+            } else if (x0 < x1) {
+              Chunk16<G> cv;
+              cv.v = v[k];
+#pragma unroll
+              for (int m = 0; m < 16 / G; ++m)
+                if (m * G >= x0 && m * G < x1)
+                  *reinterpret_cast<typename PieceOf<G>::type*>(slot + m * G) = cv.e[m];
+            }
+          }
+        }
+      }
+      __syncthreads();
+      // phase B: regions -> strided rows
+      const int32_t nB = nS;
+      for (int32_t e = threadIdx.x; e < nB; e += blockDim.x) {
+        const uint32_t i = dense ? 0u : fdiv((uint32_t)e, p.div_Cs);
+        const int32_t c = dense ? e : e - (int32_t)i * p.Cs;
+        char* a = const_cast<char*>(srow0) + (int64_t)i * p.P;
+        const int32_t o0 = 16 * c - (int32_t)(reinterpret_cast<uintptr_t>(a) & 15u);
+        const int x0 = o0 < 0 ? -o0 : 0;
+        const int x1 = seg_len - o0 < 16 ? seg_len - o0 : 16;
+        if (x0 >= x1) continue;
+        if (x0 == 0 && x1 == 16) {
+          const uint4 v = p.R >= 16 ? strided_pieces_full<G, false>(sm, rbase, p,
+                                                                    make_uint4(0, 0, 0, 0), o0,
+                                                                    (int32_t)i)
+                                    : strided_pieces<G, false>(sm, rbase, p, make_uint4(0, 0, 0, 0),
+                                                               0, 16, o0, (int32_t)i);
+          st_stream(reinterpret_cast<uint4*>(a + o0), v);
+        } else {
+          const uint4 v = strided_pieces<G, false>(sm, rbase, p, make_uint4(0, 0, 0, 0), x0, x1,
+                                                   o0, (int32_t)i);
+          store_pieces<G>(a + o0, v, x0, x1);
+        }
+      }
+    }
+    __syncthreads();  // the regions are reused by the next unit
   }
 }
 

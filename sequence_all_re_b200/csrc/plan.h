@@ -60,6 +60,11 @@ constexpr int kVecResidentCtasPerSm = 6;
 constexpr int64_t kStageTileTargetBytes = 16 * 1024;
 constexpr int64_t kStageSmemMax = 96 * 1024;
 constexpr int kStageBlock = 256;
+// AUTO re-aligns through shared memory only what the vector kernel would move
+// in pieces of at most this many bytes: measured on B200, 8-byte vectors
+// (0.86-0.91 of the copy bandwidth on 200-byte runs and on slabs 8 bytes off
+// 16) beat the staged kernel, 4- and 2-byte vectors (0.27-0.55) lose to it.
+constexpr int kStageMaxPiece = 4;
 // Unit numbering: 0 = destination rank outermost, 1 = innermost.
 constexpr int kDefaultOrder = 1;
 // Host-buffer entry point: sequence chunks its H2D copies, kernels and D2H
@@ -123,55 +128,38 @@ inline const char* tma_blocker(const void* const* in, void* const* out, int64_t 
 }
 
 // Geometry of the re-aligning (staged) path for runs of R bytes, ng head
-// groups per strided row (HDE = ng * R bytes, rows pitch_bytes apart) and
-// S_local rows:
-//   * rows per unit: about kStageTileTargetBytes of strided-side bytes (or
-//     rows_cap when set), fewer if needed so that both sides of a unit span at
-//     most kStageMaxChunks 16-byte chunks (a unit's in-side is held in
-//     registers, kStageMaxChunks / 256 chunks per thread) and its regions fit
-//     kStageSmemMax;
-//   * Cs / Cg: 16-byte chunks scanned per strided row / per gathered range;
-//   * shared memory: ng regions of RS bytes (RS = 16 * Cg rounded to an odd
-//     number of 16-byte chunks, so that consecutive regions start in
-//     different banks) and two arrays of ng 4-byte region offsets.
-// Returns false if not even one row fits.
+// groups per strided row (HDE = ng * R bytes) and S_local rows: the rows per
+// unit (about kStageTileTargetBytes of strided-side bytes, or rows_cap when
+// set), the 16-byte chunks scanned per strided row (Cs) and per gathered range
+// (Cg), and the shared memory of a CTA: ng regions of RS bytes (RS = 16*Cg
+// rounded to an odd number of 16-byte chunks, so that consecutive regions
+// start in different shared-memory banks) and ng 4-byte region offsets.
+// Returns false if not even one row fits kStageSmemMax.
 struct StageGeometry {
   int64_t rows = 0, tiles = 0, Cs = 0, Cg = 0, RS = 0, smem_bytes = 0;
 };
 
-constexpr int64_t kStageMaxChunks = 1024;   // 256 threads x 4 chunks
-constexpr int kStageCtasPerSm = 4;
-
-inline bool stage_geometry(int64_t R, int64_t ng, int64_t S, int rows_cap, int64_t pitch_bytes,
-                           StageGeometry* g) {
+inline bool stage_geometry(int64_t R, int64_t ng, int64_t S, int rows_cap, StageGeometry* g) {
   const int64_t HDE = ng * R;
   if (R < 1 || ng < 1 || S < 1 || HDE >= (int64_t(1) << 30)) return false;
-  const bool dense = pitch_bytes == HDE;
-  const int64_t Cs = (HDE + 30) / 16;
-  auto fits = [&](int64_t rows, int64_t* Cg, int64_t* RS, int64_t* smem) {
-    const int64_t strided_chunks = dense ? (rows * HDE + 30) / 16 : rows * Cs;
-    *Cg = (rows * R + 30) / 16;
-    *RS = 16 * (*Cg % 2 ? *Cg : *Cg + 1);
-    *smem = ng * *RS + 8 * ng;
-    return strided_chunks <= kStageMaxChunks && ng * *Cg <= kStageMaxChunks &&
-           *smem <= kStageSmemMax;
-  };
   int64_t rows = rows_cap > 0 ? rows_cap : kStageTileTargetBytes / HDE;
   if (rows < 1) rows = 1;
   if (rows > S) rows = S;
-  // closed-form upper bounds, then the exact check
-  const int64_t by_strided = dense ? (16 * kStageMaxChunks - 30) / HDE : kStageMaxChunks / Cs;
-  if (rows > by_strided) rows = by_strided > 1 ? by_strided : 1;
-  int64_t Cg = 0, RS = 0, smem = 0;
-  while (rows > 1 && !fits(rows, &Cg, &RS, &smem)) --rows;
-  if (!fits(rows, &Cg, &RS, &smem)) return false;
-  g->rows = rows;
-  g->tiles = (S + rows - 1) / rows;
-  g->Cs = Cs;
-  g->Cg = Cg;
-  g->RS = RS;
-  g->smem_bytes = (smem + 15) / 16 * 16;
-  return true;
+  for (; rows >= 1; rows = rows > 1 ? rows / 2 : 0) {
+    const int64_t Cg = (rows * R + 30) / 16;
+    const int64_t RS = 16 * (Cg % 2 ? Cg : Cg + 1);
+    const int64_t smem = ng * RS + 4 * ng;
+    if (smem <= kStageSmemMax && rows * HDE < (int64_t(1) << 30)) {
+      g->rows = rows;
+      g->tiles = (S + rows - 1) / rows;
+      g->Cs = (HDE + 30) / 16;
+      g->Cg = Cg;
+      g->RS = RS;
+      g->smem_bytes = (smem + 15) / 16 * 16;
+      return true;
+    }
+  }
+  return false;
 }
 
 // Public tuning struct -> internal knobs, with range checks (NULL = defaults).
@@ -491,18 +479,18 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     // pieces narrower than 16 bytes (or what it is forced onto), except
     // one-output launches.
     const bool forced_stage = forced_path == ULYSSES_A2A_PATH_STAGED;
-    if (forced_stage || (forced_path == ULYSSES_A2A_PATH_AUTO && v < 16 && only_out < 0)) {
+    if (forced_stage || (forced_path == ULYSSES_A2A_PATH_AUTO && v <= kStageMaxPiece && only_out < 0)) {
       StageGeometry sg;
-      if (stage_geometry(row_bytes, (int64_t)w * ntensors, S, tune.rows_per_tile, pitch * E, &sg)) {
+      if (stage_geometry(row_bytes, (int64_t)w * ntensors, S, tune.rows_per_tile, &sg)) {
         const int64_t nbl = chunked ? 1 : B;
         int64_t su;
         if (mul_overflows((int64_t)w * nbl, sg.tiles, &su) || su >= (int64_t(1) << 31)) {
           set_err(err, "%lld staged work units exceed the 2^31 limit", su);
           return ULYSSES_A2A_ERR_UNSUPPORTED;
         }
-        // a persistent grid: kStageCtasPerSm CTAs per SM (or ctas_per_sm)
-        const int64_t sgrid =
-            (int64_t)num_sms * (tune.ctas_per_sm > 0 ? tune.ctas_per_sm : kStageCtasPerSm);
+        // one short-lived CTA per unit (the hardware hands them to SMs as they
+        // free up), or a grid-stride grid of ctas_per_sm CTAs per SM
+        const int64_t sgrid = tune.ctas_per_sm > 0 ? (int64_t)num_sms * tune.ctas_per_sm : su;
         p->path = ULYSSES_A2A_PATH_STAGED;
         p->rows_per_tile = sg.rows;
         p->tiles_per_block = sg.tiles;
@@ -512,8 +500,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
         p->block = kStageBlock;
         p->grid = (int32_t)(su < sgrid ? su : sgrid);
       } else if (forced_stage) {
-        set_err(err, "staged path forced but one row of %lld bytes is too large for it (at most "
-                     "1024 16-byte chunks per side of a unit, 96 KB of shared memory)",
+        set_err(err, "staged path forced but one row of %lld bytes does not fit its shared memory",
                 row_bytes * w * ntensors);
         return ULYSSES_A2A_ERR_UNSUPPORTED;
       }

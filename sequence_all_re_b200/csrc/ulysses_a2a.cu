@@ -34,9 +34,7 @@ using ua2a::VecParams;
 
 static_assert(ua2a::kVecResidentCtasPerSm == ua2a::kVecMinBlocksPerSm,
               "the planner's VEC residency must match the kernel's launch bound");
-static_assert(ua2a::kStageMaxChunks == ua2a::kStageThreads * ua2a::kStageChunksPerThread,
-              "the planner's staged-unit chunk limit must match what the kernel's threads hold");
-static_assert(ua2a::kStageBlock == ua2a::kStageThreads, "staged CTA size");
+
 
 namespace ua2a {
 
@@ -286,7 +284,7 @@ StageParams stage_params(int64_t S, int w, int ntensors, int E, const ulysses_a2
   p.rows_per_tile = (int32_t)pl.rows_per_tile;
   p.units = (uint32_t)units;
   StageGeometry sg;
-  stage_geometry(pl.row_bytes, p.ng, S, (int)pl.rows_per_tile, pl.row_pitch * E, &sg);
+  stage_geometry(pl.row_bytes, p.ng, S, (int)pl.rows_per_tile, &sg);
   p.RS = (int32_t)sg.RS;
   p.Cs = (int32_t)sg.Cs;
   p.Cg = (int32_t)sg.Cg;

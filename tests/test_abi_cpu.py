@@ -172,19 +172,18 @@ def test_runs_off_16_bytes_take_the_staged_path():
 def test_staged_geometry():
     # 200-byte runs, 8 head groups of 1600-byte rows: units of 10 rows (16 KB),
     # one per (b, j, tile) covering every head group
+    # (8-byte vectors: AUTO keeps the vector path, so the staged path is forced)
     rc, p, _ = plan(8, 2, 4725, 8, 100)
+    assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 8
+    rc, p, _ = plan(8, 2, 4725, 8, 100, forced_path=PATH_STAGED)
     assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 8
     assert p.rows_per_tile == 16 * 1024 // 1600 == 10 and p.tail_rows == 4725 % 10
-    # a persistent grid of 4 CTAs per SM (148 SMs), each taking every 592nd unit
-    assert p.units == 8 * 2 * p.tiles_per_block and p.grid == 148 * 4 and p.block == 256
+    # one short-lived CTA per unit
+    assert p.units == 8 * 2 * p.tiles_per_block and p.grid == p.units and p.block == 256
     cg = (10 * 200 + 30) // 16
-    assert p.smem_bytes == (8 * 16 * (cg if cg % 2 else cg + 1) + 8 * 8 + 15) // 16 * 16
-    # a unit's in-side is held in registers: at most 1024 16-byte chunks per side
-    assert (10 * 1600 + 30) // 16 <= 1024 and 8 * cg <= 1024
-    rc, p, _ = plan(4, 1, 8192, 24, 128, forced_path=PATH_STAGED, rows_per_tile=8)
-    assert rc == OK and p.rows_per_tile == 2        # (2 * 6144 + 30) // 16 = 769 chunks
+    assert p.smem_bytes == (8 * 16 * (cg if cg % 2 else cg + 1) + 4 * 8 + 15) // 16 * 16
     # chunked: one plane per launch
-    rc, p, _ = plan(8, 2, 4725, 8, 100, chunked=1)
+    rc, p, _ = plan(8, 2, 4725, 8, 100, chunked=1, forced_path=PATH_STAGED)
     assert rc == OK and p.units == 8 * p.tiles_per_block and p.launches == 2
     # forced on an aligned shape, the pieces are 16 bytes
     rc, p, _ = plan(4, 1, 8192, 24, 128, forced_path=PATH_STAGED)
@@ -201,9 +200,13 @@ def test_vec_when_misaligned_pointer():
     ins, outs = fake_slabs(w, B * S * H * D * E)
     outs[1] += 8
     rc, p, _ = ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E)
-    assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 8
+    assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 8     # 8-byte vectors: VEC
+    outs[1] += 2
+    rc, p, _ = ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E)
+    assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 2  # 2-byte pieces: staged
     rc, p, _ = ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E, forced_path=PATH_VEC)
-    assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 8
+    assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 2
+    outs[1] -= 2
     rc, p, msg = ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E, forced_path=PATH_TMA)
     assert rc == ERR_UNSUPPORTED and "aligned" in msg
 
@@ -436,9 +439,11 @@ def test_pitch_smaller_than_a_row_is_rejected():
 def test_pitch_alignment_selects_the_vector_width():
     # pitch * E = (512 + 4) * 2 bytes: 8-byte aligned rows only
     rc, p, _ = plan_ex(4, 1, 64, 8, 64, 8 * 64 + 4)
-    assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 8
-    rc, p, _ = plan_ex(4, 1, 64, 8, 64, 8 * 64 + 4, forced_path=PATH_VEC)
     assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 8
+    rc, p, _ = plan_ex(4, 1, 64, 8, 64, 8 * 64 + 2)          # 4-byte aligned rows: staged
+    assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 4
+    rc, p, _ = plan_ex(4, 1, 64, 8, 64, 8 * 64 + 2, forced_path=PATH_VEC)
+    assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 4
     rc, _, msg = plan_ex(4, 1, 64, 8, 64, 8 * 64 + 4, forced_path=PATH_TMA)
     assert rc == ERR_UNSUPPORTED and "pitch" in msg
 
@@ -570,12 +575,11 @@ from hypothesis import strategies as st  # noqa: E402
 
 
 def _one_row_fits_stage(R, ng):
-    """Whether one strided row fits the staged path: at most 1024 16-byte
-    chunks per side, and 96 KB of shared memory for ng regions of (R + 30) // 16
-    chunks, rounded to an odd count, plus two arrays of ng 4-byte offsets."""
+    """Whether one strided row fits the staged path's 96 KB of shared memory:
+    ng regions of (R + 30) // 16 chunks, rounded to an odd count, plus ng
+    4-byte region offsets."""
     cg = (R + 30) // 16
-    return (ng * 16 * (cg if cg % 2 else cg + 1) + 8 * ng <= 96 * 1024
-            and (ng * R + 30) // 16 <= 1024 and ng * cg <= 1024)
+    return ng * 16 * (cg if cg % 2 else cg + 1) + 4 * ng <= 96 * 1024
 
 
 @settings(max_examples=300, deadline=None, derandomize=True, database=None)
@@ -610,17 +614,13 @@ def test_planner_invariants(w, hw, B, S, D, E, mode, chunked, path, rows, ntenso
         hde = ntensors * hw * w * D * E
         assert 1 <= p.rows_per_tile <= S and p.tiles_per_block == -(-S // p.rows_per_tile)
         assert p.rows_per_tile == 1 or p.rows_per_tile * hde <= 16 * 1024 or rows
-        assert p.units == w * nb * p.tiles_per_block and p.grid == min(p.units, 148 * 4)
+        assert p.units == w * nb * p.tiles_per_block and p.grid == p.units
         assert p.block == 256 and p.smem_bytes <= 96 * 1024
-        cg = (p.rows_per_tile * p.row_bytes + 30) // 16
-        strided = ((p.rows_per_tile * hde + 30) // 16 if p.row_pitch * E == hde
-                   else p.rows_per_tile * ((hde + 30) // 16))
-        assert strided <= 1024 and ntensors * w * cg <= 1024
         v = p.vec_bytes
         assert p.row_bytes % v == 0 and (p.row_pitch * E) % v == 0
         assert v == 16 or (p.row_bytes % (2 * v) or (p.row_pitch * E) % (2 * v))
         if path == PATH_AUTO:
-            assert v < 16
+            assert v <= 4
         return
     # tiles cover every sequence row exactly once per (r, b, j) block
     assert 1 <= p.rows_per_tile <= min(S, 256)
@@ -646,7 +646,7 @@ def test_planner_invariants(w, hw, B, S, D, E, mode, chunked, path, rows, ntenso
         v = p.vec_bytes
         assert v in (1, 2, 4, 8, 16) and p.row_bytes % v == 0 and (p.row_pitch * E) % v == 0
         # AUTO leaves narrower vectors to the staged path unless a row is too long
-        assert path == PATH_VEC or v == 16 or not _one_row_fits_stage(hw * D * E, ntensors * w)
+        assert path == PATH_VEC or v >= 8 or not _one_row_fits_stage(hw * D * E, ntensors * w)
         # the widest width the run length and the pitch allow (pointers are 4 KiB aligned)
         assert v == 16 or (p.row_bytes % (2 * v) or (p.row_pitch * E) % (2 * v))
         assert p.grid == p.units and p.block == 256

@@ -229,9 +229,10 @@ def test_nan_payloads_and_signed_zero_survive():
 
 @pytest.mark.parametrize("offset,vec", [(8, 8), (4, 4), (2, 2), (1, 1)])
 def test_misaligned_pointers_select_narrower_pieces(offset, vec):
-    # a base off the 16-byte boundary: AUTO re-aligns through shared memory in
-    # pieces of the alignment the bases allow; the vector path, when forced,
-    # uses vectors of that width
+    # a base off the 16-byte boundary: AUTO moves 8-byte vectors, or re-aligns
+    # through shared memory in pieces of the alignment the bases allow when
+    # that is 4 bytes or less; the vector path, when forced, uses vectors of
+    # that width
     w, B, S, H, D = 2, 2, 21, 4, 64
     E = 2 if offset % 2 == 0 else 1
     if E == 2:
@@ -242,11 +243,11 @@ def test_misaligned_pointers_select_narrower_pieces(offset, vec):
         xd = [t.cuda() for t in xs]
         g = Guarded(oracle.output_shape(tuple(xs[0].shape), 0, w), xs[0].dtype, w, offset=offset)
         plan = a2a.plan(xd, 0, out=g.slabs)
-        assert plan["path"] == PATH_STAGED and plan["vec_bytes"] == vec
+        assert plan["path"] == (PATH_STAGED if vec <= 4 else PATH_VEC) and plan["vec_bytes"] == vec
         a2a.set_path(PATH_VEC)
         plan = a2a.plan(xd, 0, out=g.slabs)
         assert plan["path"] == PATH_VEC and plan["vec_bytes"] == vec
-    for path in (PATH_AUTO, PATH_VEC):
+    for path in (PATH_AUTO, PATH_VEC, PATH_STAGED):
         for chunked in (False, True):
             run_case(xs, 0, out_offset=offset, path=path, chunked=chunked)
             run_case(xs, 0, in_offset=offset, path=path, chunked=chunked)
@@ -556,11 +557,11 @@ def test_mode1_writes_into_packed_slots(path):
                 assert torch.equal(bits(packed[j][:, :, c].cpu().contiguous()), bits(want[j]))
 
 
-@pytest.mark.parametrize("path", [PATH_AUTO, PATH_VEC], ids=["auto", "vec"])
+@pytest.mark.parametrize("path", [PATH_AUTO, PATH_VEC, PATH_STAGED], ids=["auto", "vec", "staged"])
 def test_odd_row_pitch_uses_narrower_pieces(path):
-    # rows of H*D + 4 bf16 elements: 8-byte aligned only, so 8-byte pieces
-    # (staged, AUTO) or 8-byte vectors (VEC); the 4 trailing elements of every
-    # row stay untouched
+    # rows of H*D + 4 bf16 elements: 8-byte aligned only, so 8-byte vectors
+    # (VEC, also AUTO's choice) or 8-byte pieces (staged, forced); the 4
+    # trailing elements of every row stay untouched
     w, B, S, H, D = 2, 2, 19, 4, 32
     pitch = H * D + 4
     bufs_cpu = normal_slabs((B * S * pitch,), w, "bf16", seed0=720)
@@ -570,7 +571,7 @@ def test_odd_row_pitch_uses_narrower_pieces(path):
         bufs = [t.cuda() for t in bufs_cpu]
         views = [t.as_strided((B, S, H, D), (S * pitch, pitch, D, 1)) for t in bufs]
         p = a2a.plan(views, 0)
-        assert p["path"] == (PATH_STAGED if path == PATH_AUTO else PATH_VEC)
+        assert p["path"] == (PATH_STAGED if path == PATH_STAGED else PATH_VEC)
         assert p["vec_bytes"] == 8 and p["row_pitch"] == pitch
         out = a2a.run(views, 0)
         for r in range(w):

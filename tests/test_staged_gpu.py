@@ -28,10 +28,10 @@ NARROW = [
     # (w, B, S_local, H, D, E): runs of (H/w)*D*E bytes, not a multiple of 16
     (4, 2, 100, 4, 3, 2),       # 6-byte runs: 2-byte pieces
     (4, 1, 77, 4, 3, 4),        # 12-byte runs: 4-byte pieces
-    (8, 2, 53, 8, 100, 2),      # 200-byte runs: 8-byte pieces, ragged tiles
+    (8, 2, 53, 8, 100, 2),      # 200-byte runs: 8-byte pieces (AUTO: 8-byte vectors)
     (3, 2, 29, 6, 5, 1),        # 10-byte runs: 2-byte pieces, odd rank count
     (2, 3, 33, 2, 7, 1),        # 7-byte runs: 1-byte pieces
-    (2, 2, 40, 2, 1, 8),        # 8-byte runs
+    (2, 2, 40, 2, 1, 8),        # 8-byte runs (AUTO: 8-byte vectors)
     (16, 1, 21, 16, 3, 2),      # w = 16
     (1, 2, 31, 3, 5, 2),        # w = 1: a copy
     (5, 1, 4000, 5, 3, 2),      # many rows per unit
@@ -42,14 +42,18 @@ NARROW = [
 @pytest.mark.parametrize("mode", [0, 1])
 @pytest.mark.parametrize("chunked", [False, True], ids=["whole", "per_plane"])
 def test_narrow_runs_take_the_staged_path(case, mode, chunked):
+    # AUTO re-aligns pieces of 4 bytes or less through shared memory and moves
+    # 8-byte ones as vectors; the staged path forced gives the same bytes
     w, B, S, H, D, E = case
     shape = slab_shape(mode, w, B, S, H, D)
     xs = [t.view(INT[E]).reshape(shape)
           for t in random_byte_slabs(shape[:-1] + (shape[-1] * E,), w, seed0=100 + w + D)]
     with UlyssesA2A(0, E) as a2a:
         p = a2a.plan([t.cuda() for t in xs], mode)
-        assert p["path"] == PATH_STAGED and p["vec_bytes"] < 16
+        assert p["vec_bytes"] < 16
+        assert p["path"] == (PATH_STAGED if p["vec_bytes"] <= 4 else PATH_VEC)
         run_case(xs, mode, chunked=chunked, a2a=a2a)
+        run_case(xs, mode, chunked=chunked, a2a=a2a, path=PATH_STAGED)
 
 
 SHAPES = [
@@ -92,6 +96,7 @@ def test_pitched_slabs_through_the_staged_path():
     pitch = 3 * H * D + 4
     bufs_cpu = normal_slabs((B * S * pitch,), w, "bf16", seed0=400)
     with UlyssesA2A(0, 2) as a2a:
+        a2a.set_path(PATH_STAGED)                 # 8-byte pieces: AUTO would take VEC
         bufs = [t.cuda() for t in bufs_cpu]
         for c in range(3):
             views = [t[c * H * D:].as_strided((B, S, H, D), (S * pitch, pitch, D, 1)) for t in bufs]

@@ -36,7 +36,7 @@ CASES = [
     (2, 2, 17, 4, 3, "bf16", 0, 0, STAGED),       # 12-byte runs: re-aligned in shared memory
     (2, 3, 17, 4, 3, "bf16", 1, 0, STAGED),       # chunked
     (4, 2, 33, 8, 64, "bf16", 0, 2, STAGED),      # slab bases 2 bytes off 16
-    (4, 2, 33, 8, 64, "bf16", 1, 8, STAGED),      # chunked, bases 8 bytes off 16
+    (4, 2, 33, 8, 64, "bf16", 1, 8, VEC),         # chunked, bases 8 bytes off 16: 8-byte vectors
 ]
 
 
