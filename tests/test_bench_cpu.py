@@ -11,11 +11,12 @@ import bench  # noqa: E402
 from sequence_all_re_b200 import _lib  # noqa: E402
 
 
-def plan_dict(w, B, S, H, D, path=_lib.PATH_AUTO):
-    step = (B * S * H * D * 2 + 4095) // 4096 * 4096
-    ins = [(1 << 40) + k * step for k in range(w)]
-    outs = [(1 << 40) + (w + k) * step for k in range(w)]
-    rc, p, msg = _lib.ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, 2, forced_path=path)
+def plan_dict(w, B, S, H, D, path=_lib.PATH_AUTO, E=2, off=0):
+    """The plan of a call whose slabs sit `off` bytes past 4 KiB boundaries."""
+    step = (B * S * H * D * E + 4095) // 4096 * 4096 + 4096
+    ins = [(1 << 40) + k * step + off for k in range(w)]
+    outs = [(1 << 40) + (w + k) * step + off for k in range(w)]
+    rc, p, msg = _lib.ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E, forced_path=path)
     assert rc == _lib.OK, msg
     return p.as_dict()
 
@@ -24,14 +25,22 @@ def test_committed_captures_match_the_current_kernels_and_plans():
     traffic = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))["workloads"]
     for key, entry in traffic.items():
         path, shape = key.split(":")
-        w, B, S, H, D = (int(part[1:]) for part in shape.split("_")[:5])
+        parts = shape.split("_")
+        w, B, S, H, D = (int(part[1:]) for part in parts[:5])
+        E = {"bf16": 2, "fp32": 4}[parts[5]]
+        off = int(parts[6][4:]) if len(parts) > 6 else 0
+        # the planner chooses this kernel for the captured shape (AUTO) ...
+        assert plan_dict(w, B, S, H, D, _lib.PATH_AUTO, E, off)["path"] == {
+            "tma": _lib.PATH_TMA, "vec": _lib.PATH_VEC, "staged": _lib.PATH_STAGED}[path] or (
+            key == "vec:w4_B1_S8192_H24_D128_bf16")          # the VEC capture of a TMA shape
+        # ... and the capture matches its launch shape and code
         p = plan_dict(w, B, S, H, D, {"tma": _lib.PATH_TMA, "vec": _lib.PATH_VEC,
-                                      "staged": _lib.PATH_STAGED}[path])
+                                      "staged": _lib.PATH_STAGED}[path], E, off)
         got, why = bench.ncu_traffic(key, p, 0)
         assert why == "ncu", (key, why)
         assert got == entry["dram_bytes_per_launch"]
         # DRAM reads of a launch cover the payload (no re-reads beyond a few per mille)
-        payload = w * B * S * H * D * 2
+        payload = w * B * S * H * D * E
         for m in ("mode0", "mode1"):
             assert 0.999 * payload <= entry[m]["dram_read"] <= 1.002 * payload, (key, m)
 
