@@ -76,7 +76,7 @@ extern "C" {
 /* ---- copy paths ------------------------------------------------------- */
 #define ULYSSES_A2A_PATH_AUTO 0  /* TMA when the shape allows it; else VEC, or
                                     STAGED when VEC could only use vectors
-                                    narrower than 16 bytes                   */
+                                    of 4 bytes or less                       */
 #define ULYSSES_A2A_PATH_TMA  1  /* cp.async.bulk.tensor load -> smem -> store */
 #define ULYSSES_A2A_PATH_VEC  2  /* 16/8/4/2/1-byte LDG/STG copy               */
 #define ULYSSES_A2A_PATH_STAGED 3 /* 16-byte LDG/STG, re-aligned in shared

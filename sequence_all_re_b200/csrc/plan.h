@@ -476,8 +476,8 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     p->grid = (int32_t)(units < g ? units : g);
 
     // The re-aligning path takes what the vector path could only move in
-    // pieces narrower than 16 bytes (or what it is forced onto), except
-    // one-output launches.
+    // pieces of kStageMaxPiece bytes or less (or what it is forced onto),
+    // except one-output launches.
     const bool forced_stage = forced_path == ULYSSES_A2A_PATH_STAGED;
     if (forced_stage || (forced_path == ULYSSES_A2A_PATH_AUTO && v <= kStageMaxPiece && only_out < 0)) {
       StageGeometry sg;
