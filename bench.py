@@ -802,8 +802,14 @@ def run_ours(args):
 
     exchange = None
     if world > 1 and not args.no_exchange:
-        exchange = exchange_arms(dist, device, rank, world, min(args.steps, 200),
-                                 max(3, args.warmup), wl)
+        # the exchange arms run after `value` is taken; an error that every rank
+        # meets (a window that cannot be mapped, say) is recorded in the line
+        # instead of losing it
+        try:
+            exchange = exchange_arms(dist, device, rank, world, min(args.steps, 200),
+                                     max(3, args.warmup), wl)
+        except Exception as e:          # noqa: BLE001 (reported in the line)
+            exchange = {"error": f"{type(e).__name__}: {e}"[:300]}
 
     full_sweep = None
     if args.sweep and rank == 0:

@@ -60,6 +60,17 @@ constexpr int kVecResidentCtasPerSm = 6;
 constexpr int64_t kStageTileTargetBytes = 16 * 1024;
 constexpr int64_t kStageSmemMax = 96 * 1024;
 constexpr int kStageBlock = 256;
+// AUTO moves launches of at most this many payload bytes with the vector
+// kernel even where TMA could take them: measured on B200 in CUDA-graph
+// replays, a vector launch costs about 0.6-1 us less (128 KiB: 1.3-1.5 us
+// against 2.0 us; 8 MiB: 2.9 against 3.7 us; 64 MiB: 19.5 against 20.9 us)
+// since its CTAs retire once their stores are issued, while a TMA tile waits
+// for its load and then for its store to read shared memory; from 192 MiB on
+// the two paths are within 2 % of each other.
+constexpr int64_t kVecSmallLaunchBytes = int64_t(64) << 20;
+// Smallest vector unit: small launches get units of payload / (2 * SMs),
+// down to this size, so that every SM has work.
+constexpr int64_t kVecMinTileBytes = 2 * 1024;
 // AUTO re-aligns through shared memory only what the vector kernel would move
 // in pieces of at most this many bytes: measured on B200, 8-byte vectors
 // (0.86-0.91 of the copy bandwidth on 200-byte runs and on slabs 8 bytes off
@@ -340,10 +351,18 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     path = ULYSSES_A2A_PATH_VEC;  // the staged path is decided with the vector width below
   } else {
     path = blocker ? ULYSSES_A2A_PATH_VEC : ULYSSES_A2A_PATH_TMA;
+    if (path == ULYSSES_A2A_PATH_TMA && payload / (chunked ? B : 1) <= kVecSmallLaunchBytes)
+      path = ULYSSES_A2A_PATH_VEC;  // small launches: the vector kernel's latency is lower
   }
 
-  // sequence rows per work unit
-  int64_t rows = (path == ULYSSES_A2A_PATH_TMA ? kTmaTileTargetBytes : kTileTargetBytes) / row_bytes;
+  // sequence rows per work unit; a small vector launch gets smaller units so
+  // that about two per SM exist
+  int64_t unit_target = path == ULYSSES_A2A_PATH_TMA ? kTmaTileTargetBytes : kTileTargetBytes;
+  if (path == ULYSSES_A2A_PATH_VEC) {
+    const int64_t spread = payload / (chunked ? B : 1) / (2 * (int64_t)num_sms);
+    if (spread < unit_target) unit_target = spread > kVecMinTileBytes ? spread : kVecMinTileBytes;
+  }
+  int64_t rows = unit_target / row_bytes;
   if (tune.rows_per_tile > 0) rows = tune.rows_per_tile;
   if (rows < 1) rows = 1;
   if (rows > kTmaMaxBoxDim) rows = kTmaMaxBoxDim;

@@ -143,10 +143,31 @@ def test_plan_windowed_chunked_variant():
 
 
 def test_plan_tiny_workload():
+    # 64 KiB: AUTO takes the vector kernel (lower latency below 64 MiB), with
+    # the smallest units (2 KB: 8 rows of 256 B) so that every SM gets work
     rc, p, _ = plan(2, 1, 64, 4, 64)
+    assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 16
+    assert p.rows_per_tile == 8 and p.tail_rows == 0 and p.tiles_per_block == 8
+    assert p.units == 2 * 2 * 8 and p.grid == p.units
+    # forced onto TMA: one-tile CTAs of 32 rows
+    rc, p, _ = plan(2, 1, 64, 4, 64, forced_path=PATH_TMA)
     assert rc == OK and p.path == PATH_TMA
     assert p.rows_per_tile == 32 and p.tail_rows == 0 and p.tiles_per_block == 2
     assert p.units == 8 and p.chunk_units == 1 and p.grid == 8
+
+
+def test_auto_switches_to_tma_above_64_mib_per_launch():
+    # w=4, H=16, D=128 bf16: 16 KB per sequence row of all ranks
+    rc, p, _ = plan(4, 1, 4096, 16, 128)                # 64 MiB: vector kernel
+    assert rc == OK and p.path == PATH_VEC and p.payload_bytes == 64 << 20
+    assert p.rows_per_tile == 12 * 1024 // (4 * 128 * 2)   # 12 KB units again
+    rc, p, _ = plan(4, 1, 4097, 16, 128)                # just above: TMA
+    assert rc == OK and p.path == PATH_TMA
+    # chunked: the launch is one plane
+    rc, p, _ = plan(4, 2, 4096, 16, 128)                # 128 MiB in one launch: TMA
+    assert rc == OK and p.path == PATH_TMA
+    rc, p, _ = plan(4, 2, 4096, 16, 128, chunked=1)     # 64 MiB per launch: vector
+    assert rc == OK and p.path == PATH_VEC
 
 
 def test_rows_never_exceed_sequence():
@@ -284,28 +305,28 @@ def test_ring_split_between_producers_loads_and_stores():
 def test_large_rows_reduce_stages_then_producers():
     # 24 KB rows: four producers keep two 24 KB stages each (192 KB)
     # persistent schedule
-    rc, p, _ = plan(2, 1, 16, 128, 192, chunk_units=0)
+    rc, p, _ = plan(2, 1, 16, 128, 192, chunk_units=0, forced_path=PATH_TMA)
     assert rc == OK and p.path == PATH_TMA and p.rows_per_tile == 1
     assert p.row_bytes == 24 * 1024
     assert (p.producers, p.stages, p.smem_bytes) == (4, 8, 192 * 1024)
     # 32 KB rows: two stages for four producers would not fit; three producers do
-    rc, p, _ = plan(2, 1, 16, 128, 256, chunk_units=0)
+    rc, p, _ = plan(2, 1, 16, 128, 256, chunk_units=0, forced_path=PATH_TMA)
     assert rc == OK and p.row_bytes == 32 * 1024
     assert (p.producers, p.stages, p.smem_bytes) == (3, 6, 192 * 1024)
     # 64 KB rows: one producer with a three-stage ring
-    rc, p, _ = plan(2, 1, 8, 256, 256, chunk_units=0)
+    rc, p, _ = plan(2, 1, 8, 256, 256, chunk_units=0, forced_path=PATH_TMA)
     assert rc == OK and p.path == PATH_TMA and p.row_bytes == 64 * 1024
     assert (p.producers, p.stages, p.lookahead, p.smem_bytes) == (1, 3, 2, 192 * 1024)
     # default (chunked grid): one producer, one tile; the residency cap reserves
     # shared memory for round(100 KB / tile) CTAs per SM (24 KB tiles: 4 CTAs)
-    rc, p, _ = plan(2, 1, 16, 128, 192)
+    rc, p, _ = plan(2, 1, 16, 128, 192, forced_path=PATH_TMA)
     assert (p.producers, p.stages, p.chunk_units) == (1, 1, 1)
     assert p.smem_bytes == (228 * 1024 // 4 - 1024) // 1024 * 1024
     # 64 KB tiles: cap round(100 / 64) = 2 CTAs per SM (113 KB each)
-    rc, p, _ = plan(2, 1, 8, 256, 256)
+    rc, p, _ = plan(2, 1, 8, 256, 256, forced_path=PATH_TMA)
     assert (p.producers, p.stages, p.chunk_units, p.smem_bytes) == (1, 1, 1, 113 * 1024)
     # a tile larger than the cap's share keeps its own size (cap 1 is 220 KB max)
-    rc, p, _ = plan(2, 1, 8, 256, 256, ctas_per_sm=8)
+    rc, p, _ = plan(2, 1, 8, 256, 256, ctas_per_sm=8, forced_path=PATH_TMA)
     assert p.smem_bytes == 64 * 1024
 
 
@@ -427,7 +448,7 @@ def plan_ex(w, B, S, H, D, pitch, mode=0, E=2, base=1 << 40, **kw):
 def test_pitch_defaults_to_dense_and_is_reported():
     rc, p, _ = plan_ex(4, 1, 64, 8, 64, 0)
     assert rc == OK and p.row_pitch == 8 * 64
-    rc, p, _ = plan_ex(4, 1, 64, 8, 64, 3 * 8 * 64)
+    rc, p, _ = plan_ex(4, 1, 64, 8, 64, 3 * 8 * 64, forced_path=PATH_TMA)
     assert rc == OK and p.row_pitch == 3 * 8 * 64 and p.path == PATH_TMA
 
 

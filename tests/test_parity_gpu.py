@@ -770,6 +770,7 @@ def test_tma_box_and_tile_limits():
     w, B, S, H, D = 2, 2, 5, 256, 256
     with UlyssesA2A(0, 2) as a2a:
         xs = normal_slabs((B, S, H, D), w, "bf16", seed0=950)
+        a2a.set_path(PATH_TMA)      # (AUTO would take the vector kernel for so small a call)
         p = a2a.plan([t.cuda() for t in xs], 0)
         assert p["path"] == PATH_TMA and p["rows_per_tile"] == 1 and p["row_bytes"] == 64 * 1024
         for mode, x in ((0, xs), (1, oracle.ulysses_a2a(xs, 0))):
@@ -806,7 +807,11 @@ def test_environment_overrides_set_the_initial_knobs(monkeypatch):
         a2a.set_path(PATH_AUTO)
         a2a.set_tuning()
         assert a2a.settings() == (PATH_AUTO, dict(_lib.TuningT.DEFAULTS))
-        assert a2a.plan([t.cuda() for t in xs], 0)["path"] == PATH_TMA
+        p = a2a.plan([t.cuda() for t in xs], 0)      # 768 KiB: AUTO's vector kernel
+        assert p["path"] == PATH_VEC and p["grid"] == p["units"]
+        big = [torch.empty((1, 65536, 8, 64), dtype=torch.bfloat16, device="cuda") for _ in range(4)]
+        assert a2a.plan(big, 0)["path"] == PATH_TMA   # 256 MiB: TMA
+        del big
         del out
 
 

@@ -29,8 +29,9 @@ CASES = [
     # (w, B, S_local, H, D, dtype, chunked, base offset in bytes, the path AUTO takes)
     (4, 1, 8192, 24, 128, "bf16", 0, 0, TMA),
     (8, 2, 4725, 40, 128, "bf16", 1, 0, TMA),     # chunked, ragged tail
-    (2, 3, 37, 4, 64, "bf16", 1, 0, TMA),         # chunked
-    (4, 2, 45, 8, 128, "fp32", 0, 0, TMA),        # fp32
+    (4, 1, 16384, 8, 128, "fp32", 0, 0, TMA),     # fp32 (256 MiB)
+    (2, 3, 37, 4, 64, "bf16", 1, 0, VEC),         # small calls: the vector kernel, chunked
+    (4, 2, 45, 8, 128, "fp32", 0, 0, VEC),        # fp32
     (16, 2, 19, 16, 64, "bf16", 0, 0, VEC),       # w = 16: the vector path
     (16, 3, 19, 16, 64, "bf16", 1, 0, VEC),       # the vector path, chunked
     (2, 2, 17, 4, 3, "bf16", 0, 0, STAGED),       # 12-byte runs: re-aligned in shared memory
@@ -114,20 +115,29 @@ def test_noalloc_matches_the_oracle_and_run_on_two_calls_in_a_row(case, mode):
 
 
 def test_noalloc_rejects_more_tma_planes_than_status_records():
-    w, B, S, H, D = 2, 65, 2, 2, 8        # 16-byte runs: TMA, one record per plane
+    # planes of just over 64 MiB (the TMA path takes launches above that): a
+    # chunked call over 65 of them needs 65 status records
+    w, B, S, H, D = 2, 65, 4100, 32, 128
     stream = torch.cuda.current_stream()
-    xs = [t.cuda() for t in normal_slabs((B, S, H, D), w, "bf16")]
+    xs = [torch.randint(-30000, 30000, (B, S, H, D), dtype=torch.int16, device="cuda")
+          .view(torch.bfloat16) for _ in range(w)]
     outs = [torch.zeros((B, S * w, H // w, D), dtype=torch.bfloat16, device="cuda") for _ in range(w)]
     rc, msg = _noalloc(xs, outs, (w, B, S, H, D), 0, 1, 2, stream)
     assert rc == _lib.ERR_UNSUPPORTED
     assert "64" in msg and "planes" in msg
     torch.cuda.synchronize()
-    assert all(bool((o == 0).all()) for o in outs), "a rejected call must launch nothing"
-    # the same data unchunked needs one record and is accepted
+    assert all(int(o.view(torch.int16).abs().sum()) == 0 for o in outs), \
+        "a rejected call must launch nothing"
+    # the same data unchunked needs one record and is accepted; every plane is
+    # re-laid out on its own, so planes 0 and 64 are checked against the oracle
     rc, msg = _noalloc(xs, outs, (w, B, S, H, D), 0, 0, 2, stream)
     assert rc == _lib.OK, msg
-    want = oracle.ulysses_a2a([t.cpu() for t in xs], 0)
-    assert all(torch.equal(o.cpu().view(torch.int16), e.view(torch.int16)) for o, e in zip(outs, want))
+    for b in (0, B - 1):
+        want = oracle.ulysses_a2a([t[b:b + 1].cpu() for t in xs], 0)
+        for o, e in zip(outs, want):
+            assert torch.equal(o[b:b + 1].cpu().view(torch.int16), e.view(torch.int16)), b
+    del xs, outs
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("shape", [(2, 65, 3, 2, 3), (16, 65, 3, 16, 64)],
