@@ -145,6 +145,57 @@ __device__ __forceinline__ uint4 strided_pieces(unsigned char* sm, const int32_t
   return c.v;
 }
 
+// A whole 16-byte chunk to / from 16 consecutive bytes of shared memory at
+// byte offset `at` (which must be even): one 16-, two 8- or four 4-byte accesses
+// when `at` allows them, else (at = 2 mod 4) a 2-byte access, three 4-byte
+// accesses 2 bytes into the chunk (their words assembled with byte
+// permutes: bytes 2..5 of the chunk are the upper half of word 0 and the
+// lower half of word 1, and so on) and a final 2-byte access.
+__device__ __forceinline__ void smem_put16(unsigned char* sm, int32_t at, const uint4& v) {
+  unsigned char* d = sm + at;
+  if ((at & 15) == 0) {
+    *reinterpret_cast<uint4*>(d) = v;
+  } else if ((at & 7) == 0) {
+    reinterpret_cast<uint2*>(d)[0] = make_uint2(v.x, v.y);
+    reinterpret_cast<uint2*>(d)[1] = make_uint2(v.z, v.w);
+  } else if ((at & 3) == 0) {
+    uint32_t* q = reinterpret_cast<uint32_t*>(d);
+    q[0] = v.x;
+    q[1] = v.y;
+    q[2] = v.z;
+    q[3] = v.w;
+  } else {
+    *reinterpret_cast<unsigned short*>(d) = (unsigned short)v.x;
+    *reinterpret_cast<uint32_t*>(d + 2) = __byte_perm(v.x, v.y, 0x5432);
+    *reinterpret_cast<uint32_t*>(d + 6) = __byte_perm(v.y, v.z, 0x5432);
+    *reinterpret_cast<uint32_t*>(d + 10) = __byte_perm(v.z, v.w, 0x5432);
+    *reinterpret_cast<unsigned short*>(d + 14) = (unsigned short)(v.w >> 16);
+  }
+}
+
+__device__ __forceinline__ uint4 smem_get16(const unsigned char* sm, int32_t at) {
+  const unsigned char* d = sm + at;
+  if ((at & 15) == 0) return *reinterpret_cast<const uint4*>(d);
+  uint4 v;
+  if ((at & 7) == 0) {
+    const uint2 a = reinterpret_cast<const uint2*>(d)[0];
+    const uint2 b = reinterpret_cast<const uint2*>(d)[1];
+    v = make_uint4(a.x, a.y, b.x, b.y);
+  } else if ((at & 3) == 0) {
+    const uint32_t* q = reinterpret_cast<const uint32_t*>(d);
+    v = make_uint4(q[0], q[1], q[2], q[3]);
+  } else {
+    const uint32_t h0 = *reinterpret_cast<const unsigned short*>(d);
+    const uint32_t m1 = *reinterpret_cast<const uint32_t*>(d + 2);
+    const uint32_t m2 = *reinterpret_cast<const uint32_t*>(d + 6);
+    const uint32_t m3 = *reinterpret_cast<const uint32_t*>(d + 10);
+    const uint32_t h4 = *reinterpret_cast<const unsigned short*>(d + 14);
+    v = make_uint4(__byte_perm(h0, m1, 0x5410), __byte_perm(m1, m2, 0x5432),
+                   __byte_perm(m2, m3, 0x5432), __byte_perm(m3, h4, 0x5432));
+  }
+  return v;
+}
+
 // The same pieces for a whole chunk (x0 = 0, x1 = 16, so o0 >= 0) when a run
 // is at least 16 bytes long: the chunk then meets at most one head-group
 // boundary, lim bytes in, and byte x goes to at1 + x before it and to
@@ -163,6 +214,13 @@ __device__ __forceinline__ uint4 strided_pieces_full(unsigned char* sm, const in
   int32_t iR = (i0 + (int32_t)di) * p.R;
   const int32_t at1 = rbase[g] + iR + col;
   const int32_t lim = p.R - col;  // bytes before the next head group
+  if (G >= 2 && lim >= 16) {      // the whole chunk lands contiguously (at1 is even)
+    if (STORE) {
+      smem_put16(sm, at1, c.v);
+      return c.v;
+    }
+    return smem_get16(sm, at1);
+  }
   int32_t at2 = at1;
   if (lim < 16) {
     if (++g == p.ng) {            // the next head group starts the next row
