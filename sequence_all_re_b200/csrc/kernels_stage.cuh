@@ -26,7 +26,9 @@
 //   * the strided side moves as aligned 16-byte global vectors too, each one
 //     split into (or assembled from) G-byte pieces at their places in the
 //     regions, where G (1..16) is the largest power of two dividing R, P and
-//     every slab base address, so that every piece is G-aligned on both sides.
+//     every slab base address, so that every piece is G-aligned on both sides;
+//     a chunk whose 16 bytes land contiguously in one region moves as aligned
+//     shared-memory words instead.
 // Mode 0: strided rows -> regions (phase A), regions -> gathered ranges (B).
 // Mode 1: gathered ranges -> regions (phase A), regions -> strided rows (B).
 // Global bytes outside the unit are never read or written: a partial chunk
