@@ -431,9 +431,10 @@ def isolated_call(a2a, src, dst, mode, stream, reps, flush, acc, sampler=None):
 def bandwidth_sweep(device, peak, payload_exps=range(17, 32), dtypes=(("bf16", 2), ("fp32", 4)),
                     ws=(2, 4, 8), sampler=None, long_payload=None, long_seconds=1.0):
     """Payloads 2^e bytes (e in payload_exps), w = 2/4/8, H = 8w, D = 128, B = 1,
-    U[-1,1) values, both modes. Payloads under 64 MiB: device time per call from
-    CUDA-graph replays of back-to-back calls; larger: back-to-back loops of at
-    least 0.25 s (long_seconds for the long_payload bf16 points)."""
+    U[-1,1) values, both modes. Payloads up to 64 MiB: device time per call from
+    CUDA-graph replays of back-to-back calls (a call issued from Python can take
+    longer on the host than its kernel on the device); larger: back-to-back
+    loops of at least 0.25 s (long_seconds for the long_payload bf16 points)."""
     from sequence_all_re_b200 import UlyssesA2A
 
     stream = torch.cuda.Stream(device)
@@ -460,7 +461,7 @@ def bandwidth_sweep(device, peak, payload_exps=range(17, 32), dtypes=(("bf16", 2
                 row = {"dtype": dtype, "w": w, "payload_bytes": P, "S_local": S,
                        "l2_assisted": 2 * P <= l2}
                 for mode, (src, dst) in ((0, (x, y)), (1, (y, x))):
-                    if P < (64 << 20):
+                    if P <= (64 << 20):         # a host-side call can take longer than the kernel
                         calls = max(1, min(64, (256 << 20) // P))
                         reps = max(3, min(50, (8 << 30) // (P * calls)))
                         ms = graph_ms_per_call(a2a, src, dst, mode, calls, reps, stream)
