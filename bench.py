@@ -179,7 +179,7 @@ def _code_only(text: str) -> str:
 KERNEL_FILES = {"tma": "kernels_tma.cuh", "vec": "kernels_vec.cuh", "staged": "kernels_stage.cuh"}
 PATH_NAMES = {1: "tma", 2: "vec", 3: "staged"}
 LAUNCH_FIELDS = ("path", "rows_per_tile", "producers", "stages", "lookahead", "chunk_units",
-                 "order", "grid", "block", "smem_bytes", "vec_bytes")
+                 "order", "grid", "block", "smem_bytes", "vec_bytes", "peeled")
 
 
 def kernel_source_hash(path):
@@ -518,11 +518,12 @@ def vec_shape_block(device, peak, sampler, seconds=0.5):
         if not all(torch.equal(z[k], x[k]) for k in range(w)):
             raise SystemExit(f"vector-path shape {name}: round trip mismatch")
         out[name] = {"payload_bytes": P, "path": PATH_NAMES[p["path"]],
-                     "vec_bytes": p["vec_bytes"], "row_bytes": p["row_bytes"],
-                     "base_offset_bytes": off, **res}
+                     "vec_bytes": p["vec_bytes"], "peeled": p["peeled"],
+                     "row_bytes": p["row_bytes"], "base_offset_bytes": off, **res}
         # the other of the two paths, forced: the vector kernel where AUTO
-        # re-aligns, the staged kernel where AUTO moves narrow vectors
-        other = {3: 2, 2: 3 if p["vec_bytes"] < 16 else None}.get(p["path"])
+        # re-aligns, the staged kernel where AUTO moves narrow vectors or
+        # peeled 16-byte windows
+        other = {3: 2, 2: 3 if (p["vec_bytes"] < 16 or p["peeled"]) else None}.get(p["path"])
         if other is not None:
             a2a.set_path(other)
             po = a2a.plan(x, 0, out=y)
@@ -533,7 +534,7 @@ def vec_shape_block(device, peak, sampler, seconds=0.5):
             if not all(torch.equal(z[k], x[k]) for k in range(w)):
                 raise SystemExit(f"shape {name}: round trip mismatch ({PATH_NAMES[other]} forced)")
             out[name][f"{PATH_NAMES[other]}_forced"] = {
-                "vec_bytes": po["vec_bytes"],
+                "vec_bytes": po["vec_bytes"], "peeled": po["peeled"],
                 **{m: {k: v for k, v in forced[m].items() if k != "clocks"} for m in forced}}
         a2a.close()
         del x, y, z

@@ -76,9 +76,11 @@ extern "C" {
 /* ---- copy paths ------------------------------------------------------- */
 #define ULYSSES_A2A_PATH_AUTO 0  /* TMA when the shape allows it; else VEC, or
                                     STAGED when VEC could only use vectors
-                                    of 4 bytes or less                       */
+                                    of 4 bytes or less and cannot peel them
+                                    (see plan_t.peeled)                     */
 #define ULYSSES_A2A_PATH_TMA  1  /* cp.async.bulk.tensor load -> smem -> store */
-#define ULYSSES_A2A_PATH_VEC  2  /* 16/8/4/2/1-byte LDG/STG copy               */
+#define ULYSSES_A2A_PATH_VEC  2  /* 16/8/4/2/1-byte LDG/STG copy, or 16-byte
+                                    vectors between peeled heads and tails   */
 #define ULYSSES_A2A_PATH_STAGED 3 /* 16-byte LDG/STG, re-aligned in shared
                                     memory: runs or bases off 16 bytes     */
 
@@ -116,6 +118,14 @@ typedef struct ulysses_a2a_plan_t {
                                 robin); n = n consecutive units per CTA     */
     int64_t row_pitch;       /* elements between rows of the [B,S_local,H,D]
                                 side (H*D when dense)                       */
+    int32_t peeled;          /* VEC path: 1 = every slab starts the same a
+                                bytes past a 16-byte boundary and runs and
+                                rows are multiples of 16 bytes (runs of 64+):
+                                each run moves as 16-byte vectors between a
+                                head of 16 - a and a tail of a bytes, moved
+                                in aligned pieces by the same CTAs;
+                                vec_bytes is then 16                        */
+    int32_t reserved;        /* 0                                             */
 } ulysses_a2a_plan_t;
 
 /* One call's arguments, for ulysses_a2a_run_ex / ulysses_a2a_plan_ex. Same

@@ -24,7 +24,11 @@ import torch
 from . import _lib
 from ._lib import A2AError, PATH_AUTO, PATH_STAGED, PATH_TMA, PATH_VEC  # noqa: F401
 
-__all__ = ["UlyssesA2A", "A2AError", "output_shape", "mode0_local_tuple",
+# torch's current stream as a raw handle (the public torch.cuda.current_stream
+# wraps the same handle in a Stream object)
+_raw_current_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+__all__ = ["UlyssesA2A", "A2AError", "output_shape", "mode0_local_tuple", "marshal_slabs",
            "PATH_AUTO", "PATH_TMA", "PATH_VEC", "PATH_STAGED"]
 
 
@@ -45,6 +49,82 @@ def mode0_local_tuple(in_shape, mode: int, w: int) -> tuple:
     return (int(B), int(S_global) // w, int(H_local) * w, int(D))
 
 
+def row_pitch(ts, allow_pitch: bool) -> int:
+    """Row pitch (elements) shared by [B, S, H, D] tensors: 0 when contiguous,
+    else p for views whose strides are (S*p, p, D, 1) with p >= H*D (for
+    example q, k or v of a packed [B, S, 3, H, D] projection output)."""
+    if all(t.is_contiguous() for t in ts):
+        return 0
+    if not allow_pitch:
+        raise ValueError("rank slabs must be contiguous")
+    B, S, H, D = ts[0].shape
+    pitch = None
+    for t in ts:
+        st = t.stride()
+        p = st[1]
+        ok = st[3] == 1 and (H == 1 or st[2] == D) and p >= H * D and (B == 1 or st[0] == S * p)
+        if not ok or (pitch is not None and p != pitch):
+            raise ValueError("a [B, S, H, D] slab must be contiguous or a view with strides "
+                             "(S*p, p, D, 1), p >= H*D, shared by all slabs")
+        pitch = p
+    return pitch
+
+
+def marshal_slabs(xs, mode: int, out, device_type: str, elem_bytes: int,
+                  allow_pitch: bool = False):
+    """Checks one call's slabs and turns them into the C ABI's arguments.
+
+    Returns (w, (B, S_local, H, D), out, input pointers, output pointers, row
+    pitch of the [B, S, H, D] side in elements, 0 when contiguous), allocating
+    the outputs when ``out`` is None; raises ValueError on slabs the op cannot
+    take. One pass over each list, reading only cheap tensor attributes: this
+    runs on every call, and on small launches its cost is of the kernel's
+    order. Whether each pointer lies in the context device's memory, inside
+    its allocation, the library checks itself."""
+    w = len(xs)
+    if w < 1:
+        raise ValueError("need at least one rank slab")
+    if mode != 0 and mode != 1:
+        raise ValueError("mode must be 0 or 1")
+    x0 = xs[0]
+    shape, dt = x0.shape, x0.dtype
+    if len(shape) != 4:
+        raise ValueError("rank slabs are 4D")
+    if x0.element_size() != elem_bytes:
+        raise ValueError(f"context handles {elem_bytes}-byte elements")
+    cuda = device_type == "cuda"
+    in_ptrs, in_dense = [], True
+    for t in xs:
+        if t.shape != shape or t.dtype != dt:
+            raise ValueError("rank slabs must share shape and dtype")
+        if t.is_cuda != cuda or (not cuda and t.device.type != device_type):
+            raise ValueError(f"rank slabs must be on {device_type}")
+        in_dense = in_dense and t.is_contiguous()
+        in_ptrs.append(t.data_ptr())
+    B, S, H, D = mode0_local_tuple(shape, mode, w)
+    oshape = output_shape(shape, mode, w)
+    if out is None:
+        kw = {"dtype": dt, "device": x0.device}
+        if not cuda:
+            kw["pin_memory"] = x0.is_pinned()
+        out = [torch.empty(oshape, **kw) for _ in range(w)]
+    elif len(out) != w:
+        raise ValueError("need one output per rank")
+    out_ptrs, out_dense = [], True
+    for o in out:
+        if o.shape != oshape or o.dtype != dt:
+            raise ValueError(f"outputs must be {oshape} {dt}")
+        out_dense = out_dense and o.is_contiguous()
+        out_ptrs.append(o.data_ptr())
+    # the [B, S, H, D] side (inputs in mode 0, outputs in mode 1) may be pitched
+    strided, strided_dense, dense = ((xs, in_dense, out_dense) if mode == 0
+                                     else (out, out_dense, in_dense))
+    if not dense:
+        raise ValueError("the [B, S_local*w, H/w, D] slabs must be contiguous")
+    pitch = 0 if strided_dense else row_pitch(strided, allow_pitch)
+    return w, (B, S, H, D), out, in_ptrs, out_ptrs, pitch
+
+
 class UlyssesA2A:
     """A library context bound to one CUDA device and one element size."""
 
@@ -52,6 +132,8 @@ class UlyssesA2A:
         dev = torch.device("cuda", device) if isinstance(device, int) else torch.device(device)
         self.device = dev
         self.elem_bytes = int(elem_bytes)
+        self._device_index = dev.index or 0
+        self._desc = _lib.DescBuffer()
         self._ctx = _lib.ulysses_a2a_create(dev.index or 0, self.elem_bytes)
 
     # ------------------------------------------------------------------ knobs
@@ -83,63 +165,15 @@ class UlyssesA2A:
             raise A2AError(rc, self.last_error())
 
     # ------------------------------------------------------------- the op
-    @staticmethod
-    def _row_pitch(ts, allow_pitch):
-        """Row pitch (elements) shared by [B, S, H, D] tensors: 0 when contiguous,
-        else p for views whose strides are (S*p, p, D, 1) with p >= H*D (for
-        example q, k or v of a packed [B, S, 3, H, D] projection output)."""
-        if all(t.is_contiguous() for t in ts):
-            return 0
-        if not allow_pitch:
-            raise ValueError("rank slabs must be contiguous")
-        B, S, H, D = ts[0].shape
-        pitch = None
-        for t in ts:
-            st = t.stride()
-            p = st[1]
-            ok = st[3] == 1 and (H == 1 or st[2] == D) and p >= H * D and (B == 1 or st[0] == S * p)
-            if not ok or (pitch is not None and p != pitch):
-                raise ValueError("a [B, S, H, D] slab must be contiguous or a view with strides "
-                                 "(S*p, p, D, 1), p >= H*D, shared by all slabs")
-            pitch = p
-        return pitch
-
-    def _prepare(self, xs, mode, out, device_type, allow_pitch=False):
-        w = len(xs)
-        if w < 1:
-            raise ValueError("need at least one rank slab")
-        shape = tuple(xs[0].shape)
-        if len(shape) != 4:
-            raise ValueError("rank slabs are 4D")
-        for t in xs:
-            if tuple(t.shape) != shape or t.dtype != xs[0].dtype:
-                raise ValueError("rank slabs must share shape and dtype")
-            if t.element_size() != self.elem_bytes:
-                raise ValueError(f"context handles {self.elem_bytes}-byte elements")
-            if t.device.type != device_type:
-                raise ValueError(f"rank slabs must be on {device_type}")
-        if mode not in (0, 1):
-            raise ValueError("mode must be 0 or 1")
-        B, S, H, D = mode0_local_tuple(shape, mode, w)
-        oshape = output_shape(shape, mode, w)
-        if out is None:
-            kw = {"dtype": xs[0].dtype, "device": xs[0].device}
-            if device_type == "cpu":
-                kw["pin_memory"] = xs[0].is_pinned()
-            out = [torch.empty(oshape, **kw) for _ in range(w)]
-        else:
-            if len(out) != w:
-                raise ValueError("need one output per rank")
-            for o in out:
-                if tuple(o.shape) != oshape or o.dtype != xs[0].dtype:
-                    raise ValueError(f"outputs must be {oshape} {xs[0].dtype}")
-        # the [B, S, H, D] side (inputs in mode 0, outputs in mode 1) may be pitched
-        strided, dense = (xs, out) if mode == 0 else (out, xs)
-        pitch = self._row_pitch(strided, allow_pitch)
-        if not all(t.is_contiguous() for t in dense):
-            raise ValueError("the [B, S_local*w, H/w, D] slabs must be contiguous")
-        self._last_pitch = pitch
-        return w, (B, S, H, D), out
+    def _stream_handle(self, stream) -> int:
+        """cudaStream_t of ``stream`` (a torch stream or a raw handle); None is
+        torch's current stream on this context's device, read without building
+        a Stream object (that costs microseconds per call)."""
+        if stream is None:
+            if _raw_current_stream is not None:
+                return _raw_current_stream(self._device_index)
+            return torch.cuda.current_stream(self.device).cuda_stream
+        return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
     def run(self, xs, mode: int, chunked: bool = False, out=None, stream=None):
         """Re-layout device slabs ``xs`` (list of w tensors); returns the w outputs.
@@ -149,14 +183,10 @@ class UlyssesA2A:
         projection output: it is read or written in place. Asynchronous on
         ``stream`` (default: torch's current stream on the device).
         """
-        w, (B, S, H, D), out = self._prepare(xs, mode, out, "cuda", allow_pitch=True)
-        if stream is None:
-            stream = torch.cuda.current_stream(self.device)
-        handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
-        rc = _lib.ulysses_a2a_run_ex(self._ctx, [t.data_ptr() or 0 for t in xs],
-                                     [o.data_ptr() or 0 for o in out], B, S, H, D, w, mode,
-                                     int(chunked), self._last_pitch, handle)
-        self._check(rc)
+        w, (B, S, H, D), out, ip, op, pitch = marshal_slabs(xs, mode, out, "cuda", self.elem_bytes,
+                                                            allow_pitch=True)
+        ref = self._desc.fill(ip, op, B, S, H, D, w, mode, int(chunked), pitch)
+        self._check(_lib.run_ex_ref(self._ctx, ref, self._stream_handle(stream)))
         return out
 
     def run_packed(self, xs, mode: int, chunked: bool = False, out=None, stream=None):
@@ -205,43 +235,32 @@ class UlyssesA2A:
                     or not t.is_contiguous() or t.element_size() != self.elem_bytes):
                 raise ValueError(f"every slab must be a contiguous {shape} CUDA tensor of "
                                  f"{self.elem_bytes}-byte elements")
-        if stream is None:
-            stream = torch.cuda.current_stream(self.device)
-        handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
-        rc = _lib.ulysses_a2a_run_ex(self._ctx, [t.data_ptr() or 0 for t in ins],
-                                     [o.data_ptr() or 0 for o in flat_out], B, S, H, D, w, mode,
-                                     int(chunked), 0, handle, ntensors=T)
-        self._check(rc)
+        ref = self._desc.fill([t.data_ptr() for t in ins], [o.data_ptr() for o in flat_out],
+                              B, S, H, D, w, mode, int(chunked), 0, T)
+        self._check(_lib.run_ex_ref(self._ctx, ref, self._stream_handle(stream)))
         return out
 
     def run_host(self, xs, mode: int, chunked: bool = False, out=None, stream=None):
         """Same op on host slabs: H2D copies, the kernel, D2H copies; returns when done."""
-        w, (B, S, H, D), out = self._prepare(xs, mode, out, "cpu")
-        if stream is None:
-            stream = torch.cuda.current_stream(self.device)
-        handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
-        rc = _lib.ulysses_a2a_run_host(self._ctx, [t.data_ptr() for t in xs],
-                                       [o.data_ptr() for o in out], B, S, H, D, w, mode,
-                                       int(chunked), handle)
+        w, (B, S, H, D), out, ip, op, _ = marshal_slabs(xs, mode, out, "cpu", self.elem_bytes)
+        rc = _lib.ulysses_a2a_run_host(self._ctx, ip, op, B, S, H, D, w, mode, int(chunked),
+                                       self._stream_handle(stream))
         self._check(rc)
         return out
 
     def status(self, stream=None) -> None:
         """Synchronise ``stream``; raise if a kernel of this context gave up a wait."""
-        if stream is None:
-            stream = torch.cuda.current_stream(self.device)
-        handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
-        self._check(_lib.ulysses_a2a_status(self._ctx, handle))
+        self._check(_lib.ulysses_a2a_status(self._ctx, self._stream_handle(stream)))
 
     def plan(self, xs, mode: int, chunked: bool = False, out=None, knobs=None) -> dict:
         """The path and geometry a run with these tensors would use (host only), with
         this context's forced path and tuning, or the given ``knobs`` dict instead."""
-        w, (B, S, H, D), out = self._prepare(xs, mode, out, xs[0].device.type, allow_pitch=True)
+        w, (B, S, H, D), out, ip, op, pitch = marshal_slabs(xs, mode, out, xs[0].device.type,
+                                                            self.elem_bytes, allow_pitch=True)
         path, current = self.settings()
-        rc, p, msg = _lib.ulysses_a2a_plan_ex([t.data_ptr() for t in xs],
-                                              [o.data_ptr() for o in out], B, S, H, D, w, mode,
+        rc, p, msg = _lib.ulysses_a2a_plan_ex(ip, op, B, S, H, D, w, mode,
                                               int(chunked), self.elem_bytes,
-                                              row_pitch=self._last_pitch, forced_path=path,
+                                              row_pitch=pitch, forced_path=path,
                                               **(current if knobs is None else knobs))
         if rc != _lib.OK:
             raise A2AError(rc, msg)

@@ -83,6 +83,8 @@ class PlanT(ctypes.Structure):
         ("order", ctypes.c_int32),
         ("chunk_units", ctypes.c_int32),
         ("row_pitch", ctypes.c_int64),
+        ("peeled", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
     ]
 
     def as_dict(self) -> dict:
@@ -143,6 +145,41 @@ def make_desc(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, row_pitch=0
               int(B), int(S_local), int(H), int(D), int(w), int(mode), int(chunked),
               int(ntensors), int(row_pitch))
     return d, (ins, outs)
+
+
+class DescBuffer:
+    """One DescT and its two pointer arrays, refilled in place call after call.
+
+    Building a fresh descriptor (structure, arrays, casts) costs several
+    microseconds of Python per call, as much as a small launch's kernel. A
+    context serves one host thread at a time, so one buffer per context is
+    enough; the arrays grow when a call passes more slabs than they hold."""
+
+    def __init__(self, capacity: int = 16):
+        self.desc = DescT()
+        self.ref = ctypes.byref(self.desc)
+        self._cap = 0
+        self._grow(capacity)
+
+    def _grow(self, n: int) -> None:
+        self.ins = (ctypes.c_void_p * n)()
+        self.outs = (ctypes.c_void_p * n)()
+        self.desc.in_slabs = ctypes.cast(self.ins, ctypes.POINTER(ctypes.c_void_p))
+        self.desc.out_slabs = ctypes.cast(self.outs, ctypes.POINTER(ctypes.c_void_p))
+        self._cap = n
+
+    def fill(self, in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, row_pitch=0,
+             ntensors=0):
+        """Writes one call's arguments; returns the reference to pass to the library."""
+        ni, no = len(in_ptrs), len(out_ptrs)
+        if ni > self._cap or no > self._cap:
+            self._grow(max(ni, no))
+        self.ins[:ni] = in_ptrs
+        self.outs[:no] = out_ptrs
+        d = self.desc
+        d.B, d.S_local, d.H, d.D = B, S_local, H, D
+        d.w, d.mode, d.chunked, d.ntensors, d.row_pitch = w, mode, chunked, ntensors, row_pitch
+        return self.ref
 
 
 class A2AError(RuntimeError):
@@ -314,6 +351,11 @@ def ulysses_a2a_run_ex(ctx, in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunke
                        stream, ntensors=0) -> int:
     d, keep = make_desc(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, row_pitch, ntensors)
     return lib.ulysses_a2a_run_ex(ctx, ctypes.byref(d), ctypes.c_void_p(int(stream)))
+
+
+def run_ex_ref(ctx, desc_ref, stream) -> int:
+    """ulysses_a2a_run_ex on a descriptor already filled (a DescBuffer's ``ref``)."""
+    return lib.ulysses_a2a_run_ex(ctx, desc_ref, stream)
 
 
 def ulysses_a2a_plan_ex(in_ptrs, out_ptrs, B, S_local, H, D, w, mode, chunked, elem_bytes,

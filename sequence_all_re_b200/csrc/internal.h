@@ -98,8 +98,14 @@ int check_residency(ulysses_a2a_ctx* ctx, const void* const* ptrs, int w, int64_
 // Kernel launches (programmatic stream serialization).
 cudaError_t launch_tma(int mode, int grid, int block, size_t smem, cudaStream_t st,
                        const TmaParams& p);
-cudaError_t launch_vec(const VecParams& p, int vec_bytes, int mode, int grid, int block,
-                       cudaStream_t st);
+cudaError_t launch_vec(const VecParams& p, int vec_bytes, int peeled, int mode, int grid,
+                       int block, cudaStream_t st);
+// VEC-path kernel parameters for a plan (b0 left for the caller): nr head
+// groups from r0 in steps of r_stride, nj sequence blocks from j0, nb planes
+// and nt tiles of each (r, b, j) block from tile0, `units` units in all.
+VecParams vec_params(const void* const* in, void* const* out, int nin, int nout, int64_t S, int w,
+                     int E, const ulysses_a2a_plan_t& pl, int64_t units, int64_t nb, int64_t nt,
+                     int nr, int nj, uint32_t r0, uint32_t r_stride, uint32_t j0, int64_t tile0);
 cudaError_t launch_stage(const StageParams& p, int piece_bytes, int mode, int grid, int block,
                          size_t smem, cudaStream_t st);
 // Let every staged kernel use up to kStageSmemMax of dynamic shared memory.

@@ -257,27 +257,11 @@ static int ua2a_impl_run_noalloc(const void* const* in_slabs, void* const* out_s
         return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "staged kernel launch failed (plane %lld)", l);
     }
   } else {
-    VecParams p{};
-    for (int k = 0; k < w; ++k) {
-      p.in[k] = static_cast<const char*>(in_slabs[k]);
-      p.out[k] = static_cast<char*>(out_slabs[k]);
-    }
-    p.S_local = S_local;
-    p.r_stride = 1;
-    p.nv = pl.row_bytes / pl.vec_bytes;
-    p.srow = pl.row_pitch * elem_bytes / pl.vec_bytes;
-    p.w = w;
-    p.rows_per_tile = (int32_t)pl.rows_per_tile;
-    p.units = (uint32_t)pl.units;
-    p.order = pl.order;
-    p.div_T = ua2a::FastDiv((uint32_t)pl.tiles_per_block);
-    p.div_nr = ua2a::FastDiv((uint32_t)w);
-    p.div_nj = ua2a::FastDiv((uint32_t)w);
-    p.div_nb = ua2a::FastDiv((uint32_t)nb);
-    p.div_nv = ua2a::FastDiv((uint32_t)p.nv);
+    VecParams p = vec_params(in_slabs, out_slabs, w, w, S_local, w, elem_bytes, pl, pl.units, nb,
+                             pl.tiles_per_block, w, w, 0u, 1u, 0u, 0);
     for (int l = 0; l < pl.launches; ++l) {
       p.b0 = chunked ? l : 0;
-      e = launch_vec(p, pl.vec_bytes, mode, pl.grid, pl.block, st_);
+      e = launch_vec(p, pl.vec_bytes, pl.peeled, mode, pl.grid, pl.block, st_);
       if (e != cudaSuccess)
         return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "VEC kernel launch failed (plane %lld)", l);
     }

@@ -138,6 +138,25 @@ inline const char* tma_blocker(const void* const* in, void* const* out, int64_t 
   return nullptr;
 }
 
+// Peeled vector path: runs of at least this many bytes (shorter ones are
+// mostly head and tail).
+constexpr int64_t kPeelMinRunBytes = 64;
+
+// Offset a (1..15) past a 16-byte boundary shared by every slab a call reads
+// or writes, when its runs (run_bytes) and rows (pitch_bytes) are whole
+// multiples of 16 bytes, so that every run on either side starts a bytes past
+// a boundary; else 0.
+inline int common_offset(const void* const* in, int nin, void* const* out, int nout,
+                         int64_t run_bytes, int64_t pitch_bytes) {
+  if (run_bytes % 16 != 0 || pitch_bytes % 16 != 0 || nin < 1) return 0;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(in[0]) & 15u;
+  for (int k = 0; k < nin; ++k)
+    if ((reinterpret_cast<uintptr_t>(in[k]) & 15u) != a) return 0;
+  for (int k = 0; k < nout; ++k)
+    if ((reinterpret_cast<uintptr_t>(out[k]) & 15u) != a) return 0;
+  return (int)a;
+}
+
 // Geometry of the re-aligning (staged) path for runs of R bytes, ng head
 // groups per strided row (HDE = ng * R bytes) and S_local rows: the rows per
 // unit (about kStageTileTargetBytes of strided-side bytes, or rows_cap when
@@ -483,10 +502,17 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
       set_err(err, "one VEC tile exceeds 2^31 vectors");
       return ULYSSES_A2A_ERR_UNSUPPORTED;
     }
+    // Runs that start at one offset past a 16-byte boundary on both sides move
+    // as 16-byte vectors between a peeled head and tail (not one-output
+    // launches, whose inputs are other ranks' windows).
     // one CTA per unit (units < 2^31 was checked above), or a grid-stride
     // grid of ctas_per_sm CTAs per SM when that knob is set
     int64_t g = tune.ctas_per_sm > 0 ? (int64_t)num_sms * tune.ctas_per_sm : units;
-    p->vec_bytes = v;
+    const bool peel = v < 16 && only_out < 0 && forced_path != ULYSSES_A2A_PATH_STAGED &&
+                      row_bytes >= kPeelMinRunBytes &&
+                      common_offset(in, nin, out, nout, row_bytes, pitch * E) != 0;
+    p->vec_bytes = peel ? 16 : v;
+    p->peeled = peel ? 1 : 0;
     p->stages = 0;
     p->lookahead = 0;
     p->producers = 0;
@@ -498,7 +524,8 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     // pieces of kStageMaxPiece bytes or less (or what it is forced onto),
     // except one-output launches.
     const bool forced_stage = forced_path == ULYSSES_A2A_PATH_STAGED;
-    if (forced_stage || (forced_path == ULYSSES_A2A_PATH_AUTO && v <= kStageMaxPiece && only_out < 0)) {
+    if (forced_stage ||
+        (forced_path == ULYSSES_A2A_PATH_AUTO && !peel && v <= kStageMaxPiece && only_out < 0)) {
       StageGeometry sg;
       if (stage_geometry(row_bytes, (int64_t)w * ntensors, S, tune.rows_per_tile, &sg)) {
         const int64_t nbl = chunked ? 1 : B;

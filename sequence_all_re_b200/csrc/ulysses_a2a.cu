@@ -223,8 +223,11 @@ cudaError_t launch_vec_t(const VecParams& p, int mode, int grid, int block, cuda
                    : launch_pdl(ua2a::ua2a_vec_kernel<V, 1, 4>, grid, block, 0, st, p);
 }
 
-cudaError_t launch_vec(const VecParams& p, int vec_bytes, int mode, int grid, int block,
-                       cudaStream_t st) {
+cudaError_t launch_vec(const VecParams& p, int vec_bytes, int peeled, int mode, int grid,
+                       int block, cudaStream_t st) {
+  if (peeled)
+    return mode == 0 ? launch_pdl(ua2a::ua2a_peel_kernel<0, 4>, grid, block, 0, st, p)
+                     : launch_pdl(ua2a::ua2a_peel_kernel<1, 4>, grid, block, 0, st, p);
   switch (vec_bytes) {
     case 16: return launch_vec_t<uint4>(p, mode, grid, block, st);
     case 8: return launch_vec_t<uint2>(p, mode, grid, block, st);
@@ -270,6 +273,38 @@ cudaError_t stage_allow_max_smem() {
   if (e == cudaSuccess) e = stage_allow_t<2>();
   if (e == cudaSuccess) e = stage_allow_t<1>();
   return e;
+}
+
+VecParams vec_params(const void* const* in, void* const* out, int nin, int nout, int64_t S, int w,
+                     int E, const ulysses_a2a_plan_t& pl, int64_t units, int64_t nb, int64_t nt,
+                     int nr, int nj, uint32_t r0, uint32_t r_stride, uint32_t j0, int64_t tile0) {
+  VecParams p{};
+  for (int k = 0; k < nin; ++k) p.in[k] = static_cast<const char*>(in[k]);
+  for (int k = 0; k < nout; ++k) p.out[k] = static_cast<char*>(out[k]);
+  p.S_local = S;
+  p.srow = pl.row_pitch * E / pl.vec_bytes;
+  if (pl.peeled) {
+    // whole 16-byte vectors between each run's head and tail
+    p.run = pl.row_bytes;
+    p.nv = pl.row_bytes / 16 - 1;
+    p.head = 16 - (int32_t)(reinterpret_cast<uintptr_t>(in[0]) & 15u);
+  } else {
+    p.nv = pl.row_bytes / pl.vec_bytes;
+  }
+  p.w = w;
+  p.rows_per_tile = (int32_t)pl.rows_per_tile;
+  p.units = (uint32_t)units;
+  p.order = pl.order;
+  p.tile0 = (uint32_t)tile0;
+  p.r0 = r0;
+  p.r_stride = r_stride;
+  p.j0 = j0;
+  p.div_T = ua2a::FastDiv((uint32_t)nt);
+  p.div_nr = ua2a::FastDiv((uint32_t)nr);
+  p.div_nj = ua2a::FastDiv((uint32_t)nj);
+  p.div_nb = ua2a::FastDiv((uint32_t)nb);
+  p.div_nv = ua2a::FastDiv((uint32_t)p.nv);
+  return p;
 }
 
 StageParams stage_params(int64_t S, int w, int ntensors, int E, const ulysses_a2a_plan_t& pl,
@@ -375,30 +410,15 @@ int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, in
     }
     return ULYSSES_A2A_OK;
   }
-  VecParams p{};
   const int nin = mode == 0 ? w : w * ntensors;
   const int nout = mode == 0 ? w * ntensors : w;
-  for (int k = 0; k < nin; ++k) p.in[k] = static_cast<const char*>(in[k]);
-  for (int k = 0; k < nout; ++k) p.out[k] = static_cast<char*>(out[k]);
-  p.S_local = S;
-  p.nv = pl.row_bytes / pl.vec_bytes;
-  p.srow = pl.row_pitch * ctx->elem_bytes / pl.vec_bytes;
-  p.w = w;
-  p.rows_per_tile = (int32_t)pl.rows_per_tile;
-  p.units = (uint32_t)units;
-  p.order = pl.order;
-  p.tile0 = (uint32_t)tile0;
-  p.r0 = (only_out >= 0 && mode == 0) ? (uint32_t)only_out : 0u;
-  p.r_stride = (only_out >= 0 && mode == 0) ? (uint32_t)w : 1u;
-  p.j0 = (only_out >= 0 && mode == 1) ? (uint32_t)only_out : 0u;
-  p.div_T = ua2a::FastDiv((uint32_t)nt);
-  p.div_nr = ua2a::FastDiv((uint32_t)nr);
-  p.div_nj = ua2a::FastDiv((uint32_t)nj);
-  p.div_nb = ua2a::FastDiv((uint32_t)nb);
-  p.div_nv = ua2a::FastDiv((uint32_t)p.nv);
+  VecParams p = vec_params(in, out, nin, nout, S, w, ctx->elem_bytes, pl, units, nb, nt, nr, nj,
+                           (only_out >= 0 && mode == 0) ? (uint32_t)only_out : 0u,
+                           (only_out >= 0 && mode == 0) ? (uint32_t)w : 1u,
+                           (only_out >= 0 && mode == 1) ? (uint32_t)only_out : 0u, tile0);
   for (int l = 0; l < launches; ++l) {
     p.b0 = chunked ? l : 0;
-    cudaError_t e = launch_vec(p, pl.vec_bytes, mode, grid, pl.block, st);
+    cudaError_t e = launch_vec(p, pl.vec_bytes, pl.peeled, mode, grid, pl.block, st);
     if (e != cudaSuccess) return cuda_fail(ctx, "VEC kernel launch", e);
     ctx->launches++;
   }

@@ -37,6 +37,7 @@ import torch
 import torch.distributed as dist
 
 from . import UlyssesA2A, _lib, mode0_local_tuple, output_shape
+from . import row_pitch as slab_row_pitch
 from ._lib import A2AError
 
 __all__ = ["PeerExchange", "NativePeer"]
@@ -400,7 +401,7 @@ class PeerExchange:
         elif tuple(out.shape) != oshape or out.dtype != x.dtype or out.device != x.device:
             raise ValueError(f"out must be {oshape} {x.dtype} on {x.device}")
         strided, dense = (x, out) if mode == 0 else (out, x)
-        pitch = UlyssesA2A._row_pitch([strided], allow_pitch=True)
+        pitch = slab_row_pitch([strided], allow_pitch=True)
         if not dense.is_contiguous():
             raise ValueError("the [B, S_local*w, H/w, D] slab must be contiguous")
         if B * S * H * D == 0:

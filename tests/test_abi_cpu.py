@@ -55,8 +55,9 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_plan_struct_layout_matches_header():
-    # int32 path, vec_bytes; 6 x int64; 6 x int32; int64; 2 x int32; int64 -> 104 bytes
-    assert ctypes.sizeof(_lib.PlanT) == 104
+    # int32 path, vec_bytes; 6 x int64; 6 x int32; int64; 2 x int32; int64; 2 x int32
+    # -> 112 bytes
+    assert ctypes.sizeof(_lib.PlanT) == 112
     # two pointers, 4 x int64, 4 x int32, int64 -> 72 bytes
     assert ctypes.sizeof(_lib.DescT) == 72
 
@@ -225,11 +226,80 @@ def test_vec_when_misaligned_pointer():
     outs[1] += 2
     rc, p, _ = ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E)
     assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 2  # 2-byte pieces: staged
+    assert p.peeled == 0                                            # (offsets differ)
     rc, p, _ = ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E, forced_path=PATH_VEC)
     assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 2
     outs[1] -= 2
     rc, p, msg = ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E, forced_path=PATH_TMA)
     assert rc == ERR_UNSUPPORTED and "aligned" in msg
+
+
+def test_runs_at_one_offset_are_peeled():
+    # slabs that all start the same number of bytes past a 16-byte boundary,
+    # runs and rows of whole 16-byte multiples: every run starts at that offset
+    # on both sides, so the vector kernel moves its 16-byte vectors between a
+    # peeled head and tail
+    w, B, S, H, D, E = 4, 2, 45, 8, 64, 2             # 256-byte runs
+    for off in (2, 4, 6, 8, 10, 14):
+        for mode in (0, 1):
+            ins, outs = fake_slabs(w, B * S * H * D * E)
+            ins, outs = [a + off for a in ins], [a + off for a in outs]
+            rc, p, _ = ulysses_a2a_plan(ins, outs, B, S, H, D, w, mode, 0, E)
+            assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 16 and p.peeled == 1
+            assert p.grid == p.units                  # one CTA per unit
+            rc, p, _ = ulysses_a2a_plan(ins, outs, B, S, H, D, w, mode, 1, E)
+            assert rc == OK and p.peeled == 1 and p.launches == B and p.grid == p.units
+            # forced staged stays staged; forced VEC takes the windows too
+            rc, p, _ = ulysses_a2a_plan(ins, outs, B, S, H, D, w, mode, 0, E,
+                                        forced_path=PATH_STAGED)
+            assert rc == OK and p.path == PATH_STAGED and p.peeled == 0
+            rc, p, _ = ulysses_a2a_plan(ins, outs, B, S, H, D, w, mode, 0, E, forced_path=PATH_VEC)
+            assert rc == OK and p.path == PATH_VEC and p.peeled == 1
+            # one slab off by another amount: offsets no longer match
+            outs[w - 1] += 2
+            rc, p, _ = ulysses_a2a_plan(ins, outs, B, S, H, D, w, mode, 0, E)
+            assert rc == OK and p.peeled == 0 and p.vec_bytes == 2
+    # aligned slabs keep whole 16-byte vectors (nothing to peel)
+    rc, p, _ = plan(4, 2, 45, 8, 64, forced_path=PATH_VEC)
+    assert rc == OK and p.vec_bytes == 16 and p.peeled == 0
+    # runs shorter than 64 bytes are not peeled
+    ins, outs = fake_slabs(2, 2 * 9 * 2 * 32 * 2)
+    ins, outs = [a + 2 for a in ins], [a + 2 for a in outs]
+    rc, p, _ = ulysses_a2a_plan(ins, outs, 2, 9, 2, 24, 2, 0, 0, 2)      # 48-byte runs
+    assert rc == OK and p.peeled == 0 and p.path == PATH_STAGED
+    rc, p, _ = ulysses_a2a_plan(ins, outs, 2, 9, 2, 32, 2, 0, 0, 2)      # 64-byte runs
+    assert rc == OK and p.peeled == 1
+    # runs whose offsets drift from row to row (66-byte runs in 132-byte rows,
+    # E = 1; 300-byte runs at w = 1) are not peeled
+    ins, outs = fake_slabs(2, 2 * 11 * 4 * 33)
+    rc, p, _ = ulysses_a2a_plan([a + 5 for a in ins], [a + 5 for a in outs], 2, 11, 4, 33, 2, 0,
+                                0, 1)
+    assert rc == OK and p.peeled == 0
+    ins, outs = fake_slabs(1, 2 * 9 * 4 * 40 * 2)
+    rc, p, _ = ulysses_a2a_plan([ins[0] + 10], [outs[0] + 10], 2, 9, 3, 50, 1, 0, 0, 2)
+    assert rc == OK and p.peeled == 0 and p.row_bytes == 300
+    rc, p, _ = ulysses_a2a_plan([ins[0] + 10], [outs[0] + 10], 2, 9, 4, 40, 1, 0, 0, 2)
+    assert rc == OK and p.peeled == 1 and p.row_bytes == 320
+
+
+def test_peeled_pitched_and_packed_plans():
+    # q of a packed [B, S, 3, H, D] buffer 6 bytes past a boundary, the dense
+    # side 6 bytes past too (rows of 3*H*D*E bytes, a multiple of 16): peeled
+    w, B, S, H, D, E = 4, 2, 37, 8, 64, 2
+    pitch = 3 * H * D
+    rc, p, _ = plan_ex(w, B, S, H, D, pitch, base=(1 << 40) + 6)
+    assert rc == OK and p.path == PATH_VEC and p.peeled == 1 and p.row_pitch == pitch
+    # a pitch that moves the offset by 4 bytes per row: not peeled
+    rc, p, _ = plan_ex(w, B, S, H, D, pitch + 2, base=(1 << 40) + 6)
+    assert rc == OK and p.peeled == 0
+    # T = 3 head-packed tensors, every slab 2 bytes off
+    step = (B * S * 3 * H * D * E + 4095) // 4096 * 4096
+    strided = [(1 << 40) + 2 + k * step for k in range(w)]
+    gathered = [(1 << 44) + 2 + k * step for k in range(3 * w)]
+    for mode in (0, 1):
+        ins, outs = (strided, gathered) if mode == 0 else (gathered, strided)
+        rc, p, _ = _lib.ulysses_a2a_plan_ex(ins, outs, B, S, H, D, w, mode, 0, E, ntensors=3)
+        assert rc == OK and p.path == PATH_VEC and p.peeled == 1
 
 
 def test_vec_when_too_many_ranks_for_tma():
@@ -663,11 +733,13 @@ def test_planner_invariants(w, hw, B, S, D, E, mode, chunked, path, rows, ntenso
         assert p.smem_bytes <= 220 * 1024
         assert p.grid == -(-p.units // p.chunk_units)
     else:
-        assert p.path == PATH_VEC
+        assert p.path == PATH_VEC and p.block == 256
+        # 4 KiB-aligned slabs share no offset past a 16-byte boundary: never peeled
+        assert p.peeled == 0
+        assert p.grid == p.units
         v = p.vec_bytes
         assert v in (1, 2, 4, 8, 16) and p.row_bytes % v == 0 and (p.row_pitch * E) % v == 0
         # AUTO leaves narrower vectors to the staged path unless a row is too long
         assert path == PATH_VEC or v >= 8 or not _one_row_fits_stage(hw * D * E, ntensors * w)
         # the widest width the run length and the pitch allow (pointers are 4 KiB aligned)
         assert v == 16 or (p.row_bytes % (2 * v) or (p.row_pitch * E) % (2 * v))
-        assert p.grid == p.units and p.block == 256

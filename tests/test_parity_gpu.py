@@ -736,6 +736,31 @@ def test_two_contexts_on_two_streams_concurrently():
             assert torch.equal(bits(yb[k].cpu()), bits(wb[k]))
 
 
+def test_default_stream_is_torchs_current_stream():
+    # run() without a stream queues on torch's current stream, inside a
+    # `torch.cuda.stream` block too: it must see the inputs written there after
+    # a long kernel on that stream (on any other stream it would read them early)
+    w, B, S, H, D = 2, 1, 64, 4, 128
+    cpu = normal_slabs((B, S, H, D), w, "bf16", seed0=911)
+    want = oracle.ulysses_a2a(cpu, 0)
+    s = torch.cuda.Stream()
+    with UlyssesA2A(0, 2) as a2a:
+        assert a2a._stream_handle(None) == torch.cuda.current_stream().cuda_stream
+        xs = [torch.zeros(B, S, H, D, dtype=torch.bfloat16, device="cuda") for _ in range(w)]
+        staged = [c.cuda() for c in cpu]
+        torch.cuda.synchronize()
+        with torch.cuda.stream(s):
+            assert a2a._stream_handle(None) == s.cuda_stream
+            torch.cuda._sleep(20_000_000)
+            for x, c in zip(xs, staged):
+                x.copy_(c)
+            ys = a2a.run(xs, 0)
+        s.synchronize()
+        a2a.status(s)
+        for k in range(w):
+            assert torch.equal(bits(ys[k].cpu()), bits(want[k]))
+
+
 # ---- edge sizes: empty, maximum rank count, box limits, a 2 GiB payload -------
 
 def test_empty_relayouts_launch_nothing():

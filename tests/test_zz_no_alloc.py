@@ -36,8 +36,8 @@ CASES = [
     (16, 3, 19, 16, 64, "bf16", 1, 0, VEC),       # the vector path, chunked
     (2, 2, 17, 4, 3, "bf16", 0, 0, STAGED),       # 12-byte runs: re-aligned in shared memory
     (2, 3, 17, 4, 3, "bf16", 1, 0, STAGED),       # chunked
-    (4, 2, 33, 8, 64, "bf16", 0, 2, STAGED),      # slab bases 2 bytes off 16
-    (4, 2, 33, 8, 64, "bf16", 1, 8, VEC),         # chunked, bases 8 bytes off 16: 8-byte vectors
+    (4, 2, 33, 8, 64, "bf16", 0, 2, VEC),         # every slab 2 bytes off 16: 16-byte windows
+    (4, 2, 33, 8, 64, "bf16", 1, 8, VEC),         # chunked, 8 bytes off: 16-byte windows
 ]
 
 
@@ -81,19 +81,21 @@ def test_noalloc_matches_the_oracle_and_run_on_two_calls_in_a_row(case, mode):
     cpu1 = make(in_shape, w, dtype, seed0=40 + mode)
     cpu2 = make(in_shape, w, dtype, seed0=60 + mode)
     first, second = _device_slabs(cpu1, off), _device_slabs(cpu2, off)
-    plan = UlyssesA2A(0, E).plan(first, mode, chunked=bool(chunked))
+    out1 = _poisoned(out_shape, first[0].dtype, w, off)
+    out2 = _poisoned(out_shape, first[0].dtype, w, off)
+    plan = UlyssesA2A(0, E).plan(first, mode, chunked=bool(chunked), out=out1)
     assert plan["path"] == path
 
     # expected outputs: the CPU oracle, and the regular entry point
     oracle1 = oracle.ulysses_a2a(cpu1, mode)
     oracle2 = oracle.ulysses_a2a(cpu2, mode)
     with UlyssesA2A(0, E) as a2a:
-        run1 = a2a.run(first, mode, chunked=bool(chunked))
-        run2 = a2a.run(second, mode, chunked=bool(chunked))
+        # the regular entry point on outputs at the same offset (same path)
+        ref1, ref2 = (_poisoned(out_shape, first[0].dtype, w, off) for _ in range(2))
+        run1 = a2a.run(first, mode, chunked=bool(chunked), out=ref1)
+        run2 = a2a.run(second, mode, chunked=bool(chunked), out=ref2)
         a2a.status()
 
-    out1 = _poisoned(out_shape, first[0].dtype, w, off)
-    out2 = _poisoned(out_shape, first[0].dtype, w, off)
     torch.cuda.synchronize()
     rc, msg = _noalloc(first, out1, (w, B, S, H, D), mode, chunked, E, stream)
     assert rc == _lib.OK, msg
