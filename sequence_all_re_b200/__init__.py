@@ -28,8 +28,8 @@ from ._lib import A2AError, PATH_AUTO, PATH_STAGED, PATH_TMA, PATH_VEC  # noqa: 
 # wraps the same handle in a Stream object)
 _raw_current_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
 
-__all__ = ["UlyssesA2A", "A2AError", "output_shape", "mode0_local_tuple", "marshal_slabs",
-           "PATH_AUTO", "PATH_TMA", "PATH_VEC", "PATH_STAGED"]
+__all__ = ["UlyssesA2A", "BoundRun", "A2AError", "output_shape", "mode0_local_tuple",
+           "marshal_slabs", "PATH_AUTO", "PATH_TMA", "PATH_VEC", "PATH_STAGED"]
 
 
 def output_shape(in_shape, mode: int, w: int) -> tuple:
@@ -125,6 +125,29 @@ def marshal_slabs(xs, mode: int, out, device_type: str, elem_bytes: int,
     return w, (B, S, H, D), out, in_ptrs, out_ptrs, pitch
 
 
+class BoundRun:
+    """One ``UlyssesA2A.run`` call whose arguments were checked and marshalled
+    when it was bound (``UlyssesA2A.bind``); calling it launches the re-layout
+    on ``stream`` (default: torch's current stream) and returns the outputs."""
+
+    def __init__(self, a2a, xs, out, in_ptrs, out_ptrs, dims, w, mode, chunked, pitch):
+        self._a2a = a2a
+        self._slabs = xs + list(out)
+        self._ptrs = in_ptrs + out_ptrs
+        self.out = out
+        self._desc = _lib.DescBuffer(max(len(in_ptrs), len(out_ptrs)))
+        B, S, H, D = dims
+        self._ref = self._desc.fill(in_ptrs, out_ptrs, B, S, H, D, w, mode, chunked, pitch)
+
+    def __call__(self, stream=None):
+        for t, ptr in zip(self._slabs, self._ptrs):
+            if t.data_ptr() != ptr:
+                raise ValueError("a bound slab was reallocated since bind(); bind again")
+        a2a = self._a2a
+        a2a._check(_lib.run_ex_ref(a2a._ctx, self._ref, a2a._stream_handle(stream)))
+        return self.out
+
+
 class UlyssesA2A:
     """A library context bound to one CUDA device and one element size."""
 
@@ -188,6 +211,16 @@ class UlyssesA2A:
         ref = self._desc.fill(ip, op, B, S, H, D, w, mode, int(chunked), pitch)
         self._check(_lib.run_ex_ref(self._ctx, ref, self._stream_handle(stream)))
         return out
+
+    def bind(self, xs, mode: int, chunked: bool = False, out=None) -> "BoundRun":
+        """``run`` with its slabs checked and marshalled once, for callers that
+        re-lay out the same buffers call after call: the returned object's
+        ``__call__(stream=None)`` re-reads only the slabs' data pointers (a slab
+        reallocated since, by ``resize_`` or ``set_``, raises) and launches.
+        The object keeps the slabs alive; their contents may change freely."""
+        w, dims, out, ip, op, pitch = marshal_slabs(xs, mode, out, "cuda", self.elem_bytes,
+                                                    allow_pitch=True)
+        return BoundRun(self, list(xs), out, ip, op, dims, w, mode, int(chunked), pitch)
 
     def run_packed(self, xs, mode: int, chunked: bool = False, out=None, stream=None):
         """Re-layout T tensors packed along the head dimension in one launch.

@@ -761,6 +761,57 @@ def test_default_stream_is_torchs_current_stream():
             assert torch.equal(bits(ys[k].cpu()), bits(want[k]))
 
 
+def test_bound_calls_follow_the_slabs_contents():
+    # bind once, call many times: each call re-lays out the slabs' current
+    # contents; a chunked binding launches once per plane
+    w, B, S, H, D = 4, 3, 77, 8, 64
+    with UlyssesA2A(0, 2) as a2a:
+        xs = [torch.empty(B, S, H, D, dtype=torch.bfloat16, device="cuda") for _ in range(w)]
+        for chunked in (False, True):
+            call = a2a.bind(xs, 0, chunked=chunked)
+            for seed in (931, 932):
+                cpu = normal_slabs((B, S, H, D), w, "bf16", seed0=seed)
+                for x, c in zip(xs, cpu):
+                    x.copy_(c)
+                n0 = a2a.launch_count
+                ys = call()
+                assert a2a.launch_count - n0 == (B if chunked else 1)
+                a2a.status()
+                want = oracle.ulysses_a2a(cpu, 0)
+                for r in range(w):
+                    assert torch.equal(bits(ys[r].cpu()), bits(want[r])), (chunked, seed, r)
+        # mode 1 back into row-pitched q slots of a packed buffer
+        pitch = 3 * H * D
+        packed = torch.full((w, B * S * pitch), float("nan"), dtype=torch.bfloat16, device="cuda")
+        views = [packed[k].as_strided((B, S, H, D), (S * pitch, pitch, D, 1)) for k in range(w)]
+        back = a2a.bind(ys, 1, out=views)
+        assert back() is back.out
+        a2a.status()
+        for j in range(w):
+            assert torch.equal(bits(views[j].cpu()), bits(cpu[j]))
+
+
+def test_bound_call_refuses_a_reallocated_slab():
+    w, B, S, H, D = 2, 1, 16, 4, 64
+    with UlyssesA2A(0, 2) as a2a:
+        xs = [torch.zeros(B, S, H, D, dtype=torch.bfloat16, device="cuda") for _ in range(w)]
+        call = a2a.bind(xs, 0)
+        call()
+        n0 = a2a.launch_count
+        xs[1].set_(torch.zeros(B, S, H, D, dtype=torch.bfloat16, device="cuda"))
+        with pytest.raises(ValueError, match="reallocated"):
+            call()
+        call = a2a.bind(xs, 0)                              # an output slab, this time
+        call()
+        n0 = a2a.launch_count
+        out = call.out[0]
+        out.resize_(2 * out.numel())                        # grows: a new allocation
+        with pytest.raises(ValueError, match="reallocated"):
+            call()
+        assert a2a.launch_count == n0                       # nothing was launched
+        a2a.status()
+
+
 # ---- edge sizes: empty, maximum rank count, box limits, a 2 GiB payload -------
 
 def test_empty_relayouts_launch_nothing():
