@@ -27,7 +27,8 @@ The same line carries, on one GPU:
                   (H = 8w, D = 128, B = 1), bf16 and fp32 U[-1,1), both modes;
                   the 512 MiB bf16 points (w_sweep_512MiB) run >= 1 s per mode;
   vec_shapes      shapes only the vector path takes: 200-byte and 6/12-byte
-                  rows, slab bases 8 and 2 bytes off a 16-byte boundary, w = 16;
+                  rows, slab bases 8 and 2 bytes off a 16-byte boundary (both sides,
+                  or the [B, S, H, D] side only), w = 16;
   e2e             the step through the host-buffer entry point (pinned slabs);
   cpu_baseline    the CPU oracle on a sample of the headline workload: the
                   OpenMP build on every host core, and the single-threaded one.
@@ -100,26 +101,38 @@ VEC_SHAPES = {
     "rows6B_w4_S2796202_H4_D3": (4, 1, 2796202, 4, 3, 2, 0),        # 6-byte runs
     "base8_w4_S8192_H24_D128": (4, 1, 8192, 24, 128, 2, 8),         # bases 8 B off
     "base2_w4_S8192_H24_D128": (4, 1, 8192, 24, 128, 2, 2),         # bases 2 B off
+    # [B, S, H, D] slabs 2 B off, the [B, S*w, H/w, D] slabs aligned
+    "base2in_w4_S8192_H24_D128": (4, 1, 8192, 24, 128, 2, 2, 0),
     "w16_S4096_H32_D128": (16, 1, 4096, 32, 128, 2, 0),             # w above the TMA limit
 }
 
 
 # Every workload --workload accepts: the table above, and the vector-path shapes
 # (element size and base offset as listed there).
-ALL_WORKLOADS = {**{n: dict(v, E=2, off=0) for n, v in WORKLOADS.items()},
-                 **{n: dict(w=v[0], B=v[1], S_local=v[2], H=v[3], D=v[4], E=v[5], off=v[6])
+# off: the [B, S, H, D] slabs' bytes past a 16-byte boundary; goff: the
+# [B, S*w, H/w, D] slabs' (the same unless a shape gives an eighth field).
+ALL_WORKLOADS = {**{n: dict(v, E=2, off=0, goff=0) for n, v in WORKLOADS.items()},
+                 **{n: dict(w=v[0], B=v[1], S_local=v[2], H=v[3], D=v[4], E=v[5], off=v[6],
+                            goff=v[7] if len(v) > 7 else v[6])
                     for n, v in VEC_SHAPES.items()}}
 DTYPE_OF = {2: "bf16", 4: "fp32"}
 INT_OF = {2: torch.int16, 4: torch.int32}
 
 
-def workload_key(w, B, S, H, D, path, E=2, off=0):
-    return f"{path}:w{w}_B{B}_S{S}_H{H}_D{D}_{DTYPE_OF[E]}" + (f"_base{off}" if off else "")
+def workload_key(w, B, S, H, D, path, E=2, off=0, goff=None):
+    goff = off if goff is None else goff
+    tail = (f"_base{off}" if off else "") if goff == off else f"_base{off}_gathered{goff}"
+    return f"{path}:w{w}_B{B}_S{S}_H{H}_D{D}_{DTYPE_OF[E]}" + tail
 
 
-def workload_name(w, B, S, H, D, chunked, E=2, off=0):
+def workload_name(w, B, S, H, D, chunked, E=2, off=0, goff=None):
     how = {0: "", 1: ", chunked per plane", 2: ", chunked through the staging window"}[chunked]
-    base = f", slab bases {off} bytes past a 16-byte boundary" if off else ""
+    goff = off if goff is None else goff
+    if goff != off:
+        base = (f", [B, S, H, D] slab bases {off} bytes and the others {goff} bytes past a "
+                "16-byte boundary")
+    else:
+        base = f", slab bases {off} bytes past a 16-byte boundary" if off else ""
     return (f"ulysses_a2a w={w} B={B} S_local={S} H={H} D={D} {DTYPE_OF[E]}{base}, "
             f"step = mode 0 + mode 1{how}")
 
@@ -176,7 +189,8 @@ def _code_only(text: str) -> str:
     return " ".join(text.split())
 
 
-KERNEL_FILES = {"tma": "kernels_tma.cuh", "vec": "kernels_vec.cuh", "staged": "kernels_stage.cuh"}
+KERNEL_FILES = {"tma": "kernels_tma.cuh", "vec": "kernels_vec.cuh", "peel": "kernels_peel.cuh",
+                "staged": "kernels_stage.cuh"}
 PATH_NAMES = {1: "tma", 2: "vec", 3: "staged"}
 LAUNCH_FIELDS = ("path", "rows_per_tile", "producers", "stages", "lookahead", "chunk_units",
                  "order", "grid", "block", "smem_bytes", "vec_bytes", "peeled")
@@ -203,7 +217,9 @@ def ncu_traffic(key, plan, chunked):
         return None, "no ncu traffic summary"
     if not entry:
         return None, "no ncu capture of this kernel and workload"
-    if entry.get("kernel_hash") != kernel_source_hash(key.split(":")[0]):
+    # the vector path's peeled and shifted kernels live in a file of their own
+    kernel = "peel" if plan.get("peeled") else key.split(":")[0]
+    if entry.get("kernel_hash") != kernel_source_hash(kernel):
         return None, "kernel changed since the ncu counters were taken"
     launch = entry.get("launch", {})
     if chunked or any(launch.get(f) != plan[f] for f in LAUNCH_FIELDS):
@@ -505,11 +521,13 @@ def vec_shape_block(device, peak, sampler, seconds=0.5):
 
     stream = torch.cuda.Stream(device)
     out = {}
-    for name, (w, B, S, H, D, E, off) in VEC_SHAPES.items():
+    for name, shape in VEC_SHAPES.items():
+        w, B, S, H, D, E, off = shape[:7]
+        goff = shape[7] if len(shape) > 7 else off
         dt = {2: "bf16", 4: "fp32"}[E]
         a2a = UlyssesA2A(device.index or 0, E)
         x = make_inputs(w, B, S, H, D, dt, device, offset_bytes=off)
-        y = empty_slabs(w, (B, S * w, H // w, D), x[0].dtype, device, off)
+        y = empty_slabs(w, (B, S * w, H // w, D), x[0].dtype, device, goff)
         z = empty_slabs(w, (B, S, H, D), x[0].dtype, device, off)
         p = a2a.plan(x, 0, out=y)
         P = w * B * S * H * D * E
@@ -519,7 +537,8 @@ def vec_shape_block(device, peak, sampler, seconds=0.5):
             raise SystemExit(f"vector-path shape {name}: round trip mismatch")
         out[name] = {"payload_bytes": P, "path": PATH_NAMES[p["path"]],
                      "vec_bytes": p["vec_bytes"], "peeled": p["peeled"],
-                     "row_bytes": p["row_bytes"], "base_offset_bytes": off, **res}
+                     "row_bytes": p["row_bytes"], "base_offset_bytes": off,
+                     "gathered_base_offset_bytes": goff, **res}
         # the other of the two paths, forced: the vector kernel where AUTO
         # re-aligns, the staged kernel where AUTO moves narrow vectors or
         # peeled 16-byte windows
@@ -669,20 +688,21 @@ def run_ours(args):
 
     sampler = ClockSampler(local_rank).start()
     wl = ALL_WORKLOADS[args.workload]
-    w, B, S, H, D, E, off = (wl[k] for k in ("w", "B", "S_local", "H", "D", "E", "off"))
+    w, B, S, H, D, E, off, goff = (wl[k] for k in ("w", "B", "S_local", "H", "D", "E", "off",
+                                                   "goff"))
     P = w * B * S * H * D * E
     a2a = UlyssesA2A(local_rank, E)
     a2a.set_path({"auto": 0, "tma": 1, "vec": 2, "staged": 3}[args.path])
     chunked = args.chunked
     stream = torch.cuda.Stream(device)
     x = make_inputs(w, B, S, H, D, DTYPE_OF[E], device, offset_bytes=off)
-    y = empty_slabs(w, (B, S * w, H // w, D), x[0].dtype, device, off)
+    y = empty_slabs(w, (B, S * w, H // w, D), x[0].dtype, device, goff)
     z = empty_slabs(w, (B, S, H, D), x[0].dtype, device, off)
     # mode 1 reads its own slabs (a seeded copy of mode 0's result), not y
     with torch.cuda.stream(stream):
         a2a.run(x, 0, out=y, stream=stream)
     torch.cuda.synchronize()
-    y2 = empty_slabs(w, (B, S * w, H // w, D), x[0].dtype, device, off)
+    y2 = empty_slabs(w, (B, S * w, H // w, D), x[0].dtype, device, goff)
     for a, b in zip(y2, y):
         a.copy_(b)
     plan = a2a.plan(x, 0, chunked=chunked, out=y)
@@ -709,7 +729,7 @@ def run_ours(args):
     avg_launch_ms = total_ms / launches
     bytes_per_launch = 2 * P * 2 * args.steps // launches       # 2 calls of 2P per step
     achieved = bytes_per_launch / (avg_launch_ms / 1e3) / 1e9
-    key = workload_key(w, B, S, H, D, PATH_NAMES[plan["path"]], E, off)
+    key = workload_key(w, B, S, H, D, PATH_NAMES[plan["path"]], E, off, goff)
     traffic_bytes, traffic_src = ncu_traffic(key, plan, chunked)
 
     extras = {}
@@ -836,7 +856,7 @@ def run_ours(args):
         "dtype": DTYPE_OF[E],
         "data": "synthetic",
         "config": {
-            "workload": workload_name(w, B, S, H, D, chunked, E, off),
+            "workload": workload_name(w, B, S, H, D, chunked, E, off, goff),
             "name": args.workload,
             "w": w, "B": B, "S_local": S, "H": H, "D": D,
             "payload_bytes_per_call": P,
@@ -1314,7 +1334,8 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": dt,
         "data": "synthetic",
-        "config": {"workload": workload_name(w, B, S, H, D, 0, E, wl["off"]), "name": args.workload,
+        "config": {"workload": workload_name(w, B, S, H, D, 0, E, wl["off"], wl["goff"]),
+                   "name": args.workload,
                    "w": w, "B": B, "S_local": S, "H": H, "D": D},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
                          "kind": "oracle", "sample": sample, "threads": threads,

@@ -80,7 +80,8 @@ extern "C" {
                                     (see plan_t.peeled)                     */
 #define ULYSSES_A2A_PATH_TMA  1  /* cp.async.bulk.tensor load -> smem -> store */
 #define ULYSSES_A2A_PATH_VEC  2  /* 16/8/4/2/1-byte LDG/STG copy, or 16-byte
-                                    vectors between peeled heads and tails   */
+                                    vectors between peeled heads and tails
+                                    (plan_t.peeled)                          */
 #define ULYSSES_A2A_PATH_STAGED 3 /* 16-byte LDG/STG, re-aligned in shared
                                     memory: runs or bases off 16 bytes     */
 
@@ -118,12 +119,15 @@ typedef struct ulysses_a2a_plan_t {
                                 robin); n = n consecutive units per CTA     */
     int64_t row_pitch;       /* elements between rows of the [B,S_local,H,D]
                                 side (H*D when dense)                       */
-    int32_t peeled;          /* VEC path: 1 = every slab starts the same a
-                                bytes past a 16-byte boundary and runs and
-                                rows are multiples of 16 bytes (runs of 64+):
-                                each run moves as 16-byte vectors between a
-                                head of 16 - a and a tail of a bytes, moved
-                                in aligned pieces by the same CTAs;
+    int32_t peeled;          /* VEC path, runs and rows multiples of 16
+                                bytes, runs of 64+: 1 = every slab starts the
+                                same a bytes past a 16-byte boundary; each run
+                                moves as 16-byte vectors between a head of
+                                16 - a and a tail of a bytes, moved in aligned
+                                pieces by the same CTAs. 2 = the input slabs
+                                share one offset and the output slabs another:
+                                each destination vector (and head and tail) is
+                                two aligned source vectors joined by a shift.
                                 vec_bytes is then 16                        */
     int32_t reserved;        /* 0                                             */
 } ulysses_a2a_plan_t;

@@ -15,6 +15,7 @@
 #include <string>
 #include <vector>
 
+#include "kernels_peel.cuh"
 #include "kernels_stage.cuh"
 #include "kernels_tma.cuh"
 #include "kernels_vec.cuh"

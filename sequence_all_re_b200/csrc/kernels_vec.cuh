@@ -20,16 +20,6 @@
 // multi-GPU exchange writes its own output slab (one per tensor when T
 // tensors are head-packed: head groups t*w + rank, r_stride = w) and reads
 // every rank's published input through peer mappings.
-//
-// Peeled variant (ua2a_peel_kernel): when every slab starts the same number
-// of bytes a past a 16-byte boundary and runs and rows are whole multiples of
-// 16 bytes, every run on either side starts a bytes past a boundary. The
-// whole-vector kernel could then only move 2-byte pieces (for a = 2), yet each
-// run is 16 - a head bytes, then L*E/16 - 1 aligned 16-byte vectors, then a
-// tail bytes, at the same offsets on both sides. The peeled kernel moves the
-// vectors as the whole-vector kernel does (shifted by the head), and each
-// run's head and tail in aligned pieces of 8, 4, 2 and 1 bytes held in the
-// same registers, all of a thread's loads in flight before its stores.
 #pragma once
 
 #include <cstdint>
@@ -87,7 +77,10 @@ struct VecParams {
   // the 8-byte mode-0 whole-vector kernel 8 registers (40 instead of 32), and
   // with them two of its eight resident CTAs per SM.
   int64_t run;           // bytes per run, L*E
-  int32_t head;          // bytes before a run's first 16-byte boundary
+  int32_t head;          // bytes before a run's first 16-byte boundary (on the
+                         // destination side)
+  int32_t shift;         // shifted launches: source offset minus destination
+                         // offset past their 16-byte boundaries, mod 16 (1..15)
 };
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) { return __ldcs(p); }
@@ -202,125 +195,6 @@ __global__ void __launch_bounds__(256, vec_min_blocks_per_sm<V>())
           const uint32_t c = e - row * nv;
           const int64_t off = (MODE == 0) ? (int64_t)e : (int64_t)row * strided_row + c;
           st_stream(dst + off, v[k]);
-        }
-      }
-    }
-  }
-}
-
-// Aligned pieces of bytes [x0, x1) of a 16-byte window, x0 = 0 or x1 = 16: a
-// run's head (x0 = its start offset, x1 = 16) or its tail (x0 = 0, x1 = the
-// tail's length). They split into at most one piece each of 8, 4, 2 and 1
-// bytes, whose offsets follow from the binary digits of x0 (head) or x1 (tail).
-struct WindowPieces {
-  uint32_t o8, o4, o2, o1;  // offsets in the window
-  bool f8, f4, f2, f1;      // which pieces exist
-};
-
-__device__ __forceinline__ WindowPieces window_pieces(uint32_t x0, uint32_t x1) {
-  WindowPieces w;
-  if (x0 > 0) {  // head: climb from x0 to 16 in growing aligned pieces
-    uint32_t q = x0;
-    w.f1 = q & 1; w.o1 = q; q += w.f1 ? 1 : 0;
-    w.f2 = q & 2; w.o2 = q; q += w.f2 ? 2 : 0;
-    w.f4 = q & 4; w.o4 = q; q += w.f4 ? 4 : 0;
-    w.f8 = q & 8; w.o8 = q;
-  } else {       // tail: [0, x1) in shrinking pieces
-    w.f8 = x1 & 8; w.o8 = 0;
-    w.f4 = x1 & 4; w.o4 = x1 & 8;
-    w.f2 = x1 & 2; w.o2 = x1 & 12;
-    w.f1 = x1 & 1; w.o1 = x1 & 14;
-  }
-  return w;
-}
-
-// The pieces of one partial window, held in four registers: the 8-byte piece
-// in x, y, the 4-byte in z, the 2- and 1-byte in w.
-__device__ __forceinline__ uint4 load_pieces(const char* win, const WindowPieces& pc) {
-  uint4 v = make_uint4(0u, 0u, 0u, 0u);
-  if (pc.f8) {
-    const uint2 t = ld_stream(reinterpret_cast<const uint2*>(win + pc.o8));
-    v.x = t.x;
-    v.y = t.y;
-  }
-  if (pc.f4) v.z = ld_stream(reinterpret_cast<const unsigned int*>(win + pc.o4));
-  if (pc.f2) v.w = ld_stream(reinterpret_cast<const unsigned short*>(win + pc.o2));
-  if (pc.f1) v.w |= (uint32_t)ld_stream(reinterpret_cast<const unsigned char*>(win + pc.o1)) << 16;
-  return v;
-}
-
-__device__ __forceinline__ void store_pieces(char* win, const WindowPieces& pc, uint4 v) {
-  if (pc.f8) st_stream(reinterpret_cast<uint2*>(win + pc.o8), make_uint2(v.x, v.y));
-  if (pc.f4) st_stream(reinterpret_cast<unsigned int*>(win + pc.o4), v.z);
-  if (pc.f2) st_stream(reinterpret_cast<unsigned short*>(win + pc.o2), (unsigned short)(v.w & 0xFFFFu));
-  if (pc.f1) st_stream(reinterpret_cast<unsigned char*>(win + pc.o1), (unsigned char)(v.w >> 16));
-}
-
-// The peeled variant (see the top of this file). p.nv = whole vectors per
-// run (L*E/16 - 1), p.srow in 16-byte vectors, p.head = 16 - a. A unit's
-// index space is its rows' whole vectors, then two edge items per row (the
-// run's head, then its tail), so the edge pieces of a unit are in flight with
-// its vectors and their 32-byte sectors, shared with the neighbouring vectors,
-// are read from DRAM once. A unit whose vectors would not be 16-byte aligned
-// on both sides is not touched (the host picks this kernel only when every
-// slab starts a bytes past a boundary and runs and rows are 16-byte multiples).
-template <int MODE, int U>
-__global__ void __launch_bounds__(256, kVecMinBlocksPerSm)
-    ua2a_peel_kernel(const __grid_constant__ VecParams p) {
-#if UA2A_PDL
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-#endif
-  const int64_t run = p.run;
-  const uint32_t nv = (uint32_t)p.nv;
-  const uint32_t nrun = (uint32_t)(run >> 4);  // 16-byte vectors between gathered rows
-  const int64_t strided_row = p.srow;          // 16-byte vectors between strided rows
-  const uint32_t a = 16u - (uint32_t)p.head;   // run start past its 16-byte boundary
-  const uint32_t step = blockDim.x * U;
-  for (uint32_t u = blockIdx.x; u < p.units; u += gridDim.x) {
-    const VecUnit x = vec_unit(p, u);
-    // first run of the unit, from its start (the vectors begin `head` bytes in)
-    const int64_t soff = (x.b * p.S_local + x.s0) * strided_row * 16 + (int64_t)x.r * run;
-    const int64_t goff = ((x.b * p.w + x.j) * p.S_local + x.s0) * run;
-    const char* sb = MODE == 0 ? p.in[x.j] + soff : p.in[x.r] + goff;
-    char* db = MODE == 0 ? p.out[x.r] + goff : p.out[x.j] + soff;
-    if (((((uintptr_t)sb + p.head) | ((uintptr_t)db + p.head)) & 15) != 0) continue;
-    const int64_t src_row = MODE == 0 ? strided_row : (int64_t)nrun;  // in vectors
-    const int64_t dst_row = MODE == 0 ? (int64_t)nrun : strided_row;
-    const uint4* src = reinterpret_cast<const uint4*>(sb + p.head);
-    uint4* dst = reinterpret_cast<uint4*>(db + p.head);
-    const uint32_t nvec = (uint32_t)(x.rows * nv);
-    const uint32_t n = nvec + 2u * (uint32_t)x.rows;
-    for (uint32_t base = threadIdx.x; base < n; base += step) {
-      uint4 v[U];
-#pragma unroll
-      for (int k = 0; k < U; ++k) {
-        const uint32_t e = base + k * blockDim.x;
-        if (e < nvec) {
-          const uint32_t row = fdiv(e, p.div_nv);
-          const uint32_t c = e - row * nv;
-          v[k] = ld_stream(src + (int64_t)row * src_row + c);
-        } else if (e < n) {
-          // head: window src[row*src_row] - 16, bytes [a, 16); tail: window
-          // src[row*src_row + nv], bytes [0, a)
-          const uint32_t i = e - nvec;
-          const char* w = reinterpret_cast<const char*>(src + (int64_t)(i >> 1) * src_row +
-                                                        ((i & 1) ? nv : 0)) - ((i & 1) ? 0 : 16);
-          v[k] = load_pieces(w, (i & 1) ? window_pieces(0, a) : window_pieces(a, 16));
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < U; ++k) {
-        const uint32_t e = base + k * blockDim.x;
-        if (e < nvec) {
-          const uint32_t row = fdiv(e, p.div_nv);
-          const uint32_t c = e - row * nv;
-          st_stream(dst + (int64_t)row * dst_row + c, v[k]);
-        } else if (e < n) {
-          const uint32_t i = e - nvec;
-          char* w = reinterpret_cast<char*>(dst + (int64_t)(i >> 1) * dst_row + ((i & 1) ? nv : 0)) -
-                    ((i & 1) ? 0 : 16);
-          store_pieces(w, (i & 1) ? window_pieces(0, a) : window_pieces(a, 16), v[k]);
         }
       }
     }

@@ -142,19 +142,23 @@ inline const char* tma_blocker(const void* const* in, void* const* out, int64_t 
 // mostly head and tail).
 constexpr int64_t kPeelMinRunBytes = 64;
 
-// Offset a (1..15) past a 16-byte boundary shared by every slab a call reads
-// or writes, when its runs (run_bytes) and rows (pitch_bytes) are whole
-// multiples of 16 bytes, so that every run on either side starts a bytes past
-// a boundary; else 0.
-inline int common_offset(const void* const* in, int nin, void* const* out, int nout,
-                         int64_t run_bytes, int64_t pitch_bytes) {
-  if (run_bytes % 16 != 0 || pitch_bytes % 16 != 0 || nin < 1) return 0;
-  const uintptr_t a = reinterpret_cast<uintptr_t>(in[0]) & 15u;
+// Offsets past a 16-byte boundary shared by every input slab (*a_in) and by
+// every output slab (*a_out) of a call whose runs (run_bytes) and rows
+// (pitch_bytes) are whole multiples of 16 bytes: every run then starts *a_in
+// bytes past a boundary on the input side and *a_out on the output side.
+// False when the slabs of a side differ, or a run or a row is no multiple of 16.
+inline bool side_offsets(const void* const* in, int nin, void* const* out, int nout,
+                         int64_t run_bytes, int64_t pitch_bytes, int* a_in, int* a_out) {
+  if (run_bytes % 16 != 0 || pitch_bytes % 16 != 0 || nin < 1 || nout < 1) return false;
+  const uintptr_t ai = reinterpret_cast<uintptr_t>(in[0]) & 15u;
+  const uintptr_t ao = reinterpret_cast<uintptr_t>(out[0]) & 15u;
   for (int k = 0; k < nin; ++k)
-    if ((reinterpret_cast<uintptr_t>(in[k]) & 15u) != a) return 0;
+    if ((reinterpret_cast<uintptr_t>(in[k]) & 15u) != ai) return false;
   for (int k = 0; k < nout; ++k)
-    if ((reinterpret_cast<uintptr_t>(out[k]) & 15u) != a) return 0;
-  return (int)a;
+    if ((reinterpret_cast<uintptr_t>(out[k]) & 15u) != ao) return false;
+  *a_in = (int)ai;
+  *a_out = (int)ao;
+  return true;
 }
 
 // Geometry of the re-aligning (staged) path for runs of R bytes, ng head
@@ -502,17 +506,21 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
       set_err(err, "one VEC tile exceeds 2^31 vectors");
       return ULYSSES_A2A_ERR_UNSUPPORTED;
     }
-    // Runs that start at one offset past a 16-byte boundary on both sides move
-    // as 16-byte vectors between a peeled head and tail (not one-output
-    // launches, whose inputs are other ranks' windows).
     // one CTA per unit (units < 2^31 was checked above), or a grid-stride
     // grid of ctas_per_sm CTAs per SM when that knob is set
     int64_t g = tune.ctas_per_sm > 0 ? (int64_t)num_sms * tune.ctas_per_sm : units;
-    const bool peel = v < 16 && only_out < 0 && forced_path != ULYSSES_A2A_PATH_STAGED &&
-                      row_bytes >= kPeelMinRunBytes &&
-                      common_offset(in, nin, out, nout, row_bytes, pitch * E) != 0;
-    p->vec_bytes = peel ? 16 : v;
-    p->peeled = peel ? 1 : 0;
+    // Runs that start at one offset past a 16-byte boundary on each side move
+    // as 16-byte destination vectors between a peeled head and tail: straight
+    // when the two offsets are equal (peeled = 1), each vector joined from two
+    // aligned source vectors when they differ (peeled = 2). Not one-output
+    // launches, whose inputs are other ranks' windows.
+    int a_in = 0, a_out = 0;
+    const bool sides = v < 16 && only_out < 0 && forced_path != ULYSSES_A2A_PATH_STAGED &&
+                       row_bytes >= kPeelMinRunBytes &&
+                       side_offsets(in, nin, out, nout, row_bytes, pitch * E, &a_in, &a_out);
+    const int peeled = !sides ? 0 : (a_in == a_out ? 1 : 2);
+    p->vec_bytes = peeled ? 16 : v;
+    p->peeled = peeled;
     p->stages = 0;
     p->lookahead = 0;
     p->producers = 0;
@@ -525,7 +533,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     // except one-output launches.
     const bool forced_stage = forced_path == ULYSSES_A2A_PATH_STAGED;
     if (forced_stage ||
-        (forced_path == ULYSSES_A2A_PATH_AUTO && !peel && v <= kStageMaxPiece && only_out < 0)) {
+        (forced_path == ULYSSES_A2A_PATH_AUTO && !peeled && v <= kStageMaxPiece && only_out < 0)) {
       StageGeometry sg;
       if (stage_geometry(row_bytes, (int64_t)w * ntensors, S, tune.rows_per_tile, &sg)) {
         const int64_t nbl = chunked ? 1 : B;

@@ -223,8 +223,20 @@ cudaError_t launch_vec_t(const VecParams& p, int mode, int grid, int block, cuda
                    : launch_pdl(ua2a::ua2a_vec_kernel<V, 1, 4>, grid, block, 0, st, p);
 }
 
+template <int MODE>
+cudaError_t launch_shift_t(const VecParams& p, int grid, int block, cudaStream_t st) {
+  switch (p.shift >> 2) {
+    case 0: return launch_pdl(ua2a::ua2a_shift_kernel<MODE, 0>, grid, block, 0, st, p);
+    case 1: return launch_pdl(ua2a::ua2a_shift_kernel<MODE, 1>, grid, block, 0, st, p);
+    case 2: return launch_pdl(ua2a::ua2a_shift_kernel<MODE, 2>, grid, block, 0, st, p);
+    default: return launch_pdl(ua2a::ua2a_shift_kernel<MODE, 3>, grid, block, 0, st, p);
+  }
+}
+
 cudaError_t launch_vec(const VecParams& p, int vec_bytes, int peeled, int mode, int grid,
                        int block, cudaStream_t st) {
+  if (peeled == 2)
+    return mode == 0 ? launch_shift_t<0>(p, grid, block, st) : launch_shift_t<1>(p, grid, block, st);
   if (peeled)
     return mode == 0 ? launch_pdl(ua2a::ua2a_peel_kernel<0, 4>, grid, block, 0, st, p)
                      : launch_pdl(ua2a::ua2a_peel_kernel<1, 4>, grid, block, 0, st, p);
@@ -284,10 +296,14 @@ VecParams vec_params(const void* const* in, void* const* out, int nin, int nout,
   p.S_local = S;
   p.srow = pl.row_pitch * E / pl.vec_bytes;
   if (pl.peeled) {
-    // whole 16-byte vectors between each run's head and tail
+    // whole 16-byte destination vectors between each run's head and tail; the
+    // source runs start `shift` bytes further past their boundary
+    const int32_t a_in = (int32_t)(reinterpret_cast<uintptr_t>(in[0]) & 15u);
+    const int32_t a_out = (int32_t)(reinterpret_cast<uintptr_t>(out[0]) & 15u);
     p.run = pl.row_bytes;
-    p.nv = pl.row_bytes / 16 - 1;
-    p.head = 16 - (int32_t)(reinterpret_cast<uintptr_t>(in[0]) & 15u);
+    p.nv = pl.row_bytes / 16 - (a_out ? 1 : 0);
+    p.head = (16 - a_out) & 15;
+    p.shift = (a_in - a_out) & 15;
   } else {
     p.nv = pl.row_bytes / pl.vec_bytes;
   }

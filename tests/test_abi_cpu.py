@@ -282,6 +282,35 @@ def test_runs_at_one_offset_are_peeled():
     assert rc == OK and p.peeled == 1 and p.row_bytes == 320
 
 
+def test_inputs_and_outputs_at_two_offsets_are_shifted():
+    # the input slabs share one offset past a 16-byte boundary, the outputs
+    # another: peeled = 2 (each destination vector joined from two aligned
+    # source vectors), for every pair of different offsets
+    w, B, S, H, D, E = 4, 2, 45, 8, 64, 2
+    ins, outs = fake_slabs(w, B * S * H * D * E, gap=256)
+    for a_in in range(0, 16, 2):
+        for a_out in range(0, 16, 2):
+            if a_in == a_out:
+                continue
+            for mode in (0, 1):
+                rc, p, _ = ulysses_a2a_plan([a + a_in for a in ins], [a + a_out for a in outs],
+                                            B, S, H, D, w, mode, 0, E)
+                assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 16 and p.peeled == 2
+                assert p.grid == p.units
+    # one output off by a third amount: no shared output offset, so staged
+    o2 = [a + 4 for a in outs]
+    o2[1] += 2
+    rc, p, _ = ulysses_a2a_plan([a + 2 for a in ins], o2, B, S, H, D, w, 0, 0, E)
+    assert rc == OK and p.peeled == 0 and p.path == PATH_STAGED
+    # forced staged stays staged; runs under 64 bytes are not shifted
+    rc, p, _ = ulysses_a2a_plan([a + 2 for a in ins], outs, B, S, H, D, w, 0, 0, E,
+                                forced_path=PATH_STAGED)
+    assert rc == OK and p.path == PATH_STAGED
+    ins2, outs2 = fake_slabs(2, 2 * 9 * 2 * 24 * 2, gap=256)
+    rc, p, _ = ulysses_a2a_plan([a + 2 for a in ins2], outs2, 2, 9, 2, 24, 2, 0, 0, 2)
+    assert rc == OK and p.peeled == 0
+
+
 def test_peeled_pitched_and_packed_plans():
     # q of a packed [B, S, 3, H, D] buffer 6 bytes past a boundary, the dense
     # side 6 bytes past too (rows of 3*H*D*E bytes, a multiple of 16): peeled

@@ -11,11 +11,13 @@ import bench  # noqa: E402
 from sequence_all_re_b200 import _lib  # noqa: E402
 
 
-def plan_dict(w, B, S, H, D, path=_lib.PATH_AUTO, E=2, off=0):
-    """The plan of a call whose slabs sit `off` bytes past 4 KiB boundaries."""
+def plan_dict(w, B, S, H, D, path=_lib.PATH_AUTO, E=2, off=0, goff=None):
+    """The plan of a mode-0 call whose input slabs sit `off` bytes past 4 KiB
+    boundaries and whose output slabs sit `goff` (default: `off`) bytes past."""
+    goff = off if goff is None else goff
     step = (B * S * H * D * E + 4095) // 4096 * 4096 + 4096
     ins = [(1 << 40) + k * step + off for k in range(w)]
-    outs = [(1 << 40) + (w + k) * step + off for k in range(w)]
+    outs = [(1 << 40) + (w + k) * step + goff for k in range(w)]
     rc, p, msg = _lib.ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E, forced_path=path)
     assert rc == _lib.OK, msg
     return p.as_dict()
@@ -29,13 +31,14 @@ def test_committed_captures_match_the_current_kernels_and_plans():
         w, B, S, H, D = (int(part[1:]) for part in parts[:5])
         E = {"bf16": 2, "fp32": 4}[parts[5]]
         off = int(parts[6][4:]) if len(parts) > 6 else 0
+        goff = int(parts[7][8:]) if len(parts) > 7 else off     # "_gathered<n>"
         # the planner chooses this kernel for the captured shape (AUTO) ...
-        assert plan_dict(w, B, S, H, D, _lib.PATH_AUTO, E, off)["path"] == {
+        assert plan_dict(w, B, S, H, D, _lib.PATH_AUTO, E, off, goff)["path"] == {
             "tma": _lib.PATH_TMA, "vec": _lib.PATH_VEC, "staged": _lib.PATH_STAGED}[path] or (
             key == "vec:w4_B1_S8192_H24_D128_bf16")          # the VEC capture of a TMA shape
         # ... and the capture matches its launch shape and code
         p = plan_dict(w, B, S, H, D, {"tma": _lib.PATH_TMA, "vec": _lib.PATH_VEC,
-                                      "staged": _lib.PATH_STAGED}[path], E, off)
+                                      "staged": _lib.PATH_STAGED}[path], E, off, goff)
         got, why = bench.ncu_traffic(key, p, 0)
         assert why == "ncu", (key, why)
         assert got == entry["dram_bytes_per_launch"]
@@ -85,8 +88,22 @@ def test_fractions_count_twice_the_payload():
 
 
 def test_vector_shapes_are_named_by_their_sizes_and_leave_the_tma_path():
-    for name, (w, B, S, H, D, E, off) in bench.VEC_SHAPES.items():
+    for name, shape in bench.VEC_SHAPES.items():
+        w, B, S, H, D, E, off = shape[:7]
+        goff = shape[7] if len(shape) > 7 else off
         assert f"w{w}_" in name and f"S{S}_" in name and f"H{H}_" in name and f"D{D}" in name
         row = (H // w) * D * E
-        tma_blocked = row % 16 != 0 or off % 16 != 0 or w > 8
+        tma_blocked = row % 16 != 0 or off % 16 != 0 or goff % 16 != 0 or w > 8
         assert tma_blocked, name
+        wl = bench.ALL_WORKLOADS[name]
+        assert (wl["off"], wl["goff"]) == (off, goff)
+
+
+def test_one_sided_offsets_are_keyed_apart():
+    assert bench.workload_key(4, 1, 8, 24, 128, "vec", 2, 2) == "vec:w4_B1_S8_H24_D128_bf16_base2"
+    assert bench.workload_key(4, 1, 8, 24, 128, "vec", 2, 2, 0) == \
+        "vec:w4_B1_S8_H24_D128_bf16_base2_gathered0"
+    # the bench's one-sided shape takes the shifted vector kernel in both modes
+    w, B, S, H, D, E, off, goff = bench.VEC_SHAPES["base2in_w4_S8192_H24_D128"]
+    p = plan_dict(w, B, S, H, D, _lib.PATH_AUTO, E, off, goff)
+    assert p["path"] == _lib.PATH_VEC and p["peeled"] == 2

@@ -38,11 +38,13 @@ def _offset_slabs(cpu, offset):
     return out
 
 
-def _check(a2a, xs_cpu, mode, offset, chunked, expect_peeled=True):
+def _check(a2a, xs_cpu, mode, offset, chunked, expect_peeled=True, out_offset=None):
+    """Inputs `offset` bytes past a boundary, outputs `out_offset` (default: the
+    same); the plan must be the peeled form expected (1 = one offset, 2 = two)."""
     w = len(xs_cpu)
     xs = _offset_slabs(xs_cpu, offset)
     oshape = oracle.output_shape(tuple(xs_cpu[0].shape), mode, w)
-    g = Guarded(oshape, xs_cpu[0].dtype, w, offset=offset)
+    g = Guarded(oshape, xs_cpu[0].dtype, w, offset=offset if out_offset is None else out_offset)
     p = a2a.plan(xs, mode, chunked=chunked, out=g.slabs)
     assert p["path"] == PATH_VEC and p["peeled"] == int(expect_peeled), p
     a2a.run(xs, mode, chunked=chunked, out=g.slabs)
@@ -86,6 +88,67 @@ def test_slabs_at_one_offset_every_offset(case, mode):
         # the vector path forced takes the same windows
         a2a.set_path(PATH_VEC)
         _check(a2a, xs, mode, _offsets(E)[0], False)
+
+
+@pytest.mark.parametrize("E", [1, 2, 4, 8])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_inputs_and_outputs_at_two_offsets(E, mode):
+    # every pair of different offsets (multiples of E) on the two sides: each
+    # destination vector, head and tail is joined from two aligned source
+    # vectors (peeled = 2)
+    w, B, S, H, D = 4, 2, 29, 8, 128 // E
+    shape = slab_shape(mode, w, B, S, H, D)
+    xs = [t.view(INT[E]).reshape(shape)
+          for t in random_byte_slabs(shape[:-1] + (shape[-1] * E,), w, seed0=770 + E + mode)]
+    offs = list(range(0, 16, E))
+    with UlyssesA2A(0, E) as a2a:
+        for a_in in offs:
+            for a_out in offs:
+                if a_in != a_out:
+                    _check(a2a, xs, mode, a_in, (a_in + a_out) % 2 == 0, expect_peeled=2,
+                           out_offset=a_out)
+
+
+def test_shifted_round_trip_chunked_and_pitched():
+    # inputs 2 bytes off, outputs 10 off, chunked per plane; then mode 1 from
+    # aligned slabs into q slots of a packed buffer 6 bytes off
+    w, B, S, H, D = 4, 3, 100, 8, 128
+    xs = normal_slabs((B, S, H, D), w, "bf16", seed0=780)
+    with UlyssesA2A(0, 2) as a2a:
+        ys = _check(a2a, xs, 0, 2, True, expect_peeled=2, out_offset=10)
+        pitch = 3 * H * D
+        bufs = _offset_slabs([torch.full((B * S * pitch,), float("nan"), dtype=torch.bfloat16)
+                              for _ in range(w)], 6)
+        views = [t.as_strided((B, S, H, D), (S * pitch, pitch, D, 1)) for t in bufs]
+        dense = [y.cuda() for y in ys]
+        p = a2a.plan(dense, 1, out=views)
+        assert p["peeled"] == 2 and p["row_pitch"] == pitch
+        a2a.run(dense, 1, out=views)
+        a2a.status()
+        for j in range(w):
+            got = bufs[j].cpu().view(B * S, pitch)
+            assert torch.equal(bits(got[:, :H * D].contiguous()), bits(xs[j].reshape(B * S, H * D)))
+            assert bool(torch.isnan(got[:, H * D:].float()).all()), "another slot was written"
+
+
+def test_shifted_packed_tensors():
+    w, B, S, H, D, T = 4, 2, 41, 8, 64, 3
+    packed_cpu = normal_slabs((B, S, T, H, D), w, "bf16", seed0=790)
+    flat = [t.reshape(-1) for t in packed_cpu]
+    with UlyssesA2A(0, 2) as a2a:
+        packed = _offset_slabs(packed_cpu, 14)
+        outs = [[_offset_slabs([torch.empty(B, S * w, H // w, D, dtype=torch.bfloat16)], 4)[0]
+                 for _ in range(w)] for _ in range(T)]
+        flat_out = [o.data_ptr() for per_t in outs for o in per_t]
+        rc, p, msg = _lib.ulysses_a2a_plan_ex([t.data_ptr() for t in packed], flat_out, B, S, H, D,
+                                              w, 0, 0, 2, ntensors=T)
+        assert rc == _lib.OK and p.peeled == 2, msg
+        a2a.run_packed(packed, 0, out=outs)
+        a2a.status()
+        for t in range(T):
+            want = oracle.ulysses_a2a_pitched(flat, 0, w, B, S, H, D, T * H * D, offset=t * H * D)
+            for r in range(w):
+                assert torch.equal(bits(outs[t][r].cpu()).reshape(-1), bits(want[r])), (t, r)
 
 
 def test_round_trip_through_peeled_launches():
@@ -213,10 +276,11 @@ def test_peeled_launch_captures_into_a_cuda_graph():
 
 def test_randomized_shared_offset_cases():
     """60 seeded random cases: rank counts 1..16, ragged S_local, element sizes
-    1/2/4/8, one random base offset shared by every slab, random unit sizes;
-    each checked against the oracle whichever path the planner takes, and
-    the peeled form required wherever its conditions hold (an offset, runs
-    of 64 bytes or more and a multiple of 16)."""
+    1/2/4/8, a random base offset for the inputs and, half the time, another
+    for the outputs, random unit sizes; each checked against the oracle
+    whichever path the planner takes, and the peeled form (1 for one offset,
+    2 for two) required wherever its conditions hold (an offset, runs of 64
+    bytes or more and a multiple of 16)."""
     rng = random.Random(760)
     n_peeled = 0
     ctxs = {}
@@ -230,6 +294,7 @@ def test_randomized_shared_offset_cases():
             B, S = rng.randint(1, 3), rng.randint(1, 70)
             mode = rng.choice([0, 1])
             off = rng.randrange(0, 16, E) if E < 16 else 0
+            off_out = off if rng.random() < 0.5 else rng.randrange(0, 16, E)
             shape = slab_shape(mode, w, B, S, H, D)
             xs = [t.view(INT[E]).reshape(shape)
                   for t in random_byte_slabs(shape[:-1] + (shape[-1] * E,), w, seed0=900 + case)]
@@ -238,12 +303,12 @@ def test_randomized_shared_offset_cases():
             a2a.set_tuning(rows_per_tile=rng.choice([0, 0, 1, 5]))
             dev = _offset_slabs(xs, off)
             oshape = oracle.output_shape(shape, mode, w)
-            g = Guarded(oshape, xs[0].dtype, w, offset=off)
+            g = Guarded(oshape, xs[0].dtype, w, offset=off_out)
             chunked = rng.choice([False, True])
             p = a2a.plan(dev, mode, chunked=chunked, out=g.slabs)
             run_bytes = hw * D * E
-            if off % 16 and run_bytes >= 64 and run_bytes % 16 == 0:
-                assert p["peeled"] == 1, (case, p)
+            if (off or off_out) and run_bytes >= 64 and run_bytes % 16 == 0:
+                assert p["peeled"] == (1 if off == off_out else 2), (case, p)
             n_peeled += p["peeled"]
             a2a.run(dev, mode, chunked=chunked, out=g.slabs)
             a2a.status()
