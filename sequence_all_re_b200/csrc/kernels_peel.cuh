@@ -56,8 +56,9 @@ __device__ __forceinline__ WindowPieces window_pieces(uint32_t x0, uint32_t x1) 
   return w;
 }
 
-// The pieces of one partial window, held in four registers: the 8-byte piece
-// in x, y, the 4-byte in z, the 2- and 1-byte in w.
+// The pieces of one partial window, packed in four registers: the 8-byte
+// piece in x, y, the 4-byte in z, the 2- and 1-byte in w (store_pieces takes
+// them back from there).
 __device__ __forceinline__ uint4 load_pieces(const char* win, const WindowPieces& pc) {
   uint4 v = make_uint4(0u, 0u, 0u, 0u);
   if (pc.f8) {
@@ -86,8 +87,19 @@ __device__ __forceinline__ void store_pieces(char* win, const WindowPieces& pc, 
 // are read from DRAM once. A unit whose vectors would not be 16-byte aligned
 // on both sides is not touched (the host picks this kernel only when every
 // slab starts a bytes past a boundary and runs and rows are 16-byte multiples).
+// Resident CTAs per SM the peeled kernel's launch bound asks for, and its
+// items per thread (build-time switches). More bytes in flight lose here, as
+// on the TMA path: slab bases 2 bytes off, 4 items at 6 CTAs per SM: 0.96 /
+// 0.94 of the copy bandwidth; 6 at 5: 0.87 / 0.86; 8 at 4: 0.79 / 0.79.
+#ifndef UA2A_PEEL_MIN_BLOCKS
+#define UA2A_PEEL_MIN_BLOCKS 6
+#endif
+#ifndef UA2A_PEEL_ITEMS
+#define UA2A_PEEL_ITEMS 4
+#endif
+
 template <int MODE, int U>
-__global__ void __launch_bounds__(256, kVecMinBlocksPerSm)
+__global__ void __launch_bounds__(256, UA2A_PEEL_MIN_BLOCKS)
     ua2a_peel_kernel(const __grid_constant__ VecParams p) {
 #if UA2A_PDL
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -149,6 +161,28 @@ __global__ void __launch_bounds__(256, kVecMinBlocksPerSm)
   }
 }
 
+// Word i (0..3) of v.
+__device__ __forceinline__ uint32_t word_of(const uint4& v, uint32_t i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// The pieces of a window held at their own byte positions in v (byte x of the
+// window in byte x of v, as a funnel shift leaves them), stored at win. Every
+// piece is aligned to its size, so it lies within one word, or two for the
+// 8-byte piece.
+__device__ __forceinline__ void store_window_pieces(char* win, const WindowPieces& pc, const uint4& v) {
+  if (pc.f8)
+    st_stream(reinterpret_cast<uint2*>(win + pc.o8),
+              make_uint2(word_of(v, pc.o8 >> 2), word_of(v, (pc.o8 >> 2) + 1)));
+  if (pc.f4) st_stream(reinterpret_cast<unsigned int*>(win + pc.o4), word_of(v, pc.o4 >> 2));
+  if (pc.f2)
+    st_stream(reinterpret_cast<unsigned short*>(win + pc.o2),
+              (unsigned short)(word_of(v, pc.o2 >> 2) >> (8 * (pc.o2 & 3))));
+  if (pc.f1)
+    st_stream(reinterpret_cast<unsigned char*>(win + pc.o1),
+              (unsigned char)(word_of(v, pc.o1 >> 2) >> (8 * (pc.o1 & 3))));
+}
+
 // Bytes d .. d + 15 of the 32 bytes a, b (a first), for d = 4*Q + sh/8:
 // word i of the result is the funnel shift of words Q + i, Q + i + 1.
 template <int Q>
@@ -168,14 +202,27 @@ __device__ __forceinline__ uint4 funnel16(const uint4& a, const uint4& b, uint32
 // A unit whose aligned addresses do not line up is not touched (the host
 // picks this kernel only when every slab on each side shares that side's
 // offset and runs and rows are 16-byte multiples).
+// Items per thread in flight (two loads each) and resident CTAs per SM the
+// launch bound asks for (build-time switches). 4 items at 5 CTAs per SM (up to
+// 51 registers) keep 80 KB of distinct source vectors in flight per SM; 2 at 6
+// kept 48 KB and left the kernel waiting on memory (slab bases 2 bytes off on
+// one side: 0.91 / 0.88 of the copy bandwidth against 1.00 / 0.94; 3 at 5:
+// 1.01 / 0.93; 4 at 4: 0.92 / 0.87).
+#ifndef UA2A_SHIFT_ITEMS
+#define UA2A_SHIFT_ITEMS 4
+#endif
+#ifndef UA2A_SHIFT_MIN_BLOCKS
+#define UA2A_SHIFT_MIN_BLOCKS 5
+#endif
+
 template <int MODE, int Q>
-__global__ void __launch_bounds__(256, kVecMinBlocksPerSm)
+__global__ void __launch_bounds__(256, UA2A_SHIFT_MIN_BLOCKS)
     ua2a_shift_kernel(const __grid_constant__ VecParams p) {
 #if UA2A_PDL
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
 #endif
-  constexpr int U = 2;  // items per thread in flight (two loads each)
+  constexpr int U = UA2A_SHIFT_ITEMS;
   const int64_t run = p.run;
   const uint32_t nv = (uint32_t)p.nv;
   const uint32_t nrun = (uint32_t)(run >> 4);
@@ -236,8 +283,8 @@ __global__ void __launch_bounds__(256, kVecMinBlocksPerSm)
           const uint32_t i = e - nvec;
           const bool tail = i & 1;
           char* w = reinterpret_cast<char*>(dst + (int64_t)(i >> 1) * dst_row + (tail ? (int64_t)nv : -1));
-          store_pieces(w, tail ? window_pieces(0, ad) : window_pieces(ad, 16),
-                       funnel16<Q>(v0[k], v1[k], sh));
+          store_window_pieces(w, tail ? window_pieces(0, ad) : window_pieces(ad, 16),
+                              funnel16<Q>(v0[k], v1[k], sh));
         }
       }
     }

@@ -238,8 +238,8 @@ cudaError_t launch_vec(const VecParams& p, int vec_bytes, int peeled, int mode, 
   if (peeled == 2)
     return mode == 0 ? launch_shift_t<0>(p, grid, block, st) : launch_shift_t<1>(p, grid, block, st);
   if (peeled)
-    return mode == 0 ? launch_pdl(ua2a::ua2a_peel_kernel<0, 4>, grid, block, 0, st, p)
-                     : launch_pdl(ua2a::ua2a_peel_kernel<1, 4>, grid, block, 0, st, p);
+    return mode == 0 ? launch_pdl(ua2a::ua2a_peel_kernel<0, UA2A_PEEL_ITEMS>, grid, block, 0, st, p)
+                     : launch_pdl(ua2a::ua2a_peel_kernel<1, UA2A_PEEL_ITEMS>, grid, block, 0, st, p);
   switch (vec_bytes) {
     case 16: return launch_vec_t<uint4>(p, mode, grid, block, st);
     case 8: return launch_vec_t<uint2>(p, mode, grid, block, st);

@@ -227,12 +227,12 @@ def test_nan_payloads_and_signed_zero_survive():
 
 # ---- alignment: misaligned slabs take the narrower vector path --------------
 
-@pytest.mark.parametrize("offset,vec", [(8, 8), (4, 4), (2, 2), (1, 1)])
-def test_misaligned_pointers_select_narrower_pieces(offset, vec):
-    # a base off the 16-byte boundary: AUTO moves 8-byte vectors, or re-aligns
-    # through shared memory in pieces of the alignment the bases allow when
-    # that is 4 bytes or less; the vector path, when forced, uses vectors of
-    # that width
+@pytest.mark.parametrize("offset", [8, 4, 2, 1])
+def test_one_sided_offsets_take_the_shifted_vector_kernel(offset):
+    # slabs off the 16-byte boundary on one side only (runs and rows of whole
+    # 16-byte multiples): AUTO and the vector path forced join 16-byte vectors
+    # across the two offsets (peeled = 2); the staged path, forced, re-aligns
+    # in shared memory in pieces of the alignment the bases allow
     w, B, S, H, D = 2, 2, 21, 4, 64
     E = 2 if offset % 2 == 0 else 1
     if E == 2:
@@ -242,11 +242,13 @@ def test_misaligned_pointers_select_narrower_pieces(offset, vec):
     with UlyssesA2A(0, E) as a2a:
         xd = [t.cuda() for t in xs]
         g = Guarded(oracle.output_shape(tuple(xs[0].shape), 0, w), xs[0].dtype, w, offset=offset)
+        for path in (PATH_AUTO, PATH_VEC):
+            a2a.set_path(path)
+            plan = a2a.plan(xd, 0, out=g.slabs)
+            assert plan["path"] == PATH_VEC and plan["vec_bytes"] == 16 and plan["peeled"] == 2
+        a2a.set_path(PATH_STAGED)
         plan = a2a.plan(xd, 0, out=g.slabs)
-        assert plan["path"] == (PATH_STAGED if vec <= 4 else PATH_VEC) and plan["vec_bytes"] == vec
-        a2a.set_path(PATH_VEC)
-        plan = a2a.plan(xd, 0, out=g.slabs)
-        assert plan["path"] == PATH_VEC and plan["vec_bytes"] == vec
+        assert plan["path"] == PATH_STAGED and plan["vec_bytes"] == min(offset, 16)
     for path in (PATH_AUTO, PATH_VEC, PATH_STAGED):
         for chunked in (False, True):
             run_case(xs, 0, out_offset=offset, path=path, chunked=chunked)
