@@ -85,9 +85,13 @@ def test_slabs_at_one_offset_every_offset(case, mode):
         for off in _offsets(E):
             for chunked in (False, True):
                 _check(a2a, xs, mode, off, chunked)
-        # the vector path forced takes the same windows
+        # the vector path forced takes the same windows; so does a grid-stride
+        # grid of one CTA per SM over one-row units
         a2a.set_path(PATH_VEC)
         _check(a2a, xs, mode, _offsets(E)[0], False)
+        a2a.set_tuning(ctas_per_sm=1, rows_per_tile=1)
+        _check(a2a, xs, mode, _offsets(E)[-1], True)
+        _check(a2a, xs, mode, _offsets(E)[0], False, expect_peeled=2, out_offset=0)
 
 
 @pytest.mark.parametrize("E", [1, 2, 4, 8])
@@ -300,7 +304,9 @@ def test_randomized_shared_offset_cases():
                   for t in random_byte_slabs(shape[:-1] + (shape[-1] * E,), w, seed0=900 + case)]
             a2a = ctxs.setdefault(E, UlyssesA2A(0, E))
             a2a.set_path(PATH_AUTO)
-            a2a.set_tuning(rows_per_tile=rng.choice([0, 0, 1, 5]))
+            # unit sizes, both unit numberings, and grid-stride grids
+            a2a.set_tuning(rows_per_tile=rng.choice([0, 0, 1, 5]), order=rng.choice([-1, 0, 1]),
+                           ctas_per_sm=rng.choice([0, 0, 1, 3]))
             dev = _offset_slabs(xs, off)
             oshape = oracle.output_shape(shape, mode, w)
             g = Guarded(oshape, xs[0].dtype, w, offset=off_out)
