@@ -38,7 +38,13 @@ CASES = [
     (2, 3, 17, 4, 3, "bf16", 1, 0, STAGED),       # chunked
     (4, 2, 33, 8, 64, "bf16", 0, 2, VEC),         # every slab 2 bytes off 16: 16-byte windows
     (4, 2, 33, 8, 64, "bf16", 1, 8, VEC),         # chunked, 8 bytes off: 16-byte windows
+    (4, 2, 33, 8, 64, "bf16", 1, (6, 0), VEC),    # inputs 6 bytes off, outputs aligned: joined
 ]
+
+
+def _offsets(off):
+    """(input offset, output offset) of a case: one number for both, or a pair."""
+    return off if isinstance(off, tuple) else (off, off)
 
 
 def _device_slabs(cpu_slabs, offset):
@@ -72,6 +78,7 @@ def _noalloc(xs, outs, shape, mode, chunked, E, stream):
 @pytest.mark.parametrize("mode", [0, 1])
 def test_noalloc_matches_the_oracle_and_run_on_two_calls_in_a_row(case, mode):
     w, B, S, H, D, dtype, chunked, off, path = case
+    off, out_off = _offsets(off)
     E = 2 if dtype == "bf16" else 4
     torch.cuda.set_device(0)
     stream = torch.cuda.current_stream()
@@ -81,17 +88,18 @@ def test_noalloc_matches_the_oracle_and_run_on_two_calls_in_a_row(case, mode):
     cpu1 = make(in_shape, w, dtype, seed0=40 + mode)
     cpu2 = make(in_shape, w, dtype, seed0=60 + mode)
     first, second = _device_slabs(cpu1, off), _device_slabs(cpu2, off)
-    out1 = _poisoned(out_shape, first[0].dtype, w, off)
-    out2 = _poisoned(out_shape, first[0].dtype, w, off)
+    out1 = _poisoned(out_shape, first[0].dtype, w, out_off)
+    out2 = _poisoned(out_shape, first[0].dtype, w, out_off)
     plan = UlyssesA2A(0, E).plan(first, mode, chunked=bool(chunked), out=out1)
     assert plan["path"] == path
+    assert plan["peeled"] == (0 if not (off or out_off) or path != VEC else (1 if off == out_off else 2))
 
     # expected outputs: the CPU oracle, and the regular entry point
     oracle1 = oracle.ulysses_a2a(cpu1, mode)
     oracle2 = oracle.ulysses_a2a(cpu2, mode)
     with UlyssesA2A(0, E) as a2a:
         # the regular entry point on outputs at the same offset (same path)
-        ref1, ref2 = (_poisoned(out_shape, first[0].dtype, w, off) for _ in range(2))
+        ref1, ref2 = (_poisoned(out_shape, first[0].dtype, w, out_off) for _ in range(2))
         run1 = a2a.run(first, mode, chunked=bool(chunked), out=ref1)
         run2 = a2a.run(second, mode, chunked=bool(chunked), out=ref2)
         a2a.status()
