@@ -541,7 +541,7 @@ def vec_shape_block(device, peak, sampler, seconds=0.5):
                      "gathered_base_offset_bytes": goff, **res}
         # the other of the two paths, forced: the vector kernel where AUTO
         # re-aligns, the staged kernel where AUTO moves narrow vectors or
-        # peeled 16-byte windows
+        # 16-byte vectors between peeled heads and tails
         other = {3: 2, 2: 3 if (p["vec_bytes"] < 16 or p["peeled"]) else None}.get(p["path"])
         if other is not None:
             a2a.set_path(other)
