@@ -869,6 +869,64 @@ def test_two_gib_payload_full_compare():
     run_case(y, 1)
 
 
+def _big_slabs(shape, w, offset, seed0):
+    """w seeded random int16 slabs of `shape` viewed as bf16, each `offset` bytes
+    into its own allocation, drawn on the device (4 GiB slabs are too large to
+    draw on the host and copy)."""
+    n = 2
+    for v in shape:
+        n *= v
+    out = []
+    for k in range(w):
+        raw = torch.empty(n + offset, dtype=torch.uint8, device="cuda")
+        t = raw[offset:].view(torch.int16).view(shape)
+        g = torch.Generator(device="cuda")
+        g.manual_seed(seed0 + k)
+        t.random_(-32768, 32767, generator=g)
+        out.append(t.view(torch.bfloat16))
+    return out
+
+
+@pytest.mark.parametrize("path, in_off, out_off", [
+    (PATH_AUTO, 0, 0), (PATH_VEC, 0, 0), (PATH_STAGED, 0, 0),
+    (PATH_AUTO, 2, 2), (PATH_AUTO, 2, 0)],
+    ids=["tma", "vec", "staged", "peeled", "shifted"])
+def test_slabs_over_4_gib(path, in_off, out_off):
+    # w = 2, B = 2, S_local = 2^19 + 3 (ragged), H = 16, D = 128, bf16: every
+    # slab is 4 GiB + 24 KB, so byte offsets inside a slab pass 2^32; the
+    # kernels' address arithmetic must be 64-bit throughout. Expected rows come
+    # from the oracle on one-row sub-slabs (the map sends row (b, s) of every
+    # x_j to rows (b, j*S_local + s) of the outputs); the round trip is checked
+    # in full on the device.
+    w, B, S, H, D = 2, 2, (1 << 19) + 3, 16, 128
+    Hw = H // w
+    xs = _big_slabs((B, S, H, D), w, in_off, seed0=980)
+    assert xs[0].numel() * 2 > (1 << 32)
+    with UlyssesA2A(0, 2) as a2a:
+        a2a.set_path(path)
+        ys = _big_slabs((B, S * w, Hw, D), w, out_off, seed0=990)
+        p = a2a.plan(xs, 0, out=ys)
+        assert p["peeled"] == (0 if not in_off else (1 if in_off == out_off else 2))
+        a2a.run(xs, 0, out=ys)
+        a2a.status()
+        g = torch.Generator().manual_seed(970)
+        rows = [(int(torch.randint(0, B, (1,), generator=g)), int(torch.randint(0, S, (1,), generator=g)))
+                for _ in range(24)] + [(B - 1, S - 1), (0, 0), (1, S // 2)]
+        for b, s in rows:
+            sub = [x[b:b + 1, s:s + 1].cpu() for x in xs]
+            want = oracle.ulysses_a2a(sub, 0)          # out_r[0, j, h', d]
+            for r in range(w):
+                got = ys[r][b, [j * S + s for j in range(w)]].cpu().unsqueeze(0)
+                assert torch.equal(bits(got), bits(want[r])), (b, s, r)
+        zs = _big_slabs((B, S, H, D), w, in_off, seed0=995)
+        a2a.run(ys, 1, out=zs)
+        a2a.status()
+        for k in range(w):
+            assert torch.equal(zs[k].view(torch.int16), xs[k].view(torch.int16)), k
+    del xs, ys, zs
+    torch.cuda.empty_cache()
+
+
 def test_environment_overrides_set_the_initial_knobs(monkeypatch):
     monkeypatch.setenv("ULYSSES_A2A_FORCE_PATH", "vec")
     monkeypatch.setenv("ULYSSES_A2A_CTAS_PER_SM", "8")
