@@ -10,22 +10,26 @@ The communicator follows the FastVideo API docs' ulysses_a2a helper:
 * a device window per rank, built once (``_build``) and reused call after
   call; a call that needs more bytes closes and rebuilds it (window grow in
   ``try_all_to_all_4D``);
-* ``chunked=True`` runs the exchange plane by plane on one-plane views, each
-  plane complete before the next reuses the window (``run_armed``);
+* ``chunked=True`` runs the exchange plane by plane on one-plane views
+  (``run_armed``);
 * the result owns its storage and never aliases the window;
 * teardown is collective (``close``): synchronise, agree, release.
 
 One exchange (per call, or per plane when chunked), as in the pypto-lib pull
 request "pipeline HCA AllToAll into O-A", which publishes into a distributed
 window and has consumers load from it after a handshake:
-barrier -> publish (own input into own window) -> barrier -> pull (one kernel
-reads this rank's share out of every window over NVLink and writes the local
-output). With ``input_buffer()`` the producer of the slab writes it into the
-window itself (that pull request's publishing workers), and the first barrier
-and the publish copy drop out. The barriers are collectives of the process group on the caller's
-stream (NCCL: a one-element all-reduce, stream ordered, no host wait) or, for
-host-only backends such as gloo, a stream synchronise plus a group barrier.
-No kernel waits for another GPU.
+publish (own input into one half of own window) -> barrier -> pull (one
+kernel reads this rank's share out of that half of every window over NVLink
+and writes the local output). Exchanges use the two halves of the windows in
+turn, so a publish needs no barrier of its own: the half it overwrites was
+last read two exchanges back, and the previous exchange's barrier completed
+on every rank after that rank's pull from it (each rank's exchanges are
+ordered on one stream). With ``input_buffer()`` the producer of the slab
+writes it into the next half itself (that pull request's publishing workers),
+and the publish copy drops out. The barrier is a collective of the process
+group on the caller's stream (NCCL: a one-element all-reduce, stream ordered,
+no host wait) or, for host-only backends such as gloo, a stream synchronise
+plus a group barrier. No kernel waits for another GPU.
 
 Every copy runs in ``libulysses_a2a.so`` (``ulysses_a2a_peer_*``); this module
 only sequences the calls and the group's collectives.
@@ -96,15 +100,16 @@ class NativePeer:
     def window(self, rank: int) -> int:
         return _lib.ulysses_a2a_peer_window(self._peer, rank) if self._peer is not None else 0
 
-    def window_tensor(self, shape, dtype) -> torch.Tensor:
-        """This rank's window as a dense tensor (no copy; valid until the window
-        is released)."""
+    def window_tensor(self, shape, dtype, offset: int = 0) -> torch.Tensor:
+        """This rank's window from byte ``offset`` on as a dense tensor (no copy;
+        valid until the window is released)."""
         n = torch.empty((), dtype=dtype).element_size()
         for v in shape:
             n *= int(v)
-        if self._peer is None or n > self._nbytes:
+        if self._peer is None or offset + n > self._nbytes:
             raise ValueError("the window is not built or is smaller than the tensor")
-        raw = torch.as_tensor(_DeviceBytes(self.window(self._rank), n), device=self.device)
+        raw = torch.as_tensor(_DeviceBytes(self.window(self._rank) + offset, n),
+                              device=self.device)
         return raw.view(dtype).view(tuple(shape))
 
     def unmap(self) -> None:
@@ -160,10 +165,11 @@ class PeerExchange:
         self.barrier_kind = barrier
         self._flag = (torch.zeros(1, dtype=torch.int32, device=self.device)
                       if barrier == "stream" else None)
-        self._nbytes = 0
+        self._nbytes = 0               # each rank's window: two halves of _nbytes // 2
+        self._half = 0                 # the half the next exchange publishes into
         self._armed = False
         self._agreed = set()           # call signatures every rank has confirmed
-        self._in_place = None          # window address handed out by input_buffer()
+        self._in_place = None          # (address, offset) handed out by input_buffer()
         self.disabled_reason = None
 
     # ---------------------------------------------------------- group helpers
@@ -273,23 +279,42 @@ class PeerExchange:
             self._agreed.add(sig)
 
     def _ensure_window(self, need: int) -> None:
-        if need > self._nbytes:
+        """Windows whose two halves hold at least ``need`` bytes each (256-byte
+        aligned halves)."""
+        span = (need + 255) // 256 * 256
+        if 2 * span > self._nbytes:
             if self._armed and not self.close():
                 raise RuntimeError("window teardown before growing failed")
-            if not self.build(need):
+            if not self.build(2 * span):
                 self._disable("a rank could not build its window")
                 raise RuntimeError("peer exchange: window build failed on some rank")
+            self._half = 0
+            self._in_place = None
+
+    def _take_half(self) -> int:
+        """Byte offset of the window half this exchange publishes into and pulls
+        from; the next exchange takes the other half. A half that
+        input_buffer() handed out and no exchange used is taken again (it was
+        never read, and taking the other one would overwrite the half the last
+        exchange's pulls may still read)."""
+        if self._in_place is not None:
+            self._in_place = None
+            self._half ^= 1
+        off = self._half * (self._nbytes // 2)
+        self._half ^= 1
+        return off
 
     def input_buffer(self, shape, dtype=torch.bfloat16, stream=None) -> torch.Tensor:
         """This rank's window as a dense tensor of ``shape``, for an in-place input.
 
-        Collective: every rank calls it with the same shape. It takes the
-        barrier after which no rank reads the windows any more, so the caller
-        may write its slab straight into the returned tensor (for example as
-        the output of the projection that produces it) and then pass that
-        tensor to ``all_to_all_4d`` with ``chunked=False``, which skips the
-        publish copy and its barrier. The tensor is valid until the window is
-        rebuilt or closed.
+        Collective: every rank calls it with the same shape. It hands out the
+        window half the next exchange uses, which no rank reads any more once
+        the previous exchange's barrier has passed on this rank's stream, so
+        the caller may write its slab straight into the returned tensor on
+        that stream (for example as the output of the projection that produces
+        it) and then pass that tensor to ``all_to_all_4d`` with
+        ``chunked=False``, which skips the publish copy. The tensor is valid
+        until the window is rebuilt or closed.
         """
         if self.disabled_reason is not None:
             raise RuntimeError(f"peer exchange disabled: {self.disabled_reason}")
@@ -301,15 +326,13 @@ class PeerExchange:
             need *= v
         self._agree_signature(("input_buffer", shape, dtype))
         self._ensure_window(need)
-        if stream is None:
-            stream = self.native.current_stream()
-        self._barrier(stream)         # every rank is done reading the windows
-        t = self.native.window_tensor(shape, dtype)
-        self._in_place = t.data_ptr()
+        off = self._take_half()
+        t = self.native.window_tensor(shape, dtype, off)
+        self._in_place = (t.data_ptr(), off)
         return t
 
     def all_to_all_4d_packed(self, x, mode: int, out=None, stream=None):
-        """Exchange T tensors packed along the head dimension with one barrier pair.
+        """Exchange T tensors packed along the head dimension with one barrier.
 
         mode 0: ``x`` is this rank's contiguous [B, S_local, T, H, D] slab (for
         example its packed q/k/v projection output); returns T tensors
@@ -319,7 +342,7 @@ class PeerExchange:
         the packed [B, S_local, T, H, D] slab (``out`` may be given). The T
         slabs share the window at consecutive offsets, and each is pulled
         into its slot of the packed output.
-        Same bytes as T calls of ``all_to_all_4d``; 2 barriers instead of 2T,
+        Same bytes as T calls of ``all_to_all_4d``; one barrier instead of T,
         and one pull launch for all T tensors.
         """
         if self.disabled_reason is not None:
@@ -358,20 +381,21 @@ class PeerExchange:
         if slab == 0:
             return outs
         self._agree_signature(("packed", mode, T, B, S, H, D, dtype))
+        if mode == 1 and not outs.is_contiguous():
+            raise ValueError("the packed output must be contiguous")
         self._ensure_window(T * slab)
         if stream is None:
             stream = self.native.current_stream()
-        self._barrier(stream)        # every rank is done reading the windows
+        off = self._take_half()
         if mode == 0:
             # the packed rows published whole: T*H heads of D
-            self.native.publish(x, B, S, T * H, D, 0, 0, stream)
+            self.native.publish(x, B, S, T * H, D, 0, 0, stream, window_offset=off)
         else:
             for t in range(T):
-                self.native.publish(srcs[t], B, S, H, D, 1, 0, stream, window_offset=t * slab)
+                self.native.publish(srcs[t], B, S, H, D, 1, 0, stream,
+                                    window_offset=off + t * slab)
         self._barrier(stream)        # every window holds its slabs
-        if mode == 1 and not outs.is_contiguous():
-            raise ValueError("the packed output must be contiguous")
-        self.native.pull_packed(outs, T, B, S, H, D, mode, stream)
+        self.native.pull_packed(outs, T, B, S, H, D, mode, stream, window_offset=off)
         return outs
 
     def all_to_all_4d(self, x: torch.Tensor, mode: int, chunked: bool = False, out=None,
@@ -408,26 +432,32 @@ class PeerExchange:
             return out
         planes = B if chunked else 1
         need = (1 if chunked else B) * S * H * D * self.elem_bytes
-        in_place = self._armed and x.data_ptr() == self.native.window(self.rank)
+        own = self.native.window(self.rank) if self._armed else 0
+        in_place = own != 0 and own <= x.data_ptr() < own + self._nbytes
         self._agree_signature((mode, bool(chunked), B, S, H, D, x.dtype, in_place))
         if stream is None:
             stream = self.native.current_stream()
         if in_place:
-            # the slab was written into the window after input_buffer()'s barrier
-            if chunked or not x.is_contiguous() or self._in_place != x.data_ptr():
+            # the slab was written into the half input_buffer() handed out
+            if (chunked or not x.is_contiguous() or self._in_place is None
+                    or self._in_place[0] != x.data_ptr()):
                 raise ValueError("an input in the window must come from input_buffer() and be "
                                  "exchanged whole (chunked=False)")
+            off = self._in_place[1]
             self._in_place = None
             self._barrier(stream)    # every window holds its slab
-            self.native.pull(out, B, S, H, D, mode, pitch if mode == 1 else 0, stream)
+            self.native.pull(out, B, S, H, D, mode, pitch if mode == 1 else 0, stream,
+                             window_offset=off)
             return out
         self._ensure_window(need)
         nb = 1 if chunked else B
         for b in range(planes):
             xv = x[b:b + 1] if chunked else x
             ov = out[b:b + 1] if chunked else out
-            self._barrier(stream)    # every rank is done reading the windows
-            self.native.publish(xv, nb, S, H, D, mode, pitch if mode == 0 else 0, stream)
+            off = self._take_half()
+            self.native.publish(xv, nb, S, H, D, mode, pitch if mode == 0 else 0, stream,
+                                window_offset=off)
             self._barrier(stream)    # every window holds this plane
-            self.native.pull(ov, nb, S, H, D, mode, pitch if mode == 1 else 0, stream)
+            self.native.pull(ov, nb, S, H, D, mode, pitch if mode == 1 else 0, stream,
+                             window_offset=off)
         return out

@@ -3,14 +3,14 @@
 The native peer object is replaced by a stand-in whose windows are POSIX
 shared memory and whose pull assembles the rank's output from the other
 process's window with tensor slicing. What is under test is the sequencing
-that PeerExchange owns: the record exchange, the barrier before every publish
-and before every pull, window growth (collective close + rebuild), the
-agreement on call signatures, and collective teardown. Delays make a missing
-barrier visible. Rank 1 publishes late, so rank 0, pulling without the
-barrier before the pull, would read rank 1's window before it is written; rank
-1 also pulls late, so rank 0, publishing its next call without the barrier
-before the publish, would overwrite its window while rank 1 still reads it.
-Expected values come from the oracle.
+that PeerExchange owns: the record exchange, the one barrier of an exchange
+(before its pull), the two window halves that exchanges use in turn, window
+growth (collective close + rebuild), the agreement on call signatures, and
+collective teardown. Delays make a missing barrier or a reused half visible.
+Rank 1 publishes late, so rank 0, pulling without the barrier, would read rank
+1's window before it is written; rank 1 also pulls late, so rank 0,
+publishing its next exchanges into the same half, would overwrite it while
+rank 1 still reads it. Expected values come from the oracle.
 """
 
 import os
@@ -43,6 +43,7 @@ class ShmNative:
         self.pull_delay = pull_delay
         self.fail_create = fail_create
         self.launch_count = 0
+        self.halves = []           # the window offset of every pull
 
     def create(self, rank, world, nbytes):
         if self.fail_create:
@@ -78,11 +79,11 @@ class ShmNative:
             return 0
         return torch.frombuffer(shm.buf, dtype=torch.uint8, count=1).data_ptr()
 
-    def window_tensor(self, shape, dtype):
+    def window_tensor(self, shape, dtype, offset=0):
         n = 1
         for v in shape:
             n *= v
-        return torch.frombuffer(self.own.buf, dtype=dtype, count=n).view(shape)
+        return torch.frombuffer(self.own.buf, dtype=dtype, count=n, offset=offset).view(shape)
 
     def publish(self, x, B, S, H, D, mode, row_pitch, stream, window_offset=0):
         time.sleep(self.publish_delay)
@@ -94,6 +95,7 @@ class ShmNative:
 
     def pull(self, out, B, S, H, D, mode, row_pitch, stream, window_offset=0):
         time.sleep(self.pull_delay)
+        self.halves.append(window_offset)
         w, k = self.world, self.rank
         Hw = H // w
         if mode == 0:
@@ -111,6 +113,7 @@ class ShmNative:
     def pull_packed(self, outs, T, B, S, H, D, mode, stream, window_offset=0):
         """The T tensors of a head-packed exchange at once (one native launch)."""
         time.sleep(self.pull_delay)
+        self.halves.append(window_offset)
         w, k = self.world, self.rank
         Hw = H // w
         slab_bytes = B * S * H * D * self.elem_bytes
@@ -183,11 +186,12 @@ def _worker(rank, world, port, scenario, q):
                 rep["ok"].append(torch.equal(got.view(torch.int16), want.view(torch.int16)))
             rep["closed"] = ex.close()
             rep["log"] = native.log
+            rep["halves"] = native.halves
         elif scenario == "in_place":
-            # rank 1 writes its slab late and pulls late: without the barrier in
-            # input_buffer() rank 0 would overwrite its window while rank 1 still
-            # reads it; without the one before the pull, rank 0 would read rank
-            # 1's window before the slab is in it
+            # rank 1 writes its slab late and pulls late: input_buffer() hands
+            # out the half no rank reads any more (rank 0 writing into the half
+            # rank 1 still reads would show); without the barrier before the
+            # pull, rank 0 would read rank 1's window before the slab is in it
             native = ShmNative(rank, pull_delay=0.2 if rank == 1 else 0.0)
             ex = PeerExchange(native=native, elem_bytes=2)
             shape = (2, 5, 4, 8)
@@ -201,11 +205,16 @@ def _worker(rank, world, port, scenario, q):
                 del buf
                 want = oracle.ulysses_a2a(xs, 0)[rank]
                 rep["ok"].append(torch.equal(got.view(torch.int16), want.view(torch.int16)))
-            # an ordinary call still works after in-place ones
-            xs = normal_slabs(shape, world, "bf16", seed0=2000)
-            got = ex.all_to_all_4d(xs[rank].clone(), 0)
-            rep["ok"].append(torch.equal(got.view(torch.int16),
-                                         oracle.ulysses_a2a(xs, 0)[rank].view(torch.int16)))
+            # an ordinary call still works after in-place ones, also after an
+            # input_buffer() that no exchange used (its half is taken again)
+            for seed in (2000, 2010):
+                if seed == 2010:
+                    ex.input_buffer(shape, torch.bfloat16)
+                xs = normal_slabs(shape, world, "bf16", seed0=seed)
+                got = ex.all_to_all_4d(xs[rank].clone(), 0)
+                rep["ok"].append(torch.equal(got.view(torch.int16),
+                                             oracle.ulysses_a2a(xs, 0)[rank].view(torch.int16)))
+            rep["halves"] = native.halves
             rep["closed"] = ex.close()
             rep["log"] = native.log
         elif scenario == "autograd":
@@ -242,6 +251,7 @@ def _worker(rank, world, port, scenario, q):
             rep["ok"].append(torch.equal(back.view(torch.int16), packed[rank].view(torch.int16)))
             rep["closed"] = ex.close()
             rep["log"] = native.log
+            rep["halves"] = native.halves
         elif scenario == "split_close":
             # rank 1 believes its window is gone while rank 0's is armed
             native = ShmNative(rank)
@@ -302,23 +312,30 @@ def test_exchange_sequence_barriers_and_growth():
         assert rep["closed"] is True
         log = rep["log"]
         creates = [e[1] for e in log if isinstance(e, tuple) and e[0] == "create"]
-        # 2*5*4*8*2 bytes for the first three calls (one plane when chunked fits),
-        # then the larger slab after a collective close
-        assert creates == [2 * 5 * 4 * 8 * 2, 16 * 8 * 8 * 2]
+        # two halves of 2*5*4*8*2 = 640 bytes (256-byte aligned: 768) for the
+        # first three calls (one plane when chunked fits), then two of the
+        # larger slab's 2048 after a collective close
+        assert creates == [2 * 768, 2 * 2048]
         ops = [e for e in log if isinstance(e, str)]
         # one publish + one pull per exchange, per plane when chunked
         assert ops == ["publish", "pull"] * (1 + 1 + 2 + 1)
+        # the exchanges (planes, when chunked) alternate between the two
+        # halves, from the first after each build
+        assert rep["halves"] == [0, 768, 0, 768, 0]
         assert log.index(("unmap",)) < log.index(("release",))
 
 
 def test_in_place_input_skips_the_publish():
     for rep in _run("in_place", 300):
         assert rep["errors"] == [], rep
-        assert rep["ok"] == [True] * 4, rep
+        assert rep["ok"] == [True] * 5, rep
         assert rep["closed"] is True
         ops = [e for e in rep["log"] if isinstance(e, str)]
-        # three in-place exchanges pull without publishing, then one ordinary one
-        assert ops == ["pull"] * 3 + ["publish", "pull"]
+        # three in-place exchanges pull without publishing, then two ordinary ones
+        assert ops == ["pull"] * 3 + ["publish", "pull"] * 2
+        # halves 0, 1, 0 in place; then 1; the unused input_buffer() takes 0,
+        # which the next exchange takes again
+        assert rep["halves"] == [0, 768, 0, 768, 0], rep["halves"]
 
 
 def test_autograd_backward_is_the_inverse_exchange():
@@ -328,14 +345,17 @@ def test_autograd_backward_is_the_inverse_exchange():
         assert rep["closed"] is True
 
 
-def test_packed_exchange_uses_one_barrier_pair_and_one_pull():
+def test_packed_exchange_uses_one_barrier_and_one_pull():
     for rep in _run("packed", 500):
         assert rep["errors"] == [], rep
         assert rep["ok"] == [True] * 4, rep
         assert rep["closed"] is True
         ops = [e for e in rep["log"] if isinstance(e, str)]
-        # one pull (one native launch) for the three tensors in each mode
+        # one pull (one native launch) for the three tensors in each mode, the
+        # two exchanges in the two halves (T*B*S*H*D*2 = 1920 bytes, 256-byte
+        # aligned: 2048)
         assert ops == ["publish", "pull"] + ["publish"] * 3 + ["pull"]
+        assert rep["halves"] == [0, 2048]
 
 
 def test_split_teardown_leaks_instead_of_freeing():
