@@ -113,6 +113,29 @@ def test_inputs_and_outputs_at_two_offsets(E, mode):
                            out_offset=a_out)
 
 
+@pytest.mark.parametrize("mode", [0, 1])
+def test_offset_slabs_through_the_staging_window(mode):
+    # chunked = 2 copies every plane into the context's (aligned) window and
+    # re-lays it out from there into the caller's slabs, 6 bytes off: the
+    # shifted kernel in mode 0 (aligned window -> offset outputs); in mode 1
+    # the window holds the gathered plane and the outputs are offset too
+    w, B, S, H, D = 4, 3, 45, 8, 64
+    shape = slab_shape(mode, w, B, S, H, D)
+    xs_cpu = normal_slabs(shape, w, "bf16", seed0=785 + mode)
+    with UlyssesA2A(0, 2) as a2a:
+        xs = _offset_slabs(xs_cpu, 6)
+        oshape = oracle.output_shape(shape, mode, w)
+        g = Guarded(oshape, torch.bfloat16, w, offset=6)
+        n0 = a2a.launch_count
+        a2a.run(xs, mode, chunked=2, out=g.slabs)
+        a2a.status()
+        assert a2a.launch_count - n0 == B
+        want = oracle.ulysses_a2a(xs_cpu, mode)
+        for k in range(w):
+            assert torch.equal(bits(g.slabs[k].cpu()), bits(want[k])), k
+        g.check_guards()
+
+
 def test_shifted_round_trip_chunked_and_pitched():
     # inputs 2 bytes off, outputs 10 off, chunked per plane; then mode 1 from
     # aligned slabs into q slots of a packed buffer 6 bytes off
