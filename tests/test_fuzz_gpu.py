@@ -4,7 +4,9 @@ Each case draws the rank count (1..16), element size (1/2/4/8), B, S_local, H,
 D, mode, chunking (per plane, through the staging window or not), a row pitch
 on the [B, S_local, H, D] side, input and output base offsets past a 16-byte
 boundary (independently), head-packed tensors (T = 2, 3), a forced path (or
-AUTO) and the tuning knobs (rows per unit, unit order, grid-stride grids).
+AUTO), the tuning knobs (rows per unit, unit order, grid-stride grids) and the
+entry point: ``run``, a bound call, the allocation-free C entry point, or the
+host-buffer call (the last two for dense, unpacked slabs).
 The element map is the one the FastVideo API docs give for ``run_armed``
 (device_communicators/ulysses_a2a). Expected values come from the oracle
 (the pitched form for pitched and packed cases); outputs are poisoned and
@@ -56,11 +58,37 @@ def _one_case(rng, case, ctxs):
     a2a.set_tuning(rows_per_tile=rng.choice([0, 0, 1, 3, 7]), order=rng.choice([-1, 0, 1]),
                    ctas_per_sm=rng.choice([0, 0, 0, 1, 3]))
     dt = INT[E]
+    entry = rng.choice(["run", "run", "run", "bind", "noalloc", "host"])
+    if entry in ("noalloc", "host") and (T != 1 or gap or chunked == 2):
+        entry = "run"
+    if entry == "host":
+        path = PATH_AUTO
+        a2a.set_path(path)
+        off_in = off_out = 0
+    if entry == "noalloc":
+        path = PATH_AUTO                    # the allocation-free call takes AUTO's path
     P = T * H * D + gap                     # row pitch of the [B, S, (T,) H, D] side
     n_p = (B * S - 1) * P + T * H * D
     gshape = (B, S * w, H // w, D)
     desc = f"case {case}: E={E} w={w} B={B} S={S} H={H} D={D} mode={mode} chunked={chunked} " \
-           f"T={T} gap={gap} off={off_in}/{off_out} path={path}"
+           f"T={T} gap={gap} off={off_in}/{off_out} path={path} entry={entry}"
+
+    def call(xs, m, out):
+        if entry == "bind":
+            return a2a.bind(xs, m, chunked=chunked, out=out)()
+        if entry == "noalloc":
+            rc, msg = _lib.ulysses_a2a_run_noalloc([t.data_ptr() for t in xs],
+                                                   [o.data_ptr() for o in out], B, S, H, D, w, m,
+                                                   chunked, E, torch.cuda.current_stream().cuda_stream,
+                                                   wait=1)
+            assert rc == _lib.OK, (desc, msg)
+            return out
+        if entry == "host":
+            res = a2a.run_host([t.cpu().pin_memory() for t in xs], m, chunked=bool(chunked))
+            for o, r in zip(out, res):
+                o.copy_(r)
+            return out
+        return a2a.run(xs, m, chunked=chunked, out=out)
     try:
         if T == 1:
             bufs = [t.view(dt) for t in random_byte_slabs((n_p * E,), w, seed0=50000 + case)]
@@ -68,7 +96,7 @@ def _one_case(rng, case, ctxs):
                 want = oracle.ulysses_a2a_pitched(bufs, 0, w, B, S, H, D, P)
                 xs = [_at_offset(t, off_in).as_strided((B, S, H, D), (S * P, P, D, 1)) for t in bufs]
                 g = Guarded(gshape, dt, w, offset=off_out)
-                a2a.run(xs, 0, chunked=chunked, out=g.slabs)
+                call(xs, 0, g.slabs)
                 a2a.status()
                 for r in range(w):
                     assert torch.equal(bits(g.slabs[r].cpu()).reshape(-1), bits(want[r]).reshape(-1)), \
@@ -79,7 +107,7 @@ def _one_case(rng, case, ctxs):
                 xs = [_at_offset(y, off_in) for y in ys]
                 outs = [_at_offset(torch.full((n_p,), -1, dtype=dt), off_out) for _ in range(w)]
                 views = [o.as_strided((B, S, H, D), (S * P, P, D, 1)) for o in outs]
-                a2a.run(xs, 1, chunked=chunked, out=views)
+                call(xs, 1, views)
                 a2a.status()
                 for j in range(w):
                     got = outs[j].cpu()
