@@ -217,9 +217,14 @@ cudaError_t launch_tma(int mode, int grid, int block, size_t smem, cudaStream_t 
                    : launch_pdl(ua2a::ua2a_tma_kernel<1>, grid, block, smem, st, p);
 }
 
+// Vectors in flight per thread: 4, and 6 for the 8-byte mode-0 kernel, which
+// holds them in its 32 registers (8 CTAs per SM) without spilling and so keeps
+// as many bytes in flight per SM as the 16-byte kernel (200-byte runs, mode 0:
+// 0.93 -> 0.96 of the copy bandwidth). Its mode-1 twin spills at 5.
 template <typename V>
 cudaError_t launch_vec_t(const VecParams& p, int mode, int grid, int block, cudaStream_t st) {
-  return mode == 0 ? launch_pdl(ua2a::ua2a_vec_kernel<V, 0, 4>, grid, block, 0, st, p)
+  constexpr int kU0 = sizeof(V) == 8 ? 6 : 4;
+  return mode == 0 ? launch_pdl(ua2a::ua2a_vec_kernel<V, 0, kU0>, grid, block, 0, st, p)
                    : launch_pdl(ua2a::ua2a_vec_kernel<V, 1, 4>, grid, block, 0, st, p);
 }
 
