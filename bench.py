@@ -105,6 +105,27 @@ VEC_SHAPES = {
     "base2in_w4_S8192_H24_D128": (4, 1, 8192, 24, 128, 2, 2, 0),
     "w16_S4096_H32_D128": (16, 1, 4096, 32, 128, 2, 0),             # w above the TMA limit
 }
+# Dense shapes with runs off 16 bytes (about 256 MiB each; bf16 unless noted):
+# name -> (w, B, S, H, D, element bytes). --staged-forms times each on the
+# staged path's two forms, and on the vector path; the first eight have
+# pieces of 4 bytes or less, the others 8 bytes.
+STAGED_FORM_SHAPES = {
+    "w4_S2796202_H4_D3": (4, 1, 2796202, 4, 3, 2),             # 6-byte runs, 4 regions
+    "w8_S699050_H8_D3": (8, 1, 699050, 8, 3, 2),                # 6-byte runs, 8 regions
+    "w16_S174762_H16_D3": (16, 1, 174762, 16, 3, 2),            # 6-byte runs, 16 regions
+    "w3_S2982616_H3_D5": (3, 1, 2982616, 3, 5, 2),              # 10-byte runs
+    "w4_S1398101_H4_D3_fp32": (4, 1, 1398101, 4, 3, 4),         # 12-byte runs
+    "w2_S13421772_H2_D5_u8": (2, 1, 13421772, 2, 5, 1),         # 5-byte runs, 1-byte pieces
+    "w4_S838860_H8_D5": (4, 1, 838860, 8, 5, 2),                # 20-byte runs
+    "w8_S116508_H8_D9_fp32": (8, 1, 116508, 8, 9, 4),           # 36-byte runs
+    "w4_S2097152_H4_D4": (4, 1, 2097152, 4, 4, 2),              # 8-byte runs
+    "w4_S2796202_H4_D6_fp32": (4, 1, 2796202, 4, 6, 4),         # 24-byte runs
+    "w4_S419430_H4_D20": (4, 1, 419430, 4, 20, 2),              # 40-byte runs
+    "w4_S233016_H4_D36": (4, 1, 233016, 4, 36, 2),              # 72-byte runs
+    "w4_S161319_H4_D52": (4, 1, 161319, 4, 52, 2),              # 104-byte runs
+    "w4_S123361_H4_D68": (4, 1, 123361, 4, 68, 2),              # 136-byte runs
+    "w8_S41943_H8_D100": (8, 1, 41943, 8, 100, 2),              # 200-byte runs
+}
 
 
 # Every workload --workload accepts: the table above, and the vector-path shapes
@@ -115,7 +136,7 @@ ALL_WORKLOADS = {**{n: dict(v, E=2, off=0, goff=0) for n, v in WORKLOADS.items()
                  **{n: dict(w=v[0], B=v[1], S_local=v[2], H=v[3], D=v[4], E=v[5], off=v[6],
                             goff=v[7] if len(v) > 7 else v[6])
                     for n, v in VEC_SHAPES.items()}}
-DTYPE_OF = {2: "bf16", 4: "fp32"}
+DTYPE_OF = {1: "u8", 2: "bf16", 4: "fp32"}
 INT_OF = {2: torch.int16, 4: torch.int32}
 
 
@@ -190,10 +211,10 @@ def _code_only(text: str) -> str:
 
 
 KERNEL_FILES = {"tma": "kernels_tma.cuh", "vec": "kernels_vec.cuh", "peel": "kernels_peel.cuh",
-                "staged": "kernels_stage.cuh"}
+                "staged": "kernels_stage.cuh", "phase": "kernels_phase.cuh"}
 PATH_NAMES = {1: "tma", 2: "vec", 3: "staged"}
 LAUNCH_FIELDS = ("path", "rows_per_tile", "producers", "stages", "lookahead", "chunk_units",
-                 "order", "grid", "block", "smem_bytes", "vec_bytes", "peeled")
+                 "order", "grid", "block", "smem_bytes", "vec_bytes", "peeled", "fixed_phase")
 
 
 def kernel_source_hash(path):
@@ -217,8 +238,10 @@ def ncu_traffic(key, plan, chunked):
         return None, "no ncu traffic summary"
     if not entry:
         return None, "no ncu capture of this kernel and workload"
-    # the vector path's peeled and shifted kernels live in a file of their own
-    kernel = "peel" if plan.get("peeled") else key.split(":")[0]
+    # the vector path's peeled and shifted kernels, and the staged path's
+    # fixed-phase kernel, live in files of their own
+    kernel = ("peel" if plan.get("peeled") else
+              "phase" if plan.get("fixed_phase") else key.split(":")[0])
     if entry.get("kernel_hash") != kernel_source_hash(kernel):
         return None, "kernel changed since the ncu counters were taken"
     launch = entry.get("launch", {})
@@ -322,15 +345,19 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- our arm
 def make_inputs(w, B, S, H, D, dtype, device, seed0=1234, offset_bytes=0):
-    """Seeded N(0,1) slabs drawn on the device generator (values do not affect
-    timing); with offset_bytes each slab starts that many bytes past the start
-    of its own allocation (a base off the 16-byte boundary)."""
-    dt = {"bf16": torch.bfloat16, "fp32": torch.float32}[dtype]
+    """Seeded N(0,1) slabs (uniform bytes for "u8") drawn on the device
+    generator (values do not affect timing); with offset_bytes each slab starts
+    that many bytes past the start of its own allocation (a base off the 16-byte
+    boundary)."""
+    dt = {"bf16": torch.bfloat16, "fp32": torch.float32, "u8": torch.uint8}[dtype]
     xs = []
     for k in range(w):
         g = torch.Generator(device=device)
         g.manual_seed(seed0 + k)
-        v = torch.randn((B, S, H, D), generator=g, device=device, dtype=torch.float32).to(dt)
+        if dt == torch.uint8:
+            v = torch.randint(0, 256, (B, S, H, D), generator=g, device=device, dtype=dt)
+        else:
+            v = torch.randn((B, S, H, D), generator=g, device=device, dtype=torch.float32).to(dt)
         if offset_bytes:
             n = v.numel() * v.element_size()
             raw = torch.empty(n + offset_bytes, dtype=torch.uint8, device=device)
@@ -537,6 +564,7 @@ def vec_shape_block(device, peak, sampler, seconds=0.5):
             raise SystemExit(f"vector-path shape {name}: round trip mismatch")
         out[name] = {"payload_bytes": P, "path": PATH_NAMES[p["path"]],
                      "vec_bytes": p["vec_bytes"], "peeled": p["peeled"],
+                     "fixed_phase": p["fixed_phase"],
                      "row_bytes": p["row_bytes"], "base_offset_bytes": off,
                      "gathered_base_offset_bytes": goff, **res}
         # the other of the two paths, forced: the vector kernel where AUTO
@@ -559,6 +587,58 @@ def vec_shape_block(device, peak, sampler, seconds=0.5):
         del x, y, z
         torch.cuda.empty_cache()
     return out
+
+
+def staged_forms_block(device, peak, sampler, seconds=0.5):
+    """STAGED_FORM_SHAPES on the path AUTO picks, on the staged path's
+    fixed-phase and per-piece forms, and on the vector path: fractions per mode."""
+    from sequence_all_re_b200 import UlyssesA2A
+
+    stream = torch.cuda.Stream(device)
+    out = {}
+    for name, (w, B, S, H, D, E) in STAGED_FORM_SHAPES.items():
+        a2a = UlyssesA2A(device.index or 0, E)
+        x = make_inputs(w, B, S, H, D, DTYPE_OF[E], device)
+        y = empty_slabs(w, (B, S * w, H // w, D), x[0].dtype, device)
+        z = empty_slabs(w, (B, S, H, D), x[0].dtype, device)
+        P = w * B * S * H * D * E
+        row = {"payload_bytes": P, "row_bytes": (H // w) * D * E}
+        for label, path, knobs in (("auto", 0, {}), ("fixed_phase", 3, {}),
+                                   ("per_piece", 3, {"staged_form": 1}), ("vec", 2, {})):
+            a2a.set_path(path)
+            a2a.set_tuning(**knobs)
+            p = a2a.plan(x, 0, out=y)
+            for t in z:
+                t.zero_()
+            res = per_mode_block(a2a, x, y, z, P, stream, peak, sampler, seconds)
+            torch.cuda.synchronize()
+            if not all(torch.equal(z[k], x[k]) for k in range(w)):
+                raise SystemExit(f"shape {name}: round trip mismatch ({label})")
+            row[label] = {"path": PATH_NAMES[p["path"]], "vec_bytes": p["vec_bytes"],
+                          "fixed_phase": p["fixed_phase"],
+                          "mode0": res["mode0"]["frac"], "mode1": res["mode1"]["frac"],
+                          "sm_mhz": (res["mode0"]["clocks"] or {}).get("sm_mhz")}
+        out[name] = row
+        a2a.close()
+        del x, y, z
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_staged_forms(args):
+    """The staged path's two forms and the vector path on STAGED_FORM_SHAPES
+    (each mode back to back for >= 0.5 s); prints its own line."""
+    if args.gpus != 1:
+        raise SystemExit("--staged-forms runs on one GPU")
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    peak, peak_src = hbm_peak()
+    sampler = ClockSampler(0).start()
+    res = staged_forms_block(device, peak, sampler)
+    sampler.stop()
+    print(json.dumps({"metric": "fraction of the measured copy bandwidth per form, back to "
+                                "back, 2 x payload per call",
+                      "peak": peak, "peak_source": peak_src, "shapes": res}), flush=True)
 
 
 def cpu_oracle_baseline(w, B, S, H, D, budget_s=12.0, E=2):
@@ -1385,6 +1465,9 @@ def main():
     ap.add_argument("--tuning-sweep", action="store_true",
                     help="time the schedule knobs one at a time on two workloads (prints its "
                          "own line)")
+    ap.add_argument("--staged-forms", action="store_true",
+                    help="time the staged path's fixed-phase and per-piece forms and the "
+                         "vector path on dense narrow-run shapes (prints its own line)")
     ap.add_argument("--peer-one-gpu", action="store_true",
                     help="time the multi-GPU exchange's publish and pull kernels with the w "
                          "ranks as contexts on one GPU (prints its own line)")
@@ -1402,6 +1485,8 @@ def main():
         run_packed(args)
     elif args.tuning_sweep:
         run_tuning_sweep(args)
+    elif args.staged_forms:
+        run_staged_forms(args)
     else:
         run_ours(args)
 

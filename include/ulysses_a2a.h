@@ -129,7 +129,13 @@ typedef struct ulysses_a2a_plan_t {
                                 each destination vector (and head and tail) is
                                 two aligned source vectors joined by a shift.
                                 vec_bytes is then 16                        */
-    int32_t reserved;        /* 0                                             */
+    int32_t fixed_phase;     /* STAGED path: 1 = the [B,S_local,H,D] side is
+                                dense and the gathered slabs share one
+                                offset past a 16-byte boundary: each thread
+                                takes strided chunks that share one offset
+                                modulo a strided row, so it works out where
+                                their pieces go once per work unit; 0 = every
+                                chunk's pieces are placed one by one        */
 } ulysses_a2a_plan_t;
 
 /* One call's arguments, for ulysses_a2a_run_ex / ulysses_a2a_plan_ex. Same
@@ -270,6 +276,9 @@ typedef struct ulysses_a2a_tuning_t {
     int32_t host_chunks;    /* host-buffer entry point: sequence chunks its
                                copies and kernels are pipelined over, 1..64;
                                0 = default                                */
+    int32_t staged_form;    /* STAGED path: 0 = the fixed-phase form where it
+                               applies (default; see plan_t.fixed_phase),
+                               1 = the per-piece form always              */
 } ulysses_a2a_tuning_t;
 
 /* Apply tuning to later runs (NULL restores every default). Values outside

@@ -84,7 +84,7 @@ class PlanT(ctypes.Structure):
         ("chunk_units", ctypes.c_int32),
         ("row_pitch", ctypes.c_int64),
         ("peeled", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("fixed_phase", ctypes.c_int32),
     ]
 
     def as_dict(self) -> dict:
@@ -103,10 +103,11 @@ class TuningT(ctypes.Structure):
         ("order", ctypes.c_int32),
         ("chunk_units", ctypes.c_int32),
         ("host_chunks", ctypes.c_int32),
+        ("staged_form", ctypes.c_int32),
     ]
 
     DEFAULTS = dict(rows_per_tile=0, ctas_per_sm=0, stages=0, lookahead=0, producers=0,
-                    order=-1, chunk_units=-1, host_chunks=0)
+                    order=-1, chunk_units=-1, host_chunks=0, staged_form=0)
 
     @classmethod
     def make(cls, **kw):

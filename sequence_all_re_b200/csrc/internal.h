@@ -16,6 +16,7 @@
 #include <vector>
 
 #include "kernels_peel.cuh"
+#include "kernels_phase.cuh"
 #include "kernels_stage.cuh"
 #include "kernels_tma.cuh"
 #include "kernels_vec.cuh"
@@ -107,9 +108,12 @@ cudaError_t launch_vec(const VecParams& p, int vec_bytes, int peeled, int mode, 
 VecParams vec_params(const void* const* in, void* const* out, int nin, int nout, int64_t S, int w,
                      int E, const ulysses_a2a_plan_t& pl, int64_t units, int64_t nb, int64_t nt,
                      int nr, int nj, uint32_t r0, uint32_t r_stride, uint32_t j0, int64_t tile0);
-cudaError_t launch_stage(const StageParams& p, int piece_bytes, int mode, int grid, int block,
-                         size_t smem, cudaStream_t st);
-// Let every staged kernel use up to kStageSmemMax of dynamic shared memory.
+// One staged launch: the fixed-phase kernel when fixed_phase is set (pieces
+// of 8 bytes or less), else the per-piece kernel.
+cudaError_t launch_stage(const StageParams& p, int piece_bytes, int fixed_phase, int mode, int grid,
+                         int block, size_t smem, cudaStream_t st);
+// Let every staged kernel (both forms) use up to kStageSmemMax of dynamic
+// shared memory.
 cudaError_t stage_allow_max_smem();
 // Staged-kernel parameters for a plan (slab pointers, tile0 and b0 left for
 // the caller): nt tiles per (b, j) block, `units` units in the launch.

@@ -1,0 +1,283 @@
+// kernels_phase.cuh - fixed-phase form of the re-aligning copy path of the
+// Ulysses 4D all-to-all re-layout, for shapes whose [B, S_local, H, D] side is
+// dense (rows HDE = ng * R bytes apart) and whose gathered slabs all start the
+// same number of bytes past a 16-byte boundary.
+//
+// Element map as on the other paths (FastVideo API docs, device_communicators/
+// ulysses_a2a, `run_armed`): mode 0 out_r[b, j*S_local + s, h', d] =
+// x_j[b, s, r*(H/w) + h', d]; mode 1 is its inverse.
+//
+// Units, regions and the gathered side are those of the staged kernel
+// (kernels_stage.cuh): unit (b, j, t) is S_tile rows s0.. of plane b of strided
+// slab j with the matching row range of every gathered slab g (R = (H/w)*D*E
+// bytes per row and slab, ng gathered slabs: w, or T*w for T head-packed
+// tensors). Shared memory holds ng regions RS bytes apart; region g holds
+// range g starting a_g bytes in, a_g being the ranges' common address mod 16,
+// so the gathered side moves as aligned 16-byte vectors.
+//
+// The strided side of a unit is one contiguous segment of rows * HDE bytes,
+// moved as aligned 16-byte global chunks as well. Chunk c holds segment bytes
+// o .. o + 15 with o = 16c - a_s (a_s: the segment's address mod 16); byte o
+// is byte o mod R of run q = o / R, that is of head group q mod ng in row
+// q / ng, which region g = q mod ng holds at a_g + (q / ng) * R + o mod R.
+// Relative to row i0 = floor(o / HDE), the shared-memory places of a chunk's
+// 16 / G pieces (G bytes each, G dividing R, HDE and every base address)
+// depend only on o mod HDE. Thread t takes the chunks c = t + m * nthr, with
+// nthr a multiple of HDE / gcd(HDE, 16): 16 * nthr is then a multiple of HDE,
+// every chunk of the thread has the same o mod HDE, and chunk m starts
+// step_rows = 16 * nthr / HDE rows after chunk m - 1. So a thread works out
+// its piece offsets once per unit, and a piece costs one add and one shared
+// access.
+//
+// Mode 0: strided chunks -> pieces into the regions (phase A), regions ->
+// gathered ranges (phase B). Mode 1: gathered ranges -> regions (A), pieces
+// from the regions -> strided chunks (B). Global bytes outside the unit are
+// never read or written: a partial chunk at either end of a range or segment
+// moves only its valid pieces.
+#pragma once
+
+#include <cstdint>
+
+#include "kernels_stage.cuh"  // PieceOf, Chunk16, load_pieces, store_pieces
+#include "kernels_vec.cuh"    // FastDiv, fdiv, streaming load/store helpers, PDL switch
+#include "ulysses_a2a.h"
+
+namespace ua2a {
+
+struct PhaseParams {
+  const char* in[ULYSSES_A2A_MAX_W];
+  char* out[ULYSSES_A2A_MAX_W];
+  int64_t S_local;
+  int64_t b0;             // first plane of this launch
+  int32_t R;              // bytes of one run, (H/w)*D*E
+  int32_t HDE;            // bytes of one strided row, ng * R (dense)
+  int32_t w;              // sequence blocks (j)
+  int32_t ng;             // head groups per strided row, and gathered slabs
+  int32_t rows_per_tile;  // S_tile
+  uint32_t units;         // nb * w * T
+  uint32_t tile0;         // first tile of each (b, j) block in this launch
+  int32_t RS;             // bytes per region in shared memory (a multiple of 16)
+  int32_t Cg;             // 16-byte chunks scanned per gathered range: (S_tile*R + 30) / 16
+  int32_t nthr;           // threads moving strided chunks, a multiple of HDE / gcd(HDE, 16)
+  int32_t step_rows;      // 16 * nthr / HDE
+  FastDiv div_T;          // tiles per (b, j) block in this launch
+  FastDiv div_w;
+  FastDiv div_R;
+  FastDiv div_HDE;
+  FastDiv div_Cg;
+};
+
+// Strided chunks in flight per thread (mode 0; 2 with 1-byte pieces, whose 16
+// offsets leave no registers for more) and gathered loads in flight per
+// thread (mode 1).
+constexpr int kPhaseUnroll = 4;
+
+// Shared-memory offsets of the 16 / G pieces of a strided chunk whose byte 0
+// is byte kap (0 <= kap < HDE) of a strided row, from that row's place in
+// region 0: piece n is byte col of the run of head group g in row dr (0 or
+// later) of the regions.
+template <int G>
+__device__ __forceinline__ void piece_offsets(int32_t (&off)[16 / G], int32_t kap, int32_t R,
+                                              int32_t RS, int32_t ng, const FastDiv& div_R) {
+  int32_t g = (int32_t)fdiv((uint32_t)kap, div_R);
+  int32_t col = kap - g * R;
+  int32_t dr = 0;
+#pragma unroll
+  for (int n = 0; n < 16 / G; ++n) {
+    off[n] = g * RS + dr * R + col;
+    col += G;
+    if (col == R) {  // the next piece starts the next run
+      col = 0;
+      if (++g == ng) {
+        g = 0;
+        ++dr;
+      }
+    }
+  }
+}
+
+// 256-thread CTAs; at least 5 resident per SM (4 with 1-byte pieces, whose
+// mode-1 instance spills at 48 registers).
+constexpr int kPhaseMinBlocksPerSm = 5;
+
+template <int G, int MODE>
+__global__ void __launch_bounds__(256, G == 1 ? 4 : kPhaseMinBlocksPerSm)
+    ua2a_phase_kernel(const __grid_constant__ PhaseParams p) {
+  using PT = typename PieceOf<G>::type;
+  constexpr int NP = 16 / G;  // pieces per chunk
+  extern __shared__ __align__(16) unsigned char sm[];
+#if UA2A_PDL
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
+  const int32_t R = p.R;
+  const int32_t HDE = p.HDE;
+  const int32_t RS = p.RS;
+  const int32_t tid = (int32_t)threadIdx.x;
+  for (uint32_t u = blockIdx.x; u < p.units; u += gridDim.x) {
+    // u = (b_rel * w + j) * T + t
+    const uint32_t q = fdiv(u, p.div_T);
+    const uint32_t t = u - q * p.div_T.d;
+    const uint32_t bl = fdiv(q, p.div_w);
+    const uint32_t j = q - bl * p.div_w.d;
+    const int64_t b = p.b0 + bl;
+    const int64_t s0 = (int64_t)(p.tile0 + t) * p.rows_per_tile;
+    const int64_t left = p.S_local - s0;
+    const int32_t rows = (int32_t)(left < p.rows_per_tile ? left : p.rows_per_tile);
+    const int32_t L = rows * R;      // bytes of each gathered range of this unit
+    const int32_t segB = rows * HDE;  // bytes of the strided segment
+    // the unit's range in every gathered slab, and its segment of strided slab j
+    const int64_t goff = ((b * p.w + j) * p.S_local + s0) * (int64_t)R;
+    const uintptr_t seg = reinterpret_cast<uintptr_t>(MODE == 0 ? p.in[j] : p.out[j]) +
+                          (uintptr_t)((b * p.S_local + s0) * (int64_t)HDE);
+    const int32_t a_s = (int32_t)(seg & 15u);
+    const int32_t a_g =
+        (int32_t)((reinterpret_cast<uintptr_t>(MODE == 0 ? p.out[0] : p.in[0]) + (uintptr_t)goff) & 15u);
+    char* const seg16 = reinterpret_cast<char*>(seg - (uintptr_t)a_s);  // 16-byte aligned
+    const int32_t nS = (a_s + segB + 15) >> 4;  // strided chunks of the segment
+
+    // This thread's strided chunks c = tid + m * nthr: the row i0 of its first
+    // chunk's byte 0 (o may be negative, o >= -15, so i0 >= -1 - 15 / HDE) and
+    // its phase kap = o - i0 * HDE. Chunk m's pieces sit at
+    // base0 + m * dbase + off[n] (>= 0 for every piece inside the segment).
+    const int32_t o_first = 16 * tid - a_s;
+    const int32_t i0 = (int32_t)fdiv((uint32_t)(o_first + 16 * HDE), p.div_HDE) - 16;
+    const int32_t kap = o_first - i0 * HDE;
+    const int32_t base0 = a_g + i0 * R;
+    const int32_t dbase = p.step_rows * R;
+    const bool mover = tid < p.nthr;
+    int32_t off[NP];
+
+    if (MODE == 0) {
+      // phase A: strided chunks -> regions, U loads in flight
+      constexpr int U = G == 1 ? 2 : kPhaseUnroll;
+      if (mover) {
+        piece_offsets<G>(off, kap, R, RS, p.ng, p.div_R);
+        for (int32_t m0 = 0; tid + m0 * p.nthr < nS; m0 += U) {
+          uint4 v[U];
+#pragma unroll
+          for (int k = 0; k < U; ++k) {
+            const int32_t c = tid + (m0 + k) * p.nthr;
+            if (c < nS) {
+              const int32_t o = 16 * c - a_s;
+              const int x0 = o < 0 ? -o : 0;
+              const int x1 = segB - o < 16 ? segB - o : 16;
+              if (x0 == 0 && x1 == 16)
+                v[k] = ld_stream(reinterpret_cast<const uint4*>(seg16 + 16 * c));
+              else
+                v[k] = load_pieces<G>(seg16 + 16 * c, x0, x1);
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < U; ++k) {
+            const int32_t c = tid + (m0 + k) * p.nthr;
+            if (c < nS) {
+              const int32_t o = 16 * c - a_s;
+              const int x0 = o < 0 ? -o : 0;
+              const int x1 = segB - o < 16 ? segB - o : 16;
+              const int32_t at = base0 + (m0 + k) * dbase;
+              Chunk16<G> cv;
+              cv.v = v[k];
+              if (x0 == 0 && x1 == 16) {
+#pragma unroll
+                for (int n = 0; n < NP; ++n) *reinterpret_cast<PT*>(sm + (at + off[n])) = cv.e[n];
+              } else {
+#pragma unroll
+                for (int n = 0; n < NP; ++n)
+                  if (n * G >= x0 && n * G < x1) *reinterpret_cast<PT*>(sm + (at + off[n])) = cv.e[n];
+              }
+            }
+          }
+        }
+      }
+      __syncthreads();
+      // phase B: regions -> gathered ranges, aligned on both sides
+      const int32_t nB = p.ng * p.Cg;
+      for (int32_t e = tid; e < nB; e += (int32_t)blockDim.x) {
+        const int32_t g = (int32_t)fdiv((uint32_t)e, p.div_Cg);
+        const int32_t c = e - g * p.Cg;
+        const int32_t o0 = 16 * c - a_g;
+        const int x0 = o0 < 0 ? -o0 : 0;
+        const int x1 = L - o0 < 16 ? L - o0 : 16;
+        if (x0 >= x1) continue;
+        char* d = p.out[g] + (goff + o0);
+        const uint4 v = *reinterpret_cast<const uint4*>(sm + (g * RS + 16 * c));
+        if (x0 == 0 && x1 == 16)
+          st_stream(reinterpret_cast<uint4*>(d), v);
+        else
+          store_pieces<G>(d, v, x0, x1);
+      }
+    } else {
+      // phase A: gathered ranges -> regions, kPhaseUnroll loads in flight
+      const int32_t nA = p.ng * p.Cg;
+      for (int32_t e0 = tid; e0 < nA; e0 += (int32_t)blockDim.x * kPhaseUnroll) {
+        uint4 v[kPhaseUnroll];
+#pragma unroll
+        for (int k = 0; k < kPhaseUnroll; ++k) {
+          const int32_t e = e0 + k * (int32_t)blockDim.x;
+          if (e < nA) {
+            const int32_t g = (int32_t)fdiv((uint32_t)e, p.div_Cg);
+            const int32_t c = e - g * p.Cg;
+            const int32_t o0 = 16 * c - a_g;
+            const int x0 = o0 < 0 ? -o0 : 0;
+            const int x1 = L - o0 < 16 ? L - o0 : 16;
+            const char* s = p.in[g] + (goff + o0);
+            if (x0 == 0 && x1 == 16)
+              v[k] = ld_stream(reinterpret_cast<const uint4*>(s));
+            else if (x0 < x1)
+              v[k] = load_pieces<G>(s, x0, x1);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kPhaseUnroll; ++k) {
+          const int32_t e = e0 + k * (int32_t)blockDim.x;
+          if (e < nA) {
+            const int32_t g = (int32_t)fdiv((uint32_t)e, p.div_Cg);
+            const int32_t c = e - g * p.Cg;
+            const int32_t o0 = 16 * c - a_g;
+            const int x0 = o0 < 0 ? -o0 : 0;
+            const int x1 = L - o0 < 16 ? L - o0 : 16;
+            unsigned char* slot = sm + (g * RS + 16 * c);
+            if (x0 == 0 && x1 == 16) {
+              *reinterpret_cast<uint4*>(slot) = v[k];
+            } else if (x0 < x1) {
+              Chunk16<G> cv;
+              cv.v = v[k];
+#pragma unroll
+              for (int n = 0; n < NP; ++n)
+                if (n * G >= x0 && n * G < x1) *reinterpret_cast<PT*>(slot + n * G) = cv.e[n];
+            }
+          }
+        }
+      }
+      __syncthreads();
+      // phase B: pieces from the regions -> strided chunks
+      if (mover) {
+        piece_offsets<G>(off, kap, R, RS, p.ng, p.div_R);
+        for (int32_t m = 0;; ++m) {
+          const int32_t c = tid + m * p.nthr;
+          if (c >= nS) break;
+          const int32_t o = 16 * c - a_s;
+          const int x0 = o < 0 ? -o : 0;
+          const int x1 = segB - o < 16 ? segB - o : 16;
+          const int32_t at = base0 + m * dbase;
+          Chunk16<G> cv;
+          if (x0 == 0 && x1 == 16) {
+#pragma unroll
+            for (int n = 0; n < NP; ++n) cv.e[n] = *reinterpret_cast<const PT*>(sm + (at + off[n]));
+            st_stream(reinterpret_cast<uint4*>(seg16 + 16 * c), cv.v);
+          } else {
+            cv.v = make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int n = 0; n < NP; ++n)
+              if (n * G >= x0 && n * G < x1) cv.e[n] = *reinterpret_cast<const PT*>(sm + (at + off[n]));
+            store_pieces<G>(seg16 + 16 * c, cv.v, x0, x1);
+          }
+        }
+      }
+    }
+    __syncthreads();  // the regions are reused by the next unit
+  }
+}
+
+}  // namespace ua2a

@@ -252,7 +252,8 @@ static int ua2a_impl_run_noalloc(const void* const* in_slabs, void* const* out_s
     }
     for (int l = 0; l < pl.launches; ++l) {
       p.b0 = chunked ? l : 0;
-      e = launch_stage(p, pl.vec_bytes, mode, pl.grid, pl.block, (size_t)pl.smem_bytes, st_);
+      e = launch_stage(p, pl.vec_bytes, pl.fixed_phase, mode, pl.grid, pl.block,
+                       (size_t)pl.smem_bytes, st_);
       if (e != cudaSuccess)
         return noalloc_report(err, errlen, ULYSSES_A2A_ERR_CUDA, "staged kernel launch failed (plane %lld)", l);
     }

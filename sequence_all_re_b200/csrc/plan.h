@@ -60,6 +60,14 @@ constexpr int kVecResidentCtasPerSm = 6;
 constexpr int64_t kStageTileTargetBytes = 16 * 1024;
 constexpr int64_t kStageSmemMax = 96 * 1024;
 constexpr int kStageBlock = 256;
+// Its fixed-phase form (kernels_phase.cuh): strided-side bytes per work unit,
+// and the fewest of the kStageBlock threads that must move strided chunks (a
+// multiple of HDE / gcd(HDE, 16) of them do). Measured on B200 (6- and
+// 12-byte runs, mode 0 / mode 1 of the copy bandwidth): units of 8 KB
+// 0.52 / 0.43 and 0.68 / 0.67, 16 KB 0.72 / 0.53 and 0.87 / 0.83, 32 KB
+// 0.74 / 0.62 and 0.91 / 0.89, 48 KB 0.70 / 0.65 and 0.76 / 0.79.
+constexpr int64_t kPhaseTileTargetBytes = 32 * 1024;
+constexpr int kPhaseMinMovers = 192;
 // AUTO moves launches of at most this many payload bytes with the vector
 // kernel even where TMA could take them: measured on B200 in CUDA-graph
 // replays, a vector launch costs about 0.6-1 us less (128 KiB: 1.3-1.5 us
@@ -99,6 +107,7 @@ struct Tuning {
   int order = -1;         // unit numbering (-1 = default)
   int chunk_units = -1;   // TMA: units per CTA (0 = persistent grid, -1 = default)
   int host_chunks = 0;    // host-buffer path pipeline depth (0 = default)
+  int staged_form = 0;    // staged path: 0 = fixed-phase form where it applies, 1 = per-piece
 };
 
 inline bool mul_overflows(int64_t a, int64_t b, int64_t* out) {
@@ -163,25 +172,33 @@ inline bool side_offsets(const void* const* in, int nin, void* const* out, int n
 
 // Geometry of the re-aligning (staged) path for runs of R bytes, ng head
 // groups per strided row (HDE = ng * R bytes) and S_local rows: the rows per
-// unit (about kStageTileTargetBytes of strided-side bytes, or rows_cap when
-// set), the 16-byte chunks scanned per strided row (Cs) and per gathered range
-// (Cg), and the shared memory of a CTA: ng regions of RS bytes (RS = 16*Cg
-// rounded to an odd number of 16-byte chunks, so that consecutive regions
-// start in different shared-memory banks) and ng 4-byte region offsets.
+// unit (about kStageTileTargetBytes of strided-side bytes, kPhaseTileTargetBytes
+// in the fixed-phase form, or rows_cap when set), the 16-byte chunks scanned
+// per strided row (Cs) and per gathered range (Cg), and the shared memory of a
+// CTA: ng regions of RS bytes and ng 4-byte region offsets. RS is 16*Cg
+// rounded up to an odd number of 16-byte chunks, so that consecutive regions
+// start in different shared-memory banks; in the fixed-phase form with at most
+// 4 regions, to a multiple of 128 bytes instead: one warp's 32 strided chunks
+// then cover at least 128 bytes of every region, and regions that start in
+// the same bank gave the fewest conflicts (modelled: 1.5 against 3.0
+// wavefronts per access on 6-byte runs; measured: 0.81 / 0.64 against
+// 0.74 / 0.62 of the copy bandwidth).
 // Returns false if not even one row fits kStageSmemMax.
 struct StageGeometry {
   int64_t rows = 0, tiles = 0, Cs = 0, Cg = 0, RS = 0, smem_bytes = 0;
 };
 
-inline bool stage_geometry(int64_t R, int64_t ng, int64_t S, int rows_cap, StageGeometry* g) {
+inline bool stage_geometry(int64_t R, int64_t ng, int64_t S, int rows_cap, StageGeometry* g,
+                           bool fixed_phase = false) {
   const int64_t HDE = ng * R;
   if (R < 1 || ng < 1 || S < 1 || HDE >= (int64_t(1) << 30)) return false;
-  int64_t rows = rows_cap > 0 ? rows_cap : kStageTileTargetBytes / HDE;
+  int64_t rows = rows_cap > 0 ? rows_cap
+                              : (fixed_phase ? kPhaseTileTargetBytes : kStageTileTargetBytes) / HDE;
   if (rows < 1) rows = 1;
   if (rows > S) rows = S;
   for (; rows >= 1; rows = rows > 1 ? rows / 2 : 0) {
     const int64_t Cg = (rows * R + 30) / 16;
-    const int64_t RS = 16 * (Cg % 2 ? Cg : Cg + 1);
+    const int64_t RS = 16 * (fixed_phase && ng <= 4 ? (Cg + 7) / 8 * 8 : (Cg % 2 ? Cg : Cg + 1));
     const int64_t smem = ng * RS + 4 * ng;
     if (smem <= kStageSmemMax && rows * HDE < (int64_t(1) << 30)) {
       g->rows = rows;
@@ -194,6 +211,16 @@ inline bool stage_geometry(int64_t R, int64_t ng, int64_t S, int rows_cap, Stage
     }
   }
   return false;
+}
+
+// Threads of a kStageBlock-thread CTA that move strided chunks in the
+// fixed-phase form for strided rows of HDE bytes: the largest multiple of
+// HDE / gcd(HDE, 16) up to kStageBlock (0 when there is none).
+inline int64_t phase_movers(int64_t HDE) {
+  int64_t g = 16;
+  while (HDE % g != 0) g >>= 1;
+  const int64_t period = HDE / g;
+  return period <= kStageBlock ? period * (kStageBlock / period) : 0;
 }
 
 // Public tuning struct -> internal knobs, with range checks (NULL = defaults).
@@ -212,6 +239,7 @@ inline bool tuning_from(const ulysses_a2a_tuning_t* t, Tuning* out, std::string*
   if (t->order < -1 || t->order > 1) return bad("order");
   if (t->chunk_units < -1) return bad("chunk_units");
   if (t->host_chunks < 0 || t->host_chunks > kHostMaxChunks) return bad("host_chunks");
+  if (t->staged_form < 0 || t->staged_form > 1) return bad("staged_form");
   out->rows_per_tile = t->rows_per_tile;
   out->ctas_per_sm = t->ctas_per_sm;
   out->stages = t->stages;
@@ -220,6 +248,7 @@ inline bool tuning_from(const ulysses_a2a_tuning_t* t, Tuning* out, std::string*
   out->order = t->order;
   out->chunk_units = t->chunk_units;
   out->host_chunks = t->host_chunks;
+  out->staged_form = t->staged_form;
   return true;
 }
 
@@ -534,8 +563,22 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     const bool forced_stage = forced_path == ULYSSES_A2A_PATH_STAGED;
     if (forced_stage ||
         (forced_path == ULYSSES_A2A_PATH_AUTO && !peeled && v <= kStageMaxPiece && only_out < 0)) {
+      // The fixed-phase form takes a dense [B, S, H, D] side whose gathered
+      // slabs share one offset past a 16-byte boundary, in pieces of at most
+      // 8 bytes, when enough threads can move strided chunks (unless the
+      // per-piece form is asked for).
+      const int ng = w * ntensors;
+      const int64_t HDE = row_bytes * ng;
+      bool fixed_phase = tune.staged_form == 0 && pitch * E == HDE && v <= 8 &&
+                         phase_movers(HDE) >= kPhaseMinMovers;
+      {
+        const void* const* gs = mode == 0 ? const_cast<const void* const*>(out) : in;
+        for (int k = 1; k < ng && fixed_phase; ++k)
+          fixed_phase = (reinterpret_cast<uintptr_t>(gs[k]) & 15u) ==
+                        (reinterpret_cast<uintptr_t>(gs[0]) & 15u);
+      }
       StageGeometry sg;
-      if (stage_geometry(row_bytes, (int64_t)w * ntensors, S, tune.rows_per_tile, &sg)) {
+      if (stage_geometry(row_bytes, ng, S, tune.rows_per_tile, &sg, fixed_phase)) {
         const int64_t nbl = chunked ? 1 : B;
         int64_t su;
         if (mul_overflows((int64_t)w * nbl, sg.tiles, &su) || su >= (int64_t(1) << 31)) {
@@ -546,6 +589,7 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
         // free up), or a grid-stride grid of ctas_per_sm CTAs per SM
         const int64_t sgrid = tune.ctas_per_sm > 0 ? (int64_t)num_sms * tune.ctas_per_sm : su;
         p->path = ULYSSES_A2A_PATH_STAGED;
+        p->fixed_phase = fixed_phase ? 1 : 0;
         p->rows_per_tile = sg.rows;
         p->tiles_per_block = sg.tiles;
         p->tail_rows = S % sg.rows;

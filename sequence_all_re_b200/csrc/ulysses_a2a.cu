@@ -261,8 +261,54 @@ cudaError_t launch_stage_t(const StageParams& p, int mode, int grid, int block, 
                    : launch_pdl(ua2a::ua2a_stage_kernel<G, 1>, grid, block, smem, st, p);
 }
 
-cudaError_t launch_stage(const StageParams& p, int piece_bytes, int mode, int grid, int block,
-                         size_t smem, cudaStream_t st) {
+// The fixed-phase kernel's parameters from the staged kernel's: the same
+// units and regions, plus the threads that move strided chunks and the rows
+// between a thread's consecutive chunks.
+PhaseParams phase_params(const StageParams& s) {
+  PhaseParams p{};
+  for (int k = 0; k < ULYSSES_A2A_MAX_W; ++k) {
+    p.in[k] = s.in[k];
+    p.out[k] = s.out[k];
+  }
+  p.S_local = s.S_local;
+  p.b0 = s.b0;
+  p.R = s.R;
+  p.HDE = s.HDE;
+  p.w = s.w;
+  p.ng = s.ng;
+  p.rows_per_tile = s.rows_per_tile;
+  p.units = s.units;
+  p.tile0 = s.tile0;
+  p.RS = s.RS;
+  p.Cg = s.Cg;
+  p.nthr = (int32_t)ua2a::phase_movers(s.HDE);
+  p.step_rows = 16 * p.nthr / s.HDE;
+  p.div_T = s.div_T;
+  p.div_w = s.div_w;
+  p.div_R = s.div_R;
+  p.div_HDE = ua2a::FastDiv((uint32_t)s.HDE);
+  p.div_Cg = s.div_Cg;
+  return p;
+}
+
+template <int G>
+cudaError_t launch_phase_t(const PhaseParams& p, int mode, int grid, int block, size_t smem,
+                           cudaStream_t st) {
+  return mode == 0 ? launch_pdl(ua2a::ua2a_phase_kernel<G, 0>, grid, block, smem, st, p)
+                   : launch_pdl(ua2a::ua2a_phase_kernel<G, 1>, grid, block, smem, st, p);
+}
+
+cudaError_t launch_stage(const StageParams& p, int piece_bytes, int fixed_phase, int mode, int grid,
+                         int block, size_t smem, cudaStream_t st) {
+  if (fixed_phase) {
+    const PhaseParams q = phase_params(p);
+    switch (piece_bytes) {
+      case 8: return launch_phase_t<8>(q, mode, grid, block, smem, st);
+      case 4: return launch_phase_t<4>(q, mode, grid, block, smem, st);
+      case 2: return launch_phase_t<2>(q, mode, grid, block, smem, st);
+      default: return launch_phase_t<1>(q, mode, grid, block, smem, st);
+    }
+  }
   switch (piece_bytes) {
     case 16: return launch_stage_t<16>(p, mode, grid, block, smem, st);
     case 8: return launch_stage_t<8>(p, mode, grid, block, smem, st);
@@ -283,8 +329,23 @@ cudaError_t stage_allow_t() {
   return e;
 }
 
+template <int G>
+cudaError_t phase_allow_t() {
+  cudaError_t e = cudaFuncSetAttribute(ua2a::ua2a_phase_kernel<G, 0>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)ua2a::kStageSmemMax);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(ua2a::ua2a_phase_kernel<G, 1>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ua2a::kStageSmemMax);
+  return e;
+}
+
 cudaError_t stage_allow_max_smem() {
-  cudaError_t e = stage_allow_t<16>();
+  cudaError_t e = phase_allow_t<8>();
+  if (e == cudaSuccess) e = phase_allow_t<4>();
+  if (e == cudaSuccess) e = phase_allow_t<2>();
+  if (e == cudaSuccess) e = phase_allow_t<1>();
+  if (e == cudaSuccess) e = stage_allow_t<16>();
   if (e == cudaSuccess) e = stage_allow_t<8>();
   if (e == cudaSuccess) e = stage_allow_t<4>();
   if (e == cudaSuccess) e = stage_allow_t<2>();
@@ -340,7 +401,7 @@ StageParams stage_params(int64_t S, int w, int ntensors, int E, const ulysses_a2
   p.rows_per_tile = (int32_t)pl.rows_per_tile;
   p.units = (uint32_t)units;
   StageGeometry sg;
-  stage_geometry(pl.row_bytes, p.ng, S, (int)pl.rows_per_tile, &sg);
+  stage_geometry(pl.row_bytes, p.ng, S, (int)pl.rows_per_tile, &sg, pl.fixed_phase != 0);
   p.RS = (int32_t)sg.RS;
   p.Cs = (int32_t)sg.Cs;
   p.Cg = (int32_t)sg.Cg;
@@ -393,7 +454,8 @@ int run_device(ulysses_a2a_ctx* ctx, const void* const* in, void* const* out, in
     }
     for (int l = 0; l < launches; ++l) {
       p.b0 = chunked ? l : 0;
-      cudaError_t e = launch_stage(p, pl.vec_bytes, mode, grid, pl.block, (size_t)pl.smem_bytes, st);
+      cudaError_t e = launch_stage(p, pl.vec_bytes, pl.fixed_phase, mode, grid, pl.block,
+                                   (size_t)pl.smem_bytes, st);
       if (e != cudaSuccess) return cuda_fail(ctx, "staged kernel launch", e);
       ctx->launches++;
     }
@@ -893,6 +955,7 @@ static int ua2a_impl_get_settings(const ulysses_a2a_ctx* ctx, int32_t* path,
     t->order = u.order;
     t->chunk_units = u.chunk_units;
     t->host_chunks = u.host_chunks;
+    t->staged_form = u.staged_form;
   }
   return ULYSSES_A2A_OK;
 }

@@ -55,8 +55,8 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_plan_struct_layout_matches_header():
-    # int32 path, vec_bytes; 6 x int64; 6 x int32; int64; 2 x int32; int64; 2 x int32
-    # -> 112 bytes
+    # int32 path, vec_bytes; 6 x int64; 6 x int32; int64; 2 x int32; int64;
+    # 2 x int32 (peeled, fixed_phase) -> 112 bytes
     assert ctypes.sizeof(_lib.PlanT) == 112
     # two pointers, 4 x int64, 4 x int32, int64 -> 72 bytes
     assert ctypes.sizeof(_lib.DescT) == 72
@@ -192,13 +192,19 @@ def test_runs_off_16_bytes_take_the_staged_path():
 
 
 def test_staged_geometry():
-    # 200-byte runs, 8 head groups of 1600-byte rows: units of 10 rows (16 KB),
-    # one per (b, j, tile) covering every head group
+    # 200-byte runs, 8 head groups of 1600-byte rows: one unit per (b, j, tile)
+    # covering every head group
     # (8-byte vectors: AUTO keeps the vector path, so the staged path is forced)
     rc, p, _ = plan(8, 2, 4725, 8, 100)
     assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 8
+    # dense and aligned alike, the fixed-phase form: units of 32 KB (20 rows)
     rc, p, _ = plan(8, 2, 4725, 8, 100, forced_path=PATH_STAGED)
-    assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 8
+    assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 8 and p.fixed_phase == 1
+    assert p.rows_per_tile == 32 * 1024 // 1600 == 20 and p.tail_rows == 4725 % 20
+    # a pitched [B, S, H, D] side (rows of 8 * 100 + 4 elements): the per-piece
+    # form, units of 16 KB (10 rows)
+    rc, p, _ = plan_ex(8, 2, 4725, 8, 100, 8 * 100 + 4, forced_path=PATH_STAGED)
+    assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 8 and p.fixed_phase == 0
     assert p.rows_per_tile == 16 * 1024 // 1600 == 10 and p.tail_rows == 4725 % 10
     # one short-lived CTA per unit
     assert p.units == 8 * 2 * p.tiles_per_block and p.grid == p.units and p.block == 256
@@ -215,6 +221,62 @@ def test_staged_geometry():
     assert rc == OK and p.path == PATH_VEC
     rc, _, msg = plan(4, 1, 16, 4 * 8, 512, E=8, forced_path=PATH_STAGED)
     assert rc == ERR_UNSUPPORTED and "shared memory" in msg
+
+
+def test_staged_fixed_phase_form():
+    # a dense [B, S, H, D] side with gathered slabs at one offset: the fixed-
+    # phase form (each thread's strided chunks share one phase within a row)
+    for w, H, D, E, piece in ((4, 4, 3, 2, 2), (4, 4, 3, 4, 4), (2, 2, 5, 1, 1), (3, 3, 5, 2, 2),
+                             (3, 6, 5, 2, 4)):
+        for mode in (0, 1):
+            rc, p, _ = plan(w, 2, 1000, H, D, mode=mode, E=E)
+            assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == piece
+            assert p.fixed_phase == 1, (w, H, D, E, mode)
+            rc, p, _ = plan(w, 2, 1000, H, D, mode=mode, E=E, forced_path=PATH_STAGED)
+            assert rc == OK and p.fixed_phase == 1
+    # units of 32 KB of strided rows (6-byte runs, 24-byte rows), one CTA
+    # each; with at most 4 regions they sit 128 bytes apart
+    rc, p, _ = plan(4, 1, 100000, 4, 3)
+    assert p.rows_per_tile == 32 * 1024 // 24 and p.grid == p.units == 4 * p.tiles_per_block
+    cg = (p.rows_per_tile * 6 + 30) // 16
+    assert p.smem_bytes == (4 * 16 * ((cg + 7) // 8 * 8) + 4 * 4 + 15) // 16 * 16
+    # with more regions, an odd number of 16-byte chunks apart
+    rc, p, _ = plan(8, 1, 100000, 8, 3)
+    cg = (p.rows_per_tile * 6 + 30) // 16
+    assert p.fixed_phase == 1 and p.rows_per_tile == 32 * 1024 // 48
+    assert p.smem_bytes == (8 * 16 * (cg if cg % 2 else cg + 1) + 4 * 8 + 15) // 16 * 16
+    # gathered slabs at one offset past 16 bytes, strided slabs at others
+    w, B, S, H, D, E = 4, 1, 64, 4, 3, 2
+    ins, outs = fake_slabs(w, B * S * H * D * E)
+    rc, p, _ = ulysses_a2a_plan([a + 2 * k for k, a in enumerate(ins)], [a + 6 for a in outs],
+                                B, S, H, D, w, 0, 0, E)
+    assert rc == OK and p.path == PATH_STAGED and p.fixed_phase == 1
+    # the per-piece form when asked for
+    rc, p, _ = plan(4, 2, 1000, 4, 3, staged_form=1)
+    assert rc == OK and p.path == PATH_STAGED and p.fixed_phase == 0
+    assert p.rows_per_tile == 16 * 1024 // 24
+    # gathered slabs at different offsets: per-piece form
+    rc, p, _ = ulysses_a2a_plan(ins, [a + 2 * k for k, a in enumerate(outs)], B, S, H, D, w, 0, 0, E)
+    assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 2 and p.fixed_phase == 0
+    rc, p, _ = ulysses_a2a_plan([a + 2 * k for k, a in enumerate(outs)], ins, B, S, H, D, w, 1, 0, E)
+    assert rc == OK and p.path == PATH_STAGED and p.fixed_phase == 0
+    # a pitched [B, S, H, D] side: per-piece form
+    rc, p, _ = plan_ex(4, 2, 37, 4, 3, 4 * 3 + 1)
+    assert rc == OK and p.path == PATH_STAGED and p.fixed_phase == 0
+    # 16-byte pieces (forced on an aligned shape): per-piece form
+    rc, p, _ = plan(4, 1, 8192, 24, 128, forced_path=PATH_STAGED)
+    assert rc == OK and p.vec_bytes == 16 and p.fixed_phase == 0
+    # rows whose phase period leaves too few of the 256 threads moving chunks:
+    # 87-byte rows (period 87, 2 * 87 = 174 threads) take the per-piece form,
+    # 81-byte rows (period 81, 3 * 81 = 243 threads) the fixed-phase one
+    rc, p, _ = plan(3, 1, 64, 3, 29, E=1)
+    assert rc == OK and p.path == PATH_STAGED and p.fixed_phase == 0
+    rc, p, _ = plan(3, 1, 64, 3, 27, E=1)
+    assert rc == OK and p.path == PATH_STAGED and p.fixed_phase == 1
+    # the VEC and TMA paths never set it
+    for args in ((4, 1, 8192, 24, 128), (8, 2, 4725, 8, 100)):
+        rc, p, _ = plan(*args)
+        assert rc == OK and p.path != PATH_STAGED and p.fixed_phase == 0
 
 
 def test_vec_when_misaligned_pointer():
@@ -379,14 +441,15 @@ def test_tuning_knobs():
 @pytest.mark.parametrize("knob,value", [("rows_per_tile", 257), ("rows_per_tile", -1),
                                         ("ctas_per_sm", 33), ("stages", 33), ("producers", 9),
                                         ("order", 2), ("chunk_units", -2), ("lookahead", -1),
-                                        ("host_chunks", 65), ("host_chunks", -1)])
+                                        ("host_chunks", 65), ("host_chunks", -1),
+                                        ("staged_form", 2), ("staged_form", -1)])
 def test_tuning_out_of_range_is_rejected(knob, value):
     rc, _, msg = plan(4, 1, 64, 8, 64, **{knob: value})
     assert rc == ERR_INVALID and knob in msg
 
 
 def test_tuning_struct_layout():
-    assert ctypes.sizeof(_lib.TuningT) == 32
+    assert ctypes.sizeof(_lib.TuningT) == 36
 
 
 def test_ring_split_between_producers_loads_and_stores():
@@ -733,7 +796,7 @@ def test_planner_invariants(w, hw, B, S, D, E, mode, chunked, path, rows, ntenso
         assert path in (PATH_AUTO, PATH_STAGED)
         hde = ntensors * hw * w * D * E
         assert 1 <= p.rows_per_tile <= S and p.tiles_per_block == -(-S // p.rows_per_tile)
-        assert p.rows_per_tile == 1 or p.rows_per_tile * hde <= 16 * 1024 or rows
+        assert p.rows_per_tile == 1 or p.rows_per_tile * hde <= (32 if p.fixed_phase else 16) * 1024 or rows
         assert p.units == w * nb * p.tiles_per_block and p.grid == p.units
         assert p.block == 256 and p.smem_bytes <= 96 * 1024
         v = p.vec_bytes

@@ -99,6 +99,17 @@ def test_vector_shapes_are_named_by_their_sizes_and_leave_the_tma_path():
         assert (wl["off"], wl["goff"]) == (off, goff)
 
 
+def test_staged_form_shapes_are_named_by_their_sizes_and_dense():
+    for name, (w, B, S, H, D, E) in bench.STAGED_FORM_SHAPES.items():
+        parts = {p[0]: p[1:] for p in name.split("_")}
+        assert (int(parts["w"]), int(parts["S"]), int(parts["H"]), int(parts["D"])) == (w, S, H, D)
+        assert ("fp32" in name) == (E == 4) and ("u8" in name) == (E == 1)
+        row = (H // w) * D * E
+        assert row % 16 != 0                   # TMA cannot take them
+        p = plan_dict(w, B, S, H, D, _lib.PATH_STAGED, E)
+        assert p["path"] == _lib.PATH_STAGED and p["fixed_phase"] == 1, name
+
+
 def test_one_sided_offsets_are_keyed_apart():
     assert bench.workload_key(4, 1, 8, 24, 128, "vec", 2, 2) == "vec:w4_B1_S8_H24_D128_bf16_base2"
     assert bench.workload_key(4, 1, 8, 24, 128, "vec", 2, 2, 0) == \

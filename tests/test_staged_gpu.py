@@ -54,6 +54,11 @@ def test_narrow_runs_take_the_staged_path(case, mode, chunked):
         assert p["path"] == (PATH_STAGED if p["vec_bytes"] <= 4 else PATH_VEC)
         run_case(xs, mode, chunked=chunked, a2a=a2a)
         run_case(xs, mode, chunked=chunked, a2a=a2a, path=PATH_STAGED)
+        # dense rows and aligned slabs: the fixed-phase form, unless the
+        # per-piece form is asked for
+        assert a2a.plan([t.cuda() for t in xs], mode)["fixed_phase"] == 1
+        run_case(xs, mode, chunked=chunked, a2a=a2a, path=PATH_STAGED, tuning=dict(staged_form=1))
+        assert a2a.plan([t.cuda() for t in xs], mode)["fixed_phase"] == 0
 
 
 SHAPES = [
@@ -86,6 +91,106 @@ def test_misaligned_bases_every_offset(offset, side):
     for mode, src in ((0, xs), (1, ys)):
         for chunked in (False, True):
             run_case(src, mode, chunked=chunked, **kw)
+
+
+class _GuardedAt:
+    """Output slabs at per-slab byte offsets past a 16-byte boundary, poisoned,
+    with 64 guard bytes on either side."""
+
+    def __init__(self, shape, dtype, offsets):
+        self.nbytes = torch.empty(shape, dtype=dtype, device="meta").numel() * \
+            torch.empty((), dtype=dtype).element_size()
+        self.offsets = list(offsets)
+        self.bufs, self.slabs = [], []
+        for off in offsets:
+            lo = 64 + off
+            buf = torch.full((self.nbytes + 128 + 16,), 0x5A, dtype=torch.uint8, device="cuda")
+            buf[lo:lo + self.nbytes].fill_(0xFF)
+            self.bufs.append(buf)
+            self.slabs.append(buf[lo:lo + self.nbytes].view(dtype).view(shape))
+
+    def check_guards(self):
+        for buf, off in zip(self.bufs, self.offsets):
+            lo = 64 + off
+            assert bool((buf[:lo] == 0x5A).all()), "bytes before an output slab were written"
+            assert bool((buf[lo + self.nbytes:] == 0x5A).all()), "bytes after an output slab were written"
+
+
+def _at(t, off):
+    raw = torch.empty(t.numel() * t.element_size() + off, dtype=torch.uint8, device="cuda")
+    v = raw[off:].view(t.dtype).view(t.shape)
+    v.copy_(t)
+    return v
+
+
+def _run_at(a2a, xs_cpu, mode, in_offs, out_offs, chunked, fixed_phase):
+    """One call with slab k of the inputs in_offs[k] and of the outputs out_offs[k]
+    bytes past a 16-byte boundary; the plan's form is checked, then every byte
+    against the oracle and the bytes around the outputs."""
+    w = len(xs_cpu)
+    xs = [_at(t, o) for t, o in zip(xs_cpu, in_offs)]
+    g = _GuardedAt(oracle.output_shape(tuple(xs_cpu[0].shape), mode, w), xs_cpu[0].dtype, out_offs)
+    p = a2a.plan(xs, mode, out=g.slabs)
+    assert p["path"] == PATH_STAGED and p["fixed_phase"] == fixed_phase, p
+    a2a.run(xs, mode, chunked=chunked, out=g.slabs)
+    a2a.status()
+    want = oracle.ulysses_a2a(xs_cpu, mode)
+    for k in range(w):
+        assert torch.equal(bits(g.slabs[k].cpu()), bits(want[k])), k
+    g.check_guards()
+
+
+# (w, B, S_local, H, D, E): dense narrow runs of 6, 12, 5, 10, 20 and 36 bytes
+PHASE = [(4, 2, 300, 4, 3, 2), (4, 1, 257, 4, 3, 4), (2, 2, 97, 2, 5, 1), (3, 2, 151, 3, 5, 2),
+         (3, 1, 211, 6, 5, 2), (8, 1, 99, 8, 9, 4)]
+
+
+@pytest.mark.parametrize("case", PHASE, ids=lambda c: "w{}B{}S{}H{}D{}E{}".format(*c))
+@pytest.mark.parametrize("mode", [0, 1])
+def test_fixed_phase_form_every_offset(case, mode):
+    # the gathered slabs at one offset (every piece-aligned value), the strided
+    # slabs each at its own: the fixed-phase kernel, whole and per plane
+    w, B, S, H, D, E = case
+    shape = slab_shape(mode, w, B, S, H, D)
+    xs = [t.view(INT[E]).reshape(shape)
+          for t in random_byte_slabs(shape[:-1] + (shape[-1] * E,), w, seed0=900 + S)]
+    G = 1
+    while G < 8 and ((H // w) * D * E) % (2 * G) == 0:
+        G *= 2
+    with UlyssesA2A(0, E) as a2a:
+        for a in range(0, 16, G):
+            strided = [(a + 3 * G * k) % 16 for k in range(w)]
+            gathered = [a] * w
+            ins, outs = (strided, gathered) if mode == 0 else (gathered, strided)
+            for chunked in (False, True):
+                _run_at(a2a, xs, mode, ins, outs, chunked, 1)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_per_piece_form_when_gathered_offsets_differ(mode):
+    w, B, S, H, D, E = 4, 2, 300, 4, 3, 2
+    shape = slab_shape(mode, w, B, S, H, D)
+    xs = [t.view(torch.int16).reshape(shape)
+          for t in random_byte_slabs(shape[:-1] + (shape[-1] * E,), w, seed0=950)]
+    with UlyssesA2A(0, E) as a2a:
+        gathered, strided = [0, 2, 4, 6], [2] * w
+        ins, outs = (strided, gathered) if mode == 0 else (gathered, strided)
+        _run_at(a2a, xs, mode, ins, outs, False, 0)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_fixed_phase_form_with_few_rows_per_unit(mode):
+    # units of 1, 2 and 5 rows (24 to 120 strided bytes): most threads move no
+    # strided chunk, and a unit's first and last chunks are partial
+    w, B, S, H, D, E = 4, 2, 37, 4, 3, 2
+    shape = slab_shape(mode, w, B, S, H, D)
+    xs = [t.view(torch.int16).reshape(shape)
+          for t in random_byte_slabs(shape[:-1] + (shape[-1] * E,), w, seed0=960)]
+    with UlyssesA2A(0, E) as a2a:
+        for rows in (1, 2, 5):
+            a2a.set_tuning(rows_per_tile=rows)
+            _run_at(a2a, xs, mode, [2] * w, [6] * w, False, 1)
+            _run_at(a2a, xs, mode, [0] * w, [0] * w, True, 1)
 
 
 def test_pitched_slabs_through_the_staged_path():
