@@ -79,11 +79,19 @@ constexpr int64_t kVecSmallLaunchBytes = int64_t(64) << 20;
 // Smallest vector unit: small launches get units of payload / (2 * SMs),
 // down to this size, so that every SM has work.
 constexpr int64_t kVecMinTileBytes = 2 * 1024;
-// AUTO re-aligns through shared memory only what the vector kernel would move
-// in pieces of at most this many bytes: measured on B200, 8-byte vectors
-// (0.86-0.91 of the copy bandwidth on 200-byte runs and on slabs 8 bytes off
-// 16) beat the staged kernel, 4- and 2-byte vectors (0.27-0.55) lose to it.
+// AUTO re-aligns through shared memory what the vector kernel would move in
+// pieces of at most kStageMaxPiece bytes, and 8-byte-granular runs shorter
+// than kPhaseOverVec8Run bytes when the fixed-phase form applies. Measured on
+// B200 (mode 0 / mode 1 of the copy bandwidth, bench.py --staged-forms):
+// 4-, 2- and 1-byte vectors reach 0.16-0.66 against 0.63-0.92 for the
+// fixed-phase form; 8-byte vectors 0.43 / 0.45 on 8-byte runs, 0.80 / 0.82 on
+// 24, 0.87 / 0.58 on 40 and 0.90 / 0.61 on 72 (a run of few vectors pays the
+// vector kernel's per-vector decode), against 0.97 / 0.83, 0.91 / 0.81,
+// 0.88 / 0.81 and 0.89 / 0.80 for the fixed-phase form; from 104-byte runs on
+// the vectors win (0.91 / 0.84 against 0.85 / 0.81; 136: 0.92 / 0.93 against
+// 0.85 / 0.81).
 constexpr int kStageMaxPiece = 4;
+constexpr int64_t kPhaseOverVec8Run = 96;
 // Unit numbering: 0 = destination rank outermost, 1 = innermost.
 constexpr int kDefaultOrder = 1;
 // Host-buffer entry point: sequence chunks its H2D copies, kernels and D2H
@@ -557,26 +565,29 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     p->block = kVecBlock;
     p->grid = (int32_t)(units < g ? units : g);
 
+    // The staged path's fixed-phase form takes a dense [B, S, H, D] side whose
+    // gathered slabs share one offset past a 16-byte boundary, in pieces of at
+    // most 8 bytes, when enough threads can move strided chunks (unless the
+    // per-piece form is asked for).
+    const int ng = w * ntensors;
+    const int64_t HDE = row_bytes * ng;
+    bool fixed_phase = tune.staged_form == 0 && pitch * E == HDE && v <= 8 &&
+                       phase_movers(HDE) >= kPhaseMinMovers;
+    {
+      const void* const* gs = mode == 0 ? const_cast<const void* const*>(out) : in;
+      for (int k = 1; k < ng && fixed_phase; ++k)
+        fixed_phase = (reinterpret_cast<uintptr_t>(gs[k]) & 15u) ==
+                      (reinterpret_cast<uintptr_t>(gs[0]) & 15u);
+    }
     // The re-aligning path takes what the vector path could only move in
-    // pieces of kStageMaxPiece bytes or less (or what it is forced onto),
-    // except one-output launches.
+    // pieces of kStageMaxPiece bytes or less, and short 8-byte-granular runs
+    // that the fixed-phase form takes (or what it is forced onto), except
+    // one-output launches.
     const bool forced_stage = forced_path == ULYSSES_A2A_PATH_STAGED;
-    if (forced_stage ||
-        (forced_path == ULYSSES_A2A_PATH_AUTO && !peeled && v <= kStageMaxPiece && only_out < 0)) {
-      // The fixed-phase form takes a dense [B, S, H, D] side whose gathered
-      // slabs share one offset past a 16-byte boundary, in pieces of at most
-      // 8 bytes, when enough threads can move strided chunks (unless the
-      // per-piece form is asked for).
-      const int ng = w * ntensors;
-      const int64_t HDE = row_bytes * ng;
-      bool fixed_phase = tune.staged_form == 0 && pitch * E == HDE && v <= 8 &&
-                         phase_movers(HDE) >= kPhaseMinMovers;
-      {
-        const void* const* gs = mode == 0 ? const_cast<const void* const*>(out) : in;
-        for (int k = 1; k < ng && fixed_phase; ++k)
-          fixed_phase = (reinterpret_cast<uintptr_t>(gs[k]) & 15u) ==
-                        (reinterpret_cast<uintptr_t>(gs[0]) & 15u);
-      }
+    const bool auto_stage =
+        forced_path == ULYSSES_A2A_PATH_AUTO && !peeled && only_out < 0 &&
+        (v <= kStageMaxPiece || (v == 8 && fixed_phase && row_bytes < kPhaseOverVec8Run));
+    if (forced_stage || auto_stage) {
       StageGeometry sg;
       if (stage_geometry(row_bytes, ng, S, tune.rows_per_tile, &sg, fixed_phase)) {
         const int64_t nbl = chunked ? 1 : B;

@@ -803,7 +803,7 @@ def test_planner_invariants(w, hw, B, S, D, E, mode, chunked, path, rows, ntenso
         assert p.row_bytes % v == 0 and (p.row_pitch * E) % v == 0
         assert v == 16 or (p.row_bytes % (2 * v) or (p.row_pitch * E) % (2 * v))
         if path == PATH_AUTO:
-            assert v <= 4
+            assert v <= 4 or (v == 8 and p.fixed_phase and p.row_bytes < 96)
         return
     # tiles cover every sequence row exactly once per (r, b, j) block
     assert 1 <= p.rows_per_tile <= min(S, 256)
@@ -831,7 +831,13 @@ def test_planner_invariants(w, hw, B, S, D, E, mode, chunked, path, rows, ntenso
         assert p.grid == p.units
         v = p.vec_bytes
         assert v in (1, 2, 4, 8, 16) and p.row_bytes % v == 0 and (p.row_pitch * E) % v == 0
-        # AUTO leaves narrower vectors to the staged path unless a row is too long
+        # AUTO leaves narrower vectors to the staged path unless a row is too long,
+        # and 8-byte vectors of runs under 96 bytes to its fixed-phase form
         assert path == PATH_VEC or v >= 8 or not _one_row_fits_stage(hw * D * E, ntensors * w)
+        if path == PATH_AUTO and v == 8 and p.row_bytes < 96:
+            rc2, p2, _ = _lib.ulysses_a2a_plan_ex(ins, outs, B, S, H, D, w, mode, chunked, E,
+                                                  forced_path=PATH_STAGED, ntensors=ntensors,
+                                                  rows_per_tile=rows)
+            assert rc2 != OK or p2.fixed_phase == 0
         # the widest width the run length and the pitch allow (pointers are 4 KiB aligned)
         assert v == 16 or (p.row_bytes % (2 * v) or (p.row_pitch * E) % (2 * v))

@@ -31,7 +31,7 @@ NARROW = [
     (8, 2, 53, 8, 100, 2),      # 200-byte runs: 8-byte pieces (AUTO: 8-byte vectors)
     (3, 2, 29, 6, 5, 1),        # 10-byte runs: 2-byte pieces, odd rank count
     (2, 3, 33, 2, 7, 1),        # 7-byte runs: 1-byte pieces
-    (2, 2, 40, 2, 1, 8),        # 8-byte runs (AUTO: 8-byte vectors)
+    (2, 2, 40, 2, 1, 8),        # 8-byte runs (AUTO: the fixed-phase form, 8-byte pieces)
     (16, 1, 21, 16, 3, 2),      # w = 16
     (1, 2, 31, 3, 5, 2),        # w = 1: a copy
     (5, 1, 4000, 5, 3, 2),      # many rows per unit
@@ -42,8 +42,8 @@ NARROW = [
 @pytest.mark.parametrize("mode", [0, 1])
 @pytest.mark.parametrize("chunked", [False, True], ids=["whole", "per_plane"])
 def test_narrow_runs_take_the_staged_path(case, mode, chunked):
-    # AUTO re-aligns pieces of 4 bytes or less through shared memory and moves
-    # 8-byte ones as vectors; the staged path forced gives the same bytes
+    # AUTO re-aligns pieces of 4 bytes or less through shared memory, and
+    # 8-byte ones of short runs; the staged path forced gives the same bytes
     w, B, S, H, D, E = case
     shape = slab_shape(mode, w, B, S, H, D)
     xs = [t.view(INT[E]).reshape(shape)
@@ -51,7 +51,8 @@ def test_narrow_runs_take_the_staged_path(case, mode, chunked):
     with UlyssesA2A(0, E) as a2a:
         p = a2a.plan([t.cuda() for t in xs], mode)
         assert p["vec_bytes"] < 16
-        assert p["path"] == (PATH_STAGED if p["vec_bytes"] <= 4 else PATH_VEC)
+        # (8-byte vectors stay on the vector path from 96-byte runs on)
+        assert p["path"] == (PATH_STAGED if p["vec_bytes"] <= 4 or p["row_bytes"] < 96 else PATH_VEC)
         run_case(xs, mode, chunked=chunked, a2a=a2a)
         run_case(xs, mode, chunked=chunked, a2a=a2a, path=PATH_STAGED)
         # dense rows and aligned slabs: the fixed-phase form, unless the

@@ -36,6 +36,7 @@ CASES = [
     (16, 3, 19, 16, 64, "bf16", 1, 0, VEC),       # the vector path, chunked
     (2, 2, 17, 4, 3, "bf16", 0, 0, STAGED),       # 12-byte runs: re-aligned in shared memory
     (2, 3, 17, 4, 3, "bf16", 1, 0, STAGED),       # chunked
+    (4, 2, 33, 4, 4, "bf16", 0, 0, STAGED),       # 8-byte runs: the fixed-phase form
     (4, 2, 33, 8, 64, "bf16", 0, 2, VEC),         # every slab 2 bytes off 16: peeled vectors
     (4, 2, 33, 8, 64, "bf16", 1, 8, VEC),         # chunked, 8 bytes off: peeled vectors
     (4, 2, 33, 8, 64, "bf16", 1, (6, 0), VEC),    # inputs 6 bytes off, outputs aligned: joined
