@@ -62,8 +62,9 @@ constexpr int64_t kStageSmemMax = 96 * 1024;
 constexpr int kStageBlock = 256;
 // Its fixed-phase form (kernels_phase.cuh): strided-side bytes per work unit,
 // and the fewest of the kStageBlock threads that must move strided chunks (a
-// multiple of HDE / gcd(HDE, 16) of them do). Measured on B200 (6- and
-// 12-byte runs, mode 0 / mode 1 of the copy bandwidth): units of 8 KB
+// multiple of HDE / gcd(HDE, 16) of them do). Measured on B200 with this
+// constant rebuilt at each size (6- and 12-byte runs, mode 0 / mode 1 of the
+// copy bandwidth, regions an odd number of chunks apart): units of 8 KB
 // 0.52 / 0.43 and 0.68 / 0.67, 16 KB 0.72 / 0.53 and 0.87 / 0.83, 32 KB
 // 0.74 / 0.62 and 0.91 / 0.89, 48 KB 0.70 / 0.65 and 0.76 / 0.79.
 constexpr int64_t kPhaseTileTargetBytes = 32 * 1024;
