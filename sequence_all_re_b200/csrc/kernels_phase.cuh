@@ -65,6 +65,7 @@ struct PhaseParams {
   FastDiv div_R;
   FastDiv div_HDE;
   FastDiv div_Cg;
+  FastDiv div_ng;
 };
 
 // Strided chunks in flight per thread (mode 0; 2 with 1-byte pieces, whose 16
@@ -94,6 +95,23 @@ __device__ __forceinline__ void piece_offsets(int32_t (&off)[16 / G], int32_t ka
       }
     }
   }
+}
+
+// Asynchronous 16-byte copy global -> shared (cp.async, cached in L2 only):
+// the data goes to shared memory without passing through registers, so a
+// thread can have all its chunks of a unit in flight at once. Both
+// addresses must be 16-byte aligned.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Wait until at most N of this thread's committed groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // 256-thread CTAs; at least 5 resident per SM (4 with 1-byte pieces, whose
@@ -208,73 +226,72 @@ __global__ void __launch_bounds__(256, G == 1 ? 4 : kPhaseMinBlocksPerSm)
           store_pieces<G>(d, v, x0, x1);
       }
     } else {
-      // phase A: gathered ranges -> regions, kPhaseUnroll loads in flight
+      // phase A: gathered ranges -> regions by cp.async, numbered region-
+      // fastest (e = c * ng + g), so that each thread issues the chunks
+      // holding the unit's first rowsA rows (c < cgA) before the rest: two
+      // commit groups. The strided chunks inside those rows (c < cA) are
+      // assembled while the second group is still in flight.
+      const int32_t rowsA = rows >> 1;
+      const int32_t cgA = (a_g + rowsA * R + 15) >> 4;
+      const int32_t cA = (a_s + rowsA * HDE) >> 4;
       const int32_t nA = p.ng * p.Cg;
-      for (int32_t e0 = tid; e0 < nA; e0 += (int32_t)blockDim.x * kPhaseUnroll) {
-        uint4 v[kPhaseUnroll];
-#pragma unroll
-        for (int k = 0; k < kPhaseUnroll; ++k) {
-          const int32_t e = e0 + k * (int32_t)blockDim.x;
-          if (e < nA) {
-            const int32_t g = (int32_t)fdiv((uint32_t)e, p.div_Cg);
-            const int32_t c = e - g * p.Cg;
-            const int32_t o0 = 16 * c - a_g;
-            const int x0 = o0 < 0 ? -o0 : 0;
-            const int x1 = L - o0 < 16 ? L - o0 : 16;
-            const char* s = p.in[g] + (goff + o0);
-            if (x0 == 0 && x1 == 16)
-              v[k] = ld_stream(reinterpret_cast<const uint4*>(s));
-            else if (x0 < x1)
-              v[k] = load_pieces<G>(s, x0, x1);
-          }
+      bool first_open = true;
+      for (int32_t e = tid; e < nA; e += (int32_t)blockDim.x) {
+        const int32_t c = (int32_t)fdiv((uint32_t)e, p.div_ng);
+        const int32_t g = e - c * p.ng;
+        if (first_open && c >= cgA) {
+          cp_async_commit();
+          first_open = false;
         }
+        const int32_t o0 = 16 * c - a_g;
+        const int x0 = o0 < 0 ? -o0 : 0;
+        const int x1 = L - o0 < 16 ? L - o0 : 16;
+        if (x0 >= x1) continue;
+        const char* src = p.in[g] + (goff + o0);
+        unsigned char* slot = sm + (g * RS + 16 * c);
+        if (x0 == 0 && x1 == 16) {
+          cp_async16(slot, src);
+        } else {  // a partial chunk at either end of a range: its valid pieces
+          Chunk16<G> cv;
+          cv.v = load_pieces<G>(src, x0, x1);
 #pragma unroll
-        for (int k = 0; k < kPhaseUnroll; ++k) {
-          const int32_t e = e0 + k * (int32_t)blockDim.x;
-          if (e < nA) {
-            const int32_t g = (int32_t)fdiv((uint32_t)e, p.div_Cg);
-            const int32_t c = e - g * p.Cg;
-            const int32_t o0 = 16 * c - a_g;
-            const int x0 = o0 < 0 ? -o0 : 0;
-            const int x1 = L - o0 < 16 ? L - o0 : 16;
-            unsigned char* slot = sm + (g * RS + 16 * c);
-            if (x0 == 0 && x1 == 16) {
-              *reinterpret_cast<uint4*>(slot) = v[k];
-            } else if (x0 < x1) {
-              Chunk16<G> cv;
-              cv.v = v[k];
-#pragma unroll
-              for (int n = 0; n < NP; ++n)
-                if (n * G >= x0 && n * G < x1) *reinterpret_cast<PT*>(slot + n * G) = cv.e[n];
-            }
-          }
+          for (int n = 0; n < NP; ++n)
+            if (n * G >= x0 && n * G < x1) *reinterpret_cast<PT*>(slot + n * G) = cv.e[n];
         }
       }
+      if (first_open) cp_async_commit();
+      cp_async_commit();
+      // phase B: pieces from the regions -> strided chunks, first those of
+      // the first rowsA rows, then (once every copy has landed) the rest
+      auto gather = [&](int32_t c, int32_t m) {
+        const int32_t o = 16 * c - a_s;
+        const int x0 = o < 0 ? -o : 0;
+        const int x1 = segB - o < 16 ? segB - o : 16;
+        const int32_t at = base0 + m * dbase;
+        Chunk16<G> cv;
+        if (x0 == 0 && x1 == 16) {
+#pragma unroll
+          for (int n = 0; n < NP; ++n) cv.e[n] = *reinterpret_cast<const PT*>(sm + (at + off[n]));
+          st_stream(reinterpret_cast<uint4*>(seg16 + 16 * c), cv.v);
+        } else {
+          cv.v = make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int n = 0; n < NP; ++n)
+            if (n * G >= x0 && n * G < x1) cv.e[n] = *reinterpret_cast<const PT*>(sm + (at + off[n]));
+          store_pieces<G>(seg16 + 16 * c, cv.v, x0, x1);
+        }
+      };
+      cp_async_wait<1>();
       __syncthreads();
-      // phase B: pieces from the regions -> strided chunks
+      int32_t m = 0;
       if (mover) {
         piece_offsets<G>(off, kap, R, RS, p.ng, p.div_R);
-        for (int32_t m = 0;; ++m) {
-          const int32_t c = tid + m * p.nthr;
-          if (c >= nS) break;
-          const int32_t o = 16 * c - a_s;
-          const int x0 = o < 0 ? -o : 0;
-          const int x1 = segB - o < 16 ? segB - o : 16;
-          const int32_t at = base0 + m * dbase;
-          Chunk16<G> cv;
-          if (x0 == 0 && x1 == 16) {
-#pragma unroll
-            for (int n = 0; n < NP; ++n) cv.e[n] = *reinterpret_cast<const PT*>(sm + (at + off[n]));
-            st_stream(reinterpret_cast<uint4*>(seg16 + 16 * c), cv.v);
-          } else {
-            cv.v = make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int n = 0; n < NP; ++n)
-              if (n * G >= x0 && n * G < x1) cv.e[n] = *reinterpret_cast<const PT*>(sm + (at + off[n]));
-            store_pieces<G>(seg16 + 16 * c, cv.v, x0, x1);
-          }
-        }
+        for (; tid + m * p.nthr < cA; ++m) gather(tid + m * p.nthr, m);
       }
+      cp_async_wait<0>();
+      __syncthreads();
+      if (mover)
+        for (; tid + m * p.nthr < nS; ++m) gather(tid + m * p.nthr, m);
     }
     __syncthreads();  // the regions are reused by the next unit
   }

@@ -288,6 +288,7 @@ PhaseParams phase_params(const StageParams& s) {
   p.div_R = s.div_R;
   p.div_HDE = ua2a::FastDiv((uint32_t)s.HDE);
   p.div_Cg = s.div_Cg;
+  p.div_ng = ua2a::FastDiv((uint32_t)s.ng);
   return p;
 }
 
