@@ -562,9 +562,10 @@ def vec_shape_block(device, peak, sampler, seconds=0.5):
         torch.cuda.synchronize()
         if not all(torch.equal(z[k], x[k]) for k in range(w)):
             raise SystemExit(f"vector-path shape {name}: round trip mismatch")
+        p1 = a2a.plan(y, 1, out=z)
         out[name] = {"payload_bytes": P, "path": PATH_NAMES[p["path"]],
                      "vec_bytes": p["vec_bytes"], "peeled": p["peeled"],
-                     "fixed_phase": p["fixed_phase"],
+                     "fixed_phase": p["fixed_phase"], "mode1_path": PATH_NAMES[p1["path"]],
                      "row_bytes": p["row_bytes"], "base_offset_bytes": off,
                      "gathered_base_offset_bytes": goff, **res}
         # the other of the two paths, forced: the vector kernel where AUTO
@@ -607,7 +608,7 @@ def staged_forms_block(device, peak, sampler, seconds=0.5):
                                    ("per_piece", 3, {"staged_form": 1}), ("vec", 2, {})):
             a2a.set_path(path)
             a2a.set_tuning(**knobs)
-            p = a2a.plan(x, 0, out=y)
+            p, p1 = a2a.plan(x, 0, out=y), a2a.plan(y, 1, out=z)
             for t in z:
                 t.zero_()
             res = per_mode_block(a2a, x, y, z, P, stream, peak, sampler, seconds)
@@ -615,7 +616,8 @@ def staged_forms_block(device, peak, sampler, seconds=0.5):
             if not all(torch.equal(z[k], x[k]) for k in range(w)):
                 raise SystemExit(f"shape {name}: round trip mismatch ({label})")
             row[label] = {"path": PATH_NAMES[p["path"]], "vec_bytes": p["vec_bytes"],
-                          "fixed_phase": p["fixed_phase"],
+                          "fixed_phase": p["fixed_phase"], "mode1_path": PATH_NAMES[p1["path"]],
+                          "mode1_fixed_phase": p1["fixed_phase"],
                           "mode0": res["mode0"]["frac"], "mode1": res["mode1"]["frac"],
                           "sm_mhz": (res["mode0"]["clocks"] or {}).get("sm_mhz")}
         out[name] = row

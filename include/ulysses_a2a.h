@@ -78,8 +78,8 @@ extern "C" {
                                     STAGED when VEC could only use vectors
                                     of 4 bytes or less and cannot peel them
                                     (see plan_t.peeled), or 8-byte vectors
-                                    on runs under 96 bytes that the staged
-                                    path's fixed-phase form takes           */
+                                    that the staged path's fixed-phase form
+                                    takes (mode 0: runs under 96 bytes)     */
 #define ULYSSES_A2A_PATH_TMA  1  /* cp.async.bulk.tensor load -> smem -> store */
 #define ULYSSES_A2A_PATH_VEC  2  /* 16/8/4/2/1-byte LDG/STG copy, or 16-byte
                                     vectors between peeled heads and tails

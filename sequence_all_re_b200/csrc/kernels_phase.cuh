@@ -108,6 +108,22 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
+// Bytes [x0, x1) of the aligned 16-byte global chunk at h as G-byte loads
+// cached in L2 with the normal policy, as cp.async.cg caches the whole chunks
+// beside them: a partial chunk shares its 32-byte sector with a neighbour that
+// cp.async reads, and an evict-first load would let that sector leave L2 in
+// between (the other bytes of the result are zero and never used).
+template <int G>
+__device__ __forceinline__ uint4 load_pieces_l2(const char* h, int x0, int x1) {
+  using PT = typename PieceOf<G>::type;
+  Chunk16<G> c;
+  c.v = make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int k = 0; k < 16 / G; ++k)
+    if (k * G >= x0 && k * G < x1) c.e[k] = __ldcg(reinterpret_cast<const PT*>(h + k * G));
+  return c.v;
+}
+
 // Wait until at most N of this thread's committed groups are still in flight.
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
@@ -234,15 +250,22 @@ __global__ void __launch_bounds__(256, G == 1 ? 4 : kPhaseMinBlocksPerSm)
       const int32_t rowsA = rows >> 1;
       const int32_t cgA = (a_g + rowsA * R + 15) >> 4;
       const int32_t cA = (a_s + rowsA * HDE) >> 4;
-      const int32_t nA = p.ng * p.Cg;
+      // Blocks of 8 chunks (128 bytes) of one region, regions fastest:
+      // e = (cb * ng + g) * 8 + k moves chunk c = cb * 8 + k of region g; the
+      // first group takes whole blocks up to cgA8 >= cgA.
+      const int32_t cgA8 = (cgA + 7) & ~7;
+      const int32_t nA = p.ng * ((p.Cg + 7) & ~7);
       bool first_open = true;
       for (int32_t e = tid; e < nA; e += (int32_t)blockDim.x) {
-        const int32_t c = (int32_t)fdiv((uint32_t)e, p.div_ng);
-        const int32_t g = e - c * p.ng;
-        if (first_open && c >= cgA) {
+        const int32_t q = e >> 3;
+        const int32_t cb = (int32_t)fdiv((uint32_t)q, p.div_ng);
+        const int32_t g = q - cb * p.ng;
+        const int32_t c = cb * 8 + (e & 7);
+        if (first_open && c >= cgA8) {
           cp_async_commit();
           first_open = false;
         }
+        if (c >= p.Cg) continue;
         const int32_t o0 = 16 * c - a_g;
         const int x0 = o0 < 0 ? -o0 : 0;
         const int x1 = L - o0 < 16 ? L - o0 : 16;
@@ -253,7 +276,7 @@ __global__ void __launch_bounds__(256, G == 1 ? 4 : kPhaseMinBlocksPerSm)
           cp_async16(slot, src);
         } else {  // a partial chunk at either end of a range: its valid pieces
           Chunk16<G> cv;
-          cv.v = load_pieces<G>(src, x0, x1);
+          cv.v = load_pieces_l2<G>(src, x0, x1);
 #pragma unroll
           for (int n = 0; n < NP; ++n)
             if (n * G >= x0 && n * G < x1) *reinterpret_cast<PT*>(slot + n * G) = cv.e[n];

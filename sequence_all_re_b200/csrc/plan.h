@@ -81,16 +81,16 @@ constexpr int64_t kVecSmallLaunchBytes = int64_t(64) << 20;
 // down to this size, so that every SM has work.
 constexpr int64_t kVecMinTileBytes = 2 * 1024;
 // AUTO re-aligns through shared memory what the vector kernel would move in
-// pieces of at most kStageMaxPiece bytes, and 8-byte-granular runs shorter
-// than kPhaseOverVec8Run bytes when the fixed-phase form applies. Measured on
-// B200 (mode 0 / mode 1 of the copy bandwidth, bench.py --staged-forms):
-// 4-, 2- and 1-byte vectors reach 0.16-0.66 against 0.63-0.92 for the
-// fixed-phase form; 8-byte vectors 0.43 / 0.45 on 8-byte runs, 0.80 / 0.82 on
-// 24, 0.87 / 0.58 on 40 and 0.90 / 0.61 on 72 (a run of few vectors pays the
-// vector kernel's per-vector decode), against 0.97 / 0.83, 0.91 / 0.81,
-// 0.88 / 0.81 and 0.89 / 0.80 for the fixed-phase form; from 104-byte runs on
-// the vectors win (0.91 / 0.84 against 0.85 / 0.81; 136: 0.92 / 0.93 against
-// 0.85 / 0.81).
+// pieces of at most kStageMaxPiece bytes, and 8-byte-granular runs when the
+// fixed-phase form applies: in mode 1 always, in mode 0 below
+// kPhaseOverVec8Run bytes. Measured on B200 (mode 0 / mode 1 of the copy
+// bandwidth, bench.py --staged-forms): 4-, 2- and 1-byte vectors reach
+// 0.16-0.54 against 0.60-0.97 for the fixed-phase form. 8-byte vectors: 0.43 /
+// 0.45 on 8-byte runs, 0.75 / 0.79 on 24, 0.84 / 0.66 on 40, 0.87 / 0.61 on 72
+// (a run of few vectors pays the vector kernel's per-vector decode), 0.88 /
+// 0.69-0.88 on 104, 0.89 / 0.88-0.91 on 136 and 0.89 / 0.92 on 200, against
+// 0.93 / 1.01, 0.88 / 1.01, 0.85 / 0.97, 0.85 / 0.96, 0.84 / 0.96, 0.85 / 0.96
+// and 0.85 / 0.95 for the fixed-phase form.
 constexpr int kStageMaxPiece = 4;
 constexpr int64_t kPhaseOverVec8Run = 96;
 // Unit numbering: 0 = destination rank outermost, 1 = innermost.
@@ -581,13 +581,14 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
                       (reinterpret_cast<uintptr_t>(gs[0]) & 15u);
     }
     // The re-aligning path takes what the vector path could only move in
-    // pieces of kStageMaxPiece bytes or less, and short 8-byte-granular runs
-    // that the fixed-phase form takes (or what it is forced onto), except
-    // one-output launches.
+    // pieces of kStageMaxPiece bytes or less, and 8-byte-granular runs that
+    // the fixed-phase form takes (mode 0: runs under kPhaseOverVec8Run bytes),
+    // or what it is forced onto, except one-output launches.
     const bool forced_stage = forced_path == ULYSSES_A2A_PATH_STAGED;
     const bool auto_stage =
         forced_path == ULYSSES_A2A_PATH_AUTO && !peeled && only_out < 0 &&
-        (v <= kStageMaxPiece || (v == 8 && fixed_phase && row_bytes < kPhaseOverVec8Run));
+        (v <= kStageMaxPiece ||
+         (v == 8 && fixed_phase && (mode == 1 || row_bytes < kPhaseOverVec8Run)));
     if (forced_stage || auto_stage) {
       StageGeometry sg;
       if (stage_geometry(row_bytes, ng, S, tune.rows_per_tile, &sg, fixed_phase)) {
