@@ -4,7 +4,8 @@ Each case draws the rank count (1..16), element size (1/2/4/8), B, S_local, H,
 D, mode, chunking (per plane, through the staging window or not), a row pitch
 on the [B, S_local, H, D] side, input and output base offsets past a 16-byte
 boundary (independently), head-packed tensors (T = 2, 3), a forced path (or
-AUTO), the tuning knobs (rows per unit, unit order, grid-stride grids) and the
+AUTO), the tuning knobs (rows per unit, unit order, grid-stride grids, the
+staged path's fixed-phase or per-piece form) and the
 entry point: ``run``, a bound call, the allocation-free C entry point, or the
 host-buffer call (the last two for dense, unpacked slabs).
 The element map is the one the FastVideo API docs give for ``run_armed``
@@ -55,8 +56,9 @@ def _one_case(rng, case, ctxs):
     path = rng.choice([PATH_AUTO, PATH_AUTO, PATH_AUTO, PATH_TMA, PATH_VEC, PATH_STAGED])
     a2a = ctxs[E]
     a2a.set_path(path)
+    form = rng.choice([0, 0, 1])
     a2a.set_tuning(rows_per_tile=rng.choice([0, 0, 1, 3, 7]), order=rng.choice([-1, 0, 1]),
-                   ctas_per_sm=rng.choice([0, 0, 0, 1, 3]))
+                   ctas_per_sm=rng.choice([0, 0, 0, 1, 3]), staged_form=form)
     dt = INT[E]
     entry = rng.choice(["run", "run", "run", "bind", "noalloc", "host"])
     if entry in ("noalloc", "host") and (T != 1 or gap or chunked == 2):
@@ -71,7 +73,7 @@ def _one_case(rng, case, ctxs):
     n_p = (B * S - 1) * P + T * H * D
     gshape = (B, S * w, H // w, D)
     desc = f"case {case}: E={E} w={w} B={B} S={S} H={H} D={D} mode={mode} chunked={chunked} " \
-           f"T={T} gap={gap} off={off_in}/{off_out} path={path} entry={entry}"
+           f"T={T} gap={gap} off={off_in}/{off_out} path={path} form={form} entry={entry}"
 
     def call(xs, m, out):
         if entry == "bind":
