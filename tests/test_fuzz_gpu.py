@@ -12,8 +12,9 @@ The element map is the one the FastVideo API docs give for ``run_armed``
 (device_communicators/ulysses_a2a). Expected values come from the oracle
 (the pitched form for pitched and packed cases); outputs are poisoned and
 fenced, gaps between pitched rows must stay untouched. A forced path that
-cannot take the shape (TMA on an unaligned or packed call) must be refused
-before any launch.
+cannot take the shape (TMA on an unaligned or packed call, the staged path on
+a strided row longer than its shared memory) must be refused before any
+launch.
 """
 
 import random
@@ -144,8 +145,10 @@ def _one_case(rng, case, ctxs):
                     assert torch.equal(back[j].cpu(), packed[j]), (desc, j)
         return "ran"
     except A2AError as e:
-        # only a forced TMA path may be refused (a shape it cannot describe)
-        assert path == PATH_TMA and e.code == _lib.ERR_UNSUPPORTED, (desc, str(e))
+        # only a forced path may be refused: TMA on a shape it cannot describe,
+        # the staged path on a strided row too long for its shared memory
+        assert e.code == _lib.ERR_UNSUPPORTED and (
+            path == PATH_TMA or (path == PATH_STAGED and "shared memory" in str(e))), (desc, str(e))
         return "refused"
 
 
