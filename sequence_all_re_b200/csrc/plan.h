@@ -68,7 +68,11 @@ constexpr int kStageBlock = 256;
 // 0.52 / 0.43 and 0.68 / 0.67, 16 KB 0.72 / 0.53 and 0.87 / 0.83, 32 KB
 // 0.74 / 0.62 and 0.91 / 0.89, 48 KB 0.70 / 0.65 and 0.76 / 0.79.
 constexpr int64_t kPhaseTileTargetBytes = 32 * 1024;
-constexpr int kPhaseMinMovers = 192;
+// With 128 or more movers the fixed-phase form still beats the per-piece one
+// (measured, mode 0 / mode 1: 135 movers, 10-byte runs 0.52 / 0.59 against
+// 0.43 / 0.37; 175 movers, 5-byte runs 0.44 / 0.41 against 0.23 / 0.21); a
+// phase period of at most 256 chunks always leaves more than 128.
+constexpr int kPhaseMinMovers = 128;
 // AUTO moves launches of at most this many payload bytes with the vector
 // kernel even where TMA could take them: measured on B200 in CUDA-graph
 // replays, a vector launch costs about 0.6-1 us less (128 KiB: 1.3-1.5 us

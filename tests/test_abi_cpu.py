@@ -269,13 +269,14 @@ def test_staged_fixed_phase_form():
     # 16-byte pieces (forced on an aligned shape): per-piece form
     rc, p, _ = plan(4, 1, 8192, 24, 128, forced_path=PATH_STAGED)
     assert rc == OK and p.vec_bytes == 16 and p.fixed_phase == 0
-    # rows whose phase period leaves too few of the 256 threads moving chunks:
-    # 87-byte rows (period 87, 2 * 87 = 174 threads) take the per-piece form,
-    # 81-byte rows (period 81, 3 * 81 = 243 threads) the fixed-phase one
-    rc, p, _ = plan(3, 1, 64, 3, 29, E=1)
+    # rows whose phase period exceeds 256 chunks leave no thread a fixed phase:
+    # 261-byte rows take the per-piece form; 87-byte rows (period 87, 2 * 87 =
+    # 174 threads move chunks) and 81-byte rows (3 * 81 = 243) the fixed-phase one
+    rc, p, _ = plan(3, 1, 64, 3, 87, E=1)
     assert rc == OK and p.path == PATH_STAGED and p.fixed_phase == 0
-    rc, p, _ = plan(3, 1, 64, 3, 27, E=1)
-    assert rc == OK and p.path == PATH_STAGED and p.fixed_phase == 1
+    for D in (29, 27):
+        rc, p, _ = plan(3, 1, 64, 3, D, E=1)
+        assert rc == OK and p.path == PATH_STAGED and p.fixed_phase == 1
     # the VEC and TMA paths never set it
     for args in ((4, 1, 8192, 24, 128), (8, 2, 4725, 8, 100)):
         rc, p, _ = plan(*args)

@@ -55,7 +55,7 @@ def replay_unit(R, ng, G, rows, S_tile, a_s, a_g):
     HDE = ng * R
     Cg, RS = region_stride(R, ng, S_tile)
     nthr = phase_movers(HDE)
-    assert nthr >= 192 and (16 * nthr) % HDE == 0
+    assert nthr >= 128 and (16 * nthr) % HDE == 0
     step_rows = 16 * nthr // HDE
     segB, L = rows * HDE, rows * R
     nS = (a_s + segB + 15) >> 4
@@ -114,8 +114,8 @@ SHAPES = [(6, 2), (12, 4), (3, 1), (10, 2), (5, 1), (20, 4), (24, 8), (36, 4), (
 def test_fixed_phase_piece_placement(R, G):
     rng = random.Random(1000 + R)
     cases = 0
-    for ng in (1, 2, 3, 4, 6, 8, 16, 24, 64):
-        if phase_movers(ng * R) < 192:
+    for ng in (1, 2, 3, 4, 6, 8, 16, 24, 27, 35, 64):
+        if phase_movers(ng * R) < 128:
             continue
         for _ in range(3):
             S_tile = rng.choice([1, 2, 3, 5, 64, max(1, 32768 // (ng * R))])
