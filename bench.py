@@ -107,7 +107,7 @@ VEC_SHAPES = {
 }
 # Dense shapes with runs off 16 bytes (about 256 MiB each; bf16 unless noted):
 # name -> (w, B, S, H, D, element bytes). --staged-forms times each on the
-# staged path's two forms, and on the vector path; the first eight have
+# staged path's two forms, and on the vector path; the first ten have
 # pieces of 4 bytes or less, the others 8 bytes.
 STAGED_FORM_SHAPES = {
     "w4_S2796202_H4_D3": (4, 1, 2796202, 4, 3, 2),             # 6-byte runs, 4 regions
@@ -118,6 +118,8 @@ STAGED_FORM_SHAPES = {
     "w2_S13421772_H2_D5_u8": (2, 1, 13421772, 2, 5, 1),         # 5-byte runs, 1-byte pieces
     "w4_S838860_H8_D5": (4, 1, 838860, 8, 5, 2),                # 20-byte runs
     "w8_S116508_H8_D9_fp32": (8, 1, 116508, 8, 9, 4),           # 36-byte runs
+    "w27_S36822_H27_D5": (27, 1, 36822, 27, 5, 2),              # 10-byte runs, 135 movers
+    "w35_S43826_H35_D5_u8": (35, 1, 43826, 35, 5, 1),           # 5-byte runs, 175 movers
     "w4_S2097152_H4_D4": (4, 1, 2097152, 4, 4, 2),              # 8-byte runs
     "w4_S2796202_H4_D6_fp32": (4, 1, 2796202, 4, 6, 4),         # 24-byte runs
     "w4_S419430_H4_D20": (4, 1, 419430, 4, 20, 2),              # 40-byte runs
