@@ -79,7 +79,7 @@ extern "C" {
                                     of 4 bytes or less and cannot peel them
                                     (see plan_t.peeled), or 8-byte vectors
                                     that the staged path's fixed-phase form
-                                    takes (mode 0: runs under 96 bytes)     */
+                                    takes                                   */
 #define ULYSSES_A2A_PATH_TMA  1  /* cp.async.bulk.tensor load -> smem -> store */
 #define ULYSSES_A2A_PATH_VEC  2  /* 16/8/4/2/1-byte LDG/STG copy, or 16-byte
                                     vectors between peeled heads and tails

@@ -68,7 +68,18 @@ struct PhaseParams {
   FastDiv div_HDE;
   FastDiv div_Cg;
   FastDiv div_ng;
+  // mode 0: threads that build gathered chunks (a multiple of R / gcd(R, 16)),
+  // and the region chunk count padded to such a multiple
+  int32_t nthr0;
+  int32_t Cpad;
+  FastDiv div_Cpad;
 };
+
+// Mode 0 keeps the strided segment in shared memory as loaded, its 16-byte
+// chunks permuted within each 128-byte block: byte x sits at swz(x). Bits 4-6
+// are XORed with bits 9-11, which spreads one warp's piece accesses (16*ng
+// bytes apart in the segment) over the banks.
+__device__ __forceinline__ int32_t swz(int32_t x) { return x ^ (((x >> 9) & 7) << 4); }
 
 // Strided chunks in flight per thread in mode 0 (2 with 1-byte pieces, whose
 // 16 offsets leave no registers for more). Measured on B200 against 6 and 8
@@ -185,7 +196,95 @@ __global__ void __launch_bounds__(256, G == 1 ? 4 : kPhaseMinBlocksPerSm)
     const bool mover = tid < p.nthr;
     int32_t off[NP];
 
-    if (MODE == 0) {
+    if constexpr (MODE == 0 && G >= 4) {
+      // Pieces of 4 bytes or more: gather form.
+      // phase A: the strided segment's chunks land by cp.async in the
+      // swizzled image, in two commit groups: those holding the unit's first
+      // rowsA rows (c < cI1) first.
+      const int32_t rowsA = rows >> 1;
+      const int32_t cI1 = (a_s + rowsA * HDE + 15) >> 4;
+      {
+        bool first_open = true;
+        for (int32_t c = tid; c < nS; c += (int32_t)blockDim.x) {
+          if (first_open && c >= cI1) {
+            cp_async_commit();
+            first_open = false;
+          }
+          const int32_t o = 16 * c - a_s;
+          unsigned char* dst = sm + swz(16 * c);
+          if (o >= 0 && segB - o >= 16) {
+            cp_async16(dst, seg16 + 16 * c);
+          } else {  // a partial chunk at either end of the segment: its valid pieces
+            const int x0 = o < 0 ? -o : 0;
+            const int x1 = segB - o < 16 ? segB - o : 16;
+            Chunk16<G> cv;
+            cv.v = load_pieces_l2<G>(seg16 + 16 * c, x0, x1);
+#pragma unroll
+            for (int n = 0; n < NP; ++n)
+              if (n * G >= x0 && n * G < x1) *reinterpret_cast<PT*>(dst + n * G) = cv.e[n];
+          }
+        }
+        if (first_open) cp_async_commit();
+        cp_async_commit();
+      }
+      // phase B: gathered chunks built from the image and stored. Thread tid
+      // takes chunks e = tid + m * nthr0 of the ng regions laid end to end,
+      // Cpad chunks each; chunk c of region g holds region bytes
+      // q = 16c - a_g .. q + 15, byte q being byte q mod R of row q / R of
+      // head group g, segment byte (q / R) * HDE + g * R + q mod R. All of a
+      // thread's chunks share q mod R, so the segment offsets of its pieces
+      // from row q0 / R, group g are one list.
+      const int32_t r_n = (a_g + L + 15) >> 4;        // chunks holding range bytes
+      const int32_t cB1 = (a_g + rowsA * R) >> 4;     // chunks inside the first rowsA rows
+      const bool mover0 = tid < p.nthr0;
+      if (mover0) {
+        const int32_t q = 16 * tid - a_g + 16 * R;    // >= 0, same phase as 16 * tid - a_g
+        int32_t col = q - (int32_t)fdiv((uint32_t)q, p.div_R) * R;
+        int32_t drow = 0;
+#pragma unroll
+        for (int n = 0; n < NP; ++n) {
+          off[n] = drow * HDE + col;
+          col += G;
+          if (col == R) {
+            col = 0;
+            ++drow;
+          }
+        }
+      }
+      auto build = [&](int32_t e, bool first) {
+        const int32_t g = (int32_t)fdiv((uint32_t)e, p.div_Cpad);
+        const int32_t c = e - g * p.Cpad;
+        if (c >= r_n || (c < cB1) != first) return;
+        const int32_t q0 = 16 * c - a_g;
+        const int32_t i0 = (int32_t)fdiv((uint32_t)(q0 + 16 * R), p.div_R) - 16;  // floor(q0 / R)
+        const int32_t base = a_s + i0 * HDE + g * R;
+        char* d = p.out[g] + (goff + q0);
+        Chunk16<G> cv;
+        if (q0 >= 0 && L - q0 >= 16) {
+#pragma unroll
+          for (int n = 0; n < NP; ++n) cv.e[n] = *reinterpret_cast<const PT*>(sm + swz(base + off[n]));
+          st_stream(reinterpret_cast<uint4*>(d), cv.v);
+        } else {
+          const int x0 = q0 < 0 ? -q0 : 0;
+          const int x1 = L - q0 < 16 ? L - q0 : 16;
+          cv.v = make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int n = 0; n < NP; ++n)
+            if (n * G >= x0 && n * G < x1) cv.e[n] = *reinterpret_cast<const PT*>(sm + swz(base + off[n]));
+          store_pieces<G>(d, cv.v, x0, x1);
+        }
+      };
+      const int32_t nE = p.ng * p.Cpad;
+      cp_async_wait<1>();
+      __syncthreads();
+      if (mover0)
+        for (int32_t e = tid; e < nE; e += p.nthr0) build(e, true);
+      cp_async_wait<0>();
+      __syncthreads();
+      if (mover0)
+        for (int32_t e = tid; e < nE; e += p.nthr0) build(e, false);
+    } else if constexpr (MODE == 0) {
+      // Pieces of 2 bytes or less: scatter form.
       // phase A: strided chunks -> regions, U loads in flight
       constexpr int U = G == 1 ? 2 : kPhaseUnroll;
       if (mover) {

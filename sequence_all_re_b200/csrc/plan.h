@@ -86,17 +86,13 @@ constexpr int64_t kVecSmallLaunchBytes = int64_t(64) << 20;
 constexpr int64_t kVecMinTileBytes = 2 * 1024;
 // AUTO re-aligns through shared memory what the vector kernel would move in
 // pieces of at most kStageMaxPiece bytes, and 8-byte-granular runs when the
-// fixed-phase form applies: in mode 1 always, in mode 0 below
-// kPhaseOverVec8Run bytes. Measured on B200 (mode 0 / mode 1 of the copy
+// fixed-phase form applies. Measured on B200 (mode 0 / mode 1 of the copy
 // bandwidth, bench.py --staged-forms): 4-, 2- and 1-byte vectors reach
-// 0.16-0.54 against 0.60-0.97 for the fixed-phase form. 8-byte vectors: 0.43 /
-// 0.45 on 8-byte runs, 0.75 / 0.79 on 24, 0.84 / 0.66 on 40, 0.87 / 0.61 on 72
-// (a run of few vectors pays the vector kernel's per-vector decode), 0.88 /
-// 0.69-0.88 on 104, 0.89 / 0.88-0.91 on 136 and 0.89 / 0.92 on 200, against
-// 0.93 / 1.01, 0.88 / 1.01, 0.85 / 0.97, 0.85 / 0.96, 0.84 / 0.96, 0.85 / 0.96
-// and 0.85 / 0.95 for the fixed-phase form.
+// 0.16-0.53 against 0.44-0.98 for the fixed-phase form; 8-byte vectors 0.44 /
+// 0.45 on 8-byte runs, 0.77 / 0.81 on 24, 0.85 / 0.58 on 40, 0.89 / 0.71 on
+// 72, 0.90 / 0.84 on 104, 0.91 / 0.92 on 136 and 0.91 / 0.94 on 200, against
+// 0.99-1.03 / 0.96-1.03 for the fixed-phase form (its mode-0 gather).
 constexpr int kStageMaxPiece = 4;
-constexpr int64_t kPhaseOverVec8Run = 96;
 // Unit numbering: 0 = destination rank outermost, 1 = innermost.
 constexpr int kDefaultOrder = 1;
 // Host-buffer entry point: sequence chunks its H2D copies, kernels and D2H
@@ -202,7 +198,7 @@ struct StageGeometry {
 };
 
 inline bool stage_geometry(int64_t R, int64_t ng, int64_t S, int rows_cap, StageGeometry* g,
-                           bool fixed_phase = false) {
+                           bool fixed_phase = false, bool image = false) {
   const int64_t HDE = ng * R;
   if (R < 1 || ng < 1 || S < 1 || HDE >= (int64_t(1) << 30)) return false;
   int64_t rows = rows_cap > 0 ? rows_cap
@@ -212,7 +208,11 @@ inline bool stage_geometry(int64_t R, int64_t ng, int64_t S, int rows_cap, Stage
   for (; rows >= 1; rows = rows > 1 ? rows / 2 : 0) {
     const int64_t Cg = (rows * R + 30) / 16;
     const int64_t RS = 16 * (fixed_phase && ng <= 4 ? (Cg + 7) / 8 * 8 : (Cg % 2 ? Cg : Cg + 1));
-    const int64_t smem = ng * RS + 4 * ng;
+    // the fixed-phase form's mode-0 gather (pieces of 4 bytes or more) holds
+    // the strided segment's 16-byte chunks as loaded (at most
+    // (rows * HDE + 30) / 16 of them, swizzled within 128-byte blocks); every
+    // other launch holds the ng regions
+    const int64_t smem = image ? (16 * ((rows * HDE + 30) / 16) + 127) / 128 * 128 : ng * RS + 4 * ng;
     if (smem <= kStageSmemMax && rows * HDE < (int64_t(1) << 30)) {
       g->rows = rows;
       g->tiles = (S + rows - 1) / rows;
@@ -586,16 +586,15 @@ inline int make_plan(const void* const* in, void* const* out, int64_t B, int64_t
     }
     // The re-aligning path takes what the vector path could only move in
     // pieces of kStageMaxPiece bytes or less, and 8-byte-granular runs that
-    // the fixed-phase form takes (mode 0: runs under kPhaseOverVec8Run bytes),
-    // or what it is forced onto, except one-output launches.
+    // the fixed-phase form takes, or what it is forced onto, except
+    // one-output launches.
     const bool forced_stage = forced_path == ULYSSES_A2A_PATH_STAGED;
-    const bool auto_stage =
-        forced_path == ULYSSES_A2A_PATH_AUTO && !peeled && only_out < 0 &&
-        (v <= kStageMaxPiece ||
-         (v == 8 && fixed_phase && (mode == 1 || row_bytes < kPhaseOverVec8Run)));
+    const bool auto_stage = forced_path == ULYSSES_A2A_PATH_AUTO && !peeled && only_out < 0 &&
+                            (v <= kStageMaxPiece || (v == 8 && fixed_phase));
     if (forced_stage || auto_stage) {
       StageGeometry sg;
-      if (stage_geometry(row_bytes, ng, S, tune.rows_per_tile, &sg, fixed_phase)) {
+      if (stage_geometry(row_bytes, ng, S, tune.rows_per_tile, &sg, fixed_phase,
+                         fixed_phase && mode == 0 && v >= 4)) {
         const int64_t nbl = chunked ? 1 : B;
         int64_t su;
         if (mul_overflows((int64_t)w * nbl, sg.tiles, &su) || su >= (int64_t(1) << 31)) {

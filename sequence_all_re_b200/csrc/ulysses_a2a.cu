@@ -289,6 +289,14 @@ PhaseParams phase_params(const StageParams& s) {
   p.div_HDE = ua2a::FastDiv((uint32_t)s.HDE);
   p.div_Cg = s.div_Cg;
   p.div_ng = ua2a::FastDiv((uint32_t)s.ng);
+  // mode 0: gathered chunks c + m * Rp of a region share their phase (16 * Rp
+  // is a multiple of R); regions padded to Cpad chunks, a multiple of Rp
+  int64_t gr = 16;
+  while (s.R % gr != 0) gr >>= 1;
+  const int64_t Rp = s.R / gr;
+  p.nthr0 = (int32_t)(Rp * (256 / Rp));
+  p.Cpad = (int32_t)((s.Cg + Rp - 1) / Rp * Rp);
+  p.div_Cpad = ua2a::FastDiv((uint32_t)p.Cpad);
   return p;
 }
 

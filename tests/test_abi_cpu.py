@@ -195,11 +195,10 @@ def test_staged_geometry():
     # 200-byte runs, 8 head groups of 1600-byte rows: one unit per (b, j, tile)
     # covering every head group
     # (8-byte vectors: AUTO keeps the vector path, so the staged path is forced)
-    rc, p, _ = plan(8, 2, 4725, 8, 100)
-    assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 8
-    # (mode 1: the fixed-phase form)
-    rc, p, _ = plan(8, 2, 4725, 8, 100, mode=1)
-    assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 8 and p.fixed_phase == 1
+    # AUTO: the fixed-phase form (8-byte pieces), both modes
+    for mode in (0, 1):
+        rc, p, _ = plan(8, 2, 4725, 8, 100, mode=mode)
+        assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 8 and p.fixed_phase == 1
     # dense and aligned alike, the fixed-phase form: units of 32 KB (20 rows)
     rc, p, _ = plan(8, 2, 4725, 8, 100, forced_path=PATH_STAGED)
     assert rc == OK and p.path == PATH_STAGED and p.vec_bytes == 8 and p.fixed_phase == 1
@@ -277,10 +276,11 @@ def test_staged_fixed_phase_form():
     for D in (29, 27):
         rc, p, _ = plan(3, 1, 64, 3, D, E=1)
         assert rc == OK and p.path == PATH_STAGED and p.fixed_phase == 1
-    # the VEC and TMA paths never set it
-    for args in ((4, 1, 8192, 24, 128), (8, 2, 4725, 8, 100)):
-        rc, p, _ = plan(*args)
-        assert rc == OK and p.path != PATH_STAGED and p.fixed_phase == 0
+    # the VEC and TMA paths never set it (8-byte vectors on a pitched side)
+    rc, p, _ = plan(4, 1, 8192, 24, 128)
+    assert rc == OK and p.path == PATH_TMA and p.fixed_phase == 0
+    rc, p, _ = plan_ex(8, 2, 4725, 8, 100, 8 * 100 + 4)
+    assert rc == OK and p.path == PATH_VEC and p.vec_bytes == 8 and p.fixed_phase == 0
 
 
 def test_vec_when_misaligned_pointer():
@@ -807,7 +807,7 @@ def test_planner_invariants(w, hw, B, S, D, E, mode, chunked, path, rows, ntenso
         assert p.row_bytes % v == 0 and (p.row_pitch * E) % v == 0
         assert v == 16 or (p.row_bytes % (2 * v) or (p.row_pitch * E) % (2 * v))
         if path == PATH_AUTO:
-            assert v <= 4 or (v == 8 and p.fixed_phase and (mode == 1 or p.row_bytes < 96))
+            assert v <= 4 or (v == 8 and p.fixed_phase)
         return
     # tiles cover every sequence row exactly once per (r, b, j) block
     assert 1 <= p.rows_per_tile <= min(S, 256)
@@ -836,9 +836,9 @@ def test_planner_invariants(w, hw, B, S, D, E, mode, chunked, path, rows, ntenso
         v = p.vec_bytes
         assert v in (1, 2, 4, 8, 16) and p.row_bytes % v == 0 and (p.row_pitch * E) % v == 0
         # AUTO leaves narrower vectors to the staged path unless a row is too long,
-        # and 8-byte vectors to its fixed-phase form (mode 0: runs under 96 bytes)
+        # and 8-byte vectors to its fixed-phase form where that applies
         assert path == PATH_VEC or v >= 8 or not _one_row_fits_stage(hw * D * E, ntensors * w)
-        if path == PATH_AUTO and v == 8 and (mode == 1 or p.row_bytes < 96):
+        if path == PATH_AUTO and v == 8:
             rc2, p2, _ = _lib.ulysses_a2a_plan_ex(ins, outs, B, S, H, D, w, mode, chunked, E,
                                                   forced_path=PATH_STAGED, ntensors=ntensors,
                                                   rows_per_tile=rows)

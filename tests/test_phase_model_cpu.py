@@ -14,7 +14,11 @@ checks, for units of many shapes and offsets:
 - mode 1's load batches: the strided chunks assembled before the second wait
   (c < cA) read only region chunks of the first batch (whole 8-chunk blocks up
   to cgA8), and each thread issues all its first-batch chunks before any of
-  the second.
+  the second;
+- mode 0 with pieces of 4 bytes or more (gather form): the segment's chunks
+  occupy distinct places of the swizzled image, every gathered byte comes from
+  the segment byte the element map names, exactly once, and the chunks built
+  before the second wait read only image chunks of the first load batch.
 The model is checked against the element map, not against the GPU; the GPU
 tests compare the kernel itself with the oracle.
 """
@@ -134,18 +138,95 @@ def test_mover_count_is_a_multiple_of_the_phase_period():
 
 
 def test_model_geometry_matches_the_planner():
-    # the model's unit rows and region stride are the ones the library plans
+    # the model's unit rows, region stride and mode-0 image are the ones the
+    # library plans (mode 0 with pieces of 4 bytes or more: the image only)
     from sequence_all_re_b200 import _lib
     for w, H, D, E in ((4, 4, 3, 2), (8, 8, 3, 2), (16, 16, 3, 2), (3, 3, 5, 2), (4, 4, 3, 4),
-                       (2, 2, 5, 1), (4, 8, 5, 2), (8, 8, 9, 4)):
+                       (2, 2, 5, 1), (4, 8, 5, 2), (8, 8, 9, 4), (4, 4, 4, 2)):
         B, S = 1, 100000
         R, ng = (H // w) * D * E, w
         slab = B * S * H * D * E
         step = (slab + 4095) // 4096 * 4096
-        ins = [(1 << 40) + k * step for k in range(w)]
-        outs = [(1 << 44) + k * step for k in range(w)]
-        rc, p, msg = _lib.ulysses_a2a_plan(ins, outs, B, S, H, D, w, 0, 0, E)
-        assert rc == _lib.OK and p.path == _lib.PATH_STAGED and p.fixed_phase == 1, msg
-        assert p.rows_per_tile == 32768 // (ng * R)
-        _, RS = region_stride(R, ng, p.rows_per_tile)
-        assert p.smem_bytes == (ng * RS + 4 * ng + 15) // 16 * 16
+        strided = [(1 << 40) + k * step for k in range(w)]
+        gathered = [(1 << 44) + k * step for k in range(w)]
+        for mode in (0, 1):
+            ins, outs = (strided, gathered) if mode == 0 else (gathered, strided)
+            rc, p, msg = _lib.ulysses_a2a_plan(ins, outs, B, S, H, D, w, mode, 0, E)
+            assert rc == _lib.OK and p.path == _lib.PATH_STAGED and p.fixed_phase == 1, msg
+            assert p.rows_per_tile == 32768 // (ng * R)
+            if mode == 0 and p.vec_bytes >= 4:
+                chunks = (p.rows_per_tile * ng * R + 30) // 16
+                assert p.smem_bytes == (16 * chunks + 127) // 128 * 128
+            else:
+                _, RS = region_stride(R, ng, p.rows_per_tile)
+                assert p.smem_bytes == (ng * RS + 4 * ng + 15) // 16 * 16
+
+
+def swz(x):
+    return x ^ (((x >> 9) & 7) << 4)
+
+
+def replay_gather_unit(R, ng, G, rows, S_tile, a_s, a_g):
+    """Mode 0 with pieces of G >= 4 bytes: the segment's chunks at swizzled
+    places of an image; threads build gathered chunks e = t + m*nthr0 of the
+    regions laid end to end (Cpad chunks each), all of a thread's chunks
+    sharing their phase within a run."""
+    HDE = ng * R
+    segB, L = rows * HDE, rows * R
+    nS = (a_s + segB + 15) >> 4
+    Cg = (S_tile * R + 30) // 16
+    Rp = R // math.gcd(R, 16)
+    nthr0 = Rp * (256 // Rp)
+    Cpad = (Cg + Rp - 1) // Rp * Rp
+    image = (16 * ((S_tile * HDE + 30) // 16) + 127) // 128 * 128
+    r_n = (a_g + L + 15) >> 4
+    rowsA = rows >> 1
+    cI1 = (a_s + rowsA * HDE + 15) >> 4
+    cB1 = (a_g + rowsA * R) >> 4
+    # the image: chunk c at swz(16c), all inside the allocation
+    places = {swz(16 * c) for c in range(nS)}
+    assert len(places) == nS and max(places) + 16 <= image
+    got = {}
+    for tid in range(nthr0):
+        q = 16 * tid - a_g + 16 * R
+        col, drow, off = q % R, 0, []
+        for _ in range(16 // G):
+            off.append(drow * HDE + col)
+            col += G
+            if col == R:
+                col, drow = 0, drow + 1
+        for e in range(tid, ng * Cpad, nthr0):
+            g, c = divmod(e, Cpad)
+            if c >= r_n:
+                continue
+            q0 = 16 * c - a_g
+            i0 = (q0 + 16 * R) // R - 16
+            base = a_s + i0 * HDE + g * R
+            for n in range(16 // G):
+                qq = q0 + n * G
+                if not 0 <= qq < L:
+                    continue
+                pos = base + off[n]                    # a_s + segment byte
+                seg = pos - a_s
+                i, cc = divmod(qq, R)
+                assert seg == i * HDE + g * R + cc     # the element map
+                assert 0 <= seg < segB and swz(pos) + G <= image
+                if c < cB1:
+                    assert (pos >> 4) < cI1, "built before its load batch landed"
+                for b in range(G):
+                    assert (g, qq + b) not in got
+                    got[(g, qq + b)] = seg + b
+    assert len(got) == ng * L
+
+
+@pytest.mark.parametrize("R,G", [(12, 4), (20, 4), (36, 4), (8, 8), (24, 8), (200, 8), (4, 4), (40, 8)],
+                         ids=lambda v: str(v))
+def test_mode0_gather_placement(R, G):
+    rng = random.Random(2000 + R)
+    for ng in (1, 2, 3, 4, 8, 16, 27):
+        if phase_movers(ng * R) < 128:
+            continue
+        for _ in range(3):
+            S_tile = rng.choice([1, 2, 3, 64, max(1, 32768 // (ng * R))])
+            rows = rng.randint(1, S_tile)
+            replay_gather_unit(R, ng, G, rows, S_tile, rng.randrange(0, 16, G), rng.randrange(0, 16, G))

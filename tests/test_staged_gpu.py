@@ -28,7 +28,7 @@ NARROW = [
     # (w, B, S_local, H, D, E): runs of (H/w)*D*E bytes, not a multiple of 16
     (4, 2, 100, 4, 3, 2),       # 6-byte runs: 2-byte pieces
     (4, 1, 77, 4, 3, 4),        # 12-byte runs: 4-byte pieces
-    (8, 2, 53, 8, 100, 2),      # 200-byte runs: 8-byte pieces (AUTO, mode 0: 8-byte vectors)
+    (8, 2, 53, 8, 100, 2),      # 200-byte runs: 8-byte pieces
     (3, 2, 29, 6, 5, 1),        # 10-byte runs: 2-byte pieces, odd rank count
     (2, 3, 33, 2, 7, 1),        # 7-byte runs: 1-byte pieces
     (2, 2, 40, 2, 1, 8),        # 8-byte runs (AUTO: the fixed-phase form, 8-byte pieces)
@@ -43,7 +43,8 @@ NARROW = [
 @pytest.mark.parametrize("chunked", [False, True], ids=["whole", "per_plane"])
 def test_narrow_runs_take_the_staged_path(case, mode, chunked):
     # AUTO re-aligns pieces of 4 bytes or less through shared memory, and
-    # 8-byte ones of short runs; the staged path forced gives the same bytes
+    # 8-byte ones where the fixed-phase form applies; the staged path forced
+    # gives the same bytes
     w, B, S, H, D, E = case
     shape = slab_shape(mode, w, B, S, H, D)
     xs = [t.view(INT[E]).reshape(shape)
@@ -51,9 +52,8 @@ def test_narrow_runs_take_the_staged_path(case, mode, chunked):
     with UlyssesA2A(0, E) as a2a:
         p = a2a.plan([t.cuda() for t in xs], mode)
         assert p["vec_bytes"] < 16
-        # (8-byte vectors stay on the vector path in mode 0 from 96-byte runs on)
-        assert p["path"] == (PATH_STAGED if p["vec_bytes"] <= 4 or p["row_bytes"] < 96 or mode == 1
-                             else PATH_VEC)
+        # (8-byte pieces too: the fixed-phase form applies to every case here)
+        assert p["path"] == PATH_STAGED
         run_case(xs, mode, chunked=chunked, a2a=a2a)
         run_case(xs, mode, chunked=chunked, a2a=a2a, path=PATH_STAGED)
         # dense rows and aligned slabs: the fixed-phase form, unless the
