@@ -29,13 +29,18 @@
 // its piece offsets once per unit, and a piece costs one add and one shared
 // access.
 //
-// Mode 0: strided chunks -> pieces into the regions (phase A, loads held in
-// registers), regions -> gathered ranges (phase B). Mode 1: gathered ranges ->
-// regions by cp.async in two commit groups (A), pieces from the regions ->
-// strided chunks (B), the first half of the unit's rows assembled while the
-// second group is in flight. Global bytes outside the unit are never read or
-// written: a partial chunk at either end of a range or segment moves only its
-// valid pieces.
+// Mode 1: gathered ranges -> regions by cp.async in two commit groups (A),
+// pieces from the regions -> strided chunks (B), the first half of the unit's
+// rows assembled while the second group is in flight.
+// Mode 0, pieces of 2 bytes or less (scatter form): strided chunks -> pieces
+// into the regions (A, loads held in registers), regions -> gathered ranges
+// (B). Mode 0, pieces of 4 or 8 bytes (gather form): the strided segment lands
+// by cp.async in a swizzled image (no regions), in two commit groups, and
+// threads build whole gathered chunks from it, each thread's chunks sharing
+// one phase within a run (the same offset argument, with period
+// R / gcd(R, 16) chunks).
+// Global bytes outside the unit are never read or written: a partial chunk at
+// either end of a range or segment moves only its valid pieces.
 #pragma once
 
 #include <cstdint>
