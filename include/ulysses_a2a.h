@@ -134,8 +134,11 @@ typedef struct ulysses_a2a_plan_t {
     int32_t fixed_phase;     /* STAGED path: 1 = the [B,S_local,H,D] side is
                                 dense and the gathered slabs share one
                                 offset past a 16-byte boundary: each thread
-                                takes strided chunks that share one offset
-                                modulo a strided row, so it works out where
+                                takes chunks that share one offset modulo a
+                                strided row (or, for mode 0 with pieces of
+                                4 or 8 bytes, gathered chunks that share one
+                                offset modulo a run, built from an image of
+                                the strided rows), so it works out where
                                 their pieces go once per work unit; 0 = every
                                 chunk's pieces are placed one by one        */
 } ulysses_a2a_plan_t;
